@@ -1,0 +1,231 @@
+"""Block configurations and seeded synthetic inputs for the sparse MoE FFN block.
+
+This module is shared by the CUDA path's tests/benchmark and by the oracle's
+tests. It holds shapes, seeds and the synthetic checkpoint encoder (the 4-bit
+affine quantiser that stands in for a converted checkpoint); it holds none of
+the block's forward arithmetic.
+
+Shapes follow the pages' models:
+  * the Klear-46B-A2.5B sparse block (hidden 2048, 256 experts, top-8, one
+    shared expert) -- "Klear sparse MoE family" PR, opening paragraph;
+  * Kimi K3's latent MoE (hidden 7168, latent 3584) -- ferrox latent_moe.rs,
+    module doc comment;
+  * a clamped-SwiGLU routed family with a fused interleaved gate_up plane and
+    linear biases -- libmir-metal clamped_routed/experts/mod.rs, ExpertLayout;
+  * 4-bit affine stacked expert planes with group 64 -- mlxcel issue #974,
+    "What exists" / the Jamba2-Mini checkpoint description.
+
+Recipe (every tensor is drawn independently so that generation can run in
+parallel and weights do not depend on the token count):
+  generator seed = 20261202 + 1000*config_id + crc32(tensor name) (+ T for x)
+  x ~ N(0,1); all weights ~ N(0, 0.02); the select-only expert bias ~ N(0, 0.1);
+  linear biases ~ N(0, 0.02); the RMSNorm weight = 1 + N(0, 0.1).
+  Draws are fp32, then cast to the storage dtype.
+"""
+from __future__ import annotations
+
+import dataclasses
+import zlib
+from concurrent.futures import ThreadPoolExecutor
+from typing import Dict, Optional
+
+import numpy as np
+import torch
+
+# Enum codes; the same integers appear in include/moe.h.
+SCORING = {"softmax_all": 0, "sigmoid": 1, "softmax_topk": 2}
+ACTIVATION = {"swiglu": 0, "swiglu_clamped": 1}
+DTYPE = {"f32": 0, "bf16": 1, "q4": 2}
+SHARED = {"none": 0, "add": 1, "blend": 2}
+
+
+@dataclasses.dataclass(frozen=True)
+class MoeSpec:
+    name: str
+    config_id: int
+    hidden: int
+    num_experts: int
+    top_k: int
+    intermediate: int
+    scoring: str = "sigmoid"
+    norm_topk_prob: bool = False
+    routed_scaling_factor: float = 1.0
+    activation: str = "swiglu"
+    swiglu_limit: float = 7.0
+    swiglu_alpha: float = 1.702
+    gate_up_interleaved: bool = False
+    has_expert_bias: bool = False
+    has_router_bias: bool = False
+    has_selection_bias: bool = False
+    act_dtype: str = "bf16"
+    weight_format: str = "bf16"
+    group_size: int = 64
+    bits: int = 4
+    shared_mode: str = "none"
+    shared_intermediate: int = 0
+    latent_dim: int = 0
+    latent_use_norm: bool = False
+    rms_eps: float = 1e-6
+    token_counts: tuple = ()
+
+    @property
+    def expert_in(self) -> int:
+        """K of the routed experts: the latent width when latent, else hidden."""
+        return self.latent_dim if self.latent_dim else self.hidden
+
+    def replace(self, **kw) -> "MoeSpec":
+        return dataclasses.replace(self, **kw)
+
+
+# The five workloads.
+TINY_F32 = MoeSpec(
+    name="tiny_f32", config_id=1, hidden=64, num_experts=8, top_k=2, intermediate=32,
+    scoring="softmax_all", norm_topk_prob=False, act_dtype="f32", weight_format="f32",
+    token_counts=(16,))
+KLEAR_BF16 = MoeSpec(
+    name="klear_bf16", config_id=2, hidden=2048, num_experts=256, top_k=8, intermediate=768,
+    scoring="sigmoid", has_selection_bias=True, norm_topk_prob=True,
+    shared_mode="blend", shared_intermediate=768, token_counts=(1, 8, 64, 4096))
+KLEAR_Q4 = KLEAR_BF16.replace(name="klear_q4", config_id=3, weight_format="q4",
+                              token_counts=(1, 32, 2048))
+CLAMPED_BF16 = MoeSpec(
+    name="clamped_bf16", config_id=4, hidden=2880, num_experts=128, top_k=4, intermediate=2880,
+    scoring="softmax_topk", activation="swiglu_clamped", gate_up_interleaved=True,
+    has_expert_bias=True, token_counts=(1, 8192))
+LATENT_BF16 = MoeSpec(
+    name="latent_bf16", config_id=5, hidden=7168, num_experts=384, top_k=8, intermediate=2048,
+    scoring="sigmoid", has_selection_bias=True, norm_topk_prob=True,
+    shared_mode="add", shared_intermediate=2048, latent_dim=3584, latent_use_norm=True,
+    rms_eps=1e-6, token_counts=(1, 128, 8192))
+
+WORKLOADS = {s.name: s for s in (TINY_F32, KLEAR_BF16, KLEAR_Q4, CLAMPED_BF16, LATENT_BF16)}
+
+BASE_SEED = 20261202
+
+
+def _seed(spec: MoeSpec, name: str, extra: int = 0) -> int:
+    return (BASE_SEED + 1000 * spec.config_id + zlib.crc32(name.encode()) + extra) % (2 ** 63)
+
+
+def _normal(shape, std: float, seed: int, mean: float = 0.0) -> torch.Tensor:
+    g = torch.Generator(device="cpu")
+    g.manual_seed(seed)
+    t = torch.randn(shape, generator=g, dtype=torch.float32)
+    if std != 1.0:
+        t.mul_(std)
+    if mean != 0.0:
+        t.add_(mean)
+    return t
+
+
+def _storage(t: torch.Tensor, dtype: str) -> torch.Tensor:
+    if dtype == "f32":
+        return t.contiguous()
+    return t.to(torch.bfloat16).contiguous()
+
+
+def quantize_affine_q4(w: torch.Tensor, group_size: int):
+    """Encode fp32 planes [..., K] as a synthetic 4-bit affine checkpoint.
+
+    Per group of `group_size` consecutive input elements: scale = (max-min)/15
+    and bias = min, both rounded to bf16 first; q = clamp(round((w-bias)/scale),
+    0, 15). Eight codes pack into one uint32, element j of a row at bits
+    4*(j mod 8) of word j/8. Returns (packed words [..., K/8] as int32 bit patterns, scales bf16
+    [..., K/group], biases bf16 [..., K/group]).
+    """
+    *lead, k = w.shape
+    assert k % group_size == 0 and k % 8 == 0
+    g = w.reshape(*lead, k // group_size, group_size)
+    mn = g.amin(dim=-1)
+    mx = g.amax(dim=-1)
+    scale = ((mx - mn) / 15.0).clamp_min(1e-8).to(torch.bfloat16)
+    bias = mn.to(torch.bfloat16)
+    q = torch.round((g - bias.float().unsqueeze(-1)) / scale.float().unsqueeze(-1)).clamp_(0, 15)
+    q = q.to(torch.int64).reshape(*lead, k // 8, 8)
+    shifts = torch.arange(8, dtype=torch.int64) * 4
+    packed = (q << shifts).sum(dim=-1)
+    packed = packed.bitwise_and(0xFFFFFFFF).numpy().astype(np.uint32).view(np.int32)
+    # torch has no general uint32 arithmetic: the words travel as int32 bit patterns.
+    return torch.from_numpy(packed.copy()), scale.contiguous(), bias.contiguous()
+
+
+def _expert_plane(spec: MoeSpec, name: str, rows: int, cols: int, pool) -> Dict[str, torch.Tensor]:
+    """One stacked expert projection [E, rows, cols] in the spec's weight format.
+
+    Each expert is drawn from its own generator so the draws run in parallel.
+    """
+    e_count = spec.num_experts
+
+    def one(e):
+        w = _normal((rows, cols), 0.02, _seed(spec, f"{name}/{e}"))
+        if spec.weight_format == "q4":
+            return quantize_affine_q4(w, spec.group_size)
+        return (_storage(w, spec.weight_format),)
+
+    parts = list(pool.map(one, range(e_count)))
+    if spec.weight_format == "q4":
+        stem = name[:-2]  # "gate_w" -> companions "gate_s" (scales), "gate_z" (biases)
+        return {name: torch.stack([p[0] for p in parts]),
+                stem + "_s": torch.stack([p[1] for p in parts]),
+                stem + "_z": torch.stack([p[2] for p in parts])}
+    return {name: torch.stack([p[0] for p in parts])}
+
+
+def make_weights(spec: MoeSpec, threads: Optional[int] = None) -> Dict[str, torch.Tensor]:
+    """All block weights on the CPU, keyed by the C ABI's moe_weights field names."""
+    H, E, I = spec.hidden, spec.num_experts, spec.intermediate
+    K = spec.expert_in
+    act = spec.act_dtype
+    w: Dict[str, torch.Tensor] = {}
+    w["router_w"] = _storage(_normal((E, H), 0.02, _seed(spec, "router_w")), act)
+    if spec.has_router_bias:
+        w["router_b"] = _storage(_normal((E,), 0.02, _seed(spec, "router_b")), act)
+    if spec.has_selection_bias:
+        w["selection_bias"] = _normal((E,), 0.1, _seed(spec, "selection_bias"))
+    if spec.shared_mode == "blend":
+        w["coef_w"] = _storage(_normal((2, H), 0.02, _seed(spec, "coef_w")), act)
+        w["coef_b"] = _storage(_normal((2,), 0.02, _seed(spec, "coef_b")), act)
+    with ThreadPoolExecutor(max_workers=threads or max(1, torch.get_num_threads())) as pool:
+        if spec.gate_up_interleaved:
+            w.update(_expert_plane(spec, "gate_up_w", 2 * I, K, pool))
+        else:
+            w.update(_expert_plane(spec, "gate_w", I, K, pool))
+            w.update(_expert_plane(spec, "up_w", I, K, pool))
+        w.update(_expert_plane(spec, "down_w", K, I, pool))
+    if spec.has_expert_bias:
+        if spec.gate_up_interleaved:
+            w["gate_up_b"] = _storage(_normal((E, 2 * I), 0.02, _seed(spec, "gate_up_b")), act)
+        else:
+            w["gate_b"] = _storage(_normal((E, I), 0.02, _seed(spec, "gate_b")), act)
+            w["up_b"] = _storage(_normal((E, I), 0.02, _seed(spec, "up_b")), act)
+        w["down_b"] = _storage(_normal((E, K), 0.02, _seed(spec, "down_b")), act)
+    if spec.shared_mode != "none":
+        Is = spec.shared_intermediate
+        w["shared_gate_w"] = _storage(_normal((Is, H), 0.02, _seed(spec, "shared_gate_w")), act)
+        w["shared_up_w"] = _storage(_normal((Is, H), 0.02, _seed(spec, "shared_up_w")), act)
+        w["shared_down_w"] = _storage(_normal((H, Is), 0.02, _seed(spec, "shared_down_w")), act)
+    if spec.latent_dim:
+        L = spec.latent_dim
+        w["latent_down_w"] = _storage(_normal((L, H), 0.02, _seed(spec, "latent_down_w")), act)
+        w["latent_up_w"] = _storage(_normal((H, L), 0.02, _seed(spec, "latent_up_w")), act)
+        if spec.latent_use_norm:
+            w["latent_norm_w"] = _storage(
+                _normal((L,), 0.1, _seed(spec, "latent_norm_w"), mean=1.0), act)
+    return w
+
+
+def make_x(spec: MoeSpec, T: int, scale: float = 1.0) -> torch.Tensor:
+    """Block input [T, hidden] ~ N(0, scale^2) in the activation dtype."""
+    x = _normal((T, spec.hidden), scale, _seed(spec, "x", extra=T))
+    return _storage(x, spec.act_dtype)
+
+
+def to_numpy_storage(t: torch.Tensor) -> np.ndarray:
+    """Bit-exact numpy view of a stored tensor: bf16 -> uint16, f32 -> float32,
+    packed 4-bit words (int32) -> uint32."""
+    t = t.contiguous()
+    if t.dtype == torch.bfloat16:
+        return t.view(torch.int16).numpy().view(np.uint16)
+    if t.dtype == torch.int32:
+        return t.numpy().view(np.uint32)
+    return t.numpy()

@@ -1,0 +1,59 @@
+"""Tiny block variants used by the oracle pins and the small parity cases.
+
+Each variant exercises one branch of the block: sigmoid routing with a
+select-only bias and the shared-expert blend (Klear PR items 2-3), softmax
+over the top-k logits with clamped SwiGLU on an interleaved gate_up plane with
+biases (libmir-metal clamped_routed ExpertLayout::DenseFused), 4-bit affine
+planes (mlxcel issue #974), and the latent variant (ferrox latent_moe.rs).
+"""
+import numpy as np
+
+from sparse_moe_ffn_gemv_b200 import inputs
+from sparse_moe_ffn_gemv_b200.inputs import MoeSpec
+
+SIG_BLEND = MoeSpec(
+    name="t_sig_blend", config_id=101, hidden=48, num_experts=6, top_k=3, intermediate=16,
+    scoring="sigmoid", has_selection_bias=True, norm_topk_prob=True,
+    shared_mode="blend", shared_intermediate=24)
+CLAMPED = MoeSpec(
+    name="t_clamped", config_id=102, hidden=40, num_experts=5, top_k=2, intermediate=24,
+    scoring="softmax_topk", activation="swiglu_clamped", gate_up_interleaved=True,
+    has_expert_bias=True)
+Q4 = MoeSpec(
+    name="t_q4", config_id=103, hidden=128, num_experts=4, top_k=2, intermediate=64,
+    scoring="sigmoid", has_selection_bias=True, norm_topk_prob=True, weight_format="q4",
+    group_size=64, shared_mode="blend", shared_intermediate=32)
+LATENT = MoeSpec(
+    name="t_latent", config_id=104, hidden=48, num_experts=6, top_k=2, intermediate=16,
+    scoring="sigmoid", has_selection_bias=True, norm_topk_prob=True, shared_mode="add",
+    shared_intermediate=20, latent_dim=24, latent_use_norm=True)
+ROUTER_BIAS = MoeSpec(
+    name="t_router_bias", config_id=105, hidden=32, num_experts=7, top_k=3, intermediate=8,
+    scoring="softmax_all", has_router_bias=True, norm_topk_prob=True, shared_mode="add",
+    shared_intermediate=8, act_dtype="f32", weight_format="f32")
+SEPARATE_BIAS = MoeSpec(
+    name="t_sep_bias", config_id=106, hidden=64, num_experts=4, top_k=2, intermediate=32,
+    scoring="sigmoid", norm_topk_prob=False, has_expert_bias=True, weight_format="q4",
+    group_size=32)
+LATENT_NONORM = LATENT.replace(name="t_latent_nonorm", config_id=107, latent_use_norm=False)
+
+ALL = [inputs.TINY_F32, SIG_BLEND, CLAMPED, Q4, LATENT, ROUTER_BIAS, SEPARATE_BIAS,
+       LATENT_NONORM]
+
+
+def np_weights(spec, scale_weights: float = 1.0):
+    """Stored weights as bit-exact numpy arrays (the oracle's input form)."""
+    w = inputs.make_weights(spec, threads=4)
+    return {k: inputs.to_numpy_storage(v) for k, v in w.items()}
+
+
+def np_x(spec, T, scale=1.0):
+    return inputs.to_numpy_storage(inputs.make_x(spec, T, scale))
+
+
+def to_bf16_bits(a: np.ndarray) -> np.ndarray:
+    """float64 values that are exactly representable in bf16 -> bf16 bit patterns."""
+    f = np.ascontiguousarray(a, dtype=np.float32)
+    bits = f.view(np.uint32)
+    assert np.all((bits & 0xFFFF) == 0), "value not exact in bf16"
+    return (bits >> 16).astype(np.uint16)
