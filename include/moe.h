@@ -1,0 +1,220 @@
+/*
+ * moe.h -- C ABI of the sparse Mixture-of-Experts FFN block forward on B200.
+ *
+ * The block (Klear sparse MoE family PR, items 2-3; libmir-metal
+ * clamped_routed/experts/mod.rs, ClampedRoutedExperts::forward/execute;
+ * ferrox latent_moe.rs, kimi_latent_moe_forward):
+ *
+ *   logits = x Wr^T (+ b_r)                           router, fp32 logits
+ *   scores = softmax(logits) | sigmoid(logits) | logits   (per `scoring`)
+ *   keys   = scores (+ selection_bias)                    select-only bias
+ *   idx    = top-k(keys), descending, ties -> lower expert index
+ *   w      = scores[idx] | softmax(logits[idx]); optionally w /= sum(w)
+ *   u      = x, or z = x Wdp^T for the latent variant
+ *   y_r    = sum_j w_j * Wd[e_j] act(Wg[e_j] u + bg, Wu[e_j] u + bu) (+ bd)
+ *   latent: y_r = Wup (rmsnorm(y_r) * gamma)
+ *   y      = y_r | y_r + s | y_r * c0 + s * c1,   s = shared expert(x),
+ *            (c0, c1) = softmax(x Wc^T + b_c)
+ *
+ * Conventions for every call:
+ *  - All pointers are DEVICE pointers unless stated otherwise. The caller
+ *    allocates, owns and frees every buffer, the workspace included; the
+ *    library never allocates device memory, never frees, and keeps no pointer
+ *    after a call returns.
+ *  - Calls are asynchronous on `stream` (a cudaStream_t; NULL = legacy default
+ *    stream). T (the token count) is the product of the input's leading dims;
+ *    T == 0 returns MOE_OK and launches nothing.
+ *  - Errors are returned as moe_status, never thrown and never aborted across
+ *    this boundary (mlxcel issue #974: an exception crossing an FFI boundary is
+ *    an uncatchable abort). Everything checkable on the host is checked before
+ *    the first launch, so a failed call launched nothing.
+ *  - Row-major layouts; weights are [out, in] (ferrox KimiExpertWeights:
+ *    w1 gate [ffn, in], w2 down [in, ffn], w3 up [ffn, in]) and routed experts
+ *    are stacked [E, out, in] (mlxcel issue #974, switch_mlp planes).
+ *  - Every device pointer must be 16-byte aligned and every row length in
+ *    bytes a multiple of 16 (hidden, intermediate, latent and shared widths
+ *    multiples of 8 for bf16, of 4 for f32).
+ *
+ * Library: libmoe_b200.so (sm_100a). Thread-safe: calls keep no global state.
+ */
+#ifndef MOE_B200_H
+#define MOE_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define MOE_API __attribute__((visibility("default")))
+#else
+#define MOE_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same object as cudaStream_t; declared here so that callers need no CUDA header. */
+typedef struct CUstream_st *moe_stream_t;
+
+typedef enum moe_status {
+    MOE_OK = 0,
+    MOE_ERR_INVALID_ARGUMENT = 1,     /* NULL/misaligned pointer, bad enum, bad size  */
+    MOE_ERR_SHAPE_OVERFLOW = 2,       /* a size product overflows the index types     */
+    MOE_ERR_INVALID_QUANTIZATION = 3, /* bits / group_size not supported              */
+    MOE_ERR_MISSING_TENSOR = 4,       /* a tensor the config needs is NULL            */
+    MOE_ERR_UNSUPPORTED = 5,          /* valid on the pages, not built here           */
+    MOE_ERR_CUDA = 6,                 /* a CUDA launch/runtime call failed            */
+    MOE_ERR_DEVICE_CHECK = 7,         /* a kernel found an out-of-range expert id     */
+    MOE_ERR_DEVICE_TIMEOUT = 8,       /* a bounded device wait gave up                */
+    MOE_ERR_WORKSPACE_TOO_SMALL = 9   /* ws_bytes below moe_workspace_size(cfg, T)    */
+} moe_status;
+
+enum moe_scoring {
+    MOE_SCORING_SOFTMAX_ALL = 0,   /* softmax over all E logits, then top-k            */
+    MOE_SCORING_SIGMOID = 1,       /* sigmoid of fp32 logits (Klear PR item 3)          */
+    MOE_SCORING_SOFTMAX_TOPK = 2   /* top-k logits, softmax over the k (router_top_k_unit) */
+};
+enum moe_activation {
+    MOE_ACT_SWIGLU = 0,            /* silu(g) * v                                       */
+    MOE_ACT_SWIGLU_CLAMPED = 1     /* g'=min(g,limit), v'=clamp(v,-limit,limit),
+                                      g' * sigmoid(alpha g') * (v' + 1)                 */
+};
+enum moe_dtype {
+    MOE_DTYPE_F32 = 0,
+    MOE_DTYPE_BF16 = 1,
+    MOE_DTYPE_Q4_AFFINE = 2        /* weights only: packed 4-bit codes + bf16 scale/bias */
+};
+enum moe_shared_mode {
+    MOE_SHARED_NONE = 0,
+    MOE_SHARED_ADD = 1,            /* y = y_r + s (ferrox latent_moe.rs)                */
+    MOE_SHARED_BLEND = 2           /* y = y_r * c0 + s * c1 (Klear PR item 2)           */
+};
+
+/* Plain-data description of one block. Checked by moe_config_validate. */
+typedef struct moe_config {
+    int32_t hidden;                /* H                                                 */
+    int32_t num_experts;           /* E                                                 */
+    int32_t top_k;                 /* k, 1 <= k <= E, k <= 16                           */
+    int32_t intermediate;          /* I, routed expert intermediate width               */
+    int32_t scoring;               /* enum moe_scoring                                  */
+    int32_t norm_topk_prob;        /* 1: w /= sum(w) over the k                         */
+    float routed_scaling_factor;   /* must be 1.0 (Klear PR item 3: not applied)        */
+    int32_t activation;            /* enum moe_activation                               */
+    float swiglu_limit;            /* clamp limit (clamped only), finite > 0            */
+    float swiglu_alpha;            /* sigmoid slope (clamped only), finite              */
+    int32_t gate_up_interleaved;   /* 1: one [E, 2I, K] plane, row 2i gate, 2i+1 up     */
+    int32_t has_expert_bias;       /* 1: gate/up and down linear biases                 */
+    int32_t has_router_bias;       /* 1: router bias b_r [E]                            */
+    int32_t has_selection_bias;    /* 1: select-only bias [E] (f32)                     */
+    int32_t act_dtype;             /* MOE_DTYPE_F32 or MOE_DTYPE_BF16: x, y and every
+                                      non-routed weight                                 */
+    int32_t weight_format;         /* routed planes: F32 (needs act F32), BF16, Q4_AFFINE */
+    int32_t group_size;            /* Q4 only: 32, 64 or 128                            */
+    int32_t bits;                  /* Q4 only: 4                                        */
+    int32_t shared_mode;           /* enum moe_shared_mode                              */
+    int32_t shared_intermediate;   /* Is (> 0 iff shared_mode != NONE)                  */
+    int32_t latent_dim;            /* L; 0 = no latent projection                       */
+    int32_t latent_use_norm;       /* 1: RMSNorm of the combined latent                 */
+    float rms_eps;                 /* RMSNorm epsilon, finite > 0                       */
+} moe_config;
+
+/*
+ * Device pointers to the block's tensors (NULL where the config does not use
+ * them). Dense tensors are in act_dtype except selection_bias (f32).
+ *   router_w [E, H]   router_b [E]   selection_bias [E] f32
+ *   coef_w [2, H]     coef_b [2]                                (BLEND)
+ *   gate_w, up_w [E, I, K]  or  gate_up_w [E, 2I, K]            K = L or H
+ *   down_w [E, K, I]
+ *   gate_b, up_b [E, I] or gate_up_b [E, 2I];  down_b [E, K]    (expert bias)
+ *   Q4: gate_w/up_w/down_w hold uint32 words [E, rows, cols/8] (element j of a
+ *       row at bits 4*(j mod 8) of word j/8), gate_s/up_s/down_s the bf16
+ *       scales and gate_z/up_z/down_z the bf16 biases [E, rows, cols/group];
+ *       weight = scale * q + bias.
+ *   shared_gate_w, shared_up_w [Is, H]; shared_down_w [H, Is]
+ *   latent_down_w [L, H]; latent_up_w [H, L]; latent_norm_w [L]
+ */
+typedef struct moe_weights {
+    const void *router_w, *router_b, *selection_bias, *coef_w, *coef_b;
+    const void *gate_w, *up_w, *gate_up_w, *gate_b, *up_b, *gate_up_b, *down_w, *down_b;
+    const void *gate_s, *gate_z, *up_s, *up_z, *down_s, *down_z;
+    const void *shared_gate_w, *shared_up_w, *shared_down_w;
+    const void *latent_down_w, *latent_up_w, *latent_norm_w;
+} moe_weights;
+
+/* Checks a config on the host (Klear PR "Other guards": zero checks before
+ * divisibility, 1 <= k <= E, finite positive eps; mlxcel issue #974: bits and
+ * group_size bounded before use). No device work. */
+MOE_API moe_status moe_config_validate(const moe_config *cfg);
+
+/* Checks that every tensor the config needs is present (MOE_ERR_MISSING_TENSOR,
+ * e.g. a blend without its coefficient head) and 16-byte aligned. Host only. */
+MOE_API moe_status moe_weights_validate(const moe_config *cfg, const moe_weights *w);
+
+/* Bytes of workspace needed for up to max_tokens tokens (the same value serves
+ * every call below). *bytes is written on MOE_OK only. Host only. */
+MOE_API moe_status moe_workspace_size(const moe_config *cfg, int64_t max_tokens, size_t *bytes);
+
+/* Router (a1 + a2): fp32 logits of x [T, H], scoring, select-only bias, top-k
+ * and the combine weights; for BLEND also the 2-way coefficients.
+ * Writes topk_idx [T, k] int32 (descending selection key, ties to the lower
+ * index), topk_w [T, k] f32, coef [T, 2] f32 (BLEND; may be NULL otherwise).
+ * Klear PR item 3; libmir-metal forward: router -> router_top_k_unit. */
+MOE_API moe_status moe_route(const moe_config *cfg, const moe_weights *w, const void *x, int64_t T,
+                     int32_t *topk_idx, float *topk_w, float *coef,
+                     void *ws, size_t ws_bytes, moe_stream_t stream);
+
+/* Permutation (a3): groups the T*k slots (slot s = t*k + j) by expert with a
+ * stable counting sort. Writes expert_offsets [E+1] (exclusive prefix of the
+ * per-expert counts), sorted_slot [T*k] (expert 0's slots ascending, then
+ * expert 1's, ...) and slot_pos [T*k] (its inverse). An expert id outside
+ * [0, E) sets MOE_ERR_DEVICE_CHECK in the workspace status word (see
+ * moe_read_device_status) and that slot is dropped. */
+MOE_API moe_status moe_permute(const moe_config *cfg, const int32_t *topk_idx, int64_t T,
+                       int32_t *expert_offsets, int32_t *sorted_slot, int32_t *slot_pos,
+                       void *ws, size_t ws_bytes, moe_stream_t stream);
+
+/* Routed experts (a4 + a5): y_acc [T, K] f32 = sum over each token's k slots of
+ * topk_w[slot] * expert(u[token]) with u [T, K] in act_dtype (K = L for the
+ * latent variant, else H). Overwrites y_acc. The expert_offsets / sorted_slot
+ * inputs are moe_permute's outputs for the same topk_idx.
+ * libmir-metal execute (gate_up then down weighted by routing.weights);
+ * ferrox kimi_latent_moe_forward (combined += w * expert(latent)). */
+MOE_API moe_status moe_grouped_ffn(const moe_config *cfg, const moe_weights *w, const void *u, int64_t T,
+                           const int32_t *expert_offsets, const int32_t *sorted_slot,
+                           const float *topk_w, float *y_acc,
+                           void *ws, size_t ws_bytes, moe_stream_t stream);
+
+/* Latent down projection (first half of a8): z [T, L] (act_dtype) = x Wdp^T.
+ * ferrox kimi_latent_moe_forward: latent = down_proj(hidden). */
+MOE_API moe_status moe_latent_down(const moe_config *cfg, const moe_weights *w, const void *x, int64_t T,
+                           void *z, void *ws, size_t ws_bytes, moe_stream_t stream);
+
+/* Combine (a6 + a7, and the tail of a8): from the routed sum y_acc [T, K] f32,
+ * computes the shared expert on x, then y [T, H] (act_dtype) = y_r, y_r + s or
+ * y_r * coef[:, 0] + s * coef[:, 1]; for the latent variant y_r = Wup
+ * (rmsnorm(y_acc) * gamma) first. coef [T, 2] is moe_route's (BLEND only).
+ * Klear PR item 2; ferrox kimi_latent_moe_forward (rms_norm, up_proj, + shared). */
+MOE_API moe_status moe_combine(const moe_config *cfg, const moe_weights *w, const float *y_acc,
+                       const void *x, const float *coef, int64_t T, void *y,
+                       void *ws, size_t ws_bytes, moe_stream_t stream);
+
+/* The whole block: y [T, H] = block(x [T, H]), act_dtype in and out. */
+MOE_API moe_status moe_block_forward(const moe_config *cfg, const moe_weights *w, const void *x,
+                             int64_t T, void *y, void *ws, size_t ws_bytes, moe_stream_t stream);
+
+/* Synchronises `stream`, returns the status word that device-side checks
+ * write into the workspace (MOE_OK, MOE_ERR_DEVICE_CHECK or
+ * MOE_ERR_DEVICE_TIMEOUT) and clears it. A new workspace must be cleared once
+ * with this call or zero-filled before first use. */
+MOE_API moe_status moe_read_device_status(void *ws, moe_stream_t stream);
+
+/* Clears the workspace status word, asynchronously on `stream`. */
+MOE_API moe_status moe_clear_device_status(void *ws, moe_stream_t stream);
+
+/* Static, NUL-terminated description of a status code. */
+MOE_API const char *moe_status_string(moe_status status);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* MOE_B200_H */

@@ -1,0 +1,525 @@
+// api.cu -- the C ABI: host-side validation, workspace layout and launch order.
+//
+// Every check that the host can make runs before the first launch (Klear PR
+// "Other guards": zero checks before divisibility, k within 1..=E, positive
+// finite eps, a blend without its coefficient head rejected; mlxcel issue #974:
+// quantisation parameters bounded where they enter, errors returned instead of
+// an abort crossing the boundary).
+#include <algorithm>
+#include <cmath>
+#include <cstring>
+
+#include "common.cuh"
+#include "internal.h"
+
+namespace moe {
+
+int64_t max_routed_tiles(const moe_config& c, int64_t T) {
+    (void)c;
+    (void)T;
+    return 0;
+}
+
+WsLayout ws_layout(const moe_config& c, int64_t T) {
+    WsLayout L{};
+    size_t off = 0;
+    auto take = [&](int64_t bytes) {
+        const size_t o = off;
+        off = align256(off + size_t(bytes > 0 ? bytes : 0));
+        return o;
+    };
+    const int64_t E = c.num_experts, k = c.top_k, I = c.intermediate, H = c.hidden;
+    const int64_t K = expert_in(c), Ld = c.latent_dim, Is = c.shared_intermediate;
+    const int64_t ab = act_bytes(c);
+    L.T = T;
+    L.ld_logits = int((E + 2 + 3) & ~int64_t(3));
+    L.n_chunks = int((T * k + kPermChunk - 1) / kPermChunk);
+    L.status = take(256);
+    L.logits = take(T * L.ld_logits * 4);
+    L.topk_idx = take(T * k * 4);
+    L.topk_w = take(T * k * 4);
+    L.coef = take(T * 2 * 4);
+    L.offsets = take((E + 1) * 4);
+    L.sorted_slot = take(T * k * 4);
+    L.slot_pos = take(T * k * 4);
+    L.active = take((E + 1) * 4);
+    L.chunk_hist = take(int64_t(L.n_chunks > 0 ? L.n_chunks : 1) * E * 4);
+    L.h = take(T * k * I * ab);
+    L.hs = take(T * Is * ab);
+    L.y_acc = take(T * K * 4);
+    L.s_acc = take(c.shared_mode != MOE_SHARED_NONE ? T * H * 4 : 0);
+    L.z = take(Ld ? T * Ld * ab : 0);
+    L.nrm = take(Ld ? T * Ld * ab : 0);
+    L.uperm = take(0);
+    L.tiles = take(0);
+    L.total = off;
+    return L;
+}
+
+}  // namespace moe
+
+using namespace moe;
+
+namespace {
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+bool finite_pos(float v) { return std::isfinite(v) && v > 0.f; }
+
+moe_status validate_config(const moe_config* c) {
+    if (!c) return MOE_ERR_INVALID_ARGUMENT;
+    // zero / sign checks first, divisibility afterwards
+    if (c->hidden <= 0 || c->num_experts <= 0 || c->top_k <= 0 || c->intermediate <= 0)
+        return MOE_ERR_INVALID_ARGUMENT;
+    if (c->top_k > c->num_experts || c->top_k > kMaxTopK || c->num_experts > kMaxExperts)
+        return MOE_ERR_INVALID_ARGUMENT;
+    if (c->scoring < MOE_SCORING_SOFTMAX_ALL || c->scoring > MOE_SCORING_SOFTMAX_TOPK)
+        return MOE_ERR_INVALID_ARGUMENT;
+    if (c->activation != MOE_ACT_SWIGLU && c->activation != MOE_ACT_SWIGLU_CLAMPED)
+        return MOE_ERR_INVALID_ARGUMENT;
+    if (c->shared_mode < MOE_SHARED_NONE || c->shared_mode > MOE_SHARED_BLEND) return MOE_ERR_INVALID_ARGUMENT;
+    if (c->act_dtype != MOE_DTYPE_F32 && c->act_dtype != MOE_DTYPE_BF16) return MOE_ERR_INVALID_ARGUMENT;
+    if (c->weight_format < MOE_DTYPE_F32 || c->weight_format > MOE_DTYPE_Q4_AFFINE)
+        return MOE_ERR_INVALID_ARGUMENT;
+    if (c->shared_intermediate < 0 || c->latent_dim < 0) return MOE_ERR_INVALID_ARGUMENT;
+    if ((c->shared_mode == MOE_SHARED_NONE) != (c->shared_intermediate == 0)) return MOE_ERR_INVALID_ARGUMENT;
+    if (c->latent_use_norm && !c->latent_dim) return MOE_ERR_INVALID_ARGUMENT;
+    if (c->latent_use_norm && !finite_pos(c->rms_eps)) return MOE_ERR_INVALID_ARGUMENT;
+    if (c->activation == MOE_ACT_SWIGLU_CLAMPED &&
+        (!finite_pos(c->swiglu_limit) || !std::isfinite(c->swiglu_alpha)))
+        return MOE_ERR_INVALID_ARGUMENT;
+    // routed_scaling_factor: declared by some checkpoints, never applied (Klear PR item 3)
+    if (c->routed_scaling_factor != 1.0f) return MOE_ERR_UNSUPPORTED;
+    // weight format <-> activation dtype
+    if ((c->weight_format == MOE_DTYPE_F32) != (c->act_dtype == MOE_DTYPE_F32)) return MOE_ERR_UNSUPPORTED;
+    const int K = expert_in(*c);
+    if (c->weight_format == MOE_DTYPE_Q4_AFFINE) {
+        if (c->bits != 4) return MOE_ERR_INVALID_QUANTIZATION;
+        if (c->group_size != 32 && c->group_size != 64 && c->group_size != 128)
+            return MOE_ERR_INVALID_QUANTIZATION;
+        if (K % c->group_size != 0 || c->intermediate % c->group_size != 0)
+            return MOE_ERR_INVALID_QUANTIZATION;
+        if (c->gate_up_interleaved) return MOE_ERR_UNSUPPORTED;
+    }
+    // 16-byte rows
+    const int q = c->act_dtype == MOE_DTYPE_F32 ? 4 : 8;
+    if (c->hidden % q || c->intermediate % q || K % q || c->shared_intermediate % q) return MOE_ERR_INVALID_ARGUMENT;
+    // sizes of the stacked planes must fit the index arithmetic
+    const int64_t plane = int64_t(c->num_experts) * 2 * c->intermediate * K;
+    if (plane / c->num_experts / 2 / c->intermediate != K || plane > (int64_t(1) << 46))
+        return MOE_ERR_SHAPE_OVERFLOW;
+    return MOE_OK;
+}
+
+moe_status validate_weights(const moe_config* c, const moe_weights* w) {
+    if (!w) return MOE_ERR_INVALID_ARGUMENT;
+    auto need = [](const void* p) { return p != nullptr; };
+    if (!need(w->router_w)) return MOE_ERR_MISSING_TENSOR;
+    if (c->has_router_bias && !need(w->router_b)) return MOE_ERR_MISSING_TENSOR;
+    if (c->has_selection_bias && !need(w->selection_bias)) return MOE_ERR_MISSING_TENSOR;
+    if (c->shared_mode == MOE_SHARED_BLEND && (!need(w->coef_w) || !need(w->coef_b))) return MOE_ERR_MISSING_TENSOR;
+    if (c->gate_up_interleaved) {
+        if (!need(w->gate_up_w)) return MOE_ERR_MISSING_TENSOR;
+        if (c->has_expert_bias && !need(w->gate_up_b)) return MOE_ERR_MISSING_TENSOR;
+    } else {
+        if (!need(w->gate_w) || !need(w->up_w)) return MOE_ERR_MISSING_TENSOR;
+        if (c->has_expert_bias && (!need(w->gate_b) || !need(w->up_b))) return MOE_ERR_MISSING_TENSOR;
+    }
+    if (!need(w->down_w)) return MOE_ERR_MISSING_TENSOR;
+    if (c->has_expert_bias && !need(w->down_b)) return MOE_ERR_MISSING_TENSOR;
+    if (c->weight_format == MOE_DTYPE_Q4_AFFINE) {
+        const void* q[] = {w->gate_s, w->gate_z, w->up_s, w->up_z, w->down_s, w->down_z};
+        for (const void* p : q)
+            if (!need(p)) return MOE_ERR_MISSING_TENSOR;
+    }
+    if (c->shared_mode != MOE_SHARED_NONE &&
+        (!need(w->shared_gate_w) || !need(w->shared_up_w) || !need(w->shared_down_w)))
+        return MOE_ERR_MISSING_TENSOR;
+    if (c->latent_dim && (!need(w->latent_down_w) || !need(w->latent_up_w))) return MOE_ERR_MISSING_TENSOR;
+    if (c->latent_use_norm && !need(w->latent_norm_w)) return MOE_ERR_MISSING_TENSOR;
+    const void* all[] = {w->router_w, w->router_b, w->selection_bias, w->coef_w, w->coef_b,
+                         w->gate_w, w->up_w, w->gate_up_w, w->gate_b, w->up_b, w->gate_up_b,
+                         w->down_w, w->down_b, w->gate_s, w->gate_z, w->up_s, w->up_z,
+                         w->down_s, w->down_z, w->shared_gate_w, w->shared_up_w, w->shared_down_w,
+                         w->latent_down_w, w->latent_up_w, w->latent_norm_w};
+    for (const void* p : all)
+        if (p && !aligned16(p)) return MOE_ERR_INVALID_ARGUMENT;
+    return MOE_OK;
+}
+
+moe_status check_tokens(const moe_config* c, int64_t T) {
+    if (T < 0) return MOE_ERR_INVALID_ARGUMENT;
+    const int64_t Kmax = std::max(std::max<int64_t>(c->hidden, c->intermediate), std::max<int64_t>(expert_in(*c), c->shared_intermediate));
+    if (T > (int64_t(1) << 26) || T * c->top_k >= (int64_t(1) << 31) || T * c->top_k * Kmax >= (int64_t(1) << 46))
+        return MOE_ERR_SHAPE_OVERFLOW;
+    return MOE_OK;
+}
+
+moe_status check_ptr(const void* p) {
+    if (!p) return MOE_ERR_INVALID_ARGUMENT;
+    return aligned16(p) ? MOE_OK : MOE_ERR_INVALID_ARGUMENT;
+}
+
+#define MOE_CHECK(expr)                          \
+    do {                                         \
+        const moe_status _s = (expr);            \
+        if (_s != MOE_OK) return _s;             \
+    } while (0)
+#define MOE_CUDA(expr)                                  \
+    do {                                                \
+        if ((expr) != cudaSuccess) return MOE_ERR_CUDA; \
+    } while (0)
+
+// Common preamble of every computing call: config, weights, tokens, workspace.
+moe_status prelude(const moe_config* c, const moe_weights* w, int64_t T, void* ws, size_t ws_bytes,
+                   WsLayout* L) {
+    MOE_CHECK(validate_config(c));
+    if (w) MOE_CHECK(validate_weights(c, w));
+    MOE_CHECK(check_tokens(c, T));
+    if (T == 0) return MOE_OK;
+    MOE_CHECK(check_ptr(ws));
+    *L = ws_layout(*c, T);
+    if (ws_bytes < L->total) return MOE_ERR_WORKSPACE_TOO_SMALL;
+    return MOE_OK;
+}
+
+template <typename P> P* at(void* ws, size_t off) { return reinterpret_cast<P*>(static_cast<char*>(ws) + off); }
+
+// a1 + a2
+moe_status run_route(const moe_config* c, const moe_weights* w, const void* x, int64_t T, int32_t* idx,
+                     float* wts, float* coef, float* zero, int64_t zero_cols, void* ws, const WsLayout& L,
+                     cudaStream_t s) {
+    const bool blend = c->shared_mode == MOE_SHARED_BLEND;
+    DenseGemvArgs r;
+    r.W0 = w->router_w;
+    r.b0 = c->has_router_bias ? w->router_b : nullptr;
+    r.rows0 = c->num_experts;
+    if (blend) {
+        r.W1 = w->coef_w;
+        r.b1 = w->coef_b;
+        r.rows1 = 2;
+    }
+    r.u = x;
+    r.T = T;
+    r.K = c->hidden;
+    r.out = at<float>(ws, L.logits);
+    r.ld_out = L.ld_logits;
+    r.out_f32 = 1;
+    r.act_dtype = c->act_dtype;
+    MOE_CUDA(launch_dense_gemv(r, s));
+    TopkArgs t;
+    t.logits = at<float>(ws, L.logits);
+    t.ld = L.ld_logits;
+    t.T = T;
+    t.E = c->num_experts;
+    t.k = c->top_k;
+    t.scoring = c->scoring;
+    t.norm = c->norm_topk_prob;
+    t.has_sel = c->has_selection_bias;
+    t.sel_bias = static_cast<const float*>(w->selection_bias);
+    t.blend = blend;
+    t.idx = idx;
+    t.w = wts;
+    t.coef = coef;
+    t.zero = zero;
+    t.zero_cols = zero_cols;
+    MOE_CUDA(launch_topk(t, s));
+    return MOE_OK;
+}
+
+// a3
+moe_status run_permute(const moe_config* c, const int32_t* idx, int64_t T, int32_t* offsets,
+                       int32_t* sorted_slot, int32_t* slot_pos, void* ws, const WsLayout& L, cudaStream_t s) {
+    PermuteArgs p;
+    p.idx = idx;
+    p.S = T * c->top_k;
+    p.E = c->num_experts;
+    p.offsets = offsets;
+    p.sorted_slot = sorted_slot;
+    p.slot_pos = slot_pos;
+    p.active = at<int32_t>(ws, L.active);
+    p.chunk_hist = at<int32_t>(ws, L.chunk_hist);
+    p.n_chunks = L.n_chunks;
+    p.status = at<int>(ws, L.status);
+    MOE_CUDA(launch_permute(p, s));
+    return MOE_OK;
+}
+
+// a4 + a5 (+ a6 when with_shared): y_acc must be zero on entry.
+moe_status run_experts(const moe_config* c, const moe_weights* w, const void* u, const void* x, int64_t T,
+                       const int32_t* offsets, const int32_t* sorted_slot, const float* topk_w,
+                       float* y_acc, bool with_routed, bool with_shared, void* ws, const WsLayout& L,
+                       cudaStream_t s) {
+    const int K = expert_in(*c);
+    const int64_t groups = with_routed ? std::min<int64_t>(c->num_experts, T * c->top_k) : 0;
+    const bool sh = with_shared && c->shared_mode != MOE_SHARED_NONE;
+    GateUpArgs g;
+    g.wf = c->weight_format;
+    g.interleaved = c->gate_up_interleaved;
+    g.has_bias = c->has_expert_bias;
+    g.group_size = c->group_size;
+    g.gate_w = w->gate_w; g.up_w = w->up_w; g.gate_up_w = w->gate_up_w;
+    g.gate_s = w->gate_s; g.gate_z = w->gate_z; g.up_s = w->up_s; g.up_z = w->up_z;
+    g.gate_b = w->gate_b; g.up_b = w->up_b; g.gate_up_b = w->gate_up_b;
+    g.offsets = offsets;
+    g.sorted_slot = sorted_slot;
+    g.active = at<int32_t>(ws, L.active);
+    g.k = c->top_k;
+    g.I = c->intermediate;
+    g.K = K;
+    g.routed_groups = int(groups);
+    g.u = u;
+    g.h = at<void>(ws, L.h);
+    if (sh) {
+        g.sg_w = w->shared_gate_w;
+        g.su_w = w->shared_up_w;
+        g.shared_I = c->shared_intermediate;
+        g.Hs = c->hidden;
+        g.xs = x;
+        g.hs = at<void>(ws, L.hs);
+    }
+    g.T = T;
+    g.act = c->activation;
+    g.limit = c->swiglu_limit;
+    g.alpha = c->swiglu_alpha;
+    MOE_CUDA(launch_gateup_gemv(g, s));
+    DownArgs d;
+    d.wf = c->weight_format;
+    d.has_bias = c->has_expert_bias;
+    d.group_size = c->group_size;
+    d.down_w = w->down_w; d.down_s = w->down_s; d.down_z = w->down_z; d.down_b = w->down_b;
+    d.offsets = offsets;
+    d.sorted_slot = sorted_slot;
+    d.active = at<int32_t>(ws, L.active);
+    d.topk_w = topk_w;
+    d.k = c->top_k;
+    d.I = c->intermediate;
+    d.K = K;
+    d.routed_groups = int(groups);
+    d.h = at<void>(ws, L.h);
+    d.y_acc = y_acc;
+    if (sh) {
+        d.sd_w = w->shared_down_w;
+        d.shared_I = c->shared_intermediate;
+        d.Hs = c->hidden;
+        d.hs = at<void>(ws, L.hs);
+        d.s_acc = at<float>(ws, L.s_acc);
+    }
+    d.T = T;
+    MOE_CUDA(launch_down_gemv(d, s));
+    return MOE_OK;
+}
+
+// a8 (first half): z = x Wdp^T
+moe_status run_latent_down(const moe_config* c, const moe_weights* w, const void* x, int64_t T, void* z,
+                           cudaStream_t s) {
+    DenseGemvArgs r;
+    r.W0 = w->latent_down_w;
+    r.rows0 = c->latent_dim;
+    r.u = x;
+    r.T = T;
+    r.K = c->hidden;
+    r.out = z;
+    r.ld_out = c->latent_dim;
+    r.out_f32 = 0;
+    r.act_dtype = c->act_dtype;
+    MOE_CUDA(launch_dense_gemv(r, s));
+    return MOE_OK;
+}
+
+// a7 (and the tail of a8): s_acc already holds the shared expert when shared_mode != NONE.
+moe_status run_output(const moe_config* c, const moe_weights* w, const float* y_acc, const float* coef,
+                      int64_t T, void* y, void* ws, const WsLayout& L, cudaStream_t s) {
+    const float* s_acc = c->shared_mode != MOE_SHARED_NONE ? at<float>(ws, L.s_acc) : nullptr;
+    if (!c->latent_dim) {
+        MOE_CUDA(launch_combine(y_acc, s_acc, coef, c->shared_mode, T, c->hidden, y, c->act_dtype, s));
+        return MOE_OK;
+    }
+    const void* n = y_acc;
+    bool n_f32 = true;
+    if (c->latent_use_norm) {
+        MOE_CUDA(launch_rmsnorm(y_acc, w->latent_norm_w, c->rms_eps, T, c->latent_dim, at<void>(ws, L.nrm),
+                                c->act_dtype, s));
+        n = at<void>(ws, L.nrm);
+        n_f32 = false;
+    }
+    if (n_f32) {
+        // no norm: round the routed latent sum to the activation dtype first
+        MOE_CUDA(launch_combine(y_acc, nullptr, nullptr, MOE_SHARED_NONE, T, c->latent_dim, at<void>(ws, L.nrm),
+                                c->act_dtype, s));
+        n = at<void>(ws, L.nrm);
+    }
+    if (c->shared_mode == MOE_SHARED_BLEND) return MOE_ERR_UNSUPPORTED;  // rejected earlier
+    DenseGemvArgs r;
+    r.W0 = w->latent_up_w;
+    r.rows0 = c->hidden;
+    r.u = n;
+    r.T = T;
+    r.K = c->latent_dim;
+    r.out = y;
+    r.ld_out = c->hidden;
+    r.out_f32 = c->act_dtype == MOE_DTYPE_F32;
+    r.addend = s_acc;
+    r.ld_add = c->hidden;
+    r.act_dtype = c->act_dtype;
+    MOE_CUDA(launch_dense_gemv(r, s));
+    return MOE_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+moe_status moe_config_validate(const moe_config* cfg) {
+    MOE_CHECK(validate_config(cfg));
+    if (cfg->latent_dim && cfg->shared_mode == MOE_SHARED_BLEND) return MOE_ERR_UNSUPPORTED;
+    return MOE_OK;
+}
+
+moe_status moe_weights_validate(const moe_config* cfg, const moe_weights* w) {
+    MOE_CHECK(moe_config_validate(cfg));
+    return validate_weights(cfg, w);
+}
+
+moe_status moe_workspace_size(const moe_config* cfg, int64_t max_tokens, size_t* bytes) {
+    MOE_CHECK(moe_config_validate(cfg));
+    if (!bytes) return MOE_ERR_INVALID_ARGUMENT;
+    MOE_CHECK(check_tokens(cfg, max_tokens));
+    *bytes = ws_layout(*cfg, max_tokens).total;
+    return MOE_OK;
+}
+
+moe_status moe_route(const moe_config* cfg, const moe_weights* w, const void* x, int64_t T, int32_t* topk_idx,
+                     float* topk_w, float* coef, void* ws, size_t ws_bytes, moe_stream_t stream) {
+    MOE_CHECK(moe_config_validate(cfg));
+    WsLayout L;
+    MOE_CHECK(prelude(cfg, w, T, ws, ws_bytes, &L));
+    if (T == 0) return MOE_OK;
+    MOE_CHECK(check_ptr(x));
+    MOE_CHECK(check_ptr(topk_idx));
+    MOE_CHECK(check_ptr(topk_w));
+    if (cfg->shared_mode == MOE_SHARED_BLEND) MOE_CHECK(check_ptr(coef));
+    return run_route(cfg, w, x, T, topk_idx, topk_w, coef, nullptr, 0, ws, L, (cudaStream_t)stream);
+}
+
+moe_status moe_permute(const moe_config* cfg, const int32_t* topk_idx, int64_t T, int32_t* expert_offsets,
+                       int32_t* sorted_slot, int32_t* slot_pos, void* ws, size_t ws_bytes, moe_stream_t stream) {
+    MOE_CHECK(moe_config_validate(cfg));
+    WsLayout L;
+    MOE_CHECK(prelude(cfg, nullptr, T, ws, ws_bytes, &L));
+    if (T == 0) return MOE_OK;
+    MOE_CHECK(check_ptr(topk_idx));
+    MOE_CHECK(check_ptr(expert_offsets));
+    MOE_CHECK(check_ptr(sorted_slot));
+    MOE_CHECK(check_ptr(slot_pos));
+    return run_permute(cfg, topk_idx, T, expert_offsets, sorted_slot, slot_pos, ws, L, (cudaStream_t)stream);
+}
+
+moe_status moe_grouped_ffn(const moe_config* cfg, const moe_weights* w, const void* u, int64_t T,
+                           const int32_t* expert_offsets, const int32_t* sorted_slot, const float* topk_w,
+                           float* y_acc, void* ws, size_t ws_bytes, moe_stream_t stream) {
+    MOE_CHECK(moe_config_validate(cfg));
+    WsLayout L;
+    MOE_CHECK(prelude(cfg, w, T, ws, ws_bytes, &L));
+    if (T == 0) return MOE_OK;
+    MOE_CHECK(check_ptr(u));
+    MOE_CHECK(check_ptr(expert_offsets));
+    MOE_CHECK(check_ptr(sorted_slot));
+    MOE_CHECK(check_ptr(topk_w));
+    MOE_CHECK(check_ptr(y_acc));
+    cudaStream_t s = (cudaStream_t)stream;
+    MOE_CUDA(cudaMemsetAsync(y_acc, 0, size_t(T) * expert_in(*cfg) * sizeof(float), s));
+    MOE_CUDA(launch_active_list(expert_offsets, cfg->num_experts, at<int32_t>(ws, L.active), s));
+    return run_experts(cfg, w, u, nullptr, T, expert_offsets, sorted_slot, topk_w, y_acc, true, false, ws, L, s);
+}
+
+moe_status moe_latent_down(const moe_config* cfg, const moe_weights* w, const void* x, int64_t T, void* z,
+                           void* ws, size_t ws_bytes, moe_stream_t stream) {
+    MOE_CHECK(moe_config_validate(cfg));
+    if (!cfg->latent_dim) return MOE_ERR_INVALID_ARGUMENT;
+    WsLayout L;
+    MOE_CHECK(prelude(cfg, w, T, ws, ws_bytes, &L));
+    if (T == 0) return MOE_OK;
+    MOE_CHECK(check_ptr(x));
+    MOE_CHECK(check_ptr(z));
+    return run_latent_down(cfg, w, x, T, z, (cudaStream_t)stream);
+}
+
+moe_status moe_combine(const moe_config* cfg, const moe_weights* w, const float* y_acc, const void* x,
+                       const float* coef, int64_t T, void* y, void* ws, size_t ws_bytes, moe_stream_t stream) {
+    MOE_CHECK(moe_config_validate(cfg));
+    WsLayout L;
+    MOE_CHECK(prelude(cfg, w, T, ws, ws_bytes, &L));
+    if (T == 0) return MOE_OK;
+    MOE_CHECK(check_ptr(y_acc));
+    MOE_CHECK(check_ptr(x));
+    MOE_CHECK(check_ptr(y));
+    if (cfg->shared_mode == MOE_SHARED_BLEND) MOE_CHECK(check_ptr(coef));
+    cudaStream_t s = (cudaStream_t)stream;
+    if (cfg->shared_mode != MOE_SHARED_NONE)
+        MOE_CHECK(run_experts(cfg, w, nullptr, x, T, nullptr, nullptr, nullptr, nullptr, false, true, ws, L, s));
+    return run_output(cfg, w, y_acc, coef, T, y, ws, L, s);
+}
+
+moe_status moe_block_forward(const moe_config* cfg, const moe_weights* w, const void* x, int64_t T, void* y,
+                             void* ws, size_t ws_bytes, moe_stream_t stream) {
+    MOE_CHECK(moe_config_validate(cfg));
+    WsLayout L;
+    MOE_CHECK(prelude(cfg, w, T, ws, ws_bytes, &L));
+    if (T == 0) return MOE_OK;
+    MOE_CHECK(check_ptr(x));
+    MOE_CHECK(check_ptr(y));
+    cudaStream_t s = (cudaStream_t)stream;
+    const int K = expert_in(*cfg);
+    float* y_acc = at<float>(ws, L.y_acc);
+    int32_t* idx = at<int32_t>(ws, L.topk_idx);
+    float* wts = at<float>(ws, L.topk_w);
+    float* coef = at<float>(ws, L.coef);
+    MOE_CHECK(run_route(cfg, w, x, T, idx, wts, coef, y_acc, K, ws, L, s));
+    const void* u = x;
+    if (cfg->latent_dim) {
+        MOE_CHECK(run_latent_down(cfg, w, x, T, at<void>(ws, L.z), s));
+        u = at<void>(ws, L.z);
+    }
+    int32_t* offsets = at<int32_t>(ws, L.offsets);
+    int32_t* sorted_slot = at<int32_t>(ws, L.sorted_slot);
+    MOE_CHECK(run_permute(cfg, idx, T, offsets, sorted_slot, at<int32_t>(ws, L.slot_pos), ws, L, s));
+    MOE_CHECK(run_experts(cfg, w, u, x, T, offsets, sorted_slot, wts, y_acc, true, true, ws, L, s));
+    return run_output(cfg, w, y_acc, coef, T, y, ws, L, s);
+}
+
+moe_status moe_read_device_status(void* ws, moe_stream_t stream) {
+    if (!ws) return MOE_ERR_INVALID_ARGUMENT;
+    int status = 0;
+    cudaStream_t s = (cudaStream_t)stream;
+    MOE_CUDA(cudaMemcpyAsync(&status, ws, sizeof(int), cudaMemcpyDeviceToHost, s));
+    MOE_CUDA(cudaStreamSynchronize(s));
+    MOE_CUDA(cudaMemsetAsync(ws, 0, sizeof(int), s));
+    MOE_CUDA(cudaStreamSynchronize(s));
+    if (status == MOE_ERR_DEVICE_CHECK || status == MOE_ERR_DEVICE_TIMEOUT) return moe_status(status);
+    return status == 0 ? MOE_OK : MOE_ERR_CUDA;
+}
+
+moe_status moe_clear_device_status(void* ws, moe_stream_t stream) {
+    if (!ws) return MOE_ERR_INVALID_ARGUMENT;
+    MOE_CUDA(cudaMemsetAsync(ws, 0, sizeof(int), (cudaStream_t)stream));
+    return MOE_OK;
+}
+
+const char* moe_status_string(moe_status s) {
+    switch (s) {
+        case MOE_OK: return "ok";
+        case MOE_ERR_INVALID_ARGUMENT: return "invalid argument";
+        case MOE_ERR_SHAPE_OVERFLOW: return "shape overflow";
+        case MOE_ERR_INVALID_QUANTIZATION: return "invalid quantization parameters";
+        case MOE_ERR_MISSING_TENSOR: return "missing tensor";
+        case MOE_ERR_UNSUPPORTED: return "unsupported configuration";
+        case MOE_ERR_CUDA: return "CUDA error";
+        case MOE_ERR_DEVICE_CHECK: return "device-side check failed (expert id out of range)";
+        case MOE_ERR_DEVICE_TIMEOUT: return "device-side wait timed out";
+        case MOE_ERR_WORKSPACE_TOO_SMALL: return "workspace too small";
+    }
+    return "unknown status";
+}
+
+}  // extern "C"

@@ -1,0 +1,92 @@
+// combine.cu -- routed/shared combine (a7) and the latent RMSNorm (a8).
+//
+// Klear PR item 2: y = y_experts * coef[0] + shared * coef[1] (blend); ferrox
+// latent_moe.rs: output = routed_out + shared (add), and
+// combined = rms_norm(combined) with a [latent] weight before up_proj.
+#include <algorithm>
+
+#include "common.cuh"
+#include "internal.h"
+
+namespace moe {
+
+namespace {
+
+template <typename AT>
+__global__ void __launch_bounds__(256) combine_kernel(const float* __restrict__ y_acc,
+                                                      const float* __restrict__ s_acc,
+                                                      const float* __restrict__ coef, int mode,
+                                                      int64_t T, int H, AT* __restrict__ y) {
+    const int64_t n4 = T * H / 4;
+    for (int64_t i = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; i < n4;
+         i += int64_t(gridDim.x) * blockDim.x) {
+        const int64_t t = (i * 4) / H;
+        float4 r = reinterpret_cast<const float4*>(y_acc)[i];
+        if (mode != MOE_SHARED_NONE) {
+            const float4 sv = reinterpret_cast<const float4*>(s_acc)[i];
+            if (mode == MOE_SHARED_ADD) {
+                r.x += sv.x; r.y += sv.y; r.z += sv.z; r.w += sv.w;
+            } else {
+                const float c0 = coef[2 * t], c1 = coef[2 * t + 1];
+                r.x = r.x * c0 + sv.x * c1;
+                r.y = r.y * c0 + sv.y * c1;
+                r.z = r.z * c0 + sv.z * c1;
+                r.w = r.w * c0 + sv.w * c1;
+            }
+        }
+        AT* o = y + i * 4;
+        o[0] = from_f<AT>(r.x);
+        o[1] = from_f<AT>(r.y);
+        o[2] = from_f<AT>(r.z);
+        o[3] = from_f<AT>(r.w);
+    }
+}
+
+template <typename AT>
+__global__ void __launch_bounds__(256) rmsnorm_kernel(const float* __restrict__ y_acc,
+                                                      const AT* __restrict__ gamma, float eps,
+                                                      int L, AT* __restrict__ out) {
+    __shared__ float red[8];
+    const int64_t t = blockIdx.x;
+    const float* row = y_acc + t * L;
+    float ss = 0.f;
+    for (int c = threadIdx.x; c < L; c += blockDim.x) ss = fmaf(row[c], row[c], ss);
+    ss = warp_sum(ss);
+    if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = ss;
+    __syncthreads();
+    float tot = 0.f;
+#pragma unroll
+    for (int w = 0; w < 8; ++w) tot += red[w];
+    const float inv = rsqrtf(tot / float(L) + eps);
+    for (int c = threadIdx.x; c < L; c += blockDim.x)
+        out[t * L + c] = from_f<AT>(row[c] * inv * to_f<AT>(gamma[c]));
+}
+
+}  // namespace
+
+cudaError_t launch_combine(const float* y_acc, const float* s_acc, const float* coef, int mode,
+                           int64_t T, int H, void* y, int act_dtype, cudaStream_t s) {
+    if (T == 0) return cudaSuccess;
+    const int64_t n4 = T * H / 4;
+    const unsigned grid = unsigned(std::min<int64_t>((n4 + 255) / 256, 148 * 16));
+    if (act_dtype == kF32)
+        combine_kernel<float><<<grid, 256, 0, s>>>(y_acc, s_acc, coef, mode, T, H, static_cast<float*>(y));
+    else
+        combine_kernel<__nv_bfloat16><<<grid, 256, 0, s>>>(y_acc, s_acc, coef, mode, T, H,
+                                                           static_cast<__nv_bfloat16*>(y));
+    return cudaGetLastError();
+}
+
+cudaError_t launch_rmsnorm(const float* y_acc, const void* gamma, float eps, int64_t T, int L,
+                           void* out, int act_dtype, cudaStream_t s) {
+    if (T == 0) return cudaSuccess;
+    if (act_dtype == kF32)
+        rmsnorm_kernel<float><<<unsigned(T), 256, 0, s>>>(y_acc, static_cast<const float*>(gamma), eps, L,
+                                                          static_cast<float*>(out));
+    else
+        rmsnorm_kernel<__nv_bfloat16><<<unsigned(T), 256, 0, s>>>(
+            y_acc, static_cast<const __nv_bfloat16*>(gamma), eps, L, static_cast<__nv_bfloat16*>(out));
+    return cudaGetLastError();
+}
+
+}  // namespace moe

@@ -1,0 +1,112 @@
+// common.cuh -- internal helpers shared by the library's CUDA sources.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/moe.h"
+
+namespace moe {
+
+constexpr int kWarp = 32;
+constexpr int kMaxTopK = 16;
+constexpr int kMaxExperts = 512;
+
+// Weight formats / act dtypes (same integers as enum moe_dtype).
+constexpr int kF32 = MOE_DTYPE_F32;
+constexpr int kBF16 = MOE_DTYPE_BF16;
+constexpr int kQ4 = MOE_DTYPE_Q4_AFFINE;
+
+// ---------------------------------------------------------------- workspace
+// Every call carves its scratch out of the caller's workspace at fixed
+// 256-byte-aligned offsets that depend only on (config, max_tokens).
+struct WsLayout {
+    size_t status;       // int32 status word (+ pad)
+    size_t logits;       // f32 [T, ld_logits]: E router logits, then 2 coefficient logits
+    size_t topk_idx;     // int32 [T, k]
+    size_t topk_w;       // f32 [T, k]
+    size_t coef;         // f32 [T, 2]
+    size_t offsets;      // int32 [E + 1]
+    size_t sorted_slot;  // int32 [T * k]
+    size_t slot_pos;     // int32 [T * k]
+    size_t active;       // int32 [E + 1]: n_active, then the active expert ids
+    size_t chunk_hist;   // int32 [n_chunks, E]
+    size_t h;            // act [T * k, I]: routed intermediate, sorted order
+    size_t hs;           // act [T, Is]: shared intermediate
+    size_t y_acc;        // f32 [T, K]: routed sum
+    size_t s_acc;        // f32 [T, H]: shared expert output
+    size_t z;            // act [T, L]: latent input of the experts
+    size_t nrm;          // act [T, L]: normalised latent
+    size_t uperm;        // bf16 [T * k, K]: expert inputs gathered in sorted order
+    size_t tiles;        // int32 tile list of the tensor-core path
+    size_t total;
+    int ld_logits;
+    int n_chunks;
+    int64_t T;
+};
+
+constexpr int kPermChunk = 2048;  // slots per permutation chunk
+
+inline size_t align256(size_t v) { return (v + 255) & ~size_t(255); }
+inline int act_bytes(const moe_config& c) { return c.act_dtype == kF32 ? 4 : 2; }
+inline int expert_in(const moe_config& c) { return c.latent_dim ? c.latent_dim : c.hidden; }
+
+// Upper bound of tensor-core tiles for the routed gate/up and down GEMMs.
+int64_t max_routed_tiles(const moe_config& c, int64_t T);
+
+WsLayout ws_layout(const moe_config& c, int64_t T);
+
+// ---------------------------------------------------------------- device helpers
+__device__ __forceinline__ uint4 ld_stream16(const void* p) {
+    uint4 r;
+    asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w) : "l"(p));
+    return r;
+}
+
+__device__ __forceinline__ float bf16lo(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf16hi(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
+
+__device__ __forceinline__ void unpack8(const uint4 v, float (&f)[8]) {
+    f[0] = bf16lo(v.x); f[1] = bf16hi(v.x); f[2] = bf16lo(v.y); f[3] = bf16hi(v.y);
+    f[4] = bf16lo(v.z); f[5] = bf16hi(v.z); f[6] = bf16lo(v.w); f[7] = bf16hi(v.w);
+}
+
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+    return v;
+}
+
+__device__ __forceinline__ float warp_max(float v) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+    return v;
+}
+
+template <typename AT> __device__ __forceinline__ float to_f(AT v);
+template <> __device__ __forceinline__ float to_f<float>(float v) { return v; }
+template <> __device__ __forceinline__ float to_f<__nv_bfloat16>(__nv_bfloat16 v) {
+    return __bfloat162float(v);
+}
+template <typename AT> __device__ __forceinline__ AT from_f(float v);
+template <> __device__ __forceinline__ float from_f<float>(float v) { return v; }
+template <> __device__ __forceinline__ __nv_bfloat16 from_f<__nv_bfloat16>(float v) {
+    return __float2bfloat16_rn(v);
+}
+
+// SwiGLU / clamped SwiGLU on fp32 pre-activations.
+__device__ __forceinline__ float act_apply(int act, float g, float v, float limit, float alpha) {
+    if (act == MOE_ACT_SWIGLU) return g / (1.0f + expf(-g)) * v;
+    float gc = fminf(g, limit);
+    float vc = fminf(fmaxf(v, -limit), limit);
+    return gc / (1.0f + expf(-alpha * gc)) * (vc + 1.0f);
+}
+
+// Sticky device status word (first error wins).
+__device__ __forceinline__ void set_status(int* status, int code) {
+    if (status) atomicCAS(status, 0, code);
+}
+
+}  // namespace moe

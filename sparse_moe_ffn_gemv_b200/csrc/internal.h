@@ -1,0 +1,80 @@
+// internal.h -- host-side launchers shared by the library's translation units.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/moe.h"
+
+namespace moe {
+
+// out[t, r] = sum_c W[r, c] u[t, c] (+ bias[r]) (+ addend[t, r]) for the rows of
+// W0 followed by the rows of W1 (the router and the coefficient head share a pass).
+struct DenseGemvArgs {
+    const void* W0 = nullptr; const void* b0 = nullptr; int rows0 = 0;
+    const void* W1 = nullptr; const void* b1 = nullptr; int rows1 = 0;
+    const void* u = nullptr; int64_t T = 0; int K = 0;
+    void* out = nullptr; int ld_out = 0; int out_f32 = 0;
+    const float* addend = nullptr; int ld_add = 0;
+    int act_dtype = MOE_DTYPE_BF16;
+};
+cudaError_t launch_dense_gemv(const DenseGemvArgs& a, cudaStream_t s);
+
+struct TopkArgs {
+    const float* logits = nullptr; int ld = 0; int64_t T = 0;
+    int E = 0, k = 0, scoring = 0, norm = 0, has_sel = 0, blend = 0;
+    const float* sel_bias = nullptr;
+    int32_t* idx = nullptr; float* w = nullptr; float* coef = nullptr;
+    float* zero = nullptr; int64_t zero_cols = 0;  // rows of this buffer are cleared per token
+};
+cudaError_t launch_topk(const TopkArgs& a, cudaStream_t s);
+
+struct PermuteArgs {
+    const int32_t* idx = nullptr; int64_t S = 0; int E = 0;
+    int32_t* offsets = nullptr; int32_t* sorted_slot = nullptr; int32_t* slot_pos = nullptr;
+    int32_t* active = nullptr; int32_t* chunk_hist = nullptr; int n_chunks = 0;
+    int* status = nullptr;
+};
+cudaError_t launch_permute(const PermuteArgs& a, cudaStream_t s);
+// active[0] = number of experts with tokens, active[1..] their ids, from offsets [E + 1].
+cudaError_t launch_active_list(const int32_t* offsets, int E, int32_t* active, cudaStream_t s);
+
+// Routed + shared gate/up on CUDA cores: h = act(Wg u + bg, Wu u + bu).
+struct GateUpArgs {
+    int wf = MOE_DTYPE_BF16, interleaved = 0, has_bias = 0, group_size = 64;
+    const void *gate_w = nullptr, *up_w = nullptr, *gate_up_w = nullptr;
+    const void *gate_s = nullptr, *gate_z = nullptr, *up_s = nullptr, *up_z = nullptr;
+    const void *gate_b = nullptr, *up_b = nullptr, *gate_up_b = nullptr;
+    const int32_t *offsets = nullptr, *sorted_slot = nullptr, *active = nullptr;
+    int k = 1, I = 0, K = 0, routed_groups = 0;  // routed_groups: bound on active experts
+    const void* u = nullptr; void* h = nullptr;
+    // shared expert (dense group over all T tokens), shared_I == 0 disables it
+    const void *sg_w = nullptr, *su_w = nullptr; int shared_I = 0, Hs = 0;
+    const void* xs = nullptr; void* hs = nullptr;
+    int64_t T = 0;
+    int act = 0; float limit = 7.f, alpha = 1.702f;
+};
+cudaError_t launch_gateup_gemv(const GateUpArgs& a, cudaStream_t s);
+
+// Routed + shared down on CUDA cores: y_acc[token] += w * (Wd h + bd); s_acc = Wsd hs.
+struct DownArgs {
+    int wf = MOE_DTYPE_BF16, has_bias = 0, group_size = 64;
+    const void *down_w = nullptr, *down_s = nullptr, *down_z = nullptr, *down_b = nullptr;
+    const int32_t *offsets = nullptr, *sorted_slot = nullptr, *active = nullptr;
+    const float* topk_w = nullptr;
+    int k = 1, I = 0, K = 0, routed_groups = 0;
+    const void* h = nullptr; float* y_acc = nullptr;
+    const void* sd_w = nullptr; int shared_I = 0, Hs = 0; const void* hs = nullptr;
+    float* s_acc = nullptr;
+    int64_t T = 0;
+};
+cudaError_t launch_down_gemv(const DownArgs& a, cudaStream_t s);
+
+// y = y_acc | y_acc + s | c0 y_acc + c1 s, stored in act dtype.
+cudaError_t launch_combine(const float* y_acc, const float* s_acc, const float* coef, int mode,
+                           int64_t T, int H, void* y, int act_dtype, cudaStream_t s);
+// nrm = y_acc / sqrt(mean(y_acc^2) + eps) * gamma (act dtype), per token row of width L.
+cudaError_t launch_rmsnorm(const float* y_acc, const void* gamma, float eps, int64_t T, int L,
+                           void* out, int act_dtype, cudaStream_t s);
+
+}  // namespace moe

@@ -1,0 +1,221 @@
+"""CUDA path vs the fp64 oracle, element by element, through the C ABI (GPU only).
+
+Small cases compare every token; full-size cases (the launch configurations
+the benchmark times) compare the expert choice of every token and the outputs
+of sampled tokens (the block is per-token independent, so a sample is exact).
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from parity import check_block
+from sparse_moe_ffn_gemv_b200 import inputs
+from sparse_moe_ffn_gemv_b200 import moe as M
+import tiny_specs as ts
+
+pytestmark = pytest.mark.gpu
+
+_W_CACHE = {}
+
+
+def weights(spec):
+    key = spec.name
+    if key not in _W_CACHE:
+        _W_CACHE.clear()          # keep one big weight set in host memory at a time
+        cpu = inputs.make_weights(spec)
+        _W_CACHE[key] = (cpu, {k: inputs.to_numpy_storage(v) for k, v in cpu.items()})
+    return _W_CACHE[key]
+
+
+def run_gpu(spec, wcpu, x_cpu, block=None):
+    T = x_cpu.shape[0]
+    blk = block or M.MoeBlock(spec, wcpu, max_tokens=T)
+    x = x_cpu.cuda()
+    y = blk.forward(x)
+    idx = torch.empty((T, spec.top_k), dtype=torch.int32, device="cuda")
+    w = torch.empty((T, spec.top_k), dtype=torch.float32, device="cuda")
+    coef = torch.empty((T, 2), dtype=torch.float32, device="cuda")
+    M.moe_route(blk.cfg, blk.w, x, T, idx, w, coef, blk.ws)
+    torch.cuda.synchronize()
+    assert blk.device_status() == 0
+    return (y.float().cpu().numpy(), idx.cpu().numpy(), w.cpu().numpy(), coef.cpu().numpy())
+
+
+def full_check(spec, T, x_scale=1.0, wnp_override=None):
+    wcpu, wnp = weights(spec) if wnp_override is None else wnp_override
+    x_cpu = inputs.make_x(spec, T, x_scale)
+    x_np = inputs.to_numpy_storage(x_cpu)
+    y, idx, w, coef = run_gpu(spec, wcpu, x_cpu)
+    orc = oracle.forward(spec, wnp, x_np)
+    res = check_block(spec, wnp, x_np, np.arange(T), y, idx, orc=orc, label=f"{spec.name} T={T}")
+    # combine weights and blend coefficients where the expert sets agree
+    for t in range(T):
+        if set(idx[t]) == set(orc["idx"][t]):
+            pos = {e: j for j, e in enumerate(orc["idx"][t])}
+            ow = np.array([orc["w"][t][pos[e]] for e in idx[t]])
+            np.testing.assert_allclose(w[t], ow, rtol=2e-5, atol=1e-6)
+    if spec.shared_mode == "blend":
+        np.testing.assert_allclose(coef, orc["coef"], rtol=1e-4, atol=1e-6)
+    return res
+
+
+SMALL = [
+    (inputs.TINY_F32, 16, 1.0),
+    (ts.SIG_BLEND, 13, 1.0),
+    (ts.CLAMPED, 11, 60.0),
+    (ts.Q4, 9, 1.0),
+    (ts.LATENT, 10, 1.0),
+    (ts.ROUTER_BIAS, 12, 1.0),
+    (ts.SEPARATE_BIAS, 7, 1.0),
+    (ts.LATENT_NONORM, 5, 1.0),
+    (inputs.TINY_F32, 64, 1.0),          # 16 tokens per expert: several token passes
+    (inputs.KLEAR_BF16, 1, 1.0),
+    (inputs.KLEAR_BF16, 8, 1.0),
+    (inputs.KLEAR_BF16, 37, 1.0),
+    (inputs.KLEAR_BF16, 64, 1.0),
+    (inputs.KLEAR_Q4, 1, 1.0),
+    (inputs.KLEAR_Q4, 32, 1.0),
+    (inputs.CLAMPED_BF16, 1, 1.0),
+    (inputs.CLAMPED_BF16, 8, 1.0),
+    (inputs.CLAMPED_BF16, 8, 8.0),       # clamp stress: x * 8 engages the +-7 clamp
+    (inputs.LATENT_BF16, 1, 1.0),
+    (inputs.LATENT_BF16, 9, 1.0),
+]
+
+
+@pytest.mark.parametrize("spec,T,scale", SMALL, ids=[f"{s.name}-T{T}-x{sc:g}" for s, T, sc in SMALL])
+def test_block_matches_oracle_small(spec, T, scale):
+    full_check(spec, T, scale)
+
+
+FULL = [  # (spec, T, sampled tokens for the output check)
+    (inputs.KLEAR_BF16, 4096, 48),
+    (inputs.KLEAR_Q4, 2048, 32),
+    (inputs.CLAMPED_BF16, 8192, 16),
+    (inputs.LATENT_BF16, 128, 24),
+    (inputs.LATENT_BF16, 8192, 8),
+]
+
+
+@pytest.mark.slow
+@pytest.mark.parametrize("spec,T,n_sample", FULL, ids=[f"{s.name}-T{T}" for s, T, _ in FULL])
+def test_block_matches_oracle_full_size(spec, T, n_sample):
+    wcpu, wnp = weights(spec)
+    x_cpu = inputs.make_x(spec, T)
+    x_np = inputs.to_numpy_storage(x_cpu)
+    y, idx, _, _ = run_gpu(spec, wcpu, x_cpu)
+    # expert choice of every token
+    routed = oracle.forward(spec, wnp, x_np, route_only=True)
+    from parity import index_mismatches
+    ties = index_mismatches(idx, routed, spec.top_k)
+    assert len(ties) <= max(2, T // 200)
+    # outputs of sampled tokens: first, last, and a seeded spread (ragged tail included)
+    rng = np.random.default_rng(T)
+    tokens = np.unique(np.concatenate([[0, T - 1], rng.choice(T, size=n_sample - 2, replace=False)]))
+    check_block(spec, wnp, x_np, tokens, y[tokens], idx[tokens], label=f"{spec.name} T={T}")
+
+
+def test_all_tokens_routed_to_one_expert():
+    """Degenerate routing: a huge select-only bias puts expert 3 in every token's set,
+    so one group holds every token."""
+    spec = inputs.KLEAR_BF16
+    wcpu, wnp = weights(spec)
+    wcpu = dict(wcpu)
+    sb = wcpu["selection_bias"].clone()
+    sb[3] = 10.0
+    wcpu["selection_bias"] = sb
+    wnp = dict(wnp, selection_bias=sb.numpy())
+    T = 300
+    x_cpu = inputs.make_x(spec, T)
+    y, idx, _, _ = run_gpu(spec, wcpu, x_cpu)
+    assert (idx == 3).any(axis=1).all()
+    x_np = inputs.to_numpy_storage(x_cpu)
+    tokens = np.arange(0, T, 7)
+    check_block(spec, wnp, x_np, tokens, y[tokens], idx[tokens], label="one-expert")
+
+
+@pytest.mark.parametrize("spec", [ts.SIG_BLEND.replace(top_k=6, name="t_kE", config_id=120),
+                                  inputs.TINY_F32.replace(num_experts=1, top_k=1, name="t_E1",
+                                                          config_id=121)],
+                         ids=["k_equals_E", "single_expert"])
+def test_degenerate_expert_counts(spec):
+    full_check(spec, 9)
+
+
+def test_stepwise_calls_equal_block_forward_and_permutation_is_exact():
+    spec = inputs.KLEAR_BF16
+    wcpu, _ = weights(spec)
+    T, k, E, H = 70, spec.top_k, spec.num_experts, spec.hidden
+    blk = M.MoeBlock(spec, wcpu, max_tokens=T)
+    x = inputs.make_x(spec, T).cuda()
+    y_block = blk.forward(x).float()
+    dev = dict(dtype=torch.int32, device="cuda")
+    idx = torch.empty((T, k), **dev)
+    w = torch.empty((T, k), dtype=torch.float32, device="cuda")
+    coef = torch.empty((T, 2), dtype=torch.float32, device="cuda")
+    off = torch.empty(E + 1, **dev)
+    ss = torch.empty(T * k, **dev)
+    sp = torch.empty(T * k, **dev)
+    y_acc = torch.empty((T, H), dtype=torch.float32, device="cuda")
+    y = torch.empty((T, H), dtype=torch.bfloat16, device="cuda")
+    M.moe_route(blk.cfg, blk.w, x, T, idx, w, coef, blk.ws)
+    M.moe_permute(blk.cfg, idx, T, off, ss, sp, blk.ws)
+    M.moe_grouped_ffn(blk.cfg, blk.w, x, T, off, ss, w, y_acc, blk.ws)
+    M.moe_combine(blk.cfg, blk.w, y_acc, x, coef, T, y, blk.ws)
+    torch.cuda.synchronize()
+    o_off, o_ss, o_sp = oracle.permute(idx.cpu().numpy(), E)
+    np.testing.assert_array_equal(off.cpu().numpy(), o_off)
+    np.testing.assert_array_equal(ss.cpu().numpy(), o_ss)
+    np.testing.assert_array_equal(sp.cpu().numpy(), o_sp)
+    rms = float(y_block.pow(2).mean().sqrt())
+    assert float((y.float() - y_block).abs().max()) <= 1e-2 * rms
+
+
+def test_permutation_bit_exact_across_chunks():
+    """More than one 2048-slot chunk, ragged tail, empty experts."""
+    spec = inputs.KLEAR_BF16
+    cfg = M.config_from_spec(spec)
+    T, k, E = 1000, spec.top_k, spec.num_experts
+    g = torch.Generator().manual_seed(5)
+    idx = torch.stack([torch.randperm(E, generator=g)[:k] for _ in range(T)]).to(torch.int32)
+    idx[idx == 17] = 16    # expert 17 empty, 16 doubled in some rows -> still valid ids
+    ws = torch.zeros(M.moe_workspace_size(cfg, T), dtype=torch.uint8, device="cuda")
+    dev = dict(dtype=torch.int32, device="cuda")
+    off, ss, sp = torch.empty(E + 1, **dev), torch.empty(T * k, **dev), torch.empty(T * k, **dev)
+    M.moe_permute(cfg, idx.cuda(), T, off, ss, sp, ws)
+    torch.cuda.synchronize()
+    o_off, o_ss, o_sp = oracle.permute(idx.numpy(), E)
+    np.testing.assert_array_equal(off.cpu().numpy(), o_off)
+    np.testing.assert_array_equal(ss.cpu().numpy(), o_ss)
+    np.testing.assert_array_equal(sp.cpu().numpy(), o_sp)
+    assert M.moe_read_device_status(ws) == 0
+
+
+def test_out_of_range_expert_id_sets_the_device_status():
+    spec = inputs.KLEAR_BF16
+    cfg = M.config_from_spec(spec)
+    T, k, E = 4, spec.top_k, spec.num_experts
+    idx = torch.arange(T * k, dtype=torch.int32).reshape(T, k)
+    idx[2, 5] = 999
+    ws = torch.zeros(M.moe_workspace_size(cfg, T), dtype=torch.uint8, device="cuda")
+    dev = dict(dtype=torch.int32, device="cuda")
+    off, ss, sp = torch.empty(E + 1, **dev), torch.empty(T * k, **dev), torch.empty(T * k, **dev)
+    M.moe_permute(cfg, idx.cuda(), T, off, ss, sp, ws)
+    assert M.STATUS[M.moe_read_device_status(ws)] == "MOE_ERR_DEVICE_CHECK"
+    assert M.moe_read_device_status(ws) == 0       # read clears it
+    assert int(off[-1]) == T * k - 1                # the bad slot was dropped
+
+
+def test_batch_equals_tokens_one_at_a_time_on_gpu():
+    """Klear PR validation (causality check): a token's output does not depend on the batch."""
+    spec = inputs.KLEAR_BF16
+    wcpu, _ = weights(spec)
+    T = 24
+    blk = M.MoeBlock(spec, wcpu, max_tokens=T)
+    x = inputs.make_x(spec, T).cuda()
+    y = blk.forward(x).float()
+    rms = float(y.pow(2).mean().sqrt())
+    for t in (0, 5, 23):
+        y1 = blk.forward(x[t:t + 1].contiguous()).float()
+        assert float((y1[0] - y[t]).abs().max()) <= 2e-2 * rms

@@ -26,7 +26,7 @@ Q4 = MoeSpec(
 LATENT = MoeSpec(
     name="t_latent", config_id=104, hidden=48, num_experts=6, top_k=2, intermediate=16,
     scoring="sigmoid", has_selection_bias=True, norm_topk_prob=True, shared_mode="add",
-    shared_intermediate=20, latent_dim=24, latent_use_norm=True)
+    shared_intermediate=24, latent_dim=24, latent_use_norm=True)
 ROUTER_BIAS = MoeSpec(
     name="t_router_bias", config_id=105, hidden=32, num_experts=7, top_k=3, intermediate=8,
     scoring="softmax_all", has_router_bias=True, norm_topk_prob=True, shared_mode="add",
