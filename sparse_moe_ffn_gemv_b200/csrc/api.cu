@@ -7,6 +7,7 @@
 // an abort crossing the boundary).
 #include <algorithm>
 #include <cmath>
+#include <cstdlib>
 #include <cstring>
 
 #include "common.cuh"
@@ -15,9 +16,8 @@
 namespace moe {
 
 int64_t max_routed_tiles(const moe_config& c, int64_t T) {
-    (void)c;
-    (void)T;
-    return 0;
+    const int64_t S = T * c.top_k;
+    return (S + kTcBN - 1) / kTcBN + std::min<int64_t>(c.num_experts, S);
 }
 
 WsLayout ws_layout(const moe_config& c, int64_t T) {
@@ -50,8 +50,9 @@ WsLayout ws_layout(const moe_config& c, int64_t T) {
     L.s_acc = take(c.shared_mode != MOE_SHARED_NONE ? T * H * 4 : 0);
     L.z = take(Ld ? T * Ld * ab : 0);
     L.nrm = take(Ld ? T * Ld * ab : 0);
-    L.uperm = take(0);
-    L.tiles = take(0);
+    const bool tc = c.act_dtype == MOE_DTYPE_BF16 && c.weight_format == MOE_DTYPE_BF16;
+    L.uperm = take(tc ? T * k * K * 2 : 0);
+    L.tiles = take((E + 1) * 4);
     L.total = off;
     return L;
 }
@@ -160,6 +161,29 @@ moe_status check_ptr(const void* p) {
     return aligned16(p) ? MOE_OK : MOE_ERR_INVALID_ARGUMENT;
 }
 
+// Which engine runs a GEMM: weight-streaming CUDA-core kernels (few tokens per
+// weight row) or the tcgen05 tensor-core kernel (many). MOE_PATH=gemv|tc forces one
+// where both are possible (used by the tests to cross-check the two).
+enum { kPathAuto = 0, kPathGemv = 1, kPathTc = 2 };
+int path_override() {
+    const char* e = getenv("MOE_PATH");
+    if (!e) return kPathAuto;
+    if (!strcmp(e, "gemv")) return kPathGemv;
+    if (!strcmp(e, "tc")) return kPathTc;
+    return kPathAuto;
+}
+bool dense_tc(const moe_config* c, int64_t T, int K) {
+    if (c->act_dtype != MOE_DTYPE_BF16 || K % 64 != 0) return false;
+    const int o = path_override();
+    return o == kPathTc || (o == kPathAuto && T >= 64);
+}
+bool routed_tc(const moe_config* c, int64_t T) {
+    if (c->act_dtype != MOE_DTYPE_BF16 || c->weight_format != MOE_DTYPE_BF16) return false;
+    if (expert_in(*c) % 64 != 0 || c->intermediate % 64 != 0) return false;
+    const int o = path_override();
+    return o == kPathTc || (o == kPathAuto && T * c->top_k >= 8 * int64_t(c->num_experts));
+}
+
 #define MOE_CHECK(expr)                          \
     do {                                         \
         const moe_status _s = (expr);            \
@@ -206,7 +230,31 @@ moe_status run_route(const moe_config* c, const moe_weights* w, const void* x, i
     r.ld_out = L.ld_logits;
     r.out_f32 = 1;
     r.act_dtype = c->act_dtype;
-    MOE_CUDA(launch_dense_gemv(r, s));
+    if (dense_tc(c, T, c->hidden)) {
+        TcParams P;
+        const int np = blend ? 2 : 1;
+        for (int i = 0; i < np; ++i) {
+            TcProblem& p = P.p[i];
+            p.mode = kEpiStoreF32;
+            p.M = i == 0 ? c->num_experts : 2;
+            p.K = c->hidden;
+            p.m_blocks = (p.M + 127) / 128;
+            p.rows = int(T);
+            p.n_tiles = int((T + kTcBN - 1) / kTcBN);
+            p.bias0 = i == 0 ? r.b0 : r.b1;
+            p.out = at<float>(ws, L.logits) + (i == 0 ? 0 : c->num_experts);
+            p.ld_out = L.ld_logits;
+            if (!tc_weight_map(&P.a0[i], i == 0 ? r.W0 : r.W1, 1, p.M, c->hidden, false) ||
+                !tc_token_map(&P.b[i], x, T, c->hidden, kTcBN))
+                return MOE_ERR_CUDA;
+        }
+        P.nprob = np;
+        P.status = at<int>(ws, L.status);
+        const int64_t tiles = int64_t(P.p[0].m_blocks) * P.p[0].n_tiles + (np > 1 ? P.p[1].n_tiles : 0);
+        MOE_CUDA(launch_tc_gemm(P, false, tiles, s));
+    } else {
+        MOE_CUDA(launch_dense_gemv(r, s));
+    }
     TopkArgs t;
     t.logits = at<float>(ws, L.logits);
     t.ld = L.ld_logits;
@@ -229,7 +277,8 @@ moe_status run_route(const moe_config* c, const moe_weights* w, const void* x, i
 
 // a3
 moe_status run_permute(const moe_config* c, const int32_t* idx, int64_t T, int32_t* offsets,
-                       int32_t* sorted_slot, int32_t* slot_pos, void* ws, const WsLayout& L, cudaStream_t s) {
+                       int32_t* sorted_slot, int32_t* slot_pos, void* ws, const WsLayout& L, cudaStream_t s,
+                       bool tc_tiles) {
     PermuteArgs p;
     p.idx = idx;
     p.S = T * c->top_k;
@@ -241,7 +290,111 @@ moe_status run_permute(const moe_config* c, const int32_t* idx, int64_t T, int32
     p.chunk_hist = at<int32_t>(ws, L.chunk_hist);
     p.n_chunks = L.n_chunks;
     p.status = at<int>(ws, L.status);
+    if (tc_tiles) {
+        p.tile_bn = kTcBN;
+        p.tile_start = at<int32_t>(ws, L.tiles);
+    }
     MOE_CUDA(launch_permute(p, s));
+    return MOE_OK;
+}
+
+// Tensor-core part of a4 + a5 (+ a6): the routed groups (rtc) and/or the shared expert (stc).
+moe_status run_experts_tc(const moe_config* c, const moe_weights* w, const void* u, const void* x, int64_t T,
+                          const int32_t* offsets, const int32_t* sorted_slot, const float* topk_w, float* y_acc,
+                          bool rtc, bool stc, void* ws, const WsLayout& L, cudaStream_t s) {
+    const int K = expert_in(*c), I = c->intermediate, E = c->num_experts, k = c->top_k, H = c->hidden;
+    const int Is = c->shared_intermediate;
+    const int64_t S = T * k;
+    const int64_t n_dense = (T + kTcBN - 1) / kTcBN;
+    void* uperm = at<void>(ws, L.uperm);
+    void* h = at<void>(ws, L.h);
+    void* hs = at<void>(ws, L.hs);
+    const int32_t* tiles = at<int32_t>(ws, L.tiles);
+    if (rtc) MOE_CUDA(launch_gather_rows(u, K, sorted_slot, k, S, uperm, s));
+    {  // gate/up + activation
+        TcParams P;
+        int np = 0;
+        int64_t max_tiles = 0;
+        if (stc) {
+            TcProblem& p = P.p[np];
+            p.mode = kEpiGateUp;
+            p.M = Is; p.K = H; p.m_blocks = (Is + 127) / 128;
+            p.rows = int(T); p.n_tiles = int(n_dense);
+            p.out = hs; p.ld_out = Is;
+            if (!tc_weight_map(&P.a0[np], w->shared_gate_w, 1, Is, H, false) ||
+                !tc_weight_map(&P.a1[np], w->shared_up_w, 1, Is, H, false) ||
+                !tc_token_map(&P.b[np], x, T, H, kTcBN))
+                return MOE_ERR_CUDA;
+            max_tiles += int64_t(p.m_blocks) * p.n_tiles;
+            ++np;
+        }
+        if (rtc) {
+            TcProblem& p = P.p[np];
+            p.mode = kEpiGateUp;
+            p.M = I; p.K = K; p.m_blocks = (I + 127) / 128;
+            p.grouped = 1; p.num_groups = E; p.offsets = offsets; p.tile_start = tiles;
+            p.out = h; p.ld_out = I;
+            p.interleaved = c->gate_up_interleaved;
+            if (c->has_expert_bias) {
+                if (c->gate_up_interleaved) {
+                    p.bias0 = w->gate_up_b;
+                    p.bias_interleaved = 1;
+                } else {
+                    p.bias0 = w->gate_b;
+                    p.bias1 = w->up_b;
+                }
+            }
+            bool ok;
+            if (c->gate_up_interleaved) {
+                ok = tc_weight_map(&P.a0[np], w->gate_up_w, E, I, K, true);
+            } else {
+                ok = tc_weight_map(&P.a0[np], w->gate_w, E, I, K, false) &&
+                     tc_weight_map(&P.a1[np], w->up_w, E, I, K, false);
+            }
+            if (!ok || !tc_token_map(&P.b[np], uperm, S, K, kTcBN)) return MOE_ERR_CUDA;
+            max_tiles += int64_t(p.m_blocks) * max_routed_tiles(*c, T);
+            ++np;
+        }
+        P.nprob = np;
+        P.status = at<int>(ws, L.status);
+        P.act = c->activation;
+        P.limit = c->swiglu_limit;
+        P.alpha = c->swiglu_alpha;
+        MOE_CUDA(launch_tc_gemm(P, true, max_tiles, s));
+    }
+    {  // down (+ weighted scatter into the routed sum)
+        TcParams P;
+        int np = 0;
+        int64_t max_tiles = 0;
+        if (stc) {
+            TcProblem& p = P.p[np];
+            p.mode = kEpiStoreF32;
+            p.M = H; p.K = Is; p.m_blocks = (H + 127) / 128;
+            p.rows = int(T); p.n_tiles = int(n_dense);
+            p.out = at<float>(ws, L.s_acc); p.ld_out = H;
+            if (!tc_weight_map(&P.a0[np], w->shared_down_w, 1, H, Is, false) ||
+                !tc_token_map(&P.b[np], hs, T, Is, kTcBN))
+                return MOE_ERR_CUDA;
+            max_tiles += int64_t(p.m_blocks) * p.n_tiles;
+            ++np;
+        }
+        if (rtc) {
+            TcProblem& p = P.p[np];
+            p.mode = kEpiScatter;
+            p.M = K; p.K = I; p.m_blocks = (K + 127) / 128;
+            p.grouped = 1; p.num_groups = E; p.offsets = offsets; p.tile_start = tiles;
+            p.sorted_slot = sorted_slot; p.topk_w = topk_w; p.k = k;
+            p.bias0 = c->has_expert_bias ? w->down_b : nullptr;
+            p.out = y_acc; p.ld_out = K;
+            if (!tc_weight_map(&P.a0[np], w->down_w, E, K, I, false) || !tc_token_map(&P.b[np], h, S, I, kTcBN))
+                return MOE_ERR_CUDA;
+            max_tiles += int64_t(p.m_blocks) * max_routed_tiles(*c, T);
+            ++np;
+        }
+        P.nprob = np;
+        P.status = at<int>(ws, L.status);
+        MOE_CUDA(launch_tc_gemm(P, false, max_tiles, s));
+    }
     return MOE_OK;
 }
 
@@ -251,8 +404,13 @@ moe_status run_experts(const moe_config* c, const moe_weights* w, const void* u,
                        float* y_acc, bool with_routed, bool with_shared, void* ws, const WsLayout& L,
                        cudaStream_t s) {
     const int K = expert_in(*c);
-    const int64_t groups = with_routed ? std::min<int64_t>(c->num_experts, T * c->top_k) : 0;
     const bool sh = with_shared && c->shared_mode != MOE_SHARED_NONE;
+    const bool rtc = with_routed && routed_tc(c, T);
+    const bool stc = sh && c->shared_intermediate % 64 == 0 && dense_tc(c, T, c->hidden);
+    if (rtc || stc)
+        MOE_CHECK(run_experts_tc(c, w, u, x, T, offsets, sorted_slot, topk_w, y_acc, rtc, stc, ws, L, s));
+    const int64_t groups = (with_routed && !rtc) ? std::min<int64_t>(c->num_experts, T * c->top_k) : 0;
+    if (groups == 0 && (!sh || stc)) return MOE_OK;
     GateUpArgs g;
     g.wf = c->weight_format;
     g.interleaved = c->gate_up_interleaved;
@@ -270,7 +428,7 @@ moe_status run_experts(const moe_config* c, const moe_weights* w, const void* u,
     g.routed_groups = int(groups);
     g.u = u;
     g.h = at<void>(ws, L.h);
-    if (sh) {
+    if (sh && !stc) {
         g.sg_w = w->shared_gate_w;
         g.su_w = w->shared_up_w;
         g.shared_I = c->shared_intermediate;
@@ -298,7 +456,7 @@ moe_status run_experts(const moe_config* c, const moe_weights* w, const void* u,
     d.routed_groups = int(groups);
     d.h = at<void>(ws, L.h);
     d.y_acc = y_acc;
-    if (sh) {
+    if (sh && !stc) {
         d.sd_w = w->shared_down_w;
         d.shared_I = c->shared_intermediate;
         d.Hs = c->hidden;
@@ -312,7 +470,7 @@ moe_status run_experts(const moe_config* c, const moe_weights* w, const void* u,
 
 // a8 (first half): z = x Wdp^T
 moe_status run_latent_down(const moe_config* c, const moe_weights* w, const void* x, int64_t T, void* z,
-                           cudaStream_t s) {
+                           int* status, cudaStream_t s) {
     DenseGemvArgs r;
     r.W0 = w->latent_down_w;
     r.rows0 = c->latent_dim;
@@ -323,6 +481,20 @@ moe_status run_latent_down(const moe_config* c, const moe_weights* w, const void
     r.ld_out = c->latent_dim;
     r.out_f32 = 0;
     r.act_dtype = c->act_dtype;
+    if (dense_tc(c, T, c->hidden) && c->latent_dim % 64 == 0) {
+        TcParams P;
+        TcProblem& p = P.p[0];
+        p.mode = kEpiStoreAct;
+        p.M = c->latent_dim; p.K = c->hidden; p.m_blocks = (p.M + 127) / 128;
+        p.rows = int(T); p.n_tiles = int((T + kTcBN - 1) / kTcBN);
+        p.out = z; p.ld_out = c->latent_dim;
+        if (!tc_weight_map(&P.a0[0], w->latent_down_w, 1, p.M, p.K, false) || !tc_token_map(&P.b[0], x, T, p.K, kTcBN))
+            return MOE_ERR_CUDA;
+        P.nprob = 1;
+        P.status = status;
+        MOE_CUDA(launch_tc_gemm(P, false, int64_t(p.m_blocks) * p.n_tiles, s));
+        return MOE_OK;
+    }
     MOE_CUDA(launch_dense_gemv(r, s));
     return MOE_OK;
 }
@@ -362,6 +534,21 @@ moe_status run_output(const moe_config* c, const moe_weights* w, const float* y_
     r.addend = s_acc;
     r.ld_add = c->hidden;
     r.act_dtype = c->act_dtype;
+    if (dense_tc(c, T, c->latent_dim) && c->hidden % 64 == 0) {
+        TcParams P;
+        TcProblem& p = P.p[0];
+        p.mode = kEpiStoreAct;
+        p.M = c->hidden; p.K = c->latent_dim; p.m_blocks = (p.M + 127) / 128;
+        p.rows = int(T); p.n_tiles = int((T + kTcBN - 1) / kTcBN);
+        p.out = y; p.ld_out = c->hidden;
+        p.addend = s_acc; p.ld_add = c->hidden;
+        if (!tc_weight_map(&P.a0[0], w->latent_up_w, 1, p.M, p.K, false) || !tc_token_map(&P.b[0], n, T, p.K, kTcBN))
+            return MOE_ERR_CUDA;
+        P.nprob = 1;
+        P.status = at<int>(ws, L.status);
+        MOE_CUDA(launch_tc_gemm(P, false, int64_t(p.m_blocks) * p.n_tiles, s));
+        return MOE_OK;
+    }
     MOE_CUDA(launch_dense_gemv(r, s));
     return MOE_OK;
 }
@@ -412,7 +599,8 @@ moe_status moe_permute(const moe_config* cfg, const int32_t* topk_idx, int64_t T
     MOE_CHECK(check_ptr(expert_offsets));
     MOE_CHECK(check_ptr(sorted_slot));
     MOE_CHECK(check_ptr(slot_pos));
-    return run_permute(cfg, topk_idx, T, expert_offsets, sorted_slot, slot_pos, ws, L, (cudaStream_t)stream);
+    return run_permute(cfg, topk_idx, T, expert_offsets, sorted_slot, slot_pos, ws, L, (cudaStream_t)stream,
+                       false);
 }
 
 moe_status moe_grouped_ffn(const moe_config* cfg, const moe_weights* w, const void* u, int64_t T,
@@ -430,6 +618,8 @@ moe_status moe_grouped_ffn(const moe_config* cfg, const moe_weights* w, const vo
     cudaStream_t s = (cudaStream_t)stream;
     MOE_CUDA(cudaMemsetAsync(y_acc, 0, size_t(T) * expert_in(*cfg) * sizeof(float), s));
     MOE_CUDA(launch_active_list(expert_offsets, cfg->num_experts, at<int32_t>(ws, L.active), s));
+    if (routed_tc(cfg, T))
+        MOE_CUDA(launch_tile_start(expert_offsets, cfg->num_experts, kTcBN, at<int32_t>(ws, L.tiles), s));
     return run_experts(cfg, w, u, nullptr, T, expert_offsets, sorted_slot, topk_w, y_acc, true, false, ws, L, s);
 }
 
@@ -442,7 +632,7 @@ moe_status moe_latent_down(const moe_config* cfg, const moe_weights* w, const vo
     if (T == 0) return MOE_OK;
     MOE_CHECK(check_ptr(x));
     MOE_CHECK(check_ptr(z));
-    return run_latent_down(cfg, w, x, T, z, (cudaStream_t)stream);
+    return run_latent_down(cfg, w, x, T, z, at<int>(ws, L.status), (cudaStream_t)stream);
 }
 
 moe_status moe_combine(const moe_config* cfg, const moe_weights* w, const float* y_acc, const void* x,
@@ -478,12 +668,13 @@ moe_status moe_block_forward(const moe_config* cfg, const moe_weights* w, const 
     MOE_CHECK(run_route(cfg, w, x, T, idx, wts, coef, y_acc, K, ws, L, s));
     const void* u = x;
     if (cfg->latent_dim) {
-        MOE_CHECK(run_latent_down(cfg, w, x, T, at<void>(ws, L.z), s));
+        MOE_CHECK(run_latent_down(cfg, w, x, T, at<void>(ws, L.z), at<int>(ws, L.status), s));
         u = at<void>(ws, L.z);
     }
     int32_t* offsets = at<int32_t>(ws, L.offsets);
     int32_t* sorted_slot = at<int32_t>(ws, L.sorted_slot);
-    MOE_CHECK(run_permute(cfg, idx, T, offsets, sorted_slot, at<int32_t>(ws, L.slot_pos), ws, L, s));
+    MOE_CHECK(run_permute(cfg, idx, T, offsets, sorted_slot, at<int32_t>(ws, L.slot_pos), ws, L, s,
+                          routed_tc(cfg, T)));
     MOE_CHECK(run_experts(cfg, w, u, x, T, offsets, sorted_slot, wts, y_acc, true, true, ws, L, s));
     return run_output(cfg, w, y_acc, coef, T, y, ws, L, s);
 }

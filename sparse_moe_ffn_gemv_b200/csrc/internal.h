@@ -1,8 +1,10 @@
 // internal.h -- host-side launchers shared by the library's translation units.
 #pragma once
 
+#include <cuda.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
+#include <string.h>
 
 #include "../../include/moe.h"
 
@@ -34,10 +36,19 @@ struct PermuteArgs {
     int32_t* offsets = nullptr; int32_t* sorted_slot = nullptr; int32_t* slot_pos = nullptr;
     int32_t* active = nullptr; int32_t* chunk_hist = nullptr; int n_chunks = 0;
     int* status = nullptr;
+    int tile_bn = 0;                 // > 0: also write tile_start[E + 1], the exclusive prefix
+    int32_t* tile_start = nullptr;   //      of ceil(count_e / tile_bn) (tensor-core tile list)
 };
 cudaError_t launch_permute(const PermuteArgs& a, cudaStream_t s);
 // active[0] = number of experts with tokens, active[1..] their ids, from offsets [E + 1].
 cudaError_t launch_active_list(const int32_t* offsets, int E, int32_t* active, cudaStream_t s);
+
+// dst[p, :] = src[sorted_slot[p] / k, :] for p < S (rows of K bf16): expert inputs in
+// sorted order for the tensor-core path.
+cudaError_t launch_gather_rows(const void* src, int K, const int32_t* sorted_slot, int k, int64_t S,
+                               void* dst, cudaStream_t s);
+// tile_start from offsets (moe_grouped_ffn called with a caller-made permutation).
+cudaError_t launch_tile_start(const int32_t* offsets, int E, int tile_bn, int32_t* tile_start, cudaStream_t s);
 
 // Routed + shared gate/up on CUDA cores: h = act(Wg u + bg, Wu u + bu).
 struct GateUpArgs {
@@ -76,5 +87,48 @@ cudaError_t launch_combine(const float* y_acc, const float* s_acc, const float* 
 // nrm = y_acc / sqrt(mean(y_acc^2) + eps) * gamma (act dtype), per token row of width L.
 cudaError_t launch_rmsnorm(const float* y_acc, const void* gamma, float eps, int64_t T, int L,
                            void* out, int act_dtype, cudaStream_t s);
+
+// ------------------------------------------------------------------ tensor-core GEMM
+constexpr int kTcBN = 128;  // token columns per tile
+enum { kEpiGateUp = 0, kEpiScatter = 1, kEpiStoreF32 = 2, kEpiStoreAct = 3 };
+
+// One GEMM problem of a tensor-core launch: D[M rows, tokens] = W[M, K] . U[tokens, K]^T.
+struct TcProblem {
+    int mode = kEpiStoreF32;
+    int M = 0, K = 0, m_blocks = 0;
+    int grouped = 0;                       // 1: expert groups (offsets / tile_start), 0: one dense group
+    int rows = 0, n_tiles = 0, bn = kTcBN; // dense: token rows and their tiles
+    int num_groups = 0;
+    const int32_t* offsets = nullptr;      // [E + 1] sorted-row offsets of the groups
+    const int32_t* tile_start = nullptr;   // [E + 1] prefix of token tiles per group
+    const int32_t* sorted_slot = nullptr;  // scatter: sorted row -> slot
+    const float* topk_w = nullptr;         // scatter: slot -> combine weight
+    int k = 1;
+    const void* bias0 = nullptr;           // bf16 [groups, M] (or [groups, 2M] interleaved gate/up)
+    const void* bias1 = nullptr;           // bf16 [groups, M] (up bias, separate layout)
+    int bias_interleaved = 0, interleaved = 0;
+    void* out = nullptr; int ld_out = 0;
+    const float* addend = nullptr; int ld_add = 0;
+};
+
+struct alignas(64) TcParams {
+    TcParams() {  // unused tensor maps stay zero; the problems keep their defaults
+        memset(static_cast<void*>(a0), 0, sizeof(a0));
+        memset(static_cast<void*>(a1), 0, sizeof(a1));
+        memset(static_cast<void*>(b), 0, sizeof(b));
+    }
+    CUtensorMap a0[2];  // weights (gate / single)
+    CUtensorMap a1[2];  // weights (up), gate/up mode with separate planes
+    CUtensorMap b[2];   // tokens
+    TcProblem p[2];
+    int nprob = 0;
+    int* status = nullptr;
+    int act = 0;
+    float limit = 7.f, alpha = 1.702f;
+};
+
+bool tc_weight_map(CUtensorMap* m, const void* w, int E, int R, int K, bool interleaved);
+bool tc_token_map(CUtensorMap* m, const void* u, int64_t rows, int K, int bn);
+cudaError_t launch_tc_gemm(TcParams& P, bool gateup, int64_t max_tiles, cudaStream_t s);
 
 }  // namespace moe

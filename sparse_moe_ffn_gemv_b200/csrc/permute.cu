@@ -101,6 +101,15 @@ __global__ void __launch_bounds__(kPlaceThreads) place_kernel(PermuteArgs a) {
     }
     __syncthreads();
     for (int e = tid; e < E; e += kPlaceThreads) flag_buf[e] = scan_buf[e] > 0 ? 1 : 0;
+    if (chunk == 0 && a.tile_bn > 0) {
+        // tensor-core tile prefix: tiles of expert e = ceil(count_e / tile_bn)
+        for (int e = tid; e < E; e += kPlaceThreads) cnt[0][e] = (scan_buf[e] + a.tile_bn - 1) / a.tile_bn;
+        __syncthreads();
+        const int ntiles = block_exclusive_scan(&cnt[0][0], E, warp_tot);
+        for (int e = tid; e < E; e += kPlaceThreads) a.tile_start[e] = cnt[0][e];
+        if (tid == 0) a.tile_start[E] = ntiles;
+        for (int e = tid; e < E; e += kPlaceThreads) cnt[0][e] = 0;
+    }
     __syncthreads();
     const int total = block_exclusive_scan(scan_buf, E, warp_tot);
     const int n_active = block_exclusive_scan(flag_buf, E, warp_tot);
@@ -164,7 +173,47 @@ __global__ void __launch_bounds__(kPlaceThreads) active_kernel(const int32_t* of
     if (tid == 0) active[0] = n;
 }
 
+__global__ void __launch_bounds__(kPlaceThreads) tile_start_kernel(const int32_t* offsets, int E, int bn,
+                                                                 int32_t* tile_start) {
+    __shared__ int v[kPermE];
+    __shared__ int warp_tot[kPlaceWarps + 1];
+    const int tid = threadIdx.x;
+    if (tid < E) v[tid] = (offsets[tid + 1] - offsets[tid] + bn - 1) / bn;
+    __syncthreads();
+    const int n = block_exclusive_scan(v, E, warp_tot);
+    if (tid < E) tile_start[tid] = v[tid];
+    if (tid == 0) tile_start[E] = n;
+}
+
+// One warp per destination row, 16-byte vectors.
+__global__ void __launch_bounds__(256) gather_rows_kernel(const uint4* __restrict__ src, int vpr,
+                                                          const int32_t* __restrict__ sorted_slot, int k,
+                                                          int64_t S, uint4* __restrict__ dst) {
+    const int lane = threadIdx.x & 31;
+    const int64_t p = (int64_t(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+    if (p >= S) return;
+    const int64_t row = sorted_slot[p] / k;
+    const uint4* s = src + row * vpr;
+    uint4* d = dst + p * vpr;
+    for (int c = lane; c < vpr; c += 32) d[c] = s[c];
+}
+
 }  // namespace
+
+cudaError_t launch_gather_rows(const void* src, int K, const int32_t* sorted_slot, int k, int64_t S, void* dst,
+                               cudaStream_t s) {
+    if (S == 0) return cudaSuccess;
+    const int vpr = K * 2 / 16;
+    const unsigned grid = unsigned((S * 32 + 255) / 256);
+    gather_rows_kernel<<<grid, 256, 0, s>>>(static_cast<const uint4*>(src), vpr, sorted_slot, k, S,
+                                            static_cast<uint4*>(dst));
+    return cudaGetLastError();
+}
+
+cudaError_t launch_tile_start(const int32_t* offsets, int E, int tile_bn, int32_t* tile_start, cudaStream_t s) {
+    tile_start_kernel<<<1, kPlaceThreads, 0, s>>>(offsets, E, tile_bn, tile_start);
+    return cudaGetLastError();
+}
 
 cudaError_t launch_active_list(const int32_t* offsets, int E, int32_t* active, cudaStream_t s) {
     active_kernel<<<1, kPlaceThreads, 0, s>>>(offsets, E, active);

@@ -1,0 +1,505 @@
+// umma.cu -- tensor-core (tcgen05 / TMEM) grouped GEMM fed by TMA, for prefill-sized batches.
+//
+// D[128 weight rows, BN tokens] = W[128, K] . U[BN, K]^T per tile ("weights as M"): every
+// expert group is padded only to the token tile, and each weight tile is read from HBM once
+// and shared by the token tiles of its group through L2.
+//
+// One persistent CTA per SM, warp-specialised:
+//   warp 0      TMA producer: weight tile(s) + token tile per 64-wide K block into a
+//               STAGES-deep shared-memory ring (128-byte swizzle)
+//   warp 1      MMA issuer (one thread): tcgen05.mma kind::f16, bf16 x bf16 -> fp32 in
+//               TMEM; two accumulators (gate, up) in gate/up mode
+//   warps 2..5  epilogue: tcgen05.ld, then SwiGLU / clamped SwiGLU -> bf16 h (gate/up),
+//               weighted scatter-add into the fp32 routed sum (down), or a plain store
+// TMEM holds two accumulator sets so the epilogue of one tile overlaps the main loop of
+// the next. Every mbarrier wait is bounded by %globaltimer; a wait that gives up records
+// MOE_ERR_DEVICE_TIMEOUT in the status word, drains its own outstanding copies / MMAs and
+// returns, and TMEM is always freed.
+//
+// Block math (libmir-metal execute: gate_up with biases and limit, then down weighted by
+// routing.weights and summed; ferrox KimiExpertWeights::forward: down(act(gate, up))).
+#include <cuda.h>
+
+#include <mutex>
+
+#include "common.cuh"
+#include "internal.h"
+
+namespace moe {
+
+namespace {
+
+constexpr int kBM = 128;          // weight rows per tile (MMA M)
+constexpr int kBK = 64;           // K per stage: one 128-byte swizzle atom of bf16
+constexpr int kTcThreads = 192;   // 6 warps
+constexpr uint64_t kWaitNs = 2000000000ull;  // 2 s bound on any single wait
+
+__device__ __forceinline__ uint32_t su32(const void* p) {
+    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+__device__ __forceinline__ uint64_t gtimer() {
+    uint64_t t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+__device__ __forceinline__ void mbar_init(uint64_t* b, uint32_t count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(su32(b)), "r"(count));
+}
+__device__ __forceinline__ void mbar_expect_tx(uint64_t* b, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(su32(b)), "r"(bytes) : "memory");
+}
+__device__ __forceinline__ void mbar_arrive(uint64_t* b) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(su32(b)) : "memory");
+}
+__device__ __forceinline__ bool mbar_try(uint64_t* b, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(su32(b)), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+// Bounded wait for the phase with the given parity; false = gave up.
+__device__ __forceinline__ bool mbar_wait(uint64_t* b, uint32_t parity, uint64_t deadline) {
+    for (uint32_t i = 0;; ++i) {
+        if (mbar_try(b, parity)) return true;
+        if ((i & 63u) == 63u && gtimer() > deadline) return false;
+    }
+}
+
+__device__ __forceinline__ void tma_2d(void* dst, const CUtensorMap* m, uint64_t* bar, int c0, int c1) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%3, %4}], [%2];" ::"r"(su32(dst)),
+        "l"(reinterpret_cast<uint64_t>(m)), "r"(su32(bar)), "r"(c0), "r"(c1)
+        : "memory");
+}
+__device__ __forceinline__ void tma_3d(void* dst, const CUtensorMap* m, uint64_t* bar, int c0, int c1, int c2) {
+    asm volatile(
+        "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%3, %4, %5}], [%2];" ::"r"(su32(dst)),
+        "l"(reinterpret_cast<uint64_t>(m)), "r"(su32(bar)), "r"(c0), "r"(c1), "r"(c2)
+        : "memory");
+}
+__device__ __forceinline__ void tma_4d(void* dst, const CUtensorMap* m, uint64_t* bar, int c0, int c1, int c2,
+                                       int c3) {
+    asm volatile(
+        "cp.async.bulk.tensor.4d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%3, %4, %5, %6}], [%2];" ::"r"(su32(dst)),
+        "l"(reinterpret_cast<uint64_t>(m)), "r"(su32(bar)), "r"(c0), "r"(c1), "r"(c2), "r"(c3)
+        : "memory");
+}
+__device__ __forceinline__ void prefetch_tmap(const CUtensorMap* m) {
+    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(m)) : "memory");
+}
+
+__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+
+// Shared-memory matrix descriptor: K-major, 128-byte swizzle, 8-row groups 1024 B apart.
+__device__ __forceinline__ uint64_t smem_desc(uint32_t saddr) {
+    return uint64_t((saddr & 0x3FFFFu) >> 4) | (uint64_t(1) << 16) | (uint64_t(1024 >> 4) << 32) |
+           (uint64_t(1) << 46) | (uint64_t(2) << 61);
+}
+// Instruction descriptor: kind::f16, A = B = bf16, D = f32, both K-major, M = 128, N = n.
+__host__ __device__ constexpr uint32_t idesc_bf16(int n) {
+    return (1u << 4) | (1u << 7) | (1u << 10) | (uint32_t(n >> 3) << 17) | (uint32_t(kBM >> 4) << 24);
+}
+
+__device__ __forceinline__ void umma(uint32_t d, uint64_t a, uint64_t b, uint32_t idesc, uint32_t acc) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d),
+        "l"(a), "l"(b), "r"(idesc), "r"(acc)
+        : "memory");
+}
+__device__ __forceinline__ void umma_commit(uint64_t* bar) {
+    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(su32(bar))
+                 : "memory");
+}
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {
+    uint32_t r[32];
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+        "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]),
+          "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]),
+          "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]),
+          "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+        : "r"(taddr));
+    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+    for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+// Where one tile lives.
+struct TileInfo {
+    int prob;      // problem index
+    int group;     // expert id (grouped) or 0
+    int mb;        // weight-row block
+    int row0;      // first B row (sorted position or token) of the tile
+    int nvalid;    // valid token columns
+};
+
+__device__ __forceinline__ int problem_tiles(const TcProblem& p) {
+    if (p.grouped) return p.tile_start[p.num_groups] * p.m_blocks;
+    return p.n_tiles * p.m_blocks;
+}
+
+__device__ __forceinline__ TileInfo decode_tile(const TcParams& P, int tile, int t0) {
+    TileInfo ti;
+    int local = tile;
+    ti.prob = 0;
+    if (P.nprob > 1 && tile >= t0) {
+        ti.prob = 1;
+        local = tile - t0;
+    }
+    const TcProblem& p = P.p[ti.prob];
+    if (!p.grouped) {
+        ti.group = 0;
+        ti.mb = local / p.n_tiles;
+        const int nb = local - ti.mb * p.n_tiles;
+        ti.row0 = nb * p.bn;
+        ti.nvalid = min(p.bn, p.rows - ti.row0);
+        return ti;
+    }
+    // largest e with tile_start[e] * m_blocks <= local (that expert is non-empty)
+    int lo = 0, hi = p.num_groups - 1;
+    while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (p.tile_start[mid] * p.m_blocks <= local) lo = mid;
+        else hi = mid - 1;
+    }
+    const int e = lo;
+    const int ts = p.tile_start[e];
+    const int nbe = p.tile_start[e + 1] - ts;
+    const int l = local - ts * p.m_blocks;
+    ti.group = e;
+    ti.mb = l / nbe;
+    const int nb = l - ti.mb * nbe;
+    const int off = p.offsets[e];
+    const int cnt = p.offsets[e + 1] - off;
+    ti.row0 = off + nb * p.bn;
+    ti.nvalid = min(p.bn, cnt - nb * p.bn);
+    return ti;
+}
+
+template <bool GATEUP, int BN, int STAGES>
+struct TcShape {
+    static constexpr int A_BYTES = kBM * kBK * 2;                // 16 KB
+    static constexpr int B_BYTES = BN * kBK * 2;
+    static constexpr int STAGE_BYTES = A_BYTES * (GATEUP ? 2 : 1) + B_BYTES;
+    static constexpr int ACC_COLS = GATEUP ? 2 * BN : BN;        // per accumulator set
+    static constexpr int TMEM_COLS = 2 * ACC_COLS;               // double-buffered
+    static constexpr int SMEM = STAGES * STAGE_BYTES + 1024 /*align*/ + 256 /*barriers*/;
+    static_assert(TMEM_COLS <= 512 && (TMEM_COLS & (TMEM_COLS - 1)) == 0, "TMEM columns");
+    static_assert(BN % 32 == 0 && BN >= 32 && BN <= 256, "BN");
+};
+
+__device__ __forceinline__ float bf16_at(const void* p, int64_t i) {
+    return __bfloat162float(reinterpret_cast<const __nv_bfloat16*>(p)[i]);
+}
+
+template <bool GATEUP, int BN, int STAGES>
+__global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_constant__ TcParams P) {
+    using S = TcShape<GATEUP, BN, STAGES>;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem + STAGES * S::STAGE_BYTES);
+    uint64_t* empty = full + STAGES;
+    uint64_t* acc_full = empty + STAGES;
+    uint64_t* acc_empty = acc_full + 2;
+    uint64_t* drain = acc_empty + 2;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    if (warp == 0) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(su32(tmem_slot)),
+                     "r"(uint32_t(S::TMEM_COLS)));
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
+    }
+    if (warp == 1 && lane == 0) {
+        for (int s = 0; s < STAGES; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], 1);
+        }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&acc_full[b], 1);
+            mbar_init(&acc_empty[b], 4);  // one arrive per epilogue warp
+        }
+        mbar_init(drain, 1);
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+    }
+    if (warp == 2 && lane == 0) {
+        for (int i = 0; i < P.nprob; ++i) {
+            prefetch_tmap(&P.a0[i]);
+            if (GATEUP && !P.p[i].interleaved) prefetch_tmap(&P.a1[i]);
+            prefetch_tmap(&P.b[i]);
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem_base = *tmem_slot;
+
+    const int t0 = problem_tiles(P.p[0]);
+    const int total = t0 + (P.nprob > 1 ? problem_tiles(P.p[1]) : 0);
+    const uint64_t deadline = gtimer() + kWaitNs;
+    bool timed_out = false;
+
+    if (warp == 0) {
+        if (lane == 0) {
+            // ---------------------------------------------------------- TMA producer
+            uint32_t stage = 0, phase = 0;
+            uint32_t armed = 0;  // bit s: stage s was filled at least once
+            uint32_t last_par = 0;
+            for (int tile = blockIdx.x; tile < total && !timed_out; tile += gridDim.x) {
+                const TileInfo ti = decode_tile(P, tile, t0);
+                const TcProblem& p = P.p[ti.prob];
+                const int nk = p.K / kBK;
+                for (int kb = 0; kb < nk; ++kb) {
+                    if (!mbar_wait(&empty[stage], phase ^ 1u, deadline)) {
+                        timed_out = true;
+                        break;
+                    }
+                    uint8_t* sb = smem + stage * S::STAGE_BYTES;
+                    mbar_expect_tx(&full[stage], S::STAGE_BYTES);
+                    const int kc = kb * kBK;
+                    const int mrow = ti.mb * kBM;
+                    if (p.interleaved) {  // [E, I, 2, K]: plane 0 = gate rows, 1 = up rows
+                        tma_4d(sb, &P.a0[ti.prob], &full[stage], kc, 0, mrow, ti.group);
+                        if (GATEUP) tma_4d(sb + S::A_BYTES, &P.a0[ti.prob], &full[stage], kc, 1, mrow, ti.group);
+                    } else {
+                        tma_3d(sb, &P.a0[ti.prob], &full[stage], kc, mrow, ti.group);
+                        if (GATEUP) tma_3d(sb + S::A_BYTES, &P.a1[ti.prob], &full[stage], kc, mrow, ti.group);
+                    }
+                    tma_2d(sb + S::A_BYTES * (GATEUP ? 2 : 1), &P.b[ti.prob], &full[stage], kc, ti.row0);
+                    armed |= 1u << stage;
+                    last_par = (last_par & ~(1u << stage)) | (phase << stage);
+                    if (++stage == STAGES) {
+                        stage = 0;
+                        phase ^= 1u;
+                    }
+                }
+            }
+            // drain: every copy this thread issued has landed before the CTA can exit
+            const uint64_t dl2 = gtimer() + kWaitNs;
+            for (int s = 0; s < STAGES; ++s)
+                if ((armed >> s) & 1u) mbar_wait(&full[s], (last_par >> s) & 1u, dl2);
+            if (timed_out) set_status(P.status, MOE_ERR_DEVICE_TIMEOUT);
+        }
+    } else if (warp == 1) {
+        if (lane == 0) {
+            // ---------------------------------------------------------- MMA issuer
+            uint32_t stage = 0, phase = 0, it = 0;
+            constexpr uint32_t idesc = idesc_bf16(BN);
+            for (int tile = blockIdx.x; tile < total && !timed_out; tile += gridDim.x, ++it) {
+                const TileInfo ti = decode_tile(P, tile, t0);
+                const TcProblem& p = P.p[ti.prob];
+                const uint32_t ab = it & 1u, aph = (it >> 1) & 1u;
+                if (!mbar_wait(&acc_empty[ab], aph ^ 1u, deadline)) {
+                    timed_out = true;
+                    break;
+                }
+                tc_fence_after();
+                const uint32_t d0 = tmem_base + ab * S::ACC_COLS;
+                const int nk = p.K / kBK;
+                for (int kb = 0; kb < nk; ++kb) {
+                    if (!mbar_wait(&full[stage], phase, deadline)) {
+                        timed_out = true;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint32_t sa = su32(smem + stage * S::STAGE_BYTES);
+                    const uint32_t sbb = sa + S::A_BYTES * (GATEUP ? 2 : 1);
+#pragma unroll
+                    for (int k = 0; k < kBK / 16; ++k) {
+                        const uint64_t bdesc = smem_desc(sbb + k * 32);
+                        const uint32_t acc = (kb > 0 || k > 0) ? 1u : 0u;
+                        umma(d0, smem_desc(sa + k * 32), bdesc, idesc, acc);
+                        if (GATEUP) umma(d0 + BN, smem_desc(sa + S::A_BYTES + k * 32), bdesc, idesc, acc);
+                    }
+                    umma_commit(&empty[stage]);
+                    if (++stage == STAGES) {
+                        stage = 0;
+                        phase ^= 1u;
+                    }
+                }
+                if (timed_out) break;
+                umma_commit(&acc_full[ab]);
+            }
+            // drain: all MMAs issued by this thread have completed
+            umma_commit(drain);
+            mbar_wait(drain, 0, gtimer() + kWaitNs);
+            if (timed_out) set_status(P.status, MOE_ERR_DEVICE_TIMEOUT);
+        }
+    } else {
+        // -------------------------------------------------------------- epilogue (128 threads)
+        const int q = warp & 3;                  // TMEM lane quarter of this warp
+        const int lrow = q * 32 + lane;          // accumulator row = weight row in the tile
+        uint32_t it = 0;
+        for (int tile = blockIdx.x; tile < total; tile += gridDim.x, ++it) {
+            const TileInfo ti = decode_tile(P, tile, t0);
+            const TcProblem& p = P.p[ti.prob];
+            const uint32_t ab = it & 1u, aph = (it >> 1) & 1u;
+            if (!mbar_wait(&acc_full[ab], aph, deadline)) {
+                set_status(P.status, MOE_ERR_DEVICE_TIMEOUT);
+                break;
+            }
+            tc_fence_after();
+            const uint32_t tbase = tmem_base + (uint32_t(q * 32) << 16) + ab * S::ACC_COLS;
+            const int r = ti.mb * kBM + lrow;    // weight row (intermediate unit or output row)
+            const bool rv = r < p.M;
+            float bias0 = 0.f, bias1 = 0.f;
+            if (rv && p.bias0) {
+                if (GATEUP && p.bias_interleaved) {
+                    bias0 = bf16_at(p.bias0, int64_t(ti.group) * 2 * p.M + 2 * r);
+                    bias1 = bf16_at(p.bias0, int64_t(ti.group) * 2 * p.M + 2 * r + 1);
+                } else {
+                    bias0 = bf16_at(p.bias0, int64_t(ti.group) * p.M + r);
+                    if (GATEUP) bias1 = bf16_at(p.bias1, int64_t(ti.group) * p.M + r);
+                }
+            }
+#pragma unroll 1
+            for (int c = 0; c < BN; c += 32) {
+                float g[32];
+                tmem_ld32(tbase + c, g);
+                if constexpr (GATEUP) {
+                    float u[32];
+                    tmem_ld32(tbase + BN + c, u);
+                    __nv_bfloat16* out = reinterpret_cast<__nv_bfloat16*>(p.out);
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) {
+                        const int n = c + j;
+                        if (rv && n < ti.nvalid)
+                            out[int64_t(ti.row0 + n) * p.ld_out + r] =
+                                __float2bfloat16_rn(act_apply(P.act, g[j] + bias0, u[j] + bias1, P.limit, P.alpha));
+                    }
+                } else if (p.mode == kEpiScatter) {
+                    float* out = reinterpret_cast<float*>(p.out);
+#pragma unroll 4
+                    for (int j = 0; j < 32; ++j) {
+                        const int n = c + j;
+                        if (rv && n < ti.nvalid) {
+                            const int slot = p.sorted_slot[ti.row0 + n];
+                            const int64_t token = slot / p.k;
+                            atomicAdd(out + token * p.ld_out + r, p.topk_w[slot] * (g[j] + bias0));
+                        }
+                    }
+                } else if (p.mode == kEpiStoreF32) {
+                    float* out = reinterpret_cast<float*>(p.out);
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) {
+                        const int n = c + j;
+                        if (rv && n < ti.nvalid) out[int64_t(ti.row0 + n) * p.ld_out + r] = g[j] + bias0;
+                    }
+                } else {  // kEpiStoreAct (+ optional fp32 addend)
+                    __nv_bfloat16* out = reinterpret_cast<__nv_bfloat16*>(p.out);
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) {
+                        const int n = c + j;
+                        if (rv && n < ti.nvalid) {
+                            float v = g[j] + bias0;
+                            if (p.addend) v += p.addend[int64_t(ti.row0 + n) * p.ld_add + r];
+                            out[int64_t(ti.row0 + n) * p.ld_out + r] = __float2bfloat16_rn(v);
+                        }
+                    }
+                }
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&acc_empty[ab]);
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) {
+        tc_fence_after();
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base),
+                     "r"(uint32_t(S::TMEM_COLS)));
+    }
+}
+
+// ------------------------------------------------------------------ host side
+using EncodeFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                              const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                              CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeFn encode_fn() {
+    static EncodeFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeFn>(p);
+    });
+    return fn;
+}
+
+bool encode(CUtensorMap* m, const void* base, int rank, const cuuint64_t* dims, const cuuint64_t* strides,
+            const cuuint32_t* box) {
+    EncodeFn fn = encode_fn();
+    if (!fn) return false;
+    cuuint32_t es[5] = {1, 1, 1, 1, 1};
+    return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, cuuint32_t(rank), const_cast<void*>(base), dims, strides, box,
+              es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+int sm_count() {
+    int dev = 0, n = 148;
+    if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    return n;
+}
+
+template <bool GATEUP, int BN, int STAGES>
+cudaError_t launch_tc_t(TcParams& P, int64_t max_tiles, cudaStream_t s) {
+    using S = TcShape<GATEUP, BN, STAGES>;
+    auto kern = tc_gemm_kernel<GATEUP, BN, STAGES>;
+    cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, S::SMEM);
+    if (err != cudaSuccess) return err;
+    const int grid = int(std::min<int64_t>(max_tiles, sm_count()));
+    if (grid <= 0) return cudaSuccess;
+    kern<<<grid, kTcThreads, S::SMEM, s>>>(P);
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+// Weight operand: [E, R, K] bf16 (E = 1 for a dense matrix), or the interleaved
+// [E, 2R, K] gate_up plane viewed as [E, R, 2, K].
+bool tc_weight_map(CUtensorMap* m, const void* w, int E, int R, int K, bool interleaved) {
+    if (interleaved) {
+        const cuuint64_t dims[4] = {cuuint64_t(K), 2, cuuint64_t(R), cuuint64_t(E)};
+        const cuuint64_t strides[3] = {cuuint64_t(K) * 2, cuuint64_t(K) * 4, cuuint64_t(R) * K * 4};
+        const cuuint32_t box[4] = {kBK, 1, kBM, 1};
+        return encode(m, w, 4, dims, strides, box);
+    }
+    const cuuint64_t dims[3] = {cuuint64_t(K), cuuint64_t(R), cuuint64_t(E)};
+    const cuuint64_t strides[2] = {cuuint64_t(K) * 2, cuuint64_t(R) * K * 2};
+    const cuuint32_t box[3] = {kBK, kBM, 1};
+    return encode(m, w, 3, dims, strides, box);
+}
+
+// Token operand: [rows, K] bf16, box of bn rows.
+bool tc_token_map(CUtensorMap* m, const void* u, int64_t rows, int K, int bn) {
+    const cuuint64_t dims[2] = {cuuint64_t(K), cuuint64_t(rows)};
+    const cuuint64_t strides[1] = {cuuint64_t(K) * 2};
+    const cuuint32_t box[2] = {kBK, cuuint32_t(bn)};
+    return encode(m, u, 2, dims, strides, box);
+}
+
+cudaError_t launch_tc_gemm(TcParams& P, bool gateup, int64_t max_tiles, cudaStream_t s) {
+    if (gateup) return launch_tc_t<true, kTcBN, 4>(P, max_tiles, s);
+    return launch_tc_t<false, kTcBN, 6>(P, max_tiles, s);
+}
+
+}  // namespace moe

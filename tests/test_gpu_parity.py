@@ -219,3 +219,35 @@ def test_batch_equals_tokens_one_at_a_time_on_gpu():
     for t in (0, 5, 23):
         y1 = blk.forward(x[t:t + 1].contiguous()).float()
         assert float((y1[0] - y[t]).abs().max()) <= 2e-2 * rms
+
+
+TC_SMALL = [  # tensor-core path forced: ragged groups, partial tiles, interleaved + biases, latent
+    (inputs.KLEAR_BF16, 37),
+    (inputs.KLEAR_BF16, 200),
+    (inputs.CLAMPED_BF16, 40),
+    (inputs.LATENT_BF16, 9),
+]
+
+
+@pytest.mark.parametrize("spec,T", TC_SMALL, ids=[f"{s.name}-T{T}" for s, T in TC_SMALL])
+def test_tensor_core_path_matches_oracle(spec, T, monkeypatch):
+    monkeypatch.setenv("MOE_PATH", "tc")
+    full_check(spec, T)
+
+
+@pytest.mark.parametrize("spec,T", [(inputs.KLEAR_BF16, 96), (inputs.CLAMPED_BF16, 64),
+                                    (inputs.LATENT_BF16, 64)], ids=["klear", "clamped", "latent"])
+def test_weight_streaming_and_tensor_core_paths_agree(spec, T, monkeypatch):
+    """The decode-sized engine and the batched engine give the same block output
+    (cf. the Klear PR's caveat on a fused decode kernel that was not byte-identical)."""
+    wcpu, _ = weights(spec)
+    x = inputs.make_x(spec, T).cuda()
+    blk = M.MoeBlock(spec, wcpu, max_tokens=T)
+    monkeypatch.setenv("MOE_PATH", "gemv")
+    y_g = blk.forward(x).float()
+    monkeypatch.setenv("MOE_PATH", "tc")
+    y_t = blk.forward(x).float()
+    torch.cuda.synchronize()
+    rms = float(y_g.pow(2).mean().sqrt())
+    assert float((y_g - y_t).abs().max()) <= 2e-2 * rms
+    assert blk.device_status() == 0
