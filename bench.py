@@ -151,7 +151,7 @@ def kernels_per_step(block, x, y) -> int:
     """Kernel nodes in a CUDA graph of one step (the library's own launches)."""
     try:
         from cuda.bindings import runtime as rt
-        g = torch.cuda.CUDAGraph()
+        g = torch.cuda.CUDAGraph(keep_graph=True)
         s = torch.cuda.Stream()
         s.wait_stream(torch.cuda.current_stream())
         with torch.cuda.stream(s):
