@@ -6,7 +6,10 @@ except where the oracle's k-th and (k+1)-th selection keys lie within 1e-5, in
 which case a swap among experts whose keys lie in that band is accepted and
 the token's output is checked against the oracle evaluated with the GPU's
 expert set (several sets are then correct); outputs within max abs error
-<= 2e-2 * rms(output) for bf16 / 4-bit and <= 1e-4 for fp32.
+<= 2e-2 * rms(output) for bf16 / 4-bit and <= 1e-4 for fp32. A bf16 output
+cannot hold the exact value: rounding it alone moves an element by up to half
+a bf16 ulp (2^-9 relative), which exceeds 2e-2 * rms where |y| > ~5 rms, so
+each bf16 element may also differ by half an ulp of the exact value.
 """
 import numpy as np
 
@@ -22,6 +25,22 @@ def tolerance(spec, y_ref: np.ndarray) -> float:
         return ABS_TOL_F32
     rms = float(np.sqrt(np.mean(y_ref.astype(np.float64) ** 2)))
     return REL_TOL_BF16 * rms
+
+
+def half_ulp_bf16(v: np.ndarray) -> np.ndarray:
+    """Largest error of rounding the exact value v to bf16 (8 significant bits)."""
+    a = np.abs(v.astype(np.float64))
+    e = np.floor(np.log2(np.where(a > 0, a, 1.0)))
+    return np.where(a > 0, np.exp2(e - 8), 0.0)
+
+
+def bound(spec, y_ref: np.ndarray) -> np.ndarray:
+    """Per-element bound: the bar on the arithmetic, plus (bf16 outputs) the output
+    format's own rounding of the exact value, which no bf16 result can avoid."""
+    tol = tolerance(spec, y_ref)
+    if spec.act_dtype == "f32":
+        return np.full(y_ref.shape, tol)
+    return tol + half_ulp_bf16(y_ref)
 
 
 def index_mismatches(gpu_idx: np.ndarray, orc: dict, k: int):
@@ -58,9 +77,14 @@ def check_block(spec, w_np, x_np, tokens, y_gpu: np.ndarray, idx_gpu: np.ndarray
     for i in ties:
         y_ref[i], _ = oracle.forward_with_indices(spec, w_np, x_np, int(tokens[i]), idx_gpu[i])
     tol = tolerance(spec, orc["y"])
+    lim = bound(spec, y_ref)
     err = np.abs(y_gpu.astype(np.float64) - y_ref)
     worst = float(err.max()) if err.size else 0.0
     assert np.all(np.isfinite(y_gpu)), f"{label}: non-finite output"
-    assert worst <= tol, (f"{label}: max abs error {worst:.3e} > tolerance {tol:.3e} "
-                          f"(token {tokens[np.unravel_index(err.argmax(), err.shape)[0]]})")
-    return {"max_abs_err": worst, "tol": tol, "ties": len(ties), "tokens": len(tokens)}
+    over = err > lim
+    if over.any():
+        i = np.unravel_index(np.argmax(err - lim), err.shape)
+        raise AssertionError(f"{label}: error {err[i]:.3e} > bound {lim[i]:.3e} at token {tokens[i[0]]} "
+                             f"col {i[1]} (bar {tol:.3e}, ref {y_ref[i]:.4f})")
+    return {"max_abs_err": worst, "tol": tol, "ties": len(ties), "tokens": len(tokens),
+            "within_bar_frac": float(np.mean(err <= tol))}

@@ -251,3 +251,29 @@ def test_weight_streaming_and_tensor_core_paths_agree(spec, T, monkeypatch):
     rms = float(y_g.pow(2).mean().sqrt())
     assert float((y_g - y_t).abs().max()) <= 2e-2 * rms
     assert blk.device_status() == 0
+
+
+@pytest.mark.parametrize("path", ["gemv", "tc"])
+def test_routed_sum_in_fp32_meets_the_plain_bar(path, monkeypatch):
+    """The routed sum y_acc is fp32 (no output rounding): it meets 2e-2 * rms with no
+    allowance, on both engines."""
+    monkeypatch.setenv("MOE_PATH", path)
+    spec = inputs.KLEAR_BF16
+    wcpu, wnp = weights(spec)
+    T, k, E, H = 200, spec.top_k, spec.num_experts, spec.hidden
+    blk = M.MoeBlock(spec, wcpu, max_tokens=T)
+    x_cpu = inputs.make_x(spec, T)
+    x = x_cpu.cuda()
+    dev = dict(dtype=torch.int32, device="cuda")
+    idx, w = torch.empty((T, k), **dev), torch.empty((T, k), dtype=torch.float32, device="cuda")
+    coef = torch.empty((T, 2), dtype=torch.float32, device="cuda")
+    off, ss, sp = torch.empty(E + 1, **dev), torch.empty(T * k, **dev), torch.empty(T * k, **dev)
+    y_acc = torch.empty((T, H), dtype=torch.float32, device="cuda")
+    M.moe_route(blk.cfg, blk.w, x, T, idx, w, coef, blk.ws)
+    M.moe_permute(blk.cfg, idx, T, off, ss, sp, blk.ws)
+    M.moe_grouped_ffn(blk.cfg, blk.w, x, T, off, ss, w, y_acc, blk.ws)
+    torch.cuda.synchronize()
+    ref = oracle.forward(spec.replace(shared_mode="none"), wnp, inputs.to_numpy_storage(x_cpu))
+    assert np.array_equal(np.sort(idx.cpu().numpy(), 1), np.sort(ref["idx"], 1))
+    rms = np.sqrt(np.mean(ref["y"] ** 2))
+    assert np.abs(y_acc.cpu().numpy() - ref["y"]).max() <= 2e-2 * rms
