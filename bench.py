@@ -159,7 +159,9 @@ def kernels_per_step(block, x, y) -> int:
             block.forward(x, y, stream=s)
             g.capture_end()
         torch.cuda.current_stream().wait_stream(s)
-        err, nodes, n = rt.cudaGraphGetNodes(g.raw_cuda_graph())
+        graph = g.raw_cuda_graph()
+        err, _, n = rt.cudaGraphGetNodes(graph)          # first call: the count only
+        err, nodes, n = rt.cudaGraphGetNodes(graph, n)
         count = 0
         for node in nodes:
             e2, t = rt.cudaGraphNodeGetType(node)

@@ -52,6 +52,7 @@ WsLayout ws_layout(const moe_config& c, int64_t T) {
     L.nrm = take(Ld ? T * Ld * ab : 0);
     const bool tc = c.act_dtype == MOE_DTYPE_BF16 && c.weight_format == MOE_DTYPE_BF16;
     L.uperm = take(tc ? T * k * K * 2 : 0);
+    L.oslot = take(tc ? T * k * K * 4 : 0);
     L.tiles = take((E + 1) * 4);
     L.total = off;
     return L;
@@ -299,8 +300,10 @@ moe_status run_permute(const moe_config* c, const int32_t* idx, int64_t T, int32
 }
 
 // Tensor-core part of a4 + a5 (+ a6): the routed groups (rtc) and/or the shared expert (stc).
+// The routed down GEMM writes every slot's weighted output row (oslot); a token's routed
+// sum is the sum of its k rows, taken by the combine.
 moe_status run_experts_tc(const moe_config* c, const moe_weights* w, const void* u, const void* x, int64_t T,
-                          const int32_t* offsets, const int32_t* sorted_slot, const float* topk_w, float* y_acc,
+                          const int32_t* offsets, const int32_t* sorted_slot, const float* topk_w,
                           bool rtc, bool stc, void* ws, const WsLayout& L, cudaStream_t s) {
     const int K = expert_in(*c), I = c->intermediate, E = c->num_experts, k = c->top_k, H = c->hidden;
     const int Is = c->shared_intermediate;
@@ -380,12 +383,12 @@ moe_status run_experts_tc(const moe_config* c, const moe_weights* w, const void*
         }
         if (rtc) {
             TcProblem& p = P.p[np];
-            p.mode = kEpiScatter;
+            p.mode = kEpiSlotRows;
             p.M = K; p.K = I; p.m_blocks = (K + 127) / 128;
             p.grouped = 1; p.num_groups = E; p.offsets = offsets; p.tile_start = tiles;
             p.sorted_slot = sorted_slot; p.topk_w = topk_w; p.k = k;
             p.bias0 = c->has_expert_bias ? w->down_b : nullptr;
-            p.out = y_acc; p.ld_out = K;
+            p.out = at<float>(ws, L.oslot); p.ld_out = K;
             if (!tc_weight_map(&P.a0[np], w->down_w, E, K, I, false) || !tc_token_map(&P.b[np], h, S, I, kTcBN))
                 return MOE_ERR_CUDA;
             max_tiles += int64_t(p.m_blocks) * max_routed_tiles(*c, T);
@@ -398,17 +401,29 @@ moe_status run_experts_tc(const moe_config* c, const moe_weights* w, const void*
     return MOE_OK;
 }
 
-// a4 + a5 (+ a6 when with_shared): y_acc must be zero on entry.
+// Where the routed sum lives after run_experts: token t's sum is the sum of rows
+// [t*nsum, (t+1)*nsum) of `rows` (width K).
+struct RoutedSum {
+    const float* rows = nullptr;
+    int nsum = 1;
+};
+
+// a4 + a5 (+ a6 when with_shared). On the weight-streaming path y_acc must be zero on
+// entry (scatter-add); the tensor-core path writes per-slot rows instead.
 moe_status run_experts(const moe_config* c, const moe_weights* w, const void* u, const void* x, int64_t T,
                        const int32_t* offsets, const int32_t* sorted_slot, const float* topk_w,
                        float* y_acc, bool with_routed, bool with_shared, void* ws, const WsLayout& L,
-                       cudaStream_t s) {
+                       cudaStream_t s, RoutedSum* sum) {
     const int K = expert_in(*c);
     const bool sh = with_shared && c->shared_mode != MOE_SHARED_NONE;
     const bool rtc = with_routed && routed_tc(c, T);
     const bool stc = sh && c->shared_intermediate % 64 == 0 && dense_tc(c, T, c->hidden);
+    if (sum) {
+        sum->rows = rtc ? at<float>(ws, L.oslot) : y_acc;
+        sum->nsum = rtc ? c->top_k : 1;
+    }
     if (rtc || stc)
-        MOE_CHECK(run_experts_tc(c, w, u, x, T, offsets, sorted_slot, topk_w, y_acc, rtc, stc, ws, L, s));
+        MOE_CHECK(run_experts_tc(c, w, u, x, T, offsets, sorted_slot, topk_w, rtc, stc, ws, L, s));
     const int64_t groups = (with_routed && !rtc) ? std::min<int64_t>(c->num_experts, T * c->top_k) : 0;
     if (groups == 0 && (!sh || stc)) return MOE_OK;
     GateUpArgs g;
@@ -500,27 +515,23 @@ moe_status run_latent_down(const moe_config* c, const moe_weights* w, const void
 }
 
 // a7 (and the tail of a8): s_acc already holds the shared expert when shared_mode != NONE.
-moe_status run_output(const moe_config* c, const moe_weights* w, const float* y_acc, const float* coef,
+moe_status run_output(const moe_config* c, const moe_weights* w, RoutedSum rs, const float* coef,
                       int64_t T, void* y, void* ws, const WsLayout& L, cudaStream_t s) {
     const float* s_acc = c->shared_mode != MOE_SHARED_NONE ? at<float>(ws, L.s_acc) : nullptr;
     if (!c->latent_dim) {
-        MOE_CUDA(launch_combine(y_acc, s_acc, coef, c->shared_mode, T, c->hidden, y, c->act_dtype, s));
+        MOE_CUDA(launch_combine(rs.rows, rs.nsum, s_acc, coef, c->shared_mode, T, c->hidden, y, c->act_dtype, s));
         return MOE_OK;
     }
-    const void* n = y_acc;
-    bool n_f32 = true;
+    const void* n = nullptr;
     if (c->latent_use_norm) {
-        MOE_CUDA(launch_rmsnorm(y_acc, w->latent_norm_w, c->rms_eps, T, c->latent_dim, at<void>(ws, L.nrm),
-                                c->act_dtype, s));
-        n = at<void>(ws, L.nrm);
-        n_f32 = false;
+        MOE_CUDA(launch_rmsnorm(rs.rows, rs.nsum, w->latent_norm_w, c->rms_eps, T, c->latent_dim,
+                                at<void>(ws, L.nrm), c->act_dtype, s));
+    } else {
+        // no norm: the routed latent sum rounded to the activation dtype
+        MOE_CUDA(launch_combine(rs.rows, rs.nsum, nullptr, nullptr, MOE_SHARED_NONE, T, c->latent_dim,
+                                at<void>(ws, L.nrm), c->act_dtype, s));
     }
-    if (n_f32) {
-        // no norm: round the routed latent sum to the activation dtype first
-        MOE_CUDA(launch_combine(y_acc, nullptr, nullptr, MOE_SHARED_NONE, T, c->latent_dim, at<void>(ws, L.nrm),
-                                c->act_dtype, s));
-        n = at<void>(ws, L.nrm);
-    }
+    n = at<void>(ws, L.nrm);
     if (c->shared_mode == MOE_SHARED_BLEND) return MOE_ERR_UNSUPPORTED;  // rejected earlier
     DenseGemvArgs r;
     r.W0 = w->latent_up_w;
@@ -620,7 +631,13 @@ moe_status moe_grouped_ffn(const moe_config* cfg, const moe_weights* w, const vo
     MOE_CUDA(launch_active_list(expert_offsets, cfg->num_experts, at<int32_t>(ws, L.active), s));
     if (routed_tc(cfg, T))
         MOE_CUDA(launch_tile_start(expert_offsets, cfg->num_experts, kTcBN, at<int32_t>(ws, L.tiles), s));
-    return run_experts(cfg, w, u, nullptr, T, expert_offsets, sorted_slot, topk_w, y_acc, true, false, ws, L, s);
+    RoutedSum rs;
+    MOE_CHECK(run_experts(cfg, w, u, nullptr, T, expert_offsets, sorted_slot, topk_w, y_acc, true, false, ws, L, s,
+                          &rs));
+    if (rs.rows != y_acc)  // per-slot rows: sum each token's k rows into y_acc
+        MOE_CUDA(launch_combine(rs.rows, rs.nsum, nullptr, nullptr, MOE_SHARED_NONE, T, expert_in(*cfg), y_acc,
+                                cfg->act_dtype, s, true));
+    return MOE_OK;
 }
 
 moe_status moe_latent_down(const moe_config* cfg, const moe_weights* w, const void* x, int64_t T, void* z,
@@ -647,8 +664,11 @@ moe_status moe_combine(const moe_config* cfg, const moe_weights* w, const float*
     if (cfg->shared_mode == MOE_SHARED_BLEND) MOE_CHECK(check_ptr(coef));
     cudaStream_t s = (cudaStream_t)stream;
     if (cfg->shared_mode != MOE_SHARED_NONE)
-        MOE_CHECK(run_experts(cfg, w, nullptr, x, T, nullptr, nullptr, nullptr, nullptr, false, true, ws, L, s));
-    return run_output(cfg, w, y_acc, coef, T, y, ws, L, s);
+        MOE_CHECK(run_experts(cfg, w, nullptr, x, T, nullptr, nullptr, nullptr, nullptr, false, true, ws, L, s,
+                              nullptr));
+    RoutedSum rs;
+    rs.rows = y_acc;
+    return run_output(cfg, w, rs, coef, T, y, ws, L, s);
 }
 
 moe_status moe_block_forward(const moe_config* cfg, const moe_weights* w, const void* x, int64_t T, void* y,
@@ -665,7 +685,9 @@ moe_status moe_block_forward(const moe_config* cfg, const moe_weights* w, const 
     int32_t* idx = at<int32_t>(ws, L.topk_idx);
     float* wts = at<float>(ws, L.topk_w);
     float* coef = at<float>(ws, L.coef);
-    MOE_CHECK(run_route(cfg, w, x, T, idx, wts, coef, y_acc, K, ws, L, s));
+    // the weight-streaming path scatter-adds into y_acc: its rows are cleared by the router
+    const bool rtc = routed_tc(cfg, T);
+    MOE_CHECK(run_route(cfg, w, x, T, idx, wts, coef, rtc ? nullptr : y_acc, K, ws, L, s));
     const void* u = x;
     if (cfg->latent_dim) {
         MOE_CHECK(run_latent_down(cfg, w, x, T, at<void>(ws, L.z), at<int>(ws, L.status), s));
@@ -673,10 +695,10 @@ moe_status moe_block_forward(const moe_config* cfg, const moe_weights* w, const 
     }
     int32_t* offsets = at<int32_t>(ws, L.offsets);
     int32_t* sorted_slot = at<int32_t>(ws, L.sorted_slot);
-    MOE_CHECK(run_permute(cfg, idx, T, offsets, sorted_slot, at<int32_t>(ws, L.slot_pos), ws, L, s,
-                          routed_tc(cfg, T)));
-    MOE_CHECK(run_experts(cfg, w, u, x, T, offsets, sorted_slot, wts, y_acc, true, true, ws, L, s));
-    return run_output(cfg, w, y_acc, coef, T, y, ws, L, s);
+    MOE_CHECK(run_permute(cfg, idx, T, offsets, sorted_slot, at<int32_t>(ws, L.slot_pos), ws, L, s, rtc));
+    RoutedSum rs;
+    MOE_CHECK(run_experts(cfg, w, u, x, T, offsets, sorted_slot, wts, y_acc, true, true, ws, L, s, &rs));
+    return run_output(cfg, w, rs, coef, T, y, ws, L, s);
 }
 
 moe_status moe_read_device_status(void* ws, moe_stream_t stream) {

@@ -12,16 +12,28 @@ namespace moe {
 
 namespace {
 
+__device__ __forceinline__ float4 routed_sum(const float* __restrict__ rows, int nsum, int64_t t, int64_t c4,
+                                             int H4) {
+    const float4* p = reinterpret_cast<const float4*>(rows) + (t * nsum) * H4 + c4;
+    float4 r = p[0];
+    for (int j = 1; j < nsum; ++j) {
+        const float4 v = p[int64_t(j) * H4];
+        r.x += v.x; r.y += v.y; r.z += v.z; r.w += v.w;
+    }
+    return r;
+}
+
 template <typename AT>
-__global__ void __launch_bounds__(256) combine_kernel(const float* __restrict__ y_acc,
+__global__ void __launch_bounds__(256) combine_kernel(const float* __restrict__ rows, int nsum,
                                                       const float* __restrict__ s_acc,
                                                       const float* __restrict__ coef, int mode,
                                                       int64_t T, int H, AT* __restrict__ y) {
-    const int64_t n4 = T * H / 4;
+    const int H4 = H / 4;
+    const int64_t n4 = T * H4;
     for (int64_t i = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; i < n4;
          i += int64_t(gridDim.x) * blockDim.x) {
-        const int64_t t = (i * 4) / H;
-        float4 r = reinterpret_cast<const float4*>(y_acc)[i];
+        const int64_t t = i / H4;
+        float4 r = routed_sum(rows, nsum, t, i - t * H4, H4);
         if (mode != MOE_SHARED_NONE) {
             const float4 sv = reinterpret_cast<const float4*>(s_acc)[i];
             if (mode == MOE_SHARED_ADD) {
@@ -43,14 +55,20 @@ __global__ void __launch_bounds__(256) combine_kernel(const float* __restrict__ 
 }
 
 template <typename AT>
-__global__ void __launch_bounds__(256) rmsnorm_kernel(const float* __restrict__ y_acc,
+__global__ void __launch_bounds__(256) rmsnorm_kernel(const float* __restrict__ rows, int nsum,
                                                       const AT* __restrict__ gamma, float eps,
                                                       int L, AT* __restrict__ out) {
+    extern __shared__ float rsum[];   // the routed sum of this token, L floats
     __shared__ float red[8];
     const int64_t t = blockIdx.x;
-    const float* row = y_acc + t * L;
+    const int L4 = L / 4;
     float ss = 0.f;
-    for (int c = threadIdx.x; c < L; c += blockDim.x) ss = fmaf(row[c], row[c], ss);
+    for (int c4 = threadIdx.x; c4 < L4; c4 += blockDim.x) {
+        const float4 v = routed_sum(rows, nsum, t, c4, L4);
+        reinterpret_cast<float4*>(rsum)[c4] = v;
+        ss = fmaf(v.x, v.x, fmaf(v.y, v.y, fmaf(v.z, v.z, fmaf(v.w, v.w, ss))));
+    }
+    const float* row = rsum;
     ss = warp_sum(ss);
     if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = ss;
     __syncthreads();
@@ -64,28 +82,33 @@ __global__ void __launch_bounds__(256) rmsnorm_kernel(const float* __restrict__ 
 
 }  // namespace
 
-cudaError_t launch_combine(const float* y_acc, const float* s_acc, const float* coef, int mode,
-                           int64_t T, int H, void* y, int act_dtype, cudaStream_t s) {
+cudaError_t launch_combine(const float* rows, int nsum, const float* s_acc, const float* coef, int mode,
+                           int64_t T, int H, void* y, int act_dtype, cudaStream_t s, bool out_f32) {
     if (T == 0) return cudaSuccess;
     const int64_t n4 = T * H / 4;
     const unsigned grid = unsigned(std::min<int64_t>((n4 + 255) / 256, 148 * 16));
-    if (act_dtype == kF32)
-        combine_kernel<float><<<grid, 256, 0, s>>>(y_acc, s_acc, coef, mode, T, H, static_cast<float*>(y));
+    if (act_dtype == kF32 || out_f32)
+        combine_kernel<float><<<grid, 256, 0, s>>>(rows, nsum, s_acc, coef, mode, T, H, static_cast<float*>(y));
     else
-        combine_kernel<__nv_bfloat16><<<grid, 256, 0, s>>>(y_acc, s_acc, coef, mode, T, H,
+        combine_kernel<__nv_bfloat16><<<grid, 256, 0, s>>>(rows, nsum, s_acc, coef, mode, T, H,
                                                            static_cast<__nv_bfloat16*>(y));
     return cudaGetLastError();
 }
 
-cudaError_t launch_rmsnorm(const float* y_acc, const void* gamma, float eps, int64_t T, int L,
+cudaError_t launch_rmsnorm(const float* rows, int nsum, const void* gamma, float eps, int64_t T, int L,
                            void* out, int act_dtype, cudaStream_t s) {
     if (T == 0) return cudaSuccess;
-    if (act_dtype == kF32)
-        rmsnorm_kernel<float><<<unsigned(T), 256, 0, s>>>(y_acc, static_cast<const float*>(gamma), eps, L,
-                                                          static_cast<float*>(out));
-    else
-        rmsnorm_kernel<__nv_bfloat16><<<unsigned(T), 256, 0, s>>>(
-            y_acc, static_cast<const __nv_bfloat16*>(gamma), eps, L, static_cast<__nv_bfloat16*>(out));
+    const size_t smem = size_t(L) * sizeof(float);
+    if (act_dtype == kF32) {
+        cudaFuncSetAttribute(rmsnorm_kernel<float>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
+        rmsnorm_kernel<float><<<unsigned(T), 256, smem, s>>>(rows, nsum, static_cast<const float*>(gamma), eps, L,
+                                                             static_cast<float*>(out));
+    } else {
+        cudaFuncSetAttribute(rmsnorm_kernel<__nv_bfloat16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             int(smem));
+        rmsnorm_kernel<__nv_bfloat16><<<unsigned(T), 256, smem, s>>>(
+            rows, nsum, static_cast<const __nv_bfloat16*>(gamma), eps, L, static_cast<__nv_bfloat16*>(out));
+    }
     return cudaGetLastError();
 }
 

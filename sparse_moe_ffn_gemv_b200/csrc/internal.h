@@ -81,16 +81,18 @@ struct DownArgs {
 };
 cudaError_t launch_down_gemv(const DownArgs& a, cudaStream_t s);
 
-// y = y_acc | y_acc + s | c0 y_acc + c1 s, stored in act dtype.
-cudaError_t launch_combine(const float* y_acc, const float* s_acc, const float* coef, int mode,
-                           int64_t T, int H, void* y, int act_dtype, cudaStream_t s);
-// nrm = y_acc / sqrt(mean(y_acc^2) + eps) * gamma (act dtype), per token row of width L.
-cudaError_t launch_rmsnorm(const float* y_acc, const void* gamma, float eps, int64_t T, int L,
+// The routed sum of token t is the sum of rows [t*nsum, (t+1)*nsum) of `rows` (width H):
+// nsum = 1 for an accumulated [T, H] buffer, nsum = k for per-slot weighted rows.
+// y = r | r + s | c0 r + c1 s, stored in act dtype (or f32 when out_f32).
+cudaError_t launch_combine(const float* rows, int nsum, const float* s_acc, const float* coef, int mode,
+                           int64_t T, int H, void* y, int act_dtype, cudaStream_t s, bool out_f32 = false);
+// nrm = r / sqrt(mean(r^2) + eps) * gamma (act dtype), r the routed sum as above (width L).
+cudaError_t launch_rmsnorm(const float* rows, int nsum, const void* gamma, float eps, int64_t T, int L,
                            void* out, int act_dtype, cudaStream_t s);
 
 // ------------------------------------------------------------------ tensor-core GEMM
 constexpr int kTcBN = 128;  // token columns per tile
-enum { kEpiGateUp = 0, kEpiScatter = 1, kEpiStoreF32 = 2, kEpiStoreAct = 3 };
+enum { kEpiGateUp = 0, kEpiSlotRows = 1, kEpiStoreF32 = 2, kEpiStoreAct = 3 };
 
 // One GEMM problem of a tensor-core launch: D[M rows, tokens] = W[M, K] . U[tokens, K]^T.
 struct TcProblem {
@@ -101,8 +103,8 @@ struct TcProblem {
     int num_groups = 0;
     const int32_t* offsets = nullptr;      // [E + 1] sorted-row offsets of the groups
     const int32_t* tile_start = nullptr;   // [E + 1] prefix of token tiles per group
-    const int32_t* sorted_slot = nullptr;  // scatter: sorted row -> slot
-    const float* topk_w = nullptr;         // scatter: slot -> combine weight
+    const int32_t* sorted_slot = nullptr;  // slot rows: sorted row -> slot
+    const float* topk_w = nullptr;         // slot rows: slot -> combine weight
     int k = 1;
     const void* bias0 = nullptr;           // bf16 [groups, M] (or [groups, 2M] interleaved gate/up)
     const void* bias1 = nullptr;           // bf16 [groups, M] (up bias, separate layout)

@@ -10,7 +10,7 @@
 //   warp 1      MMA issuer (one thread): tcgen05.mma kind::f16, bf16 x bf16 -> fp32 in
 //               TMEM; two accumulators (gate, up) in gate/up mode
 //   warps 2..5  epilogue: tcgen05.ld, then SwiGLU / clamped SwiGLU -> bf16 h (gate/up),
-//               weighted scatter-add into the fp32 routed sum (down), or a plain store
+//               the weighted fp32 output row of every slot (down), or a plain store
 // TMEM holds two accumulator sets so the epilogue of one tile overlaps the main loop of
 // the next. Every mbarrier wait is bounded by %globaltimer; a wait that gives up records
 // MOE_ERR_DEVICE_TIMEOUT in the status word, drains its own outstanding copies / MMAs and
@@ -381,15 +381,15 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
                             out[int64_t(ti.row0 + n) * p.ld_out + r] =
                                 __float2bfloat16_rn(act_apply(P.act, g[j] + bias0, u[j] + bias1, P.limit, P.alpha));
                     }
-                } else if (p.mode == kEpiScatter) {
+                } else if (p.mode == kEpiSlotRows) {
+                    // weighted output row of each slot; the combine sums a token's k rows
                     float* out = reinterpret_cast<float*>(p.out);
 #pragma unroll 4
                     for (int j = 0; j < 32; ++j) {
                         const int n = c + j;
                         if (rv && n < ti.nvalid) {
                             const int slot = p.sorted_slot[ti.row0 + n];
-                            const int64_t token = slot / p.k;
-                            atomicAdd(out + token * p.ld_out + r, p.topk_w[slot] * (g[j] + bias0));
+                            out[int64_t(slot) * p.ld_out + r] = p.topk_w[slot] * (g[j] + bias0);
                         }
                     }
                 } else if (p.mode == kEpiStoreF32) {
