@@ -9,7 +9,8 @@
 //               STAGES-deep shared-memory ring (128-byte swizzle)
 //   warp 1      MMA issuer (one thread): tcgen05.mma kind::f16, bf16 x bf16 -> fp32 in
 //               TMEM; two accumulators (gate, up) in gate/up mode
-//   warps 2..5  epilogue: tcgen05.ld, then SwiGLU / clamped SwiGLU -> bf16 h (gate/up),
+//   warps 2..9  epilogue (two warps per TMEM lane quarter, each half of the columns):
+//               tcgen05.ld, then SwiGLU / clamped SwiGLU -> bf16 h (gate/up),
 //               the weighted fp32 output row of every slot (down), or a plain store
 // TMEM holds two accumulator sets so the epilogue of one tile overlaps the main loop of
 // the next. Every mbarrier wait is bounded by %globaltimer; a wait that gives up records
@@ -31,7 +32,9 @@ namespace {
 
 constexpr int kBM = 128;          // weight rows per tile (MMA M)
 constexpr int kBK = 64;           // K per stage: one 128-byte swizzle atom of bf16
-constexpr int kTcThreads = 192;   // 6 warps
+constexpr int kTcThreads = 320;   // 10 warps: TMA, MMA, 8 epilogue
+constexpr int kEpiThreads = 256;
+constexpr int kMaxGroups = 512;   // expert groups whose tile table fits in shared memory
 constexpr uint64_t kWaitNs = 2000000000ull;  // 2 s bound on any single wait
 
 __device__ __forceinline__ uint32_t su32(const void* p) {
@@ -70,28 +73,43 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* b, uint32_t parity, uint64_t
     }
 }
 
-__device__ __forceinline__ void tma_2d(void* dst, const CUtensorMap* m, uint64_t* bar, int c0, int c1) {
+// L2 policies: weights stream through once (evict first); token tiles are re-read by
+// every weight-row block of their group (evict last).
+__device__ __forceinline__ uint64_t policy_evict_first() {
+    uint64_t p;
+    asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
+    return p;
+}
+__device__ __forceinline__ uint64_t policy_evict_last() {
+    uint64_t p;
+    asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(p));
+    return p;
+}
+__device__ __forceinline__ void tma_2d(void* dst, const CUtensorMap* m, uint64_t* bar, int c0, int c1,
+                                       uint64_t pol) {
     asm volatile(
-        "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
-        " [%0], [%1, {%3, %4}], [%2];" ::"r"(su32(dst)),
-        "l"(reinterpret_cast<uint64_t>(m)), "r"(su32(bar)), "r"(c0), "r"(c1)
+        "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes.L2::cache_hint"
+        " [%0], [%1, {%3, %4}], [%2], %5;" ::"r"(su32(dst)),
+        "l"(reinterpret_cast<uint64_t>(m)), "r"(su32(bar)), "r"(c0), "r"(c1), "l"(pol)
         : "memory");
 }
-__device__ __forceinline__ void tma_3d(void* dst, const CUtensorMap* m, uint64_t* bar, int c0, int c1, int c2) {
+__device__ __forceinline__ void tma_3d(void* dst, const CUtensorMap* m, uint64_t* bar, int c0, int c1, int c2,
+                                       uint64_t pol) {
     asm volatile(
-        "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
-        " [%0], [%1, {%3, %4, %5}], [%2];" ::"r"(su32(dst)),
-        "l"(reinterpret_cast<uint64_t>(m)), "r"(su32(bar)), "r"(c0), "r"(c1), "r"(c2)
+        "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes.L2::cache_hint"
+        " [%0], [%1, {%3, %4, %5}], [%2], %6;" ::"r"(su32(dst)),
+        "l"(reinterpret_cast<uint64_t>(m)), "r"(su32(bar)), "r"(c0), "r"(c1), "r"(c2), "l"(pol)
         : "memory");
 }
 __device__ __forceinline__ void tma_4d(void* dst, const CUtensorMap* m, uint64_t* bar, int c0, int c1, int c2,
-                                       int c3) {
+                                       int c3, uint64_t pol) {
     asm volatile(
-        "cp.async.bulk.tensor.4d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
-        " [%0], [%1, {%3, %4, %5, %6}], [%2];" ::"r"(su32(dst)),
-        "l"(reinterpret_cast<uint64_t>(m)), "r"(su32(bar)), "r"(c0), "r"(c1), "r"(c2), "r"(c3)
+        "cp.async.bulk.tensor.4d.shared::cluster.global.tile.mbarrier::complete_tx::bytes.L2::cache_hint"
+        " [%0], [%1, {%3, %4, %5, %6}], [%2], %7;" ::"r"(su32(dst)),
+        "l"(reinterpret_cast<uint64_t>(m)), "r"(su32(bar)), "r"(c0), "r"(c1), "r"(c2), "r"(c3), "l"(pol)
         : "memory");
 }
+__device__ __forceinline__ void epi_bar() { asm volatile("bar.sync 1, %0;" ::"r"(kEpiThreads) : "memory"); }
 __device__ __forceinline__ void prefetch_tmap(const CUtensorMap* m) {
     asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(m)) : "memory");
 }
@@ -146,12 +164,18 @@ struct TileInfo {
     int nvalid;    // valid token columns
 };
 
-__device__ __forceinline__ int problem_tiles(const TcProblem& p) {
-    if (p.grouped) return p.tile_start[p.num_groups] * p.m_blocks;
+// Tile tables of the (at most one) grouped problem, copied to shared memory at start.
+struct GroupTables {
+    int ts[kMaxGroups + 1];   // tile_start
+    int off[kMaxGroups + 1];  // offsets
+};
+
+__device__ __forceinline__ int problem_tiles(const TcProblem& p, const GroupTables& g) {
+    if (p.grouped) return g.ts[p.num_groups] * p.m_blocks;
     return p.n_tiles * p.m_blocks;
 }
 
-__device__ __forceinline__ TileInfo decode_tile(const TcParams& P, int tile, int t0) {
+__device__ __forceinline__ TileInfo decode_tile(const TcParams& P, const GroupTables& gt, int tile, int t0) {
     TileInfo ti;
     int local = tile;
     ti.prob = 0;
@@ -172,18 +196,18 @@ __device__ __forceinline__ TileInfo decode_tile(const TcParams& P, int tile, int
     int lo = 0, hi = p.num_groups - 1;
     while (lo < hi) {
         const int mid = (lo + hi + 1) >> 1;
-        if (p.tile_start[mid] * p.m_blocks <= local) lo = mid;
+        if (gt.ts[mid] * p.m_blocks <= local) lo = mid;
         else hi = mid - 1;
     }
     const int e = lo;
-    const int ts = p.tile_start[e];
-    const int nbe = p.tile_start[e + 1] - ts;
+    const int ts = gt.ts[e];
+    const int nbe = gt.ts[e + 1] - ts;
     const int l = local - ts * p.m_blocks;
     ti.group = e;
     ti.mb = l / nbe;
     const int nb = l - ti.mb * nbe;
-    const int off = p.offsets[e];
-    const int cnt = p.offsets[e + 1] - off;
+    const int off = gt.off[e];
+    const int cnt = gt.off[e + 1] - off;
     ti.row0 = off + nb * p.bn;
     ti.nvalid = min(p.bn, cnt - nb * p.bn);
     return ti;
@@ -196,10 +220,19 @@ struct TcShape {
     static constexpr int STAGE_BYTES = A_BYTES * (GATEUP ? 2 : 1) + B_BYTES;
     static constexpr int ACC_COLS = GATEUP ? 2 * BN : BN;        // per accumulator set
     static constexpr int TMEM_COLS = 2 * ACC_COLS;               // double-buffered
-    static constexpr int SMEM = STAGES * STAGE_BYTES + 1024 /*align*/ + 256 /*barriers*/;
+    static constexpr int SMEM = STAGES * STAGE_BYTES + 1024 /*align*/ + 256 /*barriers*/ +
+                                int(sizeof(GroupTables)) + 2 * BN * 4 /*epilogue slot, weight*/;
     static_assert(TMEM_COLS <= 512 && (TMEM_COLS & (TMEM_COLS - 1)) == 0, "TMEM columns");
     static_assert(BN % 32 == 0 && BN >= 32 && BN <= 256, "BN");
 };
+
+// SwiGLU / clamped SwiGLU with the fast exponential (the result is rounded to bf16).
+__device__ __forceinline__ float act_fast(int act, float g, float v, float limit, float alpha) {
+    if (act == MOE_ACT_SWIGLU) return __fdividef(g, 1.0f + __expf(-g)) * v;
+    const float gc = fminf(g, limit);
+    const float vc = fminf(fmaxf(v, -limit), limit);
+    return __fdividef(gc, 1.0f + __expf(-alpha * gc)) * (vc + 1.0f);
+}
 
 __device__ __forceinline__ float bf16_at(const void* p, int64_t i) {
     return __bfloat162float(reinterpret_cast<const __nv_bfloat16*>(p)[i]);
@@ -216,6 +249,9 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
     uint64_t* acc_empty = acc_full + 2;
     uint64_t* drain = acc_empty + 2;
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+    GroupTables& gt = *reinterpret_cast<GroupTables*>(smem + STAGES * S::STAGE_BYTES + 256);
+    int* e_slot = reinterpret_cast<int*>(&gt + 1);
+    float* e_w = reinterpret_cast<float*>(e_slot + BN);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     if (warp == 0) {
@@ -230,7 +266,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
         }
         for (int b = 0; b < 2; ++b) {
             mbar_init(&acc_full[b], 1);
-            mbar_init(&acc_empty[b], 4);  // one arrive per epilogue warp
+            mbar_init(&acc_empty[b], kEpiThreads / 32);  // one arrive per epilogue warp
         }
         mbar_init(drain, 1);
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -243,13 +279,20 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
             prefetch_tmap(&P.b[i]);
         }
     }
+    for (int i = 0; i < P.nprob; ++i) {
+        if (!P.p[i].grouped) continue;
+        for (int e = threadIdx.x; e <= P.p[i].num_groups; e += blockDim.x) {
+            gt.ts[e] = P.p[i].tile_start[e];
+            gt.off[e] = P.p[i].offsets[e];
+        }
+    }
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem_base = *tmem_slot;
 
-    const int t0 = problem_tiles(P.p[0]);
-    const int total = t0 + (P.nprob > 1 ? problem_tiles(P.p[1]) : 0);
+    const int t0 = problem_tiles(P.p[0], gt);
+    const int total = t0 + (P.nprob > 1 ? problem_tiles(P.p[1], gt) : 0);
     const uint64_t deadline = gtimer() + kWaitNs;
     bool timed_out = false;
 
@@ -259,8 +302,9 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
             uint32_t stage = 0, phase = 0;
             uint32_t armed = 0;  // bit s: stage s was filled at least once
             uint32_t last_par = 0;
+            const uint64_t pol_w = policy_evict_first(), pol_t = policy_evict_last();
             for (int tile = blockIdx.x; tile < total && !timed_out; tile += gridDim.x) {
-                const TileInfo ti = decode_tile(P, tile, t0);
+                const TileInfo ti = decode_tile(P, gt, tile, t0);
                 const TcProblem& p = P.p[ti.prob];
                 const int nk = p.K / kBK;
                 for (int kb = 0; kb < nk; ++kb) {
@@ -273,13 +317,14 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
                     const int kc = kb * kBK;
                     const int mrow = ti.mb * kBM;
                     if (p.interleaved) {  // [E, I, 2, K]: plane 0 = gate rows, 1 = up rows
-                        tma_4d(sb, &P.a0[ti.prob], &full[stage], kc, 0, mrow, ti.group);
-                        if (GATEUP) tma_4d(sb + S::A_BYTES, &P.a0[ti.prob], &full[stage], kc, 1, mrow, ti.group);
+                        tma_4d(sb, &P.a0[ti.prob], &full[stage], kc, 0, mrow, ti.group, pol_w);
+                        if (GATEUP)
+                            tma_4d(sb + S::A_BYTES, &P.a0[ti.prob], &full[stage], kc, 1, mrow, ti.group, pol_w);
                     } else {
-                        tma_3d(sb, &P.a0[ti.prob], &full[stage], kc, mrow, ti.group);
-                        if (GATEUP) tma_3d(sb + S::A_BYTES, &P.a1[ti.prob], &full[stage], kc, mrow, ti.group);
+                        tma_3d(sb, &P.a0[ti.prob], &full[stage], kc, mrow, ti.group, pol_w);
+                        if (GATEUP) tma_3d(sb + S::A_BYTES, &P.a1[ti.prob], &full[stage], kc, mrow, ti.group, pol_w);
                     }
-                    tma_2d(sb + S::A_BYTES * (GATEUP ? 2 : 1), &P.b[ti.prob], &full[stage], kc, ti.row0);
+                    tma_2d(sb + S::A_BYTES * (GATEUP ? 2 : 1), &P.b[ti.prob], &full[stage], kc, ti.row0, pol_t);
                     armed |= 1u << stage;
                     last_par = (last_par & ~(1u << stage)) | (phase << stage);
                     if (++stage == STAGES) {
@@ -300,7 +345,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
             uint32_t stage = 0, phase = 0, it = 0;
             constexpr uint32_t idesc = idesc_bf16(BN);
             for (int tile = blockIdx.x; tile < total && !timed_out; tile += gridDim.x, ++it) {
-                const TileInfo ti = decode_tile(P, tile, t0);
+                const TileInfo ti = decode_tile(P, gt, tile, t0);
                 const TcProblem& p = P.p[ti.prob];
                 const uint32_t ab = it & 1u, aph = (it >> 1) & 1u;
                 if (!mbar_wait(&acc_empty[ab], aph ^ 1u, deadline)) {
@@ -340,12 +385,14 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
             if (timed_out) set_status(P.status, MOE_ERR_DEVICE_TIMEOUT);
         }
     } else {
-        // -------------------------------------------------------------- epilogue (128 threads)
+        // -------------------------------------------------------------- epilogue (256 threads)
         const int q = warp & 3;                  // TMEM lane quarter of this warp
         const int lrow = q * 32 + lane;          // accumulator row = weight row in the tile
+        const int eid = threadIdx.x - 64;        // 0..255
+        const int c_lo = (eid >= 128) ? BN / 2 : 0;  // this warp's half of the columns
         uint32_t it = 0;
         for (int tile = blockIdx.x; tile < total; tile += gridDim.x, ++it) {
-            const TileInfo ti = decode_tile(P, tile, t0);
+            const TileInfo ti = decode_tile(P, gt, tile, t0);
             const TcProblem& p = P.p[ti.prob];
             const uint32_t ab = it & 1u, aph = (it >> 1) & 1u;
             if (!mbar_wait(&acc_full[ab], aph, deadline)) {
@@ -353,6 +400,15 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
                 break;
             }
             tc_fence_after();
+            if (!GATEUP && p.mode == kEpiSlotRows) {  // the tile's slot ids and weights, once
+                epi_bar();
+                if (eid < BN && eid < ti.nvalid) {
+                    const int slot = p.sorted_slot[ti.row0 + eid];
+                    e_slot[eid] = slot;
+                    e_w[eid] = p.topk_w[slot];
+                }
+                epi_bar();
+            }
             const uint32_t tbase = tmem_base + (uint32_t(q * 32) << 16) + ab * S::ACC_COLS;
             const int r = ti.mb * kBM + lrow;    // weight row (intermediate unit or output row)
             const bool rv = r < p.M;
@@ -367,7 +423,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
                 }
             }
 #pragma unroll 1
-            for (int c = 0; c < BN; c += 32) {
+            for (int c = c_lo; c < c_lo + BN / 2; c += 32) {
                 float g[32];
                 tmem_ld32(tbase + c, g);
                 if constexpr (GATEUP) {
@@ -379,7 +435,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
                         const int n = c + j;
                         if (rv && n < ti.nvalid)
                             out[int64_t(ti.row0 + n) * p.ld_out + r] =
-                                __float2bfloat16_rn(act_apply(P.act, g[j] + bias0, u[j] + bias1, P.limit, P.alpha));
+                                __float2bfloat16_rn(act_fast(P.act, g[j] + bias0, u[j] + bias1, P.limit, P.alpha));
                     }
                 } else if (p.mode == kEpiSlotRows) {
                     // weighted output row of each slot; the combine sums a token's k rows
@@ -387,10 +443,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
 #pragma unroll 4
                     for (int j = 0; j < 32; ++j) {
                         const int n = c + j;
-                        if (rv && n < ti.nvalid) {
-                            const int slot = p.sorted_slot[ti.row0 + n];
-                            out[int64_t(slot) * p.ld_out + r] = p.topk_w[slot] * (g[j] + bias0);
-                        }
+                        if (rv && n < ti.nvalid) out[int64_t(e_slot[n]) * p.ld_out + r] = e_w[n] * (g[j] + bias0);
                     }
                 } else if (p.mode == kEpiStoreF32) {
                     float* out = reinterpret_cast<float*>(p.out);
