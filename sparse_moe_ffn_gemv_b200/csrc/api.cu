@@ -239,7 +239,7 @@ moe_status run_route(const moe_config* c, const moe_weights* w, const void* x, i
             p.mode = kEpiStoreF32;
             p.M = i == 0 ? c->num_experts : 2;
             p.K = c->hidden;
-            p.m_blocks = (p.M + 127) / 128;
+            p.m_blocks = (p.M + kTcRows - 1) / kTcRows;
             p.rows = int(T);
             p.n_tiles = int((T + kTcBN - 1) / kTcBN);
             p.bias0 = i == 0 ? r.b0 : r.b1;
@@ -321,7 +321,7 @@ moe_status run_experts_tc(const moe_config* c, const moe_weights* w, const void*
         if (stc) {
             TcProblem& p = P.p[np];
             p.mode = kEpiGateUp;
-            p.M = Is; p.K = H; p.m_blocks = (Is + 127) / 128;
+            p.M = Is; p.K = H; p.m_blocks = (Is + kTcRowsGateUp - 1) / kTcRowsGateUp;
             p.rows = int(T); p.n_tiles = int(n_dense);
             p.out = hs; p.ld_out = Is;
             if (!tc_weight_map(&P.a0[np], w->shared_gate_w, 1, Is, H, false) ||
@@ -334,7 +334,7 @@ moe_status run_experts_tc(const moe_config* c, const moe_weights* w, const void*
         if (rtc) {
             TcProblem& p = P.p[np];
             p.mode = kEpiGateUp;
-            p.M = I; p.K = K; p.m_blocks = (I + 127) / 128;
+            p.M = I; p.K = K; p.m_blocks = (I + kTcRowsGateUp - 1) / kTcRowsGateUp;
             p.grouped = 1; p.num_groups = E; p.offsets = offsets; p.tile_start = tiles;
             p.out = h; p.ld_out = I;
             p.interleaved = c->gate_up_interleaved;
@@ -372,7 +372,7 @@ moe_status run_experts_tc(const moe_config* c, const moe_weights* w, const void*
         if (stc) {
             TcProblem& p = P.p[np];
             p.mode = kEpiStoreF32;
-            p.M = H; p.K = Is; p.m_blocks = (H + 127) / 128;
+            p.M = H; p.K = Is; p.m_blocks = (H + kTcRows - 1) / kTcRows;
             p.rows = int(T); p.n_tiles = int(n_dense);
             p.out = at<float>(ws, L.s_acc); p.ld_out = H;
             if (!tc_weight_map(&P.a0[np], w->shared_down_w, 1, H, Is, false) ||
@@ -384,7 +384,7 @@ moe_status run_experts_tc(const moe_config* c, const moe_weights* w, const void*
         if (rtc) {
             TcProblem& p = P.p[np];
             p.mode = kEpiSlotRows;
-            p.M = K; p.K = I; p.m_blocks = (K + 127) / 128;
+            p.M = K; p.K = I; p.m_blocks = (K + kTcRows - 1) / kTcRows;
             p.grouped = 1; p.num_groups = E; p.offsets = offsets; p.tile_start = tiles;
             p.sorted_slot = sorted_slot; p.topk_w = topk_w; p.k = k;
             p.bias0 = c->has_expert_bias ? w->down_b : nullptr;
@@ -500,7 +500,7 @@ moe_status run_latent_down(const moe_config* c, const moe_weights* w, const void
         TcParams P;
         TcProblem& p = P.p[0];
         p.mode = kEpiStoreAct;
-        p.M = c->latent_dim; p.K = c->hidden; p.m_blocks = (p.M + 127) / 128;
+        p.M = c->latent_dim; p.K = c->hidden; p.m_blocks = (p.M + kTcRows - 1) / kTcRows;
         p.rows = int(T); p.n_tiles = int((T + kTcBN - 1) / kTcBN);
         p.out = z; p.ld_out = c->latent_dim;
         if (!tc_weight_map(&P.a0[0], w->latent_down_w, 1, p.M, p.K, false) || !tc_token_map(&P.b[0], x, T, p.K, kTcBN))
@@ -549,7 +549,7 @@ moe_status run_output(const moe_config* c, const moe_weights* w, RoutedSum rs, c
         TcParams P;
         TcProblem& p = P.p[0];
         p.mode = kEpiStoreAct;
-        p.M = c->hidden; p.K = c->latent_dim; p.m_blocks = (p.M + 127) / 128;
+        p.M = c->hidden; p.K = c->latent_dim; p.m_blocks = (p.M + kTcRows - 1) / kTcRows;
         p.rows = int(T); p.n_tiles = int((T + kTcBN - 1) / kTcBN);
         p.out = y; p.ld_out = c->hidden;
         p.addend = s_acc; p.ld_add = c->hidden;

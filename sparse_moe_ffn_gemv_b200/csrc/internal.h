@@ -91,13 +91,15 @@ cudaError_t launch_rmsnorm(const float* rows, int nsum, const void* gamma, float
                            void* out, int act_dtype, cudaStream_t s);
 
 // ------------------------------------------------------------------ tensor-core GEMM
-constexpr int kTcBN = 128;  // token columns per tile
+constexpr int kTcBN = 128;       // token columns per tile
+constexpr int kTcRowsGateUp = 128;  // intermediate units per gate/up tile (gate + up rows)
+constexpr int kTcRows = 256;        // output rows per tile of the other GEMMs
 enum { kEpiGateUp = 0, kEpiSlotRows = 1, kEpiStoreF32 = 2, kEpiStoreAct = 3 };
 
 // One GEMM problem of a tensor-core launch: D[M rows, tokens] = W[M, K] . U[tokens, K]^T.
 struct TcProblem {
     int mode = kEpiStoreF32;
-    int M = 0, K = 0, m_blocks = 0;
+    int M = 0, K = 0, m_blocks = 0;        // m_blocks = ceil(M / rows per tile)
     int grouped = 0;                       // 1: expert groups (offsets / tile_start), 0: one dense group
     int rows = 0, n_tiles = 0, bn = kTcBN; // dense: token rows and their tiles
     int num_groups = 0;

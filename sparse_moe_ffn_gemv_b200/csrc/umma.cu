@@ -1,6 +1,6 @@
 // umma.cu -- tensor-core (tcgen05 / TMEM) grouped GEMM fed by TMA, for prefill-sized batches.
 //
-// D[128 weight rows, BN tokens] = W[128, K] . U[BN, K]^T per tile ("weights as M"): every
+// D[weight rows, BN tokens] = W[rows, K] . U[BN, K]^T per tile ("weights as M"): every
 // expert group is padded only to the token tile, and each weight tile is read from HBM once
 // and shared by the token tiles of its group through L2.
 //
@@ -30,7 +30,7 @@ namespace moe {
 
 namespace {
 
-constexpr int kBM = 128;          // weight rows per tile (MMA M)
+constexpr int kBM = 128;          // weight rows per MMA (M)
 constexpr int kBK = 64;           // K per stage: one 128-byte swizzle atom of bf16
 constexpr int kTcThreads = 320;   // 10 warps: TMA, MMA, 8 epilogue
 constexpr int kEpiThreads = 256;
@@ -213,13 +213,16 @@ __device__ __forceinline__ TileInfo decode_tile(const TcParams& P, const GroupTa
     return ti;
 }
 
+// Every tile carries two 128-row weight operands that share one token tile: the gate and
+// up rows of 128 intermediate units (gate/up), or 256 consecutive output rows (others).
 template <bool GATEUP, int BN, int STAGES>
 struct TcShape {
     static constexpr int A_BYTES = kBM * kBK * 2;                // 16 KB
     static constexpr int B_BYTES = BN * kBK * 2;
-    static constexpr int STAGE_BYTES = A_BYTES * (GATEUP ? 2 : 1) + B_BYTES;
-    static constexpr int ACC_COLS = GATEUP ? 2 * BN : BN;        // per accumulator set
+    static constexpr int STAGE_BYTES = 2 * A_BYTES + B_BYTES;
+    static constexpr int ACC_COLS = 2 * BN;                      // per accumulator set
     static constexpr int TMEM_COLS = 2 * ACC_COLS;               // double-buffered
+    static constexpr int ROWS = GATEUP ? kBM : 2 * kBM;          // weight rows per tile
     static constexpr int SMEM = STAGES * STAGE_BYTES + 1024 /*align*/ + 256 /*barriers*/ +
                                 int(sizeof(GroupTables)) + 2 * BN * 4 /*epilogue slot, weight*/;
     static_assert(TMEM_COLS <= 512 && (TMEM_COLS & (TMEM_COLS - 1)) == 0, "TMEM columns");
@@ -315,16 +318,18 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
                     uint8_t* sb = smem + stage * S::STAGE_BYTES;
                     mbar_expect_tx(&full[stage], S::STAGE_BYTES);
                     const int kc = kb * kBK;
-                    const int mrow = ti.mb * kBM;
-                    if (p.interleaved) {  // [E, I, 2, K]: plane 0 = gate rows, 1 = up rows
+                    const int mrow = ti.mb * S::ROWS;
+                    if (!GATEUP) {  // rows [mrow, mrow + 128) and [mrow + 128, mrow + 256)
+                        tma_3d(sb, &P.a0[ti.prob], &full[stage], kc, mrow, ti.group, pol_w);
+                        tma_3d(sb + S::A_BYTES, &P.a0[ti.prob], &full[stage], kc, mrow + kBM, ti.group, pol_w);
+                    } else if (p.interleaved) {  // [E, I, 2, K]: plane 0 = gate rows, 1 = up rows
                         tma_4d(sb, &P.a0[ti.prob], &full[stage], kc, 0, mrow, ti.group, pol_w);
-                        if (GATEUP)
-                            tma_4d(sb + S::A_BYTES, &P.a0[ti.prob], &full[stage], kc, 1, mrow, ti.group, pol_w);
+                        tma_4d(sb + S::A_BYTES, &P.a0[ti.prob], &full[stage], kc, 1, mrow, ti.group, pol_w);
                     } else {
                         tma_3d(sb, &P.a0[ti.prob], &full[stage], kc, mrow, ti.group, pol_w);
-                        if (GATEUP) tma_3d(sb + S::A_BYTES, &P.a1[ti.prob], &full[stage], kc, mrow, ti.group, pol_w);
+                        tma_3d(sb + S::A_BYTES, &P.a1[ti.prob], &full[stage], kc, mrow, ti.group, pol_w);
                     }
-                    tma_2d(sb + S::A_BYTES * (GATEUP ? 2 : 1), &P.b[ti.prob], &full[stage], kc, ti.row0, pol_t);
+                    tma_2d(sb + 2 * S::A_BYTES, &P.b[ti.prob], &full[stage], kc, ti.row0, pol_t);
                     armed |= 1u << stage;
                     last_par = (last_par & ~(1u << stage)) | (phase << stage);
                     if (++stage == STAGES) {
@@ -362,13 +367,13 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
                     }
                     tc_fence_after();
                     const uint32_t sa = su32(smem + stage * S::STAGE_BYTES);
-                    const uint32_t sbb = sa + S::A_BYTES * (GATEUP ? 2 : 1);
+                    const uint32_t sbb = sa + 2 * S::A_BYTES;
 #pragma unroll
                     for (int k = 0; k < kBK / 16; ++k) {
                         const uint64_t bdesc = smem_desc(sbb + k * 32);
                         const uint32_t acc = (kb > 0 || k > 0) ? 1u : 0u;
                         umma(d0, smem_desc(sa + k * 32), bdesc, idesc, acc);
-                        if (GATEUP) umma(d0 + BN, smem_desc(sa + S::A_BYTES + k * 32), bdesc, idesc, acc);
+                        umma(d0 + BN, smem_desc(sa + S::A_BYTES + k * 32), bdesc, idesc, acc);
                     }
                     umma_commit(&empty[stage]);
                     if (++stage == STAGES) {
@@ -409,8 +414,11 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
                 }
                 epi_bar();
             }
-            const uint32_t tbase = tmem_base + (uint32_t(q * 32) << 16) + ab * S::ACC_COLS;
-            const int r = ti.mb * kBM + lrow;    // weight row (intermediate unit or output row)
+            const uint32_t tbase0 = tmem_base + (uint32_t(q * 32) << 16) + ab * S::ACC_COLS;
+#pragma unroll 1
+            for (int a = 0; a < (GATEUP ? 1 : 2); ++a) {
+            const uint32_t tbase = tbase0 + a * BN;
+            const int r = ti.mb * S::ROWS + a * kBM + lrow;  // weight row (unit or output row)
             const bool rv = r < p.M;
             float bias0 = 0.f, bias1 = 0.f;
             if (rv && p.bias0) {
@@ -465,6 +473,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
                     }
                 }
             }
+            }  // accumulator a
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&acc_empty[ab]);
@@ -552,7 +561,7 @@ bool tc_token_map(CUtensorMap* m, const void* u, int64_t rows, int K, int bn) {
 
 cudaError_t launch_tc_gemm(TcParams& P, bool gateup, int64_t max_tiles, cudaStream_t s) {
     if (gateup) return launch_tc_t<true, kTcBN, 4>(P, max_tiles, s);
-    return launch_tc_t<false, kTcBN, 6>(P, max_tiles, s);
+    return launch_tc_t<false, kTcBN, 4>(P, max_tiles, s);
 }
 
 }  // namespace moe
