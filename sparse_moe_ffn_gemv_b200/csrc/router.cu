@@ -16,103 +16,87 @@ namespace {
 
 constexpr int kPerLane = kMaxExperts / kWarp;  // 16 experts per lane at most
 
+// Order-preserving packing of (selection key, expert): a larger key wins, and among
+// equal keys the lower expert index wins (its complement is larger).
+__device__ __forceinline__ uint64_t pack_key(float key, int e) {
+    uint32_t u = __float_as_uint(key);
+    u = (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+    return (uint64_t(u) << 32) | uint32_t(0xFFFFFFFFu - uint32_t(e));
+}
+
+__device__ __forceinline__ uint64_t warp_max_u64(uint64_t v) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+        const uint64_t w = __shfl_xor_sync(0xffffffffu, v, o);
+        v = w > v ? w : v;
+    }
+    return v;
+}
+
 __global__ void __launch_bounds__(256) topk_kernel(TopkArgs a) {
     const int lane = threadIdx.x & 31;
     const int64_t t = (int64_t(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
     if (t >= a.T) return;
     const float* lg = a.logits + t * a.ld;
     const int E = a.E;
-    const int nper = (E + 31) >> 5;
 
-    float score[kPerLane], key[kPerLane];
+    // this lane's experts: lane, lane + 32, ...
+    float l[kPerLane];
     float m = -INFINITY;
 #pragma unroll
     for (int i = 0; i < kPerLane; ++i) {
         const int e = lane + 32 * i;
-        score[i] = (i < nper && e < E) ? lg[e] : -INFINITY;
-        m = fmaxf(m, score[i]);
+        l[i] = e < E ? lg[e] : -INFINITY;
+        m = fmaxf(m, l[i]);
     }
+    float inv_sum = 1.f;
     if (a.scoring == MOE_SCORING_SOFTMAX_ALL) {
         m = warp_max(m);
         float sum = 0.f;
 #pragma unroll
-        for (int i = 0; i < kPerLane; ++i) {
-            const int e = lane + 32 * i;
-            score[i] = (i < nper && e < E) ? expf(score[i] - m) : 0.f;
-            sum += score[i];
-        }
-        sum = warp_sum(sum);
-        const float inv = 1.0f / sum;
-#pragma unroll
-        for (int i = 0; i < kPerLane; ++i) score[i] *= inv;
-    } else if (a.scoring == MOE_SCORING_SIGMOID) {
-#pragma unroll
-        for (int i = 0; i < kPerLane; ++i) score[i] = 1.0f / (1.0f + expf(-score[i]));
+        for (int i = 0; i < kPerLane; ++i)
+            if (lane + 32 * i < E) sum += expf(l[i] - m);
+        inv_sum = 1.0f / warp_sum(sum);
     }
+    auto score_of = [&](float logit) {
+        if (a.scoring == MOE_SCORING_SOFTMAX_ALL) return expf(logit - m) * inv_sum;
+        if (a.scoring == MOE_SCORING_SIGMOID) return 1.0f / (1.0f + expf(-logit));
+        return logit;
+    };
+    uint64_t packed[kPerLane];
 #pragma unroll
     for (int i = 0; i < kPerLane; ++i) {
         const int e = lane + 32 * i;
-        const bool valid = i < nper && e < E;
-        key[i] = valid ? score[i] + (a.has_sel ? a.sel_bias[e] : 0.f) : -INFINITY;
+        packed[i] = 0;  // below every real key
+        if (e < E) packed[i] = pack_key(score_of(l[i]) + (a.has_sel ? a.sel_bias[e] : 0.f), e);
     }
-
-    // k rounds of a warp arg-max; equal keys rank the lower expert index first.
-    uint32_t taken = 0;
-    int sel[kMaxTopK];
-    float sel_score[kMaxTopK];
+    // k rounds of a warp arg-max; lane j keeps the j-th choice
+    int my_e = -1;
     for (int j = 0; j < a.k; ++j) {
-        float bk = -INFINITY;
-        int be = 0x7fffffff;
-        float bs = 0.f;
+        uint64_t best = 0;
 #pragma unroll
-        for (int i = 0; i < kPerLane; ++i) {
-            const int e = lane + 32 * i;
-            if (i < nper && e < E && !((taken >> i) & 1u) && key[i] > bk) {
-                bk = key[i];
-                be = e;
-                bs = score[i];
-            }
-        }
-        // an untaken valid key of -inf (impossible for finite logits) never beats be
+        for (int i = 0; i < kPerLane; ++i) best = packed[i] > best ? packed[i] : best;
+        best = warp_max_u64(best);
 #pragma unroll
-        for (int o = 16; o > 0; o >>= 1) {
-            const float ok = __shfl_xor_sync(0xffffffffu, bk, o);
-            const int oe = __shfl_xor_sync(0xffffffffu, be, o);
-            const float os = __shfl_xor_sync(0xffffffffu, bs, o);
-            if (ok > bk || (ok == bk && oe < be)) {
-                bk = ok;
-                be = oe;
-                bs = os;
-            }
-        }
-        if ((be & 31) == lane) taken |= 1u << (be >> 5);
-        sel[j] = be;
-        sel_score[j] = bs;
+        for (int i = 0; i < kPerLane; ++i)
+            if (packed[i] == best) packed[i] = 0;
+        if (lane == j) my_e = int(0xFFFFFFFFu - uint32_t(best & 0xFFFFFFFFu));
     }
-
-    float w[kMaxTopK];
+    // combine weights: unbiased scores of the chosen experts, or softmax over their logits
+    const bool mine = lane < a.k;
+    const float my_l = mine ? lg[my_e] : -INFINITY;
+    float w;
     if (a.scoring == MOE_SCORING_SOFTMAX_TOPK) {
-        float mm = -INFINITY;
-        for (int j = 0; j < a.k; ++j) mm = fmaxf(mm, sel_score[j]);
-        float sum = 0.f;
-        for (int j = 0; j < a.k; ++j) {
-            w[j] = expf(sel_score[j] - mm);
-            sum += w[j];
-        }
-        for (int j = 0; j < a.k; ++j) w[j] /= sum;
+        const float mm = warp_max(my_l);
+        const float ex = mine ? expf(my_l - mm) : 0.f;
+        w = ex / warp_sum(ex);
     } else {
-        for (int j = 0; j < a.k; ++j) w[j] = sel_score[j];
+        w = mine ? score_of(my_l) : 0.f;
     }
-    if (a.norm) {
-        float sum = 0.f;
-        for (int j = 0; j < a.k; ++j) sum += w[j];
-        for (int j = 0; j < a.k; ++j) w[j] /= sum;
-    }
-    for (int j = 0; j < a.k; ++j) {
-        if (lane == j) {
-            a.idx[t * a.k + j] = sel[j];
-            a.w[t * a.k + j] = w[j];
-        }
+    if (a.norm) w = w / warp_sum(w);
+    if (mine) {
+        a.idx[t * a.k + lane] = my_e;
+        a.w[t * a.k + lane] = w;
     }
     if (a.blend && lane == 0) {
         const float c0 = lg[E], c1 = lg[E + 1];
