@@ -6,7 +6,7 @@
 #include <stdint.h>
 #include <string.h>
 
-#include "../../include/moe.h"
+#include "moe.h"
 
 namespace moe {
 
