@@ -139,6 +139,30 @@ __device__ __forceinline__ void umma_commit(uint64_t* bar) {
     asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(su32(bar))
                  : "memory");
 }
+// Issue a 32-column TMEM load without waiting; the registers are valid only after
+// tmem_ld_wait on the same array (which also keeps the compiler from using them early).
+__device__ __forceinline__ void tmem_ld_issue(uint32_t taddr, uint32_t (&r)[32]) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+        "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]),
+          "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]),
+          "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]),
+          "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+        : "r"(taddr));
+}
+__device__ __forceinline__ void tmem_ld_wait(uint32_t (&r)[32]) {
+    asm volatile("tcgen05.wait::ld.sync.aligned;"
+                 : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]), "+r"(r[6]),
+                   "+r"(r[7]), "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]), "+r"(r[12]), "+r"(r[13]),
+                   "+r"(r[14]), "+r"(r[15]), "+r"(r[16]), "+r"(r[17]), "+r"(r[18]), "+r"(r[19]),
+                   "+r"(r[20]), "+r"(r[21]), "+r"(r[22]), "+r"(r[23]), "+r"(r[24]), "+r"(r[25]),
+                   "+r"(r[26]), "+r"(r[27]), "+r"(r[28]), "+r"(r[29]), "+r"(r[30]), "+r"(r[31])
+                 :
+                 : "memory");
+}
+
 __device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {
     uint32_t r[32];
     asm volatile(
@@ -414,69 +438,92 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
                 }
                 epi_bar();
             }
-            const uint32_t tbase0 = tmem_base + (uint32_t(q * 32) << 16) + ab * S::ACC_COLS;
-#pragma unroll 1
-            for (int a = 0; a < (GATEUP ? 1 : 2); ++a) {
-            const uint32_t tbase = tbase0 + a * BN;
-            const int r = ti.mb * S::ROWS + a * kBM + lrow;  // weight row (unit or output row)
-            const bool rv = r < p.M;
-            float bias0 = 0.f, bias1 = 0.f;
-            if (rv && p.bias0) {
-                if (GATEUP && p.bias_interleaved) {
-                    bias0 = bf16_at(p.bias0, int64_t(ti.group) * 2 * p.M + 2 * r);
-                    bias1 = bf16_at(p.bias0, int64_t(ti.group) * 2 * p.M + 2 * r + 1);
-                } else {
-                    bias0 = bf16_at(p.bias0, int64_t(ti.group) * p.M + r);
-                    if (GATEUP) bias1 = bf16_at(p.bias1, int64_t(ti.group) * p.M + r);
+            const uint32_t tb = tmem_base + (uint32_t(q * 32) << 16) + ab * S::ACC_COLS;
+            if constexpr (GATEUP) {
+                // gate and up of one intermediate unit for this warp's 64 token columns
+                const int r = ti.mb * S::ROWS + lrow;
+                const bool rv = r < p.M;
+                float bias0 = 0.f, bias1 = 0.f;
+                if (rv && p.bias0) {
+                    if (p.bias_interleaved) {
+                        bias0 = bf16_at(p.bias0, int64_t(ti.group) * 2 * p.M + 2 * r);
+                        bias1 = bf16_at(p.bias0, int64_t(ti.group) * 2 * p.M + 2 * r + 1);
+                    } else {
+                        bias0 = bf16_at(p.bias0, int64_t(ti.group) * p.M + r);
+                        bias1 = bf16_at(p.bias1, int64_t(ti.group) * p.M + r);
+                    }
                 }
-            }
-#pragma unroll 1
-            for (int c = c_lo; c < c_lo + BN / 2; c += 32) {
-                float g[32];
-                tmem_ld32(tbase + c, g);
-                if constexpr (GATEUP) {
-                    float u[32];
-                    tmem_ld32(tbase + BN + c, u);
-                    __nv_bfloat16* out = reinterpret_cast<__nv_bfloat16*>(p.out);
+                uint32_t hp[32];  // 64 activated values, two bf16 per register
 #pragma unroll
-                    for (int j = 0; j < 32; ++j) {
-                        const int n = c + j;
-                        if (rv && n < ti.nvalid)
-                            out[int64_t(ti.row0 + n) * p.ld_out + r] =
-                                __float2bfloat16_rn(act_fast(P.act, g[j] + bias0, u[j] + bias1, P.limit, P.alpha));
-                    }
-                } else if (p.mode == kEpiSlotRows) {
-                    // weighted output row of each slot; the combine sums a token's k rows
-                    float* out = reinterpret_cast<float*>(p.out);
-#pragma unroll 4
-                    for (int j = 0; j < 32; ++j) {
-                        const int n = c + j;
-                        if (rv && n < ti.nvalid) out[int64_t(e_slot[n]) * p.ld_out + r] = e_w[n] * (g[j] + bias0);
-                    }
-                } else if (p.mode == kEpiStoreF32) {
-                    float* out = reinterpret_cast<float*>(p.out);
+                for (int h2 = 0; h2 < 2; ++h2) {
+                    uint32_t g[32], u[32];
+                    tmem_ld_issue(tb + c_lo + 32 * h2, g);
+                    tmem_ld_issue(tb + BN + c_lo + 32 * h2, u);
+                    tmem_ld_wait(g);
+                    tmem_ld_wait(u);
 #pragma unroll
-                    for (int j = 0; j < 32; ++j) {
-                        const int n = c + j;
-                        if (rv && n < ti.nvalid) out[int64_t(ti.row0 + n) * p.ld_out + r] = g[j] + bias0;
+                    for (int j = 0; j < 32; j += 2) {
+                        const float a0 = act_fast(P.act, __uint_as_float(g[j]) + bias0,
+                                                  __uint_as_float(u[j]) + bias1, P.limit, P.alpha);
+                        const float a1 = act_fast(P.act, __uint_as_float(g[j + 1]) + bias0,
+                                                  __uint_as_float(u[j + 1]) + bias1, P.limit, P.alpha);
+                        __nv_bfloat162 v2 = __floats2bfloat162_rn(a0, a1);
+                        hp[h2 * 16 + j / 2] = *reinterpret_cast<uint32_t*>(&v2);
                     }
-                } else {  // kEpiStoreAct (+ optional fp32 addend)
-                    __nv_bfloat16* out = reinterpret_cast<__nv_bfloat16*>(p.out);
+                }
+                // the accumulator set is free for the next tile before any global store
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&acc_empty[ab]);
+                if (rv) {
+                    __nv_bfloat16* out = reinterpret_cast<__nv_bfloat16*>(p.out) + r;
 #pragma unroll
-                    for (int j = 0; j < 32; ++j) {
-                        const int n = c + j;
-                        if (rv && n < ti.nvalid) {
-                            float v = g[j] + bias0;
-                            if (p.addend) v += p.addend[int64_t(ti.row0 + n) * p.ld_add + r];
-                            out[int64_t(ti.row0 + n) * p.ld_out + r] = __float2bfloat16_rn(v);
+                    for (int j = 0; j < 64; ++j) {
+                        const int n = c_lo + j;
+                        if (n < ti.nvalid) {
+                            const uint32_t w2 = hp[j / 2];
+                            const unsigned short b = (j & 1) ? (unsigned short)(w2 >> 16) : (unsigned short)(w2 & 0xFFFFu);
+                            reinterpret_cast<unsigned short*>(out)[int64_t(ti.row0 + n) * p.ld_out] = b;
+                        }
+                    }
+                }
+            } else {
+                // two 128-row accumulators x this warp's 64 token columns, all in registers
+                uint32_t v[4][32];
+                tmem_ld_issue(tb + c_lo, v[0]);
+                tmem_ld_issue(tb + c_lo + 32, v[1]);
+                tmem_ld_issue(tb + BN + c_lo, v[2]);
+                tmem_ld_issue(tb + BN + c_lo + 32, v[3]);
+                tmem_ld_wait(v[0]);
+                tmem_ld_wait(v[1]);
+                tmem_ld_wait(v[2]);
+                tmem_ld_wait(v[3]);
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&acc_empty[ab]);
+#pragma unroll
+                for (int a = 0; a < 2; ++a) {
+                    const int r = ti.mb * S::ROWS + a * kBM + lrow;
+                    if (r >= p.M) continue;
+                    const float bias0 = p.bias0 ? bf16_at(p.bias0, int64_t(ti.group) * p.M + r) : 0.f;
+#pragma unroll
+                    for (int j = 0; j < 64; ++j) {
+                        const int n = c_lo + j;
+                        if (n >= ti.nvalid) continue;
+                        const float d = __uint_as_float(v[a * 2 + j / 32][j % 32]) + bias0;
+                        if (p.mode == kEpiSlotRows) {
+                            // weighted output row of each slot; the combine sums a token's k rows
+                            reinterpret_cast<float*>(p.out)[int64_t(e_slot[n]) * p.ld_out + r] = e_w[n] * d;
+                        } else if (p.mode == kEpiStoreF32) {
+                            reinterpret_cast<float*>(p.out)[int64_t(ti.row0 + n) * p.ld_out + r] = d;
+                        } else {  // kEpiStoreAct (+ optional fp32 addend)
+                            const float o = p.addend ? d + p.addend[int64_t(ti.row0 + n) * p.ld_add + r] : d;
+                            reinterpret_cast<__nv_bfloat16*>(p.out)[int64_t(ti.row0 + n) * p.ld_out + r] =
+                                __float2bfloat16_rn(o);
                         }
                     }
                 }
             }
-            }  // accumulator a
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&acc_empty[ab]);
         }
     }
     tc_fence_before();
