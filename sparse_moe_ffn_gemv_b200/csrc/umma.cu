@@ -248,7 +248,7 @@ struct TcShape {
     static constexpr int TMEM_COLS = 2 * ACC_COLS;               // double-buffered
     static constexpr int ROWS = GATEUP ? kBM : 2 * kBM;          // weight rows per tile
     static constexpr int SMEM = STAGES * STAGE_BYTES + 1024 /*align*/ + 256 /*barriers*/ +
-                                int(sizeof(GroupTables)) + 2 * BN * 4 /*epilogue slot, weight*/;
+                                int(sizeof(GroupTables)) + BN * 12 /*epilogue row pointers, weights*/;
     static_assert(TMEM_COLS <= 512 && (TMEM_COLS & (TMEM_COLS - 1)) == 0, "TMEM columns");
     static_assert(BN % 32 == 0 && BN >= 32 && BN <= 256, "BN");
 };
@@ -277,8 +277,8 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
     uint64_t* drain = acc_empty + 2;
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
     GroupTables& gt = *reinterpret_cast<GroupTables*>(smem + STAGES * S::STAGE_BYTES + 256);
-    int* e_slot = reinterpret_cast<int*>(&gt + 1);
-    float* e_w = reinterpret_cast<float*>(e_slot + BN);
+    float** e_row = reinterpret_cast<float**>(&gt + 1);  // output row of each token column
+    float* e_w = reinterpret_cast<float*>(e_row + BN);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     if (warp == 0) {
@@ -372,7 +372,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
         if (lane == 0) {
             // ---------------------------------------------------------- MMA issuer
             uint32_t stage = 0, phase = 0, it = 0;
-            constexpr uint32_t idesc = idesc_bf16(BN);
+            constexpr uint32_t idesc_base = idesc_bf16(BN) & ~(0x3Fu << 17);
             for (int tile = blockIdx.x; tile < total && !timed_out; tile += gridDim.x, ++it) {
                 const TileInfo ti = decode_tile(P, gt, tile, t0);
                 const TcProblem& p = P.p[ti.prob];
@@ -383,6 +383,9 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
                 }
                 tc_fence_after();
                 const uint32_t d0 = tmem_base + ab * S::ACC_COLS;
+                // MMA only over the tile's valid token columns, rounded up to the N step (16)
+                const uint32_t n_mma = uint32_t(min(BN, (ti.nvalid + 15) & ~15));
+                const uint32_t idesc = idesc_base | ((n_mma >> 3) << 17);
                 const int nk = p.K / kBK;
                 for (int kb = 0; kb < nk; ++kb) {
                     if (!mbar_wait(&full[stage], phase, deadline)) {
@@ -433,7 +436,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
                 epi_bar();
                 if (eid < BN && eid < ti.nvalid) {
                     const int slot = p.sorted_slot[ti.row0 + eid];
-                    e_slot[eid] = slot;
+                    e_row[eid] = reinterpret_cast<float*>(p.out) + int64_t(slot) * p.ld_out;
                     e_w[eid] = p.topk_w[slot];
                 }
                 epi_bar();
@@ -501,25 +504,41 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&acc_empty[ab]);
+                const bool full_tile = ti.nvalid >= c_lo + 64;
 #pragma unroll
                 for (int a = 0; a < 2; ++a) {
                     const int r = ti.mb * S::ROWS + a * kBM + lrow;
                     if (r >= p.M) continue;
                     const float bias0 = p.bias0 ? bf16_at(p.bias0, int64_t(ti.group) * p.M + r) : 0.f;
+                    const int nend = full_tile ? 64 : max(0, ti.nvalid - c_lo);
+                    if (p.mode == kEpiSlotRows) {
+                        // weighted output row of each slot; the combine sums a token's k rows
+                        if (full_tile) {
 #pragma unroll
-                    for (int j = 0; j < 64; ++j) {
-                        const int n = c_lo + j;
-                        if (n >= ti.nvalid) continue;
-                        const float d = __uint_as_float(v[a * 2 + j / 32][j % 32]) + bias0;
-                        if (p.mode == kEpiSlotRows) {
-                            // weighted output row of each slot; the combine sums a token's k rows
-                            reinterpret_cast<float*>(p.out)[int64_t(e_slot[n]) * p.ld_out + r] = e_w[n] * d;
-                        } else if (p.mode == kEpiStoreF32) {
-                            reinterpret_cast<float*>(p.out)[int64_t(ti.row0 + n) * p.ld_out + r] = d;
-                        } else {  // kEpiStoreAct (+ optional fp32 addend)
-                            const float o = p.addend ? d + p.addend[int64_t(ti.row0 + n) * p.ld_add + r] : d;
-                            reinterpret_cast<__nv_bfloat16*>(p.out)[int64_t(ti.row0 + n) * p.ld_out + r] =
-                                __float2bfloat16_rn(o);
+                            for (int j = 0; j < 64; ++j)
+                                e_row[c_lo + j][r] = e_w[c_lo + j] * (__uint_as_float(v[a * 2 + j / 32][j % 32]) + bias0);
+                        } else {
+#pragma unroll
+                            for (int j = 0; j < 64; ++j)
+                                if (j < nend)
+                                    e_row[c_lo + j][r] =
+                                        e_w[c_lo + j] * (__uint_as_float(v[a * 2 + j / 32][j % 32]) + bias0);
+                        }
+                    } else if (p.mode == kEpiStoreF32) {
+                        float* o = reinterpret_cast<float*>(p.out) + int64_t(ti.row0 + c_lo) * p.ld_out + r;
+#pragma unroll
+                        for (int j = 0; j < 64; ++j)
+                            if (j < nend) o[int64_t(j) * p.ld_out] = __uint_as_float(v[a * 2 + j / 32][j % 32]) + bias0;
+                    } else {  // kEpiStoreAct (+ optional fp32 addend)
+                        __nv_bfloat16* o = reinterpret_cast<__nv_bfloat16*>(p.out) + int64_t(ti.row0 + c_lo) * p.ld_out + r;
+                        const float* ad = p.addend ? p.addend + int64_t(ti.row0 + c_lo) * p.ld_add + r : nullptr;
+#pragma unroll
+                        for (int j = 0; j < 64; ++j) {
+                            if (j < nend) {
+                                float d = __uint_as_float(v[a * 2 + j / 32][j % 32]) + bias0;
+                                if (ad) d += ad[int64_t(j) * p.ld_add];
+                                o[int64_t(j) * p.ld_out] = __float2bfloat16_rn(d);
+                            }
                         }
                     }
                 }
