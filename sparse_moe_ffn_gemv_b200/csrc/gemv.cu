@@ -129,15 +129,6 @@ __device__ __forceinline__ void dot_rows(const char* const (&rows)[NR], const QR
     }
 }
 
-// Start pulling a weight row (and its 4-bit companions) into L2 before the block stages
-// its tokens, so the row's DRAM latency overlaps the staging and its barrier.
-__device__ __forceinline__ void prefetch_l2(const void* p, int64_t bytes) {
-    const int lane = threadIdx.x & 31;
-    const char* c = static_cast<const char*>(p);
-    for (int64_t off = int64_t(lane) * 128; off < bytes; off += 32 * 128)
-        asm volatile("prefetch.global.L2::evict_last [%0];" ::"l"(c + off));
-}
-
 // Stage tokens [p0, p0 + tt) of a group into shared memory (rows of K act values);
 // for 4-bit weights also the per-32 sums of each staged row.
 template <int WF>
@@ -232,15 +223,6 @@ __device__ void gateup_group(const GateUpArgs& a, bool shared, int e, int unit0,
     }
     const void* src = shared ? a.xs : a.u;
     AT* dst = reinterpret_cast<AT*>(shared ? a.hs : a.h);
-    if (live) {
-        prefetch_l2(rows[0], rb);
-        prefetch_l2(rows[1], rb);
-        if constexpr (WF == kQ4) {
-            const int64_t qb = int64_t(K / a.group_size) * 2;
-            prefetch_l2(q[0].s, qb); prefetch_l2(q[0].z, qb);
-            prefetch_l2(q[1].s, qb); prefetch_l2(q[1].z, qb);
-        }
-    }
     for (int64_t c = 0; c < cnt; c += kTT) {
         const int tt = int(cnt - c < kTT ? cnt - c : kTT);
         __syncthreads();
@@ -311,14 +293,6 @@ __device__ void down_group(const DownArgs& a, bool shared, int e, int row0, int6
         if (a.has_bias && live) bd = ld_act<AT>(a.down_b, gr);
     }
     const void* src = shared ? a.hs : a.h;
-    if (live) {
-        prefetch_l2(rows[0], rb);
-        if constexpr (WF == kQ4) {
-            const int64_t qb = int64_t(I / a.group_size) * 2;
-            prefetch_l2(q[0].s, qb);
-            prefetch_l2(q[0].z, qb);
-        }
-    }
     for (int64_t c = 0; c < cnt; c += kTT) {
         const int tt = int(cnt - c < kTT ? cnt - c : kTT);
         __syncthreads();
@@ -384,11 +358,6 @@ __global__ void __launch_bounds__(kThreads) dense_gemv_kernel(DenseGemvArgs a) {
     const bool live = r < rows;
     const int64_t p0 = int64_t(blockIdx.y) * kTT;
     const int tt = int(a.T - p0 < kTT ? a.T - p0 : kTT);
-    if (live) {
-        const int rr0 = r < a.rows0 ? r : r - a.rows0;
-        prefetch_l2(reinterpret_cast<const char*>(r < a.rows0 ? a.W0 : a.W1) + int64_t(rr0) * row_bytes<WF>(a.K),
-                    row_bytes<WF>(a.K));
-    }
     stage_tokens<WF>(a.u, a.K, p0, tt, nullptr, 1, us, nullptr);
     __syncthreads();
     if (!live) return;
