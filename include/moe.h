@@ -202,6 +202,27 @@ MOE_API moe_status moe_combine(const moe_config *cfg, const moe_weights *w, cons
 MOE_API moe_status moe_block_forward(const moe_config *cfg, const moe_weights *w, const void *x,
                              int64_t T, void *y, void *ws, size_t ws_bytes, moe_stream_t stream);
 
+/* Permutation without a workspace (no counterpart on the pages: an addition for
+ * callers that cannot allocate device memory). Some callers may not call cudaMalloc at
+ * the point where they route tokens: a serving loop that reserved all of its device
+ * memory up front and may not grow it, a host that owns the allocator and exposes none to
+ * plug-ins, or code recorded into a CUDA graph while the allocation would break the
+ * capture. This variant computes exactly what moe_permute computes, keeping its scratch
+ * (status word, active-expert list, per-chunk histograms, 68,096 bytes) in one fixed
+ * device array inside the library, which every GPU that loads the library holds until the
+ * process exits. Limits: T * top_k <= 65,536 slots and num_experts <= 512, else
+ * MOE_ERR_SHAPE_OVERFLOW before any launch. The caller still passes every input and
+ * output. device_status (optional, caller-owned int32 on the device, zeroed by the caller)
+ * receives MOE_ERR_DEVICE_CHECK on an out-of-range expert id; when NULL that word lives in
+ * the fixed array and is cleared on each call. No call allocates or frees anything. The
+ * first call on each device looks up the array's device address (with that device
+ * current): make that first call before any stream capture. All calls share the one array
+ * and leave their contents in it, so calls that overlap on the GPU (different streams
+ * without ordering, or different host threads) race: serialise them. */
+MOE_API moe_status moe_permute_noalloc(const moe_config *cfg, const int32_t *topk_idx, int64_t T,
+                                       int32_t *expert_offsets, int32_t *sorted_slot, int32_t *slot_pos,
+                                       int32_t *device_status, moe_stream_t stream);
+
 /* Synchronises `stream`, returns the status word that device-side checks
  * write into the workspace (MOE_OK, MOE_ERR_DEVICE_CHECK or
  * MOE_ERR_DEVICE_TIMEOUT) and clears it. A new workspace must be cleared once

@@ -7,6 +7,8 @@
 // warp match masks plus per-warp counts in shared memory, so equal experts keep
 // ascending slot order. Also emits the compact list of experts that received
 // tokens, which the expert kernels use to skip empty experts.
+#include <mutex>
+
 #include "common.cuh"
 #include "internal.h"
 
@@ -231,4 +233,78 @@ cudaError_t launch_permute(const PermuteArgs& a, cudaStream_t s) {
     return cudaGetLastError();
 }
 
+// ---------------------------------------------------------------- permutation without a workspace
+// Scratch of moe_permute_noalloc: [status word, padded to 256 B][active list, 513 ints,
+// padded to 2304 B][per-chunk histograms, 32 chunks x 512 experts]. Every GPU that loads
+// the library holds it until the process exits.
+namespace {
+constexpr int kNoAllocMaxSlots = 65536;
+constexpr int kNoAllocMaxExperts = kPermE;
+constexpr size_t kNoAllocStatus = 0;
+constexpr size_t kNoAllocActive = 256;
+constexpr size_t kNoAllocHist = 256 + 2304;
+constexpr size_t kNoAllocBytes = kNoAllocHist + size_t(kNoAllocMaxSlots / kPermChunk) * kNoAllocMaxExperts * 4;
+static_assert(kNoAllocBytes == 68096, "documented size of the fixed scratch");
+static_assert((kNoAllocMaxExperts + 1) * 4 <= 2304, "active list fits its region");
+}  // namespace
+
+static __device__ __align__(256) unsigned char g_permute_scratch[kNoAllocBytes];
+
+namespace {
+// Device address of g_permute_scratch on the current device, looked up once per device.
+cudaError_t permute_scratch(void** out) {
+    constexpr int kMaxDevices = 64;
+    static void* addr[kMaxDevices] = {};
+    static std::mutex mu;
+    int dev = 0;
+    cudaError_t err = cudaGetDevice(&dev);
+    if (err != cudaSuccess) return err;
+    if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+    std::lock_guard<std::mutex> lock(mu);
+    if (!addr[dev]) {
+        void* p = nullptr;
+        err = cudaGetSymbolAddress(&p, g_permute_scratch);
+        if (err != cudaSuccess) return err;
+        addr[dev] = p;
+    }
+    *out = addr[dev];
+    return cudaSuccess;
+}
+}  // namespace
+
 }  // namespace moe
+
+extern "C" moe_status moe_permute_noalloc(const moe_config* cfg, const int32_t* topk_idx, int64_t T,
+                                          int32_t* expert_offsets, int32_t* sorted_slot, int32_t* slot_pos,
+                                          int32_t* device_status, moe_stream_t stream) {
+    using namespace moe;
+    const moe_status vs = moe_config_validate(cfg);
+    if (vs != MOE_OK) return vs;
+    if (T < 0) return MOE_ERR_INVALID_ARGUMENT;
+    if (T == 0) return MOE_OK;
+    if (T * int64_t(cfg->top_k) > kNoAllocMaxSlots || cfg->num_experts > kNoAllocMaxExperts)
+        return MOE_ERR_SHAPE_OVERFLOW;
+    const void* ptrs[] = {topk_idx, expert_offsets, sorted_slot, slot_pos};
+    for (const void* q : ptrs)
+        if (!q || (reinterpret_cast<uintptr_t>(q) & 15u)) return MOE_ERR_INVALID_ARGUMENT;
+    if (device_status && (reinterpret_cast<uintptr_t>(device_status) & 3u)) return MOE_ERR_INVALID_ARGUMENT;
+    void* scratch = nullptr;
+    if (permute_scratch(&scratch) != cudaSuccess) return MOE_ERR_CUDA;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    char* base = static_cast<char*>(scratch);
+    int* status = device_status ? reinterpret_cast<int*>(device_status) : reinterpret_cast<int*>(base + kNoAllocStatus);
+    // the status word must start at zero; histograms and the active list are rewritten in full
+    if (!device_status && cudaMemsetAsync(status, 0, sizeof(int), s) != cudaSuccess) return MOE_ERR_CUDA;
+    PermuteArgs p;
+    p.idx = topk_idx;
+    p.S = T * cfg->top_k;
+    p.E = cfg->num_experts;
+    p.offsets = expert_offsets;
+    p.sorted_slot = sorted_slot;
+    p.slot_pos = slot_pos;
+    p.active = reinterpret_cast<int32_t*>(base + kNoAllocActive);
+    p.chunk_hist = reinterpret_cast<int32_t*>(base + kNoAllocHist);
+    p.n_chunks = int((p.S + kPermChunk - 1) / kPermChunk);
+    p.status = status;
+    return launch_permute(p, s) == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}

@@ -30,6 +30,7 @@ EXPORTS = [
     "moe_config_validate", "moe_weights_validate", "moe_workspace_size", "moe_route",
     "moe_permute", "moe_grouped_ffn", "moe_latent_down", "moe_combine", "moe_block_forward",
     "moe_read_device_status", "moe_clear_device_status", "moe_status_string",
+    "moe_permute_noalloc",
 ]
 
 STATUS = {0: "MOE_OK", 1: "MOE_ERR_INVALID_ARGUMENT", 2: "MOE_ERR_SHAPE_OVERFLOW",
@@ -90,6 +91,7 @@ def lib():
             "moe_block_forward": [cfgp, wp, vp, i64, vp, vp, sz, vp],
             "moe_read_device_status": [vp, vp],
             "moe_clear_device_status": [vp, vp],
+            "moe_permute_noalloc": [cfgp, vp, i64, vp, vp, vp, vp, vp],
         }
         for name, args in sig.items():
             fn = getattr(L, name)
@@ -194,6 +196,15 @@ def moe_combine(cfg, w, y_acc, x, coef, T, y, ws, stream=None):
 def moe_block_forward(cfg, w, x, T, y, ws, stream=None):
     _check(lib().moe_block_forward(ctypes.byref(cfg), ctypes.byref(w), _p(x), int(T), _p(y),
                                    _p(ws), ws.numel(), _stream(stream)), "moe_block_forward")
+
+
+def moe_permute_noalloc(cfg, topk_idx, T, expert_offsets, sorted_slot, slot_pos, device_status=None,
+                        stream=None):
+    """moe_permute without a workspace: the library keeps the scratch in a fixed device
+    array (for callers that cannot allocate device memory where they route tokens)."""
+    _check(lib().moe_permute_noalloc(ctypes.byref(cfg), _p(topk_idx), int(T), _p(expert_offsets),
+                                     _p(sorted_slot), _p(slot_pos), _p(device_status), _stream(stream)),
+           "moe_permute_noalloc")
 
 
 def moe_read_device_status(ws, stream=None) -> int:

@@ -32,7 +32,7 @@ def declared_symbols():
 
 def test_library_exports_every_declared_symbol():
     names = declared_symbols()
-    assert len(names) == 12
+    assert len(names) == 13
     assert sorted(M.EXPORTS) == names
     lib = M.lib()
     for n in names:
@@ -186,6 +186,18 @@ def test_zero_tokens_is_a_no_op_and_errors_precede_launches():
     # a NULL output pointer is rejected too
     assert M.STATUS[lib.moe_block_forward(ctypes.byref(cfg), ctypes.byref(w), ctypes.c_void_p(1 << 22), 4,
                                           None, ws, 1 << 30, None)] == "MOE_ERR_INVALID_ARGUMENT"
+
+
+def test_noalloc_permutation_rejects_sizes_beyond_its_fixed_scratch():
+    """The allocation-free permutation checks its limits on the host, before any launch."""
+    lib = M.lib()
+    cfg = _cfg()                      # top_k 8: 8193 tokens are 65,544 slots > 65,536
+    p = ctypes.c_void_p(1 << 22)
+    assert M.STATUS[lib.moe_permute_noalloc(ctypes.byref(cfg), p, 8193, p, p, p, None, None)] == \
+        "MOE_ERR_SHAPE_OVERFLOW"
+    assert lib.moe_permute_noalloc(ctypes.byref(cfg), p, 0, p, p, p, None, None) == 0
+    assert M.STATUS[lib.moe_permute_noalloc(ctypes.byref(_cfg(top_k=0)), p, 4, p, p, p, None, None)] == \
+        "MOE_ERR_INVALID_ARGUMENT"
 
 
 def test_status_strings():
