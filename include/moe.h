@@ -225,11 +225,13 @@ MOE_API moe_status moe_permute_noalloc(const moe_config *cfg, const int32_t *top
 
 /* Synchronises `stream`, returns the status word that device-side checks
  * write into the workspace (MOE_OK, MOE_ERR_DEVICE_CHECK or
- * MOE_ERR_DEVICE_TIMEOUT) and clears it. A new workspace must be cleared once
- * with this call or zero-filled before first use. */
+ * MOE_ERR_DEVICE_TIMEOUT) and clears it. The first 256 bytes of a workspace
+ * hold this word and a launch counter that every call leaves at zero: a new
+ * workspace must be zero-filled (or cleared with moe_clear_device_status)
+ * before its first use. */
 MOE_API moe_status moe_read_device_status(void *ws, moe_stream_t stream);
 
-/* Clears the workspace status word, asynchronously on `stream`. */
+/* Clears the workspace's 256-byte status region, asynchronously on `stream`. */
 MOE_API moe_status moe_clear_device_status(void *ws, moe_stream_t stream);
 
 /* Static, NUL-terminated description of a status code. */

@@ -185,6 +185,20 @@ bool routed_tc(const moe_config* c, int64_t T) {
     return o == kPathTc || (o == kPathAuto && T * c->top_k >= 8 * int64_t(c->num_experts));
 }
 
+// Small batches whose router, shared expert and latent projection all take the
+// weight-streaming path route in one fused launch (the permutation fits one chunk).
+bool fused_route(const moe_config* c, int64_t T) {
+    if (path_override() == kPathTc) return false;
+    if (T * c->top_k > kPermChunk) return false;
+    if (dense_tc(c, T, c->hidden) || routed_tc(c, T)) return false;
+    if (c->latent_dim && dense_tc(c, T, c->hidden)) return false;
+    return true;
+}
+
+// Word offset (in ints) of the fused routing launch's completion counter in the
+// workspace's 256-byte status region (the status word is word 0).
+constexpr int kCounterWord = 16;
+
 #define MOE_CHECK(expr)                          \
     do {                                         \
         const moe_status _s = (expr);            \
@@ -211,9 +225,9 @@ moe_status prelude(const moe_config* c, const moe_weights* w, int64_t T, void* w
 template <typename P> P* at(void* ws, size_t off) { return reinterpret_cast<P*>(static_cast<char*>(ws) + off); }
 
 // a1 + a2
-moe_status run_route(const moe_config* c, const moe_weights* w, const void* x, int64_t T, int32_t* idx,
-                     float* wts, float* coef, float* zero, int64_t zero_cols, void* ws, const WsLayout& L,
-                     cudaStream_t s) {
+// The router's dense GEMV: E router rows (+ 2 coefficient rows for the blend) -> fp32 logits.
+DenseGemvArgs router_args(const moe_config* c, const moe_weights* w, const void* x, int64_t T, void* ws,
+                          const WsLayout& L) {
     const bool blend = c->shared_mode == MOE_SHARED_BLEND;
     DenseGemvArgs r;
     r.W0 = w->router_w;
@@ -231,6 +245,33 @@ moe_status run_route(const moe_config* c, const moe_weights* w, const void* x, i
     r.ld_out = L.ld_logits;
     r.out_f32 = 1;
     r.act_dtype = c->act_dtype;
+    return r;
+}
+
+TopkArgs topk_args(const moe_config* c, const moe_weights* w, int64_t T, int32_t* idx, float* wts, float* coef,
+                   void* ws, const WsLayout& L) {
+    TopkArgs t;
+    t.logits = at<float>(ws, L.logits);
+    t.ld = L.ld_logits;
+    t.T = T;
+    t.E = c->num_experts;
+    t.k = c->top_k;
+    t.scoring = c->scoring;
+    t.norm = c->norm_topk_prob;
+    t.has_sel = c->has_selection_bias;
+    t.sel_bias = static_cast<const float*>(w->selection_bias);
+    t.blend = c->shared_mode == MOE_SHARED_BLEND;
+    t.idx = idx;
+    t.w = wts;
+    t.coef = coef;
+    return t;
+}
+
+moe_status run_route(const moe_config* c, const moe_weights* w, const void* x, int64_t T, int32_t* idx,
+                     float* wts, float* coef, float* zero, int64_t zero_cols, void* ws, const WsLayout& L,
+                     cudaStream_t s) {
+    const bool blend = c->shared_mode == MOE_SHARED_BLEND;
+    const DenseGemvArgs r = router_args(c, w, x, T, ws, L);
     if (dense_tc(c, T, c->hidden)) {
         TcParams P;
         const int np = blend ? 2 : 1;
@@ -256,20 +297,7 @@ moe_status run_route(const moe_config* c, const moe_weights* w, const void* x, i
     } else {
         MOE_CUDA(launch_dense_gemv(r, s));
     }
-    TopkArgs t;
-    t.logits = at<float>(ws, L.logits);
-    t.ld = L.ld_logits;
-    t.T = T;
-    t.E = c->num_experts;
-    t.k = c->top_k;
-    t.scoring = c->scoring;
-    t.norm = c->norm_topk_prob;
-    t.has_sel = c->has_selection_bias;
-    t.sel_bias = static_cast<const float*>(w->selection_bias);
-    t.blend = blend;
-    t.idx = idx;
-    t.w = wts;
-    t.coef = coef;
+    TopkArgs t = topk_args(c, w, T, idx, wts, coef, ws, L);
     t.zero = zero;
     t.zero_cols = zero_cols;
     MOE_CUDA(launch_topk(t, s));
@@ -413,7 +441,7 @@ struct RoutedSum {
 moe_status run_experts(const moe_config* c, const moe_weights* w, const void* u, const void* x, int64_t T,
                        const int32_t* offsets, const int32_t* sorted_slot, const float* topk_w,
                        float* y_acc, bool with_routed, bool with_shared, void* ws, const WsLayout& L,
-                       cudaStream_t s, RoutedSum* sum) {
+                       cudaStream_t s, RoutedSum* sum, bool shared_gate_up_done = false) {
     const int K = expert_in(*c);
     const bool sh = with_shared && c->shared_mode != MOE_SHARED_NONE;
     const bool rtc = with_routed && routed_tc(c, T);
@@ -443,7 +471,7 @@ moe_status run_experts(const moe_config* c, const moe_weights* w, const void* u,
     g.routed_groups = int(groups);
     g.u = u;
     g.h = at<void>(ws, L.h);
-    if (sh && !stc) {
+    if (sh && !stc && !shared_gate_up_done) {
         g.sg_w = w->shared_gate_w;
         g.su_w = w->shared_up_w;
         g.shared_I = c->shared_intermediate;
@@ -685,16 +713,61 @@ moe_status moe_block_forward(const moe_config* cfg, const moe_weights* w, const 
     int32_t* idx = at<int32_t>(ws, L.topk_idx);
     float* wts = at<float>(ws, L.topk_w);
     float* coef = at<float>(ws, L.coef);
-    // the weight-streaming path scatter-adds into y_acc: its rows are cleared by the router
     const bool rtc = routed_tc(cfg, T);
-    MOE_CHECK(run_route(cfg, w, x, T, idx, wts, coef, rtc ? nullptr : y_acc, K, ws, L, s));
-    const void* u = x;
-    if (cfg->latent_dim) {
-        MOE_CHECK(run_latent_down(cfg, w, x, T, at<void>(ws, L.z), at<int>(ws, L.status), s));
-        u = at<void>(ws, L.z);
-    }
+    const void* u = cfg->latent_dim ? at<void>(ws, L.z) : x;
     int32_t* offsets = at<int32_t>(ws, L.offsets);
     int32_t* sorted_slot = at<int32_t>(ws, L.sorted_slot);
+    const bool sh = cfg->shared_mode != MOE_SHARED_NONE;
+    if (fused_route(cfg, T)) {
+        // small batch: router, latent down, shared gate/up, top-k and permutation in one launch
+        RouteFusedArgs f;
+        f.router = router_args(cfg, w, x, T, ws, L);
+        if (cfg->latent_dim) {
+            f.latent.W0 = w->latent_down_w;
+            f.latent.rows0 = cfg->latent_dim;
+            f.latent.u = x;
+            f.latent.T = T;
+            f.latent.K = cfg->hidden;
+            f.latent.out = at<void>(ws, L.z);
+            f.latent.ld_out = cfg->latent_dim;
+            f.latent.act_dtype = cfg->act_dtype;
+        }
+        if (sh) {
+            f.shared.wf = cfg->act_dtype;
+            f.shared.sg_w = w->shared_gate_w;
+            f.shared.su_w = w->shared_up_w;
+            f.shared.shared_I = cfg->shared_intermediate;
+            f.shared.Hs = cfg->hidden;
+            f.shared.xs = x;
+            f.shared.hs = at<void>(ws, L.hs);
+            f.shared.T = T;
+            f.shared.act = cfg->activation;
+            f.shared.limit = cfg->swiglu_limit;
+            f.shared.alpha = cfg->swiglu_alpha;
+        }
+        f.topk = topk_args(cfg, w, T, idx, wts, coef, ws, L);
+        f.perm.idx = idx;
+        f.perm.S = T * cfg->top_k;
+        f.perm.E = cfg->num_experts;
+        f.perm.offsets = offsets;
+        f.perm.sorted_slot = sorted_slot;
+        f.perm.slot_pos = at<int32_t>(ws, L.slot_pos);
+        f.perm.active = at<int32_t>(ws, L.active);
+        f.perm.chunk_hist = at<int32_t>(ws, L.chunk_hist);
+        f.perm.n_chunks = 1;
+        f.perm.status = at<int>(ws, L.status);
+        f.zero = y_acc;
+        f.zero_floats = T * K;
+        f.counter = at<int>(ws, L.status) + kCounterWord;
+        MOE_CUDA(launch_route_fused(f, s));
+        RoutedSum rs;
+        MOE_CHECK(run_experts(cfg, w, u, x, T, offsets, sorted_slot, wts, y_acc, true, true, ws, L, s, &rs,
+                              /*shared_gate_up_done=*/sh));
+        return run_output(cfg, w, rs, coef, T, y, ws, L, s);
+    }
+    // the weight-streaming path scatter-adds into y_acc: its rows are cleared by the router
+    MOE_CHECK(run_route(cfg, w, x, T, idx, wts, coef, rtc ? nullptr : y_acc, K, ws, L, s));
+    if (cfg->latent_dim) MOE_CHECK(run_latent_down(cfg, w, x, T, at<void>(ws, L.z), at<int>(ws, L.status), s));
     MOE_CHECK(run_permute(cfg, idx, T, offsets, sorted_slot, at<int32_t>(ws, L.slot_pos), ws, L, s, rtc));
     RoutedSum rs;
     MOE_CHECK(run_experts(cfg, w, u, x, T, offsets, sorted_slot, wts, y_acc, true, true, ws, L, s, &rs));
@@ -715,7 +788,7 @@ moe_status moe_read_device_status(void* ws, moe_stream_t stream) {
 
 moe_status moe_clear_device_status(void* ws, moe_stream_t stream) {
     if (!ws) return MOE_ERR_INVALID_ARGUMENT;
-    MOE_CUDA(cudaMemsetAsync(ws, 0, sizeof(int), (cudaStream_t)stream));
+    MOE_CUDA(cudaMemsetAsync(ws, 0, 256, (cudaStream_t)stream));
     return MOE_OK;
 }
 

@@ -9,8 +9,7 @@
 // tokens, which the expert kernels use to skip empty experts.
 #include <mutex>
 
-#include "common.cuh"
-#include "internal.h"
+#include "permute_dev.cuh"
 
 namespace moe {
 
@@ -18,7 +17,6 @@ namespace {
 
 constexpr int kPlaceThreads = 512;
 constexpr int kPlaceWarps = kPlaceThreads / 32;
-constexpr int kPermE = 512;  // experts supported by the permutation kernels
 
 __global__ void __launch_bounds__(256) hist_kernel(PermuteArgs a) {
     __shared__ int hist[kPermE];
@@ -35,130 +33,9 @@ __global__ void __launch_bounds__(256) hist_kernel(PermuteArgs a) {
         a.chunk_hist[int64_t(blockIdx.x) * a.E + e] = hist[e];
 }
 
-// Exclusive scan of vals[0..n) in shared memory by one 512-thread block; returns the total.
-__device__ int block_exclusive_scan(int* vals, int n, int* warp_tot) {
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    // each thread owns one element (n <= 512)
-    int v = tid < n ? vals[tid] : 0;
-    int incl = v;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-        const int y = __shfl_up_sync(0xffffffffu, incl, o);
-        if (lane >= o) incl += y;
-    }
-    if (lane == 31) warp_tot[warp] = incl;
-    __syncthreads();
-    if (warp == 0) {
-        int wt = lane < kPlaceWarps ? warp_tot[lane] : 0;
-        int wi = wt;
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-            const int y = __shfl_up_sync(0xffffffffu, wi, o);
-            if (lane >= o) wi += y;
-        }
-        if (lane < kPlaceWarps) warp_tot[lane] = wi - wt;  // exclusive warp offsets
-        if (lane == kPlaceWarps - 1) warp_tot[kPlaceWarps] = wi;
-    }
-    __syncthreads();
-    if (tid < n) vals[tid] = incl - v + warp_tot[warp];
-    const int total = warp_tot[kPlaceWarps];
-    __syncthreads();
-    return total;
-}
-
 __global__ void __launch_bounds__(kPlaceThreads) place_kernel(PermuteArgs a) {
-    __shared__ int base[kPermE];
-    __shared__ int scan_buf[kPermE];
-    __shared__ int flag_buf[kPermE];
-    __shared__ int cnt[kPlaceWarps][kPermE];
-    __shared__ int warp_tot[kPlaceWarps + 1];
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int E = a.E;
-    const int chunk = blockIdx.x;
-    const int64_t s0 = int64_t(chunk) * kPermChunk;
-    const int64_t s1 = min(a.S, s0 + kPermChunk);
-
-    for (int i = tid; i < kPlaceWarps * kPermE; i += kPlaceThreads) (&cnt[0][0])[i] = 0;
-    if (a.n_chunks == 1) {
-        for (int e = tid; e < E; e += kPlaceThreads) scan_buf[e] = 0;
-        __syncthreads();
-        for (int64_t s = s0 + tid; s < s1; s += kPlaceThreads) {
-            const int e = a.idx[s];
-            if (e >= 0 && e < E) atomicAdd(&scan_buf[e], 1);
-            else set_status(a.status, MOE_ERR_DEVICE_CHECK);
-        }
-        __syncthreads();
-        for (int e = tid; e < E; e += kPlaceThreads) base[e] = 0;  // no earlier chunks
-    } else {
-        for (int e = tid; e < E; e += kPlaceThreads) {
-            int tot = 0, pre = 0;
-            for (int c = 0; c < a.n_chunks; ++c) {
-                const int h = a.chunk_hist[int64_t(c) * E + e];
-                tot += h;
-                if (c < chunk) pre += h;
-            }
-            scan_buf[e] = tot;
-            base[e] = pre;
-        }
-    }
-    __syncthreads();
-    for (int e = tid; e < E; e += kPlaceThreads) flag_buf[e] = scan_buf[e] > 0 ? 1 : 0;
-    if (chunk == 0 && a.tile_bn > 0) {
-        // tensor-core tile prefix: tiles of expert e = ceil(count_e / tile_bn)
-        for (int e = tid; e < E; e += kPlaceThreads) cnt[0][e] = (scan_buf[e] + a.tile_bn - 1) / a.tile_bn;
-        __syncthreads();
-        const int ntiles = block_exclusive_scan(&cnt[0][0], E, warp_tot);
-        for (int e = tid; e < E; e += kPlaceThreads) a.tile_start[e] = cnt[0][e];
-        if (tid == 0) a.tile_start[E] = ntiles;
-        for (int e = tid; e < E; e += kPlaceThreads) cnt[0][e] = 0;
-    }
-    __syncthreads();
-    const int total = block_exclusive_scan(scan_buf, E, warp_tot);
-    const int n_active = block_exclusive_scan(flag_buf, E, warp_tot);
-    if (chunk == 0) {
-        for (int e = tid; e < E; e += kPlaceThreads) {
-            a.offsets[e] = scan_buf[e];
-            const int next = (e + 1 < E) ? flag_buf[e + 1] : n_active;
-            if (next != flag_buf[e]) a.active[1 + flag_buf[e]] = e;
-        }
-        if (tid == 0) {
-            a.offsets[E] = total;
-            a.active[0] = n_active;
-        }
-    }
-    for (int e = tid; e < E; e += kPlaceThreads) base[e] += scan_buf[e];
-    __syncthreads();
-
-    const unsigned lt_mask = (1u << lane) - 1u;
-    for (int64_t step = s0; step < s1; step += kPlaceThreads) {
-        const int64_t s = step + tid;
-        int e = -1;
-        if (s < s1) {
-            e = a.idx[s];
-            if (e < 0 || e >= E) {
-                if (a.n_chunks > 1) set_status(a.status, MOE_ERR_DEVICE_CHECK);
-                e = -1;
-                a.slot_pos[s] = -1;
-            }
-        }
-        const unsigned peers = __match_any_sync(0xffffffffu, e);
-        const int rank = __popc(peers & lt_mask);
-        const bool leader = (peers & lt_mask) == 0;
-        if (e >= 0 && leader) cnt[warp][e] = __popc(peers);
-        __syncthreads();
-        if (e >= 0) {
-            int p = base[e] + rank;
-            for (int w = 0; w < warp; ++w) p += cnt[w][e];
-            a.sorted_slot[p] = int32_t(s);
-            a.slot_pos[s] = p;
-        }
-        __syncthreads();
-        if (e >= 0 && leader) {
-            atomicAdd(&base[e], __popc(peers));
-            cnt[warp][e] = 0;
-        }
-        __syncthreads();
-    }
+    __shared__ PlaceSmem<kPlaceThreads> sm;
+    place_chunk<kPlaceThreads>(a, blockIdx.x, sm);
 }
 
 // Compact list of the experts that hold tokens, from offsets [E + 1]
@@ -170,7 +47,7 @@ __global__ void __launch_bounds__(kPlaceThreads) active_kernel(const int32_t* of
     const int f = (tid < E && offsets[tid + 1] > offsets[tid]) ? 1 : 0;
     if (tid < E) flags[tid] = f;
     __syncthreads();
-    const int n = block_exclusive_scan(flags, E, warp_tot);
+    const int n = block_exclusive_scan<kPlaceThreads>(flags, E, warp_tot);
     if (tid < E && f) active[1 + flags[tid]] = tid;
     if (tid == 0) active[0] = n;
 }
@@ -182,7 +59,7 @@ __global__ void __launch_bounds__(kPlaceThreads) tile_start_kernel(const int32_t
     const int tid = threadIdx.x;
     if (tid < E) v[tid] = (offsets[tid + 1] - offsets[tid] + bn - 1) / bn;
     __syncthreads();
-    const int n = block_exclusive_scan(v, E, warp_tot);
+    const int n = block_exclusive_scan<kPlaceThreads>(v, E, warp_tot);
     if (tid < E) tile_start[tid] = v[tid];
     if (tid == 0) tile_start[E] = n;
 }
