@@ -28,6 +28,7 @@ __global__ void __launch_bounds__(256) combine_kernel(const float* __restrict__ 
                                                       const float* __restrict__ s_acc,
                                                       const float* __restrict__ coef, int mode,
                                                       int64_t T, int H, AT* __restrict__ y) {
+    pdl_begin();
     const int H4 = H / 4;
     const int64_t n4 = T * H4;
     for (int64_t i = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; i < n4;
@@ -58,6 +59,7 @@ template <typename AT>
 __global__ void __launch_bounds__(256) rmsnorm_kernel(const float* __restrict__ rows, int nsum,
                                                       const AT* __restrict__ gamma, float eps,
                                                       int L, AT* __restrict__ out) {
+    pdl_begin();
     extern __shared__ float rsum[];   // the routed sum of this token, L floats
     __shared__ float red[8];
     const int64_t t = blockIdx.x;
@@ -88,10 +90,10 @@ cudaError_t launch_combine(const float* rows, int nsum, const float* s_acc, cons
     const int64_t n4 = T * H / 4;
     const unsigned grid = unsigned(std::min<int64_t>((n4 + 255) / 256, 148 * 16));
     if (act_dtype == kF32 || out_f32)
-        combine_kernel<float><<<grid, 256, 0, s>>>(rows, nsum, s_acc, coef, mode, T, H, static_cast<float*>(y));
+        { const cudaError_t e_ = launch_pdl(combine_kernel<float>, dim3(grid), dim3(256), 0, s, rows, nsum, s_acc, coef, mode, T, H, static_cast<float*>(y)); if (e_ != cudaSuccess) return e_; }
     else
-        combine_kernel<__nv_bfloat16><<<grid, 256, 0, s>>>(rows, nsum, s_acc, coef, mode, T, H,
-                                                           static_cast<__nv_bfloat16*>(y));
+        { const cudaError_t e_ = launch_pdl(combine_kernel<__nv_bfloat16>, dim3(grid), dim3(256), 0, s, rows, nsum, s_acc, coef, mode, T, H,
+                                                           static_cast<__nv_bfloat16*>(y)); if (e_ != cudaSuccess) return e_; }
     return cudaGetLastError();
 }
 
@@ -101,13 +103,13 @@ cudaError_t launch_rmsnorm(const float* rows, int nsum, const void* gamma, float
     const size_t smem = size_t(L) * sizeof(float);
     if (act_dtype == kF32) {
         cudaFuncSetAttribute(rmsnorm_kernel<float>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
-        rmsnorm_kernel<float><<<unsigned(T), 256, smem, s>>>(rows, nsum, static_cast<const float*>(gamma), eps, L,
-                                                             static_cast<float*>(out));
+        { const cudaError_t e_ = launch_pdl(rmsnorm_kernel<float>, dim3(unsigned(T)), dim3(256), smem, s, rows, nsum, static_cast<const float*>(gamma), eps, L,
+                                                             static_cast<float*>(out)); if (e_ != cudaSuccess) return e_; }
     } else {
         cudaFuncSetAttribute(rmsnorm_kernel<__nv_bfloat16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              int(smem));
-        rmsnorm_kernel<__nv_bfloat16><<<unsigned(T), 256, smem, s>>>(
-            rows, nsum, static_cast<const __nv_bfloat16*>(gamma), eps, L, static_cast<__nv_bfloat16*>(out));
+        { const cudaError_t e_ = launch_pdl(rmsnorm_kernel<__nv_bfloat16>, dim3(unsigned(T)), dim3(256), smem, s, 
+            rows, nsum, static_cast<const __nv_bfloat16*>(gamma), eps, L, static_cast<__nv_bfloat16*>(out)); if (e_ != cudaSuccess) return e_; }
     }
     return cudaGetLastError();
 }

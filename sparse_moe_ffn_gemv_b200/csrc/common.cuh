@@ -4,6 +4,9 @@
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
+#include <stdlib.h>
+
+#include <utility>
 
 #include "moe.h"
 
@@ -105,9 +108,40 @@ __device__ __forceinline__ float act_apply(int act, float g, float v, float limi
     return gc / (1.0f + expf(-alpha * gc)) * (vc + 1.0f);
 }
 
+// Programmatic dependent launch: every kernel first lets the next kernel in the stream
+// begin launching, then waits until the previous kernel's results are complete and
+// visible. Touching no memory before the wait keeps plain stream-order semantics while the
+// launch latency of each kernel overlaps the tail of the one before.
+__device__ __forceinline__ void pdl_begin() {
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+
 // Sticky device status word (first error wins).
 __device__ __forceinline__ void set_status(int* status, int code) {
     if (status) atomicCAS(status, 0, code);
+}
+
+// Host: launch a kernel that begins with pdl_begin(), allowing programmatic dependent
+// launch (MOE_PDL=0 in the environment turns it off).
+inline bool pdl_enabled() {
+    const char* e = getenv("MOE_PDL");
+    return !(e && e[0] == '0');
+}
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s,
+                              Args&&... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = pdl_enabled() ? 1 : 0;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
 }
 
 }  // namespace moe

@@ -249,6 +249,7 @@ __device__ void gateup_group(const GateUpArgs& a, bool shared, int e, int unit0,
 
 template <int WF>
 __global__ void __launch_bounds__(kThreads) gateup_gemv_kernel(GateUpArgs a) {
+    pdl_begin();
     constexpr int WFD = (WF == kQ4) ? kBF16 : WF;  // the shared expert is dense
     using AT = typename Fmt<WF>::AT;
     extern __shared__ uint4 smem_raw[];
@@ -328,6 +329,7 @@ __device__ void down_group(const DownArgs& a, bool shared, int e, int row0, int6
 
 template <int WF>
 __global__ void __launch_bounds__(kThreads) down_gemv_kernel(DownArgs a) {
+    pdl_begin();
     constexpr int WFD = (WF == kQ4) ? kBF16 : WF;
     using AT = typename Fmt<WF>::AT;
     extern __shared__ uint4 smem_raw[];
@@ -351,6 +353,7 @@ __global__ void __launch_bounds__(kThreads) down_gemv_kernel(DownArgs a) {
 
 template <typename AT>
 __global__ void __launch_bounds__(kThreads) dense_gemv_kernel(DenseGemvArgs a) {
+    pdl_begin();
     constexpr int WF = sizeof(AT) == 4 ? kF32 : kBF16;
     extern __shared__ uint4 smem_raw[];
     AT* us = reinterpret_cast<AT*>(smem_raw);
@@ -434,6 +437,7 @@ __device__ void dense_rows_block(const DenseGemvArgs& a, int rblock, typename Fm
 
 template <int WFD>
 __global__ void __launch_bounds__(kThreads) route_fused_kernel(RouteFusedArgs a) {
+    pdl_begin();
     using AT = typename Fmt<WFD>::AT;
     extern __shared__ uint4 smem_raw[];
     AT* us = reinterpret_cast<AT*>(smem_raw);
@@ -497,7 +501,7 @@ cudaError_t launch_gateup_t(const GateUpArgs& a, cudaStream_t s) {
     const int64_t rblocks = int64_t(a.routed_groups) * ((a.I + kRowsPerBlock - 1) / kRowsPerBlock);
     const int64_t grid = sblocks + rblocks;
     if (grid == 0) return cudaSuccess;
-    gateup_gemv_kernel<WF><<<unsigned(grid), kThreads, smem, s>>>(a);
+    { const cudaError_t e_ = launch_pdl(gateup_gemv_kernel<WF>, dim3(unsigned(grid)), dim3(kThreads), smem, s, a); if (e_ != cudaSuccess) return e_; }
     return cudaGetLastError();
 }
 
@@ -511,7 +515,7 @@ cudaError_t launch_down_t(const DownArgs& a, cudaStream_t s) {
     const int64_t rblocks = int64_t(a.routed_groups) * ((a.K + kRowsPerBlock - 1) / kRowsPerBlock);
     const int64_t grid = sblocks + rblocks;
     if (grid == 0) return cudaSuccess;
-    down_gemv_kernel<WF><<<unsigned(grid), kThreads, smem, s>>>(a);
+    { const cudaError_t e_ = launch_pdl(down_gemv_kernel<WF>, dim3(unsigned(grid)), dim3(kThreads), smem, s, a); if (e_ != cudaSuccess) return e_; }
     return cudaGetLastError();
 }
 
@@ -544,10 +548,10 @@ cudaError_t launch_route_fused(const RouteFusedArgs& a, cudaStream_t s) {
     cudaError_t err;
     if (wf == kF32) {
         if ((err = set_smem(route_fused_kernel<kF32>, smem)) != cudaSuccess) return err;
-        route_fused_kernel<kF32><<<rblocks + lblocks + sblocks, kThreads, smem, s>>>(a);
+        { const cudaError_t e_ = launch_pdl(route_fused_kernel<kF32>, dim3(rblocks + lblocks + sblocks), dim3(kThreads), smem, s, a); if (e_ != cudaSuccess) return e_; }
     } else {
         if ((err = set_smem(route_fused_kernel<kBF16>, smem)) != cudaSuccess) return err;
-        route_fused_kernel<kBF16><<<rblocks + lblocks + sblocks, kThreads, smem, s>>>(a);
+        { const cudaError_t e_ = launch_pdl(route_fused_kernel<kBF16>, dim3(rblocks + lblocks + sblocks), dim3(kThreads), smem, s, a); if (e_ != cudaSuccess) return e_; }
     }
     return cudaGetLastError();
 }
@@ -561,11 +565,11 @@ cudaError_t launch_dense_gemv(const DenseGemvArgs& a, cudaStream_t s) {
     if (a.act_dtype == kF32) {
         const size_t smem = stage_bytes(kF32, a.K);
         if ((err = set_smem(dense_gemv_kernel<float>, smem)) != cudaSuccess) return err;
-        dense_gemv_kernel<float><<<grid, kThreads, smem, s>>>(a);
+        { const cudaError_t e_ = launch_pdl(dense_gemv_kernel<float>, dim3(grid), dim3(kThreads), smem, s, a); if (e_ != cudaSuccess) return e_; }
     } else {
         const size_t smem = stage_bytes(kBF16, a.K);
         if ((err = set_smem(dense_gemv_kernel<__nv_bfloat16>, smem)) != cudaSuccess) return err;
-        dense_gemv_kernel<__nv_bfloat16><<<grid, kThreads, smem, s>>>(a);
+        { const cudaError_t e_ = launch_pdl(dense_gemv_kernel<__nv_bfloat16>, dim3(grid), dim3(kThreads), smem, s, a); if (e_ != cudaSuccess) return e_; }
     }
     return cudaGetLastError();
 }

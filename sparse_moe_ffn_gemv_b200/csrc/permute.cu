@@ -19,6 +19,7 @@ constexpr int kPlaceThreads = 512;
 constexpr int kPlaceWarps = kPlaceThreads / 32;
 
 __global__ void __launch_bounds__(256) hist_kernel(PermuteArgs a) {
+    pdl_begin();
     __shared__ int hist[kPermE];
     for (int e = threadIdx.x; e < a.E; e += blockDim.x) hist[e] = 0;
     __syncthreads();
@@ -34,6 +35,7 @@ __global__ void __launch_bounds__(256) hist_kernel(PermuteArgs a) {
 }
 
 __global__ void __launch_bounds__(kPlaceThreads) place_kernel(PermuteArgs a) {
+    pdl_begin();
     __shared__ PlaceSmem<kPlaceThreads> sm;
     place_chunk<kPlaceThreads>(a, blockIdx.x, sm);
 }
@@ -41,6 +43,7 @@ __global__ void __launch_bounds__(kPlaceThreads) place_kernel(PermuteArgs a) {
 // Compact list of the experts that hold tokens, from offsets [E + 1]
 // (moe_grouped_ffn called with a caller-made permutation).
 __global__ void __launch_bounds__(kPlaceThreads) active_kernel(const int32_t* offsets, int E, int32_t* active) {
+    pdl_begin();
     __shared__ int flags[kPermE];
     __shared__ int warp_tot[kPlaceWarps + 1];
     const int tid = threadIdx.x;
@@ -54,6 +57,7 @@ __global__ void __launch_bounds__(kPlaceThreads) active_kernel(const int32_t* of
 
 __global__ void __launch_bounds__(kPlaceThreads) tile_start_kernel(const int32_t* offsets, int E, int bn,
                                                                  int32_t* tile_start) {
+    pdl_begin();
     __shared__ int v[kPermE];
     __shared__ int warp_tot[kPlaceWarps + 1];
     const int tid = threadIdx.x;
@@ -68,6 +72,7 @@ __global__ void __launch_bounds__(kPlaceThreads) tile_start_kernel(const int32_t
 __global__ void __launch_bounds__(256) gather_rows_kernel(const uint4* __restrict__ src, int vpr,
                                                           const int32_t* __restrict__ sorted_slot, int k,
                                                           int64_t S, uint4* __restrict__ dst) {
+    pdl_begin();
     const int lane = threadIdx.x & 31;
     const int64_t p = (int64_t(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
     if (p >= S) return;
@@ -84,29 +89,29 @@ cudaError_t launch_gather_rows(const void* src, int K, const int32_t* sorted_slo
     if (S == 0) return cudaSuccess;
     const int vpr = K * 2 / 16;
     const unsigned grid = unsigned((S * 32 + 255) / 256);
-    gather_rows_kernel<<<grid, 256, 0, s>>>(static_cast<const uint4*>(src), vpr, sorted_slot, k, S,
-                                            static_cast<uint4*>(dst));
+    { const cudaError_t e_ = launch_pdl(gather_rows_kernel, dim3(grid), dim3(256), 0, s, static_cast<const uint4*>(src), vpr, sorted_slot, k, S,
+                                            static_cast<uint4*>(dst)); if (e_ != cudaSuccess) return e_; }
     return cudaGetLastError();
 }
 
 cudaError_t launch_tile_start(const int32_t* offsets, int E, int tile_bn, int32_t* tile_start, cudaStream_t s) {
-    tile_start_kernel<<<1, kPlaceThreads, 0, s>>>(offsets, E, tile_bn, tile_start);
+    { const cudaError_t e_ = launch_pdl(tile_start_kernel, dim3(1), dim3(kPlaceThreads), 0, s, offsets, E, tile_bn, tile_start); if (e_ != cudaSuccess) return e_; }
     return cudaGetLastError();
 }
 
 cudaError_t launch_active_list(const int32_t* offsets, int E, int32_t* active, cudaStream_t s) {
-    active_kernel<<<1, kPlaceThreads, 0, s>>>(offsets, E, active);
+    { const cudaError_t e_ = launch_pdl(active_kernel, dim3(1), dim3(kPlaceThreads), 0, s, offsets, E, active); if (e_ != cudaSuccess) return e_; }
     return cudaGetLastError();
 }
 
 cudaError_t launch_permute(const PermuteArgs& a, cudaStream_t s) {
     if (a.S == 0) return cudaSuccess;
     if (a.n_chunks > 1) {
-        hist_kernel<<<a.n_chunks, 256, 0, s>>>(a);
+        { const cudaError_t e_ = launch_pdl(hist_kernel, dim3(a.n_chunks), dim3(256), 0, s, a); if (e_ != cudaSuccess) return e_; }
         cudaError_t err = cudaGetLastError();
         if (err != cudaSuccess) return err;
     }
-    place_kernel<<<a.n_chunks, kPlaceThreads, 0, s>>>(a);
+    { const cudaError_t e_ = launch_pdl(place_kernel, dim3(a.n_chunks), dim3(kPlaceThreads), 0, s, a); if (e_ != cudaSuccess) return e_; }
     return cudaGetLastError();
 }
 

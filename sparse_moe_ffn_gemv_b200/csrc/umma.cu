@@ -290,6 +290,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
             prefetch_tmap(&P.b[i]);
         }
     }
+    pdl_begin();  // everything above touches no memory that earlier kernels write
     for (int i = 0; i < P.nprob; ++i) {
         if (!P.p[i].grouped) continue;
         for (int e = threadIdx.x; e <= P.p[i].num_groups; e += blockDim.x) {
@@ -580,7 +581,7 @@ cudaError_t launch_tc_t(TcParams& P, int64_t max_tiles, cudaStream_t s) {
     if (err != cudaSuccess) return err;
     const int grid = int(std::min<int64_t>(max_tiles, sm_count()));
     if (grid <= 0) return cudaSuccess;
-    kern<<<grid, kTcThreads, S::SMEM, s>>>(P);
+    { const cudaError_t e_ = launch_pdl(kern, dim3(grid), dim3(kTcThreads), S::SMEM, s, P); if (e_ != cudaSuccess) return e_; }
     return cudaGetLastError();
 }
 
