@@ -185,20 +185,6 @@ bool routed_tc(const moe_config* c, int64_t T) {
     return o == kPathTc || (o == kPathAuto && T * c->top_k >= 8 * int64_t(c->num_experts));
 }
 
-// Small batches whose router, shared expert and latent projection all take the
-// weight-streaming path route in one fused launch (the permutation fits one chunk).
-bool fused_route(const moe_config* c, int64_t T) {
-    if (path_override() == kPathTc) return false;
-    if (T * c->top_k > kPermChunk) return false;
-    if (dense_tc(c, T, c->hidden) || routed_tc(c, T)) return false;
-    if (c->latent_dim && dense_tc(c, T, c->hidden)) return false;
-    return true;
-}
-
-// Word offset (in ints) of the fused routing launch's completion counter in the
-// workspace's 256-byte status region (the status word is word 0).
-constexpr int kCounterWord = 16;
-
 #define MOE_CHECK(expr)                          \
     do {                                         \
         const moe_status _s = (expr);            \
@@ -441,7 +427,7 @@ struct RoutedSum {
 moe_status run_experts(const moe_config* c, const moe_weights* w, const void* u, const void* x, int64_t T,
                        const int32_t* offsets, const int32_t* sorted_slot, const float* topk_w,
                        float* y_acc, bool with_routed, bool with_shared, void* ws, const WsLayout& L,
-                       cudaStream_t s, RoutedSum* sum, bool shared_gate_up_done = false) {
+                       cudaStream_t s, RoutedSum* sum) {
     const int K = expert_in(*c);
     const bool sh = with_shared && c->shared_mode != MOE_SHARED_NONE;
     const bool rtc = with_routed && routed_tc(c, T);
@@ -471,7 +457,7 @@ moe_status run_experts(const moe_config* c, const moe_weights* w, const void* u,
     g.routed_groups = int(groups);
     g.u = u;
     g.h = at<void>(ws, L.h);
-    if (sh && !stc && !shared_gate_up_done) {
+    if (sh && !stc) {
         g.sg_w = w->shared_gate_w;
         g.su_w = w->shared_up_w;
         g.shared_I = c->shared_intermediate;
@@ -717,54 +703,6 @@ moe_status moe_block_forward(const moe_config* cfg, const moe_weights* w, const 
     const void* u = cfg->latent_dim ? at<void>(ws, L.z) : x;
     int32_t* offsets = at<int32_t>(ws, L.offsets);
     int32_t* sorted_slot = at<int32_t>(ws, L.sorted_slot);
-    const bool sh = cfg->shared_mode != MOE_SHARED_NONE;
-    if (fused_route(cfg, T)) {
-        // small batch: router, latent down, shared gate/up, top-k and permutation in one launch
-        RouteFusedArgs f;
-        f.router = router_args(cfg, w, x, T, ws, L);
-        if (cfg->latent_dim) {
-            f.latent.W0 = w->latent_down_w;
-            f.latent.rows0 = cfg->latent_dim;
-            f.latent.u = x;
-            f.latent.T = T;
-            f.latent.K = cfg->hidden;
-            f.latent.out = at<void>(ws, L.z);
-            f.latent.ld_out = cfg->latent_dim;
-            f.latent.act_dtype = cfg->act_dtype;
-        }
-        if (sh) {
-            f.shared.wf = cfg->act_dtype;
-            f.shared.sg_w = w->shared_gate_w;
-            f.shared.su_w = w->shared_up_w;
-            f.shared.shared_I = cfg->shared_intermediate;
-            f.shared.Hs = cfg->hidden;
-            f.shared.xs = x;
-            f.shared.hs = at<void>(ws, L.hs);
-            f.shared.T = T;
-            f.shared.act = cfg->activation;
-            f.shared.limit = cfg->swiglu_limit;
-            f.shared.alpha = cfg->swiglu_alpha;
-        }
-        f.topk = topk_args(cfg, w, T, idx, wts, coef, ws, L);
-        f.perm.idx = idx;
-        f.perm.S = T * cfg->top_k;
-        f.perm.E = cfg->num_experts;
-        f.perm.offsets = offsets;
-        f.perm.sorted_slot = sorted_slot;
-        f.perm.slot_pos = at<int32_t>(ws, L.slot_pos);
-        f.perm.active = at<int32_t>(ws, L.active);
-        f.perm.chunk_hist = at<int32_t>(ws, L.chunk_hist);
-        f.perm.n_chunks = 1;
-        f.perm.status = at<int>(ws, L.status);
-        f.zero = y_acc;
-        f.zero_floats = T * K;
-        f.counter = at<int>(ws, L.status) + kCounterWord;
-        MOE_CUDA(launch_route_fused(f, s));
-        RoutedSum rs;
-        MOE_CHECK(run_experts(cfg, w, u, x, T, offsets, sorted_slot, wts, y_acc, true, true, ws, L, s, &rs,
-                              /*shared_gate_up_done=*/sh));
-        return run_output(cfg, w, rs, coef, T, y, ws, L, s);
-    }
     // the weight-streaming path scatter-adds into y_acc: its rows are cleared by the router
     MOE_CHECK(run_route(cfg, w, x, T, idx, wts, coef, rtc ? nullptr : y_acc, K, ws, L, s));
     if (cfg->latent_dim) MOE_CHECK(run_latent_down(cfg, w, x, T, at<void>(ws, L.z), at<int>(ws, L.status), s));

@@ -16,8 +16,6 @@
 
 #include "common.cuh"
 #include "internal.h"
-#include "permute_dev.cuh"
-#include "topk_dev.cuh"
 
 namespace moe {
 
@@ -393,91 +391,6 @@ __global__ void __launch_bounds__(kThreads) dense_gemv_kernel(DenseGemvArgs a) {
     }
 }
 
-// All rows of one 8-row block of a dense GEMV, for every token (passes of kTT tokens).
-template <int WF>
-__device__ void dense_rows_block(const DenseGemvArgs& a, int rblock, typename Fmt<WF>::AT* us) {
-    using AT = typename Fmt<WF>::AT;
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int r = rblock * kRowsPerBlock + warp;
-    const int rows = a.rows0 + a.rows1;
-    const bool live = r < rows;
-    const int rr = live ? (r < a.rows0 ? r : r - a.rows0) : 0;
-    const void* W = (live && r >= a.rows0) ? a.W1 : a.W0;
-    const void* bias = live ? (r < a.rows0 ? a.b0 : a.b1) : nullptr;
-    const char* rowp[1] = {reinterpret_cast<const char*>(W) + int64_t(rr) * row_bytes<WF>(a.K)};
-    QRow q[1] = {{nullptr, nullptr}};
-    const float b = bias ? ld_act<AT>(bias, rr) : 0.f;
-    for (int64_t p0 = 0; p0 < a.T; p0 += kTT) {
-        const int tt = int(a.T - p0 < kTT ? a.T - p0 : kTT);
-        __syncthreads();
-        stage_tokens<WF>(a.u, a.K, p0, tt, nullptr, 1, us, nullptr);
-        __syncthreads();
-        if (!live) continue;
-        float acc[1][kTT];
-#pragma unroll
-        for (int t = 0; t < kTT; ++t) acc[0][t] = 0.f;
-        dot_rows<WF, 1>(rowp, q, a.K, 64, us, nullptr, tt, acc);
-#pragma unroll
-        for (int t = 0; t < kTT; ++t) {
-            if (t >= tt) break;
-            acc[0][t] = warp_sum(acc[0][t]);
-        }
-#pragma unroll
-        for (int t = 0; t < kTT; ++t) {
-            if (t < tt && lane == t) {
-                const int64_t p = p0 + t;
-                float v = acc[0][t] + b;
-                if (a.addend) v += a.addend[p * a.ld_add + r];
-                if (a.out_f32) reinterpret_cast<float*>(a.out)[p * a.ld_out + r] = v;
-                else reinterpret_cast<AT*>(a.out)[p * a.ld_out + r] = from_f<AT>(v);
-            }
-        }
-    }
-}
-
-template <int WFD>
-__global__ void __launch_bounds__(kThreads) route_fused_kernel(RouteFusedArgs a) {
-    pdl_begin();
-    using AT = typename Fmt<WFD>::AT;
-    extern __shared__ uint4 smem_raw[];
-    AT* us = reinterpret_cast<AT*>(smem_raw);
-    __shared__ int is_last;
-    const int rblocks = (a.router.rows0 + a.router.rows1 + kRowsPerBlock - 1) / kRowsPerBlock;
-    const int lblocks = a.latent.rows0 ? (a.latent.rows0 + kRowsPerBlock - 1) / kRowsPerBlock : 0;
-    int b = blockIdx.x;
-    if (b >= rblocks) {
-        b -= rblocks;
-        if (b < lblocks) {
-            dense_rows_block<WFD>(a.latent, b, us);
-        } else {
-            b -= lblocks;
-            gateup_group<WFD>(a.shared, true, -1, b * kRowsPerBlock, 0, a.shared.T, a.shared.Hs,
-                              a.shared.shared_I, us, nullptr);
-        }
-        return;
-    }
-    if (a.zero) {  // this block's slice of the routed sum (scatter-added by the down kernel)
-        const int64_t n4 = a.zero_floats / 4;
-        const int64_t lo = n4 * b / rblocks, hi = n4 * (b + 1) / rblocks;
-        float4* z = reinterpret_cast<float4*>(a.zero);
-        for (int64_t i = lo + threadIdx.x; i < hi; i += blockDim.x) z[i] = make_float4(0.f, 0.f, 0.f, 0.f);
-    }
-    dense_rows_block<WFD>(a.router, b, us);
-    // the last router block to finish routes every token (logits published by fence + counter)
-    __syncthreads();
-    if (threadIdx.x == 0) {
-        __threadfence();
-        is_last = atomicAdd(a.counter, 1) == rblocks - 1;
-    }
-    __syncthreads();
-    if (!is_last) return;
-    __threadfence();
-    for (int64_t t = threadIdx.x >> 5; t < a.topk.T; t += kThreads / 32) topk_token(a.topk, t);
-    __syncthreads();
-    place_chunk<kThreads>(a.perm, 0, *reinterpret_cast<PlaceSmem<kThreads>*>(smem_raw));
-    if (threadIdx.x == 0) *a.counter = 0;
-}
-
 template <typename KernelT>
 cudaError_t set_smem(KernelT kernel, size_t bytes) {
     if (bytes <= 48 * 1024) return cudaSuccess;
@@ -535,25 +448,6 @@ cudaError_t launch_down_gemv(const DownArgs& a, cudaStream_t s) {
         case kBF16: return launch_down_t<kBF16>(a, s);
         default: return launch_down_t<kQ4>(a, s);
     }
-}
-
-cudaError_t launch_route_fused(const RouteFusedArgs& a, cudaStream_t s) {
-    const int wf = a.router.act_dtype;
-    size_t smem = std::max(stage_bytes(wf, a.router.K), sizeof(PlaceSmem<kThreads>));
-    if (a.latent.rows0) smem = std::max(smem, stage_bytes(wf, a.latent.K));
-    if (a.shared.shared_I) smem = std::max(smem, stage_bytes(wf, a.shared.Hs));
-    const int rblocks = (a.router.rows0 + a.router.rows1 + kRowsPerBlock - 1) / kRowsPerBlock;
-    const int lblocks = a.latent.rows0 ? (a.latent.rows0 + kRowsPerBlock - 1) / kRowsPerBlock : 0;
-    const int sblocks = a.shared.shared_I ? (a.shared.shared_I + kRowsPerBlock - 1) / kRowsPerBlock : 0;
-    cudaError_t err;
-    if (wf == kF32) {
-        if ((err = set_smem(route_fused_kernel<kF32>, smem)) != cudaSuccess) return err;
-        { const cudaError_t e_ = launch_pdl(route_fused_kernel<kF32>, dim3(rblocks + lblocks + sblocks), dim3(kThreads), smem, s, a); if (e_ != cudaSuccess) return e_; }
-    } else {
-        if ((err = set_smem(route_fused_kernel<kBF16>, smem)) != cudaSuccess) return err;
-        { const cudaError_t e_ = launch_pdl(route_fused_kernel<kBF16>, dim3(rblocks + lblocks + sblocks), dim3(kThreads), smem, s, a); if (e_ != cudaSuccess) return e_; }
-    }
-    return cudaGetLastError();
 }
 
 cudaError_t launch_dense_gemv(const DenseGemvArgs& a, cudaStream_t s) {

@@ -81,22 +81,6 @@ struct DownArgs {
 };
 cudaError_t launch_down_gemv(const DownArgs& a, cudaStream_t s);
 
-// Routing for small batches in one launch: router rows (clearing a slice of the routed
-// sum), optional latent down-projection rows, shared-expert gate/up units; the last
-// router block to finish then takes the top-k of every token and the permutation
-// (single chunk: T * k <= 2048 slots). counter must be zero on entry and is left zero.
-struct RouteFusedArgs {
-    DenseGemvArgs router;   // E router rows (+ 2 coefficient rows) -> fp32 logits
-    DenseGemvArgs latent;   // rows0 == 0: no latent projection in this launch
-    GateUpArgs shared;      // shared_I == 0: no shared expert in this launch
-    TopkArgs topk;
-    PermuteArgs perm;
-    float* zero = nullptr;
-    int64_t zero_floats = 0;
-    int* counter = nullptr;
-};
-cudaError_t launch_route_fused(const RouteFusedArgs& a, cudaStream_t s);
-
 // The routed sum of token t is the sum of rows [t*nsum, (t+1)*nsum) of `rows` (width H):
 // nsum = 1 for an accumulated [T, H] buffer, nsum = k for per-slot weighted rows.
 // y = r | r + s | c0 r + c1 s, stored in act dtype (or f32 when out_f32).
