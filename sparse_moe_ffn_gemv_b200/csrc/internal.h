@@ -90,53 +90,6 @@ cudaError_t launch_combine(const float* rows, int nsum, const float* s_acc, cons
 cudaError_t launch_rmsnorm(const float* rows, int nsum, const void* gamma, float eps, int64_t T, int L,
                            void* out, int act_dtype, cudaStream_t s);
 
-// ------------------------------------------------------------------ streamed GEMV
-// Weight-streaming launch for few tokens per weight row: a producer thread per CTA copies
-// items of R consecutive weight rows (gate/up: R/2 units, their gate and up rows) into a
-// shared-memory ring with bulk asynchronous copies; eight consumer warps multiply them with
-// the group's tokens (read through L1). One launch runs up to two parts (e.g. the shared
-// expert as a dense group and the routed experts as groups).
-enum { kStreamGateUp = 0, kStreamDown = 1, kStreamDense = 2 };
-enum { kOutAct = 0, kOutF32 = 1, kOutScatter = 2 };
-
-struct StreamPart {
-    int fmt = MOE_DTYPE_BF16;          // weight format of this part
-    int M = 0;                         // gate/up: units per group; otherwise rows per group
-    int K = 0;                         // inputs per row
-    int R = 8;                         // weight rows per item (gate/up: even)
-    const void* w0 = nullptr;          // gate (or interleaved gate_up) / single plane
-    const void* w1 = nullptr;          // up plane (separate gate/up)
-    const void *s0 = nullptr, *z0 = nullptr, *s1 = nullptr, *z1 = nullptr;  // 4-bit companions
-    int interleaved = 0;
-    int group_size = 64;
-    const void* bias0 = nullptr;       // gate (or interleaved gate_up) bias / row bias
-    const void* bias1 = nullptr;       // up bias (separate)
-    int grouped = 0;                   // 1: routed groups (active list), 0: one dense group of T tokens
-    const void* u = nullptr;           // input rows (act dtype, K each)
-    int u_by_slot = 0;                 // input row of sorted position p = sorted_slot[p] / k
-    void* out = nullptr;
-    int64_t ld_out = 0;
-    int out_kind = kOutAct;
-    const float* addend = nullptr;     // dense: out = dot + bias + addend[t, r]
-    int64_t ld_add = 0;
-};
-
-struct StreamArgs {
-    StreamPart part[2];
-    int nparts = 0;
-    int mode = kStreamGateUp;
-    int act_dtype = MOE_DTYPE_BF16;
-    const int32_t *offsets = nullptr, *sorted_slot = nullptr, *active = nullptr;
-    const float* topk_w = nullptr;
-    int k = 1;
-    int64_t T = 0;
-    int max_groups = 0;                // bound on routed groups (grid sizing)
-    int act = 0;
-    float limit = 7.f, alpha = 1.702f;
-    int* status = nullptr;
-};
-cudaError_t launch_stream(StreamArgs& a, cudaStream_t s);
-
 // ------------------------------------------------------------------ tensor-core GEMM
 constexpr int kTcBN = 128;       // token columns per tile
 constexpr int kTcRowsGateUp = 128;  // intermediate units per gate/up tile (gate + up rows)
