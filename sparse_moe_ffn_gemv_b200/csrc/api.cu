@@ -52,7 +52,7 @@ WsLayout ws_layout(const moe_config& c, int64_t T) {
     L.nrm = take(Ld ? T * Ld * ab : 0);
     const bool tc = c.act_dtype == MOE_DTYPE_BF16 && c.weight_format == MOE_DTYPE_BF16;
     L.uperm = take(tc ? T * k * K * 2 : 0);
-    L.oslot = take(tc ? T * k * K * 4 : 0);
+    L.oslot = take(tc ? T * k * K * 2 : 0);
     L.tiles = take((E + 1) * 4);
     L.total = off;
     return L;
@@ -402,7 +402,7 @@ moe_status run_experts_tc(const moe_config* c, const moe_weights* w, const void*
             p.grouped = 1; p.num_groups = E; p.offsets = offsets; p.tile_start = tiles;
             p.sorted_slot = sorted_slot; p.topk_w = topk_w; p.k = k;
             p.bias0 = c->has_expert_bias ? w->down_b : nullptr;
-            p.out = at<float>(ws, L.oslot); p.ld_out = K;
+            p.out = at<__nv_bfloat16>(ws, L.oslot); p.ld_out = K;
             if (!tc_weight_map(&P.a0[np], w->down_w, E, K, I, false) || !tc_token_map(&P.b[np], h, S, I, kTcBN))
                 return MOE_ERR_CUDA;
             max_tiles += int64_t(p.m_blocks) * max_routed_tiles(*c, T);
@@ -418,8 +418,9 @@ moe_status run_experts_tc(const moe_config* c, const moe_weights* w, const void*
 // Where the routed sum lives after run_experts: token t's sum is the sum of rows
 // [t*nsum, (t+1)*nsum) of `rows` (width K).
 struct RoutedSum {
-    const float* rows = nullptr;
+    const void* rows = nullptr;
     int nsum = 1;
+    int dtype = MOE_DTYPE_F32;  // bf16 for the tensor-core path's per-slot rows
 };
 
 // a4 + a5 (+ a6 when with_shared). On the weight-streaming path y_acc must be zero on
@@ -433,8 +434,9 @@ moe_status run_experts(const moe_config* c, const moe_weights* w, const void* u,
     const bool rtc = with_routed && routed_tc(c, T);
     const bool stc = sh && c->shared_intermediate % 64 == 0 && dense_tc(c, T, c->hidden);
     if (sum) {
-        sum->rows = rtc ? at<float>(ws, L.oslot) : y_acc;
+        sum->rows = rtc ? at<void>(ws, L.oslot) : static_cast<const void*>(y_acc);
         sum->nsum = rtc ? c->top_k : 1;
+        sum->dtype = rtc ? MOE_DTYPE_BF16 : MOE_DTYPE_F32;
     }
     if (rtc || stc)
         MOE_CHECK(run_experts_tc(c, w, u, x, T, offsets, sorted_slot, topk_w, rtc, stc, ws, L, s));
@@ -533,16 +535,16 @@ moe_status run_output(const moe_config* c, const moe_weights* w, RoutedSum rs, c
                       int64_t T, void* y, void* ws, const WsLayout& L, cudaStream_t s) {
     const float* s_acc = c->shared_mode != MOE_SHARED_NONE ? at<float>(ws, L.s_acc) : nullptr;
     if (!c->latent_dim) {
-        MOE_CUDA(launch_combine(rs.rows, rs.nsum, s_acc, coef, c->shared_mode, T, c->hidden, y, c->act_dtype, s));
+        MOE_CUDA(launch_combine(rs.rows, rs.dtype, rs.nsum, s_acc, coef, c->shared_mode, T, c->hidden, y, c->act_dtype, s));
         return MOE_OK;
     }
     const void* n = nullptr;
     if (c->latent_use_norm) {
-        MOE_CUDA(launch_rmsnorm(rs.rows, rs.nsum, w->latent_norm_w, c->rms_eps, T, c->latent_dim,
+        MOE_CUDA(launch_rmsnorm(rs.rows, rs.dtype, rs.nsum, w->latent_norm_w, c->rms_eps, T, c->latent_dim,
                                 at<void>(ws, L.nrm), c->act_dtype, s));
     } else {
         // no norm: the routed latent sum rounded to the activation dtype
-        MOE_CUDA(launch_combine(rs.rows, rs.nsum, nullptr, nullptr, MOE_SHARED_NONE, T, c->latent_dim,
+        MOE_CUDA(launch_combine(rs.rows, rs.dtype, rs.nsum, nullptr, nullptr, MOE_SHARED_NONE, T, c->latent_dim,
                                 at<void>(ws, L.nrm), c->act_dtype, s));
     }
     n = at<void>(ws, L.nrm);
@@ -649,7 +651,7 @@ moe_status moe_grouped_ffn(const moe_config* cfg, const moe_weights* w, const vo
     MOE_CHECK(run_experts(cfg, w, u, nullptr, T, expert_offsets, sorted_slot, topk_w, y_acc, true, false, ws, L, s,
                           &rs));
     if (rs.rows != y_acc)  // per-slot rows: sum each token's k rows into y_acc
-        MOE_CUDA(launch_combine(rs.rows, rs.nsum, nullptr, nullptr, MOE_SHARED_NONE, T, expert_in(*cfg), y_acc,
+        MOE_CUDA(launch_combine(rs.rows, rs.dtype, rs.nsum, nullptr, nullptr, MOE_SHARED_NONE, T, expert_in(*cfg), y_acc,
                                 cfg->act_dtype, s, true));
     return MOE_OK;
 }

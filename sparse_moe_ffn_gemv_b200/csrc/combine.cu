@@ -12,19 +12,31 @@ namespace moe {
 
 namespace {
 
-__device__ __forceinline__ float4 routed_sum(const float* __restrict__ rows, int nsum, int64_t t, int64_t c4,
-                                             int H4) {
-    const float4* p = reinterpret_cast<const float4*>(rows) + (t * nsum) * H4 + c4;
-    float4 r = p[0];
+// Four consecutive routed values of token t, columns 4*c4 .. 4*c4+3: the sum of the
+// token's nsum rows (fp32 rows, or bf16 rows as the tensor-core down GEMM writes them).
+template <typename RT>
+__device__ __forceinline__ float4 load4(const RT* p);
+template <> __device__ __forceinline__ float4 load4<float>(const float* p) {
+    return *reinterpret_cast<const float4*>(p);
+}
+template <> __device__ __forceinline__ float4 load4<__nv_bfloat16>(const __nv_bfloat16* p) {
+    const uint2 w = *reinterpret_cast<const uint2*>(p);
+    return make_float4(bf16lo(w.x), bf16hi(w.x), bf16lo(w.y), bf16hi(w.y));
+}
+
+template <typename RT>
+__device__ __forceinline__ float4 routed_sum(const RT* __restrict__ rows, int nsum, int64_t t, int64_t c4, int H4) {
+    const RT* p = rows + ((t * nsum) * H4 + c4) * 4;
+    float4 r = load4<RT>(p);
     for (int j = 1; j < nsum; ++j) {
-        const float4 v = p[int64_t(j) * H4];
+        const float4 v = load4<RT>(p + int64_t(j) * H4 * 4);
         r.x += v.x; r.y += v.y; r.z += v.z; r.w += v.w;
     }
     return r;
 }
 
-template <typename AT>
-__global__ void __launch_bounds__(256) combine_kernel(const float* __restrict__ rows, int nsum,
+template <typename AT, typename RT>
+__global__ void __launch_bounds__(256) combine_kernel(const RT* __restrict__ rows, int nsum,
                                                       const float* __restrict__ s_acc,
                                                       const float* __restrict__ coef, int mode,
                                                       int64_t T, int H, AT* __restrict__ y) {
@@ -34,7 +46,7 @@ __global__ void __launch_bounds__(256) combine_kernel(const float* __restrict__ 
     for (int64_t i = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; i < n4;
          i += int64_t(gridDim.x) * blockDim.x) {
         const int64_t t = i / H4;
-        float4 r = routed_sum(rows, nsum, t, i - t * H4, H4);
+        float4 r = routed_sum<RT>(rows, nsum, t, i - t * H4, H4);
         if (mode != MOE_SHARED_NONE) {
             const float4 sv = reinterpret_cast<const float4*>(s_acc)[i];
             if (mode == MOE_SHARED_ADD) {
@@ -55,8 +67,8 @@ __global__ void __launch_bounds__(256) combine_kernel(const float* __restrict__ 
     }
 }
 
-template <typename AT>
-__global__ void __launch_bounds__(256) rmsnorm_kernel(const float* __restrict__ rows, int nsum,
+template <typename AT, typename RT>
+__global__ void __launch_bounds__(256) rmsnorm_kernel(const RT* __restrict__ rows, int nsum,
                                                       const AT* __restrict__ gamma, float eps,
                                                       int L, AT* __restrict__ out) {
     pdl_begin();
@@ -66,7 +78,7 @@ __global__ void __launch_bounds__(256) rmsnorm_kernel(const float* __restrict__ 
     const int L4 = L / 4;
     float ss = 0.f;
     for (int c4 = threadIdx.x; c4 < L4; c4 += blockDim.x) {
-        const float4 v = routed_sum(rows, nsum, t, c4, L4);
+        const float4 v = routed_sum<RT>(rows, nsum, t, c4, L4);
         reinterpret_cast<float4*>(rsum)[c4] = v;
         ss = fmaf(v.x, v.x, fmaf(v.y, v.y, fmaf(v.z, v.z, fmaf(v.w, v.w, ss))));
     }
@@ -82,36 +94,53 @@ __global__ void __launch_bounds__(256) rmsnorm_kernel(const float* __restrict__ 
         out[t * L + c] = from_f<AT>(row[c] * inv * to_f<AT>(gamma[c]));
 }
 
-}  // namespace
-
-cudaError_t launch_combine(const float* rows, int nsum, const float* s_acc, const float* coef, int mode,
-                           int64_t T, int H, void* y, int act_dtype, cudaStream_t s, bool out_f32) {
-    if (T == 0) return cudaSuccess;
+template <typename RT>
+cudaError_t launch_combine_t(const RT* rows, int nsum, const float* s_acc, const float* coef, int mode, int64_t T,
+                             int H, void* y, int act_dtype, cudaStream_t s, bool out_f32) {
     const int64_t n4 = T * H / 4;
     const unsigned grid = unsigned(std::min<int64_t>((n4 + 255) / 256, 148 * 16));
+    cudaError_t e;
     if (act_dtype == kF32 || out_f32)
-        { const cudaError_t e_ = launch_pdl(combine_kernel<float>, dim3(grid), dim3(256), 0, s, rows, nsum, s_acc, coef, mode, T, H, static_cast<float*>(y)); if (e_ != cudaSuccess) return e_; }
+        e = launch_pdl(combine_kernel<float, RT>, dim3(grid), dim3(256), 0, s, rows, nsum, s_acc, coef, mode, T, H,
+                       static_cast<float*>(y));
     else
-        { const cudaError_t e_ = launch_pdl(combine_kernel<__nv_bfloat16>, dim3(grid), dim3(256), 0, s, rows, nsum, s_acc, coef, mode, T, H,
-                                                           static_cast<__nv_bfloat16*>(y)); if (e_ != cudaSuccess) return e_; }
+        e = launch_pdl(combine_kernel<__nv_bfloat16, RT>, dim3(grid), dim3(256), 0, s, rows, nsum, s_acc, coef, mode,
+                       T, H, static_cast<__nv_bfloat16*>(y));
+    if (e != cudaSuccess) return e;
     return cudaGetLastError();
 }
 
-cudaError_t launch_rmsnorm(const float* rows, int nsum, const void* gamma, float eps, int64_t T, int L,
-                           void* out, int act_dtype, cudaStream_t s) {
-    if (T == 0) return cudaSuccess;
+template <typename AT, typename RT>
+cudaError_t launch_rmsnorm_t(const RT* rows, int nsum, const void* gamma, float eps, int64_t T, int L, void* out,
+                             cudaStream_t s) {
     const size_t smem = size_t(L) * sizeof(float);
-    if (act_dtype == kF32) {
-        cudaFuncSetAttribute(rmsnorm_kernel<float>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
-        { const cudaError_t e_ = launch_pdl(rmsnorm_kernel<float>, dim3(unsigned(T)), dim3(256), smem, s, rows, nsum, static_cast<const float*>(gamma), eps, L,
-                                                             static_cast<float*>(out)); if (e_ != cudaSuccess) return e_; }
-    } else {
-        cudaFuncSetAttribute(rmsnorm_kernel<__nv_bfloat16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             int(smem));
-        { const cudaError_t e_ = launch_pdl(rmsnorm_kernel<__nv_bfloat16>, dim3(unsigned(T)), dim3(256), smem, s, 
-            rows, nsum, static_cast<const __nv_bfloat16*>(gamma), eps, L, static_cast<__nv_bfloat16*>(out)); if (e_ != cudaSuccess) return e_; }
-    }
+    cudaError_t e = cudaFuncSetAttribute(rmsnorm_kernel<AT, RT>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
+    if (e != cudaSuccess) return e;
+    e = launch_pdl(rmsnorm_kernel<AT, RT>, dim3(unsigned(T)), dim3(256), smem, s, rows, nsum,
+                   static_cast<const AT*>(gamma), eps, L, static_cast<AT*>(out));
+    if (e != cudaSuccess) return e;
     return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_combine(const void* rows, int rows_dtype, int nsum, const float* s_acc, const float* coef,
+                           int mode, int64_t T, int H, void* y, int act_dtype, cudaStream_t s, bool out_f32) {
+    if (T == 0) return cudaSuccess;
+    if (rows_dtype == kBF16)
+        return launch_combine_t(static_cast<const __nv_bfloat16*>(rows), nsum, s_acc, coef, mode, T, H, y, act_dtype,
+                                s, out_f32);
+    return launch_combine_t(static_cast<const float*>(rows), nsum, s_acc, coef, mode, T, H, y, act_dtype, s, out_f32);
+}
+
+cudaError_t launch_rmsnorm(const void* rows, int rows_dtype, int nsum, const void* gamma, float eps, int64_t T,
+                           int L, void* out, int act_dtype, cudaStream_t s) {
+    if (T == 0) return cudaSuccess;
+    if (act_dtype == kF32)
+        return launch_rmsnorm_t<float>(static_cast<const float*>(rows), nsum, gamma, eps, T, L, out, s);
+    if (rows_dtype == kBF16)
+        return launch_rmsnorm_t<__nv_bfloat16>(static_cast<const __nv_bfloat16*>(rows), nsum, gamma, eps, T, L, out, s);
+    return launch_rmsnorm_t<__nv_bfloat16>(static_cast<const float*>(rows), nsum, gamma, eps, T, L, out, s);
 }
 
 }  // namespace moe

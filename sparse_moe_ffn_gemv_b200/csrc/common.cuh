@@ -42,7 +42,7 @@ struct WsLayout {
     size_t z;            // act [T, L]: latent input of the experts
     size_t nrm;          // act [T, L]: normalised latent
     size_t uperm;        // bf16 [T * k, K]: expert inputs gathered in sorted order
-    size_t oslot;        // f32 [T * k, K]: weighted expert output of every slot
+    size_t oslot;        // bf16 [T * k, K]: weighted expert output of every slot
     size_t tiles;        // int32 tile list of the tensor-core path
     size_t total;
     int ld_logits;

@@ -81,14 +81,15 @@ struct DownArgs {
 };
 cudaError_t launch_down_gemv(const DownArgs& a, cudaStream_t s);
 
-// The routed sum of token t is the sum of rows [t*nsum, (t+1)*nsum) of `rows` (width H):
-// nsum = 1 for an accumulated [T, H] buffer, nsum = k for per-slot weighted rows.
-// y = r | r + s | c0 r + c1 s, stored in act dtype (or f32 when out_f32).
-cudaError_t launch_combine(const float* rows, int nsum, const float* s_acc, const float* coef, int mode,
-                           int64_t T, int H, void* y, int act_dtype, cudaStream_t s, bool out_f32 = false);
+// The routed sum of token t is the sum of rows [t*nsum, (t+1)*nsum) of `rows` (width H,
+// fp32 or bf16 as rows_dtype says): nsum = 1 for an accumulated [T, H] buffer, nsum = k
+// for per-slot weighted rows. y = r | r + s | c0 r + c1 s, stored in act dtype (or f32
+// when out_f32).
+cudaError_t launch_combine(const void* rows, int rows_dtype, int nsum, const float* s_acc, const float* coef,
+                           int mode, int64_t T, int H, void* y, int act_dtype, cudaStream_t s, bool out_f32 = false);
 // nrm = r / sqrt(mean(r^2) + eps) * gamma (act dtype), r the routed sum as above (width L).
-cudaError_t launch_rmsnorm(const float* rows, int nsum, const void* gamma, float eps, int64_t T, int L,
-                           void* out, int act_dtype, cudaStream_t s);
+cudaError_t launch_rmsnorm(const void* rows, int rows_dtype, int nsum, const void* gamma, float eps, int64_t T,
+                           int L, void* out, int act_dtype, cudaStream_t s);
 
 // ------------------------------------------------------------------ tensor-core GEMM
 constexpr int kTcBN = 128;       // token columns per tile

@@ -190,7 +190,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
     uint64_t* drain = acc_empty + 2;
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
     GroupTables& gt = *reinterpret_cast<GroupTables*>(smem + STAGES * S::STAGE_BYTES + 256);
-    float** e_row = reinterpret_cast<float**>(&gt + 1);  // output row of each token column
+    __nv_bfloat16** e_row = reinterpret_cast<__nv_bfloat16**>(&gt + 1);  // output row of each token column
     float* e_w = reinterpret_cast<float*>(e_row + BN);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -350,7 +350,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
                 epi_bar();
                 if (eid < BN && eid < ti.nvalid) {
                     const int slot = p.sorted_slot[ti.row0 + eid];
-                    e_row[eid] = reinterpret_cast<float*>(p.out) + int64_t(slot) * p.ld_out;
+                    e_row[eid] = reinterpret_cast<__nv_bfloat16*>(p.out) + int64_t(slot) * p.ld_out;
                     e_w[eid] = p.topk_w[slot];
                 }
                 epi_bar();
@@ -426,17 +426,18 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
                     const float bias0 = p.bias0 ? bf16_at(p.bias0, int64_t(ti.group) * p.M + r) : 0.f;
                     const int nend = full_tile ? 64 : max(0, ti.nvalid - c_lo);
                     if (p.mode == kEpiSlotRows) {
-                        // weighted output row of each slot; the combine sums a token's k rows
+                        // weighted output row of each slot (bf16); the combine sums a token's k rows
                         if (full_tile) {
 #pragma unroll
                             for (int j = 0; j < 64; ++j)
-                                e_row[c_lo + j][r] = e_w[c_lo + j] * (__uint_as_float(v[a * 2 + j / 32][j % 32]) + bias0);
+                                e_row[c_lo + j][r] =
+                                    __float2bfloat16_rn(e_w[c_lo + j] * (__uint_as_float(v[a * 2 + j / 32][j % 32]) + bias0));
                         } else {
 #pragma unroll
                             for (int j = 0; j < 64; ++j)
                                 if (j < nend)
-                                    e_row[c_lo + j][r] =
-                                        e_w[c_lo + j] * (__uint_as_float(v[a * 2 + j / 32][j % 32]) + bias0);
+                                    e_row[c_lo + j][r] = __float2bfloat16_rn(
+                                        e_w[c_lo + j] * (__uint_as_float(v[a * 2 + j / 32][j % 32]) + bias0));
                         }
                     } else if (p.mode == kEpiStoreF32) {
                         float* o = reinterpret_cast<float*>(p.out) + int64_t(ti.row0 + c_lo) * p.ld_out + r;
