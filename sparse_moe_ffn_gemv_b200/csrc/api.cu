@@ -178,11 +178,15 @@ bool dense_tc(const moe_config* c, int64_t T, int K) {
     const int o = path_override();
     return o == kPathTc || (o == kPathAuto && T >= 64);
 }
+// The routed experts go to the tensor cores once there are about E/4 slots: measured on
+// B200, the TMA-fed tcgen05 kernel streams the activated weights faster than the CUDA-core
+// kernels from there on, although most tiles then hold only a few tokens (Klear shape:
+// 8 tokens 149 vs 157 us, 64 tokens 279 vs 627 us; at 4 tokens the CUDA cores win).
 bool routed_tc(const moe_config* c, int64_t T) {
     if (c->act_dtype != MOE_DTYPE_BF16 || c->weight_format != MOE_DTYPE_BF16) return false;
     if (expert_in(*c) % 64 != 0 || c->intermediate % 64 != 0) return false;
     const int o = path_override();
-    return o == kPathTc || (o == kPathAuto && T * c->top_k >= 8 * int64_t(c->num_experts));
+    return o == kPathTc || (o == kPathAuto && 4 * T * c->top_k >= int64_t(c->num_experts));
 }
 
 #define MOE_CHECK(expr)                          \
@@ -432,7 +436,9 @@ moe_status run_experts(const moe_config* c, const moe_weights* w, const void* u,
     const int K = expert_in(*c);
     const bool sh = with_shared && c->shared_mode != MOE_SHARED_NONE;
     const bool rtc = with_routed && routed_tc(c, T);
-    const bool stc = sh && c->shared_intermediate % 64 == 0 && dense_tc(c, T, c->hidden);
+    // the shared expert joins the routed tensor-core launches whenever those run
+    const bool stc = sh && c->shared_intermediate % 64 == 0 && c->hidden % 64 == 0 &&
+                     c->act_dtype == MOE_DTYPE_BF16 && (dense_tc(c, T, c->hidden) || rtc);
     if (sum) {
         sum->rows = rtc ? at<void>(ws, L.oslot) : static_cast<const void*>(y_acc);
         sum->nsum = rtc ? c->top_k : 1;

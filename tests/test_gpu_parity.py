@@ -208,7 +208,11 @@ def test_out_of_range_expert_id_sets_the_device_status():
 
 
 def test_batch_equals_tokens_one_at_a_time_on_gpu():
-    """Klear PR validation (causality check): a token's output does not depend on the batch."""
+    """Klear PR validation (causality check): a token's output does not depend on the batch.
+
+    24 tokens take the tensor-core engine and one token the weight-streaming engine; each
+    is within the bar (+ half a bf16 ulp) of the exact value, so the two may differ by the
+    sum of both allowances and no more."""
     spec = inputs.KLEAR_BF16
     wcpu, _ = weights(spec)
     T = 24
@@ -218,7 +222,9 @@ def test_batch_equals_tokens_one_at_a_time_on_gpu():
     rms = float(y.pow(2).mean().sqrt())
     for t in (0, 5, 23):
         y1 = blk.forward(x[t:t + 1].contiguous()).float()
-        assert float((y1[0] - y[t]).abs().max()) <= 2e-2 * rms
+        ulp = torch.exp2(torch.floor(torch.log2(y[t].abs().clamp_min(1e-30))) - 7)
+        assert bool(((y1[0] - y[t]).abs() <= 2 * 2e-2 * rms + ulp).all())
+    assert blk.device_status() == 0
 
 
 TC_SMALL = [  # tensor-core path forced: ragged groups, partial tiles, interleaved + biases, latent
