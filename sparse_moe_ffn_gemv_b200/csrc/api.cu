@@ -257,9 +257,14 @@ TopkArgs topk_args(const moe_config* c, const moe_weights* w, int64_t T, int32_t
     return t;
 }
 
+// Where the top-k warp writes the permutation of a single token (moe_block_forward, T == 1).
+struct PermOut {
+    int32_t *offsets = nullptr, *sorted_slot = nullptr, *slot_pos = nullptr, *active = nullptr, *tiles = nullptr;
+};
+
 moe_status run_route(const moe_config* c, const moe_weights* w, const void* x, int64_t T, int32_t* idx,
                      float* wts, float* coef, float* zero, int64_t zero_cols, void* ws, const WsLayout& L,
-                     cudaStream_t s) {
+                     cudaStream_t s, const PermOut* perm = nullptr) {
     const bool blend = c->shared_mode == MOE_SHARED_BLEND;
     const DenseGemvArgs r = router_args(c, w, x, T, ws, L);
     if (dense_tc(c, T, c->hidden)) {
@@ -290,6 +295,13 @@ moe_status run_route(const moe_config* c, const moe_weights* w, const void* x, i
     TopkArgs t = topk_args(c, w, T, idx, wts, coef, ws, L);
     t.zero = zero;
     t.zero_cols = zero_cols;
+    if (perm && T == 1) {
+        t.p_offsets = perm->offsets;
+        t.p_sorted = perm->sorted_slot;
+        t.p_slot_pos = perm->slot_pos;
+        t.p_active = perm->active;
+        t.p_tiles = perm->tiles;
+    }
     MOE_CUDA(launch_topk(t, s));
     return MOE_OK;
 }
@@ -711,10 +723,17 @@ moe_status moe_block_forward(const moe_config* cfg, const moe_weights* w, const 
     const void* u = cfg->latent_dim ? at<void>(ws, L.z) : x;
     int32_t* offsets = at<int32_t>(ws, L.offsets);
     int32_t* sorted_slot = at<int32_t>(ws, L.sorted_slot);
-    // the weight-streaming path scatter-adds into y_acc: its rows are cleared by the router
-    MOE_CHECK(run_route(cfg, w, x, T, idx, wts, coef, rtc ? nullptr : y_acc, K, ws, L, s));
+    // the weight-streaming path scatter-adds into y_acc: its rows are cleared by the router;
+    // a single token's permutation comes from the top-k warp itself
+    PermOut perm;
+    perm.offsets = offsets;
+    perm.sorted_slot = sorted_slot;
+    perm.slot_pos = at<int32_t>(ws, L.slot_pos);
+    perm.active = at<int32_t>(ws, L.active);
+    perm.tiles = rtc ? at<int32_t>(ws, L.tiles) : nullptr;
+    MOE_CHECK(run_route(cfg, w, x, T, idx, wts, coef, rtc ? nullptr : y_acc, K, ws, L, s, &perm));
     if (cfg->latent_dim) MOE_CHECK(run_latent_down(cfg, w, x, T, at<void>(ws, L.z), at<int>(ws, L.status), s));
-    MOE_CHECK(run_permute(cfg, idx, T, offsets, sorted_slot, at<int32_t>(ws, L.slot_pos), ws, L, s, rtc));
+    if (T > 1) MOE_CHECK(run_permute(cfg, idx, T, offsets, sorted_slot, at<int32_t>(ws, L.slot_pos), ws, L, s, rtc));
     RoutedSum rs;
     MOE_CHECK(run_experts(cfg, w, u, x, T, offsets, sorted_slot, wts, y_acc, true, true, ws, L, s, &rs));
     return run_output(cfg, w, rs, coef, T, y, ws, L, s);

@@ -26,9 +26,12 @@ constexpr int kRowsPerBlock = 8;  // one warp per weight row / intermediate unit
 constexpr int kThreads = kRowsPerBlock * 32;
 
 template <int WF> struct Fmt;
-template <> struct Fmt<kF32> { using AT = float; static constexpr int VE = 4; static constexpr int U = 4; };
-template <> struct Fmt<kBF16> { using AT = __nv_bfloat16; static constexpr int VE = 8; static constexpr int U = 4; };
-template <> struct Fmt<kQ4> { using AT = __nv_bfloat16; static constexpr int VE = 32; static constexpr int U = 2; };
+// VE: weights per 16-byte vector; U: vectors per row in flight per lane; DR: down-projection
+// rows per warp (two short rows keep more bytes in flight; with the 4-bit dequantisation's
+// registers one row per warp keeps more warps resident, which measured faster).
+template <> struct Fmt<kF32> { using AT = float; static constexpr int VE = 4, U = 4, DR = 2; };
+template <> struct Fmt<kBF16> { using AT = __nv_bfloat16; static constexpr int VE = 8, U = 4, DR = 2; };
+template <> struct Fmt<kQ4> { using AT = __nv_bfloat16; static constexpr int VE = 32, U = 2, DR = 1; };
 
 // Row pointer of a weight matrix row in a given format (bytes per row).
 template <int WF> __host__ __device__ __forceinline__ int64_t row_bytes(int K) {
@@ -269,56 +272,73 @@ __global__ void __launch_bounds__(kThreads) gateup_gemv_kernel(GateUpArgs a) {
     gateup_group<WF>(a, false, e, (b - ai * ublocks) * kRowsPerBlock, p0, cnt, a.K, a.I, us, xsum);
 }
 
-// One block of 8 output rows of one group's down projection.
-template <int WF>
+// One block of 8 * NR output rows of one group's down projection, NR rows per warp.
+template <int WF, int NR>
 __device__ void down_group(const DownArgs& a, bool shared, int e, int row0, int64_t p0, int64_t cnt,
                            int I, int R, typename Fmt<WF>::AT* us, float* xsum) {
     using AT = typename Fmt<WF>::AT;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int r = row0 + warp;
-    const bool live = r < R;
+    const int rbase = row0 + warp * NR;
     const int64_t rb = row_bytes<WF>(I);
-    const char* rows[1];
-    QRow q[1] = {{nullptr, nullptr}};
-    float bd = 0.f;
-    if (shared) {
-        rows[0] = reinterpret_cast<const char*>(a.sd_w) + int64_t(live ? r : 0) * rb;
-    } else {
-        const int64_t gr = int64_t(e) * R + (live ? r : 0);
-        rows[0] = reinterpret_cast<const char*>(a.down_w) + gr * rb;
-        if constexpr (WF == kQ4) {
-            const int64_t ng = I / a.group_size;
-            q[0] = {reinterpret_cast<const __nv_bfloat16*>(a.down_s) + gr * ng,
-                    reinterpret_cast<const __nv_bfloat16*>(a.down_z) + gr * ng};
+    const char* rows[NR];
+    QRow q[NR];
+    float bd[NR];
+    bool live[NR];
+#pragma unroll
+    for (int i = 0; i < NR; ++i) {
+        const int r = rbase + i;
+        live[i] = r < R;
+        q[i] = {nullptr, nullptr};
+        bd[i] = 0.f;
+        if (shared) {
+            rows[i] = reinterpret_cast<const char*>(a.sd_w) + int64_t(live[i] ? r : 0) * rb;
+        } else {
+            const int64_t gr = int64_t(e) * R + (live[i] ? r : 0);
+            rows[i] = reinterpret_cast<const char*>(a.down_w) + gr * rb;
+            if constexpr (WF == kQ4) {
+                const int64_t ng = I / a.group_size;
+                q[i] = {reinterpret_cast<const __nv_bfloat16*>(a.down_s) + gr * ng,
+                        reinterpret_cast<const __nv_bfloat16*>(a.down_z) + gr * ng};
+            }
+            if (a.has_bias && live[i]) bd[i] = ld_act<AT>(a.down_b, gr);
         }
-        if (a.has_bias && live) bd = ld_act<AT>(a.down_b, gr);
     }
+    const bool any = live[0];
     const void* src = shared ? a.hs : a.h;
     for (int64_t c = 0; c < cnt; c += kTT) {
         const int tt = int(cnt - c < kTT ? cnt - c : kTT);
         __syncthreads();
         stage_tokens<WF>(src, I, p0 + c, tt, nullptr, 1, us, xsum);
         __syncthreads();
-        if (!live) continue;
-        float acc[1][kTT];
+        if (!any) continue;
+        float acc[NR][kTT];
 #pragma unroll
-        for (int t = 0; t < kTT; ++t) acc[0][t] = 0.f;
-        dot_rows<WF, 1>(rows, q, I, a.group_size, us, xsum, tt, acc);
+        for (int i = 0; i < NR; ++i)
 #pragma unroll
-        for (int t = 0; t < kTT; ++t) {
-            if (t >= tt) break;
-            acc[0][t] = warp_sum(acc[0][t]);
-        }
+            for (int t = 0; t < kTT; ++t) acc[i][t] = 0.f;
+        dot_rows<WF, NR>(rows, q, I, a.group_size, us, xsum, tt, acc);
 #pragma unroll
-        for (int t = 0; t < kTT; ++t) {
-            if (t < tt && lane == t) {
-                const int64_t p = p0 + c + t;
-                if (shared) {
-                    a.s_acc[p * a.Hs + r] = acc[0][t];
-                } else {
-                    const int slot = a.sorted_slot[p];
-                    const int64_t token = slot / a.k;
-                    atomicAdd(a.y_acc + token * R + r, a.topk_w[slot] * (acc[0][t] + bd));
+        for (int i = 0; i < NR; ++i)
+#pragma unroll
+            for (int t = 0; t < kTT; ++t) {
+                if (t >= tt) break;
+                acc[i][t] = warp_sum(acc[i][t]);
+            }
+#pragma unroll
+        for (int i = 0; i < NR; ++i) {
+            if (!live[i]) continue;
+            const int r = rbase + i;
+#pragma unroll
+            for (int t = 0; t < kTT; ++t) {
+                if (t < tt && lane == t) {
+                    const int64_t p = p0 + c + t;
+                    if (shared) {
+                        a.s_acc[p * a.Hs + r] = acc[i][t];
+                    } else {
+                        const int slot = a.sorted_slot[p];
+                        const int64_t token = slot / a.k;
+                        atomicAdd(a.y_acc + token * R + r, a.topk_w[slot] * (acc[i][t] + bd[i]));
+                    }
                 }
             }
         }
@@ -332,21 +352,22 @@ __global__ void __launch_bounds__(kThreads) down_gemv_kernel(DownArgs a) {
     using AT = typename Fmt<WF>::AT;
     extern __shared__ uint4 smem_raw[];
     AT* us = reinterpret_cast<AT*>(smem_raw);
-    const int sblocks = a.shared_I ? (a.Hs + kRowsPerBlock - 1) / kRowsPerBlock : 0;
+    constexpr int NR = Fmt<WF>::DR, RR = kRowsPerBlock * NR;  // rows per warp / per block (both parts)
+    const int sblocks = a.shared_I ? (a.Hs + RR - 1) / RR : 0;
     int b = blockIdx.x;
     if (b < sblocks) {
-        down_group<WFD>(a, true, -1, b * kRowsPerBlock, 0, a.T, a.shared_I, a.Hs, us, nullptr);
+        down_group<WFD, NR>(a, true, -1, b * RR, 0, a.T, a.shared_I, a.Hs, us, nullptr);
         return;
     }
     b -= sblocks;
-    const int rblocks = (a.K + kRowsPerBlock - 1) / kRowsPerBlock;
+    const int rblocks = (a.K + RR - 1) / RR;
     const int ai = b / rblocks;
     if (ai >= a.active[0]) return;
     const int e = a.active[1 + ai];
     const int64_t p0 = a.offsets[e];
     const int64_t cnt = a.offsets[e + 1] - p0;
     float* xsum = reinterpret_cast<float*>(us + int64_t(kTT) * a.I);
-    down_group<WF>(a, false, e, (b - ai * rblocks) * kRowsPerBlock, p0, cnt, a.I, a.K, us, xsum);
+    down_group<WF, NR>(a, false, e, (b - ai * rblocks) * RR, p0, cnt, a.I, a.K, us, xsum);
 }
 
 template <typename AT>
@@ -424,8 +445,9 @@ cudaError_t launch_down_t(const DownArgs& a, cudaStream_t s) {
     const size_t smem = std::max(stage_bytes(WF, a.I), a.shared_I ? stage_bytes(WFD, a.shared_I) : size_t(0));
     cudaError_t err = set_smem(down_gemv_kernel<WF>, smem);
     if (err != cudaSuccess) return err;
-    const int64_t sblocks = a.shared_I ? (a.Hs + kRowsPerBlock - 1) / kRowsPerBlock : 0;
-    const int64_t rblocks = int64_t(a.routed_groups) * ((a.K + kRowsPerBlock - 1) / kRowsPerBlock);
+    constexpr int RR = kRowsPerBlock * Fmt<WF>::DR;
+    const int64_t sblocks = a.shared_I ? (a.Hs + RR - 1) / RR : 0;
+    const int64_t rblocks = int64_t(a.routed_groups) * ((a.K + RR - 1) / RR);
     const int64_t grid = sblocks + rblocks;
     if (grid == 0) return cudaSuccess;
     { const cudaError_t e_ = launch_pdl(down_gemv_kernel<WF>, dim3(unsigned(grid)), dim3(kThreads), smem, s, a); if (e_ != cudaSuccess) return e_; }

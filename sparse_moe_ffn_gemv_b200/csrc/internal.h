@@ -28,6 +28,10 @@ struct TopkArgs {
     const float* sel_bias = nullptr;
     int32_t* idx = nullptr; float* w = nullptr; float* coef = nullptr;
     float* zero = nullptr; int64_t zero_cols = 0;  // rows of this buffer are cleared per token
+    // T == 1 only: the warp also writes the permutation of the token's k slots (offsets
+    // [E + 1], sorted slots, their inverse, the active list and, if set, the tile prefix)
+    int32_t *p_offsets = nullptr, *p_sorted = nullptr, *p_slot_pos = nullptr, *p_active = nullptr;
+    int32_t* p_tiles = nullptr;
 };
 cudaError_t launch_topk(const TopkArgs& a, cudaStream_t s);
 

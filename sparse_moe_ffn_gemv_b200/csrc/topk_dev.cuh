@@ -40,15 +40,17 @@ __device__ __forceinline__ void topk_token(const TopkArgs& a, int64_t t) {
     const float* lg = a.logits + t * a.ld;
     const int E = a.E;
 
-    // this lane's experts: lane, lane + 32, ...
-    float l[kPerLane];
+    // this lane's experts: lane, lane + 32, ...; logits and select-only biases loaded together
+    float l[kPerLane], sb[kPerLane];
     float m = -INFINITY;
 #pragma unroll
     for (int i = 0; i < kPerLane; ++i) {
         const int e = lane + 32 * i;
         l[i] = e < E ? __ldcg(lg + e) : -INFINITY;
-        m = fmaxf(m, l[i]);
+        sb[i] = (e < E && a.has_sel) ? __ldg(a.sel_bias + e) : 0.f;
     }
+#pragma unroll
+    for (int i = 0; i < kPerLane; ++i) m = fmaxf(m, l[i]);
     float inv_sum = 1.f;
     if (a.scoring == MOE_SCORING_SOFTMAX_ALL) {
         m = warp_max(m);
@@ -68,23 +70,33 @@ __device__ __forceinline__ void topk_token(const TopkArgs& a, int64_t t) {
     for (int i = 0; i < kPerLane; ++i) {
         const int e = lane + 32 * i;
         packed[i] = 0;  // below every real key
-        if (e < E) packed[i] = pack_key(score_of(l[i]) + (a.has_sel ? a.sel_bias[e] : 0.f), e);
+        if (e < E) packed[i] = pack_key(score_of(l[i]) + sb[i], e);
     }
-    // k rounds of a warp arg-max; lane j keeps the j-th choice
+    // k rounds of a warp arg-max; lane j keeps the j-th choice and its logit (from the
+    // registers of the lane that owns the expert)
     int my_e = -1;
+    float my_l = -INFINITY;
     for (int j = 0; j < a.k; ++j) {
         uint64_t best = 0;
 #pragma unroll
         for (int i = 0; i < kPerLane; ++i) best = packed[i] > best ? packed[i] : best;
         best = warp_max_u64(best);
+        float won = 0.f;
 #pragma unroll
         for (int i = 0; i < kPerLane; ++i)
-            if (packed[i] == best) packed[i] = 0;
-        if (lane == j) my_e = int(0xFFFFFFFFu - uint32_t(best & 0xFFFFFFFFu));
+            if (packed[i] == best) {
+                packed[i] = 0;
+                won = l[i];
+            }
+        const int e = int(0xFFFFFFFFu - uint32_t(best & 0xFFFFFFFFu));
+        won = __shfl_sync(0xffffffffu, won, e & 31);
+        if (lane == j) {
+            my_e = e;
+            my_l = won;
+        }
     }
     // combine weights: unbiased scores of the chosen experts, or softmax over their logits
     const bool mine = lane < a.k;
-    const float my_l = mine ? __ldcg(lg + my_e) : -INFINITY;
     float w;
     if (a.scoring == MOE_SCORING_SOFTMAX_TOPK) {
         const float mm = warp_max(my_l);
@@ -104,6 +116,29 @@ __device__ __forceinline__ void topk_token(const TopkArgs& a, int64_t t) {
         const float e0 = expf(c0 - cm), e1 = expf(c1 - cm);
         a.coef[t * 2 + 0] = e0 / (e0 + e1);
         a.coef[t * 2 + 1] = e1 / (e0 + e1);
+    }
+    if (a.p_offsets) {
+        // One token (t == 0): its k slots sorted by expert. The experts of a token's top-k
+        // are distinct, so a slot's rank is the number of chosen experts below its own.
+        int ek[kMaxTopK];
+#pragma unroll
+        for (int q = 0; q < kMaxTopK; ++q) ek[q] = q < a.k ? __shfl_sync(0xffffffffu, my_e, q) : 0x7fffffff;
+        if (mine) {
+            int rank = 0;
+#pragma unroll
+            for (int q = 0; q < kMaxTopK; ++q) rank += ek[q] < my_e ? 1 : 0;
+            a.p_sorted[rank] = lane;
+            a.p_slot_pos[lane] = rank;
+            a.p_active[1 + rank] = my_e;
+        }
+        for (int e = lane; e <= a.E; e += 32) {
+            int below = 0;
+#pragma unroll
+            for (int q = 0; q < kMaxTopK; ++q) below += ek[q] < e ? 1 : 0;
+            a.p_offsets[e] = below;
+            if (a.p_tiles) a.p_tiles[e] = below;  // one token per active expert: one tile each
+        }
+        if (lane == 0) a.p_active[0] = a.k;
     }
     if (a.zero) {
         float4* z = reinterpret_cast<float4*>(a.zero + t * a.zero_cols);
