@@ -50,7 +50,7 @@ WsLayout ws_layout(const moe_config& c, int64_t T) {
     L.s_acc = take(c.shared_mode != MOE_SHARED_NONE ? T * H * 4 : 0);
     L.z = take(Ld ? T * Ld * ab : 0);
     L.nrm = take(Ld ? T * Ld * ab : 0);
-    const bool tc = c.act_dtype == MOE_DTYPE_BF16 && c.weight_format == MOE_DTYPE_BF16;
+    const bool tc = c.act_dtype == MOE_DTYPE_BF16;  // bf16 or 4-bit weights
     L.uperm = take(tc ? T * k * K * 2 : 0);
     L.oslot = take(tc ? T * k * K * 2 : 0);
     L.tiles = take((E + 1) * 4);
@@ -183,7 +183,7 @@ bool dense_tc(const moe_config* c, int64_t T, int K) {
 // kernels from there on, although most tiles then hold only a few tokens (Klear shape:
 // 8 tokens 149 vs 157 us, 64 tokens 279 vs 627 us; at 4 tokens the CUDA cores win).
 bool routed_tc(const moe_config* c, int64_t T) {
-    if (c->act_dtype != MOE_DTYPE_BF16 || c->weight_format != MOE_DTYPE_BF16) return false;
+    if (c->act_dtype != MOE_DTYPE_BF16 || c->weight_format == MOE_DTYPE_F32) return false;
     if (expert_in(*c) % 64 != 0 || c->intermediate % 64 != 0) return false;
     const int o = path_override();
     return o == kPathTc || (o == kPathAuto && 4 * T * c->top_k >= int64_t(c->num_experts));
@@ -378,7 +378,12 @@ moe_status run_experts_tc(const moe_config* c, const moe_weights* w, const void*
                 }
             }
             bool ok;
-            if (c->gate_up_interleaved) {
+            if (c->weight_format == MOE_DTYPE_Q4_AFFINE) {  // dequantised in the main loop
+                p.q4 = 1;
+                p.group_size = c->group_size;
+                p.qs0 = w->gate_s; p.qz0 = w->gate_z; p.qs1 = w->up_s; p.qz1 = w->up_z;
+                ok = tc_q4_weight_map(&P.a0[np], w->gate_w, E, I, K) && tc_q4_weight_map(&P.a1[np], w->up_w, E, I, K);
+            } else if (c->gate_up_interleaved) {
                 ok = tc_weight_map(&P.a0[np], w->gate_up_w, E, I, K, true);
             } else {
                 ok = tc_weight_map(&P.a0[np], w->gate_w, E, I, K, false) &&
@@ -419,8 +424,16 @@ moe_status run_experts_tc(const moe_config* c, const moe_weights* w, const void*
             p.sorted_slot = sorted_slot; p.topk_w = topk_w; p.k = k;
             p.bias0 = c->has_expert_bias ? w->down_b : nullptr;
             p.out = at<__nv_bfloat16>(ws, L.oslot); p.ld_out = K;
-            if (!tc_weight_map(&P.a0[np], w->down_w, E, K, I, false) || !tc_token_map(&P.b[np], h, S, I, kTcBN))
-                return MOE_ERR_CUDA;
+            bool ok;
+            if (c->weight_format == MOE_DTYPE_Q4_AFFINE) {
+                p.q4 = 1;
+                p.group_size = c->group_size;
+                p.qs0 = w->down_s; p.qz0 = w->down_z;
+                ok = tc_q4_weight_map(&P.a0[np], w->down_w, E, K, I);
+            } else {
+                ok = tc_weight_map(&P.a0[np], w->down_w, E, K, I, false);
+            }
+            if (!ok || !tc_token_map(&P.b[np], h, S, I, kTcBN)) return MOE_ERR_CUDA;
             max_tiles += int64_t(p.m_blocks) * max_routed_tiles(*c, T);
             ++np;
         }

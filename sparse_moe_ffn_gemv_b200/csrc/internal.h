@@ -118,6 +118,10 @@ struct TcProblem {
     int bias_interleaved = 0, interleaved = 0;
     void* out = nullptr; int ld_out = 0;
     const float* addend = nullptr; int ld_add = 0;
+    // 4-bit affine weights (tc_q4_weight_map planes): bf16 scales / biases [groups, M, K / group_size]
+    // of the first (gate or single) and second (up) weight plane
+    int q4 = 0, group_size = 64;
+    const void *qs0 = nullptr, *qz0 = nullptr, *qs1 = nullptr, *qz1 = nullptr;
 };
 
 struct alignas(64) TcParams {
@@ -137,6 +141,9 @@ struct alignas(64) TcParams {
 };
 
 bool tc_weight_map(CUtensorMap* m, const void* w, int E, int R, int K, bool interleaved);
+// Packed 4-bit weight operand: [E, R, K / 8] uint32 words (8 codes each), one 64-wide K block
+// (8 words) x 128 rows per box, no swizzle (the kernel's dequantising warps read it).
+bool tc_q4_weight_map(CUtensorMap* m, const void* w, int E, int R, int K);
 bool tc_token_map(CUtensorMap* m, const void* u, int64_t rows, int K, int bn);
 cudaError_t launch_tc_gemm(TcParams& P, bool gateup, int64_t max_tiles, cudaStream_t s);
 

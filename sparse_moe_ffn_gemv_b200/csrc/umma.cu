@@ -11,7 +11,11 @@
 //               TMEM; two accumulators (gate, up) in gate/up mode
 //   warps 2..9  epilogue (two warps per TMEM lane quarter, each half of the columns):
 //               tcgen05.ld, then SwiGLU / clamped SwiGLU -> bf16 h (gate/up),
-//               the weighted fp32 output row of every slot (down), or a plain store
+//               the weighted bf16 output row of every slot (down), or a plain store
+//   warps 10..13 (4-bit weights only) dequantisation: the producer loads the packed words,
+//               these warps write w = scale * q + bias as bf16 into the swizzled operand
+//               layout the MMA reads (mlxcel issue #974: affine 4-bit, per-group scale
+//               and bias), one K block ahead of the MMA
 // TMEM holds two accumulator sets so the epilogue of one tile overlaps the main loop of
 // the next. Every mbarrier wait is bounded by %globaltimer; a wait that gives up records
 // MOE_ERR_DEVICE_TIMEOUT in the status word, drains its own outstanding copies / MMAs and
@@ -34,7 +38,9 @@ namespace {
 constexpr int kBM = 128;          // weight rows per MMA (M)
 constexpr int kBK = 64;           // K per stage: one 128-byte swizzle atom of bf16
 constexpr int kTcThreads = 320;   // 10 warps: TMA, MMA, 8 epilogue
+constexpr int kDqThreads = 128;   // + 4 dequantising warps for 4-bit weights
 constexpr int kEpiThreads = 256;
+constexpr int kPkBytes = kBM * kBK / 2;  // packed 4-bit weight tile: 128 rows x 32 bytes
 constexpr int kMaxGroups = 512;   // expert groups whose tile table fits in shared memory
 constexpr uint64_t kWaitNs = 2000000000ull;  // 2 s bound on any single wait
 
@@ -152,11 +158,14 @@ __device__ __forceinline__ TileInfo decode_tile(const TcParams& P, const GroupTa
 
 // Every tile carries two 128-row weight operands that share one token tile: the gate and
 // up rows of 128 intermediate units (gate/up), or 256 consecutive output rows (others).
-template <bool GATEUP, int BN, int STAGES>
+// With 4-bit weights a stage also holds the two packed tiles after the bf16 operands.
+template <bool GATEUP, int BN, int STAGES, bool Q4 = false>
 struct TcShape {
     static constexpr int A_BYTES = kBM * kBK * 2;                // 16 KB
     static constexpr int B_BYTES = BN * kBK * 2;
-    static constexpr int STAGE_BYTES = 2 * A_BYTES + B_BYTES;
+    static constexpr int PK_OFF = 2 * A_BYTES + B_BYTES;         // packed tiles (4-bit only)
+    static constexpr int STAGE_BYTES = 2 * A_BYTES + B_BYTES + (Q4 ? 2 * kPkBytes : 0);
+    static constexpr int THREADS = kTcThreads + (Q4 ? kDqThreads : 0);
     static constexpr int ACC_COLS = 2 * BN;                      // per accumulator set
     static constexpr int TMEM_COLS = 2 * ACC_COLS;               // double-buffered
     static constexpr int ROWS = GATEUP ? kBM : 2 * kBM;          // weight rows per tile
@@ -178,9 +187,40 @@ __device__ __forceinline__ float bf16_at(const void* p, int64_t i) {
     return __bfloat162float(reinterpret_cast<const __nv_bfloat16*>(p)[i]);
 }
 
-template <bool GATEUP, int BN, int STAGES>
-__global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_constant__ TcParams P) {
-    using S = TcShape<GATEUP, BN, STAGES>;
+// Eight 4-bit codes (element j in bits 4j..4j+3 of the word) -> eight bf16 weights
+// w = s * q + b, one rounding each. A code q becomes the exact bf16 128 + q by OR-ing it into
+// the mantissa of 128.0 (two codes per 32-bit pair: the pair (q_i, q_i+4) comes from the
+// same nibble position of both halves), PRMT puts neighbours together, and q = (128 + q) -
+// 128 is exact in bf16 before the single-rounding fma.
+__device__ __forceinline__ uint4 dequant8(uint32_t w, __nv_bfloat162 s2, __nv_bfloat162 b2) {
+    const uint32_t p0 = (w & 0x000F000Fu) | 0x43004300u;          // (q0, q4)
+    const uint32_t p1 = ((w >> 4) & 0x000F000Fu) | 0x43004300u;   // (q1, q5)
+    const uint32_t p2 = ((w >> 8) & 0x000F000Fu) | 0x43004300u;   // (q2, q6)
+    const uint32_t p3 = ((w >> 12) & 0x000F000Fu) | 0x43004300u;  // (q3, q7)
+    const uint32_t o[4] = {__byte_perm(p0, p1, 0x5410), __byte_perm(p2, p3, 0x5410),
+                           __byte_perm(p0, p1, 0x7632), __byte_perm(p2, p3, 0x7632)};
+    const __nv_bfloat162 off = __floats2bfloat162_rn(128.0f, 128.0f);
+    uint32_t r[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const __nv_bfloat162 q = __hsub2(*reinterpret_cast<const __nv_bfloat162*>(&o[i]), off);
+        const __nv_bfloat162 v = __hfma2(q, s2, b2);
+        r[i] = *reinterpret_cast<const uint32_t*>(&v);
+    }
+    return make_uint4(r[0], r[1], r[2], r[3]);
+}
+
+// Byte offset of row r's 16-byte chunk c (8 bf16 of one 64-wide K block) in a 128-row
+// operand tile with the 128-byte swizzle the MMA descriptor expects (8-row atoms of 1 KB,
+// chunk index XOR row within the atom).
+__device__ __forceinline__ uint32_t sw128_offset(int r, int c) {
+    return uint32_t((r >> 3) * 1024 + (r & 7) * 128 + ((c ^ (r & 7)) << 4));
+}
+
+template <bool GATEUP, int BN, int STAGES, bool Q4>
+__global__ void __launch_bounds__(TcShape<GATEUP, BN, STAGES, Q4>::THREADS, 1)
+    tc_gemm_kernel(const __grid_constant__ TcParams P) {
+    using S = TcShape<GATEUP, BN, STAGES, Q4>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint64_t* full = reinterpret_cast<uint64_t*>(smem + STAGES * S::STAGE_BYTES);
@@ -188,7 +228,8 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
     uint64_t* acc_full = empty + STAGES;
     uint64_t* acc_empty = acc_full + 2;
     uint64_t* drain = acc_empty + 2;
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+    uint64_t* dq = drain + 1;  // 4-bit: stage dequantised (STAGES barriers)
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(dq + STAGES);
     GroupTables& gt = *reinterpret_cast<GroupTables*>(smem + STAGES * S::STAGE_BYTES + 256);
     __nv_bfloat16** e_row = reinterpret_cast<__nv_bfloat16**>(&gt + 1);  // output row of each token column
     float* e_w = reinterpret_cast<float*>(e_row + BN);
@@ -209,6 +250,8 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
             mbar_init(&acc_empty[b], kEpiThreads / 32);  // one arrive per epilogue warp
         }
         mbar_init(drain, 1);
+        if (Q4)
+            for (int st = 0; st < STAGES; ++st) mbar_init(&dq[st], kDqThreads / 32);  // one arrive per warp
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
         asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
     }
@@ -254,16 +297,28 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
                         break;
                     }
                     uint8_t* sb = smem + stage * S::STAGE_BYTES;
-                    mbar_expect_tx(&full[stage], S::STAGE_BYTES);
                     const int kc = kb * kBK;
                     const int mrow = ti.mb * S::ROWS;
-                    if (!GATEUP) {  // rows [mrow, mrow + 128) and [mrow + 128, mrow + 256)
+                    if (Q4 && p.q4) {  // packed words of the two weight tiles (8 words per K block)
+                        mbar_expect_tx(&full[stage], 2 * kPkBytes + S::B_BYTES);
+                        uint8_t* pk = sb + S::PK_OFF;
+                        if (!GATEUP) {
+                            tma_3d(pk, &P.a0[ti.prob], &full[stage], kb * 8, mrow, ti.group, pol_w);
+                            tma_3d(pk + kPkBytes, &P.a0[ti.prob], &full[stage], kb * 8, mrow + kBM, ti.group, pol_w);
+                        } else {
+                            tma_3d(pk, &P.a0[ti.prob], &full[stage], kb * 8, mrow, ti.group, pol_w);
+                            tma_3d(pk + kPkBytes, &P.a1[ti.prob], &full[stage], kb * 8, mrow, ti.group, pol_w);
+                        }
+                    } else if (!GATEUP) {  // rows [mrow, mrow + 128) and [mrow + 128, mrow + 256)
+                        mbar_expect_tx(&full[stage], 2 * S::A_BYTES + S::B_BYTES);
                         tma_3d(sb, &P.a0[ti.prob], &full[stage], kc, mrow, ti.group, pol_w);
                         tma_3d(sb + S::A_BYTES, &P.a0[ti.prob], &full[stage], kc, mrow + kBM, ti.group, pol_w);
                     } else if (p.interleaved) {  // [E, I, 2, K]: plane 0 = gate rows, 1 = up rows
+                        mbar_expect_tx(&full[stage], 2 * S::A_BYTES + S::B_BYTES);
                         tma_4d(sb, &P.a0[ti.prob], &full[stage], kc, 0, mrow, ti.group, pol_w);
                         tma_4d(sb + S::A_BYTES, &P.a0[ti.prob], &full[stage], kc, 1, mrow, ti.group, pol_w);
                     } else {
+                        mbar_expect_tx(&full[stage], 2 * S::A_BYTES + S::B_BYTES);
                         tma_3d(sb, &P.a0[ti.prob], &full[stage], kc, mrow, ti.group, pol_w);
                         tma_3d(sb + S::A_BYTES, &P.a1[ti.prob], &full[stage], kc, mrow, ti.group, pol_w);
                     }
@@ -302,7 +357,9 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
                 const uint32_t idesc = idesc_base | ((n_mma >> 3) << 17);
                 const int nk = p.K / kBK;
                 for (int kb = 0; kb < nk; ++kb) {
-                    if (!mbar_wait(&full[stage], phase, deadline)) {
+                    // with 4-bit weights in the kernel every stage passes through the
+                    // dequantising warps (which only forward bf16 stages)
+                    if (!mbar_wait(Q4 ? &dq[stage] : &full[stage], phase, deadline)) {
                         timed_out = true;
                         break;
                     }
@@ -330,6 +387,89 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
             mbar_wait(drain, 0, gtimer() + kWaitNs);
             if (timed_out) set_status(P.status, MOE_ERR_DEVICE_TIMEOUT);
         }
+    } else if (Q4 && warp >= kTcThreads / 32) {
+        // ---------------------------------------------------------- dequantisation (128 threads)
+        // Thread d takes 16-byte chunk c = d % 8 (K elements 8c..8c+7 of the block) of rows
+        // d / 8 + 16 i (i < 8) of both weight tiles; its 16 scale / bias pairs for the next K
+        // block are loaded while the current block is dequantised.
+        const int d = threadIdx.x - kTcThreads;
+        const int c = d & 7, r0 = d >> 3;
+        uint32_t stage = 0, phase = 0;
+        for (int tile = blockIdx.x; tile < total && !timed_out; tile += gridDim.x) {
+            const TileInfo ti = decode_tile(P, gt, tile, t0);
+            const TcProblem& p = P.p[ti.prob];
+            const int nk = p.K / kBK;
+            if (!p.q4) {  // bf16 tile: the stage goes straight on to the MMA
+                for (int kb = 0; kb < nk; ++kb) {
+                    if (!mbar_wait(&full[stage], phase, deadline)) {
+                        timed_out = true;
+                        break;
+                    }
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&dq[stage]);
+                    if (++stage == STAGES) {
+                        stage = 0;
+                        phase ^= 1u;
+                    }
+                }
+                continue;
+            }
+            const int ng = p.K / p.group_size;
+            // scale / bias planes of the two weight tiles (this group), this thread's 16 row
+            // offsets in them (rows past M read row M - 1: their results are discarded), and
+            // the (scale, bias) pair of each row for the current and the next K block
+            const int64_t gbase = int64_t(ti.group) * p.M * ng;
+            const __nv_bfloat16* sp[2] = {static_cast<const __nv_bfloat16*>(p.qs0) + gbase,
+                                          static_cast<const __nv_bfloat16*>(GATEUP ? p.qs1 : p.qs0) + gbase};
+            const __nv_bfloat16* zp[2] = {static_cast<const __nv_bfloat16*>(p.qz0) + gbase,
+                                          static_cast<const __nv_bfloat16*>(GATEUP ? p.qz1 : p.qz0) + gbase};
+            int roff[16];
+#pragma unroll
+            for (int a = 0; a < 2; ++a)
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                    const int r = ti.mb * S::ROWS + (GATEUP ? 0 : a * kBM) + r0 + 16 * i;
+                    roff[a * 8 + i] = min(r, p.M - 1) * ng;
+                }
+            auto load_sb = [&](int kb, __nv_bfloat162 (&out)[16]) {
+                const int g = (kb * kBK + 8 * c) / p.group_size;
+#pragma unroll
+                for (int i = 0; i < 16; ++i)
+                    out[i] = __halves2bfloat162(__ldg(sp[i >> 3] + roff[i] + g), __ldg(zp[i >> 3] + roff[i] + g));
+            };
+            __nv_bfloat162 sbc[16];
+            load_sb(0, sbc);
+            for (int kb = 0; kb < nk; ++kb) {
+                __nv_bfloat162 sbn[16];
+                if (kb + 1 < nk) load_sb(kb + 1, sbn);
+                if (!mbar_wait(&full[stage], phase, deadline)) {
+                    timed_out = true;
+                    break;
+                }
+                uint8_t* sb = smem + stage * S::STAGE_BYTES;
+                const uint32_t* pk = reinterpret_cast<const uint32_t*>(sb + S::PK_OFF);
+#pragma unroll
+                for (int a = 0; a < 2; ++a)
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) {
+                        const int r = r0 + 16 * i;
+                        const uint32_t w = pk[a * (kPkBytes / 4) + r * 8 + c];
+                        const uint4 v = dequant8(w, __low2bfloat162(sbc[a * 8 + i]), __high2bfloat162(sbc[a * 8 + i]));
+                        *reinterpret_cast<uint4*>(sb + a * S::A_BYTES + sw128_offset(r, c)) = v;
+                    }
+                // generic-proxy writes, read next by the tensor cores (async proxy)
+                asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&dq[stage]);
+#pragma unroll
+                for (int i = 0; i < 16; ++i) sbc[i] = sbn[i];
+                if (++stage == STAGES) {
+                    stage = 0;
+                    phase ^= 1u;
+                }
+            }
+        }
+        if (timed_out) set_status(P.status, MOE_ERR_DEVICE_TIMEOUT);
     } else {
         // -------------------------------------------------------------- epilogue (256 threads)
         const int q = warp & 3;                  // TMEM lane quarter of this warp
@@ -405,56 +545,76 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
                     }
                 }
             } else {
-                // two 128-row accumulators x this warp's 64 token columns, all in registers
-                uint32_t v[4][32];
-                tmem_ld_issue(tb + c_lo, v[0]);
-                tmem_ld_issue(tb + c_lo + 32, v[1]);
-                tmem_ld_issue(tb + BN + c_lo, v[2]);
-                tmem_ld_issue(tb + BN + c_lo + 32, v[3]);
-                tmem_ld_wait(v[0]);
-                tmem_ld_wait(v[1]);
-                tmem_ld_wait(v[2]);
-                tmem_ld_wait(v[3]);
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&acc_empty[ab]);
+                // two 128-row accumulators x this warp's 64 token columns
                 const bool full_tile = ti.nvalid >= c_lo + 64;
-#pragma unroll
-                for (int a = 0; a < 2; ++a) {
+                const int nend = full_tile ? 64 : max(0, ti.nvalid - c_lo);
+                auto store_acc = [&](int a, const uint32_t (&va)[2][32]) {
                     const int r = ti.mb * S::ROWS + a * kBM + lrow;
-                    if (r >= p.M) continue;
+                    if (r >= p.M) return;
                     const float bias0 = p.bias0 ? bf16_at(p.bias0, int64_t(ti.group) * p.M + r) : 0.f;
-                    const int nend = full_tile ? 64 : max(0, ti.nvalid - c_lo);
                     if (p.mode == kEpiSlotRows) {
                         // weighted output row of each slot (bf16); the combine sums a token's k rows
                         if (full_tile) {
 #pragma unroll
                             for (int j = 0; j < 64; ++j)
                                 e_row[c_lo + j][r] =
-                                    __float2bfloat16_rn(e_w[c_lo + j] * (__uint_as_float(v[a * 2 + j / 32][j % 32]) + bias0));
+                                    __float2bfloat16_rn(e_w[c_lo + j] * (__uint_as_float(va[j / 32][j % 32]) + bias0));
                         } else {
 #pragma unroll
                             for (int j = 0; j < 64; ++j)
                                 if (j < nend)
                                     e_row[c_lo + j][r] = __float2bfloat16_rn(
-                                        e_w[c_lo + j] * (__uint_as_float(v[a * 2 + j / 32][j % 32]) + bias0));
+                                        e_w[c_lo + j] * (__uint_as_float(va[j / 32][j % 32]) + bias0));
                         }
                     } else if (p.mode == kEpiStoreF32) {
                         float* o = reinterpret_cast<float*>(p.out) + int64_t(ti.row0 + c_lo) * p.ld_out + r;
 #pragma unroll
                         for (int j = 0; j < 64; ++j)
-                            if (j < nend) o[int64_t(j) * p.ld_out] = __uint_as_float(v[a * 2 + j / 32][j % 32]) + bias0;
+                            if (j < nend) o[int64_t(j) * p.ld_out] = __uint_as_float(va[j / 32][j % 32]) + bias0;
                     } else {  // kEpiStoreAct (+ optional fp32 addend)
                         __nv_bfloat16* o = reinterpret_cast<__nv_bfloat16*>(p.out) + int64_t(ti.row0 + c_lo) * p.ld_out + r;
                         const float* ad = p.addend ? p.addend + int64_t(ti.row0 + c_lo) * p.ld_add + r : nullptr;
 #pragma unroll
                         for (int j = 0; j < 64; ++j) {
                             if (j < nend) {
-                                float d = __uint_as_float(v[a * 2 + j / 32][j % 32]) + bias0;
+                                float d = __uint_as_float(va[j / 32][j % 32]) + bias0;
                                 if (ad) d += ad[int64_t(j) * p.ld_add];
                                 o[int64_t(j) * p.ld_out] = __float2bfloat16_rn(d);
                             }
                         }
+                    }
+                };
+                if constexpr (!Q4) {
+                    // both accumulators in registers, the TMEM set released before any store
+                    uint32_t v[2][2][32];
+                    tmem_ld_issue(tb + c_lo, v[0][0]);
+                    tmem_ld_issue(tb + c_lo + 32, v[0][1]);
+                    tmem_ld_issue(tb + BN + c_lo, v[1][0]);
+                    tmem_ld_issue(tb + BN + c_lo + 32, v[1][1]);
+                    tmem_ld_wait(v[0][0]);
+                    tmem_ld_wait(v[0][1]);
+                    tmem_ld_wait(v[1][0]);
+                    tmem_ld_wait(v[1][1]);
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&acc_empty[ab]);
+                    store_acc(0, v[0]);
+                    store_acc(1, v[1]);
+                } else {
+                    // with the dequantising warps' share of the registers, one accumulator at a time
+#pragma unroll 1
+                    for (int a = 0; a < 2; ++a) {
+                        uint32_t v[2][32];
+                        tmem_ld_issue(tb + a * BN + c_lo, v[0]);
+                        tmem_ld_issue(tb + a * BN + c_lo + 32, v[1]);
+                        tmem_ld_wait(v[0]);
+                        tmem_ld_wait(v[1]);
+                        if (a == 1) {
+                            tc_fence_before();
+                            __syncwarp();
+                            if (lane == 0) mbar_arrive(&acc_empty[ab]);
+                        }
+                        store_acc(a, v);
                     }
                 }
             }
@@ -488,12 +648,13 @@ EncodeFn encode_fn() {
 }
 
 bool encode(CUtensorMap* m, const void* base, int rank, const cuuint64_t* dims, const cuuint64_t* strides,
-            const cuuint32_t* box) {
+            const cuuint32_t* box, CUtensorMapDataType type = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16,
+            CUtensorMapSwizzle swizzle = CU_TENSOR_MAP_SWIZZLE_128B) {
     EncodeFn fn = encode_fn();
     if (!fn) return false;
     cuuint32_t es[5] = {1, 1, 1, 1, 1};
-    return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, cuuint32_t(rank), const_cast<void*>(base), dims, strides, box,
-              es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+    return fn(m, type, cuuint32_t(rank), const_cast<void*>(base), dims, strides, box, es,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
@@ -503,15 +664,15 @@ int sm_count() {
     return n;
 }
 
-template <bool GATEUP, int BN, int STAGES>
+template <bool GATEUP, int BN, int STAGES, bool Q4>
 cudaError_t launch_tc_t(TcParams& P, int64_t max_tiles, cudaStream_t s) {
-    using S = TcShape<GATEUP, BN, STAGES>;
-    auto kern = tc_gemm_kernel<GATEUP, BN, STAGES>;
+    using S = TcShape<GATEUP, BN, STAGES, Q4>;
+    auto kern = tc_gemm_kernel<GATEUP, BN, STAGES, Q4>;
     cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, S::SMEM);
     if (err != cudaSuccess) return err;
     const int grid = int(std::min<int64_t>(max_tiles, sm_count()));
     if (grid <= 0) return cudaSuccess;
-    { const cudaError_t e_ = launch_pdl(kern, dim3(grid), dim3(kTcThreads), S::SMEM, s, P); if (e_ != cudaSuccess) return e_; }
+    { const cudaError_t e_ = launch_pdl(kern, dim3(grid), dim3(S::THREADS), S::SMEM, s, P); if (e_ != cudaSuccess) return e_; }
     return cudaGetLastError();
 }
 
@@ -540,9 +701,23 @@ bool tc_token_map(CUtensorMap* m, const void* u, int64_t rows, int K, int bn) {
     return encode(m, u, 2, dims, strides, box);
 }
 
+// Packed 4-bit plane [E, R, K / 8] uint32 (K % 64 == 0): box of 8 words x 128 rows.
+bool tc_q4_weight_map(CUtensorMap* m, const void* w, int E, int R, int K) {
+    const cuuint64_t dims[3] = {cuuint64_t(K / 8), cuuint64_t(R), cuuint64_t(E)};
+    const cuuint64_t strides[2] = {cuuint64_t(K / 8) * 4, cuuint64_t(R) * (K / 8) * 4};
+    const cuuint32_t box[3] = {8, kBM, 1};
+    return encode(m, w, 3, dims, strides, box, CU_TENSOR_MAP_DATA_TYPE_UINT32, CU_TENSOR_MAP_SWIZZLE_NONE);
+}
+
 cudaError_t launch_tc_gemm(TcParams& P, bool gateup, int64_t max_tiles, cudaStream_t s) {
-    if (gateup) return launch_tc_t<true, kTcBN, 4>(P, max_tiles, s);
-    return launch_tc_t<false, kTcBN, 4>(P, max_tiles, s);
+    bool q4 = false;
+    for (int i = 0; i < P.nprob; ++i) q4 = q4 || P.p[i].q4;
+    if (q4) {  // a stage also holds the packed tiles: three stages fit
+        if (gateup) return launch_tc_t<true, kTcBN, 3, true>(P, max_tiles, s);
+        return launch_tc_t<false, kTcBN, 3, true>(P, max_tiles, s);
+    }
+    if (gateup) return launch_tc_t<true, kTcBN, 4, false>(P, max_tiles, s);
+    return launch_tc_t<false, kTcBN, 4, false>(P, max_tiles, s);
 }
 
 }  // namespace moe

@@ -227,11 +227,13 @@ def test_batch_equals_tokens_one_at_a_time_on_gpu():
     assert blk.device_status() == 0
 
 
-TC_SMALL = [  # tensor-core path forced: ragged groups, partial tiles, interleaved + biases, latent
-    (inputs.KLEAR_BF16, 37),
+TC_SMALL = [  # tensor-core path forced: ragged groups, partial tiles, interleaved + biases, latent,
+    (inputs.KLEAR_BF16, 37),   # 4-bit weights dequantised in the main loop
     (inputs.KLEAR_BF16, 200),
     (inputs.CLAMPED_BF16, 40),
     (inputs.LATENT_BF16, 9),
+    (inputs.KLEAR_Q4, 3),
+    (inputs.KLEAR_Q4, 150),
 ]
 
 
@@ -242,7 +244,8 @@ def test_tensor_core_path_matches_oracle(spec, T, monkeypatch):
 
 
 @pytest.mark.parametrize("spec,T", [(inputs.KLEAR_BF16, 96), (inputs.CLAMPED_BF16, 64),
-                                    (inputs.LATENT_BF16, 64)], ids=["klear", "clamped", "latent"])
+                                    (inputs.LATENT_BF16, 64), (inputs.KLEAR_Q4, 96)],
+                         ids=["klear", "clamped", "latent", "klear_q4"])
 def test_weight_streaming_and_tensor_core_paths_agree(spec, T, monkeypatch):
     """The decode-sized engine and the batched engine give the same block output
     (cf. the Klear PR's caveat on a fused decode kernel that was not byte-identical)."""
