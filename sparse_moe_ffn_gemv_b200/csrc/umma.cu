@@ -389,11 +389,10 @@ __global__ void __launch_bounds__(TcShape<GATEUP, BN, STAGES, Q4>::THREADS, 1)
         }
     } else if (Q4 && warp >= kTcThreads / 32) {
         // ---------------------------------------------------------- dequantisation (128 threads)
-        // Thread d takes 16-byte chunk c = d % 8 (K elements 8c..8c+7 of the block) of rows
-        // d / 8 + 16 i (i < 8) of both weight tiles; its 16 scale / bias pairs for the next K
-        // block are loaded while the current block is dequantised.
+        // Thread d dequantises row d of both weight tiles (all 64 K elements of the block:
+        // two 16-byte loads of packed words, eight swizzled 16-byte stores per row). Its
+        // (scale, bias) pairs are loaded two K blocks ahead.
         const int d = threadIdx.x - kTcThreads;
-        const int c = d & 7, r0 = d >> 3;
         uint32_t stage = 0, phase = 0;
         for (int tile = blockIdx.x; tile < total && !timed_out; tile += gridDim.x) {
             const TileInfo ti = decode_tile(P, gt, tile, t0);
@@ -415,54 +414,62 @@ __global__ void __launch_bounds__(TcShape<GATEUP, BN, STAGES, Q4>::THREADS, 1)
                 continue;
             }
             const int ng = p.K / p.group_size;
-            // scale / bias planes of the two weight tiles (this group), this thread's 16 row
-            // offsets in them (rows past M read row M - 1: their results are discarded), and
-            // the (scale, bias) pair of each row for the current and the next K block
-            const int64_t gbase = int64_t(ti.group) * p.M * ng;
-            const __nv_bfloat16* sp[2] = {static_cast<const __nv_bfloat16*>(p.qs0) + gbase,
-                                          static_cast<const __nv_bfloat16*>(GATEUP ? p.qs1 : p.qs0) + gbase};
-            const __nv_bfloat16* zp[2] = {static_cast<const __nv_bfloat16*>(p.qz0) + gbase,
-                                          static_cast<const __nv_bfloat16*>(GATEUP ? p.qz1 : p.qz0) + gbase};
-            int roff[16];
+            // this thread's row of each weight tile in its scale / bias planes (rows past M
+            // read row M - 1: their results are discarded)
+            const __nv_bfloat16* sp[2];
+            const __nv_bfloat16* zp[2];
 #pragma unroll
-            for (int a = 0; a < 2; ++a)
+            for (int a = 0; a < 2; ++a) {
+                const int r = min(ti.mb * S::ROWS + (GATEUP ? 0 : a * kBM) + d, p.M - 1);
+                const int64_t off = (int64_t(ti.group) * p.M + r) * ng;
+                sp[a] = static_cast<const __nv_bfloat16*>((GATEUP && a == 1) ? p.qs1 : p.qs0) + off;
+                zp[a] = static_cast<const __nv_bfloat16*>((GATEUP && a == 1) ? p.qz1 : p.qz0) + off;
+            }
+            // (scale, bias) of tile a for the first and second half of K block kb (two
+            // groups per block when group_size is 32, else the same group twice)
+            auto load_sb = [&](int kb, __nv_bfloat162 (&o)[2][2]) {
 #pragma unroll
-                for (int i = 0; i < 8; ++i) {
-                    const int r = ti.mb * S::ROWS + (GATEUP ? 0 : a * kBM) + r0 + 16 * i;
-                    roff[a * 8 + i] = min(r, p.M - 1) * ng;
-                }
-            auto load_sb = [&](int kb, __nv_bfloat162 (&out)[16]) {
-                const int g = (kb * kBK + 8 * c) / p.group_size;
+                for (int a = 0; a < 2; ++a)
 #pragma unroll
-                for (int i = 0; i < 16; ++i)
-                    out[i] = __halves2bfloat162(__ldg(sp[i >> 3] + roff[i] + g), __ldg(zp[i >> 3] + roff[i] + g));
+                    for (int h = 0; h < 2; ++h) {
+                        const int g = (kb * kBK + h * 32) / p.group_size;
+                        o[a][h] = __halves2bfloat162(__ldg(sp[a] + g), __ldg(zp[a] + g));
+                    }
             };
-            __nv_bfloat162 sbc[16];
-            load_sb(0, sbc);
+            __nv_bfloat162 q0[2][2], q1[2][2];
+            load_sb(0, q0);
+            if (nk > 1) load_sb(1, q1);
             for (int kb = 0; kb < nk; ++kb) {
-                __nv_bfloat162 sbn[16];
-                if (kb + 1 < nk) load_sb(kb + 1, sbn);
+                __nv_bfloat162 q2[2][2];
+                if (kb + 2 < nk) load_sb(kb + 2, q2);
                 if (!mbar_wait(&full[stage], phase, deadline)) {
                     timed_out = true;
                     break;
                 }
                 uint8_t* sb = smem + stage * S::STAGE_BYTES;
-                const uint32_t* pk = reinterpret_cast<const uint32_t*>(sb + S::PK_OFF);
 #pragma unroll
-                for (int a = 0; a < 2; ++a)
+                for (int a = 0; a < 2; ++a) {
+                    const uint4* pk = reinterpret_cast<const uint4*>(sb + S::PK_OFF + a * kPkBytes + d * 32);
+                    const uint4 w0 = pk[0], w1 = pk[1];
+                    const uint32_t words[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
 #pragma unroll
-                    for (int i = 0; i < 8; ++i) {
-                        const int r = r0 + 16 * i;
-                        const uint32_t w = pk[a * (kPkBytes / 4) + r * 8 + c];
-                        const uint4 v = dequant8(w, __low2bfloat162(sbc[a * 8 + i]), __high2bfloat162(sbc[a * 8 + i]));
-                        *reinterpret_cast<uint4*>(sb + a * S::A_BYTES + sw128_offset(r, c)) = v;
+                    for (int c = 0; c < 8; ++c) {
+                        const __nv_bfloat162 sbv = q0[a][c >> 2];
+                        const uint4 v = dequant8(words[c], __low2bfloat162(sbv), __high2bfloat162(sbv));
+                        *reinterpret_cast<uint4*>(sb + a * S::A_BYTES + sw128_offset(d, c)) = v;
                     }
+                }
                 // generic-proxy writes, read next by the tensor cores (async proxy)
                 asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&dq[stage]);
 #pragma unroll
-                for (int i = 0; i < 16; ++i) sbc[i] = sbn[i];
+                for (int a = 0; a < 2; ++a)
+#pragma unroll
+                    for (int h = 0; h < 2; ++h) {
+                        q0[a][h] = q1[a][h];
+                        q1[a][h] = q2[a][h];
+                    }
                 if (++stage == STAGES) {
                     stage = 0;
                     phase ^= 1u;
