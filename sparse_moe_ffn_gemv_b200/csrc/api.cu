@@ -33,7 +33,7 @@ WsLayout ws_layout(const moe_config& c, int64_t T) {
     const int64_t ab = act_bytes(c);
     L.T = T;
     L.ld_logits = int((E + 2 + 3) & ~int64_t(3));
-    L.n_chunks = int((T * k + kPermChunk - 1) / kPermChunk);
+    L.n_chunks = int((T * k + kPermChunkWs - 1) / kPermChunkWs);
     L.status = take(256);
     L.logits = take(T * L.ld_logits * 4);
     L.topk_idx = take(T * k * 4);
@@ -319,6 +319,7 @@ moe_status run_permute(const moe_config* c, const int32_t* idx, int64_t T, int32
     p.slot_pos = slot_pos;
     p.active = at<int32_t>(ws, L.active);
     p.chunk_hist = at<int32_t>(ws, L.chunk_hist);
+    p.chunk = kPermChunkWs;
     p.n_chunks = L.n_chunks;
     p.status = at<int>(ws, L.status);
     if (tc_tiles) {

@@ -34,7 +34,7 @@ struct WsLayout {
     size_t sorted_slot;  // int32 [T * k]
     size_t slot_pos;     // int32 [T * k]
     size_t active;       // int32 [E + 1]: n_active, then the active expert ids
-    size_t chunk_hist;   // int32 [n_chunks, E]
+    size_t chunk_hist;   // int32 [E, n_chunks]: slots per expert in each permutation chunk
     size_t h;            // act [T * k, I]: routed intermediate, sorted order
     size_t hs;           // act [T, Is]: shared intermediate
     size_t y_acc;        // f32 [T, K]: routed sum
@@ -50,7 +50,8 @@ struct WsLayout {
     int64_t T;
 };
 
-constexpr int kPermChunk = 2048;  // slots per permutation chunk
+constexpr int kPermChunk = 2048;   // slots per permutation chunk (fixed-scratch permutation)
+constexpr int kPermChunkWs = 2048;  // slots per chunk when the workspace holds the histograms (512 measured slower)
 
 inline size_t align256(size_t v) { return (v + 255) & ~size_t(255); }
 inline int act_bytes(const moe_config& c) { return c.act_dtype == kF32 ? 4 : 2; }

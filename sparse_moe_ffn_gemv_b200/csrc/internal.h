@@ -39,6 +39,7 @@ struct PermuteArgs {
     const int32_t* idx = nullptr; int64_t S = 0; int E = 0;
     int32_t* offsets = nullptr; int32_t* sorted_slot = nullptr; int32_t* slot_pos = nullptr;
     int32_t* active = nullptr; int32_t* chunk_hist = nullptr; int n_chunks = 0;
+    int chunk = 2048;                // slots per chunk (one block each); n_chunks = ceil(S / chunk)
     int* status = nullptr;
     int tile_bn = 0;                 // > 0: also write tile_start[E + 1], the exclusive prefix
     int32_t* tile_start = nullptr;   //      of ceil(count_e / tile_bn) (tensor-core tile list)

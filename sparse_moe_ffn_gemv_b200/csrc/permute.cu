@@ -23,15 +23,15 @@ __global__ void __launch_bounds__(256) hist_kernel(PermuteArgs a) {
     __shared__ int hist[kPermE];
     for (int e = threadIdx.x; e < a.E; e += blockDim.x) hist[e] = 0;
     __syncthreads();
-    const int64_t s0 = int64_t(blockIdx.x) * kPermChunk;
-    const int64_t s1 = min(a.S, s0 + kPermChunk);
+    const int64_t s0 = int64_t(blockIdx.x) * a.chunk;
+    const int64_t s1 = min(a.S, s0 + a.chunk);
     for (int64_t s = s0 + threadIdx.x; s < s1; s += blockDim.x) {
         const int e = a.idx[s];
         if (e >= 0 && e < a.E) atomicAdd(&hist[e], 1);
     }
     __syncthreads();
     for (int e = threadIdx.x; e < a.E; e += blockDim.x)
-        a.chunk_hist[int64_t(blockIdx.x) * a.E + e] = hist[e];
+        a.chunk_hist[int64_t(e) * a.n_chunks + blockIdx.x] = hist[e];  // expert-major
 }
 
 __global__ void __launch_bounds__(kPlaceThreads) place_kernel(PermuteArgs a) {
@@ -117,7 +117,7 @@ cudaError_t launch_permute(const PermuteArgs& a, cudaStream_t s) {
 
 // ---------------------------------------------------------------- permutation without a workspace
 // Scratch of moe_permute_noalloc: [status word, padded to 256 B][active list, 513 ints,
-// padded to 2304 B][per-chunk histograms, 32 chunks x 512 experts]. Every GPU that loads
+// padded to 2304 B][per-chunk histograms, 512 experts x 32 chunks, expert-major]. Every GPU that loads
 // the library holds it until the process exits.
 namespace {
 constexpr int kNoAllocMaxSlots = 65536;
@@ -186,6 +186,7 @@ extern "C" moe_status moe_permute_noalloc(const moe_config* cfg, const int32_t* 
     p.slot_pos = slot_pos;
     p.active = reinterpret_cast<int32_t*>(base + kNoAllocActive);
     p.chunk_hist = reinterpret_cast<int32_t*>(base + kNoAllocHist);
+    p.chunk = kPermChunk;
     p.n_chunks = int((p.S + kPermChunk - 1) / kPermChunk);
     p.status = status;
     return launch_permute(p, s) == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;

@@ -78,8 +78,8 @@ __device__ void place_chunk(const PermuteArgs& a, int chunk, PlaceSmem<NT>& sm) 
     constexpr int NW = NT / 32;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int E = a.E;
-    const int64_t s0 = int64_t(chunk) * kPermChunk;
-    const int64_t s1 = min(a.S, s0 + kPermChunk);
+    const int64_t s0 = int64_t(chunk) * a.chunk;
+    const int64_t s1 = min(a.S, s0 + a.chunk);
 
     for (int i = tid; i < NW * kPermE; i += NT) (&sm.cnt[0][0])[i] = 0;
     if (a.n_chunks == 1) {
@@ -94,11 +94,14 @@ __device__ void place_chunk(const PermuteArgs& a, int chunk, PlaceSmem<NT>& sm) 
         for (int e = tid; e < E; e += NT) sm.base[e] = 0;  // no earlier chunks
     } else {
         for (int e = tid; e < E; e += NT) {
+            // this expert's counts of all chunks are contiguous (expert-major histograms)
+            const int* hrow = a.chunk_hist + int64_t(e) * a.n_chunks;
             int tot = 0, pre = 0;
+#pragma unroll 8
             for (int c = 0; c < a.n_chunks; ++c) {
-                const int h = a.chunk_hist[int64_t(c) * E + e];
+                const int h = hrow[c];
                 tot += h;
-                if (c < chunk) pre += h;
+                pre += c < chunk ? h : 0;
             }
             sm.scan_buf[e] = tot;
             sm.base[e] = pre;
