@@ -214,6 +214,24 @@ def cpu_baseline(spec, w_cpu, x_cpu, target_s: float = 10.0):
                       f"({dt2:.1f} s, fp64, OpenMP over tokens)"}
 
 
+def workload_config(spec, T, world):
+    """The `config` object of both arms' JSON lines."""
+    return {"workload": f"{spec.name} (hidden {spec.hidden}, {spec.num_experts} experts, "
+                        f"top-{spec.top_k}, intermediate {spec.intermediate})",
+            "tokens_per_gpu": T, "parallelism": f"replicas x{world}",
+            "l2": "activated weights larger than L2 (no flush needed); decode rows flush L2"}
+
+
+def max_over_ranks(v: float, dist, device) -> float:
+    """The largest of every rank's value (a step time): the whole job is as slow as its
+    slowest replica. Identity on one rank."""
+    if dist is None:
+        return float(v)
+    t = torch.tensor([float(v)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
 def reference_arm(args, rank, world):
     if rank != 0:
         return
@@ -244,8 +262,7 @@ def reference_arm(args, rank, world):
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1000 * tot / args.steps,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
             "data": "synthetic (seeded; no checkpoint)",
-            "config": {"workload": spec.name, "tokens": T, "hidden": spec.hidden,
-                       "experts": spec.num_experts, "top_k": spec.top_k},
+            "config": workload_config(spec, T, world),
             "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": threads, "kind": "oracle",
                              "sample": f"{n} tokens of the {T}-token batch per step"},
             "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
@@ -359,10 +376,7 @@ def run(args, rank, world, local, dist):
     if block.device_status() != 0:
         raise SystemExit("device status set during the timed region")
 
-    ms_t = torch.tensor([ms], device=dev)
-    if dist is not None:
-        dist.all_reduce(ms_t, op=dist.ReduceOp.MAX)
-    ms_max = float(ms_t.item())
+    ms_max = max_over_ranks(ms, dist, dev)
     value = world * T / (ms_max / 1000.0)
 
     pk, pk_src = peaks()
@@ -387,10 +401,8 @@ def run(args, rank, world, local, dist):
             y_host.copy_(y, non_blocking=True)
 
         e2e_ms = time_steps(e2e_step, args.steps, args.warmup)
-        e_ms = torch.tensor([statistics.mean(e2e_ms)], device=dev)
-        if dist is not None:
-            dist.all_reduce(e_ms, op=dist.ReduceOp.MAX)
-        e2e = {"value": world * T / (float(e_ms.item()) / 1000.0), "unit": "tokens/s",
+        e_max = max_over_ranks(statistics.mean(e2e_ms), dist, dev)
+        e2e = {"value": world * T / (e_max / 1000.0), "unit": "tokens/s",
                "h2d_bytes_per_step": T * spec.hidden * ab, "d2h_bytes_per_step": T * spec.hidden * ab}
 
     # ---- decode-sized batches (L2 flushed between iterations; graphs remove launch gaps)
@@ -433,10 +445,7 @@ def run(args, rank, world, local, dist):
             "warmup": args.warmup, "ms_per_step": ms_max, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": spec.act_dtype if spec.weight_format != "q4" else "bf16+q4",
             "data": "synthetic (seeded N(0,1) activations, N(0,0.02) weights; no checkpoint)",
-            "config": {"workload": f"{spec.name} (hidden {spec.hidden}, {spec.num_experts} experts, "
-                                   f"top-{spec.top_k}, intermediate {spec.intermediate})",
-                       "tokens_per_gpu": T, "parallelism": f"replicas x{world}",
-                       "l2": "activated weights larger than L2 (no flush needed); decode rows flush L2"},
+            "config": workload_config(spec, T, world),
             "roofline": roofline,
             "block": {"algorithmic_bytes": blk_bytes, "gbs": blk_bytes / (ms_max / 1000) / 1e9,
                       "hbm_frac": blk_bytes / (ms_max / 1000) / 1e9 / pk["hbm_gbs"],
