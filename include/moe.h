@@ -82,7 +82,9 @@ enum moe_activation {
 enum moe_dtype {
     MOE_DTYPE_F32 = 0,
     MOE_DTYPE_BF16 = 1,
-    MOE_DTYPE_Q4_AFFINE = 2        /* weights only: packed 4-bit codes + bf16 scale/bias */
+    MOE_DTYPE_Q4_AFFINE = 2,       /* weights only: packed 4-bit codes + bf16 scale/bias */
+    MOE_DTYPE_MXFP4 = 3            /* weights only: E2M1 codes + an E8M0 scale per 32
+                                      elements (OCP Microscaling Formats v1.0)          */
 };
 enum moe_shared_mode {
     MOE_SHARED_NONE = 0,
@@ -108,9 +110,10 @@ typedef struct moe_config {
     int32_t has_selection_bias;    /* 1: select-only bias [E] (f32)                     */
     int32_t act_dtype;             /* MOE_DTYPE_F32 or MOE_DTYPE_BF16: x, y and every
                                       non-routed weight                                 */
-    int32_t weight_format;         /* routed planes: F32 (needs act F32), BF16, Q4_AFFINE */
-    int32_t group_size;            /* Q4 only: 32, 64 or 128                            */
-    int32_t bits;                  /* Q4 only: 4                                        */
+    int32_t weight_format;         /* routed planes: F32 (needs act F32), BF16, Q4_AFFINE,
+                                      MXFP4 (both need act BF16, separate gate/up)      */
+    int32_t group_size;            /* Q4: 32, 64 or 128; MXFP4: 32                      */
+    int32_t bits;                  /* Q4 and MXFP4: 4                                   */
     int32_t shared_mode;           /* enum moe_shared_mode                              */
     int32_t shared_intermediate;   /* Is (> 0 iff shared_mode != NONE)                  */
     int32_t latent_dim;            /* L; 0 = no latent projection                       */
@@ -130,6 +133,11 @@ typedef struct moe_config {
  *       row at bits 4*(j mod 8) of word j/8), gate_s/up_s/down_s the bf16
  *       scales and gate_z/up_z/down_z the bf16 biases [E, rows, cols/group];
  *       weight = scale * q + bias.
+ *   MXFP4: the same uint32 words, each code an E2M1 element (bit 3 sign, bits
+ *       2..1 exponent, bit 0 mantissa: magnitudes 0, 0.5, 1, 1.5, 2, 3, 4, 6);
+ *       gate_s/up_s/down_s hold one uint8 E8M0 scale per 32 elements
+ *       [E, rows, cols/32], weight = element * 2^(scale - 127); the _z fields are
+ *       unused. A scale byte of 255 (NaN in the format) gives non-finite weights.
  *   shared_gate_w, shared_up_w [Is, H]; shared_down_w [H, Is]
  *   latent_down_w [L, H]; latent_up_w [H, L]; latent_norm_w [L]
  */

@@ -27,7 +27,7 @@ _LIB_PATH = os.path.join(_HERE, "libmoe_oracle.so")
 
 _SCORING = {"softmax_all": 0, "sigmoid": 1, "softmax_topk": 2}
 _ACT = {"swiglu": 0, "swiglu_clamped": 1}
-_DT = {"f32": 0, "bf16": 1, "q4": 2}
+_DT = {"f32": 0, "bf16": 1, "q4": 2, "mxfp4": 3}
 _SHARED = {"none": 0, "add": 1, "blend": 2}
 
 
@@ -100,6 +100,9 @@ def _load():
                                        ctypes.c_int64, ctypes.c_int32, ctypes.c_int64,
                                        ctypes.c_int64]
         lib.orc_dequant_q4.restype = ctypes.c_double
+        lib.orc_dequant_mxfp4.argtypes = [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int64, ctypes.c_int64,
+                                          ctypes.c_int64]
+        lib.orc_dequant_mxfp4.restype = ctypes.c_double
         lib.orc_max_threads.argtypes = []
         lib.orc_max_threads.restype = ctypes.c_int
         _lib = lib
@@ -129,7 +132,7 @@ def _config(spec) -> OrcConfig:
 
 def _check_storage(a: np.ndarray) -> np.ndarray:
     assert a.flags["C_CONTIGUOUS"], "oracle inputs must be C-contiguous"
-    assert a.dtype in (np.float32, np.uint16, np.uint32), a.dtype
+    assert a.dtype in (np.float32, np.uint16, np.uint32, np.uint8), a.dtype
     return a
 
 
@@ -227,3 +230,9 @@ def dequant_q4(q: np.ndarray, scales: np.ndarray, biases: np.ndarray, cols: int,
     return float(_load().orc_dequant_q4(q.ctypes.data, _check_storage(scales).ctypes.data,
                                         _check_storage(biases).ctypes.data, cols, group_size,
                                         row, col))
+
+
+def dequant_mxfp4(q: np.ndarray, scales: np.ndarray, cols: int, row: int, col: int) -> float:
+    """One MXFP4 weight W[row, col] (E2M1 element times its block's E8M0 scale)."""
+    q = _check_storage(q)
+    return float(_load().orc_dequant_mxfp4(q.ctypes.data, _check_storage(scales).ctypes.data, cols, row, col))

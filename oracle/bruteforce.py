@@ -33,7 +33,23 @@ def _dequant(q: np.ndarray, s: np.ndarray, z: np.ndarray, group: int) -> np.ndar
     return codes * scale + bias
 
 
+# OCP Microscaling Formats v1.0, FP4 E2M1: the sixteen code values (table of the spec).
+_E2M1_TABLE = np.array([0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0,
+                        -0.0, -0.5, -1.0, -1.5, -2.0, -3.0, -4.0, -6.0])
+
+
+def _dequant_mxfp4(q: np.ndarray, sbytes: np.ndarray) -> np.ndarray:
+    """Packed MXFP4 planes [..., K/8] with E8M0 scale bytes [..., K/32] -> float64 [..., K]."""
+    shifts = np.arange(8, dtype=np.uint32) * 4
+    codes = (q[..., None] >> shifts) & 0xF
+    codes = codes.reshape(*q.shape[:-1], q.shape[-1] * 8)
+    scale = np.repeat(np.exp2(sbytes.astype(np.float64) - 127.0), 32, axis=-1)
+    return _E2M1_TABLE[codes] * scale
+
+
 def _plane(spec, w, name):
+    if spec.weight_format == "mxfp4":
+        return _dequant_mxfp4(w[name], w[name[:-2] + "_s"])
     if spec.weight_format == "q4":
         stem = name[:-2]
         return _dequant(w[name], w[stem + "_s"], w[stem + "_z"], spec.group_size)

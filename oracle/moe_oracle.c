@@ -31,6 +31,13 @@
  *    the expert shape down(act(gate(x), up(x))) with [out, in] weights.
  *  - mlxcel issue #974, "What exists": stacked switch_mlp expert planes and
  *    the affine 4-bit mode (weight, scales, biases, group_size 64, bits 4).
+ *  - libmir-metal clamped_routed/experts/mod.rs, the split/u32 MXFP4 layout
+ *    (gate, up and down blocks, each with scales and a bias); the element and
+ *    scale encodings are not on the pages and come from the public OCP
+ *    Microscaling Formats (MX) Specification v1.0: blocks of 32 elements, each
+ *    element FP4 E2M1 (sign, 2 exponent bits with bias 1, 1 mantissa bit,
+ *    subnormal when the exponent field is 0), one shared E8M0 scale per block
+ *    (2^(byte - 127); byte 255 is NaN).
  *
  * Readings where the pages are silent (each listed in the design notes):
  *  - SwiGLU is silu(g) * v with silu(g) = g / (1 + e^-g).
@@ -52,7 +59,7 @@
 
 enum { ORC_SOFTMAX_ALL = 0, ORC_SIGMOID = 1, ORC_SOFTMAX_TOPK = 2 };
 enum { ORC_SWIGLU = 0, ORC_SWIGLU_CLAMPED = 1 };
-enum { ORC_F32 = 0, ORC_BF16 = 1, ORC_Q4 = 2 };
+enum { ORC_F32 = 0, ORC_BF16 = 1, ORC_Q4 = 2, ORC_MXFP4 = 3 };
 enum { ORC_SHARED_NONE = 0, ORC_SHARED_ADD = 1, ORC_SHARED_BLEND = 2 };
 
 typedef struct {
@@ -108,6 +115,22 @@ double orc_dequant_q4(const uint32_t *q, const uint16_t *scales, const uint16_t 
     return s * (double)code + b;
 }
 
+/* One MXFP4 weight W[row, col]: the E2M1 element value times its block's
+ * E8M0 scale, 32 elements per block (OCP MX v1.0). The element value is the
+ * format's definition written out: exponent field e, mantissa bit m, and
+ * (-1)^sign * 2^(e-1) * (1 + m/2) for e > 0, (-1)^sign * m/2 for e = 0. */
+double orc_dequant_mxfp4(const uint32_t *q, const uint8_t *scales, int64_t cols, int64_t row, int64_t col)
+{
+    uint32_t word = q[row * (cols / 8) + col / 8];
+    int code = (int)((word >> (4 * (col % 8))) & 0xFu);
+    int e = (code >> 1) & 3, m = code & 1;
+    double v = e > 0 ? ldexp(1.0 + 0.5 * m, e - 1) : 0.5 * m;
+    if (code & 8) v = -v;
+    int sbyte = scales[row * (cols / 32) + col / 32];
+    if (sbyte == 255) return NAN;
+    return ldexp(v, sbyte - 127);
+}
+
 /* W[e, r, c] of a stacked routed-expert plane [E, rows, cols]. */
 static double plane_at(const orc_config *cfg, const void *w, const void *s, const void *z,
                        int64_t rows, int64_t cols, int64_t e, int64_t r, int64_t c)
@@ -116,6 +139,8 @@ static double plane_at(const orc_config *cfg, const void *w, const void *s, cons
     if (cfg->weight_format == ORC_Q4)
         return orc_dequant_q4((const uint32_t *)w, (const uint16_t *)s, (const uint16_t *)z,
                               cols, cfg->group_size, row, c);
+    if (cfg->weight_format == ORC_MXFP4)
+        return orc_dequant_mxfp4((const uint32_t *)w, (const uint8_t *)s, cols, row, c);
     return dense_at(w, cfg->weight_format, row * cols + c);
 }
 

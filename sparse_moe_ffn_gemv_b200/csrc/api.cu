@@ -81,7 +81,7 @@ moe_status validate_config(const moe_config* c) {
         return MOE_ERR_INVALID_ARGUMENT;
     if (c->shared_mode < MOE_SHARED_NONE || c->shared_mode > MOE_SHARED_BLEND) return MOE_ERR_INVALID_ARGUMENT;
     if (c->act_dtype != MOE_DTYPE_F32 && c->act_dtype != MOE_DTYPE_BF16) return MOE_ERR_INVALID_ARGUMENT;
-    if (c->weight_format < MOE_DTYPE_F32 || c->weight_format > MOE_DTYPE_Q4_AFFINE)
+    if (c->weight_format < MOE_DTYPE_F32 || c->weight_format > MOE_DTYPE_MXFP4)
         return MOE_ERR_INVALID_ARGUMENT;
     if (c->shared_intermediate < 0 || c->latent_dim < 0) return MOE_ERR_INVALID_ARGUMENT;
     if ((c->shared_mode == MOE_SHARED_NONE) != (c->shared_intermediate == 0)) return MOE_ERR_INVALID_ARGUMENT;
@@ -101,6 +101,11 @@ moe_status validate_config(const moe_config* c) {
             return MOE_ERR_INVALID_QUANTIZATION;
         if (K % c->group_size != 0 || c->intermediate % c->group_size != 0)
             return MOE_ERR_INVALID_QUANTIZATION;
+        if (c->gate_up_interleaved) return MOE_ERR_UNSUPPORTED;
+    }
+    if (c->weight_format == MOE_DTYPE_MXFP4) {  // OCP MX: blocks of 32 elements, 4-bit E2M1
+        if (c->bits != 4 || c->group_size != 32) return MOE_ERR_INVALID_QUANTIZATION;
+        if (K % 64 != 0 || c->intermediate % 64 != 0) return MOE_ERR_INVALID_QUANTIZATION;
         if (c->gate_up_interleaved) return MOE_ERR_UNSUPPORTED;
     }
     // 16-byte rows
@@ -134,6 +139,8 @@ moe_status validate_weights(const moe_config* c, const moe_weights* w) {
         for (const void* p : q)
             if (!need(p)) return MOE_ERR_MISSING_TENSOR;
     }
+    if (c->weight_format == MOE_DTYPE_MXFP4 && (!need(w->gate_s) || !need(w->up_s) || !need(w->down_s)))
+        return MOE_ERR_MISSING_TENSOR;
     if (c->shared_mode != MOE_SHARED_NONE &&
         (!need(w->shared_gate_w) || !need(w->shared_up_w) || !need(w->shared_down_w)))
         return MOE_ERR_MISSING_TENSOR;
@@ -183,7 +190,8 @@ bool dense_tc(const moe_config* c, int64_t T, int K) {
 // kernels from there on, although most tiles then hold only a few tokens (Klear shape:
 // 8 tokens 149 vs 157 us, 64 tokens 279 vs 627 us; at 4 tokens the CUDA cores win).
 bool routed_tc(const moe_config* c, int64_t T) {
-    if (c->act_dtype != MOE_DTYPE_BF16 || c->weight_format == MOE_DTYPE_F32) return false;
+    if (c->act_dtype != MOE_DTYPE_BF16 || c->weight_format == MOE_DTYPE_F32 || c->weight_format == MOE_DTYPE_MXFP4)
+        return false;
     if (expert_in(*c) % 64 != 0 || c->intermediate % 64 != 0) return false;
     const int o = path_override();
     return o == kPathTc || (o == kPathAuto && 4 * T * c->top_k >= int64_t(c->num_experts));

@@ -460,7 +460,8 @@ cudaError_t launch_gateup_gemv(const GateUpArgs& a, cudaStream_t s) {
     switch (a.wf) {
         case kF32: return launch_gateup_t<kF32>(a, s);
         case kBF16: return launch_gateup_t<kBF16>(a, s);
-        default: return launch_gateup_t<kQ4>(a, s);
+        case kQ4: return launch_gateup_t<kQ4>(a, s);
+        default: return cudaErrorInvalidValue;
     }
 }
 
@@ -468,7 +469,8 @@ cudaError_t launch_down_gemv(const DownArgs& a, cudaStream_t s) {
     switch (a.wf) {
         case kF32: return launch_down_t<kF32>(a, s);
         case kBF16: return launch_down_t<kBF16>(a, s);
-        default: return launch_down_t<kQ4>(a, s);
+        case kQ4: return launch_down_t<kQ4>(a, s);
+        default: return cudaErrorInvalidValue;
     }
 }
 

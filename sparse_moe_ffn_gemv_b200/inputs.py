@@ -35,7 +35,7 @@ import torch
 # Enum codes; the same integers appear in include/moe.h.
 SCORING = {"softmax_all": 0, "sigmoid": 1, "softmax_topk": 2}
 ACTIVATION = {"swiglu": 0, "swiglu_clamped": 1}
-DTYPE = {"f32": 0, "bf16": 1, "q4": 2}
+DTYPE = {"f32": 0, "bf16": 1, "q4": 2, "mxfp4": 3}
 SHARED = {"none": 0, "add": 1, "blend": 2}
 
 
@@ -98,7 +98,12 @@ LATENT_BF16 = MoeSpec(
     shared_mode="add", shared_intermediate=2048, latent_dim=3584, latent_use_norm=True,
     rms_eps=1e-6, token_counts=(1, 128, 8192))
 
-WORKLOADS = {s.name: s for s in (TINY_F32, KLEAR_BF16, KLEAR_Q4, CLAMPED_BF16, LATENT_BF16)}
+# The clamped-routed family with MXFP4 expert planes in the split/u32 layout (libmir-metal
+# clamped_routed: gate, up and down blocks with scales and biases; not interleaved).
+CLAMPED_MXFP4 = CLAMPED_BF16.replace(name="clamped_mxfp4", config_id=6, weight_format="mxfp4",
+                                     gate_up_interleaved=False, group_size=32, token_counts=(1, 8, 8192))
+
+WORKLOADS = {s.name: s for s in (TINY_F32, KLEAR_BF16, KLEAR_Q4, CLAMPED_BF16, LATENT_BF16, CLAMPED_MXFP4)}
 
 BASE_SEED = 20261202
 
@@ -149,6 +154,36 @@ def quantize_affine_q4(w: torch.Tensor, group_size: int):
     return torch.from_numpy(packed.copy()), scale.contiguous(), bias.contiguous()
 
 
+# E2M1 magnitudes by the low three bits of a code (OCP Microscaling Formats v1.0).
+_E2M1 = torch.tensor([0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0])
+
+
+def quantize_mxfp4(w: torch.Tensor):
+    """Encode fp32 planes [..., K] as a synthetic MXFP4 checkpoint (OCP MX v1.0).
+
+    Per block of 32 consecutive input elements: the shared E8M0 scale is 2^x with
+    x = floor(log2(max |w|)) - 2 (the largest E2M1 exponent), stored as the byte x + 127;
+    each element is w / 2^x rounded to the nearest E2M1 value (ties to the smaller
+    magnitude), clamped to +-6; code = sign bit 8 | magnitude index. Codes pack as the
+    4-bit planes do: element j of a row at bits 4*(j mod 8) of word j/8. Returns (packed
+    words [..., K/8] as int32 bit patterns, scale bytes uint8 [..., K/32]).
+    """
+    *lead, k = w.shape
+    assert k % 32 == 0
+    g = w.reshape(*lead, k // 32, 32)
+    amax = g.abs().amax(dim=-1).clamp_min(2.0 ** -120)
+    x = torch.floor(torch.log2(amax)) - 2.0
+    sbyte = (x + 127).clamp(1, 254)
+    v = (g / torch.exp2(sbyte - 127).unsqueeze(-1)).clamp(-6.0, 6.0)
+    idx = (v.abs().unsqueeze(-1) - _E2M1).abs().argmin(dim=-1)  # first minimum: smaller magnitude
+    code = idx + torch.where(v < 0, 8, 0) * (idx > 0)
+    code = code.to(torch.int64).reshape(*lead, k // 8, 8)
+    shifts = torch.arange(8, dtype=torch.int64) * 4
+    packed = (code << shifts).sum(dim=-1)
+    packed = packed.bitwise_and(0xFFFFFFFF).numpy().astype(np.uint32).view(np.int32)
+    return torch.from_numpy(packed.copy()), sbyte.to(torch.uint8).contiguous()
+
+
 def _expert_plane(spec: MoeSpec, name: str, rows: int, cols: int, pool) -> Dict[str, torch.Tensor]:
     """One stacked expert projection [E, rows, cols] in the spec's weight format.
 
@@ -160,9 +195,13 @@ def _expert_plane(spec: MoeSpec, name: str, rows: int, cols: int, pool) -> Dict[
         w = _normal((rows, cols), 0.02, _seed(spec, f"{name}/{e}"))
         if spec.weight_format == "q4":
             return quantize_affine_q4(w, spec.group_size)
+        if spec.weight_format == "mxfp4":
+            return quantize_mxfp4(w)
         return (_storage(w, spec.weight_format),)
 
     parts = list(pool.map(one, range(e_count)))
+    if spec.weight_format == "mxfp4":  # "gate_w" -> "gate_s" (E8M0 scale bytes)
+        return {name: torch.stack([p[0] for p in parts]), name[:-2] + "_s": torch.stack([p[1] for p in parts])}
     if spec.weight_format == "q4":
         stem = name[:-2]  # "gate_w" -> companions "gate_s" (scales), "gate_z" (biases)
         return {name: torch.stack([p[0] for p in parts]),
@@ -222,7 +261,7 @@ def make_x(spec: MoeSpec, T: int, scale: float = 1.0) -> torch.Tensor:
 
 def to_numpy_storage(t: torch.Tensor) -> np.ndarray:
     """Bit-exact numpy view of a stored tensor: bf16 -> uint16, f32 -> float32,
-    packed 4-bit words (int32) -> uint32."""
+    packed 4-bit words (int32) -> uint32, MXFP4 scale bytes -> uint8."""
     t = t.contiguous()
     if t.dtype == torch.bfloat16:
         return t.view(torch.int16).numpy().view(np.uint16)

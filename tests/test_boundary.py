@@ -64,6 +64,7 @@ def test_enum_values_match_the_header():
     assert val("MOE_SCORING_SOFTMAX_TOPK") == inputs.SCORING["softmax_topk"]
     assert val("MOE_ACT_SWIGLU_CLAMPED") == inputs.ACTIVATION["swiglu_clamped"]
     assert val("MOE_DTYPE_Q4_AFFINE") == inputs.DTYPE["q4"]
+    assert val("MOE_DTYPE_MXFP4") == inputs.DTYPE["mxfp4"]
     assert val("MOE_SHARED_BLEND") == inputs.SHARED["blend"]
     for name, code in M.STATUS_CODE.items():
         assert val(name) == code
@@ -113,6 +114,21 @@ QUANT = [("bits 0", dict(bits=0)), ("bits 8", dict(bits=8)), ("group 0", dict(gr
 def test_hostile_quantisation_params_are_rejected(name, fields):
     assert M.moe_config_validate(_cfg(inputs.KLEAR_Q4)) == 0
     assert M.STATUS[M.moe_config_validate(_cfg(inputs.KLEAR_Q4, **fields))] == "MOE_ERR_INVALID_QUANTIZATION"
+
+
+def test_mxfp4_needs_blocks_of_32_four_bits_and_separate_gate_up():
+    assert M.moe_config_validate(_cfg(inputs.CLAMPED_MXFP4)) == 0
+    for fields in (dict(group_size=64), dict(bits=8)):
+        assert M.STATUS[M.moe_config_validate(_cfg(inputs.CLAMPED_MXFP4, **fields))] == \
+            "MOE_ERR_INVALID_QUANTIZATION"
+    assert M.STATUS[M.moe_config_validate(_cfg(inputs.CLAMPED_MXFP4, gate_up_interleaved=1))] == \
+        "MOE_ERR_UNSUPPORTED"
+    cfg = _cfg(inputs.CLAMPED_MXFP4)
+    w = _fake_weights(inputs.CLAMPED_MXFP4)
+    w.gate_z = w.up_z = w.down_z = None            # MXFP4 has no affine biases
+    assert M.moe_weights_validate(cfg, w) == 0
+    w.down_s = None                                  # but every plane needs its scales
+    assert M.STATUS[M.moe_weights_validate(cfg, w)] == "MOE_ERR_MISSING_TENSOR"
 
 
 def test_group_must_divide_the_widths():

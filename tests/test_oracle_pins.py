@@ -15,7 +15,7 @@ import torch
 import oracle
 from oracle import bruteforce
 from sparse_moe_ffn_gemv_b200 import inputs
-from tiny_specs import (ALL, CLAMPED, LATENT, LATENT_NONORM, Q4, ROUTER_BIAS, SIG_BLEND,
+from tiny_specs import (ALL, CLAMPED, LATENT, LATENT_NONORM, MXFP4, Q4, ROUTER_BIAS, SIG_BLEND,
                         np_weights, np_x, to_bf16_bits)
 
 GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
@@ -395,6 +395,56 @@ def test_q4_planes_match_the_bruteforce_unpacking_and_are_near_the_drawn_weights
                                  w["gate_z"].reshape(-1, spec.hidden // 64), spec.hidden, 64,
                                  e * spec.intermediate + r, c) == deq[e, r, c]
     assert np.abs(deq).max() < 0.2 and deq.std() == pytest.approx(0.02, rel=0.1)
+
+
+# --- MXFP4 (OCP Microscaling Formats v1.0) -----------------------------------------
+# The FP4 E2M1 value table of the specification, by code 0..15.
+SPEC_E2M1 = [0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0, -0.0, -0.5, -1.0, -1.5, -2.0, -3.0, -4.0, -6.0]
+
+
+def test_mxfp4_codes_decode_to_the_spec_table_times_the_block_scale():
+    q = np.array([[0x76543210, 0xFEDCBA98, 0x76543210, 0xFEDCBA98]], dtype=np.uint32)  # codes 0..15, twice
+    for sbyte in (127, 120, 130, 1, 254):
+        s = np.array([[sbyte]], dtype=np.uint8)
+        vals = [oracle.dequant_mxfp4(q, s, 32, 0, c) for c in range(32)]
+        assert vals == [v * 2.0 ** (sbyte - 127) for v in SPEC_E2M1 * 2]
+    assert math.isnan(oracle.dequant_mxfp4(q, np.array([[255]], dtype=np.uint8), 32, 0, 3))  # NaN scale
+    # two blocks of 32 with their own scales, element j at bits 4 * (j mod 8) of word j / 8
+    q2 = np.array([[0x00000001] + [0] * 3 + [0x60000000] + [0] * 3], dtype=np.uint32)
+    s2 = np.array([[127, 125]], dtype=np.uint8)
+    assert oracle.dequant_mxfp4(q2, s2, 64, 0, 0) == 0.5
+    assert oracle.dequant_mxfp4(q2, s2, 64, 0, 39) == 4.0 * 0.25   # code 6 = 4.0, block scale 2^-2
+
+
+def test_mxfp4_encoder_keeps_representable_values_and_matches_bruteforce_unpacking():
+    vals = torch.tensor(SPEC_E2M1[:8] + [-v for v in SPEC_E2M1[1:8]] + [6.0] * 17) * 2.0 ** -9
+    q, s = inputs.quantize_mxfp4(vals.reshape(1, 32).float())
+    qn, sn = inputs.to_numpy_storage(q), inputs.to_numpy_storage(s)
+    assert [oracle.dequant_mxfp4(qn, sn, 32, 0, c) for c in range(32)] == vals.double().tolist()
+    w = np_weights(MXFP4)
+    deq = bruteforce._dequant_mxfp4(w["gate_w"], w["gate_s"])
+    for (e, r, c) in [(0, 0, 0), (1, 5, 63), (4, 63, 127), (2, 17, 64)]:
+        assert oracle.dequant_mxfp4(w["gate_w"].reshape(-1, MXFP4.hidden // 8),
+                                    w["gate_s"].reshape(-1, MXFP4.hidden // 32), MXFP4.hidden,
+                                    e * MXFP4.intermediate + r, c) == deq[e, r, c]
+    assert np.abs(deq).max() < 0.2 and deq.std() == pytest.approx(0.02, rel=0.15)
+
+
+def test_mxfp4_block_equals_the_same_weights_stored_in_bf16():
+    """Every MXFP4 weight (at most two significant bits times a power of two) is exact in bf16:
+    the block evaluated on the packed planes equals the block on those values stored as bf16."""
+    w = np_weights(MXFP4)
+    x = np_x(MXFP4, 6, 30.0)
+    spec_bf = MXFP4.replace(name="t_mxfp4_as_bf16", weight_format="bf16")
+    wb = dict(w)
+    for name in ("gate_w", "up_w", "down_w"):
+        deq = bruteforce._dequant_mxfp4(w[name], w[name[:-2] + "_s"])
+        wb[name] = to_bf16_bits(deq)
+        del wb[name[:-2] + "_s"]
+    a = oracle.forward(MXFP4, w, x)
+    b = oracle.forward(spec_bf, wb, x)
+    np.testing.assert_array_equal(a["idx"], b["idx"])
+    np.testing.assert_array_equal(a["y"], b["y"])
 
 
 # --- permutation -----------------------------------------------------------------

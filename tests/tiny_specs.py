@@ -4,7 +4,9 @@ Each variant exercises one branch of the block: sigmoid routing with a
 select-only bias and the shared-expert blend (Klear PR items 2-3), softmax
 over the top-k logits with clamped SwiGLU on an interleaved gate_up plane with
 biases (libmir-metal clamped_routed ExpertLayout::DenseFused), 4-bit affine
-planes (mlxcel issue #974), and the latent variant (ferrox latent_moe.rs).
+planes (mlxcel issue #974), the latent variant (ferrox latent_moe.rs), and MXFP4
+planes in the clamped family's split layout (libmir-metal clamped_routed; element
+and scale encodings from the OCP Microscaling Formats v1.0 specification).
 """
 import numpy as np
 
@@ -36,9 +38,14 @@ SEPARATE_BIAS = MoeSpec(
     scoring="sigmoid", norm_topk_prob=False, has_expert_bias=True, weight_format="q4",
     group_size=32)
 LATENT_NONORM = LATENT.replace(name="t_latent_nonorm", config_id=107, latent_use_norm=False)
+# MXFP4 planes (OCP MX v1.0 encoding) in the clamped family's split layout, with biases
+MXFP4 = MoeSpec(
+    name="t_mxfp4", config_id=108, hidden=128, num_experts=5, top_k=2, intermediate=64,
+    scoring="softmax_topk", activation="swiglu_clamped", has_expert_bias=True,
+    weight_format="mxfp4", group_size=32)
 
 ALL = [inputs.TINY_F32, SIG_BLEND, CLAMPED, Q4, LATENT, ROUTER_BIAS, SEPARATE_BIAS,
-       LATENT_NONORM]
+       LATENT_NONORM, MXFP4]
 
 
 def np_weights(spec, scale_weights: float = 1.0):
