@@ -190,8 +190,7 @@ bool dense_tc(const moe_config* c, int64_t T, int K) {
 // kernels from there on, although most tiles then hold only a few tokens (Klear shape:
 // 8 tokens 149 vs 157 us, 64 tokens 279 vs 627 us; at 4 tokens the CUDA cores win).
 bool routed_tc(const moe_config* c, int64_t T) {
-    if (c->act_dtype != MOE_DTYPE_BF16 || c->weight_format == MOE_DTYPE_F32 || c->weight_format == MOE_DTYPE_MXFP4)
-        return false;
+    if (c->act_dtype != MOE_DTYPE_BF16 || c->weight_format == MOE_DTYPE_F32) return false;
     if (expert_in(*c) % 64 != 0 || c->intermediate % 64 != 0) return false;
     const int o = path_override();
     return o == kPathTc || (o == kPathAuto && 4 * T * c->top_k >= int64_t(c->num_experts));
@@ -387,8 +386,10 @@ moe_status run_experts_tc(const moe_config* c, const moe_weights* w, const void*
                 }
             }
             bool ok;
-            if (c->weight_format == MOE_DTYPE_Q4_AFFINE) {  // dequantised in the main loop
+            if (c->weight_format == MOE_DTYPE_Q4_AFFINE || c->weight_format == MOE_DTYPE_MXFP4) {
+                // packed 4-bit codes, dequantised in the main loop
                 p.q4 = 1;
+                p.mx = c->weight_format == MOE_DTYPE_MXFP4;
                 p.group_size = c->group_size;
                 p.qs0 = w->gate_s; p.qz0 = w->gate_z; p.qs1 = w->up_s; p.qz1 = w->up_z;
                 ok = tc_q4_weight_map(&P.a0[np], w->gate_w, E, I, K) && tc_q4_weight_map(&P.a1[np], w->up_w, E, I, K);
@@ -434,8 +435,9 @@ moe_status run_experts_tc(const moe_config* c, const moe_weights* w, const void*
             p.bias0 = c->has_expert_bias ? w->down_b : nullptr;
             p.out = at<__nv_bfloat16>(ws, L.oslot); p.ld_out = K;
             bool ok;
-            if (c->weight_format == MOE_DTYPE_Q4_AFFINE) {
+            if (c->weight_format == MOE_DTYPE_Q4_AFFINE || c->weight_format == MOE_DTYPE_MXFP4) {
                 p.q4 = 1;
+                p.mx = c->weight_format == MOE_DTYPE_MXFP4;
                 p.group_size = c->group_size;
                 p.qs0 = w->down_s; p.qz0 = w->down_z;
                 ok = tc_q4_weight_map(&P.a0[np], w->down_w, E, K, I);

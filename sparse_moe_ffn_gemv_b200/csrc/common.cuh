@@ -20,6 +20,7 @@ constexpr int kMaxExperts = 512;
 constexpr int kF32 = MOE_DTYPE_F32;
 constexpr int kBF16 = MOE_DTYPE_BF16;
 constexpr int kQ4 = MOE_DTYPE_Q4_AFFINE;
+constexpr int kMX4 = MOE_DTYPE_MXFP4;
 
 // ---------------------------------------------------------------- workspace
 // Every call carves its scratch out of the caller's workspace at fixed
@@ -99,6 +100,18 @@ template <typename AT> __device__ __forceinline__ AT from_f(float v);
 template <> __device__ __forceinline__ float from_f<float>(float v) { return v; }
 template <> __device__ __forceinline__ __nv_bfloat16 from_f<__nv_bfloat16>(float v) {
     return __float2bfloat16_rn(v);
+}
+
+// MXFP4 (OCP Microscaling Formats v1.0). An E2M1 code's exponent and mantissa bits, placed
+// at the bottom of a float's exponent field, give exactly the element value times 2^-126
+// (exponent field 0 is the format's subnormal, and so it is for the float): one exact
+// multiply restores it. The E8M0 block scale byte s is 2^(s - 127).
+__device__ __forceinline__ float e2m1_value(uint32_t code) {
+    const float mag = __uint_as_float((code & 7u) << 22) * 0x1p126f;
+    return __uint_as_float(__float_as_uint(mag) | ((code & 8u) << 28));
+}
+__device__ __forceinline__ float e8m0_value(uint32_t s) {
+    return __uint_as_float(s ? (s << 23) : 0x00400000u);  // 255 (NaN in the format) -> inf
 }
 
 // SwiGLU / clamped SwiGLU on fp32 pre-activations.

@@ -32,15 +32,18 @@ template <int WF> struct Fmt;
 template <> struct Fmt<kF32> { using AT = float; static constexpr int VE = 4, U = 4, DR = 2; };
 template <> struct Fmt<kBF16> { using AT = __nv_bfloat16; static constexpr int VE = 8, U = 4, DR = 2; };
 template <> struct Fmt<kQ4> { using AT = __nv_bfloat16; static constexpr int VE = 32, U = 2, DR = 1; };
+template <> struct Fmt<kMX4> { using AT = __nv_bfloat16; static constexpr int VE = 32, U = 2, DR = 1; };
+template <int WF> constexpr bool is_4bit() { return WF == kQ4 || WF == kMX4; }
 
 // Row pointer of a weight matrix row in a given format (bytes per row).
 template <int WF> __host__ __device__ __forceinline__ int64_t row_bytes(int K) {
     return WF == kF32 ? int64_t(K) * 4 : (WF == kBF16 ? int64_t(K) * 2 : int64_t(K) / 2);
 }
 
-struct QRow {  // 4-bit companions of one row: bf16 scale / bias per group
-    const __nv_bfloat16* s;
-    const __nv_bfloat16* z;
+struct QRow {  // 4-bit companions of one row
+    const __nv_bfloat16* s;  // affine: bf16 scale per group
+    const __nv_bfloat16* z;  // affine: bf16 bias per group
+    const uint8_t* e8;       // MXFP4: E8M0 scale byte per block of 32
 };
 
 // acc[r][t] += sum_c W_r[c] * u_t[c] for NR rows and tt (<= kTT) staged tokens.
@@ -92,6 +95,35 @@ __device__ __forceinline__ void dot_rows(const char* const (&rows)[NR], const QR
                         acc[r][t] = fmaf(__uint_as_float(wv[r][u].z), xv.z, acc[r][t]);
                         acc[r][t] = fmaf(__uint_as_float(wv[r][u].w), xv.w, acc[r][t]);
                     }
+                }
+            } else if constexpr (WF == kMX4) {  // one vector = one block of 32: sum_j e_j x_j times 2^(s-127)
+                float qf[NR][32], sc[NR];
+#pragma unroll
+                for (int r = 0; r < NR; ++r) {
+                    sc[r] = e8m0_value(q[r].e8[v]);
+                    const uint32_t words[4] = {wv[r][u].x, wv[r][u].y, wv[r][u].z, wv[r][u].w};
+#pragma unroll
+                    for (int i = 0; i < 4; ++i)
+#pragma unroll
+                        for (int n = 0; n < 8; ++n) qf[r][i * 8 + n] = e2m1_value(words[i] >> (4 * n));
+                }
+#pragma unroll
+                for (int t = 0; t < kTT; ++t) {
+                    if (t >= tt) break;
+                    float dq[NR];
+#pragma unroll
+                    for (int r = 0; r < NR; ++r) dq[r] = 0.f;
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        float xf[8];
+                        unpack8(*reinterpret_cast<const uint4*>(us + int64_t(t) * K + c0 + 8 * i), xf);
+#pragma unroll
+                        for (int r = 0; r < NR; ++r)
+#pragma unroll
+                            for (int n = 0; n < 8; ++n) dq[r] = fmaf(qf[r][i * 8 + n], xf[n], dq[r]);
+                    }
+#pragma unroll
+                    for (int r = 0; r < NR; ++r) acc[r][t] = fmaf(sc[r], dq[r], acc[r][t]);
                 }
             } else {  // 4-bit affine: sum_j (s q_j + b) x_j = s * sum_j q_j x_j + b * sum_j x_j
                 const int grp = c0 / group_size;
@@ -193,7 +225,7 @@ __device__ void gateup_group(const GateUpArgs& a, bool shared, int e, int unit0,
     const int i = unit0 + warp;
     const bool live = i < I;
     const char* rows[2];
-    QRow q[2] = {{nullptr, nullptr}, {nullptr, nullptr}};
+    QRow q[2] = {{nullptr, nullptr, nullptr}, {nullptr, nullptr, nullptr}};
     const int64_t rb = row_bytes<WF>(K);
     if (shared) {
         rows[0] = reinterpret_cast<const char*>(a.sg_w) + int64_t(live ? i : 0) * rb;
@@ -209,9 +241,12 @@ __device__ void gateup_group(const GateUpArgs& a, bool shared, int e, int unit0,
         if constexpr (WF == kQ4) {
             const int64_t ng = K / a.group_size;
             q[0] = {reinterpret_cast<const __nv_bfloat16*>(a.gate_s) + r0 * ng,
-                    reinterpret_cast<const __nv_bfloat16*>(a.gate_z) + r0 * ng};
+                    reinterpret_cast<const __nv_bfloat16*>(a.gate_z) + r0 * ng, nullptr};
             q[1] = {reinterpret_cast<const __nv_bfloat16*>(a.up_s) + r0 * ng,
-                    reinterpret_cast<const __nv_bfloat16*>(a.up_z) + r0 * ng};
+                    reinterpret_cast<const __nv_bfloat16*>(a.up_z) + r0 * ng, nullptr};
+        } else if constexpr (WF == kMX4) {
+            q[0] = {nullptr, nullptr, reinterpret_cast<const uint8_t*>(a.gate_s) + r0 * (K / 32)};
+            q[1] = {nullptr, nullptr, reinterpret_cast<const uint8_t*>(a.up_s) + r0 * (K / 32)};
         }
     }
     float bg = 0.f, bu = 0.f;
@@ -251,7 +286,7 @@ __device__ void gateup_group(const GateUpArgs& a, bool shared, int e, int unit0,
 template <int WF>
 __global__ void __launch_bounds__(kThreads) gateup_gemv_kernel(GateUpArgs a) {
     pdl_begin();
-    constexpr int WFD = (WF == kQ4) ? kBF16 : WF;  // the shared expert is dense
+    constexpr int WFD = is_4bit<WF>() ? kBF16 : WF;  // the shared expert is dense
     using AT = typename Fmt<WF>::AT;
     extern __shared__ uint4 smem_raw[];
     AT* us = reinterpret_cast<AT*>(smem_raw);
@@ -288,7 +323,7 @@ __device__ void down_group(const DownArgs& a, bool shared, int e, int row0, int6
     for (int i = 0; i < NR; ++i) {
         const int r = rbase + i;
         live[i] = r < R;
-        q[i] = {nullptr, nullptr};
+        q[i] = {nullptr, nullptr, nullptr};
         bd[i] = 0.f;
         if (shared) {
             rows[i] = reinterpret_cast<const char*>(a.sd_w) + int64_t(live[i] ? r : 0) * rb;
@@ -298,7 +333,9 @@ __device__ void down_group(const DownArgs& a, bool shared, int e, int row0, int6
             if constexpr (WF == kQ4) {
                 const int64_t ng = I / a.group_size;
                 q[i] = {reinterpret_cast<const __nv_bfloat16*>(a.down_s) + gr * ng,
-                        reinterpret_cast<const __nv_bfloat16*>(a.down_z) + gr * ng};
+                        reinterpret_cast<const __nv_bfloat16*>(a.down_z) + gr * ng, nullptr};
+            } else if constexpr (WF == kMX4) {
+                q[i] = {nullptr, nullptr, reinterpret_cast<const uint8_t*>(a.down_s) + gr * (I / 32)};
             }
             if (a.has_bias && live[i]) bd[i] = ld_act<AT>(a.down_b, gr);
         }
@@ -348,7 +385,7 @@ __device__ void down_group(const DownArgs& a, bool shared, int e, int row0, int6
 template <int WF>
 __global__ void __launch_bounds__(kThreads) down_gemv_kernel(DownArgs a) {
     pdl_begin();
-    constexpr int WFD = (WF == kQ4) ? kBF16 : WF;
+    constexpr int WFD = is_4bit<WF>() ? kBF16 : WF;
     using AT = typename Fmt<WF>::AT;
     extern __shared__ uint4 smem_raw[];
     AT* us = reinterpret_cast<AT*>(smem_raw);
@@ -389,7 +426,7 @@ __global__ void __launch_bounds__(kThreads) dense_gemv_kernel(DenseGemvArgs a) {
     const void* W = r < a.rows0 ? a.W0 : a.W1;
     const void* bias = r < a.rows0 ? a.b0 : a.b1;
     const char* rowp[1] = {reinterpret_cast<const char*>(W) + int64_t(rr) * row_bytes<WF>(a.K)};
-    QRow q[1] = {{nullptr, nullptr}};
+    QRow q[1] = {{nullptr, nullptr, nullptr}};
     float acc[1][kTT];
 #pragma unroll
     for (int t = 0; t < kTT; ++t) acc[0][t] = 0.f;
@@ -427,7 +464,7 @@ size_t stage_bytes(int wf, int K) {
 
 template <int WF>
 cudaError_t launch_gateup_t(const GateUpArgs& a, cudaStream_t s) {
-    constexpr int WFD = (WF == kQ4) ? kBF16 : WF;
+    constexpr int WFD = is_4bit<WF>() ? kBF16 : WF;
     const size_t smem = std::max(stage_bytes(WF, a.K), a.shared_I ? stage_bytes(WFD, a.Hs) : size_t(0));
     cudaError_t err = set_smem(gateup_gemv_kernel<WF>, smem);
     if (err != cudaSuccess) return err;
@@ -441,7 +478,7 @@ cudaError_t launch_gateup_t(const GateUpArgs& a, cudaStream_t s) {
 
 template <int WF>
 cudaError_t launch_down_t(const DownArgs& a, cudaStream_t s) {
-    constexpr int WFD = (WF == kQ4) ? kBF16 : WF;
+    constexpr int WFD = is_4bit<WF>() ? kBF16 : WF;
     const size_t smem = std::max(stage_bytes(WF, a.I), a.shared_I ? stage_bytes(WFD, a.shared_I) : size_t(0));
     cudaError_t err = set_smem(down_gemv_kernel<WF>, smem);
     if (err != cudaSuccess) return err;
@@ -461,6 +498,7 @@ cudaError_t launch_gateup_gemv(const GateUpArgs& a, cudaStream_t s) {
         case kF32: return launch_gateup_t<kF32>(a, s);
         case kBF16: return launch_gateup_t<kBF16>(a, s);
         case kQ4: return launch_gateup_t<kQ4>(a, s);
+        case kMX4: return launch_gateup_t<kMX4>(a, s);
         default: return cudaErrorInvalidValue;
     }
 }
@@ -470,6 +508,7 @@ cudaError_t launch_down_gemv(const DownArgs& a, cudaStream_t s) {
         case kF32: return launch_down_t<kF32>(a, s);
         case kBF16: return launch_down_t<kBF16>(a, s);
         case kQ4: return launch_down_t<kQ4>(a, s);
+        case kMX4: return launch_down_t<kMX4>(a, s);
         default: return cudaErrorInvalidValue;
     }
 }

@@ -123,6 +123,7 @@ struct TcProblem {
     // of the first (gate or single) and second (up) weight plane
     int q4 = 0, group_size = 64;
     const void *qs0 = nullptr, *qz0 = nullptr, *qs1 = nullptr, *qz1 = nullptr;
+    int mx = 0;  // with q4 = 1: MXFP4 codes, qs0 / qs1 the E8M0 scale bytes [groups, M, K / 32]
 };
 
 struct alignas(64) TcParams {

@@ -210,6 +210,29 @@ __device__ __forceinline__ uint4 dequant8(uint32_t w, __nv_bfloat162 s2, __nv_bf
     return make_uint4(r[0], r[1], r[2], r[3]);
 }
 
+// Eight MXFP4 codes (OCP MX v1.0 E2M1, element j in bits 4j..4j+3) -> eight bf16 weights
+// element * 2^(block scale). A code's exponent and mantissa bits placed at the bottom of a
+// bf16 exponent field give exactly the element times 2^-126 (subnormal at exponent 0, as in
+// the format); two exact power-of-two multiplies (2^126, then the block scale) finish.
+__device__ __forceinline__ uint4 dequant8_mx(uint32_t w, __nv_bfloat162 scale2) {
+    uint32_t p[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {  // (code_i, code_i+4) as bf16 bit patterns
+        const uint32_t c = (w >> (4 * i)) & 0x000F000Fu;
+        p[i] = ((c & 0x00080008u) << 12) | ((c & 0x00070007u) << 6);
+    }
+    const uint32_t o[4] = {__byte_perm(p[0], p[1], 0x5410), __byte_perm(p[2], p[3], 0x5410),
+                           __byte_perm(p[0], p[1], 0x7632), __byte_perm(p[2], p[3], 0x7632)};
+    const __nv_bfloat162 two126 = __halves2bfloat162(__ushort_as_bfloat16(0x7E80), __ushort_as_bfloat16(0x7E80));
+    uint32_t r[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const __nv_bfloat162 v = __hmul2(__hmul2(*reinterpret_cast<const __nv_bfloat162*>(&o[i]), two126), scale2);
+        r[i] = *reinterpret_cast<const uint32_t*>(&v);
+    }
+    return make_uint4(r[0], r[1], r[2], r[3]);
+}
+
 // Byte offset of row r's 16-byte chunk c (8 bf16 of one 64-wide K block) in a 128-row
 // operand tile with the 128-byte swizzle the MMA descriptor expects (8-row atoms of 1 KB,
 // chunk index XOR row within the atom).
@@ -416,24 +439,34 @@ __global__ void __launch_bounds__(TcShape<GATEUP, BN, STAGES, Q4>::THREADS, 1)
             const int ng = p.K / p.group_size;
             // this thread's row of each weight tile in its scale / bias planes (rows past M
             // read row M - 1: their results are discarded)
-            const __nv_bfloat16* sp[2];
-            const __nv_bfloat16* zp[2];
+            // (byte addresses: bf16 scales and biases, or MXFP4's one-byte scales and no biases)
+            const unsigned char* sp[2];
+            const unsigned char* zp[2];
 #pragma unroll
             for (int a = 0; a < 2; ++a) {
                 const int r = min(ti.mb * S::ROWS + (GATEUP ? 0 : a * kBM) + d, p.M - 1);
                 const int64_t off = (int64_t(ti.group) * p.M + r) * ng;
-                sp[a] = static_cast<const __nv_bfloat16*>((GATEUP && a == 1) ? p.qs1 : p.qs0) + off;
-                zp[a] = static_cast<const __nv_bfloat16*>((GATEUP && a == 1) ? p.qz1 : p.qz0) + off;
+                sp[a] = static_cast<const unsigned char*>((GATEUP && a == 1) ? p.qs1 : p.qs0) + off * (p.mx ? 1 : 2);
+                zp[a] = p.mx ? nullptr : static_cast<const unsigned char*>((GATEUP && a == 1) ? p.qz1 : p.qz0) + off * 2;
             }
             // (scale, bias) of tile a for the first and second half of K block kb (two
             // groups per block when group_size is 32, else the same group twice)
+            // (MXFP4: the scale planes hold one E8M0 byte per block of 32 at the same offsets;
+            // the pair then carries 2^(byte - 127) as bf16 twice)
             auto load_sb = [&](int kb, __nv_bfloat162 (&o)[2][2]) {
 #pragma unroll
                 for (int a = 0; a < 2; ++a)
 #pragma unroll
                     for (int h = 0; h < 2; ++h) {
                         const int g = (kb * kBK + h * 32) / p.group_size;
-                        o[a][h] = __halves2bfloat162(__ldg(sp[a] + g), __ldg(zp[a] + g));
+                        if (p.mx) {
+                            const uint32_t sbyte = __ldg(sp[a] + g);
+                            const __nv_bfloat16 sc = __ushort_as_bfloat16(uint16_t(sbyte ? (sbyte << 7) : 0x0040u));
+                            o[a][h] = __halves2bfloat162(sc, sc);
+                        } else {
+                            o[a][h] = __halves2bfloat162(__ldg(reinterpret_cast<const __nv_bfloat16*>(sp[a]) + g),
+                                                         __ldg(reinterpret_cast<const __nv_bfloat16*>(zp[a]) + g));
+                        }
                     }
             };
             __nv_bfloat162 q0[2][2], q1[2][2];
@@ -455,7 +488,8 @@ __global__ void __launch_bounds__(TcShape<GATEUP, BN, STAGES, Q4>::THREADS, 1)
 #pragma unroll
                     for (int c = 0; c < 8; ++c) {
                         const __nv_bfloat162 sbv = q0[a][c >> 2];
-                        const uint4 v = dequant8(words[c], __low2bfloat162(sbv), __high2bfloat162(sbv));
+                        const uint4 v = p.mx ? dequant8_mx(words[c], sbv)
+                                             : dequant8(words[c], __low2bfloat162(sbv), __high2bfloat162(sbv));
                         *reinterpret_cast<uint4*>(sb + a * S::A_BYTES + sw128_offset(d, c)) = v;
                     }
                 }

@@ -154,8 +154,10 @@ def quantize_affine_q4(w: torch.Tensor, group_size: int):
     return torch.from_numpy(packed.copy()), scale.contiguous(), bias.contiguous()
 
 
-# E2M1 magnitudes by the low three bits of a code (OCP Microscaling Formats v1.0).
+# E2M1 magnitudes by the low three bits of a code (OCP Microscaling Formats v1.0), and the
+# midpoints between neighbours (a magnitude rounds to the index of the first midpoint >= it).
 _E2M1 = torch.tensor([0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0])
+_E2M1_MID = (_E2M1[1:] + _E2M1[:-1]) / 2
 
 
 def quantize_mxfp4(w: torch.Tensor):
@@ -175,7 +177,7 @@ def quantize_mxfp4(w: torch.Tensor):
     x = torch.floor(torch.log2(amax)) - 2.0
     sbyte = (x + 127).clamp(1, 254)
     v = (g / torch.exp2(sbyte - 127).unsqueeze(-1)).clamp(-6.0, 6.0)
-    idx = (v.abs().unsqueeze(-1) - _E2M1).abs().argmin(dim=-1)  # first minimum: smaller magnitude
+    idx = torch.bucketize(v.abs(), _E2M1_MID)  # nearest E2M1 magnitude; a tie keeps the smaller
     code = idx + torch.where(v < 0, 8, 0) * (idx > 0)
     code = code.to(torch.int64).reshape(*lead, k // 8, 8)
     shifts = torch.arange(8, dtype=torch.int64) * 4

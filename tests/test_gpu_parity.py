@@ -81,6 +81,9 @@ SMALL = [
     (inputs.CLAMPED_BF16, 8, 8.0),       # clamp stress: x * 8 engages the +-7 clamp
     (inputs.LATENT_BF16, 1, 1.0),
     (inputs.LATENT_BF16, 9, 1.0),
+    (ts.MXFP4, 9, 30.0),                 # MXFP4 planes (tensor cores: 4 T k >= E)
+    (inputs.CLAMPED_MXFP4, 1, 1.0),      # weight-streaming kernels
+    (inputs.CLAMPED_MXFP4, 8, 8.0),      # tensor cores, clamp engaged
 ]
 
 
@@ -95,6 +98,7 @@ FULL = [  # (spec, T, sampled tokens for the output check)
     (inputs.CLAMPED_BF16, 8192, 16),
     (inputs.LATENT_BF16, 128, 24),
     (inputs.LATENT_BF16, 8192, 8),
+    (inputs.CLAMPED_MXFP4, 8192, 12),
 ]
 
 
@@ -234,7 +238,21 @@ TC_SMALL = [  # tensor-core path forced: ragged groups, partial tiles, interleav
     (inputs.LATENT_BF16, 9),
     (inputs.KLEAR_Q4, 3),
     (inputs.KLEAR_Q4, 150),
+    (inputs.CLAMPED_MXFP4, 5),
 ]
+
+
+GEMV_SMALL = [  # weight-streaming kernels forced where the auto rule picks the tensor cores
+    (ts.MXFP4, 9),
+    (inputs.CLAMPED_MXFP4, 20),
+    (inputs.KLEAR_Q4, 20),
+]
+
+
+@pytest.mark.parametrize("spec,T", GEMV_SMALL, ids=[f"{s.name}-T{T}" for s, T in GEMV_SMALL])
+def test_weight_streaming_path_matches_oracle(spec, T, monkeypatch):
+    monkeypatch.setenv("MOE_PATH", "gemv")
+    full_check(spec, T)
 
 
 @pytest.mark.parametrize("spec,T", TC_SMALL, ids=[f"{s.name}-T{T}" for s, T in TC_SMALL])
@@ -244,8 +262,9 @@ def test_tensor_core_path_matches_oracle(spec, T, monkeypatch):
 
 
 @pytest.mark.parametrize("spec,T", [(inputs.KLEAR_BF16, 96), (inputs.CLAMPED_BF16, 64),
-                                    (inputs.LATENT_BF16, 64), (inputs.KLEAR_Q4, 96)],
-                         ids=["klear", "clamped", "latent", "klear_q4"])
+                                    (inputs.LATENT_BF16, 64), (inputs.KLEAR_Q4, 96),
+                                    (inputs.CLAMPED_MXFP4, 48)],
+                         ids=["klear", "clamped", "latent", "klear_q4", "clamped_mxfp4"])
 def test_weight_streaming_and_tensor_core_paths_agree(spec, T, monkeypatch):
     """The decode-sized engine and the batched engine give the same block output
     (cf. the Klear PR's caveat on a fused decode kernel that was not byte-identical)."""
