@@ -289,7 +289,7 @@ moe_status run_route(const moe_config* c, const moe_weights* w, const void* x, i
             p.out = at<float>(ws, L.logits) + (i == 0 ? 0 : c->num_experts);
             p.ld_out = L.ld_logits;
             if (!tc_weight_map(&P.a0[i], i == 0 ? r.W0 : r.W1, 1, p.M, c->hidden, false) ||
-                !tc_token_map(&P.b[i], x, T, c->hidden, kTcBN))
+                !tc_token_map(P.b[i], x, T, c->hidden, kTcBN))
                 return MOE_ERR_CUDA;
         }
         P.nprob = np;
@@ -364,7 +364,7 @@ moe_status run_experts_tc(const moe_config* c, const moe_weights* w, const void*
             p.out = hs; p.ld_out = Is;
             if (!tc_weight_map(&P.a0[np], w->shared_gate_w, 1, Is, H, false) ||
                 !tc_weight_map(&P.a1[np], w->shared_up_w, 1, Is, H, false) ||
-                !tc_token_map(&P.b[np], x, T, H, kTcBN))
+                !tc_token_map(P.b[np], x, T, H, kTcBN))
                 return MOE_ERR_CUDA;
             max_tiles += int64_t(p.m_blocks) * p.n_tiles;
             ++np;
@@ -399,7 +399,7 @@ moe_status run_experts_tc(const moe_config* c, const moe_weights* w, const void*
                 ok = tc_weight_map(&P.a0[np], w->gate_w, E, I, K, false) &&
                      tc_weight_map(&P.a1[np], w->up_w, E, I, K, false);
             }
-            if (!ok || !tc_token_map(&P.b[np], uperm, S, K, kTcBN)) return MOE_ERR_CUDA;
+            if (!ok || !tc_token_map(P.b[np], uperm, S, K, kTcBN)) return MOE_ERR_CUDA;
             max_tiles += int64_t(p.m_blocks) * max_routed_tiles(*c, T);
             ++np;
         }
@@ -421,7 +421,7 @@ moe_status run_experts_tc(const moe_config* c, const moe_weights* w, const void*
             p.rows = int(T); p.n_tiles = int(n_dense);
             p.out = at<float>(ws, L.s_acc); p.ld_out = H;
             if (!tc_weight_map(&P.a0[np], w->shared_down_w, 1, H, Is, false) ||
-                !tc_token_map(&P.b[np], hs, T, Is, kTcBN))
+                !tc_token_map(P.b[np], hs, T, Is, kTcBN))
                 return MOE_ERR_CUDA;
             max_tiles += int64_t(p.m_blocks) * p.n_tiles;
             ++np;
@@ -444,7 +444,7 @@ moe_status run_experts_tc(const moe_config* c, const moe_weights* w, const void*
             } else {
                 ok = tc_weight_map(&P.a0[np], w->down_w, E, K, I, false);
             }
-            if (!ok || !tc_token_map(&P.b[np], h, S, I, kTcBN)) return MOE_ERR_CUDA;
+            if (!ok || !tc_token_map(P.b[np], h, S, I, kTcBN)) return MOE_ERR_CUDA;
             max_tiles += int64_t(p.m_blocks) * max_routed_tiles(*c, T);
             ++np;
         }
@@ -561,7 +561,7 @@ moe_status run_latent_down(const moe_config* c, const moe_weights* w, const void
         p.M = c->latent_dim; p.K = c->hidden; p.m_blocks = (p.M + kTcRows - 1) / kTcRows;
         p.rows = int(T); p.n_tiles = int((T + kTcBN - 1) / kTcBN);
         p.out = z; p.ld_out = c->latent_dim;
-        if (!tc_weight_map(&P.a0[0], w->latent_down_w, 1, p.M, p.K, false) || !tc_token_map(&P.b[0], x, T, p.K, kTcBN))
+        if (!tc_weight_map(&P.a0[0], w->latent_down_w, 1, p.M, p.K, false) || !tc_token_map(P.b[0], x, T, p.K, kTcBN))
             return MOE_ERR_CUDA;
         P.nprob = 1;
         P.status = status;
@@ -611,7 +611,7 @@ moe_status run_output(const moe_config* c, const moe_weights* w, RoutedSum rs, c
         p.rows = int(T); p.n_tiles = int((T + kTcBN - 1) / kTcBN);
         p.out = y; p.ld_out = c->hidden;
         p.addend = s_acc; p.ld_add = c->hidden;
-        if (!tc_weight_map(&P.a0[0], w->latent_up_w, 1, p.M, p.K, false) || !tc_token_map(&P.b[0], n, T, p.K, kTcBN))
+        if (!tc_weight_map(&P.a0[0], w->latent_up_w, 1, p.M, p.K, false) || !tc_token_map(P.b[0], n, T, p.K, kTcBN))
             return MOE_ERR_CUDA;
         P.nprob = 1;
         P.status = at<int>(ws, L.status);

@@ -134,7 +134,8 @@ struct alignas(64) TcParams {
     }
     CUtensorMap a0[2];  // weights (gate / single)
     CUtensorMap a1[2];  // weights (up), gate/up mode with separate planes
-    CUtensorMap b[2];   // tokens
+    CUtensorMap b[2][4];  // tokens, boxes of 16, 32, 64 and 128 rows (a tile loads the smallest
+                          // box that holds its valid tokens)
     TcProblem p[2];
     int nprob = 0;
     int* status = nullptr;
@@ -146,6 +147,7 @@ bool tc_weight_map(CUtensorMap* m, const void* w, int E, int R, int K, bool inte
 // Packed 4-bit weight operand: [E, R, K / 8] uint32 words (8 codes each), one 64-wide K block
 // (8 words) x 128 rows per box, no swizzle (the kernel's dequantising warps read it).
 bool tc_q4_weight_map(CUtensorMap* m, const void* w, int E, int R, int K);
+// Four maps m[0..3] of the token operand [rows, K] bf16, boxes of 16, 32, 64 and bn rows.
 bool tc_token_map(CUtensorMap* m, const void* u, int64_t rows, int K, int bn);
 cudaError_t launch_tc_gemm(TcParams& P, bool gateup, int64_t max_tiles, cudaStream_t s);
 

@@ -25,6 +25,7 @@
 // routing.weights and summed; ferrox KimiExpertWeights::forward: down(act(gate, up))).
 #include <cuda.h>
 
+#include <algorithm>
 #include <mutex>
 #include <type_traits>
 
@@ -284,7 +285,7 @@ __global__ void __launch_bounds__(TcShape<GATEUP, BN, STAGES, Q4>::THREADS, 1)
         for (int i = 0; i < P.nprob; ++i) {
             prefetch_tmap(&P.a0[i]);
             if (GATEUP && !P.p[i].interleaved) prefetch_tmap(&P.a1[i]);
-            prefetch_tmap(&P.b[i]);
+            for (int v = 0; v < 4; ++v) prefetch_tmap(&P.b[i][v]);
         }
     }
     pdl_begin();  // everything above touches no memory that earlier kernels write
@@ -324,8 +325,11 @@ __global__ void __launch_bounds__(TcShape<GATEUP, BN, STAGES, Q4>::THREADS, 1)
                     uint8_t* sb = smem + stage * S::STAGE_BYTES;
                     const int kc = kb * kBK;
                     const int mrow = ti.mb * S::ROWS;
+                    // token rows: the smallest box (16, 32, 64, BN) that holds the valid tokens
+                    const int bv = ti.nvalid <= 16 ? 0 : ti.nvalid <= 32 ? 1 : ti.nvalid <= 64 ? 2 : 3;
+                    const uint32_t b_bytes = uint32_t(min(BN, 16 << bv)) * kBK * 2;
                     if (Q4 && p.q4) {  // packed words of the two weight tiles (8 words per K block)
-                        mbar_expect_tx(&full[stage], 2 * kPkBytes + S::B_BYTES);
+                        mbar_expect_tx(&full[stage], 2 * kPkBytes + b_bytes);
                         uint8_t* pk = sb + S::PK_OFF;
                         if (!GATEUP) {
                             tma_3d(pk, &P.a0[ti.prob], &full[stage], kb * 8, mrow, ti.group, pol_w);
@@ -335,19 +339,19 @@ __global__ void __launch_bounds__(TcShape<GATEUP, BN, STAGES, Q4>::THREADS, 1)
                             tma_3d(pk + kPkBytes, &P.a1[ti.prob], &full[stage], kb * 8, mrow, ti.group, pol_w);
                         }
                     } else if (!GATEUP) {  // rows [mrow, mrow + 128) and [mrow + 128, mrow + 256)
-                        mbar_expect_tx(&full[stage], 2 * S::A_BYTES + S::B_BYTES);
+                        mbar_expect_tx(&full[stage], 2 * S::A_BYTES + b_bytes);
                         tma_3d(sb, &P.a0[ti.prob], &full[stage], kc, mrow, ti.group, pol_w);
                         tma_3d(sb + S::A_BYTES, &P.a0[ti.prob], &full[stage], kc, mrow + kBM, ti.group, pol_w);
                     } else if (p.interleaved) {  // [E, I, 2, K]: plane 0 = gate rows, 1 = up rows
-                        mbar_expect_tx(&full[stage], 2 * S::A_BYTES + S::B_BYTES);
+                        mbar_expect_tx(&full[stage], 2 * S::A_BYTES + b_bytes);
                         tma_4d(sb, &P.a0[ti.prob], &full[stage], kc, 0, mrow, ti.group, pol_w);
                         tma_4d(sb + S::A_BYTES, &P.a0[ti.prob], &full[stage], kc, 1, mrow, ti.group, pol_w);
                     } else {
-                        mbar_expect_tx(&full[stage], 2 * S::A_BYTES + S::B_BYTES);
+                        mbar_expect_tx(&full[stage], 2 * S::A_BYTES + b_bytes);
                         tma_3d(sb, &P.a0[ti.prob], &full[stage], kc, mrow, ti.group, pol_w);
                         tma_3d(sb + S::A_BYTES, &P.a1[ti.prob], &full[stage], kc, mrow, ti.group, pol_w);
                     }
-                    tma_2d(sb + 2 * S::A_BYTES, &P.b[ti.prob], &full[stage], kc, ti.row0, pol_t);
+                    tma_2d(sb + 2 * S::A_BYTES, &P.b[ti.prob][bv], &full[stage], kc, ti.row0, pol_t);
                     armed |= 1u << stage;
                     last_par = (last_par & ~(1u << stage)) | (phase << stage);
                     if (++stage == STAGES) {
@@ -746,12 +750,15 @@ bool tc_weight_map(CUtensorMap* m, const void* w, int E, int R, int K, bool inte
     return encode(m, w, 3, dims, strides, box);
 }
 
-// Token operand: [rows, K] bf16, box of bn rows.
+// Token operand: [rows, K] bf16, maps m[0..3] with boxes of 16, 32, 64 and bn rows.
 bool tc_token_map(CUtensorMap* m, const void* u, int64_t rows, int K, int bn) {
     const cuuint64_t dims[2] = {cuuint64_t(K), cuuint64_t(rows)};
     const cuuint64_t strides[1] = {cuuint64_t(K) * 2};
-    const cuuint32_t box[2] = {kBK, cuuint32_t(bn)};
-    return encode(m, u, 2, dims, strides, box);
+    for (int v = 0; v < 4; ++v) {
+        const cuuint32_t box[2] = {kBK, cuuint32_t(std::min(bn, 16 << v))};
+        if (!encode(&m[v], u, 2, dims, strides, box)) return false;
+    }
+    return true;
 }
 
 // Packed 4-bit plane [E, R, K / 8] uint32 (K % 64 == 0): box of 8 words x 128 rows.
