@@ -242,6 +242,14 @@ MOE_API moe_status moe_read_device_status(void *ws, moe_stream_t stream);
 /* Clears the workspace's 256-byte status region, asynchronously on `stream`. */
 MOE_API moe_status moe_clear_device_status(void *ws, moe_stream_t stream);
 
+/* Failure-detection self test: one CTA waits on an mbarrier that nothing ever
+ * completes, with the bounded wait every kernel of the library uses (a
+ * %globaltimer deadline of timeout_ns, 0 < timeout_ns <= 1e9). When it gives up
+ * it records MOE_ERR_DEVICE_TIMEOUT in the status word of `ws` (read it with
+ * moe_read_device_status) and returns; nothing traps or hangs. Asynchronous on
+ * `stream`; MOE_ERR_INVALID_ARGUMENT for a NULL ws or an out-of-range timeout. */
+MOE_API moe_status moe_selftest_bounded_wait(void *ws, int64_t timeout_ns, moe_stream_t stream);
+
 /* Static, NUL-terminated description of a status code. */
 MOE_API const char *moe_status_string(moe_status status);
 

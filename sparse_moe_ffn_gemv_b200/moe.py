@@ -30,7 +30,7 @@ EXPORTS = [
     "moe_config_validate", "moe_weights_validate", "moe_workspace_size", "moe_route",
     "moe_permute", "moe_grouped_ffn", "moe_latent_down", "moe_combine", "moe_block_forward",
     "moe_read_device_status", "moe_clear_device_status", "moe_status_string",
-    "moe_permute_noalloc",
+    "moe_permute_noalloc", "moe_selftest_bounded_wait",
 ]
 
 STATUS = {0: "MOE_OK", 1: "MOE_ERR_INVALID_ARGUMENT", 2: "MOE_ERR_SHAPE_OVERFLOW",
@@ -92,6 +92,7 @@ def lib():
             "moe_read_device_status": [vp, vp],
             "moe_clear_device_status": [vp, vp],
             "moe_permute_noalloc": [cfgp, vp, i64, vp, vp, vp, vp, vp],
+            "moe_selftest_bounded_wait": [vp, i64, vp],
         }
         for name, args in sig.items():
             fn = getattr(L, name)
@@ -205,6 +206,11 @@ def moe_permute_noalloc(cfg, topk_idx, T, expert_offsets, sorted_slot, slot_pos,
     _check(lib().moe_permute_noalloc(ctypes.byref(cfg), _p(topk_idx), int(T), _p(expert_offsets),
                                      _p(sorted_slot), _p(slot_pos), _p(device_status), _stream(stream)),
            "moe_permute_noalloc")
+
+
+def moe_selftest_bounded_wait(ws, timeout_ns: int, stream=None):
+    """Run the bounded-wait self test: records MOE_ERR_DEVICE_TIMEOUT in ws's status word."""
+    _check(lib().moe_selftest_bounded_wait(_p(ws), int(timeout_ns), _stream(stream)), "moe_selftest_bounded_wait")
 
 
 def moe_read_device_status(ws, stream=None) -> int:

@@ -32,7 +32,7 @@ def declared_symbols():
 
 def test_library_exports_every_declared_symbol():
     names = declared_symbols()
-    assert len(names) == 13
+    assert len(names) == 14
     assert sorted(M.EXPORTS) == names
     lib = M.lib()
     for n in names:
@@ -214,6 +214,14 @@ def test_noalloc_permutation_rejects_sizes_beyond_its_fixed_scratch():
     assert lib.moe_permute_noalloc(ctypes.byref(cfg), p, 0, p, p, p, None, None) == 0
     assert M.STATUS[lib.moe_permute_noalloc(ctypes.byref(_cfg(top_k=0)), p, 4, p, p, p, None, None)] == \
         "MOE_ERR_INVALID_ARGUMENT"
+
+
+def test_selftest_rejects_bad_arguments_before_any_launch():
+    lib = M.lib()
+    assert M.STATUS[lib.moe_selftest_bounded_wait(None, 1000, None)] == "MOE_ERR_INVALID_ARGUMENT"
+    for ns in (0, -5, 2_000_000_000):
+        assert M.STATUS[lib.moe_selftest_bounded_wait(ctypes.c_void_p(1 << 20), ns, None)] == \
+            "MOE_ERR_INVALID_ARGUMENT"
 
 
 def test_status_strings():

@@ -307,3 +307,19 @@ def test_routed_sum_in_fp32_meets_the_plain_bar(path, monkeypatch):
     assert np.array_equal(np.sort(idx.cpu().numpy(), 1), np.sort(ref["idx"], 1))
     rms = np.sqrt(np.mean(ref["y"] ** 2))
     assert np.abs(y_acc.cpu().numpy() - ref["y"]).max() <= 2e-2 * rms
+
+
+def test_bounded_device_wait_reports_a_timeout_and_the_context_stays_usable():
+    """A wait that can never complete gives up after its bound, records
+    MOE_ERR_DEVICE_TIMEOUT in the status word, and the next block forward works."""
+    spec = inputs.KLEAR_BF16
+    wcpu, _ = weights(spec)
+    blk = M.MoeBlock(spec, wcpu, max_tokens=8)
+    M.moe_clear_device_status(blk.ws)
+    M.moe_selftest_bounded_wait(blk.ws, 2_000_000)           # 2 ms
+    assert M.STATUS[blk.device_status()] == "MOE_ERR_DEVICE_TIMEOUT"
+    assert blk.device_status() == 0                          # reading clears it
+    x = inputs.make_x(spec, 8).cuda()
+    y = blk.forward(x)
+    torch.cuda.synchronize()
+    assert blk.device_status() == 0 and bool(torch.isfinite(y.float()).all())
