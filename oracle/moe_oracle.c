@@ -37,7 +37,9 @@
  *    Microscaling Formats (MX) Specification v1.0: blocks of 32 elements, each
  *    element FP4 E2M1 (sign, 2 exponent bits with bias 1, 1 mantissa bit,
  *    subnormal when the exponent field is 0), one shared E8M0 scale per block
- *    (2^(byte - 127); byte 255 is NaN).
+ *    (2^(byte - 127); byte 255 is NaN). ExpertLayout::Native's single gate_up
+ *    plane (blocks, scales, bias) is read as the interleaved gate_up: row 2i
+ *    gate, 2i+1 up, its scales / biases in the same row order.
  *
  * Readings where the pages are silent (each listed in the design notes):
  *  - SwiGLU is silu(g) * v with silu(g) = g / (1 + e^-g).
@@ -85,6 +87,7 @@ typedef struct {
     const void *gate_s, *gate_z, *up_s, *up_z, *down_s, *down_z;
     const void *shared_gate_w, *shared_up_w, *shared_down_w;
     const void *latent_down_w, *latent_up_w, *latent_norm_w;
+    const void *gate_up_s, *gate_up_z;  /* 4-bit interleaved gate_up plane */
 } orc_weights;
 
 static double bf16_bits_to_double(uint16_t b)
@@ -175,8 +178,8 @@ static void routed_expert(const orc_config *cfg, const orc_weights *w, int64_t e
         for (int64_t c = 0; c < K; ++c) {
             double wg, wu;
             if (cfg->gate_up_interleaved) {
-                wg = plane_at(cfg, w->gate_up_w, NULL, NULL, 2 * I, K, e, 2 * i, c);
-                wu = plane_at(cfg, w->gate_up_w, NULL, NULL, 2 * I, K, e, 2 * i + 1, c);
+                wg = plane_at(cfg, w->gate_up_w, w->gate_up_s, w->gate_up_z, 2 * I, K, e, 2 * i, c);
+                wu = plane_at(cfg, w->gate_up_w, w->gate_up_s, w->gate_up_z, 2 * I, K, e, 2 * i + 1, c);
             } else {
                 wg = plane_at(cfg, w->gate_w, w->gate_s, w->gate_z, I, K, e, i, c);
                 wu = plane_at(cfg, w->up_w, w->up_s, w->up_z, I, K, e, i, c);

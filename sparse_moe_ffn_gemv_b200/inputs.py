@@ -102,8 +102,13 @@ LATENT_BF16 = MoeSpec(
 # clamped_routed: gate, up and down blocks with scales and biases; not interleaved).
 CLAMPED_MXFP4 = CLAMPED_BF16.replace(name="clamped_mxfp4", config_id=6, weight_format="mxfp4",
                                      gate_up_interleaved=False, group_size=32, token_counts=(1, 8, 8192))
+# The same family in the native MXFP4 layout (libmir-metal clamped_routed ExpertLayout::Native):
+# one interleaved gate_up block plane (row 2i gate, 2i + 1 up) with its scales and bias.
+CLAMPED_MXFP4_NATIVE = CLAMPED_MXFP4.replace(name="clamped_mxfp4_native", config_id=7,
+                                             gate_up_interleaved=True)
 
-WORKLOADS = {s.name: s for s in (TINY_F32, KLEAR_BF16, KLEAR_Q4, CLAMPED_BF16, LATENT_BF16, CLAMPED_MXFP4)}
+WORKLOADS = {s.name: s for s in (TINY_F32, KLEAR_BF16, KLEAR_Q4, CLAMPED_BF16, LATENT_BF16, CLAMPED_MXFP4,
+                                 CLAMPED_MXFP4_NATIVE)}
 
 BASE_SEED = 20261202
 

@@ -15,8 +15,8 @@ import torch
 import oracle
 from oracle import bruteforce
 from sparse_moe_ffn_gemv_b200 import inputs
-from tiny_specs import (ALL, CLAMPED, LATENT, LATENT_NONORM, MXFP4, Q4, ROUTER_BIAS, SIG_BLEND,
-                        np_weights, np_x, to_bf16_bits)
+from tiny_specs import (ALL, CLAMPED, LATENT, LATENT_NONORM, MXFP4, MXFP4_NATIVE, Q4, Q4_INTERLEAVED,
+                        ROUTER_BIAS, SIG_BLEND, np_weights, np_x, to_bf16_bits)
 
 GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
 
@@ -445,6 +445,30 @@ def test_mxfp4_block_equals_the_same_weights_stored_in_bf16():
     b = oracle.forward(spec_bf, wb, x)
     np.testing.assert_array_equal(a["idx"], b["idx"])
     np.testing.assert_array_equal(a["y"], b["y"])
+
+
+@pytest.mark.parametrize("spec", [MXFP4_NATIVE, Q4_INTERLEAVED], ids=lambda s: s.name)
+def test_interleaved_4bit_block_equals_the_split_block_on_the_same_rows(spec):
+    """The native layout's single gate_up plane (libmir-metal ExpertLayout::Native), read as
+    row 2i gate and 2i + 1 up with the companions and bias in the same row order, is the split
+    layout of its even and odd rows: the two evaluations agree exactly."""
+    w = np_weights(spec)
+    x = np_x(spec, 7, 30.0)
+    split = spec.replace(name=spec.name + "_split", gate_up_interleaved=False)
+    ws = {k: v for k, v in w.items() if not k.startswith("gate_up")}
+    for comp in ("_w", "_s", "_z", "_b"):
+        if "gate_up" + comp in w:
+            plane = w["gate_up" + comp]
+            ws["gate" + comp], ws["up" + comp] = plane[:, 0::2].copy(), plane[:, 1::2].copy()
+    a = oracle.forward(spec, w, x)
+    b = oracle.forward(split, ws, x)
+    np.testing.assert_array_equal(a["idx"], b["idx"])
+    np.testing.assert_array_equal(a["y"], b["y"])
+    # and a swapped row order (up rows first) is a different block
+    wswap = dict(w)
+    g = w["gate_up_w"]
+    wswap["gate_up_w"] = np.stack([g[:, 1::2], g[:, 0::2]], axis=2).reshape(g.shape).copy()
+    assert not np.array_equal(oracle.forward(spec, wswap, x)["y"], a["y"])
 
 
 # --- permutation -----------------------------------------------------------------

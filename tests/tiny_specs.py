@@ -5,8 +5,9 @@ select-only bias and the shared-expert blend (Klear PR items 2-3), softmax
 over the top-k logits with clamped SwiGLU on an interleaved gate_up plane with
 biases (libmir-metal clamped_routed ExpertLayout::DenseFused), 4-bit affine
 planes (mlxcel issue #974), the latent variant (ferrox latent_moe.rs), and MXFP4
-planes in the clamped family's split layout (libmir-metal clamped_routed; element
-and scale encodings from the OCP Microscaling Formats v1.0 specification).
+planes in the clamped family's split and native (interleaved gate_up) layouts
+(libmir-metal clamped_routed; element and scale encodings from the OCP Microscaling
+Formats v1.0 specification).
 """
 import numpy as np
 
@@ -43,9 +44,17 @@ MXFP4 = MoeSpec(
     name="t_mxfp4", config_id=108, hidden=128, num_experts=5, top_k=2, intermediate=64,
     scoring="softmax_topk", activation="swiglu_clamped", has_expert_bias=True,
     weight_format="mxfp4", group_size=32)
+# the same family in the native layout: one interleaved gate_up block plane with its scales
+# and bias (libmir-metal clamped_routed ExpertLayout::Native)
+MXFP4_NATIVE = MXFP4.replace(name="t_mxfp4_native", config_id=109, gate_up_interleaved=True)
+# 4-bit affine on an interleaved gate_up plane (its scales and biases interleaved alike)
+Q4_INTERLEAVED = MoeSpec(
+    name="t_q4_il", config_id=110, hidden=128, num_experts=4, top_k=2, intermediate=64,
+    scoring="softmax_topk", activation="swiglu_clamped", gate_up_interleaved=True,
+    has_expert_bias=True, weight_format="q4", group_size=32)
 
 ALL = [inputs.TINY_F32, SIG_BLEND, CLAMPED, Q4, LATENT, ROUTER_BIAS, SEPARATE_BIAS,
-       LATENT_NONORM, MXFP4]
+       LATENT_NONORM, MXFP4, MXFP4_NATIVE, Q4_INTERLEAVED]
 
 
 def np_weights(spec, scale_weights: float = 1.0):
