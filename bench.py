@@ -65,9 +65,11 @@ def peaks():
 def expert_bytes(spec) -> int:
     """Bytes of one routed expert's weights (gate, up, down, biases / 4-bit companions)."""
     I, K = spec.intermediate, spec.expert_in
-    if spec.weight_format == "q4":
+    if spec.weight_format == "q4":  # packed codes + bf16 scale and bias per group
         g = spec.group_size
         b = 3 * I * K // 2 + (2 * I * (K // g) + K * (I // g)) * 2 * 2
+    elif spec.weight_format == "mxfp4":  # packed E2M1 codes + one E8M0 byte per 32
+        b = 3 * I * K // 2 + (2 * I * (K // 32) + K * (I // 32))
     else:
         b = 3 * I * K * (4 if spec.weight_format == "f32" else 2)
     if spec.has_expert_bias:
@@ -443,7 +445,7 @@ def run(args, rank, world, local, dist):
         line = {
             "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_max, "higher_is_better": True, "scaling": "weak",
-            "vs_baseline": None, "dtype": spec.act_dtype if spec.weight_format != "q4" else "bf16+q4",
+            "vs_baseline": None, "dtype": spec.act_dtype if spec.weight_format in ("bf16", "f32") else "bf16+" + spec.weight_format,
             "data": "synthetic (seeded N(0,1) activations, N(0,0.02) weights; no checkpoint)",
             "config": workload_config(spec, T, world),
             "roofline": roofline,

@@ -111,7 +111,7 @@ typedef struct moe_config {
     int32_t act_dtype;             /* MOE_DTYPE_F32 or MOE_DTYPE_BF16: x, y and every
                                       non-routed weight                                 */
     int32_t weight_format;         /* routed planes: F32 (needs act F32), BF16, Q4_AFFINE,
-                                      MXFP4 (both need act BF16, separate gate/up)      */
+                                      MXFP4 (both need act BF16)                        */
     int32_t group_size;            /* Q4: 32, 64 or 128; MXFP4: 32                      */
     int32_t bits;                  /* Q4 and MXFP4: 4                                   */
     int32_t shared_mode;           /* enum moe_shared_mode                              */
@@ -138,6 +138,11 @@ typedef struct moe_config {
  *       gate_s/up_s/down_s hold one uint8 E8M0 scale per 32 elements
  *       [E, rows, cols/32], weight = element * 2^(scale - 127); the _z fields are
  *       unused. A scale byte of 255 (NaN in the format) gives non-finite weights.
+ *   4-bit with gate_up_interleaved (libmir-metal ExpertLayout::Native: one
+ *       gate_up block plane with its scales and bias): gate_up_w holds the
+ *       words of the [E, 2I, K] plane (row 2i gate, 2i+1 up), gate_up_s (and,
+ *       for Q4, gate_up_z) its companions [E, 2I, K/group] in the same row
+ *       order; gate_s/gate_z/up_s/up_z are unused.
  *   shared_gate_w, shared_up_w [Is, H]; shared_down_w [H, Is]
  *   latent_down_w [L, H]; latent_up_w [H, L]; latent_norm_w [L]
  */
@@ -147,6 +152,7 @@ typedef struct moe_weights {
     const void *gate_s, *gate_z, *up_s, *up_z, *down_s, *down_z;
     const void *shared_gate_w, *shared_up_w, *shared_down_w;
     const void *latent_down_w, *latent_up_w, *latent_norm_w;
+    const void *gate_up_s, *gate_up_z;  /* 4-bit interleaved gate_up plane: its scales / biases */
 } moe_weights;
 
 /* Checks a config on the host (Klear PR "Other guards": zero checks before

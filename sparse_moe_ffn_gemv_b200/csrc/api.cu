@@ -101,12 +101,10 @@ moe_status validate_config(const moe_config* c) {
             return MOE_ERR_INVALID_QUANTIZATION;
         if (K % c->group_size != 0 || c->intermediate % c->group_size != 0)
             return MOE_ERR_INVALID_QUANTIZATION;
-        if (c->gate_up_interleaved) return MOE_ERR_UNSUPPORTED;
     }
     if (c->weight_format == MOE_DTYPE_MXFP4) {  // OCP MX: blocks of 32 elements, 4-bit E2M1
         if (c->bits != 4 || c->group_size != 32) return MOE_ERR_INVALID_QUANTIZATION;
         if (K % 64 != 0 || c->intermediate % 64 != 0) return MOE_ERR_INVALID_QUANTIZATION;
-        if (c->gate_up_interleaved) return MOE_ERR_UNSUPPORTED;
     }
     // 16-byte rows
     const int q = c->act_dtype == MOE_DTYPE_F32 ? 4 : 8;
@@ -134,12 +132,17 @@ moe_status validate_weights(const moe_config* c, const moe_weights* w) {
     }
     if (!need(w->down_w)) return MOE_ERR_MISSING_TENSOR;
     if (c->has_expert_bias && !need(w->down_b)) return MOE_ERR_MISSING_TENSOR;
+    // 4-bit companions: scales (and Q4 biases) of each routed plane; an interleaved gate_up
+    // plane carries its own (gate_up_s / gate_up_z, libmir-metal ExpertLayout::Native)
+    const bool il = c->gate_up_interleaved;
     if (c->weight_format == MOE_DTYPE_Q4_AFFINE) {
-        const void* q[] = {w->gate_s, w->gate_z, w->up_s, w->up_z, w->down_s, w->down_z};
+        const void* q[] = {il ? w->gate_up_s : w->gate_s, il ? w->gate_up_z : w->gate_z,
+                           il ? w->gate_up_s : w->up_s, il ? w->gate_up_z : w->up_z, w->down_s, w->down_z};
         for (const void* p : q)
             if (!need(p)) return MOE_ERR_MISSING_TENSOR;
     }
-    if (c->weight_format == MOE_DTYPE_MXFP4 && (!need(w->gate_s) || !need(w->up_s) || !need(w->down_s)))
+    if (c->weight_format == MOE_DTYPE_MXFP4 &&
+        (!need(il ? w->gate_up_s : w->gate_s) || !need(il ? w->gate_up_s : w->up_s) || !need(w->down_s)))
         return MOE_ERR_MISSING_TENSOR;
     if (c->shared_mode != MOE_SHARED_NONE &&
         (!need(w->shared_gate_w) || !need(w->shared_up_w) || !need(w->shared_down_w)))
@@ -150,7 +153,7 @@ moe_status validate_weights(const moe_config* c, const moe_weights* w) {
                          w->gate_w, w->up_w, w->gate_up_w, w->gate_b, w->up_b, w->gate_up_b,
                          w->down_w, w->down_b, w->gate_s, w->gate_z, w->up_s, w->up_z,
                          w->down_s, w->down_z, w->shared_gate_w, w->shared_up_w, w->shared_down_w,
-                         w->latent_down_w, w->latent_up_w, w->latent_norm_w};
+                         w->latent_down_w, w->latent_up_w, w->latent_norm_w, w->gate_up_s, w->gate_up_z};
     for (const void* p : all)
         if (p && !aligned16(p)) return MOE_ERR_INVALID_ARGUMENT;
     return MOE_OK;
@@ -375,7 +378,7 @@ moe_status run_experts_tc(const moe_config* c, const moe_weights* w, const void*
             p.M = I; p.K = K; p.m_blocks = (I + kTcRowsGateUp - 1) / kTcRowsGateUp;
             p.grouped = 1; p.num_groups = E; p.offsets = offsets; p.tile_start = tiles;
             p.out = h; p.ld_out = I;
-            p.interleaved = c->gate_up_interleaved;
+            p.interleaved = c->gate_up_interleaved;  // bf16 / f32 planes: one 4-D map
             if (c->has_expert_bias) {
                 if (c->gate_up_interleaved) {
                     p.bias0 = w->gate_up_b;
@@ -391,8 +394,25 @@ moe_status run_experts_tc(const moe_config* c, const moe_weights* w, const void*
                 p.q4 = 1;
                 p.mx = c->weight_format == MOE_DTYPE_MXFP4;
                 p.group_size = c->group_size;
-                p.qs0 = w->gate_s; p.qz0 = w->gate_z; p.qs1 = w->up_s; p.qz1 = w->up_z;
-                ok = tc_q4_weight_map(&P.a0[np], w->gate_w, E, I, K) && tc_q4_weight_map(&P.a1[np], w->up_w, E, I, K);
+                if (c->gate_up_interleaved) {
+                    // one [E, 2I, K] plane: gate rows 2i and up rows 2i + 1 through two maps
+                    // that step over every other row; the companions interleave the same way
+                    const int64_t ng = K / c->group_size;
+                    const int64_t sb = p.mx ? 1 : 2;  // bytes per scale
+                    p.interleaved = 0;
+                    p.qrow_step = 2;
+                    p.qs0 = w->gate_up_s;
+                    p.qs1 = static_cast<const char*>(w->gate_up_s) + ng * sb;
+                    p.qz0 = p.mx ? nullptr : w->gate_up_z;
+                    p.qz1 = p.mx ? nullptr : static_cast<const char*>(w->gate_up_z) + ng * 2;
+                    const char* gu = static_cast<const char*>(w->gate_up_w);
+                    ok = tc_q4_weight_map(&P.a0[np], gu, E, I, K, 2) &&
+                         tc_q4_weight_map(&P.a1[np], gu + int64_t(K) / 2, E, I, K, 2);
+                } else {
+                    p.qs0 = w->gate_s; p.qz0 = w->gate_z; p.qs1 = w->up_s; p.qz1 = w->up_z;
+                    ok = tc_q4_weight_map(&P.a0[np], w->gate_w, E, I, K) &&
+                         tc_q4_weight_map(&P.a1[np], w->up_w, E, I, K);
+                }
             } else if (c->gate_up_interleaved) {
                 ok = tc_weight_map(&P.a0[np], w->gate_up_w, E, I, K, true);
             } else {
@@ -490,7 +510,9 @@ moe_status run_experts(const moe_config* c, const moe_weights* w, const void* u,
     g.has_bias = c->has_expert_bias;
     g.group_size = c->group_size;
     g.gate_w = w->gate_w; g.up_w = w->up_w; g.gate_up_w = w->gate_up_w;
-    g.gate_s = w->gate_s; g.gate_z = w->gate_z; g.up_s = w->up_s; g.up_z = w->up_z;
+    g.gate_s = c->gate_up_interleaved ? w->gate_up_s : w->gate_s;
+    g.gate_z = c->gate_up_interleaved ? w->gate_up_z : w->gate_z;
+    g.up_s = w->up_s; g.up_z = w->up_z;
     g.gate_b = w->gate_b; g.up_b = w->up_b; g.gate_up_b = w->gate_up_b;
     g.offsets = offsets;
     g.sorted_slot = sorted_slot;

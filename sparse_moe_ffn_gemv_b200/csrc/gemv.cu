@@ -236,10 +236,19 @@ __device__ void gateup_group(const GateUpArgs& a, bool shared, int e, int unit0,
     if (shared) {
         rows[0] = reinterpret_cast<const char*>(a.sg_w) + int64_t(live ? i : 0) * rb;
         rows[1] = reinterpret_cast<const char*>(a.su_w) + int64_t(live ? i : 0) * rb;
-    } else if (a.interleaved) {
+    } else if (a.interleaved) {  // one plane: rows 2i (gate) and 2i + 1 (up), companions alike
         const int64_t r0 = int64_t(e) * 2 * I + 2 * int64_t(live ? i : 0);
         rows[0] = reinterpret_cast<const char*>(a.gate_up_w) + r0 * rb;
         rows[1] = rows[0] + rb;
+        if constexpr (WF == kQ4) {
+            const int64_t ng = K / a.group_size;
+            q[0] = {reinterpret_cast<const __nv_bfloat16*>(a.gate_s) + r0 * ng,
+                    reinterpret_cast<const __nv_bfloat16*>(a.gate_z) + r0 * ng, nullptr};
+            q[1] = {q[0].s + ng, q[0].z + ng, nullptr};
+        } else if constexpr (WF == kMX4) {
+            q[0] = {nullptr, nullptr, reinterpret_cast<const uint8_t*>(a.gate_s) + r0 * (K / 32)};
+            q[1] = {nullptr, nullptr, q[0].e8 + K / 32};
+        }
     } else {
         const int64_t r0 = int64_t(e) * I + (live ? i : 0);
         rows[0] = reinterpret_cast<const char*>(a.gate_w) + r0 * rb;

@@ -59,6 +59,8 @@ cudaError_t launch_tile_start(const int32_t* offsets, int E, int tile_bn, int32_
 struct GateUpArgs {
     int wf = MOE_DTYPE_BF16, interleaved = 0, has_bias = 0, group_size = 64;
     const void *gate_w = nullptr, *up_w = nullptr, *gate_up_w = nullptr;
+    // 4-bit companions; with interleaved planes gate_s / gate_z are those of gate_up_w
+    // ([E, 2I, K / group], the plane's row order)
     const void *gate_s = nullptr, *gate_z = nullptr, *up_s = nullptr, *up_z = nullptr;
     const void *gate_b = nullptr, *up_b = nullptr, *gate_up_b = nullptr;
     const int32_t *offsets = nullptr, *sorted_slot = nullptr, *active = nullptr;
@@ -124,6 +126,8 @@ struct TcProblem {
     int q4 = 0, group_size = 64;
     const void *qs0 = nullptr, *qz0 = nullptr, *qs1 = nullptr, *qz1 = nullptr;
     int mx = 0;  // with q4 = 1: MXFP4 codes, qs0 / qs1 the E8M0 scale bytes [groups, M, K / 32]
+    int qrow_step = 1;  // companion rows per unit: 2 for an interleaved gate_up plane, whose
+                        // up companions start one row after qs0 / qz0 (qs1 / qz1 = that row)
 };
 
 struct alignas(64) TcParams {
@@ -146,7 +150,9 @@ struct alignas(64) TcParams {
 bool tc_weight_map(CUtensorMap* m, const void* w, int E, int R, int K, bool interleaved);
 // Packed 4-bit weight operand: [E, R, K / 8] uint32 words (8 codes each), one 64-wide K block
 // (8 words) x 128 rows per box, no swizzle (the kernel's dequantising warps read it).
-bool tc_q4_weight_map(CUtensorMap* m, const void* w, int E, int R, int K);
+// row_step 2 views every other row of an interleaved [E, 2R, K / 8] plane from w (gate rows;
+// pass w advanced by one row for the up rows).
+bool tc_q4_weight_map(CUtensorMap* m, const void* w, int E, int R, int K, int row_step = 1);
 // Four maps m[0..3] of the token operand [rows, K] bf16, boxes of 16, 32, 64 and bn rows.
 bool tc_token_map(CUtensorMap* m, const void* u, int64_t rows, int K, int bn);
 cudaError_t launch_tc_gemm(TcParams& P, bool gateup, int64_t max_tiles, cudaStream_t s);

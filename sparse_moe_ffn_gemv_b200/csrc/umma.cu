@@ -454,7 +454,7 @@ __global__ void __launch_bounds__(TcShape<GATEUP, BN, STAGES, Q4>::THREADS, 1)
             for (int ai = 0; ai < DT; ++ai) {
                 const int a = a0 + ai;
                 const int r = min(ti.mb * S::ROWS + (GATEUP ? 0 : a * kBM) + drow, p.M - 1);
-                const int64_t off = (int64_t(ti.group) * p.M + r) * ng;
+                const int64_t off = (int64_t(ti.group) * p.M + r) * p.qrow_step * ng;
                 sp[ai] = static_cast<const unsigned char*>((GATEUP && a == 1) ? p.qs1 : p.qs0) + off * (p.mx ? 1 : 2);
                 zp[ai] = p.mx ? nullptr : static_cast<const unsigned char*>((GATEUP && a == 1) ? p.qz1 : p.qz0) + off * 2;
             }
@@ -761,10 +761,11 @@ bool tc_token_map(CUtensorMap* m, const void* u, int64_t rows, int K, int bn) {
     return true;
 }
 
-// Packed 4-bit plane [E, R, K / 8] uint32 (K % 64 == 0): box of 8 words x 128 rows.
-bool tc_q4_weight_map(CUtensorMap* m, const void* w, int E, int R, int K) {
+// Packed 4-bit plane [E, R, K / 8] uint32 (K % 64 == 0): box of 8 words x 128 rows. With
+// row_step 2 the rows of one unit are every other row of an [E, 2R, K / 8] plane.
+bool tc_q4_weight_map(CUtensorMap* m, const void* w, int E, int R, int K, int row_step) {
     const cuuint64_t dims[3] = {cuuint64_t(K / 8), cuuint64_t(R), cuuint64_t(E)};
-    const cuuint64_t strides[2] = {cuuint64_t(K / 8) * 4, cuuint64_t(R) * (K / 8) * 4};
+    const cuuint64_t strides[2] = {cuuint64_t(K / 8) * 4 * row_step, cuuint64_t(R) * (K / 8) * 4 * row_step};
     const cuuint32_t box[3] = {8, kBM, 1};
     return encode(m, w, 3, dims, strides, box, CU_TENSOR_MAP_DATA_TYPE_UINT32, CU_TENSOR_MAP_SWIZZLE_NONE);
 }

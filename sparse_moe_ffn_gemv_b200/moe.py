@@ -23,6 +23,7 @@ WEIGHT_FIELDS = [
     "gate_s", "gate_z", "up_s", "up_z", "down_s", "down_z",
     "shared_gate_w", "shared_up_w", "shared_down_w",
     "latent_down_w", "latent_up_w", "latent_norm_w",
+    "gate_up_s", "gate_up_z",
 ]
 
 # The entry points include/moe.h declares.

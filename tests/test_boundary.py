@@ -116,19 +116,36 @@ def test_hostile_quantisation_params_are_rejected(name, fields):
     assert M.STATUS[M.moe_config_validate(_cfg(inputs.KLEAR_Q4, **fields))] == "MOE_ERR_INVALID_QUANTIZATION"
 
 
-def test_mxfp4_needs_blocks_of_32_four_bits_and_separate_gate_up():
+def test_mxfp4_needs_blocks_of_32_and_four_bits():
     assert M.moe_config_validate(_cfg(inputs.CLAMPED_MXFP4)) == 0
     for fields in (dict(group_size=64), dict(bits=8)):
         assert M.STATUS[M.moe_config_validate(_cfg(inputs.CLAMPED_MXFP4, **fields))] == \
             "MOE_ERR_INVALID_QUANTIZATION"
-    assert M.STATUS[M.moe_config_validate(_cfg(inputs.CLAMPED_MXFP4, gate_up_interleaved=1))] == \
-        "MOE_ERR_UNSUPPORTED"
+    assert M.moe_config_validate(_cfg(inputs.CLAMPED_MXFP4, gate_up_interleaved=1)) == 0  # native layout
     cfg = _cfg(inputs.CLAMPED_MXFP4)
     w = _fake_weights(inputs.CLAMPED_MXFP4)
-    w.gate_z = w.up_z = w.down_z = None            # MXFP4 has no affine biases
+    w.gate_z = w.up_z = w.down_z = w.gate_up_s = w.gate_up_z = None  # no affine biases; split planes
     assert M.moe_weights_validate(cfg, w) == 0
     w.down_s = None                                  # but every plane needs its scales
     assert M.STATUS[M.moe_weights_validate(cfg, w)] == "MOE_ERR_MISSING_TENSOR"
+
+
+@pytest.mark.parametrize("fmt", ["mxfp4", "q4"])
+def test_interleaved_4bit_plane_needs_its_own_companions(fmt):
+    """With one gate_up plane (libmir-metal ExpertLayout::Native) the scales (and Q4 biases)
+    come from gate_up_s / gate_up_z; the split planes' companions are not consulted."""
+    spec = inputs.CLAMPED_MXFP4.replace(gate_up_interleaved=True, weight_format=fmt)
+    cfg = _cfg(spec)
+    w = _fake_weights(spec)
+    w.gate_s = w.gate_z = w.up_s = w.up_z = None
+    assert M.moe_weights_validate(cfg, w) == 0
+    for f in (["gate_up_s", "gate_up_z"] if fmt == "q4" else ["gate_up_s"]):
+        w2 = _fake_weights(spec)
+        setattr(w2, f, None)
+        assert M.STATUS[M.moe_weights_validate(cfg, w2)] == "MOE_ERR_MISSING_TENSOR", f
+    w3 = _fake_weights(spec)
+    w3.gate_up_s = 1 << 21 | 8                       # misaligned companion plane
+    assert M.STATUS[M.moe_weights_validate(cfg, w3)] == "MOE_ERR_INVALID_ARGUMENT"
 
 
 def test_group_must_divide_the_widths():

@@ -84,6 +84,8 @@ SMALL = [
     (ts.MXFP4, 9, 30.0),                 # MXFP4 planes (tensor cores: 4 T k >= E)
     (inputs.CLAMPED_MXFP4, 1, 1.0),      # weight-streaming kernels
     (inputs.CLAMPED_MXFP4, 8, 8.0),      # tensor cores, clamp engaged
+    (ts.MXFP4_NATIVE, 9, 30.0),          # native layout: one interleaved gate_up block plane
+    (ts.Q4_INTERLEAVED, 9, 30.0),        # 4-bit affine on an interleaved gate_up plane
 ]
 
 
@@ -117,6 +119,30 @@ def test_block_matches_oracle_full_size(spec, T, n_sample):
     # outputs of sampled tokens: first, last, and a seeded spread (ragged tail included)
     rng = np.random.default_rng(T)
     tokens = np.unique(np.concatenate([[0, T - 1], rng.choice(T, size=n_sample - 2, replace=False)]))
+    check_block(spec, wnp, x_np, tokens, y[tokens], idx[tokens], label=f"{spec.name} T={T}")
+
+
+@pytest.mark.slow
+def test_native_mxfp4_layout_at_the_clamped_shape(monkeypatch):
+    """The clamped family's native MXFP4 layout (one interleaved gate_up block plane with its
+    scales and bias, libmir-metal ExpertLayout::Native) at full shape, one weight set for all
+    cases: one token (weight-streaming), 8 tokens with the clamp engaged (tensor cores), both
+    engines forced at 5 / 20 tokens, and sampled tokens of an 8192-token batch."""
+    spec = inputs.CLAMPED_MXFP4_NATIVE
+    wcpu, wnp = weights(spec)
+    full_check(spec, 1)
+    full_check(spec, 8, 8.0)
+    monkeypatch.setenv("MOE_PATH", "tc")
+    full_check(spec, 5)
+    monkeypatch.setenv("MOE_PATH", "gemv")
+    full_check(spec, 20)
+    monkeypatch.delenv("MOE_PATH")
+    T = 8192
+    x_cpu = inputs.make_x(spec, T)
+    x_np = inputs.to_numpy_storage(x_cpu)
+    y, idx, _, _ = run_gpu(spec, wcpu, x_cpu)
+    rng = np.random.default_rng(T)
+    tokens = np.unique(np.concatenate([[0, T - 1], rng.choice(T, size=10, replace=False)]))
     check_block(spec, wnp, x_np, tokens, y[tokens], idx[tokens], label=f"{spec.name} T={T}")
 
 
@@ -239,6 +265,7 @@ TC_SMALL = [  # tensor-core path forced: ragged groups, partial tiles, interleav
     (inputs.KLEAR_Q4, 3),
     (inputs.KLEAR_Q4, 150),
     (inputs.CLAMPED_MXFP4, 5),
+    (ts.Q4_INTERLEAVED, 3),
 ]
 
 
@@ -246,6 +273,8 @@ GEMV_SMALL = [  # weight-streaming kernels forced where the auto rule picks the 
     (ts.MXFP4, 9),
     (inputs.CLAMPED_MXFP4, 20),
     (inputs.KLEAR_Q4, 20),
+    (ts.MXFP4_NATIVE, 9),
+    (ts.Q4_INTERLEAVED, 9),
 ]
 
 
