@@ -216,12 +216,25 @@ def cpu_baseline(spec, w_cpu, x_cpu, target_s: float = 10.0):
                       f"({dt2:.1f} s, fp64, OpenMP over tokens)"}
 
 
+L2_BYTES = 126 * 2**20  # B200 L2 cache
+
+
+def needs_l2_flush(spec, T) -> bool:
+    """True when the step's weights could stay in L2 between timed steps: the largest
+    possible activated set (min(E, T k) experts plus the dense weights) is under twice the
+    L2 size. Those steps are timed one by one with L2 flushed in between."""
+    most = min(spec.num_experts, T * spec.top_k) * expert_bytes(spec) + dense_bytes(spec)
+    return most < 2 * L2_BYTES
+
+
 def workload_config(spec, T, world):
     """The `config` object of both arms' JSON lines."""
+    l2 = ("L2 flushed between timed steps (activated weights could fit in L2)" if needs_l2_flush(spec, T)
+          else "activated weights larger than L2 (no flush needed)")
     return {"workload": f"{spec.name} (hidden {spec.hidden}, {spec.num_experts} experts, "
                         f"top-{spec.top_k}, intermediate {spec.intermediate})",
             "tokens_per_gpu": T, "parallelism": f"replicas x{world}",
-            "l2": "activated weights larger than L2 (no flush needed); decode rows flush L2"}
+            "l2": l2 + "; decode rows flush L2"}
 
 
 def max_over_ranks(v: float, dist, device) -> float:
@@ -344,7 +357,9 @@ def run(args, rank, world, local, dist):
 
     launches = kernels_per_step(block, x, y)
 
-    # ---- timed region: K whole steps
+    # ---- timed region: K whole steps (one by one with L2 flushed in between when the
+    # activated weights could stay in L2)
+    l2_flush = l2_flush_buffer(dev) if needs_l2_flush(spec, T) else None
     sampler = ClockSampler(local)
     for _ in range(args.warmup):
         block.forward(x, y)
@@ -353,15 +368,18 @@ def run(args, rank, world, local, dist):
     torch.cuda.synchronize()
     sampler.start()
     time.sleep(0.3)
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record()
-    for _ in range(args.steps):
-        block.forward(x, y)
-    e1.record()
-    torch.cuda.synchronize()
+    if l2_flush is None:
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(args.steps):
+            block.forward(x, y)
+        e1.record()
+        torch.cuda.synchronize()
+        ms = e0.elapsed_time(e1) / args.steps
+    else:
+        ms = statistics.mean(time_steps(lambda: block.forward(x, y), args.steps, 0, flush=l2_flush))
     if dist is not None:
         dist.barrier()
-    ms = e0.elapsed_time(e1) / args.steps
     # dominant stage (routed experts: gate/up + down kernels), same inputs, CUDA events
     off = torch.empty(spec.num_experts + 1, dtype=torch.int32, device=dev)
     ss = torch.empty(T * spec.top_k, dtype=torch.int32, device=dev)
@@ -373,7 +391,7 @@ def run(args, rank, world, local, dist):
     M.moe_permute(block.cfg, idx, T, off, ss, sp, block.ws)
     y_acc = torch.empty((T, K), dtype=torch.float32, device=dev)
     ffn_ms = time_steps(lambda: M.moe_grouped_ffn(block.cfg, block.w, u, T, off, ss, wts, y_acc, block.ws),
-                        args.steps, args.warmup)
+                        args.steps, args.warmup, flush=l2_flush)
     clocks = sampler.stop()
     if block.device_status() != 0:
         raise SystemExit("device status set during the timed region")
@@ -402,7 +420,7 @@ def run(args, rank, world, local, dist):
             block.forward(x_dev, y)
             y_host.copy_(y, non_blocking=True)
 
-        e2e_ms = time_steps(e2e_step, args.steps, args.warmup)
+        e2e_ms = time_steps(e2e_step, args.steps, args.warmup, flush=l2_flush)
         e_max = max_over_ranks(statistics.mean(e2e_ms), dist, dev)
         e2e = {"value": world * T / (e_max / 1000.0), "unit": "tokens/s",
                "h2d_bytes_per_step": T * spec.hidden * ab, "d2h_bytes_per_step": T * spec.hidden * ab}

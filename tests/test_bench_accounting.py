@@ -33,3 +33,17 @@ def test_block_flops_counts_router_experts_and_shared():
     T = 4096
     want = 2 * T * 256 * 2048 + 2 * T * 8 * 3 * 768 * 2048 + 2 * T * 3 * 768 * 2048
     assert bench.block_flops(s, T) == want
+
+
+def test_l2_flush_between_timed_steps_only_where_the_weights_could_stay_in_l2():
+    # Klear bf16 prefill: 256 experts x 9.44 MB, far above 2 x 126 MB -> no flush needed
+    assert not bench.needs_l2_flush(inputs.KLEAR_BF16, 4096)
+    assert not bench.needs_l2_flush(inputs.KLEAR_BF16, 64)      # up to 256 experts activated
+    # one token: 8 experts (76 MB bf16, 21 MB 4-bit) plus the dense weights fit in L2 twice
+    assert bench.needs_l2_flush(inputs.KLEAR_BF16, 1)
+    assert bench.needs_l2_flush(inputs.KLEAR_Q4, 1)
+    assert bench.needs_l2_flush(inputs.KLEAR_Q4, 8)             # 64 x 2.65 MB = 170 MB < 252 MB
+    assert not bench.needs_l2_flush(inputs.KLEAR_Q4, 32)        # up to 256 x 2.65 MB = 679 MB
+    for spec, T in ((inputs.KLEAR_Q4, 1), (inputs.KLEAR_BF16, 4096)):
+        cfg = bench.workload_config(spec, T, 1)
+        assert cfg["l2"].startswith("L2 flushed" if bench.needs_l2_flush(spec, T) else "activated weights larger")
