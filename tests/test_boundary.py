@@ -47,13 +47,14 @@ def test_struct_layout_matches_the_header(tmp_path):
     src.write_text('#include <stdio.h>\n#include <stddef.h>\n#include "moe.h"\nint main(void){\n'
                    'printf("%zu %zu %zu %zu %zu\\n", sizeof(moe_config), sizeof(moe_weights),'
                    ' offsetof(moe_config, rms_eps), offsetof(moe_config, routed_scaling_factor),'
-                   ' offsetof(moe_weights, latent_norm_w));return 0;}\n')
+                   ' offsetof(moe_weights, latent_norm_w)); printf("%zu\\n", offsetof(moe_weights, gate_up_z));'
+                   'return 0;}\n')
     exe = tmp_path / "layout"
     subprocess.check_call(["gcc", "-std=c11", "-I", os.path.join(ROOT, "include"), str(src), "-o", str(exe)])
     got = [int(v) for v in subprocess.check_output([str(exe)]).split()]
     assert got == [ctypes.sizeof(M.MoeConfig), ctypes.sizeof(M.MoeWeights),
                    M.MoeConfig.rms_eps.offset, M.MoeConfig.routed_scaling_factor.offset,
-                   M.MoeWeights.latent_norm_w.offset]
+                   M.MoeWeights.latent_norm_w.offset, M.MoeWeights.gate_up_z.offset]
 
 
 def test_enum_values_match_the_header():
