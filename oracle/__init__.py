@@ -46,6 +46,7 @@ class OrcConfig(ctypes.Structure):
         ("shared_mode", ctypes.c_int32), ("shared_intermediate", ctypes.c_int32),
         ("latent_dim", ctypes.c_int32), ("latent_use_norm", ctypes.c_int32),
         ("rms_eps", ctypes.c_double),
+        ("dense_weight_format", ctypes.c_int32), ("dense_group_size", ctypes.c_int32),
     ]
 
 
@@ -56,6 +57,8 @@ _WEIGHT_FIELDS = [
     "shared_gate_w", "shared_up_w", "shared_down_w",
     "latent_down_w", "latent_up_w", "latent_norm_w",
     "gate_up_s", "gate_up_z",
+    "router_s", "router_z", "shared_gate_s", "shared_gate_z", "shared_up_s", "shared_up_z",
+    "shared_down_s", "shared_down_z", "latent_down_s", "latent_down_z", "latent_up_s", "latent_up_z",
 ]
 
 
@@ -128,7 +131,9 @@ def _config(spec) -> OrcConfig:
         weight_format=_DT[spec.weight_format], group_size=spec.group_size,
         shared_mode=_SHARED[spec.shared_mode], shared_intermediate=spec.shared_intermediate,
         latent_dim=spec.latent_dim, latent_use_norm=int(spec.latent_use_norm),
-        rms_eps=float(spec.rms_eps))
+        rms_eps=float(spec.rms_eps),
+        dense_weight_format=_DT["q4"] if spec.dense_format == "q4" else _DT[spec.act_dtype],
+        dense_group_size=spec.dense_group_size)
 
 
 def _check_storage(a: np.ndarray) -> np.ndarray:

@@ -47,6 +47,15 @@ def _dequant_mxfp4(q: np.ndarray, sbytes: np.ndarray) -> np.ndarray:
     return _E2M1_TABLE[codes] * scale
 
 
+def _dense(spec, w, name):
+    """A non-routed plane (router, shared, latent): activation dtype, or 4-bit affine words
+    with their own scales / biases when the spec quantises the dense parts."""
+    if spec.dense_format == "q4":
+        stem = name[:-2]
+        return _dequant(w[name], w[stem + "_s"], w[stem + "_z"], spec.dense_group_size)
+    return _decode(w[name])
+
+
 def _plane(spec, w, name):
     if spec.weight_format == "mxfp4":
         return _dequant_mxfp4(w[name], w[name[:-2] + "_s"])
@@ -84,7 +93,7 @@ def forward(spec, weights: Dict[str, np.ndarray], x: np.ndarray) -> Dict[str, np
     X = _decode(x)
     T, H = X.shape
     E, k, I = spec.num_experts, spec.top_k, spec.intermediate
-    logits = X @ _decode(weights["router_w"]).T
+    logits = X @ _dense(spec, weights, "router_w").T
     if spec.has_router_bias:
         logits = logits + _decode(weights["router_b"])
     if spec.scoring == "softmax_all":
@@ -106,7 +115,7 @@ def forward(spec, weights: Dict[str, np.ndarray], x: np.ndarray) -> Dict[str, np
         weight = weight / weight.sum(axis=1, keepdims=True)
     weight = weight * spec.routed_scaling_factor
 
-    U = X @ _decode(weights["latent_down_w"]).T if spec.latent_dim else X   # [T, K]
+    U = X @ _dense(spec, weights, "latent_down_w").T if spec.latent_dim else X   # [T, K]
     if spec.gate_up_interleaved:
         gu = _plane(spec, weights, "gate_up_w")                              # [E, 2I, K]
         Wg, Wu = gu[:, 0::2, :], gu[:, 1::2, :]
@@ -130,13 +139,13 @@ def forward(spec, weights: Dict[str, np.ndarray], x: np.ndarray) -> Dict[str, np
         if spec.latent_use_norm:
             rms = np.sqrt(np.mean(Yr * Yr, axis=1, keepdims=True) + spec.rms_eps)
             Yr = Yr / rms * _decode(weights["latent_norm_w"])
-        Yr = Yr @ _decode(weights["latent_up_w"]).T
+        Yr = Yr @ _dense(spec, weights, "latent_up_w").T
     coef = np.zeros((T, 2))
     if spec.shared_mode == "none":
         Y = Yr
     else:
-        S = _act(spec, X @ _decode(weights["shared_gate_w"]).T,
-                 X @ _decode(weights["shared_up_w"]).T) @ _decode(weights["shared_down_w"]).T
+        S = _act(spec, X @ _dense(spec, weights, "shared_gate_w").T,
+                 X @ _dense(spec, weights, "shared_up_w").T) @ _dense(spec, weights, "shared_down_w").T
         if spec.shared_mode == "add":
             Y = Yr + S
         else:

@@ -75,6 +75,8 @@ typedef struct {
     int32_t shared_mode, shared_intermediate;
     int32_t latent_dim, latent_use_norm;
     double rms_eps;
+    int32_t dense_weight_format;  /* router, shared and latent planes: act dtype or Q4 */
+    int32_t dense_group_size;     /* Q4 group of those planes                          */
 } orc_config;
 
 /* Host pointers to the stored tensors. Dense tensors are in the activation
@@ -88,6 +90,10 @@ typedef struct {
     const void *shared_gate_w, *shared_up_w, *shared_down_w;
     const void *latent_down_w, *latent_up_w, *latent_norm_w;
     const void *gate_up_s, *gate_up_z;  /* 4-bit interleaved gate_up plane */
+    /* 4-bit dense planes: bf16 scales / biases [rows, cols / dense_group_size] */
+    const void *router_s, *router_z, *shared_gate_s, *shared_gate_z, *shared_up_s, *shared_up_z;
+    const void *shared_down_s, *shared_down_z, *latent_down_s, *latent_down_z;
+    const void *latent_up_s, *latent_up_z;
 } orc_weights;
 
 static double bf16_bits_to_double(uint16_t b)
@@ -155,13 +161,26 @@ double orc_activation(int32_t act, double g, double v, double limit, double alph
     return gc / (1.0 + exp(-alpha * gc)) * (vc + 1.0);
 }
 
-/* y[r] = sum_c W[r, c] * v[c] for a dense [rows, cols] matrix in act dtype. */
-static void dense_matvec(const void *W, int32_t dtype, int64_t rows, int64_t cols,
-                         const double *v, double *y)
+/* W[r, c] of a dense (non-routed) [rows, cols] plane: the activation dtype, or
+ * 4-bit affine words with bf16 scales / biases per dense_group_size columns (a
+ * 4-bit checkpoint quantises its dense projections too: mlxcel issue #974's
+ * Jamba study, models/jamba-v0.1-4bit's quantised dense projections). */
+static double dense_plane_at(const orc_config *cfg, const void *w, const void *s, const void *z,
+                             int64_t cols, int64_t r, int64_t c)
+{
+    if (cfg->dense_weight_format == ORC_Q4)
+        return orc_dequant_q4((const uint32_t *)w, (const uint16_t *)s, (const uint16_t *)z,
+                              cols, cfg->dense_group_size, r, c);
+    return dense_at(w, cfg->act_dtype, r * cols + c);
+}
+
+/* y[r] = sum_c W[r, c] * v[c] for a dense [rows, cols] plane. */
+static void dense_matvec(const orc_config *cfg, const void *W, const void *S, const void *Z,
+                         int64_t rows, int64_t cols, const double *v, double *y)
 {
     for (int64_t r = 0; r < rows; ++r) {
         double acc = 0.0;
-        for (int64_t c = 0; c < cols; ++c) acc += dense_at(W, dtype, r * cols + c) * v[c];
+        for (int64_t c = 0; c < cols; ++c) acc += dense_plane_at(cfg, W, S, Z, cols, r, c) * v[c];
         y[r] = acc;
     }
 }
@@ -212,16 +231,15 @@ static void shared_expert(const orc_config *cfg, const orc_weights *w, const dou
                           double *out, double *h)
 {
     const int64_t H = cfg->hidden, Is = cfg->shared_intermediate;
-    const int32_t ad = cfg->act_dtype;
     for (int64_t i = 0; i < Is; ++i) {
         double g = 0.0, v = 0.0;
         for (int64_t c = 0; c < H; ++c) {
-            g += dense_at(w->shared_gate_w, ad, i * H + c) * x[c];
-            v += dense_at(w->shared_up_w, ad, i * H + c) * x[c];
+            g += dense_plane_at(cfg, w->shared_gate_w, w->shared_gate_s, w->shared_gate_z, H, i, c) * x[c];
+            v += dense_plane_at(cfg, w->shared_up_w, w->shared_up_s, w->shared_up_z, H, i, c) * x[c];
         }
         h[i] = orc_activation(cfg->activation, g, v, cfg->swiglu_limit, cfg->swiglu_alpha);
     }
-    dense_matvec(w->shared_down_w, ad, H, Is, h, out);
+    dense_matvec(cfg, w->shared_down_w, w->shared_down_s, w->shared_down_z, H, Is, h, out);
 }
 
 /* Router for one token: logits, selection keys, the chosen experts (or the
@@ -234,7 +252,8 @@ static void route_token(const orc_config *cfg, const orc_weights *w, const doubl
     const int32_t ad = cfg->act_dtype;
     for (int64_t e = 0; e < E; ++e) {
         double acc = 0.0;
-        for (int64_t c = 0; c < H; ++c) acc += dense_at(w->router_w, ad, e * H + c) * x[c];
+        for (int64_t c = 0; c < H; ++c)
+            acc += dense_plane_at(cfg, w->router_w, w->router_s, w->router_z, H, e, c) * x[c];
         if (cfg->has_router_bias) acc += dense_at(w->router_b, ad, e);
         logits[e] = acc;
     }
@@ -317,7 +336,7 @@ static void token_forward(const orc_config *cfg, const orc_weights *w, const dou
         double *o = (double *)malloc(sizeof(double) * (size_t)K);
         double *hb = (double *)malloc(sizeof(double) * (size_t)hmax);
         double *yr = (double *)malloc(sizeof(double) * (size_t)H);
-        if (cfg->latent_dim) dense_matvec(w->latent_down_w, ad, K, H, x, u);
+        if (cfg->latent_dim) dense_matvec(cfg, w->latent_down_w, w->latent_down_s, w->latent_down_z, K, H, x, u);
         else memcpy(u, x, sizeof(double) * (size_t)K);
         for (int64_t j = 0; j < k; ++j) {
             routed_expert(cfg, w, idx[j], u, o, hb);
@@ -331,7 +350,7 @@ static void token_forward(const orc_config *cfg, const orc_weights *w, const dou
                 for (int64_t r = 0; r < K; ++r)
                     acc[r] = acc[r] * inv * dense_at(w->latent_norm_w, ad, r);
             }
-            dense_matvec(w->latent_up_w, ad, H, K, acc, yr);
+            dense_matvec(cfg, w->latent_up_w, w->latent_up_s, w->latent_up_z, H, K, acc, yr);
         } else {
             memcpy(yr, acc, sizeof(double) * (size_t)H);
         }

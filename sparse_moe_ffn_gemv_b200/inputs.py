@@ -66,6 +66,10 @@ class MoeSpec:
     latent_dim: int = 0
     latent_use_norm: bool = False
     rms_eps: float = 1e-6
+    # non-routed planes (router, shared expert, latent projections): "act" = the activation
+    # dtype, "q4" = 4-bit affine with dense_group_size (the 2-row blend head stays in act)
+    dense_format: str = "act"
+    dense_group_size: int = 64
     token_counts: tuple = ()
 
     @property
@@ -217,13 +221,24 @@ def _expert_plane(spec: MoeSpec, name: str, rows: int, cols: int, pool) -> Dict[
     return {name: torch.stack([p[0] for p in parts])}
 
 
+def _dense_plane(spec: MoeSpec, name: str, rows: int, cols: int) -> Dict[str, torch.Tensor]:
+    """One non-routed plane [rows, cols] ~ N(0, 0.02): in the activation dtype, or (dense
+    format q4) the same draw encoded 4-bit affine, "router_w" -> companions "router_s",
+    "router_z"."""
+    w = _normal((rows, cols), 0.02, _seed(spec, name))
+    if spec.dense_format == "q4":
+        q, sc, bi = quantize_affine_q4(w, spec.dense_group_size)
+        return {name: q, name[:-2] + "_s": sc, name[:-2] + "_z": bi}
+    return {name: _storage(w, spec.act_dtype)}
+
+
 def make_weights(spec: MoeSpec, threads: Optional[int] = None) -> Dict[str, torch.Tensor]:
     """All block weights on the CPU, keyed by the C ABI's moe_weights field names."""
     H, E, I = spec.hidden, spec.num_experts, spec.intermediate
     K = spec.expert_in
     act = spec.act_dtype
     w: Dict[str, torch.Tensor] = {}
-    w["router_w"] = _storage(_normal((E, H), 0.02, _seed(spec, "router_w")), act)
+    w.update(_dense_plane(spec, "router_w", E, H))
     if spec.has_router_bias:
         w["router_b"] = _storage(_normal((E,), 0.02, _seed(spec, "router_b")), act)
     if spec.has_selection_bias:
@@ -247,13 +262,13 @@ def make_weights(spec: MoeSpec, threads: Optional[int] = None) -> Dict[str, torc
         w["down_b"] = _storage(_normal((E, K), 0.02, _seed(spec, "down_b")), act)
     if spec.shared_mode != "none":
         Is = spec.shared_intermediate
-        w["shared_gate_w"] = _storage(_normal((Is, H), 0.02, _seed(spec, "shared_gate_w")), act)
-        w["shared_up_w"] = _storage(_normal((Is, H), 0.02, _seed(spec, "shared_up_w")), act)
-        w["shared_down_w"] = _storage(_normal((H, Is), 0.02, _seed(spec, "shared_down_w")), act)
+        w.update(_dense_plane(spec, "shared_gate_w", Is, H))
+        w.update(_dense_plane(spec, "shared_up_w", Is, H))
+        w.update(_dense_plane(spec, "shared_down_w", H, Is))
     if spec.latent_dim:
         L = spec.latent_dim
-        w["latent_down_w"] = _storage(_normal((L, H), 0.02, _seed(spec, "latent_down_w")), act)
-        w["latent_up_w"] = _storage(_normal((H, L), 0.02, _seed(spec, "latent_up_w")), act)
+        w.update(_dense_plane(spec, "latent_down_w", L, H))
+        w.update(_dense_plane(spec, "latent_up_w", H, L))
         if spec.latent_use_norm:
             w["latent_norm_w"] = _storage(
                 _normal((L,), 0.1, _seed(spec, "latent_norm_w"), mean=1.0), act)

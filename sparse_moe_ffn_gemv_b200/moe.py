@@ -118,6 +118,10 @@ def _check(status: int, where: str):
 
 
 def config_from_spec(spec) -> MoeConfig:
+    if getattr(spec, "dense_format", "act") != "act":
+        # 4-bit router / shared / latent planes: the oracle evaluates them, the library's
+        # kernels read those planes in the activation dtype only
+        raise ValueError(f"dense_format {spec.dense_format!r} is not supported by the CUDA library")
     return MoeConfig(
         hidden=spec.hidden, num_experts=spec.num_experts, top_k=spec.top_k,
         intermediate=spec.intermediate, scoring=inputs.SCORING[spec.scoring],

@@ -149,6 +149,15 @@ def test_interleaved_4bit_plane_needs_its_own_companions(fmt):
     assert M.STATUS[M.moe_weights_validate(cfg, w3)] == "MOE_ERR_INVALID_ARGUMENT"
 
 
+def test_4bit_dense_planes_are_refused_by_the_binding():
+    """The oracle evaluates 4-bit router / shared / latent planes; the library reads those planes
+    in the activation dtype only, so the binding refuses such a spec instead of misreading it."""
+    from tiny_specs import DENSE_Q4
+    with pytest.raises(ValueError, match="dense_format"):
+        M.config_from_spec(DENSE_Q4)
+    assert M.moe_config_validate(M.config_from_spec(DENSE_Q4.replace(dense_format="act"))) == 0
+
+
 def test_group_must_divide_the_widths():
     spec = inputs.KLEAR_Q4.replace(intermediate=800)      # 800 % 64 != 0
     assert M.STATUS[M.moe_config_validate(M.config_from_spec(spec))] == "MOE_ERR_INVALID_QUANTIZATION"

@@ -15,8 +15,8 @@ import torch
 import oracle
 from oracle import bruteforce
 from sparse_moe_ffn_gemv_b200 import inputs
-from tiny_specs import (ALL, CLAMPED, LATENT, LATENT_NONORM, MXFP4, MXFP4_NATIVE, Q4, Q4_INTERLEAVED,
-                        ROUTER_BIAS, SIG_BLEND, np_weights, np_x, to_bf16_bits)
+from tiny_specs import (ALL, CLAMPED, DENSE_Q4, LATENT, LATENT_NONORM, MXFP4, MXFP4_NATIVE, Q4,
+                        Q4_INTERLEAVED, ROUTER_BIAS, SIG_BLEND, np_weights, np_x, to_bf16_bits)
 
 GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
 
@@ -469,6 +469,57 @@ def test_interleaved_4bit_block_equals_the_split_block_on_the_same_rows(spec):
     g = w["gate_up_w"]
     wswap["gate_up_w"] = np.stack([g[:, 1::2], g[:, 0::2]], axis=2).reshape(g.shape).copy()
     assert not np.array_equal(oracle.forward(spec, wswap, x)["y"], a["y"])
+
+
+# --- 4-bit dense planes (router, shared expert, latent projections) --------------
+def _exact_q4(rows, cols, group, rng):
+    """A 4-bit affine plane whose every weight is exact in bf16: scale 2^-6, bias -8 * 2^-6,
+    so weight = (q - 8) / 64 with q in [0, 15]. Returns (words, scales, biases, values)."""
+    q = rng.integers(0, 16, size=(rows, cols)).astype(np.uint32)
+    words = np.zeros((rows, cols // 8), dtype=np.uint32)
+    for j in range(8):
+        words |= q[:, j::8] << np.uint32(4 * j)
+    s = np.full((rows, cols // group), 2.0 ** -6, dtype=np.float32)
+    z = np.full((rows, cols // group), -8 * 2.0 ** -6, dtype=np.float32)
+    return words, to_bf16_bits(s), to_bf16_bits(z), (q.astype(np.float64) - 8) / 64
+
+
+def test_dense_q4_block_equals_the_bf16_block_on_the_same_exact_values():
+    """With every dense weight exact in bf16, the block reading the 4-bit dense planes equals
+    the block reading those values stored as bf16, exactly."""
+    spec = DENSE_Q4
+    rng = np.random.default_rng(3)
+    w = np_weights(spec)
+    shapes = {"router_w": (spec.num_experts, spec.hidden),
+              "shared_gate_w": (spec.shared_intermediate, spec.hidden),
+              "shared_up_w": (spec.shared_intermediate, spec.hidden),
+              "shared_down_w": (spec.hidden, spec.shared_intermediate),
+              "latent_down_w": (spec.latent_dim, spec.hidden),
+              "latent_up_w": (spec.hidden, spec.latent_dim)}
+    wq, wb = dict(w), dict(w)
+    for name, (r, c) in shapes.items():
+        words, s, z, vals = _exact_q4(r, c, spec.dense_group_size, rng)
+        wq[name], wq[name[:-2] + "_s"], wq[name[:-2] + "_z"] = words, s, z
+        wb[name] = to_bf16_bits(vals)
+        for comp in ("_s", "_z"):
+            wb.pop(name[:-2] + comp, None)
+    x = np_x(spec, 6)
+    a = oracle.forward(spec, wq, x)
+    b = oracle.forward(spec.replace(name="t_dense_as_bf16", dense_format="act"), wb, x)
+    np.testing.assert_array_equal(a["idx"], b["idx"])
+    np.testing.assert_array_equal(a["y"], b["y"])
+    assert np.abs(a["y"]).max() > 0
+
+
+def test_dense_q4_planes_change_the_output_against_the_unquantised_draw():
+    """The 4-bit dense planes are a different block from the drawn bf16 planes (they are read,
+    not ignored), yet close to it: the quantisation error of the dense parts is small."""
+    spec = DENSE_Q4
+    x = np_x(spec, 5)
+    yq = oracle.forward(spec, np_weights(spec), x)["y"]
+    y16 = oracle.forward(spec.replace(dense_format="act"), np_weights(spec.replace(dense_format="act")), x)["y"]
+    assert not np.array_equal(yq, y16)
+    assert np.abs(yq - y16).max() < 0.5 * np.abs(y16).max()
 
 
 # --- permutation -----------------------------------------------------------------

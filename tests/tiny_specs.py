@@ -53,8 +53,17 @@ Q4_INTERLEAVED = MoeSpec(
     scoring="softmax_topk", activation="swiglu_clamped", gate_up_interleaved=True,
     has_expert_bias=True, weight_format="q4", group_size=32)
 
+# every dense plane 4-bit as well (router, shared expert, latent projections; the blend head
+# stays bf16): a 4-bit checkpoint quantises its dense projections too (mlxcel issue #974)
+DENSE_Q4 = MoeSpec(
+    name="t_dense_q4", config_id=111, hidden=64, num_experts=6, top_k=2, intermediate=32,
+    scoring="sigmoid", has_selection_bias=True, norm_topk_prob=True, weight_format="q4",
+    group_size=32, shared_mode="add", shared_intermediate=32, latent_dim=32, latent_use_norm=True,
+    dense_format="q4", dense_group_size=32)
+DENSE_Q4_BLEND = Q4.replace(name="t_dense_q4_blend", config_id=112, dense_format="q4", dense_group_size=32)
+
 ALL = [inputs.TINY_F32, SIG_BLEND, CLAMPED, Q4, LATENT, ROUTER_BIAS, SEPARATE_BIAS,
-       LATENT_NONORM, MXFP4, MXFP4_NATIVE, Q4_INTERLEAVED]
+       LATENT_NONORM, MXFP4, MXFP4_NATIVE, Q4_INTERLEAVED, DENSE_Q4, DENSE_Q4_BLEND]
 
 
 def np_weights(spec, scale_weights: float = 1.0):
