@@ -192,7 +192,12 @@ MOE_API moe_status moe_permute(const moe_config *cfg, const int32_t *topk_idx, i
  * latent variant, else H). Overwrites y_acc. The expert_offsets / sorted_slot
  * inputs are moe_permute's outputs for the same topk_idx.
  * libmir-metal execute (gate_up then down weighted by routing.weights);
- * ferrox kimi_latent_moe_forward (combined += w * expert(latent)). */
+ * ferrox kimi_latent_moe_forward (combined += w * expert(latent)).
+ * Engine: the tcgen05 tensor-core kernel once 4*T*k >= E (bf16 activations,
+ * K and I multiples of 64), else the CUDA-core weight-streaming kernels; the
+ * environment variable MOE_PATH=gemv or MOE_PATH=tc forces one of them, for
+ * the router and latent projections too (read at every call). MOE_PDL=1 enables programmatic dependent launch between the
+ * kernels (off by default: it measured slower). */
 MOE_API moe_status moe_grouped_ffn(const moe_config *cfg, const moe_weights *w, const void *u, int64_t T,
                            const int32_t *expert_offsets, const int32_t *sorted_slot,
                            const float *topk_w, float *y_acc,
