@@ -20,7 +20,9 @@
  *  - All pointers are DEVICE pointers unless stated otherwise. The caller
  *    allocates, owns and frees every buffer, the workspace included; the
  *    library never allocates device memory, never frees, and keeps no pointer
- *    after a call returns.
+ *    after a call returns. The one exception is moe_permute_noalloc, whose
+ *    scratch is a fixed device array inside the library (see its declaration:
+ *    its size, and the race between calls that overlap on the GPU).
  *  - Calls are asynchronous on `stream` (a cudaStream_t; NULL = legacy default
  *    stream). T (the token count) is the product of the input's leading dims;
  *    T == 0 returns MOE_OK and launches nothing.
@@ -35,7 +37,9 @@
  *    bytes a multiple of 16 (hidden, intermediate, latent and shared widths
  *    multiples of 8 for bf16, of 4 for f32).
  *
- * Library: libmoe_b200.so (sm_100a). Thread-safe: calls keep no global state.
+ * Library: libmoe_b200.so (sm_100a). Thread-safe: calls keep no global device
+ * state, except moe_permute_noalloc's fixed scratch array, which all of its calls
+ * share (calls of it that overlap on the GPU race; serialise them).
  */
 #ifndef MOE_B200_H
 #define MOE_B200_H
@@ -232,10 +236,13 @@ MOE_API moe_status moe_block_forward(const moe_config *cfg, const moe_weights *w
  * process exits. Limits: T * top_k <= 65,536 slots and num_experts <= 512, else
  * MOE_ERR_SHAPE_OVERFLOW before any launch. The caller still passes every input and
  * output. device_status (optional, caller-owned int32 on the device, zeroed by the caller)
- * receives MOE_ERR_DEVICE_CHECK on an out-of-range expert id; when NULL that word lives in
- * the fixed array and is cleared on each call. No call allocates or frees anything. The
- * first call on each device looks up the array's device address (with that device
- * current): make that first call before any stream capture. All calls share the one array
+ * receives MOE_ERR_DEVICE_CHECK on an out-of-range expert id, and passing it is the only
+ * way to observe that check: with device_status NULL the bad slot is still dropped, but
+ * the error goes to a word inside the fixed array that no call reads. No call allocates
+ * or frees anything. The first call on each device (and the first after the device's
+ * context was replaced, e.g. by cudaDeviceReset) looks up the array's device address
+ * with that device current: make that first call before any stream capture. All calls
+ * share the one array
  * and leave their contents in it, so calls that overlap on the GPU (different streams
  * without ordering, or different host threads) race: serialise them. */
 MOE_API moe_status moe_permute_noalloc(const moe_config *cfg, const int32_t *topk_idx, int64_t T,

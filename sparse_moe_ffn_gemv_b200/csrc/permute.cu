@@ -7,6 +7,8 @@
 // warp match masks plus per-warp counts in shared memory, so equal experts keep
 // ascending slot order. Also emits the compact list of experts that received
 // tokens, which the expert kernels use to skip empty experts.
+#include <cuda.h>
+
 #include <mutex>
 
 #include "permute_dev.cuh"
@@ -133,21 +135,49 @@ static_assert((kNoAllocMaxExperts + 1) * 4 <= 2304, "active list fits its region
 static __device__ __align__(256) unsigned char g_permute_scratch[kNoAllocBytes];
 
 namespace {
-// Device address of g_permute_scratch on the current device, looked up once per device.
+// The current context's unique id (0 if no context is current or the driver lacks the call).
+unsigned long long current_context_id() {
+    using GetCurrentFn = CUresult (*)(CUcontext*);
+    using GetIdFn = CUresult (*)(CUcontext, unsigned long long*);
+    static GetCurrentFn get_current = nullptr;
+    static GetIdFn get_id = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            get_current = reinterpret_cast<GetCurrentFn>(p);
+        if (cudaGetDriverEntryPoint("cuCtxGetId", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            get_id = reinterpret_cast<GetIdFn>(p);
+    });
+    CUcontext ctx = nullptr;
+    unsigned long long id = 0;
+    if (get_current && get_id && get_current(&ctx) == CUDA_SUCCESS && ctx && get_id(ctx, &id) == CUDA_SUCCESS)
+        return id;
+    return 0;
+}
+
+// Device address of g_permute_scratch on the current device, looked up once per device and
+// context: a context created after a device reset gets its address looked up again.
 cudaError_t permute_scratch(void** out) {
     constexpr int kMaxDevices = 64;
     static void* addr[kMaxDevices] = {};
+    static unsigned long long ctx_of[kMaxDevices] = {};
     static std::mutex mu;
     int dev = 0;
     cudaError_t err = cudaGetDevice(&dev);
     if (err != cudaSuccess) return err;
     if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
     std::lock_guard<std::mutex> lock(mu);
-    if (!addr[dev]) {
+    const unsigned long long ctx = current_context_id();
+    if (!addr[dev] || ctx == 0 || ctx != ctx_of[dev]) {
         void* p = nullptr;
-        err = cudaGetSymbolAddress(&p, g_permute_scratch);
+        err = cudaGetSymbolAddress(&p, g_permute_scratch);  // also makes the device's context current
         if (err != cudaSuccess) return err;
         addr[dev] = p;
+        ctx_of[dev] = current_context_id();
     }
     *out = addr[dev];
     return cudaSuccess;

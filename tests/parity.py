@@ -8,8 +8,14 @@ the token's output is checked against the oracle evaluated with the GPU's
 expert set (several sets are then correct); outputs within max abs error
 <= 2e-2 * rms(output) for bf16 / 4-bit and <= 1e-4 for fp32. A bf16 output
 cannot hold the exact value: rounding it alone moves an element by up to half
-a bf16 ulp (2^-9 relative), which exceeds 2e-2 * rms where |y| > ~5 rms, so
-each bf16 element may also differ by half an ulp of the exact value.
+a bf16 ulp, which is between 2^-9 and 2^-8 of |y| (8 significant bits), and so
+exceeds 2e-2 * rms where |y| > ~5 rms. Each bf16 element may therefore also
+differ by half an ulp of the exact value, and check_block shows that this
+allowance covers only output rounding: at least 99.9% of the elements meet the
+plain bar, and every element over it is large (|y| > 3 rms, where half an ulp
+is at least 0.6% of rms and the rounding of the output is what pushes it over).
+The fp32 routed sums, which no output rounding touches, are checked against the
+plain bar with no allowance (tests/test_gpu_parity.py).
 """
 import numpy as np
 
@@ -18,6 +24,9 @@ import oracle
 TIE_WINDOW = 1e-5
 REL_TOL_BF16 = 2e-2
 ABS_TOL_F32 = 1e-4
+MIN_WITHIN_BAR = 0.999   # share of bf16 output elements that must meet the plain bar (2 may
+                         # miss it in batches under 2000 elements)
+BIG_OVER_RMS = 3.0       # an element over the plain bar must have |y_ref| > this many rms
 
 
 def tolerance(spec, y_ref: np.ndarray) -> float:
@@ -36,7 +45,8 @@ def half_ulp_bf16(v: np.ndarray) -> np.ndarray:
 
 def bound(spec, y_ref: np.ndarray) -> np.ndarray:
     """Per-element bound: the bar on the arithmetic, plus (bf16 outputs) the output
-    format's own rounding of the exact value, which no bf16 result can avoid."""
+    format's own rounding of the exact value (half an ulp), which no bf16 result can
+    avoid."""
     tol = tolerance(spec, y_ref)
     if spec.act_dtype == "f32":
         return np.full(y_ref.shape, tol)
@@ -86,5 +96,16 @@ def check_block(spec, w_np, x_np, tokens, y_gpu: np.ndarray, idx_gpu: np.ndarray
         i = np.unravel_index(np.argmax(err - lim), err.shape)
         raise AssertionError(f"{label}: error {err[i]:.3e} > bound {lim[i]:.3e} at token {tokens[i[0]]} "
                              f"col {i[1]} (bar {tol:.3e}, ref {y_ref[i]:.4f})")
+    plain = err <= tol
+    within = float(np.mean(plain)) if err.size else 1.0
+    rms = float(np.sqrt(np.mean(y_ref ** 2))) if y_ref.size else 0.0
+    big = float(np.abs(y_ref[~plain]).min() / rms) if (~plain).any() else None
+    if spec.act_dtype != "f32":
+        n_over = int((~plain).sum())
+        assert n_over <= max(2, (1.0 - MIN_WITHIN_BAR) * err.size), (
+            f"{label}: {n_over} of {err.size} elements over the plain bar ({within:.5f} within)")
+        assert big is None or big > BIG_OVER_RMS, (
+            f"{label}: an element over the plain bar has |y_ref| = {big:.2f} rms (not a large element)")
     return {"max_abs_err": worst, "tol": tol, "ties": len(ties), "tokens": len(tokens),
-            "within_bar_frac": float(np.mean(err <= tol))}
+            "within_bar_frac": within, "n_over_bar": int((~plain).sum()),
+            "min_abs_ref_over_bar_in_rms": big}

@@ -47,3 +47,32 @@ def test_l2_flush_between_timed_steps_only_where_the_weights_could_stay_in_l2():
     for spec, T in ((inputs.KLEAR_Q4, 1), (inputs.KLEAR_BF16, 4096)):
         cfg = bench.workload_config(spec, T, 1)
         assert cfg["l2"].startswith("L2 flushed" if bench.needs_l2_flush(spec, T) else "activated weights larger")
+
+
+def test_expert_launch_bytes_add_up_to_the_expert_planes():
+    """The gate/up and down launches read the routed planes once: their weight bytes
+    sum to the distinct experts' bytes plus the shared planes."""
+    s = inputs.KLEAR_BF16
+    T, nd = 4096, 216
+    r = bench.kernel_roles(s, T, nd)
+    H, k, I, Is = s.hidden, s.top_k, s.intermediate, s.shared_intermediate
+    io_gu = T * H * 2 + T * H * 2 + T * k * I * 2 + T * Is * 2       # u, x in; h, hs out
+    io_dn = T * k * I * 2 + T * Is * 2 + T * H * 4 + T * H * 4       # h, hs in; sums out
+    assert r["gate/up"]["bytes"] - io_gu + r["down"]["bytes"] - io_dn == nd * bench.expert_bytes(s) + 3 * Is * H * 2
+    assert r["gate/up"]["flops"] + r["down"]["flops"] + 2 * T * 256 * 2048 == bench.block_flops(s, T)
+
+
+def test_kernel_names_from_mangled_symbols():
+    n = bench.short_kernel_name
+    assert n("_ZN3moe12_GLOBAL__N_114tc_gemm_kernelILb1ELi128ELi4ELb0EEEvNS_8TcParamsE") == "tc_gemm_kernel<1,128,4,0>"
+    assert n("_ZN3moe12_GLOBAL__N_118gateup_gemv_kernelILi1EEEvNS_10GateUpArgsE") == "gateup_gemv_kernel<1>"
+    assert n("_ZN3moe12_GLOBAL__N_111topk_kernelENS_8TopkArgsE") == "topk_kernel"
+    table = [("topk_kernel", 1.0), ("tc_gemm_kernel<1,128,4,0>", 3.0), ("tc_gemm_kernel<0,128,4,0>", 2.0)]
+    assert bench.label_expert_launches(table) == (1, 2)
+
+
+def test_headline_is_the_largest_single_gpu_workload():
+    args = bench.parse([])
+    assert (args.workload, args.tokens) == ("latent_bf16", 8192)
+    big = max(bench.PREFILL, key=lambda w: bench.block_flops(inputs.WORKLOADS[w], bench.PREFILL[w]))
+    assert big == "latent_bf16"

@@ -94,13 +94,13 @@ def test_block_matches_oracle_small(spec, T, scale):
     full_check(spec, T, scale)
 
 
-FULL = [  # (spec, T, sampled tokens for the output check)
-    (inputs.KLEAR_BF16, 4096, 48),
-    (inputs.KLEAR_Q4, 2048, 32),
-    (inputs.CLAMPED_BF16, 8192, 16),
-    (inputs.LATENT_BF16, 128, 24),
-    (inputs.LATENT_BF16, 8192, 8),
-    (inputs.CLAMPED_MXFP4, 8192, 12),
+FULL = [  # (spec, T, tokens whose outputs are compared: None = every token)
+    (inputs.KLEAR_BF16, 4096, None),
+    (inputs.KLEAR_Q4, 2048, None),
+    (inputs.CLAMPED_BF16, 8192, 512),
+    (inputs.LATENT_BF16, 128, None),
+    (inputs.LATENT_BF16, 8192, 512),
+    (inputs.CLAMPED_MXFP4, 8192, 512),
 ]
 
 
@@ -116,10 +116,13 @@ def test_block_matches_oracle_full_size(spec, T, n_sample):
     from parity import index_mismatches
     ties = index_mismatches(idx, routed, spec.top_k)
     assert len(ties) <= max(2, T // 200)
-    # outputs of sampled tokens: first, last, and a seeded spread (ragged tail included)
-    rng = np.random.default_rng(T)
-    tokens = np.unique(np.concatenate([[0, T - 1], rng.choice(T, size=n_sample - 2, replace=False)]))
-    check_block(spec, wnp, x_np, tokens, y[tokens], idx[tokens], label=f"{spec.name} T={T}")
+    if n_sample is None:  # every token's output
+        tokens = np.arange(T)
+    else:  # first, last, and a seeded spread (ragged tail included)
+        rng = np.random.default_rng(T)
+        tokens = np.unique(np.concatenate([[0, T - 1], rng.choice(T, size=n_sample - 2, replace=False)]))
+    res = check_block(spec, wnp, x_np, tokens, y[tokens], idx[tokens], label=f"{spec.name} T={T}")
+    assert res["tokens"] == len(tokens)
 
 
 @pytest.mark.slow
@@ -312,14 +315,20 @@ def test_weight_streaming_and_tensor_core_paths_agree(spec, T, monkeypatch):
     assert blk.device_status() == 0
 
 
+ROUTED_SUM = [  # (spec, T): every non-latent workload, on both engines
+    (inputs.KLEAR_BF16, 200), (inputs.KLEAR_Q4, 96), (inputs.CLAMPED_BF16, 64),
+    (inputs.CLAMPED_MXFP4, 48), (inputs.CLAMPED_MXFP4_NATIVE, 40),
+]
+
+
 @pytest.mark.parametrize("path", ["gemv", "tc"])
-def test_routed_sum_in_fp32_meets_the_plain_bar(path, monkeypatch):
+@pytest.mark.parametrize("spec,T", ROUTED_SUM, ids=[f"{s.name}-T{T}" for s, T in ROUTED_SUM])
+def test_routed_sum_in_fp32_meets_the_plain_bar(spec, T, path, monkeypatch):
     """The routed sum y_acc is fp32 (no output rounding): it meets 2e-2 * rms with no
-    allowance, on both engines."""
+    allowance, on both engines, for every non-latent workload."""
     monkeypatch.setenv("MOE_PATH", path)
-    spec = inputs.KLEAR_BF16
     wcpu, wnp = weights(spec)
-    T, k, E, H = 200, spec.top_k, spec.num_experts, spec.hidden
+    k, E, H = spec.top_k, spec.num_experts, spec.hidden
     blk = M.MoeBlock(spec, wcpu, max_tokens=T)
     x_cpu = inputs.make_x(spec, T)
     x = x_cpu.cuda()
@@ -332,10 +341,14 @@ def test_routed_sum_in_fp32_meets_the_plain_bar(path, monkeypatch):
     M.moe_permute(blk.cfg, idx, T, off, ss, sp, blk.ws)
     M.moe_grouped_ffn(blk.cfg, blk.w, x, T, off, ss, w, y_acc, blk.ws)
     torch.cuda.synchronize()
-    ref = oracle.forward(spec.replace(shared_mode="none"), wnp, inputs.to_numpy_storage(x_cpu))
-    assert np.array_equal(np.sort(idx.cpu().numpy(), 1), np.sort(ref["idx"], 1))
+    assert blk.device_status() == 0
+    ref = oracle.forward(spec.replace(shared_mode="none", shared_intermediate=0), wnp,
+                         inputs.to_numpy_storage(x_cpu))
+    from parity import index_mismatches
+    ties = index_mismatches(idx.cpu().numpy(), ref, k)       # only inside the 1e-5 window
+    same = np.setdiff1d(np.arange(T), ties)                  # tokens with the oracle's set
     rms = np.sqrt(np.mean(ref["y"] ** 2))
-    assert np.abs(y_acc.cpu().numpy() - ref["y"]).max() <= 2e-2 * rms
+    assert np.abs(y_acc.cpu().numpy()[same] - ref["y"][same]).max() <= 2e-2 * rms
 
 
 def test_bounded_device_wait_reports_a_timeout_and_the_context_stays_usable():

@@ -4,8 +4,10 @@ Some callers cannot allocate device memory at the point where they route tokens 
 serving loop with a fixed memory reservation, a host whose allocator is not exposed to
 plug-ins, code being recorded into a CUDA graph). moe_permute_noalloc keeps its scratch
 in a fixed device array inside the library. These checks compare it with moe_permute
-(workspace-based) on two calls in a row of different sizes, so contents left in the
-shared array by the first call cannot go unnoticed. This file runs last in the suite.
+(workspace-based) on calls in a row of different sizes: four 2048-slot chunks, then two
+(the per-chunk histograms of the first call's later chunks are still in the array), then
+one, so contents left in the shared array by an earlier call would show. This file runs
+last in the suite.
 """
 import numpy as np
 import pytest
@@ -28,13 +30,14 @@ def _outputs(T, k, E):
     return (torch.full((E + 1,), -7, **dev), torch.full((T * k,), -7, **dev), torch.full((T * k,), -7, **dev))
 
 
-def test_noalloc_permutation_matches_the_workspace_permutation_on_two_calls():
+def test_noalloc_permutation_matches_the_workspace_permutation_on_calls_in_a_row():
     spec = inputs.KLEAR_BF16
     cfg = M.config_from_spec(spec)
     k, E = spec.top_k, spec.num_experts
     ws = torch.zeros(M.moe_workspace_size(cfg, 1000), dtype=torch.uint8, device="cuda")
-    # call 1: 1000 tokens (four 2048-slot chunks); call 2: 37 tokens (one chunk, fewer experts)
-    for T, seed in ((1000, 11), (37, 12)):
+    # 1000 tokens (four 2048-slot chunks), 300 tokens (two chunks), 37 tokens (one chunk,
+    # experts 64..255 empty)
+    for T, seed in ((1000, 11), (300, 15), (37, 12)):
         idx = _routing(T, k, E, seed)
         if T == 37:
             idx = idx % 64                      # experts 64..255 empty on the second call
