@@ -48,10 +48,10 @@ HEADLINE = ("latent_bf16", 8192)
 # Per-workload rows: the prefill-sized batch (graded on tensor-core peak) and the
 # decode-sized batches (graded on HBM bandwidth over the activated bytes).
 PREFILL = {"klear_bf16": 4096, "klear_q4": 2048, "clamped_bf16": 8192, "latent_bf16": 8192,
-           "clamped_mxfp4": 8192}
+           "clamped_mxfp4": 8192, "klear_q4_dense": 2048}
 DECODE = {"klear_bf16": (1, 8, 64), "klear_q4": (1, 32), "clamped_bf16": (1,), "latent_bf16": (1, 128),
-          "clamped_mxfp4": (1, 8)}
-ROW_ORDER = ("latent_bf16", "klear_bf16", "klear_q4", "clamped_bf16", "clamped_mxfp4")
+          "clamped_mxfp4": (1, 8), "klear_q4_dense": (1, 32)}
+ROW_ORDER = ("latent_bf16", "klear_bf16", "klear_q4", "clamped_bf16", "clamped_mxfp4", "klear_q4_dense")
 
 
 def parse(argv=None):
@@ -102,17 +102,25 @@ def expert_bytes(spec) -> int:
     return b
 
 
+def dense_plane_bytes(spec, rows: int, cols: int) -> int:
+    """Bytes of a router / shared / latent plane: the activation dtype, or 4-bit affine words
+    with a bf16 scale and bias per dense_group_size columns."""
+    if getattr(spec, "dense_format", "act") == "q4":
+        return rows * cols // 2 + rows * (cols // spec.dense_group_size) * 4
+    return rows * cols * (4 if spec.act_dtype == "f32" else 2)
+
+
 def dense_bytes(spec) -> int:
     """Non-routed weights read once per step: router, coefficient head, shared, latent."""
     ab = 4 if spec.act_dtype == "f32" else 2
     H, E = spec.hidden, spec.num_experts
-    b = E * H * ab + (E * 4 if spec.has_selection_bias else 0)
+    b = dense_plane_bytes(spec, E, H) + (E * 4 if spec.has_selection_bias else 0)
     if spec.shared_mode == "blend":
         b += 2 * H * ab
     if spec.shared_mode != "none":
-        b += 3 * spec.shared_intermediate * H * ab
+        b += 3 * dense_plane_bytes(spec, spec.shared_intermediate, H)
     if spec.latent_dim:
-        b += 2 * spec.latent_dim * H * ab + spec.latent_dim * ab
+        b += 2 * dense_plane_bytes(spec, spec.latent_dim, H) + spec.latent_dim * ab
     return b
 
 
@@ -141,8 +149,8 @@ def kernel_roles(spec, T: int, n_distinct: int) -> dict:
     H, k, I, K, Is = spec.hidden, spec.top_k, spec.intermediate, spec.expert_in, spec.shared_intermediate
     ab = 4 if spec.act_dtype == "f32" else 2
     sh = spec.shared_mode != "none"
-    gu_w = n_distinct * 2 * plane_bytes(spec, I, K) + (2 * Is * H * ab if sh else 0)
-    dn_w = n_distinct * plane_bytes(spec, K, I) + (H * Is * ab if sh else 0)
+    gu_w = n_distinct * 2 * plane_bytes(spec, I, K) + (2 * dense_plane_bytes(spec, Is, H) if sh else 0)
+    dn_w = n_distinct * plane_bytes(spec, K, I) + (dense_plane_bytes(spec, H, Is) if sh else 0)
     if spec.has_expert_bias:
         gu_w += n_distinct * 2 * I * ab
         dn_w += n_distinct * K * ab

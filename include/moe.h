@@ -123,6 +123,10 @@ typedef struct moe_config {
     int32_t latent_dim;            /* L; 0 = no latent projection                       */
     int32_t latent_use_norm;       /* 1: RMSNorm of the combined latent                 */
     float rms_eps;                 /* RMSNorm epsilon, finite > 0                       */
+    int32_t dense_format;          /* router, shared-expert and latent planes: 0 = in
+                                      act_dtype, MOE_DTYPE_Q4_AFFINE = 4-bit affine (needs
+                                      act BF16; the 2-row blend head stays in act_dtype)  */
+    int32_t dense_group_size;      /* Q4 group of those planes: 32, 64 or 128           */
 } moe_config;
 
 /*
@@ -149,6 +153,11 @@ typedef struct moe_config {
  *       order; gate_s/gate_z/up_s/up_z are unused.
  *   shared_gate_w, shared_up_w [Is, H]; shared_down_w [H, Is]
  *   latent_down_w [L, H]; latent_up_w [H, L]; latent_norm_w [L]
+ *   dense_format Q4 (a 4-bit checkpoint quantises its dense projections too; mlxcel issue
+ *       #974, the Jamba study): router_w, shared_*_w and latent_down_w / latent_up_w hold
+ *       uint32 words [rows, cols/8] like the routed Q4 planes, and <plane>_s / <plane>_z
+ *       (router_s, router_z, shared_gate_s, ...) their bf16 scales and biases
+ *       [rows, cols/dense_group_size]. coef_w / coef_b and latent_norm_w stay in act_dtype.
  */
 typedef struct moe_weights {
     const void *router_w, *router_b, *selection_bias, *coef_w, *coef_b;
@@ -157,6 +166,9 @@ typedef struct moe_weights {
     const void *shared_gate_w, *shared_up_w, *shared_down_w;
     const void *latent_down_w, *latent_up_w, *latent_norm_w;
     const void *gate_up_s, *gate_up_z;  /* 4-bit interleaved gate_up plane: its scales / biases */
+    const void *router_s, *router_z;    /* dense_format Q4: scales / biases of each dense plane */
+    const void *shared_gate_s, *shared_gate_z, *shared_up_s, *shared_up_z, *shared_down_s, *shared_down_z;
+    const void *latent_down_s, *latent_down_z, *latent_up_s, *latent_up_z;
 } moe_weights;
 
 /* Checks a config on the host (Klear PR "Other guards": zero checks before
@@ -207,6 +219,23 @@ MOE_API moe_status moe_grouped_ffn(const moe_config *cfg, const moe_weights *w, 
                            const float *topk_w, float *y_acc,
                            void *ws, size_t ws_bytes, moe_stream_t stream);
 
+/* Routed experts of one contiguous expert range (expert-parallel sharding; the pages run
+ * the block on one device, so this call has no counterpart there). Computes what
+ * moe_grouped_ffn computes, restricted to experts [expert_begin, expert_end): y_acc [T, K]
+ * f32 = sum over each token's slots routed to those experts of topk_w[slot] *
+ * expert(u[token]), zero where a token has none. The routed planes of `w` (gate/up/down,
+ * their biases and 4-bit companions) hold ONLY these experts, stacked from expert_begin
+ * (plane g is expert expert_begin + g); the dense planes are as for moe_grouped_ffn.
+ * expert_offsets / sorted_slot / topk_w are the full permutation of all E experts, as
+ * moe_permute writes it. The partial sums of ranges that cover [0, E) add up to
+ * moe_grouped_ffn's result (one range per GPU, followed by a reduce-scatter of y_acc over
+ * the token dimension). 0 <= expert_begin < expert_end <= E, else MOE_ERR_INVALID_ARGUMENT.
+ * Overwrites y_acc. */
+MOE_API moe_status moe_grouped_ffn_experts(const moe_config *cfg, const moe_weights *w, const void *u, int64_t T,
+                                   const int32_t *expert_offsets, const int32_t *sorted_slot,
+                                   const float *topk_w, int32_t expert_begin, int32_t expert_end,
+                                   float *y_acc, void *ws, size_t ws_bytes, moe_stream_t stream);
+
 /* Latent down projection (first half of a8): z [T, L] (act_dtype) = x Wdp^T.
  * ferrox kimi_latent_moe_forward: latent = down_proj(hidden). */
 MOE_API moe_status moe_latent_down(const moe_config *cfg, const moe_weights *w, const void *x, int64_t T,
@@ -254,7 +283,8 @@ MOE_API moe_status moe_permute_noalloc(const moe_config *cfg, const int32_t *top
  * MOE_ERR_DEVICE_TIMEOUT) and clears it. The first 256 bytes of a workspace
  * hold this word and a launch counter that every call leaves at zero: a new
  * workspace must be zero-filled (or cleared with moe_clear_device_status)
- * before its first use. */
+ * before its first use. The same region holds the grid-barrier counters of the persistent
+ * decode kernel, which every launch also leaves at zero. */
 MOE_API moe_status moe_read_device_status(void *ws, moe_stream_t stream);
 
 /* Clears the workspace's 256-byte status region, asynchronously on `stream`. */
@@ -267,6 +297,15 @@ MOE_API moe_status moe_clear_device_status(void *ws, moe_stream_t stream);
  * moe_read_device_status) and returns; nothing traps or hangs. Asynchronous on
  * `stream`; MOE_ERR_INVALID_ARGUMENT for a NULL ws or an out-of-range timeout. */
 MOE_API moe_status moe_selftest_bounded_wait(void *ws, int64_t timeout_ns, moe_stream_t stream);
+
+/* Failure-detection self test of the grid barrier the persistent decode kernel uses
+ * between its phases (moe_block_forward with up to 8 tokens): one block arrives at a
+ * barrier that needs two arrivals and polls it with the same %globaltimer deadline
+ * (timeout_ns, 0 < timeout_ns <= 1e9); when it gives up it records
+ * MOE_ERR_DEVICE_TIMEOUT in the status word of `ws` and returns, and the counter is put
+ * back to zero. Asynchronous on `stream`; MOE_ERR_INVALID_ARGUMENT for a NULL ws or an
+ * out-of-range timeout. */
+MOE_API moe_status moe_selftest_grid_wait(void *ws, int64_t timeout_ns, moe_stream_t stream);
 
 /* Static, NUL-terminated description of a status code. */
 MOE_API const char *moe_status_string(moe_status status);

@@ -52,7 +52,6 @@ WsLayout ws_layout(const moe_config& c, int64_t T) {
     L.nrm = take(Ld ? T * Ld * ab : 0);
     const bool tc = c.act_dtype == MOE_DTYPE_BF16;  // bf16 or 4-bit weights
     L.uperm = take(tc ? T * k * K * 2 : 0);
-    L.oslot = take(tc ? T * k * K * 2 : 0);
     L.tiles = take((E + 1) * 4);
     L.total = off;
     return L;
@@ -67,6 +66,24 @@ namespace {
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 bool finite_pos(float v) { return std::isfinite(v) && v > 0.f; }
+
+bool dense_q4(const moe_config* c) { return c->dense_format == MOE_DTYPE_Q4_AFFINE; }
+
+// Weight operand(s) of a dense (one-group) tensor-core problem: bf16 [M, K], or 4-bit affine
+// words [M, K / 8] with bf16 scales / biases per dense_group_size columns (the second
+// operand w1 only in gate/up mode).
+bool tc_dense_weights(const moe_config* c, TcProblem& p, CUtensorMap* m0, CUtensorMap* m1, const void* w0,
+                      const void* s0, const void* z0, const void* w1, const void* s1, const void* z1, int M, int K) {
+    if (dense_q4(c)) {
+        p.q4 = 1;
+        p.mx = 0;
+        p.group_size = c->dense_group_size;
+        p.qs0 = s0; p.qz0 = z0; p.qs1 = s1; p.qz1 = z1;
+        return tc_q4_weight_map(m0, w0, 1, M, K) && (!w1 || tc_q4_weight_map(m1, w1, 1, M, K));
+    }
+    return tc_weight_map(m0, w0, 1, M, K, false) && (!w1 || tc_weight_map(m1, w1, 1, M, K, false));
+}
+
 
 moe_status validate_config(const moe_config* c) {
     if (!c) return MOE_ERR_INVALID_ARGUMENT;
@@ -105,6 +122,14 @@ moe_status validate_config(const moe_config* c) {
     if (c->weight_format == MOE_DTYPE_MXFP4) {  // OCP MX: blocks of 32 elements, 4-bit E2M1
         if (c->bits != 4 || c->group_size != 32) return MOE_ERR_INVALID_QUANTIZATION;
         if (K % 64 != 0 || c->intermediate % 64 != 0) return MOE_ERR_INVALID_QUANTIZATION;
+    }
+    // 4-bit dense planes (router, shared expert, latent projections)
+    if (c->dense_format != 0 && c->dense_format != MOE_DTYPE_Q4_AFFINE) return MOE_ERR_INVALID_ARGUMENT;
+    if (c->dense_format == MOE_DTYPE_Q4_AFFINE) {
+        if (c->act_dtype != MOE_DTYPE_BF16) return MOE_ERR_UNSUPPORTED;
+        const int g = c->dense_group_size;
+        if (g != 32 && g != 64 && g != 128) return MOE_ERR_INVALID_QUANTIZATION;
+        if (c->hidden % g || c->shared_intermediate % g || c->latent_dim % g) return MOE_ERR_INVALID_QUANTIZATION;
     }
     // 16-byte rows
     const int q = c->act_dtype == MOE_DTYPE_F32 ? 4 : 8;
@@ -149,11 +174,24 @@ moe_status validate_weights(const moe_config* c, const moe_weights* w) {
         return MOE_ERR_MISSING_TENSOR;
     if (c->latent_dim && (!need(w->latent_down_w) || !need(w->latent_up_w))) return MOE_ERR_MISSING_TENSOR;
     if (c->latent_use_norm && !need(w->latent_norm_w)) return MOE_ERR_MISSING_TENSOR;
+    if (c->dense_format == MOE_DTYPE_Q4_AFFINE) {
+        if (!need(w->router_s) || !need(w->router_z)) return MOE_ERR_MISSING_TENSOR;
+        if (c->shared_mode != MOE_SHARED_NONE &&
+            (!need(w->shared_gate_s) || !need(w->shared_gate_z) || !need(w->shared_up_s) || !need(w->shared_up_z) ||
+             !need(w->shared_down_s) || !need(w->shared_down_z)))
+            return MOE_ERR_MISSING_TENSOR;
+        if (c->latent_dim &&
+            (!need(w->latent_down_s) || !need(w->latent_down_z) || !need(w->latent_up_s) || !need(w->latent_up_z)))
+            return MOE_ERR_MISSING_TENSOR;
+    }
     const void* all[] = {w->router_w, w->router_b, w->selection_bias, w->coef_w, w->coef_b,
                          w->gate_w, w->up_w, w->gate_up_w, w->gate_b, w->up_b, w->gate_up_b,
                          w->down_w, w->down_b, w->gate_s, w->gate_z, w->up_s, w->up_z,
                          w->down_s, w->down_z, w->shared_gate_w, w->shared_up_w, w->shared_down_w,
-                         w->latent_down_w, w->latent_up_w, w->latent_norm_w, w->gate_up_s, w->gate_up_z};
+                         w->latent_down_w, w->latent_up_w, w->latent_norm_w, w->gate_up_s, w->gate_up_z,
+                         w->router_s, w->router_z, w->shared_gate_s, w->shared_gate_z, w->shared_up_s,
+                         w->shared_up_z, w->shared_down_s, w->shared_down_z, w->latent_down_s, w->latent_down_z,
+                         w->latent_up_s, w->latent_up_z};
     for (const void* p : all)
         if (p && !aligned16(p)) return MOE_ERR_INVALID_ARGUMENT;
     return MOE_OK;
@@ -175,12 +213,13 @@ moe_status check_ptr(const void* p) {
 // Which engine runs a GEMM: weight-streaming CUDA-core kernels (few tokens per
 // weight row) or the tcgen05 tensor-core kernel (many). MOE_PATH=gemv|tc forces one
 // where both are possible (used by the tests to cross-check the two).
-enum { kPathAuto = 0, kPathGemv = 1, kPathTc = 2 };
+enum { kPathAuto = 0, kPathGemv = 1, kPathTc = 2, kPathDecode = 3 };
 int path_override() {
     const char* e = getenv("MOE_PATH");
     if (!e) return kPathAuto;
     if (!strcmp(e, "gemv")) return kPathGemv;
     if (!strcmp(e, "tc")) return kPathTc;
+    if (!strcmp(e, "decode")) return kPathDecode;
     return kPathAuto;
 }
 bool dense_tc(const moe_config* c, int64_t T, int K) {
@@ -197,6 +236,57 @@ bool routed_tc(const moe_config* c, int64_t T) {
     if (expert_in(*c) % 64 != 0 || c->intermediate % 64 != 0) return false;
     const int o = path_override();
     return o == kPathTc || (o == kPathAuto && 4 * T * c->top_k >= int64_t(c->num_experts));
+}
+
+// The whole block as one persistent launch (csrc/decode.cu) for up to 8 tokens without a
+// latent projection, bf16 activations and bf16 / 4-bit routed planes; MOE_PATH=gemv or tc
+// selects the multi-kernel engines instead.
+DecodeArgs decode_args(const moe_config* c, const moe_weights* w, const void* x, int64_t T, void* y, void* ws,
+                       const WsLayout& L) {
+    DecodeArgs d;
+    d.T = int(T); d.H = c->hidden; d.E = c->num_experts; d.k = c->top_k; d.I = c->intermediate;
+    d.Is = c->shared_intermediate;
+    d.wf = c->weight_format; d.interleaved = c->gate_up_interleaved; d.has_bias = c->has_expert_bias;
+    d.group_size = c->group_size;
+    d.act = c->activation; d.limit = c->swiglu_limit; d.alpha = c->swiglu_alpha;
+    d.scoring = c->scoring; d.norm = c->norm_topk_prob; d.has_sel = c->has_selection_bias;
+    d.shared_mode = c->shared_mode;
+    d.router_w = w->router_w; d.router_b = c->has_router_bias ? w->router_b : nullptr;
+    if (c->shared_mode == MOE_SHARED_BLEND) { d.coef_w = w->coef_w; d.coef_b = w->coef_b; }
+    d.sel_bias = static_cast<const float*>(w->selection_bias);
+    d.gate_w = w->gate_w; d.up_w = w->up_w; d.gate_up_w = w->gate_up_w;
+    d.gate_s = c->gate_up_interleaved ? w->gate_up_s : w->gate_s;
+    d.gate_z = c->gate_up_interleaved ? w->gate_up_z : w->gate_z;
+    d.up_s = w->up_s; d.up_z = w->up_z;
+    d.gate_b = w->gate_b; d.up_b = w->up_b; d.gate_up_b = w->gate_up_b;
+    d.down_w = w->down_w; d.down_s = w->down_s; d.down_z = w->down_z; d.down_b = w->down_b;
+    if (c->shared_mode != MOE_SHARED_NONE) { d.sg_w = w->shared_gate_w; d.su_w = w->shared_up_w; d.sd_w = w->shared_down_w; }
+    if (dense_q4(c)) {
+        d.dense_q4 = 1;
+        d.dense_group = c->dense_group_size;
+        d.router_s = w->router_s; d.router_z = w->router_z;
+        d.sg_s = w->shared_gate_s; d.sg_z = w->shared_gate_z; d.su_s = w->shared_up_s; d.su_z = w->shared_up_z;
+        d.sd_s = w->shared_down_s; d.sd_z = w->shared_down_z;
+    }
+    d.x = x; d.y = y;
+    d.logits = reinterpret_cast<float*>(static_cast<char*>(ws) + L.logits); d.ld_logits = L.ld_logits;
+    d.h = static_cast<char*>(ws) + L.h;
+    d.hs = static_cast<char*>(ws) + L.hs;
+    d.status = reinterpret_cast<int*>(static_cast<char*>(ws) + L.status);
+    d.bar = reinterpret_cast<unsigned*>(static_cast<char*>(ws) + L.status + kDecodeBarOffset);
+    // the down rows of the activated experts are prefetched into L2 only where they fit
+    // comfortably beside the gate/up stream
+    const int64_t drow = c->weight_format == MOE_DTYPE_BF16 ? int64_t(c->intermediate) * 2 : c->intermediate / 2;
+    const int64_t most = std::min<int64_t>(c->num_experts, T * c->top_k);
+    d.l2_prefetch = most * c->hidden * drow + int64_t(c->hidden) * c->shared_intermediate * 2 <= (int64_t(40) << 20);
+    return d;
+}
+
+bool use_decode(const moe_config* c, int64_t T, const DecodeArgs& d) {
+    if (c->latent_dim || c->act_dtype != MOE_DTYPE_BF16 || c->weight_format == MOE_DTYPE_F32) return false;
+    const int o = path_override();
+    if (o == kPathGemv || o == kPathTc) return false;
+    return T >= 1 && T <= 8 && decode_smem_bytes(d) > 0;
 }
 
 #define MOE_CHECK(expr)                          \
@@ -245,6 +335,11 @@ DenseGemvArgs router_args(const moe_config* c, const moe_weights* w, const void*
     r.ld_out = L.ld_logits;
     r.out_f32 = 1;
     r.act_dtype = c->act_dtype;
+    if (dense_q4(c)) {
+        r.s0 = w->router_s;
+        r.z0 = w->router_z;
+        r.group0 = c->dense_group_size;
+    }
     return r;
 }
 
@@ -291,9 +386,10 @@ moe_status run_route(const moe_config* c, const moe_weights* w, const void* x, i
             p.bias0 = i == 0 ? r.b0 : r.b1;
             p.out = at<float>(ws, L.logits) + (i == 0 ? 0 : c->num_experts);
             p.ld_out = L.ld_logits;
-            if (!tc_weight_map(&P.a0[i], i == 0 ? r.W0 : r.W1, 1, p.M, c->hidden, false) ||
-                !tc_token_map(P.b[i], x, T, c->hidden, kTcBN))
-                return MOE_ERR_CUDA;
+            const bool wok = i == 0 ? tc_dense_weights(c, p, &P.a0[i], nullptr, r.W0, w->router_s, w->router_z, nullptr,
+                                                       nullptr, nullptr, p.M, c->hidden)
+                                    : tc_weight_map(&P.a0[i], r.W1, 1, p.M, c->hidden, false);  // blend head: act dtype
+            if (!wok || !tc_token_map(P.b[i], x, T, c->hidden, kTcBN)) return MOE_ERR_CUDA;
         }
         P.nprob = np;
         P.status = at<int>(ws, L.status);
@@ -340,13 +436,22 @@ moe_status run_permute(const moe_config* c, const int32_t* idx, int64_t T, int32
     return MOE_OK;
 }
 
+// The routed experts a call runs: [e0, e0 + ne). The routed planes of moe_weights hold
+// exactly these experts (plane g = expert e0 + g); offsets / sorted_slot stay the full
+// permutation's, and only the slots of these experts are read.
+struct ExpertRange {
+    int e0 = 0, ne = 0;
+};
+
 // Tensor-core part of a4 + a5 (+ a6): the routed groups (rtc) and/or the shared expert (stc).
-// The routed down GEMM writes every slot's weighted output row (oslot); a token's routed
-// sum is the sum of its k rows, taken by the combine.
+// The routed down GEMM's epilogue multiplies each slot's output row by its routing weight
+// and adds it into the token's fp32 routed sum y_acc, which must be zero on entry.
 moe_status run_experts_tc(const moe_config* c, const moe_weights* w, const void* u, const void* x, int64_t T,
                           const int32_t* offsets, const int32_t* sorted_slot, const float* topk_w,
-                          bool rtc, bool stc, void* ws, const WsLayout& L, cudaStream_t s) {
-    const int K = expert_in(*c), I = c->intermediate, E = c->num_experts, k = c->top_k, H = c->hidden;
+                          float* y_acc, bool rtc, bool stc, ExpertRange rg, void* ws, const WsLayout& L,
+                          cudaStream_t s) {
+    const int K = expert_in(*c), I = c->intermediate, E = rg.ne, k = c->top_k, H = c->hidden;
+    const int32_t* goff = offsets ? offsets + rg.e0 : nullptr;  // the range's offsets [ne + 1]
     const int Is = c->shared_intermediate;
     const int64_t S = T * k;
     const int64_t n_dense = (T + kTcBN - 1) / kTcBN;
@@ -354,7 +459,7 @@ moe_status run_experts_tc(const moe_config* c, const moe_weights* w, const void*
     void* h = at<void>(ws, L.h);
     void* hs = at<void>(ws, L.hs);
     const int32_t* tiles = at<int32_t>(ws, L.tiles);
-    if (rtc) MOE_CUDA(launch_gather_rows(u, K, sorted_slot, k, S, uperm, s));
+    if (rtc) MOE_CUDA(launch_gather_rows(u, K, sorted_slot, k, S, uperm, s, goff, goff + E));
     {  // gate/up + activation
         TcParams P;
         int np = 0;
@@ -365,8 +470,8 @@ moe_status run_experts_tc(const moe_config* c, const moe_weights* w, const void*
             p.M = Is; p.K = H; p.m_blocks = (Is + kTcRowsGateUp - 1) / kTcRowsGateUp;
             p.rows = int(T); p.n_tiles = int(n_dense);
             p.out = hs; p.ld_out = Is;
-            if (!tc_weight_map(&P.a0[np], w->shared_gate_w, 1, Is, H, false) ||
-                !tc_weight_map(&P.a1[np], w->shared_up_w, 1, Is, H, false) ||
+            if (!tc_dense_weights(c, p, &P.a0[np], &P.a1[np], w->shared_gate_w, w->shared_gate_s, w->shared_gate_z,
+                                  w->shared_up_w, w->shared_up_s, w->shared_up_z, Is, H) ||
                 !tc_token_map(P.b[np], x, T, H, kTcBN))
                 return MOE_ERR_CUDA;
             max_tiles += int64_t(p.m_blocks) * p.n_tiles;
@@ -376,7 +481,7 @@ moe_status run_experts_tc(const moe_config* c, const moe_weights* w, const void*
             TcProblem& p = P.p[np];
             p.mode = kEpiGateUp;
             p.M = I; p.K = K; p.m_blocks = (I + kTcRowsGateUp - 1) / kTcRowsGateUp;
-            p.grouped = 1; p.num_groups = E; p.offsets = offsets; p.tile_start = tiles;
+            p.grouped = 1; p.num_groups = E; p.offsets = goff; p.tile_start = tiles;
             p.out = h; p.ld_out = I;
             p.interleaved = c->gate_up_interleaved;  // bf16 / f32 planes: one 4-D map
             if (c->has_expert_bias) {
@@ -440,7 +545,8 @@ moe_status run_experts_tc(const moe_config* c, const moe_weights* w, const void*
             p.M = H; p.K = Is; p.m_blocks = (H + kTcRows - 1) / kTcRows;
             p.rows = int(T); p.n_tiles = int(n_dense);
             p.out = at<float>(ws, L.s_acc); p.ld_out = H;
-            if (!tc_weight_map(&P.a0[np], w->shared_down_w, 1, H, Is, false) ||
+            if (!tc_dense_weights(c, p, &P.a0[np], nullptr, w->shared_down_w, w->shared_down_s, w->shared_down_z,
+                                  nullptr, nullptr, nullptr, H, Is) ||
                 !tc_token_map(P.b[np], hs, T, Is, kTcBN))
                 return MOE_ERR_CUDA;
             max_tiles += int64_t(p.m_blocks) * p.n_tiles;
@@ -448,12 +554,12 @@ moe_status run_experts_tc(const moe_config* c, const moe_weights* w, const void*
         }
         if (rtc) {
             TcProblem& p = P.p[np];
-            p.mode = kEpiSlotRows;
+            p.mode = kEpiScatterAdd;
             p.M = K; p.K = I; p.m_blocks = (K + kTcRows - 1) / kTcRows;
-            p.grouped = 1; p.num_groups = E; p.offsets = offsets; p.tile_start = tiles;
+            p.grouped = 1; p.num_groups = E; p.offsets = goff; p.tile_start = tiles;
             p.sorted_slot = sorted_slot; p.topk_w = topk_w; p.k = k;
             p.bias0 = c->has_expert_bias ? w->down_b : nullptr;
-            p.out = at<__nv_bfloat16>(ws, L.oslot); p.ld_out = K;
+            p.out = y_acc; p.ld_out = K;
             bool ok;
             if (c->weight_format == MOE_DTYPE_Q4_AFFINE || c->weight_format == MOE_DTYPE_MXFP4) {
                 p.q4 = 1;
@@ -480,15 +586,16 @@ moe_status run_experts_tc(const moe_config* c, const moe_weights* w, const void*
 struct RoutedSum {
     const void* rows = nullptr;
     int nsum = 1;
-    int dtype = MOE_DTYPE_F32;  // bf16 for the tensor-core path's per-slot rows
+    int dtype = MOE_DTYPE_F32;
 };
 
-// a4 + a5 (+ a6 when with_shared). On the weight-streaming path y_acc must be zero on
-// entry (scatter-add); the tensor-core path writes per-slot rows instead.
+// a4 + a5 (+ a6 when with_shared). y_acc must be zero on entry: both engines add each
+// slot's weighted output into its token's row.
 moe_status run_experts(const moe_config* c, const moe_weights* w, const void* u, const void* x, int64_t T,
                        const int32_t* offsets, const int32_t* sorted_slot, const float* topk_w,
                        float* y_acc, bool with_routed, bool with_shared, void* ws, const WsLayout& L,
-                       cudaStream_t s, RoutedSum* sum) {
+                       cudaStream_t s, RoutedSum* sum, ExpertRange rg = ExpertRange{}) {
+    if (rg.ne == 0) rg.ne = c->num_experts;
     const int K = expert_in(*c);
     const bool sh = with_shared && c->shared_mode != MOE_SHARED_NONE;
     const bool rtc = with_routed && routed_tc(c, T);
@@ -496,13 +603,13 @@ moe_status run_experts(const moe_config* c, const moe_weights* w, const void* u,
     const bool stc = sh && c->shared_intermediate % 64 == 0 && c->hidden % 64 == 0 &&
                      c->act_dtype == MOE_DTYPE_BF16 && (dense_tc(c, T, c->hidden) || rtc);
     if (sum) {
-        sum->rows = rtc ? at<void>(ws, L.oslot) : static_cast<const void*>(y_acc);
-        sum->nsum = rtc ? c->top_k : 1;
-        sum->dtype = rtc ? MOE_DTYPE_BF16 : MOE_DTYPE_F32;
+        sum->rows = y_acc;
+        sum->nsum = 1;
+        sum->dtype = MOE_DTYPE_F32;
     }
     if (rtc || stc)
-        MOE_CHECK(run_experts_tc(c, w, u, x, T, offsets, sorted_slot, topk_w, rtc, stc, ws, L, s));
-    const int64_t groups = (with_routed && !rtc) ? std::min<int64_t>(c->num_experts, T * c->top_k) : 0;
+        MOE_CHECK(run_experts_tc(c, w, u, x, T, offsets, sorted_slot, topk_w, y_acc, rtc, stc, rg, ws, L, s));
+    const int64_t groups = (with_routed && !rtc) ? std::min<int64_t>(rg.ne, T * c->top_k) : 0;
     if (groups == 0 && (!sh || stc)) return MOE_OK;
     GateUpArgs g;
     g.wf = c->weight_format;
@@ -514,7 +621,7 @@ moe_status run_experts(const moe_config* c, const moe_weights* w, const void* u,
     g.gate_z = c->gate_up_interleaved ? w->gate_up_z : w->gate_z;
     g.up_s = w->up_s; g.up_z = w->up_z;
     g.gate_b = w->gate_b; g.up_b = w->up_b; g.gate_up_b = w->gate_up_b;
-    g.offsets = offsets;
+    g.offsets = offsets ? offsets + rg.e0 : nullptr;
     g.sorted_slot = sorted_slot;
     g.active = at<int32_t>(ws, L.active);
     g.k = c->top_k;
@@ -530,6 +637,11 @@ moe_status run_experts(const moe_config* c, const moe_weights* w, const void* u,
         g.Hs = c->hidden;
         g.xs = x;
         g.hs = at<void>(ws, L.hs);
+        if (dense_q4(c)) {
+            g.sg_s = w->shared_gate_s; g.sg_z = w->shared_gate_z;
+            g.su_s = w->shared_up_s; g.su_z = w->shared_up_z;
+            g.s_group = c->dense_group_size;
+        }
     }
     g.T = T;
     g.act = c->activation;
@@ -541,7 +653,7 @@ moe_status run_experts(const moe_config* c, const moe_weights* w, const void* u,
     d.has_bias = c->has_expert_bias;
     d.group_size = c->group_size;
     d.down_w = w->down_w; d.down_s = w->down_s; d.down_z = w->down_z; d.down_b = w->down_b;
-    d.offsets = offsets;
+    d.offsets = offsets ? offsets + rg.e0 : nullptr;
     d.sorted_slot = sorted_slot;
     d.active = at<int32_t>(ws, L.active);
     d.topk_w = topk_w;
@@ -557,6 +669,10 @@ moe_status run_experts(const moe_config* c, const moe_weights* w, const void* u,
         d.Hs = c->hidden;
         d.hs = at<void>(ws, L.hs);
         d.s_acc = at<float>(ws, L.s_acc);
+        if (dense_q4(c)) {
+            d.sd_s = w->shared_down_s; d.sd_z = w->shared_down_z;
+            d.s_group = c->dense_group_size;
+        }
     }
     d.T = T;
     MOE_CUDA(launch_down_gemv(d, s));
@@ -576,6 +692,11 @@ moe_status run_latent_down(const moe_config* c, const moe_weights* w, const void
     r.ld_out = c->latent_dim;
     r.out_f32 = 0;
     r.act_dtype = c->act_dtype;
+    if (dense_q4(c)) {
+        r.s0 = w->latent_down_s;
+        r.z0 = w->latent_down_z;
+        r.group0 = c->dense_group_size;
+    }
     if (dense_tc(c, T, c->hidden) && c->latent_dim % 64 == 0) {
         TcParams P;
         TcProblem& p = P.p[0];
@@ -583,7 +704,9 @@ moe_status run_latent_down(const moe_config* c, const moe_weights* w, const void
         p.M = c->latent_dim; p.K = c->hidden; p.m_blocks = (p.M + kTcRows - 1) / kTcRows;
         p.rows = int(T); p.n_tiles = int((T + kTcBN - 1) / kTcBN);
         p.out = z; p.ld_out = c->latent_dim;
-        if (!tc_weight_map(&P.a0[0], w->latent_down_w, 1, p.M, p.K, false) || !tc_token_map(P.b[0], x, T, p.K, kTcBN))
+        if (!tc_dense_weights(c, p, &P.a0[0], nullptr, w->latent_down_w, w->latent_down_s, w->latent_down_z, nullptr,
+                              nullptr, nullptr, p.M, p.K) ||
+            !tc_token_map(P.b[0], x, T, p.K, kTcBN))
             return MOE_ERR_CUDA;
         P.nprob = 1;
         P.status = status;
@@ -625,6 +748,11 @@ moe_status run_output(const moe_config* c, const moe_weights* w, RoutedSum rs, c
     r.addend = s_acc;
     r.ld_add = c->hidden;
     r.act_dtype = c->act_dtype;
+    if (dense_q4(c)) {
+        r.s0 = w->latent_up_s;
+        r.z0 = w->latent_up_z;
+        r.group0 = c->dense_group_size;
+    }
     if (dense_tc(c, T, c->latent_dim) && c->hidden % 64 == 0) {
         TcParams P;
         TcProblem& p = P.p[0];
@@ -633,7 +761,9 @@ moe_status run_output(const moe_config* c, const moe_weights* w, RoutedSum rs, c
         p.rows = int(T); p.n_tiles = int((T + kTcBN - 1) / kTcBN);
         p.out = y; p.ld_out = c->hidden;
         p.addend = s_acc; p.ld_add = c->hidden;
-        if (!tc_weight_map(&P.a0[0], w->latent_up_w, 1, p.M, p.K, false) || !tc_token_map(P.b[0], n, T, p.K, kTcBN))
+        if (!tc_dense_weights(c, p, &P.a0[0], nullptr, w->latent_up_w, w->latent_up_s, w->latent_up_z, nullptr,
+                              nullptr, nullptr, p.M, p.K) ||
+            !tc_token_map(P.b[0], n, T, p.K, kTcBN))
             return MOE_ERR_CUDA;
         P.nprob = 1;
         P.status = at<int>(ws, L.status);
@@ -694,9 +824,12 @@ moe_status moe_permute(const moe_config* cfg, const int32_t* topk_idx, int64_t T
                        false);
 }
 
-moe_status moe_grouped_ffn(const moe_config* cfg, const moe_weights* w, const void* u, int64_t T,
-                           const int32_t* expert_offsets, const int32_t* sorted_slot, const float* topk_w,
-                           float* y_acc, void* ws, size_t ws_bytes, moe_stream_t stream) {
+}  // extern "C"
+
+namespace {
+moe_status grouped_ffn_range(const moe_config* cfg, const moe_weights* w, const void* u, int64_t T,
+                             const int32_t* expert_offsets, const int32_t* sorted_slot, const float* topk_w,
+                             ExpertRange rg, float* y_acc, void* ws, size_t ws_bytes, moe_stream_t stream) {
     MOE_CHECK(moe_config_validate(cfg));
     WsLayout L;
     MOE_CHECK(prelude(cfg, w, T, ws, ws_bytes, &L));
@@ -708,16 +841,33 @@ moe_status moe_grouped_ffn(const moe_config* cfg, const moe_weights* w, const vo
     MOE_CHECK(check_ptr(y_acc));
     cudaStream_t s = (cudaStream_t)stream;
     MOE_CUDA(cudaMemsetAsync(y_acc, 0, size_t(T) * expert_in(*cfg) * sizeof(float), s));
-    MOE_CUDA(launch_active_list(expert_offsets, cfg->num_experts, at<int32_t>(ws, L.active), s));
+    MOE_CUDA(launch_active_list(expert_offsets + rg.e0, rg.ne, at<int32_t>(ws, L.active), s));
     if (routed_tc(cfg, T))
-        MOE_CUDA(launch_tile_start(expert_offsets, cfg->num_experts, kTcBN, at<int32_t>(ws, L.tiles), s));
-    RoutedSum rs;
-    MOE_CHECK(run_experts(cfg, w, u, nullptr, T, expert_offsets, sorted_slot, topk_w, y_acc, true, false, ws, L, s,
-                          &rs));
-    if (rs.rows != y_acc)  // per-slot rows: sum each token's k rows into y_acc
-        MOE_CUDA(launch_combine(rs.rows, rs.dtype, rs.nsum, nullptr, nullptr, MOE_SHARED_NONE, T, expert_in(*cfg), y_acc,
-                                cfg->act_dtype, s, true));
-    return MOE_OK;
+        MOE_CUDA(launch_tile_start(expert_offsets + rg.e0, rg.ne, kTcBN, at<int32_t>(ws, L.tiles), s));
+    return run_experts(cfg, w, u, nullptr, T, expert_offsets, sorted_slot, topk_w, y_acc, true, false, ws, L, s,
+                       nullptr, rg);
+}
+}  // namespace
+
+extern "C" {
+
+moe_status moe_grouped_ffn(const moe_config* cfg, const moe_weights* w, const void* u, int64_t T,
+                           const int32_t* expert_offsets, const int32_t* sorted_slot, const float* topk_w,
+                           float* y_acc, void* ws, size_t ws_bytes, moe_stream_t stream) {
+    if (!cfg) return MOE_ERR_INVALID_ARGUMENT;
+    return grouped_ffn_range(cfg, w, u, T, expert_offsets, sorted_slot, topk_w, ExpertRange{0, cfg->num_experts},
+                             y_acc, ws, ws_bytes, stream);
+}
+
+moe_status moe_grouped_ffn_experts(const moe_config* cfg, const moe_weights* w, const void* u, int64_t T,
+                                   const int32_t* expert_offsets, const int32_t* sorted_slot, const float* topk_w,
+                                   int32_t expert_begin, int32_t expert_end, float* y_acc, void* ws,
+                                   size_t ws_bytes, moe_stream_t stream) {
+    MOE_CHECK(moe_config_validate(cfg));
+    if (expert_begin < 0 || expert_end <= expert_begin || expert_end > cfg->num_experts)
+        return MOE_ERR_INVALID_ARGUMENT;
+    return grouped_ffn_range(cfg, w, u, T, expert_offsets, sorted_slot, topk_w,
+                             ExpertRange{expert_begin, expert_end - expert_begin}, y_acc, ws, ws_bytes, stream);
 }
 
 moe_status moe_latent_down(const moe_config* cfg, const moe_weights* w, const void* x, int64_t T, void* z,
@@ -760,6 +910,13 @@ moe_status moe_block_forward(const moe_config* cfg, const moe_weights* w, const 
     MOE_CHECK(check_ptr(x));
     MOE_CHECK(check_ptr(y));
     cudaStream_t s = (cudaStream_t)stream;
+    {
+        const DecodeArgs d = decode_args(cfg, w, x, T, y, ws, L);
+        if (use_decode(cfg, T, d)) {
+            MOE_CUDA(launch_decode(d, s));
+            return MOE_OK;
+        }
+    }
     const int K = expert_in(*cfg);
     float* y_acc = at<float>(ws, L.y_acc);
     int32_t* idx = at<int32_t>(ws, L.topk_idx);
@@ -769,15 +926,15 @@ moe_status moe_block_forward(const moe_config* cfg, const moe_weights* w, const 
     const void* u = cfg->latent_dim ? at<void>(ws, L.z) : x;
     int32_t* offsets = at<int32_t>(ws, L.offsets);
     int32_t* sorted_slot = at<int32_t>(ws, L.sorted_slot);
-    // the weight-streaming path scatter-adds into y_acc: its rows are cleared by the router;
-    // a single token's permutation comes from the top-k warp itself
+    // both engines add every slot's weighted output into y_acc: its rows are cleared by the
+    // router; a single token's permutation comes from the top-k warp itself
     PermOut perm;
     perm.offsets = offsets;
     perm.sorted_slot = sorted_slot;
     perm.slot_pos = at<int32_t>(ws, L.slot_pos);
     perm.active = at<int32_t>(ws, L.active);
     perm.tiles = rtc ? at<int32_t>(ws, L.tiles) : nullptr;
-    MOE_CHECK(run_route(cfg, w, x, T, idx, wts, coef, rtc ? nullptr : y_acc, K, ws, L, s, &perm));
+    MOE_CHECK(run_route(cfg, w, x, T, idx, wts, coef, y_acc, K, ws, L, s, &perm));
     if (cfg->latent_dim) MOE_CHECK(run_latent_down(cfg, w, x, T, at<void>(ws, L.z), at<int>(ws, L.status), s));
     if (T > 1) MOE_CHECK(run_permute(cfg, idx, T, offsets, sorted_slot, at<int32_t>(ws, L.slot_pos), ws, L, s, rtc));
     RoutedSum rs;

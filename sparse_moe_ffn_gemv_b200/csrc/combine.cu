@@ -35,6 +35,13 @@ __device__ __forceinline__ float4 routed_sum(const RT* __restrict__ rows, int ns
     return r;
 }
 
+// Four consecutive outputs in one vector store: 16 bytes of fp32 or 8 bytes of bf16.
+__device__ __forceinline__ void store4(float* o, float4 r) { *reinterpret_cast<float4*>(o) = r; }
+__device__ __forceinline__ void store4(__nv_bfloat16* o, float4 r) {
+    const __nv_bfloat162 a = __floats2bfloat162_rn(r.x, r.y), b = __floats2bfloat162_rn(r.z, r.w);
+    *reinterpret_cast<uint2*>(o) = make_uint2(*reinterpret_cast<const uint32_t*>(&a), *reinterpret_cast<const uint32_t*>(&b));
+}
+
 template <typename AT, typename RT>
 __global__ void __launch_bounds__(256) combine_kernel(const RT* __restrict__ rows, int nsum,
                                                       const float* __restrict__ s_acc,
@@ -59,11 +66,7 @@ __global__ void __launch_bounds__(256) combine_kernel(const RT* __restrict__ row
                 r.w = r.w * c0 + sv.w * c1;
             }
         }
-        AT* o = y + i * 4;
-        o[0] = from_f<AT>(r.x);
-        o[1] = from_f<AT>(r.y);
-        o[2] = from_f<AT>(r.z);
-        o[3] = from_f<AT>(r.w);
+        store4(y + i * 4, r);
     }
 }
 

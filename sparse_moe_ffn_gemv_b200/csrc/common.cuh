@@ -43,13 +43,18 @@ struct WsLayout {
     size_t z;            // act [T, L]: latent input of the experts
     size_t nrm;          // act [T, L]: normalised latent
     size_t uperm;        // bf16 [T * k, K]: expert inputs gathered in sorted order
-    size_t oslot;        // bf16 [T * k, K]: weighted expert output of every slot
     size_t tiles;        // int32 tile list of the tensor-core path
     size_t total;
     int ld_logits;
     int n_chunks;
     int64_t T;
 };
+
+// Byte offset, within the workspace's 256-byte status region, of the decode kernel's three
+// grid-barrier counters (every launch leaves them at zero).
+constexpr size_t kDecodeBarOffset = 16;
+// ... and of the counter the grid-barrier self test waits on.
+constexpr size_t kSelftestBarOffset = 32;
 
 constexpr int kPermChunk = 2048;   // slots per permutation chunk (fixed-scratch permutation)
 constexpr int kPermChunkWs = 2048;  // slots per chunk when the workspace holds the histograms (512 measured slower)

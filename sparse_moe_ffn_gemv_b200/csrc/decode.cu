@@ -1,0 +1,473 @@
+// decode.cu -- the whole block for a decode-sized batch (T <= 8 tokens) in one launch.
+//
+// At a few tokens the block is bound by reading the activated weights once from HBM, and
+// a chain of short kernels (router, top-k, gate/up, down, combine) loses most of its time to
+// the start and tail of each launch. Here one cooperative launch of one 512-thread block
+// per SM runs three phases separated by grid barriers:
+//   A  the router and coefficient-head rows (fp32 logits) and the shared expert's gate/up
+//      units (Klear PR item 2: the shared expert reads the block input x; neither depends
+//      on the routing, so they start at once);
+//   B  every block takes the top-k of the T tokens itself (Klear PR item 3: sigmoid of fp32
+//      logits, select-only bias, unbiased weights, norm_topk_prob; libmir-metal
+//      router_top_k_unit for softmax over the top-k logits), sorts the T*k slots by expert,
+//      and the grid streams the routed gate/up units of the distinct experts (one weight
+//      row pair per warp item, dotted with the tokens routed to that expert);
+//   C  each block owns a contiguous range of output rows: it stages every slot's
+//      intermediate vector, streams the down rows of its range for every distinct expert
+//      and for the shared expert, and writes y = y_r | y_r + s | c0 y_r + c1 s for its
+//      rows (libmir-metal execute: down weighted by routing.weights and summed; ferrox
+//      KimiExpertWeights::forward: down(act(gate, up))).
+// While phase B streams the gate/up rows, each block asks L2 to prefetch its phase-C down
+// rows when they fit in L2, so phase C reads them from L2.
+// Every grid-barrier wait is bounded by %globaltimer: a wait that gives up records
+// MOE_ERR_DEVICE_TIMEOUT in the status word, and the block skips the remaining phases.
+// The last block to finish resets the barrier counters, so the next launch starts from 0.
+#include <algorithm>
+
+#include "gemv_dev.cuh"
+#include "ptx.cuh"
+#include "topk_dev.cuh"
+
+namespace moe {
+
+namespace {
+
+constexpr int kDecThreads = 512;
+constexpr int kDecWarps = kDecThreads / kWarp;
+constexpr int kDecMaxSlots = kTT * kMaxTopK;  // T * k slots at most
+constexpr int kDecRowsMax = 64;               // output rows a block owns at most
+constexpr uint64_t kDecWaitNs = 2000000000ull;  // 2 s bound on a grid-barrier wait
+constexpr size_t kDecSmemMax = 200 * 1024;
+
+struct DecSmem {
+    int32_t sidx[kDecMaxSlots];  // expert of slot s = t * k + j
+    float sw[kDecMaxSlots];      // combine weight of slot s
+    float scoef[kTT * 2];        // blend coefficients of each token
+    int sorted[kDecMaxSlots];    // slots sorted by expert, ascending slot within an expert
+    int head[kDecMaxSlots];      // 1: first slot of its expert
+    int lt[kDecMaxSlots];        // slots whose expert is smaller than slot s's
+    int dexp[kDecMaxSlots];      // distinct experts, ascending
+    int doff[kDecMaxSlots + 1];  // their ranges in `sorted`
+    int n_d;                     // number of distinct experts
+    int flag;
+    float acc_r[kDecRowsMax][kTT];  // routed sum of the block's rows
+    float acc_s[kDecRowsMax][kTT];  // shared expert output of the block's rows
+};
+
+__device__ __forceinline__ void l2_prefetch(const void* p, size_t bytes) {
+    // a hint: the start is rounded up and the size down to 16 bytes, so nothing outside
+    // [p, p + bytes) is named
+    uintptr_t a = (reinterpret_cast<uintptr_t>(p) + 15) & ~uintptr_t(15);
+    const uintptr_t end = (reinterpret_cast<uintptr_t>(p) + bytes) & ~uintptr_t(15);
+    while (a < end) {
+        const uint32_t n = uint32_t(end - a < (uintptr_t(1) << 20) ? end - a : (uintptr_t(1) << 20));
+        asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(a), "r"(n) : "memory");
+        a += n;
+    }
+}
+
+__device__ __forceinline__ float bf16_ld(const void* p, int64_t i) {
+    return __bfloat162float(reinterpret_cast<const __nv_bfloat16*>(p)[i]);
+}
+
+// Copy n16 16-byte vectors from global (through L2: another block wrote them) to shared.
+__device__ __forceinline__ void copy_cg(uint4* dst, const void* src, int64_t n16) {
+    const uint4* s = reinterpret_cast<const uint4*>(src);
+    for (int64_t i = threadIdx.x; i < n16; i += blockDim.x) dst[i] = __ldcg(s + i);
+}
+
+template <int WF>
+__global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(const DecodeArgs a) {
+    using AT = __nv_bfloat16;
+    constexpr int DN = 2;  // down rows per warp item (one expert)
+    extern __shared__ uint4 dsm[];
+    __shared__ DecSmem sm;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int T = a.T, H = a.H, k = a.k, I = a.I, Is = a.Is, S = T * k;
+    const int gw = blockIdx.x * kDecWarps + warp, nw = gridDim.x * kDecWarps;
+    const uint64_t deadline = gtimer() + kDecWaitNs;
+    const int RB = (H + gridDim.x - 1) / gridDim.x;  // output rows per block
+    const int r0 = min(H, int(blockIdx.x) * RB), r1 = min(H, r0 + RB), nr = r1 - r0;
+    const bool blend = a.shared_mode == MOE_SHARED_BLEND;
+    const int64_t drb = row_bytes<WF>(I);  // bytes of one routed down row
+
+    // ------------------------------------------------------------ phase A
+    AT* xs = reinterpret_cast<AT*>(dsm);
+    float* xsum = reinterpret_cast<float*>(xs + int64_t(T) * H);  // 4-bit affine: sums per 32
+    if (WF == kQ4 || a.dense_q4) stage_tokens<kQ4>(a.x, H, 0, T, nullptr, 1, xs, xsum);
+    else stage_tokens<kBF16>(a.x, H, 0, T, nullptr, 1, xs, nullptr);
+    const int dg = a.dense_group;
+    const int64_t srb = a.dense_q4 ? Is / 2 : int64_t(Is) * 2;  // bytes of one shared down row
+    if (a.l2_prefetch && Is && threadIdx.x == 0 && nr > 0)
+        l2_prefetch(static_cast<const char*>(a.sd_w) + int64_t(r0) * srb, size_t(nr) * srb);
+    __syncthreads();
+    const int nrouter = a.E + (blend ? 2 : 0);
+    for (int it = gw; it < nrouter + Is; it += nw) {
+        if (it < nrouter) {  // one router / coefficient row -> fp32 logits of every token
+            const bool cr = it >= a.E;
+            const int rr = cr ? it - a.E : it;
+            float acc[1][kTT];
+#pragma unroll
+            for (int t = 0; t < kTT; ++t) acc[0][t] = 0.f;
+            if (a.dense_q4 && !cr) {  // 4-bit router row (the blend head stays bf16)
+                const int64_t ng = H / dg;
+                const char* rows[1] = {static_cast<const char*>(a.router_w) + int64_t(rr) * (H / 2)};
+                const QRow q[1] = {{static_cast<const __nv_bfloat16*>(a.router_s) + rr * ng,
+                                    static_cast<const __nv_bfloat16*>(a.router_z) + rr * ng, nullptr}};
+                dot_rows<kQ4, 1>(rows, q, H, dg, xs, xsum, T, acc);
+            } else {
+                const char* rows[1] = {static_cast<const char*>(cr ? a.coef_w : a.router_w) + int64_t(rr) * H * 2};
+                const QRow q[1] = {{nullptr, nullptr, nullptr}};
+                dot_rows<kBF16, 1>(rows, q, H, 64, xs, nullptr, T, acc);
+            }
+            const void* bp = cr ? a.coef_b : a.router_b;
+            const float b = bp ? bf16_ld(bp, rr) : 0.f;
+#pragma unroll
+            for (int t = 0; t < kTT; ++t) {
+                if (t >= T) break;
+                const float v = warp_sum(acc[0][t]);
+                if (lane == t) a.logits[int64_t(t) * a.ld_logits + it] = v + b;
+            }
+        } else {  // one shared gate/up unit
+            const int i = it - nrouter;
+            float acc[2][kTT];
+#pragma unroll
+            for (int r = 0; r < 2; ++r)
+#pragma unroll
+                for (int t = 0; t < kTT; ++t) acc[r][t] = 0.f;
+            if (a.dense_q4) {
+                const int64_t ng = H / dg;
+                const char* rows[2] = {static_cast<const char*>(a.sg_w) + int64_t(i) * (H / 2),
+                                       static_cast<const char*>(a.su_w) + int64_t(i) * (H / 2)};
+                const QRow q[2] = {{static_cast<const __nv_bfloat16*>(a.sg_s) + i * ng,
+                                    static_cast<const __nv_bfloat16*>(a.sg_z) + i * ng, nullptr},
+                                   {static_cast<const __nv_bfloat16*>(a.su_s) + i * ng,
+                                    static_cast<const __nv_bfloat16*>(a.su_z) + i * ng, nullptr}};
+                dot_rows<kQ4, 2>(rows, q, H, dg, xs, xsum, T, acc);
+            } else {
+                const char* rows[2] = {static_cast<const char*>(a.sg_w) + int64_t(i) * H * 2,
+                                       static_cast<const char*>(a.su_w) + int64_t(i) * H * 2};
+                const QRow q[2] = {{nullptr, nullptr, nullptr}, {nullptr, nullptr, nullptr}};
+                dot_rows<kBF16, 2>(rows, q, H, 64, xs, nullptr, T, acc);
+            }
+#pragma unroll
+            for (int t = 0; t < kTT; ++t) {
+                if (t >= T) break;
+                const float g = warp_sum(acc[0][t]), u = warp_sum(acc[1][t]);
+                if (lane == t)
+                    reinterpret_cast<AT*>(a.hs)[int64_t(t) * Is + i] =
+                        __float2bfloat16_rn(act_apply(a.act, g, u, a.limit, a.alpha));
+            }
+        }
+    }
+    bool ok = grid_barrier(&a.bar[0], gridDim.x, deadline, a.status, &sm.flag);
+
+    // ------------------------------------------------------------ phase B
+    if (ok) {
+        if (warp < T) {  // top-k of token `warp`, identical in every block
+            TopkArgs ta;
+            ta.logits = a.logits; ta.ld = a.ld_logits; ta.T = T; ta.E = a.E; ta.k = k;
+            ta.scoring = a.scoring; ta.norm = a.norm; ta.has_sel = a.has_sel; ta.sel_bias = a.sel_bias;
+            ta.blend = blend ? 1 : 0;
+            ta.idx = sm.sidx; ta.w = sm.sw; ta.coef = sm.scoef;
+            topk_token(ta, warp);
+        }
+        __syncthreads();
+        // stable counting sort of the S slots by expert (a token's k experts are distinct,
+        // so an expert holds at most T slots)
+        const int s = threadIdx.x;
+        int e = 0, lt = 0, eqb = 0;
+        if (s < S) {
+            e = sm.sidx[s];
+            for (int u = 0; u < S; ++u) {
+                const int f = sm.sidx[u];
+                lt += f < e ? 1 : 0;
+                eqb += (f == e && u < s) ? 1 : 0;
+            }
+            sm.sorted[lt + eqb] = s;
+            sm.head[s] = eqb == 0 ? 1 : 0;
+            sm.lt[s] = lt;
+        }
+        const int n_d = __syncthreads_count(s < S && eqb == 0);
+        if (s < S && eqb == 0) {
+            int d = 0;
+            for (int u = 0; u < S; ++u) d += (sm.head[u] && sm.sidx[u] < e) ? 1 : 0;
+            sm.dexp[d] = e;
+            sm.doff[d] = lt;
+        }
+        if (threadIdx.x == 0) {
+            sm.doff[n_d] = S;
+            sm.n_d = n_d;
+        }
+        __syncthreads();
+        // this block's phase-C down rows of every distinct expert, into L2
+        if (a.l2_prefetch && nr > 0)
+            for (int d = threadIdx.x; d < n_d; d += blockDim.x)
+                l2_prefetch(static_cast<const char*>(a.down_w) + (int64_t(sm.dexp[d]) * H + r0) * drb,
+                            size_t(nr) * drb);
+        // routed gate/up: one unit (gate row + up row) of one distinct expert per warp item
+        for (int it = gw; it < n_d * I; it += nw) {
+            const int d = it / I, i = it - d * I;
+            const int ex = sm.dexp[d];
+            const int sb = sm.doff[d], cnt = sm.doff[d + 1] - sb;
+            int tl[kTT];
+#pragma unroll
+            for (int j = 0; j < kTT; ++j) tl[j] = j < cnt ? sm.sorted[sb + j] / k : 0;
+            const int64_t rb = row_bytes<WF>(H);
+            const char* rows[2];
+            QRow q[2] = {{nullptr, nullptr, nullptr}, {nullptr, nullptr, nullptr}};
+            int64_t g0, g1;  // plane rows of the gate and the up weights
+            if (a.interleaved) {
+                g0 = int64_t(ex) * 2 * I + 2 * i;
+                g1 = g0 + 1;
+                rows[0] = static_cast<const char*>(a.gate_up_w) + g0 * rb;
+                rows[1] = rows[0] + rb;
+            } else {
+                g0 = g1 = int64_t(ex) * I + i;
+                rows[0] = static_cast<const char*>(a.gate_w) + g0 * rb;
+                rows[1] = static_cast<const char*>(a.up_w) + g1 * rb;
+            }
+            if constexpr (WF == kQ4) {
+                const int64_t ng = H / a.group_size;
+                const __nv_bfloat16* s0 = static_cast<const __nv_bfloat16*>(a.gate_s);
+                const __nv_bfloat16* z0 = static_cast<const __nv_bfloat16*>(a.gate_z);
+                const __nv_bfloat16* s1 = static_cast<const __nv_bfloat16*>(a.interleaved ? a.gate_s : a.up_s);
+                const __nv_bfloat16* z1 = static_cast<const __nv_bfloat16*>(a.interleaved ? a.gate_z : a.up_z);
+                q[0] = {s0 + g0 * ng, z0 + g0 * ng, nullptr};
+                q[1] = {s1 + g1 * ng, z1 + g1 * ng, nullptr};
+            } else if constexpr (WF == kMX4) {
+                const uint8_t* s0 = static_cast<const uint8_t*>(a.gate_s);
+                const uint8_t* s1 = static_cast<const uint8_t*>(a.interleaved ? a.gate_s : a.up_s);
+                q[0] = {nullptr, nullptr, s0 + g0 * (H / 32)};
+                q[1] = {nullptr, nullptr, s1 + g1 * (H / 32)};
+            }
+            float bg = 0.f, bu = 0.f;
+            if (a.has_bias) {
+                if (a.interleaved) {
+                    bg = bf16_ld(a.gate_up_b, int64_t(ex) * 2 * I + 2 * i);
+                    bu = bf16_ld(a.gate_up_b, int64_t(ex) * 2 * I + 2 * i + 1);
+                } else {
+                    bg = bf16_ld(a.gate_b, int64_t(ex) * I + i);
+                    bu = bf16_ld(a.up_b, int64_t(ex) * I + i);
+                }
+            }
+            float acc[2][kTT];
+#pragma unroll
+            for (int r = 0; r < 2; ++r)
+#pragma unroll
+                for (int t = 0; t < kTT; ++t) acc[r][t] = 0.f;
+            dot_rows<WF, 2>(rows, q, H, a.group_size, xs, xsum, cnt, acc, tl);
+#pragma unroll
+            for (int j = 0; j < kTT; ++j) {
+                if (j >= cnt) break;
+                const float g = warp_sum(acc[0][j]), u = warp_sum(acc[1][j]);
+                if (lane == j)
+                    reinterpret_cast<AT*>(a.h)[int64_t(sm.sorted[sb + j]) * I + i] =
+                        __float2bfloat16_rn(act_apply(a.act, g + bg, u + bu, a.limit, a.alpha));
+            }
+        }
+        ok = grid_barrier(&a.bar[1], gridDim.x, deadline, a.status, &sm.flag);
+    }
+
+    // ------------------------------------------------------------ phase C
+    if (ok) {
+        const int n_d = sm.n_d;
+        AT* hsm = reinterpret_cast<AT*>(dsm);                          // [S, I] by slot
+        float* hsum = reinterpret_cast<float*>(hsm + int64_t(S) * I);  // 4-bit affine: sums per 32
+        AT* hss = reinterpret_cast<AT*>(hsum + (WF == kQ4 ? int64_t(S) * (I / 32) : 0));  // [T, Is]
+        float* hssum = reinterpret_cast<float*>(hss + int64_t(T) * Is);  // 4-bit shared down: sums per 32
+        copy_cg(reinterpret_cast<uint4*>(hsm), a.h, int64_t(S) * I / 8);
+        if (Is) copy_cg(reinterpret_cast<uint4*>(hss), a.hs, int64_t(T) * Is / 8);
+        for (int i = threadIdx.x; i < nr * kTT; i += blockDim.x) {
+            sm.acc_r[i / kTT][i % kTT] = 0.f;
+            sm.acc_s[i / kTT][i % kTT] = 0.f;
+        }
+        __syncthreads();
+        if (a.dense_q4 && Is) {
+            const int nv = Is / 32;
+            for (int i = threadIdx.x; i < T * nv; i += blockDim.x) {
+                const uint4* p = reinterpret_cast<const uint4*>(hss + int64_t(i / nv) * Is + (i % nv) * 32);
+                float sum = 0.f;
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    float f[8];
+                    unpack8(p[j], f);
+#pragma unroll
+                    for (int n = 0; n < 8; ++n) sum += f[n];
+                }
+                hssum[i] = sum;
+            }
+            if (WF != kQ4) __syncthreads();
+        }
+        if constexpr (WF == kQ4) {
+            const int nv = I / 32;
+            for (int i = threadIdx.x; i < S * nv; i += blockDim.x) {
+                const uint4* p = reinterpret_cast<const uint4*>(hsm + int64_t(i / nv) * I + (i % nv) * 32);
+                float sum = 0.f;
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    float f[8];
+                    unpack8(p[j], f);
+#pragma unroll
+                    for (int n = 0; n < 8; ++n) sum += f[n];
+                }
+                hsum[i] = sum;
+            }
+            __syncthreads();
+        }
+        const int nq = (nr + DN - 1) / DN;
+        const int n_items = n_d * nq + (Is ? nq : 0);
+        for (int it = warp; it < n_items; it += kDecWarps) {
+            if (it < n_d * nq) {  // DN down rows of one distinct expert
+                const int d = it / nq, qq = it - d * nq;
+                const int ex = sm.dexp[d];
+                const int sb = sm.doff[d], cnt = sm.doff[d + 1] - sb;
+                int tl[kTT];
+#pragma unroll
+                for (int j = 0; j < kTT; ++j) tl[j] = j < cnt ? sm.sorted[sb + j] : 0;  // slot rows of hsm
+                const char* rows[DN];
+                QRow q[DN];
+                float bd[DN];
+#pragma unroll
+                for (int jr = 0; jr < DN; ++jr) {
+                    const int r = min(r0 + qq * DN + jr, r1 - 1);
+                    const int64_t gr = int64_t(ex) * H + r;
+                    rows[jr] = static_cast<const char*>(a.down_w) + gr * drb;
+                    q[jr] = {nullptr, nullptr, nullptr};
+                    if constexpr (WF == kQ4) {
+                        const int64_t ng = I / a.group_size;
+                        q[jr] = {static_cast<const __nv_bfloat16*>(a.down_s) + gr * ng,
+                                 static_cast<const __nv_bfloat16*>(a.down_z) + gr * ng, nullptr};
+                    } else if constexpr (WF == kMX4) {
+                        q[jr] = {nullptr, nullptr, static_cast<const uint8_t*>(a.down_s) + gr * (I / 32)};
+                    }
+                    bd[jr] = a.has_bias ? bf16_ld(a.down_b, gr) : 0.f;
+                }
+                float acc[DN][kTT];
+#pragma unroll
+                for (int jr = 0; jr < DN; ++jr)
+#pragma unroll
+                    for (int t = 0; t < kTT; ++t) acc[jr][t] = 0.f;
+                dot_rows<WF, DN>(rows, q, I, a.group_size, hsm, hsum, cnt, acc, tl);
+#pragma unroll
+                for (int jr = 0; jr < DN; ++jr)
+#pragma unroll
+                    for (int j = 0; j < kTT; ++j) {
+                        if (j >= cnt) break;
+                        const float v = warp_sum(acc[jr][j]);
+                        const int rl = qq * DN + jr;
+                        if (lane == 0 && rl < nr) {
+                            const int slot = tl[j];
+                            atomicAdd(&sm.acc_r[rl][slot / k], sm.sw[slot] * (v + bd[jr]));
+                        }
+                    }
+            } else {  // DN rows of the shared expert's down projection, every token
+                const int qq = it - n_d * nq;
+                const char* rows[DN];
+                QRow q[DN];
+#pragma unroll
+                for (int jr = 0; jr < DN; ++jr) {
+                    const int64_t r = min(r0 + qq * DN + jr, r1 - 1);
+                    rows[jr] = static_cast<const char*>(a.sd_w) + r * srb;
+                    q[jr] = {nullptr, nullptr, nullptr};
+                    if (a.dense_q4)
+                        q[jr] = {static_cast<const __nv_bfloat16*>(a.sd_s) + r * (Is / dg),
+                                 static_cast<const __nv_bfloat16*>(a.sd_z) + r * (Is / dg), nullptr};
+                }
+                float acc[DN][kTT];
+#pragma unroll
+                for (int jr = 0; jr < DN; ++jr)
+#pragma unroll
+                    for (int t = 0; t < kTT; ++t) acc[jr][t] = 0.f;
+                if (a.dense_q4) dot_rows<kQ4, DN>(rows, q, Is, dg, hss, hssum, T, acc);
+                else dot_rows<kBF16, DN>(rows, q, Is, 64, hss, nullptr, T, acc);
+#pragma unroll
+                for (int jr = 0; jr < DN; ++jr)
+#pragma unroll
+                    for (int t = 0; t < kTT; ++t) {
+                        if (t >= T) break;
+                        const float v = warp_sum(acc[jr][t]);
+                        const int rl = qq * DN + jr;
+                        if (lane == 0 && rl < nr) sm.acc_s[rl][t] = v;
+                    }
+            }
+        }
+        __syncthreads();
+        // y = y_r | y_r + s | c0 y_r + c1 s for the block's rows (Klear PR item 2)
+        for (int i = threadIdx.x; i < T * nr; i += blockDim.x) {
+            const int t = i / nr, rl = i - t * nr;
+            const float yr = sm.acc_r[rl][t], sv = sm.acc_s[rl][t];
+            float v = yr;
+            if (a.shared_mode == MOE_SHARED_ADD) v = yr + sv;
+            else if (blend) v = yr * sm.scoef[2 * t] + sv * sm.scoef[2 * t + 1];
+            reinterpret_cast<AT*>(a.y)[int64_t(t) * H + r0 + rl] = __float2bfloat16_rn(v);
+        }
+    }
+
+    // the last block out resets the barrier counters for the next launch
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        __threadfence();
+        if (atomicAdd(&a.bar[2], 1u) == gridDim.x - 1) {
+            a.bar[0] = 0;
+            a.bar[1] = 0;
+            __threadfence();
+            a.bar[2] = 0;
+        }
+    }
+}
+
+template <int WF>
+cudaError_t launch_decode_t(const DecodeArgs& a, size_t smem, cudaStream_t s) {
+    auto kern = decode_kernel<WF>;
+    cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
+    if (err != cudaSuccess) return err;
+    int dev = 0, sms = 0, per_sm = 0;
+    if ((err = cudaGetDevice(&dev)) != cudaSuccess) return err;
+    if ((err = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return err;
+    if ((err = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kDecThreads, smem)) != cudaSuccess)
+        return err;
+    if (per_sm < 1) return cudaErrorInvalidConfiguration;
+    const int grid = sms * std::min(per_sm, 1);  // one block per SM: every block is resident
+    if ((a.H + grid - 1) / grid > kDecRowsMax) return cudaErrorInvalidConfiguration;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(grid);
+    cfg.blockDim = dim3(kDecThreads);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeCooperative;  // co-residency of all blocks (grid barriers)
+    attr[0].val.cooperative = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    err = cudaLaunchKernelEx(&cfg, kern, a);
+    if (err != cudaSuccess) return err;
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+size_t decode_smem_bytes(const DecodeArgs& a) {
+    if (a.T < 1 || a.T > kTT || a.k > kMaxTopK || a.E > kMaxExperts) return 0;
+    if (a.wf != kBF16 && a.wf != kQ4 && a.wf != kMX4) return 0;
+    const size_t S = size_t(a.T) * a.k;
+    const bool q4 = a.wf == kQ4;
+    const size_t pa = size_t(a.T) * a.H * 2 + ((q4 || a.dense_q4) ? size_t(a.T) * (a.H / 32) * 4 : 0);
+    const size_t pc = S * a.I * 2 + (q4 ? S * (a.I / 32) * 4 : 0) + size_t(a.T) * a.Is * 2 +
+                      (a.dense_q4 ? size_t(a.T) * (a.Is / 32) * 4 : 0);
+    const size_t need = (std::max(pa, pc) + 15) & ~size_t(15);
+    return need <= kDecSmemMax ? need : 0;
+}
+
+cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t s) {
+    const size_t smem = decode_smem_bytes(a);
+    if (smem == 0) return cudaErrorInvalidValue;
+    switch (a.wf) {
+        case kBF16: return launch_decode_t<kBF16>(a, smem, s);
+        case kQ4: return launch_decode_t<kQ4>(a, smem, s);
+        case kMX4: return launch_decode_t<kMX4>(a, smem, s);
+        default: return cudaErrorInvalidValue;
+    }
+}
+
+}  // namespace moe

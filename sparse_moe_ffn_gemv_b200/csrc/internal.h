@@ -19,6 +19,8 @@ struct DenseGemvArgs {
     void* out = nullptr; int ld_out = 0; int out_f32 = 0;
     const float* addend = nullptr; int ld_add = 0;
     int act_dtype = MOE_DTYPE_BF16;
+    // W0 4-bit affine when s0 is set: words [rows0, K / 8], bf16 scales / biases [rows0, K / group0]
+    const void *s0 = nullptr, *z0 = nullptr; int group0 = 64;
 };
 cudaError_t launch_dense_gemv(const DenseGemvArgs& a, cudaStream_t s);
 
@@ -49,9 +51,9 @@ cudaError_t launch_permute(const PermuteArgs& a, cudaStream_t s);
 cudaError_t launch_active_list(const int32_t* offsets, int E, int32_t* active, cudaStream_t s);
 
 // dst[p, :] = src[sorted_slot[p] / k, :] for p < S (rows of K bf16): expert inputs in
-// sorted order for the tensor-core path.
+// sorted order for the tensor-core path; with lo / hi (device pointers) only *lo <= p < *hi.
 cudaError_t launch_gather_rows(const void* src, int K, const int32_t* sorted_slot, int k, int64_t S,
-                               void* dst, cudaStream_t s);
+                               void* dst, cudaStream_t s, const int32_t* lo = nullptr, const int32_t* hi = nullptr);
 // tile_start from offsets (moe_grouped_ffn called with a caller-made permutation).
 cudaError_t launch_tile_start(const int32_t* offsets, int E, int tile_bn, int32_t* tile_start, cudaStream_t s);
 
@@ -69,6 +71,8 @@ struct GateUpArgs {
     // shared expert (dense group over all T tokens), shared_I == 0 disables it
     const void *sg_w = nullptr, *su_w = nullptr; int shared_I = 0, Hs = 0;
     const void* xs = nullptr; void* hs = nullptr;
+    // 4-bit shared planes when sg_s is set (bf16 scales / biases per s_group columns)
+    const void *sg_s = nullptr, *sg_z = nullptr, *su_s = nullptr, *su_z = nullptr; int s_group = 64;
     int64_t T = 0;
     int act = 0; float limit = 7.f, alpha = 1.702f;
 };
@@ -84,6 +88,7 @@ struct DownArgs {
     const void* h = nullptr; float* y_acc = nullptr;
     const void* sd_w = nullptr; int shared_I = 0, Hs = 0; const void* hs = nullptr;
     float* s_acc = nullptr;
+    const void *sd_s = nullptr, *sd_z = nullptr; int s_group = 64;  // 4-bit shared down plane
     int64_t T = 0;
 };
 cudaError_t launch_down_gemv(const DownArgs& a, cudaStream_t s);
@@ -98,11 +103,44 @@ cudaError_t launch_combine(const void* rows, int rows_dtype, int nsum, const flo
 cudaError_t launch_rmsnorm(const void* rows, int rows_dtype, int nsum, const void* gamma, float eps, int64_t T,
                            int L, void* out, int act_dtype, cudaStream_t s);
 
+// ------------------------------------------------------------------ persistent decode kernel
+// The whole block for a decode-sized batch (T <= 8, no latent projection) in one cooperative
+// launch: router + coefficient rows and the shared expert's gate/up, a grid barrier, top-k
+// and the routed gate/up, a grid barrier, then the routed and shared down rows with the
+// weighted combine and the blend, each block owning a contiguous range of output rows.
+struct DecodeArgs {
+    int T = 0, H = 0, E = 0, k = 0, I = 0, Is = 0;
+    int wf = MOE_DTYPE_BF16, interleaved = 0, has_bias = 0, group_size = 64;
+    int act = 0; float limit = 7.f, alpha = 1.702f;
+    int scoring = 0, norm = 0, has_sel = 0, shared_mode = 0;
+    const void *router_w = nullptr, *router_b = nullptr, *coef_w = nullptr, *coef_b = nullptr;
+    const float* sel_bias = nullptr;
+    const void *gate_w = nullptr, *up_w = nullptr, *gate_up_w = nullptr;
+    const void *gate_s = nullptr, *gate_z = nullptr, *up_s = nullptr, *up_z = nullptr;
+    const void *gate_b = nullptr, *up_b = nullptr, *gate_up_b = nullptr;
+    const void *down_w = nullptr, *down_s = nullptr, *down_z = nullptr, *down_b = nullptr;
+    const void *sg_w = nullptr, *su_w = nullptr, *sd_w = nullptr;
+    // 4-bit router and shared planes (dense_q4): bf16 scales / biases per dense_group columns
+    int dense_q4 = 0, dense_group = 64;
+    const void *router_s = nullptr, *router_z = nullptr;
+    const void *sg_s = nullptr, *sg_z = nullptr, *su_s = nullptr, *su_z = nullptr, *sd_s = nullptr, *sd_z = nullptr;
+    const void* x = nullptr; void* y = nullptr;
+    float* logits = nullptr; int ld_logits = 0;   // workspace: fp32 router + coefficient logits
+    void* h = nullptr;                            // workspace: bf16 [T * k, I] by slot
+    void* hs = nullptr;                           // workspace: bf16 [T, Is]
+    unsigned* bar = nullptr;                      // workspace: three zeroed counters
+    int* status = nullptr;
+    int l2_prefetch = 0;                          // prefetch each block's down rows into L2
+};
+// Dynamic shared memory the decode kernel needs for a config and T (0 if it cannot run it).
+size_t decode_smem_bytes(const DecodeArgs& a);
+cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t s);
+
 // ------------------------------------------------------------------ tensor-core GEMM
 constexpr int kTcBN = 128;       // token columns per tile
 constexpr int kTcRowsGateUp = 128;  // intermediate units per gate/up tile (gate + up rows)
 constexpr int kTcRows = 256;        // output rows per tile of the other GEMMs
-enum { kEpiGateUp = 0, kEpiSlotRows = 1, kEpiStoreF32 = 2, kEpiStoreAct = 3 };
+enum { kEpiGateUp = 0, kEpiScatterAdd = 1, kEpiStoreF32 = 2, kEpiStoreAct = 3 };
 
 // One GEMM problem of a tensor-core launch: D[M rows, tokens] = W[M, K] . U[tokens, K]^T.
 struct TcProblem {
@@ -113,8 +151,8 @@ struct TcProblem {
     int num_groups = 0;
     const int32_t* offsets = nullptr;      // [E + 1] sorted-row offsets of the groups
     const int32_t* tile_start = nullptr;   // [E + 1] prefix of token tiles per group
-    const int32_t* sorted_slot = nullptr;  // slot rows: sorted row -> slot
-    const float* topk_w = nullptr;         // slot rows: slot -> combine weight
+    const int32_t* sorted_slot = nullptr;  // scatter-add: sorted row -> slot (token = slot / k)
+    const float* topk_w = nullptr;         // scatter-add: slot -> combine weight
     int k = 1;
     const void* bias0 = nullptr;           // bf16 [groups, M] (or [groups, 2M] interleaved gate/up)
     const void* bias1 = nullptr;           // bf16 [groups, M] (up bias, separate layout)

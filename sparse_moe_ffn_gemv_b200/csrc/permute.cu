@@ -70,14 +70,16 @@ __global__ void __launch_bounds__(kPlaceThreads) tile_start_kernel(const int32_t
     if (tid == 0) tile_start[E] = n;
 }
 
-// One warp per destination row, 16-byte vectors.
+// One warp per destination row, 16-byte vectors; only sorted positions in [*lo, *hi) when
+// those bounds are given (a range of experts).
 __global__ void __launch_bounds__(256) gather_rows_kernel(const uint4* __restrict__ src, int vpr,
                                                           const int32_t* __restrict__ sorted_slot, int k,
-                                                          int64_t S, uint4* __restrict__ dst) {
+                                                          int64_t S, uint4* __restrict__ dst,
+                                                          const int32_t* lo, const int32_t* hi) {
     pdl_begin();
     const int lane = threadIdx.x & 31;
     const int64_t p = (int64_t(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
-    if (p >= S) return;
+    if (p >= S || (lo && (p < *lo || p >= *hi))) return;
     const int64_t row = sorted_slot[p] / k;
     const uint4* s = src + row * vpr;
     uint4* d = dst + p * vpr;
@@ -87,12 +89,12 @@ __global__ void __launch_bounds__(256) gather_rows_kernel(const uint4* __restric
 }  // namespace
 
 cudaError_t launch_gather_rows(const void* src, int K, const int32_t* sorted_slot, int k, int64_t S, void* dst,
-                               cudaStream_t s) {
+                               cudaStream_t s, const int32_t* lo, const int32_t* hi) {
     if (S == 0) return cudaSuccess;
     const int vpr = K * 2 / 16;
     const unsigned grid = unsigned((S * 32 + 255) / 256);
     { const cudaError_t e_ = launch_pdl(gather_rows_kernel, dim3(grid), dim3(256), 0, s, static_cast<const uint4*>(src), vpr, sorted_slot, k, S,
-                                            static_cast<uint4*>(dst)); if (e_ != cudaSuccess) return e_; }
+                                            static_cast<uint4*>(dst), lo, hi); if (e_ != cudaSuccess) return e_; }
     return cudaGetLastError();
 }
 

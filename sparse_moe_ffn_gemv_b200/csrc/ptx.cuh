@@ -44,6 +44,30 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* b, uint32_t parity, uint64_t
     }
 }
 
+// Arrive at grid barrier `ctr` and wait (bounded) until `target` blocks have arrived.
+// Writes of this block before the call are visible to every block after it.
+__device__ bool grid_barrier(unsigned* ctr, unsigned target, uint64_t deadline, int* status, int* flag) {
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        __threadfence();
+        atomicAdd(ctr, 1u);
+        int ok = 1;
+        for (uint32_t i = 0;; ++i) {
+            unsigned v;
+            asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(ctr) : "memory");
+            if (v >= target) break;
+            if ((i & 15u) == 15u && gtimer() > deadline) {
+                ok = 0;
+                set_status(status, MOE_ERR_DEVICE_TIMEOUT);
+                break;
+            }
+        }
+        *flag = ok;
+    }
+    __syncthreads();
+    return *flag != 0;
+}
+
 // L2 policies: weights stream through once (evict first); token tiles are re-read by
 // every weight-row block of their group (evict last).
 __device__ __forceinline__ uint64_t policy_evict_first() {

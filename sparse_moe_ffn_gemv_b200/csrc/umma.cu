@@ -1,21 +1,31 @@
 // umma.cu -- tensor-core (tcgen05 / TMEM) grouped GEMM fed by TMA, for prefill-sized batches.
 //
-// D[weight rows, BN tokens] = W[rows, K] . U[BN, K]^T per tile ("weights as M"): every
-// expert group is padded only to the token tile, and each weight tile is read from HBM once
-// and shared by the token tiles of its group through L2.
+// D[128 token rows, 256 weight rows] = U[tokens, K] . W[rows, K]^T per tile: the tokens
+// are the MMA's M side and the tile's 256 weight rows (128 gate + 128 up rows, or 256
+// output rows) its N side, so that one 128 x 256 x 16 MMA per K step reads 12 KB of shared
+// memory (a 128 x 128 pair of MMAs sharing the token tile would read 16 KB for the same
+// work). Every expert group is padded only to the token tile, and each weight tile is read
+// from HBM once and shared by the token tiles of its group through L2.
 //
 // One persistent CTA per SM, warp-specialised:
 //   warp 0      TMA producer: weight tile(s) + token tile per 64-wide K block into a
 //               STAGES-deep shared-memory ring (128-byte swizzle)
 //   warp 1      MMA issuer (one thread): tcgen05.mma kind::f16, bf16 x bf16 -> fp32 in
-//               TMEM; two accumulators (gate, up) in gate/up mode
-//   warps 2..9  epilogue (two warps per TMEM lane quarter, each half of the columns):
-//               tcgen05.ld, then SwiGLU / clamped SwiGLU -> bf16 h (gate/up),
-//               the weighted bf16 output row of every slot (down), or a plain store
+//               TMEM, M = 128 token rows x N = 256 weight rows
+//   warps 2..9  epilogue (two warps per TMEM lane quarter, each half of the columns; one
+//               token row per thread): tcgen05.ld, then SwiGLU / clamped SwiGLU -> bf16 h
+//               (gate/up: gate and up of a unit are columns u and 128 + u), the weighted
+//               combine (down: the slot's output row times its routing weight reduced
+//               into the token's fp32 routed sum with 16-byte vector reductions), or a
+//               plain store, each thread writing contiguous 16-byte vectors
 //   warps 10..17 (4-bit weights only) dequantisation: the producer loads the packed words,
 //               these warps write w = scale * q + bias as bf16 into the swizzled operand
 //               layout the MMA reads (mlxcel issue #974: affine 4-bit, per-group scale
-//               and bias), one K block ahead of the MMA
+//               and bias). With 4-bit weights the shared memory holds two rings: a deep
+//               one of small slots (the two packed tiles + the token tile of a K block)
+//               that TMA fills far ahead, and a shallow one of bf16 operand tiles that
+//               the dequantising warps fill and the MMA drains, so that load latency,
+//               dequantisation and MMA overlap instead of sharing one stage
 // TMEM holds two accumulator sets so the epilogue of one tile overlaps the main loop of
 // the next. Every mbarrier wait is bounded by %globaltimer; a wait that gives up records
 // MOE_ERR_DEVICE_TIMEOUT in the status word, drains its own outstanding copies / MMAs and
@@ -47,7 +57,6 @@ constexpr int kPkBytes = kBM * kBK / 2;  // packed 4-bit weight tile: 128 rows x
 constexpr int kMaxGroups = 512;   // expert groups whose tile table fits in shared memory
 constexpr uint64_t kWaitNs = 2000000000ull;  // 2 s bound on any single wait
 
-__device__ __forceinline__ void epi_bar() { asm volatile("bar.sync 1, %0;" ::"r"(kEpiThreads) : "memory"); }
 __device__ __forceinline__ void prefetch_tmap(const CUtensorMap* m) {
     asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(m)) : "memory");
 }
@@ -161,21 +170,28 @@ __device__ __forceinline__ TileInfo decode_tile(const TcParams& P, const GroupTa
 
 // Every tile carries two 128-row weight operands that share one token tile: the gate and
 // up rows of 128 intermediate units (gate/up), or 256 consecutive output rows (others).
-// With 4-bit weights a stage also holds the two packed tiles after the bf16 operands.
+// bf16 weights: STAGES stages of [A0 | A1 | B]. 4-bit weights: STAGES load slots of
+// [packed 0 | packed 1 | B] (TMA), then ASTAGES operand slots of [A0 | A1] (dequantised).
 template <bool GATEUP, int BN, int STAGES, bool Q4 = false>
 struct TcShape {
     static constexpr int A_BYTES = kBM * kBK * 2;                // 16 KB
     static constexpr int B_BYTES = BN * kBK * 2;
-    static constexpr int PK_OFF = 2 * A_BYTES + B_BYTES;         // packed tiles (4-bit only)
-    static constexpr int STAGE_BYTES = 2 * A_BYTES + B_BYTES + (Q4 ? 2 * kPkBytes : 0);
+    static constexpr int ASTAGES = Q4 ? 2 : 0;                   // dequantised operand slots
+    static constexpr int B_OFF = Q4 ? 2 * kPkBytes : 2 * A_BYTES;  // token tile within a stage
+    static constexpr int STAGE_BYTES = Q4 ? 2 * kPkBytes + B_BYTES : 2 * A_BYTES + B_BYTES;
+    static constexpr int ARING_OFF = STAGES * STAGE_BYTES;       // operand ring (4-bit only)
+    static constexpr int RING_BYTES = STAGES * STAGE_BYTES + ASTAGES * 2 * A_BYTES;
     static constexpr int THREADS = kTcThreads + (Q4 ? kDqThreads : 0);
     static constexpr int ACC_COLS = 2 * BN;                      // per accumulator set
     static constexpr int TMEM_COLS = 2 * ACC_COLS;               // double-buffered
     static constexpr int ROWS = GATEUP ? kBM : 2 * kBM;          // weight rows per tile
-    static constexpr int SMEM = STAGES * STAGE_BYTES + 1024 /*align*/ + 256 /*barriers*/ +
-                                int(sizeof(GroupTables)) + BN * 12 /*epilogue row pointers, weights*/;
+    static constexpr int SMEM = RING_BYTES + 1024 /*align*/ + 256 /*barriers*/ + int(sizeof(GroupTables)) +
+                                8 * 128 * 4 /*epilogue bias tables*/;
     static_assert(TMEM_COLS <= 512 && (TMEM_COLS & (TMEM_COLS - 1)) == 0, "TMEM columns");
     static_assert(BN % 32 == 0 && BN >= 32 && BN <= 256, "BN");
+    static_assert(STAGE_BYTES % 1024 == 0 && B_OFF % 1024 == 0, "swizzle atoms stay 1 KB aligned");
+    static_assert((2 * STAGES + 5 + 2 * ASTAGES) * 8 + 4 <= 256, "barriers fit their region");
+    static_assert(SMEM <= 232448, "dynamic shared memory per block");
 };
 
 // SwiGLU / clamped SwiGLU with the fast exponential (the result is rounded to bf16).
@@ -184,6 +200,11 @@ __device__ __forceinline__ float act_fast(int act, float g, float v, float limit
     const float gc = fminf(g, limit);
     const float vc = fminf(fmaxf(v, -limit), limit);
     return __fdividef(gc, 1.0f + __expf(-alpha * gc)) * (vc + 1.0f);
+}
+
+// Fire-and-forget add of four consecutive fp32 values in global memory (16-byte aligned).
+__device__ __forceinline__ void red_add_v4(float* p, float a, float b, float c, float d) {
+    asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(p), "f"(a), "f"(b), "f"(c), "f"(d) : "memory");
 }
 
 __device__ __forceinline__ float bf16_at(const void* p, int64_t i) {
@@ -243,22 +264,40 @@ __device__ __forceinline__ uint32_t sw128_offset(int r, int c) {
     return uint32_t((r >> 3) * 1024 + (r & 7) * 128 + ((c ^ (r & 7)) << 4));
 }
 
+// The two bf16 weight tiles of K block kc of a tile, by TMA, completing on `bar`.
+template <bool GATEUP>
+__device__ __forceinline__ void load_a_bf16(uint8_t* dst, const TcParams& P, const TileInfo& ti, int mrow, int kc,
+                                            uint64_t* bar, uint64_t pol) {
+    constexpr int A_BYTES = kBM * kBK * 2;
+    if (!GATEUP) {  // rows [mrow, mrow + 128) and [mrow + 128, mrow + 256)
+        tma_3d(dst, &P.a0[ti.prob], bar, kc, mrow, ti.group, pol);
+        tma_3d(dst + A_BYTES, &P.a0[ti.prob], bar, kc, mrow + kBM, ti.group, pol);
+    } else if (P.p[ti.prob].interleaved) {  // [E, I, 2, K]: plane 0 = gate rows, 1 = up rows
+        tma_4d(dst, &P.a0[ti.prob], bar, kc, 0, mrow, ti.group, pol);
+        tma_4d(dst + A_BYTES, &P.a0[ti.prob], bar, kc, 1, mrow, ti.group, pol);
+    } else {
+        tma_3d(dst, &P.a0[ti.prob], bar, kc, mrow, ti.group, pol);
+        tma_3d(dst + A_BYTES, &P.a1[ti.prob], bar, kc, mrow, ti.group, pol);
+    }
+}
+
 template <bool GATEUP, int BN, int STAGES, bool Q4>
 __global__ void __launch_bounds__(TcShape<GATEUP, BN, STAGES, Q4>::THREADS, 1)
     tc_gemm_kernel(const __grid_constant__ TcParams P) {
     using S = TcShape<GATEUP, BN, STAGES, Q4>;
+    constexpr int AS = S::ASTAGES > 0 ? S::ASTAGES : 1;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    uint64_t* full = reinterpret_cast<uint64_t*>(smem + STAGES * S::STAGE_BYTES);
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem + S::RING_BYTES);
     uint64_t* empty = full + STAGES;
     uint64_t* acc_full = empty + STAGES;
     uint64_t* acc_empty = acc_full + 2;
     uint64_t* drain = acc_empty + 2;
-    uint64_t* dq = drain + 1;  // 4-bit: stage dequantised (STAGES barriers)
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(dq + STAGES);
-    GroupTables& gt = *reinterpret_cast<GroupTables*>(smem + STAGES * S::STAGE_BYTES + 256);
-    __nv_bfloat16** e_row = reinterpret_cast<__nv_bfloat16**>(&gt + 1);  // output row of each token column
-    float* e_w = reinterpret_cast<float*>(e_row + BN);
+    uint64_t* dq = drain + 1;       // 4-bit: operand slot filled (dequantised or loaded)
+    uint64_t* aempty = dq + AS;     // 4-bit: operand slot consumed by the MMA
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(aempty + AS);
+    GroupTables& gt = *reinterpret_cast<GroupTables*>(smem + S::RING_BYTES + 256);
+    float* sbias = reinterpret_cast<float*>(&gt + 1);  // epilogue: 128 column biases per warp
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     if (warp == 0) {
@@ -277,7 +316,10 @@ __global__ void __launch_bounds__(TcShape<GATEUP, BN, STAGES, Q4>::THREADS, 1)
         }
         mbar_init(drain, 1);
         if (Q4)
-            for (int st = 0; st < STAGES; ++st) mbar_init(&dq[st], kDqThreads / 32);  // one arrive per warp
+            for (int st = 0; st < S::ASTAGES; ++st) {
+                mbar_init(&dq[st], kDqThreads / 32);  // one arrive per dequantising warp
+                mbar_init(&aempty[st], 1);            // one MMA commit
+            }
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
         asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
     }
@@ -309,6 +351,9 @@ __global__ void __launch_bounds__(TcShape<GATEUP, BN, STAGES, Q4>::THREADS, 1)
     if (warp == 0) {
         if (lane == 0) {
             // ---------------------------------------------------------- TMA producer
+            // bf16: both weight tiles + the token tile of each K block into one stage.
+            // 4-bit: the two packed tiles + the token tile into one load slot (the
+            // dequantising warps bring bf16 tiles into the operand ring themselves).
             uint32_t stage = 0, phase = 0;
             uint32_t armed = 0;  // bit s: stage s was filled at least once
             uint32_t last_par = 0;
@@ -317,6 +362,10 @@ __global__ void __launch_bounds__(TcShape<GATEUP, BN, STAGES, Q4>::THREADS, 1)
                 const TileInfo ti = decode_tile(P, gt, tile, t0);
                 const TcProblem& p = P.p[ti.prob];
                 const int nk = p.K / kBK;
+                const int mrow = ti.mb * S::ROWS;
+                // token rows: the smallest box (16, 32, 64, BN) that holds the valid tokens
+                const int bv = ti.nvalid <= 16 ? 0 : ti.nvalid <= 32 ? 1 : ti.nvalid <= 64 ? 2 : 3;
+                const uint32_t b_bytes = uint32_t(min(BN, 16 << bv)) * kBK * 2;
                 for (int kb = 0; kb < nk; ++kb) {
                     if (!mbar_wait(&empty[stage], phase ^ 1u, deadline)) {
                         timed_out = true;
@@ -324,34 +373,22 @@ __global__ void __launch_bounds__(TcShape<GATEUP, BN, STAGES, Q4>::THREADS, 1)
                     }
                     uint8_t* sb = smem + stage * S::STAGE_BYTES;
                     const int kc = kb * kBK;
-                    const int mrow = ti.mb * S::ROWS;
-                    // token rows: the smallest box (16, 32, 64, BN) that holds the valid tokens
-                    const int bv = ti.nvalid <= 16 ? 0 : ti.nvalid <= 32 ? 1 : ti.nvalid <= 64 ? 2 : 3;
-                    const uint32_t b_bytes = uint32_t(min(BN, 16 << bv)) * kBK * 2;
-                    if (Q4 && p.q4) {  // packed words of the two weight tiles (8 words per K block)
-                        mbar_expect_tx(&full[stage], 2 * kPkBytes + b_bytes);
-                        uint8_t* pk = sb + S::PK_OFF;
-                        if (!GATEUP) {
-                            tma_3d(pk, &P.a0[ti.prob], &full[stage], kb * 8, mrow, ti.group, pol_w);
-                            tma_3d(pk + kPkBytes, &P.a0[ti.prob], &full[stage], kb * 8, mrow + kBM, ti.group, pol_w);
+                    if constexpr (Q4) {
+                        if (p.q4) {  // packed words of the two weight tiles (8 words per K block)
+                            mbar_expect_tx(&full[stage], 2 * kPkBytes + b_bytes);
+                            tma_3d(sb, &P.a0[ti.prob], &full[stage], kb * 8, mrow, ti.group, pol_w);
+                            if (!GATEUP)
+                                tma_3d(sb + kPkBytes, &P.a0[ti.prob], &full[stage], kb * 8, mrow + kBM, ti.group, pol_w);
+                            else
+                                tma_3d(sb + kPkBytes, &P.a1[ti.prob], &full[stage], kb * 8, mrow, ti.group, pol_w);
                         } else {
-                            tma_3d(pk, &P.a0[ti.prob], &full[stage], kb * 8, mrow, ti.group, pol_w);
-                            tma_3d(pk + kPkBytes, &P.a1[ti.prob], &full[stage], kb * 8, mrow, ti.group, pol_w);
+                            mbar_expect_tx(&full[stage], b_bytes);
                         }
-                    } else if (!GATEUP) {  // rows [mrow, mrow + 128) and [mrow + 128, mrow + 256)
-                        mbar_expect_tx(&full[stage], 2 * S::A_BYTES + b_bytes);
-                        tma_3d(sb, &P.a0[ti.prob], &full[stage], kc, mrow, ti.group, pol_w);
-                        tma_3d(sb + S::A_BYTES, &P.a0[ti.prob], &full[stage], kc, mrow + kBM, ti.group, pol_w);
-                    } else if (p.interleaved) {  // [E, I, 2, K]: plane 0 = gate rows, 1 = up rows
-                        mbar_expect_tx(&full[stage], 2 * S::A_BYTES + b_bytes);
-                        tma_4d(sb, &P.a0[ti.prob], &full[stage], kc, 0, mrow, ti.group, pol_w);
-                        tma_4d(sb + S::A_BYTES, &P.a0[ti.prob], &full[stage], kc, 1, mrow, ti.group, pol_w);
                     } else {
                         mbar_expect_tx(&full[stage], 2 * S::A_BYTES + b_bytes);
-                        tma_3d(sb, &P.a0[ti.prob], &full[stage], kc, mrow, ti.group, pol_w);
-                        tma_3d(sb + S::A_BYTES, &P.a1[ti.prob], &full[stage], kc, mrow, ti.group, pol_w);
+                        load_a_bf16<GATEUP>(sb, P, ti, mrow, kc, &full[stage], pol_w);
                     }
-                    tma_2d(sb + 2 * S::A_BYTES, &P.b[ti.prob][bv], &full[stage], kc, ti.row0, pol_t);
+                    tma_2d(sb + S::B_OFF, &P.b[ti.prob][bv], &full[stage], kc, ti.row0, pol_t);
                     armed |= 1u << stage;
                     last_par = (last_par & ~(1u << stage)) | (phase << stage);
                     if (++stage == STAGES) {
@@ -370,7 +407,8 @@ __global__ void __launch_bounds__(TcShape<GATEUP, BN, STAGES, Q4>::THREADS, 1)
         if (lane == 0) {
             // ---------------------------------------------------------- MMA issuer
             uint32_t stage = 0, phase = 0, it = 0;
-            constexpr uint32_t idesc_base = idesc_bf16(BN) & ~(0x3Fu << 17);
+            uint32_t astage = 0, aphase = 0;
+            constexpr uint32_t idesc = idesc_bf16(2 * kBM);  // M = 128 token rows, N = 256 weight rows
             for (int tile = blockIdx.x; tile < total && !timed_out; tile += gridDim.x, ++it) {
                 const TileInfo ti = decode_tile(P, gt, tile, t0);
                 const TcProblem& p = P.p[ti.prob];
@@ -381,31 +419,33 @@ __global__ void __launch_bounds__(TcShape<GATEUP, BN, STAGES, Q4>::THREADS, 1)
                 }
                 tc_fence_after();
                 const uint32_t d0 = tmem_base + ab * S::ACC_COLS;
-                // MMA only over the tile's valid token columns, rounded up to the N step (16)
-                const uint32_t n_mma = uint32_t(min(BN, (ti.nvalid + 15) & ~15));
-                const uint32_t idesc = idesc_base | ((n_mma >> 3) << 17);
                 const int nk = p.K / kBK;
                 for (int kb = 0; kb < nk; ++kb) {
-                    // with 4-bit weights in the kernel every stage passes through the
-                    // dequantising warps (which only forward bf16 stages)
-                    if (!mbar_wait(Q4 ? &dq[stage] : &full[stage], phase, deadline)) {
+                    // 4-bit: the operand slot is complete once the dequantising warps have
+                    // filled it, which they do only after the load slot (token tile) landed
+                    if (!mbar_wait(Q4 ? &dq[astage] : &full[stage], Q4 ? aphase : phase, deadline)) {
                         timed_out = true;
                         break;
                     }
                     tc_fence_after();
-                    const uint32_t sa = su32(smem + stage * S::STAGE_BYTES);
-                    const uint32_t sbb = sa + 2 * S::A_BYTES;
+                    // the two 128-row weight tiles lie back to back: one 256-row operand
+                    const uint32_t sw = Q4 ? su32(smem + S::ARING_OFF + astage * 2 * S::A_BYTES)
+                                           : su32(smem + stage * S::STAGE_BYTES);
+                    const uint32_t st = su32(smem + stage * S::STAGE_BYTES + S::B_OFF);
 #pragma unroll
-                    for (int k = 0; k < kBK / 16; ++k) {
-                        const uint64_t bdesc = smem_desc(sbb + k * 32);
-                        const uint32_t acc = (kb > 0 || k > 0) ? 1u : 0u;
-                        umma(d0, smem_desc(sa + k * 32), bdesc, idesc, acc);
-                        umma(d0 + BN, smem_desc(sa + S::A_BYTES + k * 32), bdesc, idesc, acc);
-                    }
+                    for (int k = 0; k < kBK / 16; ++k)
+                        umma(d0, smem_desc(st + k * 32), smem_desc(sw + k * 32), idesc, (kb > 0 || k > 0) ? 1u : 0u);
                     umma_commit(&empty[stage]);
                     if (++stage == STAGES) {
                         stage = 0;
                         phase ^= 1u;
+                    }
+                    if constexpr (Q4) {
+                        umma_commit(&aempty[astage]);
+                        if (++astage == uint32_t(S::ASTAGES)) {
+                            astage = 0;
+                            aphase ^= 1u;
+                        }
                     }
                 }
                 if (timed_out) break;
@@ -419,28 +459,50 @@ __global__ void __launch_bounds__(TcShape<GATEUP, BN, STAGES, Q4>::THREADS, 1)
     } else if (Q4 && warp >= kTcThreads / 32) {
         // ---------------------------------------------------------- dequantisation warps
         // Thread d dequantises row d % 128 of kDqTiles of the two weight tiles (all 64 K
-        // elements of the block: two 16-byte loads of packed words, eight swizzled 16-byte
-        // stores per row). Its (scale, bias) pairs are loaded two K blocks ahead.
+        // elements of the block: two 16-byte loads of packed words from the load slot, eight
+        // swizzled 16-byte stores into the operand slot). Its (scale, bias) pairs are loaded
+        // three K blocks ahead. A bf16 tile in the same launch (the shared expert) gets its
+        // operand slot filled by TMA, issued by the first dequantising thread.
         constexpr int DT = kDqTiles;
         const int d = threadIdx.x - kTcThreads;
         const int drow = d & (kBM - 1), a0 = (d / kBM) * DT;
+        const bool leader = d == 0;
         uint32_t stage = 0, phase = 0;
+        uint32_t astage = 0, aphase = 0;
+        uint32_t a_armed = 0, a_last = 0;  // leader: operand slots it filled by TMA
+        const uint64_t pol_w = policy_evict_first();
+        auto next = [&]() {
+            if (++stage == STAGES) {
+                stage = 0;
+                phase ^= 1u;
+            }
+            if (++astage == uint32_t(S::ASTAGES)) {
+                astage = 0;
+                aphase ^= 1u;
+            }
+        };
         for (int tile = blockIdx.x; tile < total && !timed_out; tile += gridDim.x) {
             const TileInfo ti = decode_tile(P, gt, tile, t0);
             const TcProblem& p = P.p[ti.prob];
             const int nk = p.K / kBK;
-            if (!p.q4) {  // bf16 tile: the stage goes straight on to the MMA
+            const int mrow = ti.mb * S::ROWS;
+            if (!p.q4) {  // bf16 tile: the leader loads both weight tiles into the operand slot
                 for (int kb = 0; kb < nk; ++kb) {
-                    if (!mbar_wait(&full[stage], phase, deadline)) {
+                    if (!mbar_wait(&full[stage], phase, deadline) || !mbar_wait(&aempty[astage], aphase ^ 1u, deadline)) {
                         timed_out = true;
                         break;
                     }
                     __syncwarp();
-                    if (lane == 0) mbar_arrive(&dq[stage]);
-                    if (++stage == STAGES) {
-                        stage = 0;
-                        phase ^= 1u;
+                    if (leader) {
+                        mbar_expect_tx(&dq[astage], 2 * S::A_BYTES);  // counts as this warp's arrive
+                        load_a_bf16<GATEUP>(smem + S::ARING_OFF + astage * 2 * S::A_BYTES, P, ti, mrow, kb * kBK,
+                                            &dq[astage], pol_w);
+                        a_armed |= 1u << astage;
+                        a_last = (a_last & ~(1u << astage)) | (aphase << astage);
+                    } else if (lane == 0) {
+                        mbar_arrive(&dq[astage]);
                     }
+                    next();
                 }
                 continue;
             }
@@ -453,7 +515,7 @@ __global__ void __launch_bounds__(TcShape<GATEUP, BN, STAGES, Q4>::THREADS, 1)
 #pragma unroll
             for (int ai = 0; ai < DT; ++ai) {
                 const int a = a0 + ai;
-                const int r = min(ti.mb * S::ROWS + (GATEUP ? 0 : a * kBM) + drow, p.M - 1);
+                const int r = min(mrow + (GATEUP ? 0 : a * kBM) + drow, p.M - 1);
                 const int64_t off = (int64_t(ti.group) * p.M + r) * p.qrow_step * ng;
                 sp[ai] = static_cast<const unsigned char*>((GATEUP && a == 1) ? p.qs1 : p.qs0) + off * (p.mx ? 1 : 2);
                 zp[ai] = p.mx ? nullptr : static_cast<const unsigned char*>((GATEUP && a == 1) ? p.qz1 : p.qz0) + off * 2;
@@ -480,21 +542,23 @@ __global__ void __launch_bounds__(TcShape<GATEUP, BN, STAGES, Q4>::THREADS, 1)
                         }
                     }
             };
-            __nv_bfloat162 q0[DT][2], q1[DT][2];
+            __nv_bfloat162 q0[DT][2], q1[DT][2], q2[DT][2];
             load_sb(0, q0);
             if (nk > 1) load_sb(1, q1);
+            if (nk > 2) load_sb(2, q2);
             for (int kb = 0; kb < nk; ++kb) {
-                __nv_bfloat162 q2[DT][2];
-                if (kb + 2 < nk) load_sb(kb + 2, q2);
-                if (!mbar_wait(&full[stage], phase, deadline)) {
+                __nv_bfloat162 q3[DT][2];
+                if (kb + 3 < nk) load_sb(kb + 3, q3);
+                if (!mbar_wait(&full[stage], phase, deadline) || !mbar_wait(&aempty[astage], aphase ^ 1u, deadline)) {
                     timed_out = true;
                     break;
                 }
-                uint8_t* sb = smem + stage * S::STAGE_BYTES;
+                const uint8_t* lb = smem + stage * S::STAGE_BYTES;
+                uint8_t* ob = smem + S::ARING_OFF + astage * 2 * S::A_BYTES;
 #pragma unroll
                 for (int ai = 0; ai < DT; ++ai) {
                     const int a = a0 + ai;
-                    const uint4* pk = reinterpret_cast<const uint4*>(sb + S::PK_OFF + a * kPkBytes + drow * 32);
+                    const uint4* pk = reinterpret_cast<const uint4*>(lb + a * kPkBytes + drow * 32);
                     const uint4 w0 = pk[0], w1 = pk[1];
                     const uint32_t words[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
 #pragma unroll
@@ -503,175 +567,192 @@ __global__ void __launch_bounds__(TcShape<GATEUP, BN, STAGES, Q4>::THREADS, 1)
                         uint4 v;
                         if constexpr (MX) v = dequant8_mx(words[c], sbv);
                         else v = dequant8(words[c], __low2bfloat162(sbv), __high2bfloat162(sbv));
-                        *reinterpret_cast<uint4*>(sb + a * S::A_BYTES + sw128_offset(drow, c)) = v;
+                        *reinterpret_cast<uint4*>(ob + a * S::A_BYTES + sw128_offset(drow, c)) = v;
                     }
                 }
                 // generic-proxy writes, read next by the tensor cores (async proxy)
                 asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
                 __syncwarp();
-                if (lane == 0) mbar_arrive(&dq[stage]);
+                if (lane == 0) mbar_arrive(&dq[astage]);
 #pragma unroll
                 for (int ai = 0; ai < DT; ++ai)
 #pragma unroll
                     for (int h = 0; h < 2; ++h) {
                         q0[ai][h] = q1[ai][h];
                         q1[ai][h] = q2[ai][h];
+                        q2[ai][h] = q3[ai][h];
                     }
-                if (++stage == STAGES) {
-                    stage = 0;
-                    phase ^= 1u;
-                }
+                next();
             }
             };
             if (p.mx) run(std::true_type{});
             else run(std::false_type{});
         }
+        // drain: the operand loads the leader issued have landed before the CTA can exit
+        if (leader) {
+            const uint64_t dl2 = gtimer() + kWaitNs;
+            for (int s = 0; s < S::ASTAGES; ++s)
+                if ((a_armed >> s) & 1u) mbar_wait(&dq[s], (a_last >> s) & 1u, dl2);
+        }
         if (timed_out) set_status(P.status, MOE_ERR_DEVICE_TIMEOUT);
     } else {
         // -------------------------------------------------------------- epilogue (256 threads)
-        const int q = warp & 3;                  // TMEM lane quarter of this warp
-        const int lrow = q * 32 + lane;          // accumulator row = weight row in the tile
-        const int eid = threadIdx.x - 64;        // 0..255
-        const int c_lo = (eid >= 128) ? BN / 2 : 0;  // this warp's half of the columns
+        // Accumulator lane = token row of the tile, column = weight row. The two warps of a
+        // TMEM lane quarter take one half each of the 256 columns; in gate/up mode a half is
+        // 64 intermediate units, read from both the gate (columns 0..127) and the up
+        // (columns 128..255) block. Each warp stages the biases of its own columns in a
+        // warp-private slice of shared memory, so that no epilogue step waits on another warp.
+        const int q = warp & 3;
+        const int tok = q * 32 + lane;  // token row of the tile
+        const int eid = threadIdx.x - 64;
+        const int half = eid >= 128 ? 1 : 0;
+        float* sb = sbias + (eid >> 5) * 128;  // this warp's column biases (warp-private)
         uint32_t it = 0;
         for (int tile = blockIdx.x; tile < total; tile += gridDim.x, ++it) {
             const TileInfo ti = decode_tile(P, gt, tile, t0);
             const TcProblem& p = P.p[ti.prob];
             const uint32_t ab = it & 1u, aph = (it >> 1) & 1u;
+            const bool tv = tok < ti.nvalid;
+            const int64_t prow = int64_t(ti.row0) + tok;
+            float wslot = 0.f;
+            float* yrow = nullptr;
+            if (!GATEUP && p.mode == kEpiScatterAdd && tv) {  // this token row's slot, before the wait
+                const int slot = p.sorted_slot[prow];
+                wslot = p.topk_w[slot];
+                yrow = reinterpret_cast<float*>(p.out) + int64_t(slot / p.k) * p.ld_out;
+            }
+            const bool has_bias = p.bias0 != nullptr;
+            if (has_bias) {  // the 128 biases of this warp's columns: 4 per lane, before the wait
+                __syncwarp();  // every lane is done with the previous tile's values
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    const int j = lane + 32 * i;
+                    float b = 0.f;
+                    if (GATEUP) {  // j < 64: gate bias of unit u0 + j, else up bias of unit u0 + j - 64
+                        const int unit = ti.mb * kBM + half * 64 + (j & 63);
+                        const int up = j >= 64 ? 1 : 0;
+                        if (unit < p.M)
+                            b = p.bias_interleaved ? bf16_at(p.bias0, (int64_t(ti.group) * p.M + unit) * 2 + up)
+                                                   : bf16_at(up ? p.bias1 : p.bias0, int64_t(ti.group) * p.M + unit);
+                    } else {
+                        const int r = ti.mb * 2 * kBM + half * kBM + j;
+                        if (r < p.M) b = bf16_at(p.bias0, int64_t(ti.group) * p.M + r);
+                    }
+                    sb[j] = b;
+                }
+                __syncwarp();
+            }
             if (!mbar_wait(&acc_full[ab], aph, deadline)) {
                 set_status(P.status, MOE_ERR_DEVICE_TIMEOUT);
                 break;
             }
             tc_fence_after();
-            if (!GATEUP && p.mode == kEpiSlotRows) {  // the tile's slot ids and weights, once
-                epi_bar();
-                if (eid < BN && eid < ti.nvalid) {
-                    const int slot = p.sorted_slot[ti.row0 + eid];
-                    e_row[eid] = reinterpret_cast<__nv_bfloat16*>(p.out) + int64_t(slot) * p.ld_out;
-                    e_w[eid] = p.topk_w[slot];
-                }
-                epi_bar();
-            }
             const uint32_t tb = tmem_base + (uint32_t(q * 32) << 16) + ab * S::ACC_COLS;
-            if constexpr (GATEUP) {
-                // gate and up of one intermediate unit for this warp's 64 token columns
-                const int r = ti.mb * S::ROWS + lrow;
-                const bool rv = r < p.M;
-                float bias0 = 0.f, bias1 = 0.f;
-                if (rv && p.bias0) {
-                    if (p.bias_interleaved) {
-                        bias0 = bf16_at(p.bias0, int64_t(ti.group) * 2 * p.M + 2 * r);
-                        bias1 = bf16_at(p.bias0, int64_t(ti.group) * 2 * p.M + 2 * r + 1);
-                    } else {
-                        bias0 = bf16_at(p.bias0, int64_t(ti.group) * p.M + r);
-                        bias1 = bf16_at(p.bias1, int64_t(ti.group) * p.M + r);
-                    }
-                }
-                uint32_t hp[32];  // 64 activated values, two bf16 per register
-#pragma unroll
-                for (int h2 = 0; h2 < 2; ++h2) {
-                    uint32_t g[32], u[32];
-                    tmem_ld_issue(tb + c_lo + 32 * h2, g);
-                    tmem_ld_issue(tb + BN + c_lo + 32 * h2, u);
-                    tmem_ld_wait(g);
-                    tmem_ld_wait(u);
-#pragma unroll
-                    for (int j = 0; j < 32; j += 2) {
-                        const float a0 = act_fast(P.act, __uint_as_float(g[j]) + bias0,
-                                                  __uint_as_float(u[j]) + bias1, P.limit, P.alpha);
-                        const float a1 = act_fast(P.act, __uint_as_float(g[j + 1]) + bias0,
-                                                  __uint_as_float(u[j + 1]) + bias1, P.limit, P.alpha);
-                        __nv_bfloat162 v2 = __floats2bfloat162_rn(a0, a1);
-                        hp[h2 * 16 + j / 2] = *reinterpret_cast<uint32_t*>(&v2);
-                    }
-                }
-                // the accumulator set is free for the next tile before any global store
+            auto release = [&]() {  // the accumulator set is free for the tile after next
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&acc_empty[ab]);
-                if (rv) {
-                    __nv_bfloat16* out = reinterpret_cast<__nv_bfloat16*>(p.out) + r;
+            };
+            if constexpr (GATEUP) {
+                // 32 units per chunk: gate and up of the same units -> 32 bf16 of h (64 bytes)
+                const int u0 = ti.mb * kBM + half * 64;
+#pragma unroll 1
+                for (int c = 0; c < 2; ++c) {
+                    uint32_t g[32], u[32];
+                    tmem_ld_issue(tb + half * 64 + 32 * c, g);
+                    tmem_ld_issue(tb + kBM + half * 64 + 32 * c, u);
+                    tmem_ld_wait(g);
+                    tmem_ld_wait(u);
+                    if (c == 1) release();
+                    const int ub = u0 + 32 * c;
+                    if (!tv || ub >= p.M) continue;
+                    const float* bg = sb + 32 * c;  // gate biases of these 32 units
+                    const float* bu = bg + 64;       // their up biases
+                    uint32_t hp[16];
 #pragma unroll
-                    for (int j = 0; j < 64; ++j) {
-                        const int n = c_lo + j;
-                        if (n < ti.nvalid) {
-                            const uint32_t w2 = hp[j / 2];
-                            const unsigned short b = (j & 1) ? (unsigned short)(w2 >> 16) : (unsigned short)(w2 & 0xFFFFu);
-                            reinterpret_cast<unsigned short*>(out)[int64_t(ti.row0 + n) * p.ld_out] = b;
+                    for (int j = 0; j < 32; j += 2) {
+                        float gg0 = __uint_as_float(g[j]), gg1 = __uint_as_float(g[j + 1]);
+                        float uu0 = __uint_as_float(u[j]), uu1 = __uint_as_float(u[j + 1]);
+                        if (has_bias) {
+                            gg0 += bg[j]; gg1 += bg[j + 1];
+                            uu0 += bu[j]; uu1 += bu[j + 1];
                         }
+                        __nv_bfloat162 v2 = __floats2bfloat162_rn(act_fast(P.act, gg0, uu0, P.limit, P.alpha),
+                                                                  act_fast(P.act, gg1, uu1, P.limit, P.alpha));
+                        hp[j / 2] = *reinterpret_cast<uint32_t*>(&v2);
                     }
+                    uint4* dst = reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(p.out) + prow * p.ld_out + ub);
+#pragma unroll
+                    for (int v = 0; v < 4; ++v) dst[v] = make_uint4(hp[4 * v], hp[4 * v + 1], hp[4 * v + 2], hp[4 * v + 3]);
                 }
             } else {
-                // two 128-row accumulators x this warp's 64 token columns
-                const bool full_tile = ti.nvalid >= c_lo + 64;
-                const int nend = full_tile ? 64 : max(0, ti.nvalid - c_lo);
-                auto store_acc = [&](int a, const uint32_t (&va)[2][32]) {
-                    const int r = ti.mb * S::ROWS + a * kBM + lrow;
-                    if (r >= p.M) return;
-                    const float bias0 = p.bias0 ? bf16_at(p.bias0, int64_t(ti.group) * p.M + r) : 0.f;
-                    if (p.mode == kEpiSlotRows) {
-                        // weighted output row of each slot (bf16); the combine sums a token's k rows
-                        if (full_tile) {
+                // 32 weight rows (output columns) per chunk, the next chunk's TMEM load in flight
+                const int rb = ti.mb * 2 * kBM + half * kBM;
+                // bf16 weights: the next chunk's TMEM load in flight while this one is stored;
+                // 4-bit weights (the dequantising warps share the register file): one at a time
+                constexpr int NB = Q4 ? 1 : 2;
+                uint32_t v[NB][32];
+                tmem_ld_issue(tb + half * kBM, v[0]);
 #pragma unroll
-                            for (int j = 0; j < 64; ++j)
-                                e_row[c_lo + j][r] =
-                                    __float2bfloat16_rn(e_w[c_lo + j] * (__uint_as_float(va[j / 32][j % 32]) + bias0));
+                for (int c = 0; c < 4; ++c) {
+                    tmem_ld_wait(v[c % NB]);
+                    if (NB == 2 && c < 3) tmem_ld_issue(tb + half * kBM + 32 * (c + 1), v[(c + 1) % NB]);
+                    if (c == 3) release();
+                    const int r0 = rb + 32 * c;
+                    float o[32];
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) o[j] = __uint_as_float(v[c % NB][j]);
+                    if (NB == 1 && c < 3) tmem_ld_issue(tb + half * kBM + 32 * (c + 1), v[0]);
+                    if (!tv || r0 >= p.M) continue;
+                    if (has_bias) {
+#pragma unroll
+                        for (int j = 0; j < 32; ++j) o[j] += sb[32 * c + j];
+                    }
+                    const bool whole = r0 + 32 <= p.M;
+                    if (p.mode == kEpiScatterAdd) {
+                        // weighted combine into the token's fp32 routed sum, 16 bytes per
+                        // reduction (libmir-metal execute: down weighted by routing.weights and
+                        // summed per token); M is a multiple of 64 here
+#pragma unroll
+                        for (int j = 0; j < 32; j += 4)
+                            red_add_v4(yrow + r0 + j, wslot * o[j], wslot * o[j + 1], wslot * o[j + 2], wslot * o[j + 3]);
+                    } else if (p.mode == kEpiStoreF32) {
+                        float* dst = reinterpret_cast<float*>(p.out) + prow * p.ld_out + r0;
+                        if (whole) {
+#pragma unroll
+                            for (int j = 0; j < 32; j += 4)
+                                *reinterpret_cast<float4*>(dst + j) = make_float4(o[j], o[j + 1], o[j + 2], o[j + 3]);
                         } else {
 #pragma unroll
-                            for (int j = 0; j < 64; ++j)
-                                if (j < nend)
-                                    e_row[c_lo + j][r] = __float2bfloat16_rn(
-                                        e_w[c_lo + j] * (__uint_as_float(va[j / 32][j % 32]) + bias0));
+                            for (int j = 0; j < 32; ++j)
+                                if (r0 + j < p.M) dst[j] = o[j];
                         }
-                    } else if (p.mode == kEpiStoreF32) {
-                        float* o = reinterpret_cast<float*>(p.out) + int64_t(ti.row0 + c_lo) * p.ld_out + r;
-#pragma unroll
-                        for (int j = 0; j < 64; ++j)
-                            if (j < nend) o[int64_t(j) * p.ld_out] = __uint_as_float(va[j / 32][j % 32]) + bias0;
                     } else {  // kEpiStoreAct (+ optional fp32 addend)
-                        __nv_bfloat16* o = reinterpret_cast<__nv_bfloat16*>(p.out) + int64_t(ti.row0 + c_lo) * p.ld_out + r;
-                        const float* ad = p.addend ? p.addend + int64_t(ti.row0 + c_lo) * p.ld_add + r : nullptr;
+                        __nv_bfloat16* dst = reinterpret_cast<__nv_bfloat16*>(p.out) + prow * p.ld_out + r0;
+                        const float* ad = p.addend ? p.addend + prow * p.ld_add + r0 : nullptr;
+                        if (whole) {
+                            if (ad) {
 #pragma unroll
-                        for (int j = 0; j < 64; ++j) {
-                            if (j < nend) {
-                                float d = __uint_as_float(va[j / 32][j % 32]) + bias0;
-                                if (ad) d += ad[int64_t(j) * p.ld_add];
-                                o[int64_t(j) * p.ld_out] = __float2bfloat16_rn(d);
+                                for (int j = 0; j < 32; j += 4) {
+                                    const float4 a4 = __ldcs(reinterpret_cast<const float4*>(ad + j));
+                                    o[j] += a4.x; o[j + 1] += a4.y; o[j + 2] += a4.z; o[j + 3] += a4.w;
+                                }
                             }
+#pragma unroll
+                            for (int w4 = 0; w4 < 4; ++w4) {
+                                uint32_t hp[4];
+#pragma unroll
+                                for (int j = 0; j < 4; ++j) {
+                                    __nv_bfloat162 v2 = __floats2bfloat162_rn(o[8 * w4 + 2 * j], o[8 * w4 + 2 * j + 1]);
+                                    hp[j] = *reinterpret_cast<uint32_t*>(&v2);
+                                }
+                                reinterpret_cast<uint4*>(dst)[w4] = make_uint4(hp[0], hp[1], hp[2], hp[3]);
+                            }
+                        } else {
+#pragma unroll
+                            for (int j = 0; j < 32; ++j)
+                                if (r0 + j < p.M) dst[j] = __float2bfloat16_rn(o[j] + (ad ? ad[j] : 0.f));
                         }
-                    }
-                };
-                if constexpr (!Q4) {
-                    // both accumulators in registers, the TMEM set released before any store
-                    uint32_t v[2][2][32];
-                    tmem_ld_issue(tb + c_lo, v[0][0]);
-                    tmem_ld_issue(tb + c_lo + 32, v[0][1]);
-                    tmem_ld_issue(tb + BN + c_lo, v[1][0]);
-                    tmem_ld_issue(tb + BN + c_lo + 32, v[1][1]);
-                    tmem_ld_wait(v[0][0]);
-                    tmem_ld_wait(v[0][1]);
-                    tmem_ld_wait(v[1][0]);
-                    tmem_ld_wait(v[1][1]);
-                    tc_fence_before();
-                    __syncwarp();
-                    if (lane == 0) mbar_arrive(&acc_empty[ab]);
-                    store_acc(0, v[0]);
-                    store_acc(1, v[1]);
-                } else {
-                    // with the dequantising warps' share of the registers, one accumulator at a time
-#pragma unroll 1
-                    for (int a = 0; a < 2; ++a) {
-                        uint32_t v[2][32];
-                        tmem_ld_issue(tb + a * BN + c_lo, v[0]);
-                        tmem_ld_issue(tb + a * BN + c_lo + 32, v[1]);
-                        tmem_ld_wait(v[0]);
-                        tmem_ld_wait(v[1]);
-                        if (a == 1) {
-                            tc_fence_before();
-                            __syncwarp();
-                            if (lane == 0) mbar_arrive(&acc_empty[ab]);
-                        }
-                        store_acc(a, v);
                     }
                 }
             }
@@ -773,9 +854,9 @@ bool tc_q4_weight_map(CUtensorMap* m, const void* w, int E, int R, int K, int ro
 cudaError_t launch_tc_gemm(TcParams& P, bool gateup, int64_t max_tiles, cudaStream_t s) {
     bool q4 = false;
     for (int i = 0; i < P.nprob; ++i) q4 = q4 || P.p[i].q4;
-    if (q4) {  // a stage also holds the packed tiles: three stages fit
-        if (gateup) return launch_tc_t<true, kTcBN, 3, true>(P, max_tiles, s);
-        return launch_tc_t<false, kTcBN, 3, true>(P, max_tiles, s);
+    if (q4) {  // six load slots (packed tiles + token tile) feed two dequantised operand slots
+        if (gateup) return launch_tc_t<true, kTcBN, 6, true>(P, max_tiles, s);
+        return launch_tc_t<false, kTcBN, 6, true>(P, max_tiles, s);
     }
     if (gateup) return launch_tc_t<true, kTcBN, 4, false>(P, max_tiles, s);
     return launch_tc_t<false, kTcBN, 4, false>(P, max_tiles, s);

@@ -111,8 +111,14 @@ CLAMPED_MXFP4 = CLAMPED_BF16.replace(name="clamped_mxfp4", config_id=6, weight_f
 CLAMPED_MXFP4_NATIVE = CLAMPED_MXFP4.replace(name="clamped_mxfp4_native", config_id=7,
                                              gate_up_interleaved=True)
 
+# The 4-bit Klear block with its dense planes 4-bit as well (router, shared expert; the 2-row
+# blend head stays bf16), as a 4-bit checkpoint quantises its dense projections too (mlxcel
+# issue #974, the Jamba study).
+KLEAR_Q4_DENSE = KLEAR_Q4.replace(name="klear_q4_dense", config_id=8, dense_format="q4", dense_group_size=64,
+                                  token_counts=(1, 32, 2048))
+
 WORKLOADS = {s.name: s for s in (TINY_F32, KLEAR_BF16, KLEAR_Q4, CLAMPED_BF16, LATENT_BF16, CLAMPED_MXFP4,
-                                 CLAMPED_MXFP4_NATIVE)}
+                                 CLAMPED_MXFP4_NATIVE, KLEAR_Q4_DENSE)}
 
 BASE_SEED = 20261202
 

@@ -24,14 +24,16 @@ WEIGHT_FIELDS = [
     "shared_gate_w", "shared_up_w", "shared_down_w",
     "latent_down_w", "latent_up_w", "latent_norm_w",
     "gate_up_s", "gate_up_z",
+    "router_s", "router_z", "shared_gate_s", "shared_gate_z", "shared_up_s", "shared_up_z",
+    "shared_down_s", "shared_down_z", "latent_down_s", "latent_down_z", "latent_up_s", "latent_up_z",
 ]
 
 # The entry points include/moe.h declares.
 EXPORTS = [
     "moe_config_validate", "moe_weights_validate", "moe_workspace_size", "moe_route",
-    "moe_permute", "moe_grouped_ffn", "moe_latent_down", "moe_combine", "moe_block_forward",
+    "moe_permute", "moe_grouped_ffn", "moe_grouped_ffn_experts", "moe_latent_down", "moe_combine", "moe_block_forward",
     "moe_read_device_status", "moe_clear_device_status", "moe_status_string",
-    "moe_permute_noalloc", "moe_selftest_bounded_wait",
+    "moe_permute_noalloc", "moe_selftest_bounded_wait", "moe_selftest_grid_wait",
 ]
 
 STATUS = {0: "MOE_OK", 1: "MOE_ERR_INVALID_ARGUMENT", 2: "MOE_ERR_SHAPE_OVERFLOW",
@@ -53,7 +55,7 @@ class MoeConfig(ctypes.Structure):
         ("weight_format", ctypes.c_int32), ("group_size", ctypes.c_int32), ("bits", ctypes.c_int32),
         ("shared_mode", ctypes.c_int32), ("shared_intermediate", ctypes.c_int32),
         ("latent_dim", ctypes.c_int32), ("latent_use_norm", ctypes.c_int32),
-        ("rms_eps", ctypes.c_float),
+        ("rms_eps", ctypes.c_float), ("dense_format", ctypes.c_int32), ("dense_group_size", ctypes.c_int32),
     ]
 
 
@@ -87,6 +89,8 @@ def lib():
             "moe_route": [cfgp, wp, vp, i64, vp, vp, vp, vp, sz, vp],
             "moe_permute": [cfgp, vp, i64, vp, vp, vp, vp, sz, vp],
             "moe_grouped_ffn": [cfgp, wp, vp, i64, vp, vp, vp, vp, vp, sz, vp],
+            "moe_grouped_ffn_experts": [cfgp, wp, vp, i64, vp, vp, vp, ctypes.c_int32, ctypes.c_int32, vp, vp, sz,
+                                        vp],
             "moe_latent_down": [cfgp, wp, vp, i64, vp, vp, sz, vp],
             "moe_combine": [cfgp, wp, vp, vp, vp, i64, vp, vp, sz, vp],
             "moe_block_forward": [cfgp, wp, vp, i64, vp, vp, sz, vp],
@@ -94,6 +98,7 @@ def lib():
             "moe_clear_device_status": [vp, vp],
             "moe_permute_noalloc": [cfgp, vp, i64, vp, vp, vp, vp, vp],
             "moe_selftest_bounded_wait": [vp, i64, vp],
+            "moe_selftest_grid_wait": [vp, i64, vp],
         }
         for name, args in sig.items():
             fn = getattr(L, name)
@@ -118,10 +123,9 @@ def _check(status: int, where: str):
 
 
 def config_from_spec(spec) -> MoeConfig:
-    if getattr(spec, "dense_format", "act") != "act":
-        # 4-bit router / shared / latent planes: the oracle evaluates them, the library's
-        # kernels read those planes in the activation dtype only
-        raise ValueError(f"dense_format {spec.dense_format!r} is not supported by the CUDA library")
+    dense = getattr(spec, "dense_format", "act")
+    if dense not in ("act", "q4"):
+        raise ValueError(f"dense_format {dense!r}")
     return MoeConfig(
         hidden=spec.hidden, num_experts=spec.num_experts, top_k=spec.top_k,
         intermediate=spec.intermediate, scoring=inputs.SCORING[spec.scoring],
@@ -134,7 +138,8 @@ def config_from_spec(spec) -> MoeConfig:
         weight_format=inputs.DTYPE[spec.weight_format], group_size=spec.group_size,
         bits=spec.bits, shared_mode=inputs.SHARED[spec.shared_mode],
         shared_intermediate=spec.shared_intermediate, latent_dim=spec.latent_dim,
-        latent_use_norm=int(spec.latent_use_norm), rms_eps=float(spec.rms_eps))
+        latent_use_norm=int(spec.latent_use_norm), rms_eps=float(spec.rms_eps),
+        dense_format=inputs.DTYPE["q4"] if dense == "q4" else 0, dense_group_size=int(spec.dense_group_size))
 
 
 def weights_struct(dev: Dict[str, torch.Tensor]) -> MoeWeights:
@@ -189,6 +194,15 @@ def moe_grouped_ffn(cfg, w, u, T, expert_offsets, sorted_slot, topk_w, y_acc, ws
                                  _p(ws), ws.numel(), _stream(stream)), "moe_grouped_ffn")
 
 
+def moe_grouped_ffn_experts(cfg, w, u, T, expert_offsets, sorted_slot, topk_w, expert_begin, expert_end,
+                            y_acc, ws, stream=None):
+    """Routed experts [expert_begin, expert_end) only; w's routed planes hold just those."""
+    _check(lib().moe_grouped_ffn_experts(ctypes.byref(cfg), ctypes.byref(w), _p(u), int(T),
+                                         _p(expert_offsets), _p(sorted_slot), _p(topk_w), int(expert_begin),
+                                         int(expert_end), _p(y_acc), _p(ws), ws.numel(), _stream(stream)),
+           "moe_grouped_ffn_experts")
+
+
 def moe_latent_down(cfg, w, x, T, z, ws, stream=None):
     _check(lib().moe_latent_down(ctypes.byref(cfg), ctypes.byref(w), _p(x), int(T), _p(z),
                                  _p(ws), ws.numel(), _stream(stream)), "moe_latent_down")
@@ -216,6 +230,11 @@ def moe_permute_noalloc(cfg, topk_idx, T, expert_offsets, sorted_slot, slot_pos,
 def moe_selftest_bounded_wait(ws, timeout_ns: int, stream=None):
     """Run the bounded-wait self test: records MOE_ERR_DEVICE_TIMEOUT in ws's status word."""
     _check(lib().moe_selftest_bounded_wait(_p(ws), int(timeout_ns), _stream(stream)), "moe_selftest_bounded_wait")
+
+
+def moe_selftest_grid_wait(ws, timeout_ns: int, stream=None):
+    """Run the grid-barrier self test: records MOE_ERR_DEVICE_TIMEOUT in ws's status word."""
+    _check(lib().moe_selftest_grid_wait(_p(ws), int(timeout_ns), _stream(stream)), "moe_selftest_grid_wait")
 
 
 def moe_read_device_status(ws, stream=None) -> int:

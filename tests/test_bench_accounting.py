@@ -76,3 +76,11 @@ def test_headline_is_the_largest_single_gpu_workload():
     assert (args.workload, args.tokens) == ("latent_bf16", 8192)
     big = max(bench.PREFILL, key=lambda w: bench.block_flops(inputs.WORKLOADS[w], bench.PREFILL[w]))
     assert big == "latent_bf16"
+
+
+def test_dense_bytes_count_4bit_dense_planes_at_their_width():
+    s = inputs.KLEAR_Q4_DENSE
+    H, E, Is, g = s.hidden, s.num_experts, s.shared_intermediate, s.dense_group_size
+    q4 = lambda r, c: r * c // 2 + r * (c // g) * 4
+    assert bench.dense_bytes(s) == q4(E, H) + E * 4 + 2 * H * 2 + 3 * q4(Is, H)
+    assert bench.dense_bytes(s) < bench.dense_bytes(inputs.KLEAR_Q4) / 3

@@ -32,7 +32,7 @@ def declared_symbols():
 
 def test_library_exports_every_declared_symbol():
     names = declared_symbols()
-    assert len(names) == 14
+    assert len(names) == 16
     assert sorted(M.EXPORTS) == names
     lib = M.lib()
     for n in names:
@@ -149,13 +149,37 @@ def test_interleaved_4bit_plane_needs_its_own_companions(fmt):
     assert M.STATUS[M.moe_weights_validate(cfg, w3)] == "MOE_ERR_INVALID_ARGUMENT"
 
 
-def test_4bit_dense_planes_are_refused_by_the_binding():
-    """The oracle evaluates 4-bit router / shared / latent planes; the library reads those planes
-    in the activation dtype only, so the binding refuses such a spec instead of misreading it."""
-    from tiny_specs import DENSE_Q4
+def test_4bit_dense_planes_are_validated_before_any_launch():
+    """4-bit router / shared / latent planes (mlxcel issue #974, the Jamba study): accepted with
+    bf16 activations and a group that divides every width; hostile parameters are refused,
+    each beside a positive control."""
+    from tiny_specs import DENSE_Q4, DENSE_Q4_BLEND
+    for spec in (DENSE_Q4, DENSE_Q4_BLEND):
+        assert M.moe_config_validate(M.config_from_spec(spec)) == 0
+    bad_group = M.config_from_spec(DENSE_Q4)
+    bad_group.dense_group_size = 48
+    assert M.STATUS[M.moe_config_validate(bad_group)] == "MOE_ERR_INVALID_QUANTIZATION"
+    assert M.STATUS[M.moe_config_validate(M.config_from_spec(DENSE_Q4.replace(dense_group_size=128)))] == \
+        "MOE_ERR_INVALID_QUANTIZATION"                       # 128 does not divide hidden 64
+    bad_fmt = M.config_from_spec(DENSE_Q4)
+    bad_fmt.dense_format = 3                                 # MXFP4 dense planes: not a dense format here
+    assert M.STATUS[M.moe_config_validate(bad_fmt)] == "MOE_ERR_INVALID_ARGUMENT"
+    f32 = M.config_from_spec(inputs.TINY_F32)
+    f32.dense_format = 2
+    assert M.STATUS[M.moe_config_validate(f32)] == "MOE_ERR_UNSUPPORTED"
     with pytest.raises(ValueError, match="dense_format"):
-        M.config_from_spec(DENSE_Q4)
-    assert M.moe_config_validate(M.config_from_spec(DENSE_Q4.replace(dense_format="act"))) == 0
+        M.config_from_spec(DENSE_Q4.replace(dense_format="mxfp4"))
+
+
+def test_4bit_dense_planes_need_their_scales_and_biases():
+    from tiny_specs import DENSE_Q4
+    cfg = M.config_from_spec(DENSE_Q4)
+    w = inputs.make_weights(DENSE_Q4, threads=2)
+    ws = M.weights_struct(w)
+    assert M.moe_weights_validate(cfg, ws) == 0
+    for f in ("router_s", "shared_down_z", "latent_up_s"):
+        broken = M.weights_struct({k: v for k, v in w.items() if k != f})
+        assert M.STATUS[M.moe_weights_validate(cfg, broken)] == "MOE_ERR_MISSING_TENSOR", f
 
 
 def test_group_must_divide_the_widths():
@@ -245,10 +269,10 @@ def test_noalloc_permutation_rejects_sizes_beyond_its_fixed_scratch():
 
 def test_selftest_rejects_bad_arguments_before_any_launch():
     lib = M.lib()
-    assert M.STATUS[lib.moe_selftest_bounded_wait(None, 1000, None)] == "MOE_ERR_INVALID_ARGUMENT"
-    for ns in (0, -5, 2_000_000_000):
-        assert M.STATUS[lib.moe_selftest_bounded_wait(ctypes.c_void_p(1 << 20), ns, None)] == \
-            "MOE_ERR_INVALID_ARGUMENT"
+    for fn in (lib.moe_selftest_bounded_wait, lib.moe_selftest_grid_wait):
+        assert M.STATUS[fn(None, 1000, None)] == "MOE_ERR_INVALID_ARGUMENT"
+        for ns in (0, -5, 2_000_000_000):
+            assert M.STATUS[fn(ctypes.c_void_p(1 << 20), ns, None)] == "MOE_ERR_INVALID_ARGUMENT"
 
 
 def test_status_strings():
