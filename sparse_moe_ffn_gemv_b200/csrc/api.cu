@@ -50,9 +50,12 @@ WsLayout ws_layout(const moe_config& c, int64_t T) {
     L.s_acc = take(c.shared_mode != MOE_SHARED_NONE ? T * H * 4 : 0);
     L.z = take(Ld ? T * Ld * ab : 0);
     L.nrm = take(Ld ? T * Ld * ab : 0);
-    const bool tc = c.act_dtype == MOE_DTYPE_BF16;  // bf16 or 4-bit weights
-    L.uperm = take(tc ? T * k * K * 2 : 0);
     L.tiles = take((E + 1) * 4);
+    // fp16 copies of the token operands of 4-bit affine problems on the tensor cores
+    const bool aff = c.weight_format == MOE_DTYPE_Q4_AFFINE, dq = c.dense_format == MOE_DTYPE_Q4_AFFINE;
+    L.x16 = take((aff && !Ld) || dq ? T * H * 2 : 0);
+    L.z16 = take(Ld && aff ? T * Ld * 2 : 0);
+    L.n16 = take(Ld && dq ? T * Ld * 2 : 0);
     L.total = off;
     return L;
 }
@@ -372,7 +375,10 @@ moe_status run_route(const moe_config* c, const moe_weights* w, const void* x, i
                      cudaStream_t s, const PermOut* perm = nullptr) {
     const bool blend = c->shared_mode == MOE_SHARED_BLEND;
     const DenseGemvArgs r = router_args(c, w, x, T, ws, L);
-    if (dense_tc(c, T, c->hidden)) {
+    // a 4-bit router stays on the weight-streaming kernel at every size: it dequantises exactly
+    // in fp32 (s * sum q x + b * sum x), while the tensor cores would round each weight, and
+    // the selection keys decide integer expert choices
+    if (dense_tc(c, T, c->hidden) && !dense_q4(c)) {
         TcParams P;
         const int np = blend ? 2 : 1;
         for (int i = 0; i < np; ++i) {
@@ -452,14 +458,18 @@ moe_status run_experts_tc(const moe_config* c, const moe_weights* w, const void*
                           cudaStream_t s) {
     const int K = expert_in(*c), I = c->intermediate, E = rg.ne, k = c->top_k, H = c->hidden;
     const int32_t* goff = offsets ? offsets + rg.e0 : nullptr;  // the range's offsets [ne + 1]
+    // 4-bit affine problems run on fp16 operands: fp16 copies of their token inputs
+    const bool aff = rtc && c->weight_format == MOE_DTYPE_Q4_AFFINE, dq = stc && dense_q4(c);
+    void* x16 = at<void>(ws, L.x16);
+    void* u16 = c->latent_dim ? at<void>(ws, L.z16) : x16;
+    if (aff) MOE_CUDA(launch_to_f16(u, T * K, u16, s));
+    if (dq && !(aff && !c->latent_dim)) MOE_CUDA(launch_to_f16(x, T * H, x16, s));
     const int Is = c->shared_intermediate;
     const int64_t S = T * k;
     const int64_t n_dense = (T + kTcBN - 1) / kTcBN;
-    void* uperm = at<void>(ws, L.uperm);
     void* h = at<void>(ws, L.h);
     void* hs = at<void>(ws, L.hs);
     const int32_t* tiles = at<int32_t>(ws, L.tiles);
-    if (rtc) MOE_CUDA(launch_gather_rows(u, K, sorted_slot, k, S, uperm, s, goff, goff + E));
     {  // gate/up + activation
         TcParams P;
         int np = 0;
@@ -470,9 +480,10 @@ moe_status run_experts_tc(const moe_config* c, const moe_weights* w, const void*
             p.M = Is; p.K = H; p.m_blocks = (Is + kTcRowsGateUp - 1) / kTcRowsGateUp;
             p.rows = int(T); p.n_tiles = int(n_dense);
             p.out = hs; p.ld_out = Is;
+            p.out_f16 = dq ? 1 : 0;  // fp16 hs for the fp16 shared down GEMM
             if (!tc_dense_weights(c, p, &P.a0[np], &P.a1[np], w->shared_gate_w, w->shared_gate_s, w->shared_gate_z,
                                   w->shared_up_w, w->shared_up_s, w->shared_up_z, Is, H) ||
-                !tc_token_map(P.b[np], x, T, H, kTcBN))
+                !tc_token_map(P.b[np], dq ? x16 : x, T, H, kTcBN))
                 return MOE_ERR_CUDA;
             max_tiles += int64_t(p.m_blocks) * p.n_tiles;
             ++np;
@@ -524,7 +535,11 @@ moe_status run_experts_tc(const moe_config* c, const moe_weights* w, const void*
                 ok = tc_weight_map(&P.a0[np], w->gate_w, E, I, K, false) &&
                      tc_weight_map(&P.a1[np], w->up_w, E, I, K, false);
             }
-            if (!ok || !tc_token_map(P.b[np], uperm, S, K, kTcBN)) return MOE_ERR_CUDA;
+            // the tile's token rows are gathered from u by slot (TMA row gather, no copy)
+            p.gather_k = k;
+            p.sorted_slot = sorted_slot;
+            p.out_f16 = aff ? 1 : 0;  // fp16 h for the fp16 routed down GEMM
+            if (!ok || !tc_gather_map(&P.b[np][0], aff ? u16 : u, T, K)) return MOE_ERR_CUDA;
             max_tiles += int64_t(p.m_blocks) * max_routed_tiles(*c, T);
             ++np;
         }
@@ -681,7 +696,8 @@ moe_status run_experts(const moe_config* c, const moe_weights* w, const void* u,
 
 // a8 (first half): z = x Wdp^T
 moe_status run_latent_down(const moe_config* c, const moe_weights* w, const void* x, int64_t T, void* z,
-                           int* status, cudaStream_t s) {
+                           void* ws, const WsLayout& L, cudaStream_t s) {
+    int* status = at<int>(ws, L.status);
     DenseGemvArgs r;
     r.W0 = w->latent_down_w;
     r.rows0 = c->latent_dim;
@@ -704,9 +720,14 @@ moe_status run_latent_down(const moe_config* c, const moe_weights* w, const void
         p.M = c->latent_dim; p.K = c->hidden; p.m_blocks = (p.M + kTcRows - 1) / kTcRows;
         p.rows = int(T); p.n_tiles = int((T + kTcBN - 1) / kTcBN);
         p.out = z; p.ld_out = c->latent_dim;
+        const void* xt = x;
+        if (dense_q4(c)) {  // fp16 operands
+            xt = static_cast<char*>(ws) + L.x16;
+            MOE_CUDA(launch_to_f16(x, T * c->hidden, const_cast<void*>(xt), s));
+        }
         if (!tc_dense_weights(c, p, &P.a0[0], nullptr, w->latent_down_w, w->latent_down_s, w->latent_down_z, nullptr,
                               nullptr, nullptr, p.M, p.K) ||
-            !tc_token_map(P.b[0], x, T, p.K, kTcBN))
+            !tc_token_map(P.b[0], xt, T, p.K, kTcBN))
             return MOE_ERR_CUDA;
         P.nprob = 1;
         P.status = status;
@@ -761,9 +782,14 @@ moe_status run_output(const moe_config* c, const moe_weights* w, RoutedSum rs, c
         p.rows = int(T); p.n_tiles = int((T + kTcBN - 1) / kTcBN);
         p.out = y; p.ld_out = c->hidden;
         p.addend = s_acc; p.ld_add = c->hidden;
+        const void* nt = n;
+        if (dense_q4(c)) {  // fp16 operands
+            nt = at<void>(ws, L.n16);
+            MOE_CUDA(launch_to_f16(n, T * c->latent_dim, const_cast<void*>(nt), s));
+        }
         if (!tc_dense_weights(c, p, &P.a0[0], nullptr, w->latent_up_w, w->latent_up_s, w->latent_up_z, nullptr,
                               nullptr, nullptr, p.M, p.K) ||
-            !tc_token_map(P.b[0], n, T, p.K, kTcBN))
+            !tc_token_map(P.b[0], nt, T, p.K, kTcBN))
             return MOE_ERR_CUDA;
         P.nprob = 1;
         P.status = at<int>(ws, L.status);
@@ -879,7 +905,7 @@ moe_status moe_latent_down(const moe_config* cfg, const moe_weights* w, const vo
     if (T == 0) return MOE_OK;
     MOE_CHECK(check_ptr(x));
     MOE_CHECK(check_ptr(z));
-    return run_latent_down(cfg, w, x, T, z, at<int>(ws, L.status), (cudaStream_t)stream);
+    return run_latent_down(cfg, w, x, T, z, ws, L, (cudaStream_t)stream);
 }
 
 moe_status moe_combine(const moe_config* cfg, const moe_weights* w, const float* y_acc, const void* x,
@@ -935,7 +961,7 @@ moe_status moe_block_forward(const moe_config* cfg, const moe_weights* w, const 
     perm.active = at<int32_t>(ws, L.active);
     perm.tiles = rtc ? at<int32_t>(ws, L.tiles) : nullptr;
     MOE_CHECK(run_route(cfg, w, x, T, idx, wts, coef, y_acc, K, ws, L, s, &perm));
-    if (cfg->latent_dim) MOE_CHECK(run_latent_down(cfg, w, x, T, at<void>(ws, L.z), at<int>(ws, L.status), s));
+    if (cfg->latent_dim) MOE_CHECK(run_latent_down(cfg, w, x, T, at<void>(ws, L.z), ws, L, s));
     if (T > 1) MOE_CHECK(run_permute(cfg, idx, T, offsets, sorted_slot, at<int32_t>(ws, L.slot_pos), ws, L, s, rtc));
     RoutedSum rs;
     MOE_CHECK(run_experts(cfg, w, u, x, T, offsets, sorted_slot, wts, y_acc, true, true, ws, L, s, &rs));

@@ -3,6 +3,8 @@
 // Klear PR item 2: y = y_experts * coef[0] + shared * coef[1] (blend); ferrox
 // latent_moe.rs: output = routed_out + shared (add), and
 // combined = rms_norm(combined) with a [latent] weight before up_proj.
+#include <cuda_fp16.h>
+
 #include <algorithm>
 
 #include "common.cuh"
@@ -97,6 +99,22 @@ __global__ void __launch_bounds__(256) rmsnorm_kernel(const RT* __restrict__ row
         out[t * L + c] = from_f<AT>(row[c] * inv * to_f<AT>(gamma[c]));
 }
 
+// Eight bf16 values -> eight fp16 values per thread (exact within fp16's range).
+__global__ void __launch_bounds__(256) to_f16_kernel(const uint4* __restrict__ src, int64_t n8, uint4* __restrict__ dst) {
+    pdl_begin();
+    for (int64_t i = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; i < n8; i += int64_t(gridDim.x) * blockDim.x) {
+        float f[8];
+        unpack8(src[i], f);
+        uint32_t h[4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            __half2 v = __floats2half2_rn(f[2 * j], f[2 * j + 1]);
+            h[j] = *reinterpret_cast<uint32_t*>(&v);
+        }
+        dst[i] = make_uint4(h[0], h[1], h[2], h[3]);
+    }
+}
+
 template <typename RT>
 cudaError_t launch_combine_t(const RT* rows, int nsum, const float* s_acc, const float* coef, int mode, int64_t T,
                              int H, void* y, int act_dtype, cudaStream_t s, bool out_f32) {
@@ -134,6 +152,16 @@ cudaError_t launch_combine(const void* rows, int rows_dtype, int nsum, const flo
         return launch_combine_t(static_cast<const __nv_bfloat16*>(rows), nsum, s_acc, coef, mode, T, H, y, act_dtype,
                                 s, out_f32);
     return launch_combine_t(static_cast<const float*>(rows), nsum, s_acc, coef, mode, T, H, y, act_dtype, s, out_f32);
+}
+
+cudaError_t launch_to_f16(const void* src, int64_t n, void* dst, cudaStream_t s) {
+    if (n == 0) return cudaSuccess;
+    const int64_t n8 = n / 8;
+    const unsigned grid = unsigned(std::min<int64_t>((n8 + 255) / 256, 148 * 8));
+    const cudaError_t e = launch_pdl(to_f16_kernel, dim3(grid), dim3(256), 0, s, static_cast<const uint4*>(src), n8,
+                                     static_cast<uint4*>(dst));
+    if (e != cudaSuccess) return e;
+    return cudaGetLastError();
 }
 
 cudaError_t launch_rmsnorm(const void* rows, int rows_dtype, int nsum, const void* gamma, float eps, int64_t T,

@@ -42,8 +42,10 @@ struct WsLayout {
     size_t s_acc;        // f32 [T, H]: shared expert output
     size_t z;            // act [T, L]: latent input of the experts
     size_t nrm;          // act [T, L]: normalised latent
-    size_t uperm;        // bf16 [T * k, K]: expert inputs gathered in sorted order
     size_t tiles;        // int32 tile list of the tensor-core path
+    size_t x16;          // fp16 [T, H]: x as the fp16 token operand (4-bit affine weights)
+    size_t z16;          // fp16 [T, L]: the latent expert input likewise
+    size_t n16;          // fp16 [T, L]: the normalised latent likewise
     size_t total;
     int ld_logits;
     int n_chunks;

@@ -166,6 +166,12 @@ struct TcProblem {
     int mx = 0;  // with q4 = 1: MXFP4 codes, qs0 / qs1 the E8M0 scale bytes [groups, M, K / 32]
     int qrow_step = 1;  // companion rows per unit: 2 for an interleaved gate_up plane, whose
                         // up companions start one row after qs0 / qz0 (qs1 / qz1 = that row)
+    int gather_k = 0;   // > 0: token row i of a tile is row sorted_slot[row0 + i] / gather_k of the
+                        // token operand, fetched by TMA row gather (b[..][0] is the gather map)
+    // 4-bit affine weights run the MMA on fp16 operands (the dequantised s * q + b rounds to
+    // 11 significant bits; bf16 keeps 8): the token operand of such a problem is fp16, and
+    // out_f16 makes a gate/up problem write its h in fp16 for the fp16 down GEMM after it.
+    int out_f16 = 0;
 };
 
 struct alignas(64) TcParams {
@@ -193,6 +199,10 @@ bool tc_weight_map(CUtensorMap* m, const void* w, int E, int R, int K, bool inte
 bool tc_q4_weight_map(CUtensorMap* m, const void* w, int E, int R, int K, int row_step = 1);
 // Four maps m[0..3] of the token operand [rows, K] bf16, boxes of 16, 32, 64 and bn rows.
 bool tc_token_map(CUtensorMap* m, const void* u, int64_t rows, int K, int bn);
+// The token operand [rows, K] bf16 for TMA row gather: a box of one row x one K block.
+bool tc_gather_map(CUtensorMap* m, const void* u, int64_t rows, int K);
+// dst[i] = fp16(src[i]) for n bf16 values (exact within fp16's range), n % 8 == 0.
+cudaError_t launch_to_f16(const void* src, int64_t n, void* dst, cudaStream_t s);
 cudaError_t launch_tc_gemm(TcParams& P, bool gateup, int64_t max_tiles, cudaStream_t s);
 
 }  // namespace moe

@@ -39,6 +39,8 @@
 #include <mutex>
 #include <type_traits>
 
+#include <cuda_fp16.h>
+
 #include "common.cuh"
 #include "internal.h"
 #include "ptx.cuh"
@@ -72,6 +74,10 @@ __device__ __forceinline__ uint64_t smem_desc(uint32_t saddr) {
 // Instruction descriptor: kind::f16, A = B = bf16, D = f32, both K-major, M = 128, N = n.
 __host__ __device__ constexpr uint32_t idesc_bf16(int n) {
     return (1u << 4) | (1u << 7) | (1u << 10) | (uint32_t(n >> 3) << 17) | (uint32_t(kBM >> 4) << 24);
+}
+// The same with A = B = fp16 (4-bit affine weights).
+__host__ __device__ constexpr uint32_t idesc_f16(int n) {
+    return (1u << 4) | (uint32_t(n >> 3) << 17) | (uint32_t(kBM >> 4) << 24);
 }
 
 __device__ __forceinline__ void umma(uint32_t d, uint64_t a, uint64_t b, uint32_t idesc, uint32_t acc) {
@@ -211,24 +217,24 @@ __device__ __forceinline__ float bf16_at(const void* p, int64_t i) {
     return __bfloat162float(reinterpret_cast<const __nv_bfloat16*>(p)[i]);
 }
 
-// Eight 4-bit codes (element j in bits 4j..4j+3 of the word) -> eight bf16 weights
-// w = s * q + b, one rounding each. A code q becomes the exact bf16 128 + q by OR-ing it into
-// the mantissa of 128.0 (two codes per 32-bit pair: the pair (q_i, q_i+4) comes from the
-// same nibble position of both halves), PRMT puts neighbours together, and q = (128 + q) -
-// 128 is exact in bf16 before the single-rounding fma.
-__device__ __forceinline__ uint4 dequant8(uint32_t w, __nv_bfloat162 s2, __nv_bfloat162 b2) {
-    const uint32_t p0 = (w & 0x000F000Fu) | 0x43004300u;          // (q0, q4)
-    const uint32_t p1 = ((w >> 4) & 0x000F000Fu) | 0x43004300u;   // (q1, q5)
-    const uint32_t p2 = ((w >> 8) & 0x000F000Fu) | 0x43004300u;   // (q2, q6)
-    const uint32_t p3 = ((w >> 12) & 0x000F000Fu) | 0x43004300u;  // (q3, q7)
+// Eight 4-bit codes (element j in bits 4j..4j+3 of the word) -> eight fp16 weights
+// w = s * q + b, one rounding each. A code q becomes the exact fp16 1024 + q by OR-ing it into
+// the mantissa of 1024.0 (two codes per 32-bit pair: the pair (q_i, q_i+4) comes from the same
+// nibble position of both halves), PRMT puts neighbours together, and q = (1024 + q) - 1024 is
+// exact before the single-rounding fma.
+__device__ __forceinline__ uint4 dequant8_f16(uint32_t w, __half2 s2, __half2 b2) {
+    const uint32_t p0 = (w & 0x000F000Fu) | 0x64006400u;          // (q0, q4)
+    const uint32_t p1 = ((w >> 4) & 0x000F000Fu) | 0x64006400u;   // (q1, q5)
+    const uint32_t p2 = ((w >> 8) & 0x000F000Fu) | 0x64006400u;   // (q2, q6)
+    const uint32_t p3 = ((w >> 12) & 0x000F000Fu) | 0x64006400u;  // (q3, q7)
     const uint32_t o[4] = {__byte_perm(p0, p1, 0x5410), __byte_perm(p2, p3, 0x5410),
                            __byte_perm(p0, p1, 0x7632), __byte_perm(p2, p3, 0x7632)};
-    const __nv_bfloat162 off = __floats2bfloat162_rn(128.0f, 128.0f);
+    const __half2 off = __floats2half2_rn(1024.0f, 1024.0f);
     uint32_t r[4];
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
-        const __nv_bfloat162 q = __hsub2(*reinterpret_cast<const __nv_bfloat162*>(&o[i]), off);
-        const __nv_bfloat162 v = __hfma2(q, s2, b2);
+        const __half2 q = __hsub2(*reinterpret_cast<const __half2*>(&o[i]), off);
+        const __half2 v = __hfma2(q, s2, b2);
         r[i] = *reinterpret_cast<const uint32_t*>(&v);
     }
     return make_uint4(r[0], r[1], r[2], r[3]);
@@ -327,7 +333,7 @@ __global__ void __launch_bounds__(TcShape<GATEUP, BN, STAGES, Q4>::THREADS, 1)
         for (int i = 0; i < P.nprob; ++i) {
             prefetch_tmap(&P.a0[i]);
             if (GATEUP && !P.p[i].interleaved) prefetch_tmap(&P.a1[i]);
-            for (int v = 0; v < 4; ++v) prefetch_tmap(&P.b[i][v]);
+            for (int v = 0; v < (P.p[i].gather_k ? 1 : 4); ++v) prefetch_tmap(&P.b[i][v]);
         }
     }
     pdl_begin();  // everything above touches no memory that earlier kernels write
@@ -349,30 +355,42 @@ __global__ void __launch_bounds__(TcShape<GATEUP, BN, STAGES, Q4>::THREADS, 1)
     bool timed_out = false;
 
     if (warp == 0) {
-        if (lane == 0) {
-            // ---------------------------------------------------------- TMA producer
-            // bf16: both weight tiles + the token tile of each K block into one stage.
-            // 4-bit: the two packed tiles + the token tile into one load slot (the
-            // dequantising warps bring bf16 tiles into the operand ring themselves).
-            uint32_t stage = 0, phase = 0;
-            uint32_t armed = 0;  // bit s: stage s was filled at least once
-            uint32_t last_par = 0;
-            const uint64_t pol_w = policy_evict_first(), pol_t = policy_evict_last();
-            for (int tile = blockIdx.x; tile < total && !timed_out; tile += gridDim.x) {
-                const TileInfo ti = decode_tile(P, gt, tile, t0);
-                const TcProblem& p = P.p[ti.prob];
-                const int nk = p.K / kBK;
-                const int mrow = ti.mb * S::ROWS;
-                // token rows: the smallest box (16, 32, 64, BN) that holds the valid tokens
-                const int bv = ti.nvalid <= 16 ? 0 : ti.nvalid <= 32 ? 1 : ti.nvalid <= 64 ? 2 : 3;
-                const uint32_t b_bytes = uint32_t(min(BN, 16 << bv)) * kBK * 2;
-                for (int kb = 0; kb < nk; ++kb) {
-                    if (!mbar_wait(&empty[stage], phase ^ 1u, deadline)) {
-                        timed_out = true;
-                        break;
-                    }
-                    uint8_t* sb = smem + stage * S::STAGE_BYTES;
-                    const int kc = kb * kBK;
+        // -------------------------------------------------------------- TMA producer (one warp)
+        // bf16: both weight tiles + the token tile of each K block into one stage.
+        // 4-bit: the two packed tiles + the token tile into one load slot (the
+        // dequantising warps bring bf16 tiles into the operand ring themselves).
+        // Lane 0 waits for the slot, arms its barrier and loads the weight tiles; the token
+        // tile is one tiled load by lane 0, or, for a gathered problem, one four-row TMA gather
+        // per lane (lane l: the tile's token rows 4l .. 4l + 3).
+        uint32_t stage = 0, phase = 0;
+        uint32_t armed = 0;  // bit s: stage s was filled at least once
+        uint32_t last_par = 0;
+        const uint64_t pol_w = policy_evict_first(), pol_t = policy_evict_last();
+        for (int tile = blockIdx.x; tile < total && !timed_out; tile += gridDim.x) {
+            const TileInfo ti = decode_tile(P, gt, tile, t0);
+            const TcProblem& p = P.p[ti.prob];
+            const int nk = p.K / kBK;
+            const int mrow = ti.mb * S::ROWS;
+            // token rows: the smallest box (16, 32, 64, BN) that holds the valid tokens
+            const int bv = ti.nvalid <= 16 ? 0 : ti.nvalid <= 32 ? 1 : ti.nvalid <= 64 ? 2 : 3;
+            const bool gath = p.gather_k > 0;
+            const int ngr = gath ? (ti.nvalid + 3) / 4 : 0;  // lanes that gather four rows
+            const uint32_t b_bytes = gath ? uint32_t(ngr) * 4 * kBK * 2 : uint32_t(min(BN, 16 << bv)) * kBK * 2;
+            int gr[4] = {0, 0, 0, 0};  // this lane's four token rows (padding rows read row 0)
+            if (gath && lane < ngr)
+#pragma unroll
+                for (int j = 0; j < 4; ++j)
+                    if (4 * lane + j < ti.nvalid) gr[j] = p.sorted_slot[ti.row0 + 4 * lane + j] / p.gather_k;
+            for (int kb = 0; kb < nk; ++kb) {
+                int ok = 1;
+                if (lane == 0) ok = mbar_wait(&empty[stage], phase ^ 1u, deadline) ? 1 : 0;
+                if (!__shfl_sync(0xffffffffu, ok, 0)) {
+                    timed_out = true;
+                    break;
+                }
+                uint8_t* sb = smem + stage * S::STAGE_BYTES;
+                const int kc = kb * kBK;
+                if (lane == 0) {
                     if constexpr (Q4) {
                         if (p.q4) {  // packed words of the two weight tiles (8 words per K block)
                             mbar_expect_tx(&full[stage], 2 * kPkBytes + b_bytes);
@@ -388,27 +406,35 @@ __global__ void __launch_bounds__(TcShape<GATEUP, BN, STAGES, Q4>::THREADS, 1)
                         mbar_expect_tx(&full[stage], 2 * S::A_BYTES + b_bytes);
                         load_a_bf16<GATEUP>(sb, P, ti, mrow, kc, &full[stage], pol_w);
                     }
-                    tma_2d(sb + S::B_OFF, &P.b[ti.prob][bv], &full[stage], kc, ti.row0, pol_t);
-                    armed |= 1u << stage;
-                    last_par = (last_par & ~(1u << stage)) | (phase << stage);
-                    if (++stage == STAGES) {
-                        stage = 0;
-                        phase ^= 1u;
-                    }
+                    if (!gath) tma_2d(sb + S::B_OFF, &P.b[ti.prob][bv], &full[stage], kc, ti.row0, pol_t);
+                }
+                __syncwarp();  // the barrier expects the gathered bytes before any gather lands
+                if (gath && lane < ngr)
+                    tma_gather4(sb + S::B_OFF + lane * 4 * kBK * 2, &P.b[ti.prob][0], &full[stage], kc, gr[0], gr[1],
+                                gr[2], gr[3], pol_t);
+                armed |= 1u << stage;
+                last_par = (last_par & ~(1u << stage)) | (phase << stage);
+                if (++stage == STAGES) {
+                    stage = 0;
+                    phase ^= 1u;
                 }
             }
-            // drain: every copy this thread issued has landed before the CTA can exit
+        }
+        // drain: every copy this warp issued has landed before the CTA can exit
+        if (lane == 0) {
             const uint64_t dl2 = gtimer() + kWaitNs;
             for (int s = 0; s < STAGES; ++s)
                 if ((armed >> s) & 1u) mbar_wait(&full[s], (last_par >> s) & 1u, dl2);
             if (timed_out) set_status(P.status, MOE_ERR_DEVICE_TIMEOUT);
         }
+        __syncwarp();
     } else if (warp == 1) {
         if (lane == 0) {
             // ---------------------------------------------------------- MMA issuer
             uint32_t stage = 0, phase = 0, it = 0;
             uint32_t astage = 0, aphase = 0;
-            constexpr uint32_t idesc = idesc_bf16(2 * kBM);  // M = 128 token rows, N = 256 weight rows
+            // M = 128 token rows, N = 256 weight rows; fp16 operands for 4-bit affine weights
+            constexpr uint32_t idesc_b = idesc_bf16(2 * kBM), idesc_h = idesc_f16(2 * kBM);
             for (int tile = blockIdx.x; tile < total && !timed_out; tile += gridDim.x, ++it) {
                 const TileInfo ti = decode_tile(P, gt, tile, t0);
                 const TcProblem& p = P.p[ti.prob];
@@ -419,6 +445,7 @@ __global__ void __launch_bounds__(TcShape<GATEUP, BN, STAGES, Q4>::THREADS, 1)
                 }
                 tc_fence_after();
                 const uint32_t d0 = tmem_base + ab * S::ACC_COLS;
+                const uint32_t idesc = (Q4 && p.q4 && !p.mx) ? idesc_h : idesc_b;
                 const int nk = p.K / kBK;
                 for (int kb = 0; kb < nk; ++kb) {
                     // 4-bit: the operand slot is complete once the dequantising warps have
@@ -536,9 +563,11 @@ __global__ void __launch_bounds__(TcShape<GATEUP, BN, STAGES, Q4>::THREADS, 1)
                             const uint32_t sbyte = __ldg(sp[ai] + g);
                             const __nv_bfloat16 sc = __ushort_as_bfloat16(uint16_t(sbyte ? (sbyte << 7) : 0x0040u));
                             o[ai][h] = __halves2bfloat162(sc, sc);
-                        } else {
-                            o[ai][h] = __halves2bfloat162(__ldg(reinterpret_cast<const __nv_bfloat16*>(sp[ai]) + g),
-                                                          __ldg(reinterpret_cast<const __nv_bfloat16*>(zp[ai]) + g));
+                        } else {  // (scale, bias) as an fp16 pair, kept in the same 32-bit register
+                            const __half2 sz = __floats2half2_rn(
+                                __bfloat162float(__ldg(reinterpret_cast<const __nv_bfloat16*>(sp[ai]) + g)),
+                                __bfloat162float(__ldg(reinterpret_cast<const __nv_bfloat16*>(zp[ai]) + g)));
+                            o[ai][h] = *reinterpret_cast<const __nv_bfloat162*>(&sz);
                         }
                     }
             };
@@ -565,8 +594,12 @@ __global__ void __launch_bounds__(TcShape<GATEUP, BN, STAGES, Q4>::THREADS, 1)
                     for (int c = 0; c < 8; ++c) {
                         const __nv_bfloat162 sbv = q0[ai][c >> 2];
                         uint4 v;
-                        if constexpr (MX) v = dequant8_mx(words[c], sbv);
-                        else v = dequant8(words[c], __low2bfloat162(sbv), __high2bfloat162(sbv));
+                        if constexpr (MX) {
+                            v = dequant8_mx(words[c], sbv);
+                        } else {
+                            const __half2 sz = *reinterpret_cast<const __half2*>(&sbv);
+                            v = dequant8_f16(words[c], __low2half2(sz), __high2half2(sz));
+                        }
                         *reinterpret_cast<uint4*>(ob + a * S::A_BYTES + sw128_offset(drow, c)) = v;
                     }
                 }
@@ -677,9 +710,15 @@ __global__ void __launch_bounds__(TcShape<GATEUP, BN, STAGES, Q4>::THREADS, 1)
                             gg0 += bg[j]; gg1 += bg[j + 1];
                             uu0 += bu[j]; uu1 += bu[j + 1];
                         }
-                        __nv_bfloat162 v2 = __floats2bfloat162_rn(act_fast(P.act, gg0, uu0, P.limit, P.alpha),
-                                                                  act_fast(P.act, gg1, uu1, P.limit, P.alpha));
-                        hp[j / 2] = *reinterpret_cast<uint32_t*>(&v2);
+                        const float a0 = act_fast(P.act, gg0, uu0, P.limit, P.alpha);
+                        const float a1 = act_fast(P.act, gg1, uu1, P.limit, P.alpha);
+                        if (p.out_f16) {
+                            __half2 v2 = __floats2half2_rn(a0, a1);
+                            hp[j / 2] = *reinterpret_cast<uint32_t*>(&v2);
+                        } else {
+                            __nv_bfloat162 v2 = __floats2bfloat162_rn(a0, a1);
+                            hp[j / 2] = *reinterpret_cast<uint32_t*>(&v2);
+                        }
                     }
                     uint4* dst = reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(p.out) + prow * p.ld_out + ub);
 #pragma unroll
@@ -840,6 +879,14 @@ bool tc_token_map(CUtensorMap* m, const void* u, int64_t rows, int K, int bn) {
         if (!encode(&m[v], u, 2, dims, strides, box)) return false;
     }
     return true;
+}
+
+// Token operand [rows, K] bf16 for TMA row gather: box of one 64-wide K block x one row.
+bool tc_gather_map(CUtensorMap* m, const void* u, int64_t rows, int K) {
+    const cuuint64_t dims[2] = {cuuint64_t(K), cuuint64_t(rows)};
+    const cuuint64_t strides[1] = {cuuint64_t(K) * 2};
+    const cuuint32_t box[2] = {kBK, 1};
+    return encode(m, u, 2, dims, strides, box);
 }
 
 // Packed 4-bit plane [E, R, K / 8] uint32 (K % 64 == 0): box of 8 words x 128 rows. With
