@@ -38,10 +38,10 @@ struct QRow {  // 4-bit companions of one row
 
 // acc[r][t] += sum_c W_r[c] * u_t[c] for NR rows and tt (<= kTT) staged tokens; u_t is row
 // t of `us` (rows of K values), or row tl[t] when a token list is given.
-template <int WF, int NR>
+template <int WF, int NR, int TT = kTT>
 __device__ __forceinline__ void dot_rows(const char* const (&rows)[NR], const QRow (&q)[NR], int K,
                                          int group_size, const typename Fmt<WF>::AT* us,
-                                         const float* xsum, int tt, float (&acc)[NR][kTT],
+                                         const float* xsum, int tt, float (&acc)[NR][TT],
                                          const int* tl = nullptr) {
     using F = Fmt<WF>;
     using AT = typename F::AT;
@@ -66,7 +66,7 @@ __device__ __forceinline__ void dot_rows(const char* const (&rows)[NR], const QR
 #pragma unroll
                 for (int r = 0; r < NR; ++r) unpack8(wv[r][u], wf[r]);
 #pragma unroll
-                for (int t = 0; t < kTT; ++t) {
+                for (int t = 0; t < TT; ++t) {
                     if (t >= tt) break;
                     float xf[8];
                     unpack8(*reinterpret_cast<const uint4*>(us + int64_t(tl ? tl[t] : t) * K + c0), xf);
@@ -77,7 +77,7 @@ __device__ __forceinline__ void dot_rows(const char* const (&rows)[NR], const QR
                 }
             } else if constexpr (WF == kF32) {
 #pragma unroll
-                for (int t = 0; t < kTT; ++t) {
+                for (int t = 0; t < TT; ++t) {
                     if (t >= tt) break;
                     const float4 xv = *reinterpret_cast<const float4*>(us + int64_t(tl ? tl[t] : t) * K + c0);
 #pragma unroll
@@ -100,7 +100,7 @@ __device__ __forceinline__ void dot_rows(const char* const (&rows)[NR], const QR
                         for (int n = 0; n < 8; ++n) qf[r][i * 8 + n] = e2m1_value(words[i] >> (4 * n));
                 }
 #pragma unroll
-                for (int t = 0; t < kTT; ++t) {
+                for (int t = 0; t < TT; ++t) {
                     if (t >= tt) break;
                     float dq[NR];
 #pragma unroll
@@ -120,11 +120,11 @@ __device__ __forceinline__ void dot_rows(const char* const (&rows)[NR], const QR
             } else {  // 4-bit affine: sum_j (s q_j + b) x_j = s * sum_j q_j x_j + b * sum_j x_j
                 // Decoded one 32-bit word (8 codes) at a time, so that only 8 codes per row are
                 // live beside the per-token partial sums (fewer registers, more resident warps).
-                float dq[NR][kTT];
+                float dq[NR][TT];
 #pragma unroll
                 for (int r = 0; r < NR; ++r)
 #pragma unroll
-                    for (int t = 0; t < kTT; ++t) dq[r][t] = 0.f;
+                    for (int t = 0; t < TT; ++t) dq[r][t] = 0.f;
 #pragma unroll
                 for (int i = 0; i < 4; ++i) {
                     float qf[NR][8];
@@ -136,7 +136,7 @@ __device__ __forceinline__ void dot_rows(const char* const (&rows)[NR], const QR
                             qf[r][n] = __uint_as_float(0x4B000000u | ((word >> (4 * n)) & 0xFu)) - 8388608.0f;
                     }
 #pragma unroll
-                    for (int t = 0; t < kTT; ++t) {
+                    for (int t = 0; t < TT; ++t) {
                         if (t >= tt) break;
                         float xf[8];
                         unpack8(*reinterpret_cast<const uint4*>(us + int64_t(tl ? tl[t] : t) * K + c0 + 8 * i), xf);
@@ -152,7 +152,7 @@ __device__ __forceinline__ void dot_rows(const char* const (&rows)[NR], const QR
                     const float sc = __bfloat162float(q[r].s[grp]);
                     const float bi = __bfloat162float(q[r].z[grp]);
 #pragma unroll
-                    for (int t = 0; t < kTT; ++t) {
+                    for (int t = 0; t < TT; ++t) {
                         if (t >= tt) break;
                         acc[r][t] = fmaf(sc, dq[r][t], fmaf(bi, xsum[(tl ? tl[t] : t) * (K / 32) + v], acc[r][t]));
                     }
