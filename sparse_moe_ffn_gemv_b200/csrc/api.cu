@@ -51,10 +51,10 @@ WsLayout ws_layout(const moe_config& c, int64_t T) {
     L.z = take(Ld ? T * Ld * ab : 0);
     L.nrm = take(Ld ? T * Ld * ab : 0);
     L.tiles = take((E + 1) * 4);
-    // fp16 copies of the token operands of 4-bit affine problems on the tensor cores
-    const bool aff = c.weight_format == MOE_DTYPE_Q4_AFFINE, dq = c.dense_format == MOE_DTYPE_Q4_AFFINE;
-    L.x16 = take((aff && !Ld) || dq ? T * H * 2 : 0);
-    L.z16 = take(Ld && aff ? T * Ld * 2 : 0);
+    L.uperm = take(c.act_dtype == MOE_DTYPE_BF16 ? T * k * K * 2 : 0);
+    // fp16 copies of the dense token operands of 4-bit dense planes on the tensor cores
+    const bool dq = c.dense_format == MOE_DTYPE_Q4_AFFINE;
+    L.x16 = take(dq ? T * H * 2 : 0);
     L.n16 = take(Ld && dq ? T * Ld * 2 : 0);
     L.total = off;
     return L;
@@ -461,12 +461,13 @@ moe_status run_experts_tc(const moe_config* c, const moe_weights* w, const void*
     // 4-bit affine problems run on fp16 operands: fp16 copies of their token inputs
     const bool aff = rtc && c->weight_format == MOE_DTYPE_Q4_AFFINE, dq = stc && dense_q4(c);
     void* x16 = at<void>(ws, L.x16);
-    void* u16 = c->latent_dim ? at<void>(ws, L.z16) : x16;
-    if (aff) MOE_CUDA(launch_to_f16(u, T * K, u16, s));
-    if (dq && !(aff && !c->latent_dim)) MOE_CUDA(launch_to_f16(x, T * H, x16, s));
     const int Is = c->shared_intermediate;
     const int64_t S = T * k;
     const int64_t n_dense = (T + kTcBN - 1) / kTcBN;
+    void* uperm = at<void>(ws, L.uperm);
+    // the routed token rows in sorted order (fp16 for 4-bit affine weights)
+    if (rtc) MOE_CUDA(launch_gather_rows(u, K, sorted_slot, k, S, uperm, s, goff, goff + E, aff));
+    if (dq) MOE_CUDA(launch_to_f16(x, T * H, x16, s));
     void* h = at<void>(ws, L.h);
     void* hs = at<void>(ws, L.hs);
     const int32_t* tiles = at<int32_t>(ws, L.tiles);
@@ -535,11 +536,8 @@ moe_status run_experts_tc(const moe_config* c, const moe_weights* w, const void*
                 ok = tc_weight_map(&P.a0[np], w->gate_w, E, I, K, false) &&
                      tc_weight_map(&P.a1[np], w->up_w, E, I, K, false);
             }
-            // the tile's token rows are gathered from u by slot (TMA row gather, no copy)
-            p.gather_k = k;
-            p.sorted_slot = sorted_slot;
             p.out_f16 = aff ? 1 : 0;  // fp16 h for the fp16 routed down GEMM
-            if (!ok || !tc_gather_map(&P.b[np][0], aff ? u16 : u, T, K)) return MOE_ERR_CUDA;
+            if (!ok || !tc_token_map(P.b[np], uperm, S, K, kTcBN)) return MOE_ERR_CUDA;
             max_tiles += int64_t(p.m_blocks) * max_routed_tiles(*c, T);
             ++np;
         }

@@ -43,8 +43,8 @@ struct WsLayout {
     size_t z;            // act [T, L]: latent input of the experts
     size_t nrm;          // act [T, L]: normalised latent
     size_t tiles;        // int32 tile list of the tensor-core path
-    size_t x16;          // fp16 [T, H]: x as the fp16 token operand (4-bit affine weights)
-    size_t z16;          // fp16 [T, L]: the latent expert input likewise
+    size_t uperm;        // [T * k, K]: routed token rows in sorted order (fp16 for 4-bit affine)
+    size_t x16;          // fp16 [T, H]: x as the fp16 token operand (4-bit dense planes)
     size_t n16;          // fp16 [T, L]: the normalised latent likewise
     size_t total;
     int ld_logits;

@@ -76,87 +76,127 @@ __device__ __forceinline__ void copy_cg(uint4* dst, const void* src, int64_t n16
     for (int64_t i = threadIdx.x; i < n16; i += blockDim.x) dst[i] = __ldcg(s + i);
 }
 
-template <int WF>
+// Rows per warp item. With one token the accumulators are few, so a warp keeps several rows
+// (two gate/up units, four down rows) in flight; with up to 8 tokens one unit / two rows.
+template <int WF, int TT> struct DecShape {
+    static constexpr bool ONE = TT == 1;
+    static constexpr int RR = ONE ? 4 : 1;                          // router rows
+    static constexpr int SU = ONE ? 2 : 1;                          // shared gate/up units
+    static constexpr int BU = (ONE && WF == kBF16) ? 2 : 1;         // routed gate/up units
+    static constexpr int DN = (ONE && WF == kBF16) ? 4 : 2;         // routed down rows
+    static constexpr int SN = ONE ? 4 : 2;                          // shared down rows
+};
+
+// acc[r][t] = sum over the row of W_r . u_t, reduced over the warp (every lane holds it).
+template <int WF, int NR, int TT>
+__device__ __forceinline__ void dot_reduce(const char* const (&rows)[NR], const QRow (&q)[NR], int K, int gs,
+                                           const __nv_bfloat16* us, const float* usum, int tt, float (&acc)[NR][TT],
+                                           const int* tl = nullptr) {
+#pragma unroll
+    for (int r = 0; r < NR; ++r)
+#pragma unroll
+        for (int t = 0; t < TT; ++t) acc[r][t] = 0.f;
+    dot_rows<WF, NR, TT>(rows, q, K, gs, us, usum, tt, acc, tl);
+#pragma unroll
+    for (int r = 0; r < NR; ++r)
+#pragma unroll
+        for (int t = 0; t < TT; ++t) {
+            if (t >= tt) break;
+            acc[r][t] = warp_sum(acc[r][t]);
+        }
+}
+
+template <int WF, int TT>
 __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(const DecodeArgs a) {
     using AT = __nv_bfloat16;
-    constexpr int DN = 2;  // down rows per warp item (one expert)
+    using Sh = DecShape<WF, TT>;
+    constexpr int DN = Sh::DN, SN = Sh::SN, RR = Sh::RR, SU = Sh::SU, BU = Sh::BU;
     extern __shared__ uint4 dsm[];
     __shared__ DecSmem sm;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int T = a.T, H = a.H, k = a.k, I = a.I, Is = a.Is, S = T * k;
+    const int T = a.T, H = a.H, k = a.k, I = a.I, Is = a.Is, S = T * k, E = a.E;
     const int gw = blockIdx.x * kDecWarps + warp, nw = gridDim.x * kDecWarps;
     const uint64_t deadline = gtimer() + kDecWaitNs;
     const int RB = (H + gridDim.x - 1) / gridDim.x;  // output rows per block
     const int r0 = min(H, int(blockIdx.x) * RB), r1 = min(H, r0 + RB), nr = r1 - r0;
     const bool blend = a.shared_mode == MOE_SHARED_BLEND;
     const int64_t drb = row_bytes<WF>(I);  // bytes of one routed down row
+    const int dg = a.dense_group;
+    const bool dq = a.dense_q4 != 0;
+    const int64_t dhb = dq ? H / 2 : int64_t(H) * 2;   // bytes of a router / shared gate/up row
+    const int64_t srb = dq ? Is / 2 : int64_t(Is) * 2;  // bytes of one shared down row
+    auto dense_q = [&](const void* sc, const void* bi, int64_t row, int cols) -> QRow {
+        if (!dq) return QRow{nullptr, nullptr, nullptr};
+        const int64_t ng = cols / dg;
+        return QRow{static_cast<const __nv_bfloat16*>(sc) + row * ng, static_cast<const __nv_bfloat16*>(bi) + row * ng,
+                    nullptr};
+    };
 
     // ------------------------------------------------------------ phase A
     AT* xs = reinterpret_cast<AT*>(dsm);
     float* xsum = reinterpret_cast<float*>(xs + int64_t(T) * H);  // 4-bit affine: sums per 32
-    if (WF == kQ4 || a.dense_q4) stage_tokens<kQ4>(a.x, H, 0, T, nullptr, 1, xs, xsum);
+    if (WF == kQ4 || dq) stage_tokens<kQ4>(a.x, H, 0, T, nullptr, 1, xs, xsum);
     else stage_tokens<kBF16>(a.x, H, 0, T, nullptr, 1, xs, nullptr);
-    const int dg = a.dense_group;
-    const int64_t srb = a.dense_q4 ? Is / 2 : int64_t(Is) * 2;  // bytes of one shared down row
     if (a.l2_prefetch && Is && threadIdx.x == 0 && nr > 0)
         l2_prefetch(static_cast<const char*>(a.sd_w) + int64_t(r0) * srb, size_t(nr) * srb);
     __syncthreads();
-    const int nrouter = a.E + (blend ? 2 : 0);
-    for (int it = gw; it < nrouter + Is; it += nw) {
-        if (it < nrouter) {  // one router / coefficient row -> fp32 logits of every token
-            const bool cr = it >= a.E;
-            const int rr = cr ? it - a.E : it;
-            float acc[1][kTT];
+    {
+        const int n_rg = (E + RR - 1) / RR;           // router row groups
+        const int n_cf = blend ? 2 : 0;                // coefficient rows (bf16)
+        const int n_sh = Is ? (Is + SU - 1) / SU : 0;  // shared gate/up unit groups
+        for (int it = gw; it < n_rg + n_cf + n_sh; it += nw) {
+            if (it < n_rg) {  // RR router rows -> fp32 logits of every token
+                const char* rows[RR];
+                QRow q[RR];
 #pragma unroll
-            for (int t = 0; t < kTT; ++t) acc[0][t] = 0.f;
-            if (a.dense_q4 && !cr) {  // 4-bit router row (the blend head stays bf16)
-                const int64_t ng = H / dg;
-                const char* rows[1] = {static_cast<const char*>(a.router_w) + int64_t(rr) * (H / 2)};
-                const QRow q[1] = {{static_cast<const __nv_bfloat16*>(a.router_s) + rr * ng,
-                                    static_cast<const __nv_bfloat16*>(a.router_z) + rr * ng, nullptr}};
-                dot_rows<kQ4, 1>(rows, q, H, dg, xs, xsum, T, acc);
-            } else {
-                const char* rows[1] = {static_cast<const char*>(cr ? a.coef_w : a.router_w) + int64_t(rr) * H * 2};
+                for (int j = 0; j < RR; ++j) {
+                    const int e = min(it * RR + j, E - 1);
+                    rows[j] = static_cast<const char*>(a.router_w) + int64_t(e) * dhb;
+                    q[j] = dense_q(a.router_s, a.router_z, e, H);
+                }
+                float acc[RR][TT];
+                if (dq) dot_reduce<kQ4, RR, TT>(rows, q, H, dg, xs, xsum, T, acc);
+                else dot_reduce<kBF16, RR, TT>(rows, q, H, 64, xs, nullptr, T, acc);
+#pragma unroll
+                for (int j = 0; j < RR; ++j) {
+                    const int e = it * RR + j;
+                    const float b = a.router_b ? bf16_ld(a.router_b, min(e, E - 1)) : 0.f;
+#pragma unroll
+                    for (int t = 0; t < TT; ++t)
+                        if (t < T && e < E && lane == t) a.logits[int64_t(t) * a.ld_logits + e] = acc[j][t] + b;
+                }
+            } else if (it < n_rg + n_cf) {  // one coefficient-head row (bf16)
+                const int c = it - n_rg;
+                const char* rows[1] = {static_cast<const char*>(a.coef_w) + int64_t(c) * H * 2};
                 const QRow q[1] = {{nullptr, nullptr, nullptr}};
-                dot_rows<kBF16, 1>(rows, q, H, 64, xs, nullptr, T, acc);
-            }
-            const void* bp = cr ? a.coef_b : a.router_b;
-            const float b = bp ? bf16_ld(bp, rr) : 0.f;
+                float acc[1][TT];
+                dot_reduce<kBF16, 1, TT>(rows, q, H, 64, xs, nullptr, T, acc);
+                const float b = bf16_ld(a.coef_b, c);
 #pragma unroll
-            for (int t = 0; t < kTT; ++t) {
-                if (t >= T) break;
-                const float v = warp_sum(acc[0][t]);
-                if (lane == t) a.logits[int64_t(t) * a.ld_logits + it] = v + b;
-            }
-        } else {  // one shared gate/up unit
-            const int i = it - nrouter;
-            float acc[2][kTT];
+                for (int t = 0; t < TT; ++t)
+                    if (t < T && lane == t) a.logits[int64_t(t) * a.ld_logits + E + c] = acc[0][t] + b;
+            } else {  // SU shared gate/up units
+                const int i0 = (it - n_rg - n_cf) * SU;
+                const char* rows[2 * SU];
+                QRow q[2 * SU];
 #pragma unroll
-            for (int r = 0; r < 2; ++r)
+                for (int j = 0; j < SU; ++j) {
+                    const int i = min(i0 + j, Is - 1);
+                    rows[j] = static_cast<const char*>(a.sg_w) + int64_t(i) * dhb;
+                    rows[SU + j] = static_cast<const char*>(a.su_w) + int64_t(i) * dhb;
+                    q[j] = dense_q(a.sg_s, a.sg_z, i, H);
+                    q[SU + j] = dense_q(a.su_s, a.su_z, i, H);
+                }
+                float acc[2 * SU][TT];
+                if (dq) dot_reduce<kQ4, 2 * SU, TT>(rows, q, H, dg, xs, xsum, T, acc);
+                else dot_reduce<kBF16, 2 * SU, TT>(rows, q, H, 64, xs, nullptr, T, acc);
 #pragma unroll
-                for (int t = 0; t < kTT; ++t) acc[r][t] = 0.f;
-            if (a.dense_q4) {
-                const int64_t ng = H / dg;
-                const char* rows[2] = {static_cast<const char*>(a.sg_w) + int64_t(i) * (H / 2),
-                                       static_cast<const char*>(a.su_w) + int64_t(i) * (H / 2)};
-                const QRow q[2] = {{static_cast<const __nv_bfloat16*>(a.sg_s) + i * ng,
-                                    static_cast<const __nv_bfloat16*>(a.sg_z) + i * ng, nullptr},
-                                   {static_cast<const __nv_bfloat16*>(a.su_s) + i * ng,
-                                    static_cast<const __nv_bfloat16*>(a.su_z) + i * ng, nullptr}};
-                dot_rows<kQ4, 2>(rows, q, H, dg, xs, xsum, T, acc);
-            } else {
-                const char* rows[2] = {static_cast<const char*>(a.sg_w) + int64_t(i) * H * 2,
-                                       static_cast<const char*>(a.su_w) + int64_t(i) * H * 2};
-                const QRow q[2] = {{nullptr, nullptr, nullptr}, {nullptr, nullptr, nullptr}};
-                dot_rows<kBF16, 2>(rows, q, H, 64, xs, nullptr, T, acc);
-            }
+                for (int j = 0; j < SU; ++j)
 #pragma unroll
-            for (int t = 0; t < kTT; ++t) {
-                if (t >= T) break;
-                const float g = warp_sum(acc[0][t]), u = warp_sum(acc[1][t]);
-                if (lane == t)
-                    reinterpret_cast<AT*>(a.hs)[int64_t(t) * Is + i] =
-                        __float2bfloat16_rn(act_apply(a.act, g, u, a.limit, a.alpha));
+                    for (int t = 0; t < TT; ++t)
+                        if (t < T && i0 + j < Is && lane == t)
+                            reinterpret_cast<AT*>(a.hs)[int64_t(t) * Is + i0 + j] = __float2bfloat16_rn(
+                                act_apply(a.act, acc[j][t], acc[SU + j][t], a.limit, a.alpha));
             }
         }
     }
@@ -166,7 +206,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(const DecodeArgs
     if (ok) {
         if (warp < T) {  // top-k of token `warp`, identical in every block
             TopkArgs ta;
-            ta.logits = a.logits; ta.ld = a.ld_logits; ta.T = T; ta.E = a.E; ta.k = k;
+            ta.logits = a.logits; ta.ld = a.ld_logits; ta.T = T; ta.E = E; ta.k = k;
             ta.scoring = a.scoring; ta.norm = a.norm; ta.has_sel = a.has_sel; ta.sel_bias = a.sel_bias;
             ta.blend = blend ? 1 : 0;
             ta.idx = sm.sidx; ta.w = sm.sw; ta.coef = sm.scoef;
@@ -205,66 +245,68 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(const DecodeArgs
             for (int d = threadIdx.x; d < n_d; d += blockDim.x)
                 l2_prefetch(static_cast<const char*>(a.down_w) + (int64_t(sm.dexp[d]) * H + r0) * drb,
                             size_t(nr) * drb);
-        // routed gate/up: one unit (gate row + up row) of one distinct expert per warp item
-        for (int it = gw; it < n_d * I; it += nw) {
-            const int d = it / I, i = it - d * I;
+        // routed gate/up: BU units (gate + up rows) of one distinct expert per warp item
+        const int ub = (I + BU - 1) / BU;
+        const int64_t rbh = row_bytes<WF>(H);
+        for (int it = gw; it < n_d * ub; it += nw) {
+            const int d = it / ub, i0 = (it - d * ub) * BU;
             const int ex = sm.dexp[d];
             const int sb = sm.doff[d], cnt = sm.doff[d + 1] - sb;
-            int tl[kTT];
+            int tl[TT];
 #pragma unroll
-            for (int j = 0; j < kTT; ++j) tl[j] = j < cnt ? sm.sorted[sb + j] / k : 0;
-            const int64_t rb = row_bytes<WF>(H);
-            const char* rows[2];
-            QRow q[2] = {{nullptr, nullptr, nullptr}, {nullptr, nullptr, nullptr}};
-            int64_t g0, g1;  // plane rows of the gate and the up weights
-            if (a.interleaved) {
-                g0 = int64_t(ex) * 2 * I + 2 * i;
-                g1 = g0 + 1;
-                rows[0] = static_cast<const char*>(a.gate_up_w) + g0 * rb;
-                rows[1] = rows[0] + rb;
-            } else {
-                g0 = g1 = int64_t(ex) * I + i;
-                rows[0] = static_cast<const char*>(a.gate_w) + g0 * rb;
-                rows[1] = static_cast<const char*>(a.up_w) + g1 * rb;
-            }
-            if constexpr (WF == kQ4) {
-                const int64_t ng = H / a.group_size;
-                const __nv_bfloat16* s0 = static_cast<const __nv_bfloat16*>(a.gate_s);
-                const __nv_bfloat16* z0 = static_cast<const __nv_bfloat16*>(a.gate_z);
-                const __nv_bfloat16* s1 = static_cast<const __nv_bfloat16*>(a.interleaved ? a.gate_s : a.up_s);
-                const __nv_bfloat16* z1 = static_cast<const __nv_bfloat16*>(a.interleaved ? a.gate_z : a.up_z);
-                q[0] = {s0 + g0 * ng, z0 + g0 * ng, nullptr};
-                q[1] = {s1 + g1 * ng, z1 + g1 * ng, nullptr};
-            } else if constexpr (WF == kMX4) {
-                const uint8_t* s0 = static_cast<const uint8_t*>(a.gate_s);
-                const uint8_t* s1 = static_cast<const uint8_t*>(a.interleaved ? a.gate_s : a.up_s);
-                q[0] = {nullptr, nullptr, s0 + g0 * (H / 32)};
-                q[1] = {nullptr, nullptr, s1 + g1 * (H / 32)};
-            }
-            float bg = 0.f, bu = 0.f;
-            if (a.has_bias) {
+            for (int j = 0; j < TT; ++j) tl[j] = j < cnt ? sm.sorted[sb + j] / k : 0;
+            const char* rows[2 * BU];
+            QRow q[2 * BU];
+            float bg[BU], bu[BU];
+#pragma unroll
+            for (int j = 0; j < BU; ++j) {
+                const int i = min(i0 + j, I - 1);
+                int64_t g0, g1;  // plane rows of the gate and the up weights
                 if (a.interleaved) {
-                    bg = bf16_ld(a.gate_up_b, int64_t(ex) * 2 * I + 2 * i);
-                    bu = bf16_ld(a.gate_up_b, int64_t(ex) * 2 * I + 2 * i + 1);
+                    g0 = int64_t(ex) * 2 * I + 2 * i;
+                    g1 = g0 + 1;
+                    rows[j] = static_cast<const char*>(a.gate_up_w) + g0 * rbh;
+                    rows[BU + j] = rows[j] + rbh;
                 } else {
-                    bg = bf16_ld(a.gate_b, int64_t(ex) * I + i);
-                    bu = bf16_ld(a.up_b, int64_t(ex) * I + i);
+                    g0 = g1 = int64_t(ex) * I + i;
+                    rows[j] = static_cast<const char*>(a.gate_w) + g0 * rbh;
+                    rows[BU + j] = static_cast<const char*>(a.up_w) + g1 * rbh;
+                }
+                q[j] = q[BU + j] = QRow{nullptr, nullptr, nullptr};
+                if constexpr (WF == kQ4) {
+                    const int64_t ng = H / a.group_size;
+                    const __nv_bfloat16* s0 = static_cast<const __nv_bfloat16*>(a.gate_s);
+                    const __nv_bfloat16* z0 = static_cast<const __nv_bfloat16*>(a.gate_z);
+                    const __nv_bfloat16* s1 = static_cast<const __nv_bfloat16*>(a.interleaved ? a.gate_s : a.up_s);
+                    const __nv_bfloat16* z1 = static_cast<const __nv_bfloat16*>(a.interleaved ? a.gate_z : a.up_z);
+                    q[j] = {s0 + g0 * ng, z0 + g0 * ng, nullptr};
+                    q[BU + j] = {s1 + g1 * ng, z1 + g1 * ng, nullptr};
+                } else if constexpr (WF == kMX4) {
+                    const uint8_t* s0 = static_cast<const uint8_t*>(a.gate_s);
+                    const uint8_t* s1 = static_cast<const uint8_t*>(a.interleaved ? a.gate_s : a.up_s);
+                    q[j] = {nullptr, nullptr, s0 + g0 * (H / 32)};
+                    q[BU + j] = {nullptr, nullptr, s1 + g1 * (H / 32)};
+                }
+                bg[j] = bu[j] = 0.f;
+                if (a.has_bias) {
+                    if (a.interleaved) {
+                        bg[j] = bf16_ld(a.gate_up_b, int64_t(ex) * 2 * I + 2 * i);
+                        bu[j] = bf16_ld(a.gate_up_b, int64_t(ex) * 2 * I + 2 * i + 1);
+                    } else {
+                        bg[j] = bf16_ld(a.gate_b, int64_t(ex) * I + i);
+                        bu[j] = bf16_ld(a.up_b, int64_t(ex) * I + i);
+                    }
                 }
             }
-            float acc[2][kTT];
+            float acc[2 * BU][TT];
+            dot_reduce<WF, 2 * BU, TT>(rows, q, H, a.group_size, xs, xsum, cnt, acc, tl);
 #pragma unroll
-            for (int r = 0; r < 2; ++r)
+            for (int j = 0; j < BU; ++j)
 #pragma unroll
-                for (int t = 0; t < kTT; ++t) acc[r][t] = 0.f;
-            dot_rows<WF, 2>(rows, q, H, a.group_size, xs, xsum, cnt, acc, tl);
-#pragma unroll
-            for (int j = 0; j < kTT; ++j) {
-                if (j >= cnt) break;
-                const float g = warp_sum(acc[0][j]), u = warp_sum(acc[1][j]);
-                if (lane == j)
-                    reinterpret_cast<AT*>(a.h)[int64_t(sm.sorted[sb + j]) * I + i] =
-                        __float2bfloat16_rn(act_apply(a.act, g + bg, u + bu, a.limit, a.alpha));
-            }
+                for (int t = 0; t < TT; ++t)
+                    if (t < cnt && i0 + j < I && lane == t)
+                        reinterpret_cast<AT*>(a.h)[int64_t(sm.sorted[sb + t]) * I + i0 + j] = __float2bfloat16_rn(
+                            act_apply(a.act, acc[j][t] + bg[j], acc[BU + j][t] + bu[j], a.limit, a.alpha));
         }
         ok = grid_barrier(&a.bar[1], gridDim.x, deadline, a.status, &sm.flag);
     }
@@ -283,10 +325,10 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(const DecodeArgs
             sm.acc_s[i / kTT][i % kTT] = 0.f;
         }
         __syncthreads();
-        if (a.dense_q4 && Is) {
-            const int nv = Is / 32;
-            for (int i = threadIdx.x; i < T * nv; i += blockDim.x) {
-                const uint4* p = reinterpret_cast<const uint4*>(hss + int64_t(i / nv) * Is + (i % nv) * 32);
+        auto sums32 = [&](const AT* rowsrc, int nrows, int cols, float* dst) {  // per-32 sums of rows
+            const int nv = cols / 32;
+            for (int i = threadIdx.x; i < nrows * nv; i += blockDim.x) {
+                const uint4* p = reinterpret_cast<const uint4*>(rowsrc + int64_t(i / nv) * cols + (i % nv) * 32);
                 float sum = 0.f;
 #pragma unroll
                 for (int j = 0; j < 4; ++j) {
@@ -295,36 +337,22 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(const DecodeArgs
 #pragma unroll
                     for (int n = 0; n < 8; ++n) sum += f[n];
                 }
-                hssum[i] = sum;
+                dst[i] = sum;
             }
-            if (WF != kQ4) __syncthreads();
-        }
-        if constexpr (WF == kQ4) {
-            const int nv = I / 32;
-            for (int i = threadIdx.x; i < S * nv; i += blockDim.x) {
-                const uint4* p = reinterpret_cast<const uint4*>(hsm + int64_t(i / nv) * I + (i % nv) * 32);
-                float sum = 0.f;
-#pragma unroll
-                for (int j = 0; j < 4; ++j) {
-                    float f[8];
-                    unpack8(p[j], f);
-#pragma unroll
-                    for (int n = 0; n < 8; ++n) sum += f[n];
-                }
-                hsum[i] = sum;
-            }
-            __syncthreads();
-        }
-        const int nq = (nr + DN - 1) / DN;
-        const int n_items = n_d * nq + (Is ? nq : 0);
+        };
+        if (dq && Is) sums32(hss, T, Is, hssum);
+        if (WF == kQ4) sums32(hsm, S, I, hsum);
+        if (WF == kQ4 || (dq && Is)) __syncthreads();
+        const int nq = (nr + DN - 1) / DN, nsq = (nr + SN - 1) / SN;
+        const int n_items = n_d * nq + (Is ? nsq : 0);
         for (int it = warp; it < n_items; it += kDecWarps) {
             if (it < n_d * nq) {  // DN down rows of one distinct expert
                 const int d = it / nq, qq = it - d * nq;
                 const int ex = sm.dexp[d];
                 const int sb = sm.doff[d], cnt = sm.doff[d + 1] - sb;
-                int tl[kTT];
+                int tl[TT];
 #pragma unroll
-                for (int j = 0; j < kTT; ++j) tl[j] = j < cnt ? sm.sorted[sb + j] : 0;  // slot rows of hsm
+                for (int j = 0; j < TT; ++j) tl[j] = j < cnt ? sm.sorted[sb + j] : 0;  // slot rows of hsm
                 const char* rows[DN];
                 QRow q[DN];
                 float bd[DN];
@@ -343,52 +371,37 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(const DecodeArgs
                     }
                     bd[jr] = a.has_bias ? bf16_ld(a.down_b, gr) : 0.f;
                 }
-                float acc[DN][kTT];
+                float acc[DN][TT];
+                dot_reduce<WF, DN, TT>(rows, q, I, a.group_size, hsm, hsum, cnt, acc, tl);
 #pragma unroll
                 for (int jr = 0; jr < DN; ++jr)
 #pragma unroll
-                    for (int t = 0; t < kTT; ++t) acc[jr][t] = 0.f;
-                dot_rows<WF, DN>(rows, q, I, a.group_size, hsm, hsum, cnt, acc, tl);
-#pragma unroll
-                for (int jr = 0; jr < DN; ++jr)
-#pragma unroll
-                    for (int j = 0; j < kTT; ++j) {
-                        if (j >= cnt) break;
-                        const float v = warp_sum(acc[jr][j]);
+                    for (int j = 0; j < TT; ++j) {
                         const int rl = qq * DN + jr;
-                        if (lane == 0 && rl < nr) {
+                        if (j < cnt && lane == 0 && rl < nr) {
                             const int slot = tl[j];
-                            atomicAdd(&sm.acc_r[rl][slot / k], sm.sw[slot] * (v + bd[jr]));
+                            atomicAdd(&sm.acc_r[rl][slot / k], sm.sw[slot] * (acc[jr][j] + bd[jr]));
                         }
                     }
-            } else {  // DN rows of the shared expert's down projection, every token
+            } else {  // SN rows of the shared expert's down projection, every token
                 const int qq = it - n_d * nq;
-                const char* rows[DN];
-                QRow q[DN];
+                const char* rows[SN];
+                QRow q[SN];
 #pragma unroll
-                for (int jr = 0; jr < DN; ++jr) {
-                    const int64_t r = min(r0 + qq * DN + jr, r1 - 1);
+                for (int jr = 0; jr < SN; ++jr) {
+                    const int64_t r = min(r0 + qq * SN + jr, r1 - 1);
                     rows[jr] = static_cast<const char*>(a.sd_w) + r * srb;
-                    q[jr] = {nullptr, nullptr, nullptr};
-                    if (a.dense_q4)
-                        q[jr] = {static_cast<const __nv_bfloat16*>(a.sd_s) + r * (Is / dg),
-                                 static_cast<const __nv_bfloat16*>(a.sd_z) + r * (Is / dg), nullptr};
+                    q[jr] = dense_q(a.sd_s, a.sd_z, r, Is);
                 }
-                float acc[DN][kTT];
+                float acc[SN][TT];
+                if (dq) dot_reduce<kQ4, SN, TT>(rows, q, Is, dg, hss, hssum, T, acc);
+                else dot_reduce<kBF16, SN, TT>(rows, q, Is, 64, hss, nullptr, T, acc);
 #pragma unroll
-                for (int jr = 0; jr < DN; ++jr)
+                for (int jr = 0; jr < SN; ++jr)
 #pragma unroll
-                    for (int t = 0; t < kTT; ++t) acc[jr][t] = 0.f;
-                if (a.dense_q4) dot_rows<kQ4, DN>(rows, q, Is, dg, hss, hssum, T, acc);
-                else dot_rows<kBF16, DN>(rows, q, Is, 64, hss, nullptr, T, acc);
-#pragma unroll
-                for (int jr = 0; jr < DN; ++jr)
-#pragma unroll
-                    for (int t = 0; t < kTT; ++t) {
-                        if (t >= T) break;
-                        const float v = warp_sum(acc[jr][t]);
-                        const int rl = qq * DN + jr;
-                        if (lane == 0 && rl < nr) sm.acc_s[rl][t] = v;
+                    for (int t = 0; t < TT; ++t) {
+                        const int rl = qq * SN + jr;
+                        if (t < T && lane == 0 && rl < nr) sm.acc_s[rl][t] = acc[jr][t];
                     }
             }
         }
@@ -419,7 +432,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(const DecodeArgs
 
 template <int WF>
 cudaError_t launch_decode_t(const DecodeArgs& a, size_t smem, cudaStream_t s) {
-    auto kern = decode_kernel<WF>;
+    auto kern = a.T == 1 ? decode_kernel<WF, 1> : decode_kernel<WF, kTT>;
     cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
     if (err != cudaSuccess) return err;
     int dev = 0, sms = 0, per_sm = 0;

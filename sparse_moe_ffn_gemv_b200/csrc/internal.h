@@ -51,9 +51,11 @@ cudaError_t launch_permute(const PermuteArgs& a, cudaStream_t s);
 cudaError_t launch_active_list(const int32_t* offsets, int E, int32_t* active, cudaStream_t s);
 
 // dst[p, :] = src[sorted_slot[p] / k, :] for p < S (rows of K bf16): expert inputs in
-// sorted order for the tensor-core path; with lo / hi (device pointers) only *lo <= p < *hi.
+// sorted order for the tensor-core path; with lo / hi (device pointers) only *lo <= p < *hi;
+// to_f16: written as fp16.
 cudaError_t launch_gather_rows(const void* src, int K, const int32_t* sorted_slot, int k, int64_t S,
-                               void* dst, cudaStream_t s, const int32_t* lo = nullptr, const int32_t* hi = nullptr);
+                               void* dst, cudaStream_t s, const int32_t* lo = nullptr, const int32_t* hi = nullptr,
+                               bool to_f16 = false);
 // tile_start from offsets (moe_grouped_ffn called with a caller-made permutation).
 cudaError_t launch_tile_start(const int32_t* offsets, int E, int tile_bn, int32_t* tile_start, cudaStream_t s);
 
@@ -166,8 +168,6 @@ struct TcProblem {
     int mx = 0;  // with q4 = 1: MXFP4 codes, qs0 / qs1 the E8M0 scale bytes [groups, M, K / 32]
     int qrow_step = 1;  // companion rows per unit: 2 for an interleaved gate_up plane, whose
                         // up companions start one row after qs0 / qz0 (qs1 / qz1 = that row)
-    int gather_k = 0;   // > 0: token row i of a tile is row sorted_slot[row0 + i] / gather_k of the
-                        // token operand, fetched by TMA row gather (b[..][0] is the gather map)
     // 4-bit affine weights run the MMA on fp16 operands (the dequantised s * q + b rounds to
     // 11 significant bits; bf16 keeps 8): the token operand of such a problem is fp16, and
     // out_f16 makes a gate/up problem write its h in fp16 for the fp16 down GEMM after it.
@@ -199,8 +199,6 @@ bool tc_weight_map(CUtensorMap* m, const void* w, int E, int R, int K, bool inte
 bool tc_q4_weight_map(CUtensorMap* m, const void* w, int E, int R, int K, int row_step = 1);
 // Four maps m[0..3] of the token operand [rows, K] bf16, boxes of 16, 32, 64 and bn rows.
 bool tc_token_map(CUtensorMap* m, const void* u, int64_t rows, int K, int bn);
-// The token operand [rows, K] bf16 for TMA row gather: a box of one row x one K block.
-bool tc_gather_map(CUtensorMap* m, const void* u, int64_t rows, int K);
 // dst[i] = fp16(src[i]) for n bf16 values (exact within fp16's range), n % 8 == 0.
 cudaError_t launch_to_f16(const void* src, int64_t n, void* dst, cudaStream_t s);
 cudaError_t launch_tc_gemm(TcParams& P, bool gateup, int64_t max_tiles, cudaStream_t s);

@@ -8,6 +8,7 @@
 // ascending slot order. Also emits the compact list of experts that received
 // tokens, which the expert kernels use to skip empty experts.
 #include <cuda.h>
+#include <cuda_fp16.h>
 
 #include <mutex>
 
@@ -71,7 +72,9 @@ __global__ void __launch_bounds__(kPlaceThreads) tile_start_kernel(const int32_t
 }
 
 // One warp per destination row, 16-byte vectors; only sorted positions in [*lo, *hi) when
-// those bounds are given (a range of experts).
+// those bounds are given (a range of experts). F16: the bf16 rows are written as fp16
+// (exact within fp16's range), the token operand of 4-bit affine weights.
+template <bool F16>
 __global__ void __launch_bounds__(256) gather_rows_kernel(const uint4* __restrict__ src, int vpr,
                                                           const int32_t* __restrict__ sorted_slot, int k,
                                                           int64_t S, uint4* __restrict__ dst,
@@ -83,18 +86,34 @@ __global__ void __launch_bounds__(256) gather_rows_kernel(const uint4* __restric
     const int64_t row = sorted_slot[p] / k;
     const uint4* s = src + row * vpr;
     uint4* d = dst + p * vpr;
-    for (int c = lane; c < vpr; c += 32) d[c] = s[c];
+    for (int c = lane; c < vpr; c += 32) {
+        if constexpr (F16) {
+            float f[8];
+            unpack8(s[c], f);
+            uint32_t h[4];
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                __half2 v = __floats2half2_rn(f[2 * j], f[2 * j + 1]);
+                h[j] = *reinterpret_cast<uint32_t*>(&v);
+            }
+            d[c] = make_uint4(h[0], h[1], h[2], h[3]);
+        } else {
+            d[c] = s[c];
+        }
+    }
 }
 
 }  // namespace
 
 cudaError_t launch_gather_rows(const void* src, int K, const int32_t* sorted_slot, int k, int64_t S, void* dst,
-                               cudaStream_t s, const int32_t* lo, const int32_t* hi) {
+                               cudaStream_t s, const int32_t* lo, const int32_t* hi, bool to_f16) {
     if (S == 0) return cudaSuccess;
     const int vpr = K * 2 / 16;
     const unsigned grid = unsigned((S * 32 + 255) / 256);
-    { const cudaError_t e_ = launch_pdl(gather_rows_kernel, dim3(grid), dim3(256), 0, s, static_cast<const uint4*>(src), vpr, sorted_slot, k, S,
-                                            static_cast<uint4*>(dst), lo, hi); if (e_ != cudaSuccess) return e_; }
+    auto kern = to_f16 ? gather_rows_kernel<true> : gather_rows_kernel<false>;
+    const cudaError_t e = launch_pdl(kern, dim3(grid), dim3(256), 0, s, static_cast<const uint4*>(src), vpr, sorted_slot,
+                                     k, S, static_cast<uint4*>(dst), lo, hi);
+    if (e != cudaSuccess) return e;
     return cudaGetLastError();
 }
 

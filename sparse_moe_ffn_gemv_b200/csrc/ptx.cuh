@@ -104,16 +104,6 @@ __device__ __forceinline__ void tma_4d(void* dst, const CUtensorMap* m, uint64_t
         "l"(reinterpret_cast<uint64_t>(m)), "r"(su32(bar)), "r"(c0), "r"(c1), "r"(c2), "r"(c3), "l"(pol)
         : "memory");
 }
-// Four rows (r0..r3) x one box of columns from c0 of a 2D tensor map whose box is one row
-// high, written to consecutive rows of shared memory from dst (TMA row gather).
-__device__ __forceinline__ void tma_gather4(void* dst, const CUtensorMap* m, uint64_t* bar, int c0, int r0, int r1,
-                                            int r2, int r3, uint64_t pol) {
-    asm volatile(
-        "cp.async.bulk.tensor.2d.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes.L2::cache_hint"
-        " [%0], [%1, {%3, %4, %5, %6, %7}], [%2], %8;" ::"r"(su32(dst)),
-        "l"(reinterpret_cast<uint64_t>(m)), "r"(su32(bar)), "r"(c0), "r"(r0), "r"(r1), "r"(r2), "r"(r3), "l"(pol)
-        : "memory");
-}
 // 1D bulk copy global -> shared, completing on an mbarrier (16-byte aligned, size % 16 == 0).
 __device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t bytes, uint64_t* bar, uint64_t pol) {
     asm volatile(

@@ -333,7 +333,7 @@ __global__ void __launch_bounds__(TcShape<GATEUP, BN, STAGES, Q4>::THREADS, 1)
         for (int i = 0; i < P.nprob; ++i) {
             prefetch_tmap(&P.a0[i]);
             if (GATEUP && !P.p[i].interleaved) prefetch_tmap(&P.a1[i]);
-            for (int v = 0; v < (P.p[i].gather_k ? 1 : 4); ++v) prefetch_tmap(&P.b[i][v]);
+            for (int v = 0; v < 4; ++v) prefetch_tmap(&P.b[i][v]);
         }
     }
     pdl_begin();  // everything above touches no memory that earlier kernels write
@@ -359,9 +359,7 @@ __global__ void __launch_bounds__(TcShape<GATEUP, BN, STAGES, Q4>::THREADS, 1)
         // bf16: both weight tiles + the token tile of each K block into one stage.
         // 4-bit: the two packed tiles + the token tile into one load slot (the
         // dequantising warps bring bf16 tiles into the operand ring themselves).
-        // Lane 0 waits for the slot, arms its barrier and loads the weight tiles; the token
-        // tile is one tiled load by lane 0, or, for a gathered problem, one four-row TMA gather
-        // per lane (lane l: the tile's token rows 4l .. 4l + 3).
+        // Lane 0 waits for the slot, arms its barrier and issues the loads.
         uint32_t stage = 0, phase = 0;
         uint32_t armed = 0;  // bit s: stage s was filled at least once
         uint32_t last_par = 0;
@@ -373,14 +371,7 @@ __global__ void __launch_bounds__(TcShape<GATEUP, BN, STAGES, Q4>::THREADS, 1)
             const int mrow = ti.mb * S::ROWS;
             // token rows: the smallest box (16, 32, 64, BN) that holds the valid tokens
             const int bv = ti.nvalid <= 16 ? 0 : ti.nvalid <= 32 ? 1 : ti.nvalid <= 64 ? 2 : 3;
-            const bool gath = p.gather_k > 0;
-            const int ngr = gath ? (ti.nvalid + 3) / 4 : 0;  // lanes that gather four rows
-            const uint32_t b_bytes = gath ? uint32_t(ngr) * 4 * kBK * 2 : uint32_t(min(BN, 16 << bv)) * kBK * 2;
-            int gr[4] = {0, 0, 0, 0};  // this lane's four token rows (padding rows read row 0)
-            if (gath && lane < ngr)
-#pragma unroll
-                for (int j = 0; j < 4; ++j)
-                    if (4 * lane + j < ti.nvalid) gr[j] = p.sorted_slot[ti.row0 + 4 * lane + j] / p.gather_k;
+            const uint32_t b_bytes = uint32_t(min(BN, 16 << bv)) * kBK * 2;
             for (int kb = 0; kb < nk; ++kb) {
                 int ok = 1;
                 if (lane == 0) ok = mbar_wait(&empty[stage], phase ^ 1u, deadline) ? 1 : 0;
@@ -406,12 +397,8 @@ __global__ void __launch_bounds__(TcShape<GATEUP, BN, STAGES, Q4>::THREADS, 1)
                         mbar_expect_tx(&full[stage], 2 * S::A_BYTES + b_bytes);
                         load_a_bf16<GATEUP>(sb, P, ti, mrow, kc, &full[stage], pol_w);
                     }
-                    if (!gath) tma_2d(sb + S::B_OFF, &P.b[ti.prob][bv], &full[stage], kc, ti.row0, pol_t);
+                    tma_2d(sb + S::B_OFF, &P.b[ti.prob][bv], &full[stage], kc, ti.row0, pol_t);
                 }
-                __syncwarp();  // the barrier expects the gathered bytes before any gather lands
-                if (gath && lane < ngr)
-                    tma_gather4(sb + S::B_OFF + lane * 4 * kBK * 2, &P.b[ti.prob][0], &full[stage], kc, gr[0], gr[1],
-                                gr[2], gr[3], pol_t);
                 armed |= 1u << stage;
                 last_par = (last_par & ~(1u << stage)) | (phase << stage);
                 if (++stage == STAGES) {
@@ -879,14 +866,6 @@ bool tc_token_map(CUtensorMap* m, const void* u, int64_t rows, int K, int bn) {
         if (!encode(&m[v], u, 2, dims, strides, box)) return false;
     }
     return true;
-}
-
-// Token operand [rows, K] bf16 for TMA row gather: box of one 64-wide K block x one row.
-bool tc_gather_map(CUtensorMap* m, const void* u, int64_t rows, int K) {
-    const cuuint64_t dims[2] = {cuuint64_t(K), cuuint64_t(rows)};
-    const cuuint64_t strides[1] = {cuuint64_t(K) * 2};
-    const cuuint32_t box[2] = {kBK, 1};
-    return encode(m, u, 2, dims, strides, box);
 }
 
 // Packed 4-bit plane [E, R, K / 8] uint32 (K % 64 == 0): box of 8 words x 128 rows. With
