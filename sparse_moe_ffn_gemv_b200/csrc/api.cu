@@ -285,11 +285,16 @@ DecodeArgs decode_args(const moe_config* c, const moe_weights* w, const void* x,
     return d;
 }
 
+// Chosen where it measured faster than both other engines on B200 (graph replay, L2
+// flushed): a single token, and MXFP4 weights up to 8 tokens. From two tokens on, the
+// tensor-core kernel streams bf16 and affine 4-bit weights faster (Klear 2 tokens: 98 vs
+// 82 us; 8 tokens: 186 vs 129 us).
 bool use_decode(const moe_config* c, int64_t T, const DecodeArgs& d) {
     if (c->latent_dim || c->act_dtype != MOE_DTYPE_BF16 || c->weight_format == MOE_DTYPE_F32) return false;
     const int o = path_override();
     if (o == kPathGemv || o == kPathTc) return false;
-    return T >= 1 && T <= 8 && decode_smem_bytes(d) > 0;
+    if (T < 1 || T > 8 || decode_smem_bytes(d) == 0) return false;
+    return o == kPathDecode || T == 1 || c->weight_format == MOE_DTYPE_MXFP4;
 }
 
 #define MOE_CHECK(expr)                          \

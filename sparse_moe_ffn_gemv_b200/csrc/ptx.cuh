@@ -36,11 +36,31 @@ __device__ __forceinline__ bool mbar_try(uint64_t* b, uint32_t parity) {
         : "memory");
     return ok != 0;
 }
+// The same test, letting the thread sleep up to `ns` nanoseconds inside the instruction
+// while the phase is incomplete (a long wait that should not take issue slots).
+__device__ __forceinline__ bool mbar_try_sleep(uint64_t* b, uint32_t parity, uint32_t ns) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(su32(b)), "r"(parity), "r"(ns)
+        : "memory");
+    return ok != 0;
+}
 // Bounded wait for the phase with the given parity; false = gave up.
 __device__ __forceinline__ bool mbar_wait(uint64_t* b, uint32_t parity, uint64_t deadline) {
     for (uint32_t i = 0;; ++i) {
         if (mbar_try(b, parity)) return true;
         if ((i & 63u) == 63u && gtimer() > deadline) return false;
+    }
+}
+// Bounded wait that sleeps inside each test (up to 2 us at a time).
+__device__ __forceinline__ bool mbar_wait_sleep(uint64_t* b, uint32_t parity, uint64_t deadline) {
+    for (;;) {
+        if (mbar_try_sleep(b, parity, 2000u)) return true;
+        if (gtimer() > deadline) return false;
     }
 }
 

@@ -51,7 +51,6 @@ namespace {
 
 constexpr int kBM = 128;          // weight rows per MMA (M)
 constexpr int kBK = 64;           // K per stage: one 128-byte swizzle atom of bf16
-constexpr int kTcThreads = 320;   // 10 warps: TMA, MMA, 8 epilogue
 constexpr int kDqThreads = 256;   // + 8 dequantising warps for 4-bit weights (4 measured 30% slower)
 constexpr int kDqTiles = 2 * kBM / kDqThreads;  // weight tiles per dequantising thread (one row each)
 constexpr int kEpiThreads = 256;
@@ -187,7 +186,12 @@ struct TcShape {
     static constexpr int STAGE_BYTES = Q4 ? 2 * kPkBytes + B_BYTES : 2 * A_BYTES + B_BYTES;
     static constexpr int ARING_OFF = STAGES * STAGE_BYTES;       // operand ring (4-bit only)
     static constexpr int RING_BYTES = STAGES * STAGE_BYTES + ASTAGES * 2 * A_BYTES;
-    static constexpr int THREADS = kTcThreads + (Q4 ? kDqThreads : 0);
+    // epilogue warps: 8 (two per TMEM lane quarter, one column half each), or 4 beside the
+    // dequantising warps (each taking both halves), which keeps the 4-bit block at 14 warps,
+    // at most 4 per SM sub-partition and so 128 registers per thread
+    static constexpr int EPI = Q4 ? 128 : kEpiThreads;
+    static constexpr int DQ_BASE = 64 + EPI;                     // first dequantising thread
+    static constexpr int THREADS = 64 + EPI + (Q4 ? kDqThreads : 0);
     static constexpr int ACC_COLS = 2 * BN;                      // per accumulator set
     static constexpr int TMEM_COLS = 2 * ACC_COLS;               // double-buffered
     static constexpr int ROWS = GATEUP ? kBM : 2 * kBM;          // weight rows per tile
@@ -318,7 +322,7 @@ __global__ void __launch_bounds__(TcShape<GATEUP, BN, STAGES, Q4>::THREADS, 1)
         }
         for (int b = 0; b < 2; ++b) {
             mbar_init(&acc_full[b], 1);
-            mbar_init(&acc_empty[b], kEpiThreads / 32);  // one arrive per epilogue warp
+            mbar_init(&acc_empty[b], S::EPI / 32);  // one arrive per epilogue warp
         }
         mbar_init(drain, 1);
         if (Q4)
@@ -470,15 +474,15 @@ __global__ void __launch_bounds__(TcShape<GATEUP, BN, STAGES, Q4>::THREADS, 1)
             mbar_wait(drain, 0, gtimer() + kWaitNs);
             if (timed_out) set_status(P.status, MOE_ERR_DEVICE_TIMEOUT);
         }
-    } else if (Q4 && warp >= kTcThreads / 32) {
+    } else if (Q4 && int(threadIdx.x) >= S::DQ_BASE) {
         // ---------------------------------------------------------- dequantisation warps
         // Thread d dequantises row d % 128 of kDqTiles of the two weight tiles (all 64 K
         // elements of the block: two 16-byte loads of packed words from the load slot, eight
         // swizzled 16-byte stores into the operand slot). Its (scale, bias) pairs are loaded
-        // three K blocks ahead. A bf16 tile in the same launch (the shared expert) gets its
+        // eight K blocks ahead. A bf16 tile in the same launch (the shared expert) gets its
         // operand slot filled by TMA, issued by the first dequantising thread.
         constexpr int DT = kDqTiles;
-        const int d = threadIdx.x - kTcThreads;
+        const int d = threadIdx.x - S::DQ_BASE;
         const int drow = d & (kBM - 1), a0 = (d / kBM) * DT;
         const bool leader = d == 0;
         uint32_t stage = 0, phase = 0;
@@ -558,13 +562,26 @@ __global__ void __launch_bounds__(TcShape<GATEUP, BN, STAGES, Q4>::THREADS, 1)
                         }
                     }
             };
-            __nv_bfloat162 q0[DT][2], q1[DT][2], q2[DT][2];
-            load_sb(0, q0);
-            if (nk > 1) load_sb(1, q1);
-            if (nk > 2) load_sb(2, q2);
+            // a ring of the next kPre K blocks' pairs in registers, refilled kPre blocks ahead
+            // (the pairs come from DRAM the first time a tile row is read)
+            constexpr int kPre = 8;
+            __nv_bfloat162 qr[kPre][DT][2];
+#pragma unroll
+            for (int j = 0; j < kPre; ++j)
+                if (j < nk) load_sb(j, qr[j]);
             for (int kb = 0; kb < nk; ++kb) {
-                __nv_bfloat162 q3[DT][2];
-                if (kb + 3 < nk) load_sb(kb + 3, q3);
+                __nv_bfloat162 q0[DT][2];
+#pragma unroll
+                for (int ai = 0; ai < DT; ++ai)
+#pragma unroll
+                    for (int h = 0; h < 2; ++h) q0[ai][h] = qr[0][ai][h];
+#pragma unroll
+                for (int j = 0; j + 1 < kPre; ++j)
+#pragma unroll
+                    for (int ai = 0; ai < DT; ++ai)
+#pragma unroll
+                        for (int h = 0; h < 2; ++h) qr[j][ai][h] = qr[j + 1][ai][h];
+                if (kb + kPre < nk) load_sb(kb + kPre, qr[kPre - 1]);
                 if (!mbar_wait(&full[stage], phase, deadline) || !mbar_wait(&aempty[astage], aphase ^ 1u, deadline)) {
                     timed_out = true;
                     break;
@@ -594,14 +611,6 @@ __global__ void __launch_bounds__(TcShape<GATEUP, BN, STAGES, Q4>::THREADS, 1)
                 asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&dq[astage]);
-#pragma unroll
-                for (int ai = 0; ai < DT; ++ai)
-#pragma unroll
-                    for (int h = 0; h < 2; ++h) {
-                        q0[ai][h] = q1[ai][h];
-                        q1[ai][h] = q2[ai][h];
-                        q2[ai][h] = q3[ai][h];
-                    }
                 next();
             }
             };
@@ -625,8 +634,9 @@ __global__ void __launch_bounds__(TcShape<GATEUP, BN, STAGES, Q4>::THREADS, 1)
         const int q = warp & 3;
         const int tok = q * 32 + lane;  // token row of the tile
         const int eid = threadIdx.x - 64;
-        const int half = eid >= 128 ? 1 : 0;
-        float* sb = sbias + (eid >> 5) * 128;  // this warp's column biases (warp-private)
+        constexpr int NH = S::EPI == kEpiThreads ? 1 : 2;  // column halves per warp
+        const int h_lo = NH == 1 ? (eid >= 128 ? 1 : 0) : 0;
+        float* sb = sbias + (eid >> 5) * 128 * NH;  // this warp's column biases (warp-private)
         uint32_t it = 0;
         for (int tile = blockIdx.x; tile < total; tile += gridDim.x, ++it) {
             const TileInfo ti = decode_tile(P, gt, tile, t0);
@@ -642,27 +652,33 @@ __global__ void __launch_bounds__(TcShape<GATEUP, BN, STAGES, Q4>::THREADS, 1)
                 yrow = reinterpret_cast<float*>(p.out) + int64_t(slot / p.k) * p.ld_out;
             }
             const bool has_bias = p.bias0 != nullptr;
-            if (has_bias) {  // the 128 biases of this warp's columns: 4 per lane, before the wait
+            if (has_bias) {  // the biases of this warp's columns (128 per half), before the wait
                 __syncwarp();  // every lane is done with the previous tile's values
 #pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                    const int j = lane + 32 * i;
-                    float b = 0.f;
-                    if (GATEUP) {  // j < 64: gate bias of unit u0 + j, else up bias of unit u0 + j - 64
-                        const int unit = ti.mb * kBM + half * 64 + (j & 63);
-                        const int up = j >= 64 ? 1 : 0;
-                        if (unit < p.M)
-                            b = p.bias_interleaved ? bf16_at(p.bias0, (int64_t(ti.group) * p.M + unit) * 2 + up)
-                                                   : bf16_at(up ? p.bias1 : p.bias0, int64_t(ti.group) * p.M + unit);
-                    } else {
-                        const int r = ti.mb * 2 * kBM + half * kBM + j;
-                        if (r < p.M) b = bf16_at(p.bias0, int64_t(ti.group) * p.M + r);
+                for (int hh = 0; hh < NH; ++hh) {
+                    const int half = h_lo + hh;
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        const int j = lane + 32 * i;
+                        float b = 0.f;
+                        if (GATEUP) {  // j < 64: gate bias of unit u0 + j, else up bias of unit u0 + j - 64
+                            const int unit = ti.mb * kBM + half * 64 + (j & 63);
+                            const int up = j >= 64 ? 1 : 0;
+                            if (unit < p.M)
+                                b = p.bias_interleaved ? bf16_at(p.bias0, (int64_t(ti.group) * p.M + unit) * 2 + up)
+                                                       : bf16_at(up ? p.bias1 : p.bias0, int64_t(ti.group) * p.M + unit);
+                        } else {
+                            const int r = ti.mb * 2 * kBM + half * kBM + j;
+                            if (r < p.M) b = bf16_at(p.bias0, int64_t(ti.group) * p.M + r);
+                        }
+                        sb[hh * 128 + j] = b;
                     }
-                    sb[j] = b;
                 }
                 __syncwarp();
             }
-            if (!mbar_wait(&acc_full[ab], aph, deadline)) {
+            // the accumulator is ready only after the tile's whole main loop: sleep in the wait
+            // rather than take issue slots from the warps that feed the MMA
+            if (!mbar_wait_sleep(&acc_full[ab], aph, deadline)) {
                 set_status(P.status, MOE_ERR_DEVICE_TIMEOUT);
                 break;
             }
@@ -673,111 +689,116 @@ __global__ void __launch_bounds__(TcShape<GATEUP, BN, STAGES, Q4>::THREADS, 1)
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&acc_empty[ab]);
             };
-            if constexpr (GATEUP) {
-                // 32 units per chunk: gate and up of the same units -> 32 bf16 of h (64 bytes)
-                const int u0 = ti.mb * kBM + half * 64;
 #pragma unroll 1
-                for (int c = 0; c < 2; ++c) {
-                    uint32_t g[32], u[32];
-                    tmem_ld_issue(tb + half * 64 + 32 * c, g);
-                    tmem_ld_issue(tb + kBM + half * 64 + 32 * c, u);
-                    tmem_ld_wait(g);
-                    tmem_ld_wait(u);
-                    if (c == 1) release();
-                    const int ub = u0 + 32 * c;
-                    if (!tv || ub >= p.M) continue;
-                    const float* bg = sb + 32 * c;  // gate biases of these 32 units
-                    const float* bu = bg + 64;       // their up biases
-                    uint32_t hp[16];
+            for (int hh = 0; hh < NH; ++hh) {
+                const int half = h_lo + hh;
+                const bool last_half = hh == NH - 1;
+                const float* sbh = sb + hh * 128;
+                if constexpr (GATEUP) {
+                    // 32 units per chunk: gate and up of the same units -> 32 values of h (64 bytes)
+                    const int u0 = ti.mb * kBM + half * 64;
+#pragma unroll 1
+                    for (int c = 0; c < 2; ++c) {
+                        uint32_t g[32], u[32];
+                        tmem_ld_issue(tb + half * 64 + 32 * c, g);
+                        tmem_ld_issue(tb + kBM + half * 64 + 32 * c, u);
+                        tmem_ld_wait(g);
+                        tmem_ld_wait(u);
+                        if (c == 1 && last_half) release();
+                        const int ub = u0 + 32 * c;
+                        if (!tv || ub >= p.M) continue;
+                        const float* bg = sbh + 32 * c;  // gate biases of these 32 units
+                        const float* bu = bg + 64;       // their up biases
+                        uint32_t hp[16];
 #pragma unroll
-                    for (int j = 0; j < 32; j += 2) {
-                        float gg0 = __uint_as_float(g[j]), gg1 = __uint_as_float(g[j + 1]);
-                        float uu0 = __uint_as_float(u[j]), uu1 = __uint_as_float(u[j + 1]);
+                        for (int j = 0; j < 32; j += 2) {
+                            float gg0 = __uint_as_float(g[j]), gg1 = __uint_as_float(g[j + 1]);
+                            float uu0 = __uint_as_float(u[j]), uu1 = __uint_as_float(u[j + 1]);
+                            if (has_bias) {
+                                gg0 += bg[j]; gg1 += bg[j + 1];
+                                uu0 += bu[j]; uu1 += bu[j + 1];
+                            }
+                            const float a0 = act_fast(P.act, gg0, uu0, P.limit, P.alpha);
+                            const float a1 = act_fast(P.act, gg1, uu1, P.limit, P.alpha);
+                            if (p.out_f16) {
+                                __half2 v2 = __floats2half2_rn(a0, a1);
+                                hp[j / 2] = *reinterpret_cast<uint32_t*>(&v2);
+                            } else {
+                                __nv_bfloat162 v2 = __floats2bfloat162_rn(a0, a1);
+                                hp[j / 2] = *reinterpret_cast<uint32_t*>(&v2);
+                            }
+                        }
+                        uint4* dst = reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(p.out) + prow * p.ld_out + ub);
+#pragma unroll
+                        for (int v = 0; v < 4; ++v) dst[v] = make_uint4(hp[4 * v], hp[4 * v + 1], hp[4 * v + 2], hp[4 * v + 3]);
+                    }
+                } else {
+                    // 32 weight rows (output columns) per chunk; bf16 weights: the next chunk's TMEM
+                    // load in flight while this one is stored; 4-bit weights: one at a time
+                    const int rb = ti.mb * 2 * kBM + half * kBM;
+                    constexpr int NB = Q4 ? 1 : 2;
+                    uint32_t v[NB][32];
+                    tmem_ld_issue(tb + half * kBM, v[0]);
+#pragma unroll
+                    for (int c = 0; c < 4; ++c) {
+                        tmem_ld_wait(v[c % NB]);
+                        if (NB == 2 && c < 3) tmem_ld_issue(tb + half * kBM + 32 * (c + 1), v[(c + 1) % NB]);
+                        if (c == 3 && last_half) release();
+                        const int r0 = rb + 32 * c;
+                        float o[32];
+#pragma unroll
+                        for (int j = 0; j < 32; ++j) o[j] = __uint_as_float(v[c % NB][j]);
+                        if (NB == 1 && c < 3) tmem_ld_issue(tb + half * kBM + 32 * (c + 1), v[0]);
+                        if (!tv || r0 >= p.M) continue;
                         if (has_bias) {
-                            gg0 += bg[j]; gg1 += bg[j + 1];
-                            uu0 += bu[j]; uu1 += bu[j + 1];
+#pragma unroll
+                            for (int j = 0; j < 32; ++j) o[j] += sbh[32 * c + j];
                         }
-                        const float a0 = act_fast(P.act, gg0, uu0, P.limit, P.alpha);
-                        const float a1 = act_fast(P.act, gg1, uu1, P.limit, P.alpha);
-                        if (p.out_f16) {
-                            __half2 v2 = __floats2half2_rn(a0, a1);
-                            hp[j / 2] = *reinterpret_cast<uint32_t*>(&v2);
-                        } else {
-                            __nv_bfloat162 v2 = __floats2bfloat162_rn(a0, a1);
-                            hp[j / 2] = *reinterpret_cast<uint32_t*>(&v2);
-                        }
-                    }
-                    uint4* dst = reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(p.out) + prow * p.ld_out + ub);
-#pragma unroll
-                    for (int v = 0; v < 4; ++v) dst[v] = make_uint4(hp[4 * v], hp[4 * v + 1], hp[4 * v + 2], hp[4 * v + 3]);
-                }
-            } else {
-                // 32 weight rows (output columns) per chunk, the next chunk's TMEM load in flight
-                const int rb = ti.mb * 2 * kBM + half * kBM;
-                // bf16 weights: the next chunk's TMEM load in flight while this one is stored;
-                // 4-bit weights (the dequantising warps share the register file): one at a time
-                constexpr int NB = Q4 ? 1 : 2;
-                uint32_t v[NB][32];
-                tmem_ld_issue(tb + half * kBM, v[0]);
-#pragma unroll
-                for (int c = 0; c < 4; ++c) {
-                    tmem_ld_wait(v[c % NB]);
-                    if (NB == 2 && c < 3) tmem_ld_issue(tb + half * kBM + 32 * (c + 1), v[(c + 1) % NB]);
-                    if (c == 3) release();
-                    const int r0 = rb + 32 * c;
-                    float o[32];
-#pragma unroll
-                    for (int j = 0; j < 32; ++j) o[j] = __uint_as_float(v[c % NB][j]);
-                    if (NB == 1 && c < 3) tmem_ld_issue(tb + half * kBM + 32 * (c + 1), v[0]);
-                    if (!tv || r0 >= p.M) continue;
-                    if (has_bias) {
-#pragma unroll
-                        for (int j = 0; j < 32; ++j) o[j] += sb[32 * c + j];
-                    }
-                    const bool whole = r0 + 32 <= p.M;
-                    if (p.mode == kEpiScatterAdd) {
-                        // weighted combine into the token's fp32 routed sum, 16 bytes per
-                        // reduction (libmir-metal execute: down weighted by routing.weights and
-                        // summed per token); M is a multiple of 64 here
-#pragma unroll
-                        for (int j = 0; j < 32; j += 4)
-                            red_add_v4(yrow + r0 + j, wslot * o[j], wslot * o[j + 1], wslot * o[j + 2], wslot * o[j + 3]);
-                    } else if (p.mode == kEpiStoreF32) {
-                        float* dst = reinterpret_cast<float*>(p.out) + prow * p.ld_out + r0;
-                        if (whole) {
+                        const bool whole = r0 + 32 <= p.M;
+                        if (p.mode == kEpiScatterAdd) {
+                            // weighted combine into the token's fp32 routed sum, 16 bytes per
+                            // reduction (libmir-metal execute: down weighted by routing.weights and
+                            // summed per token); M is a multiple of 64 here
 #pragma unroll
                             for (int j = 0; j < 32; j += 4)
-                                *reinterpret_cast<float4*>(dst + j) = make_float4(o[j], o[j + 1], o[j + 2], o[j + 3]);
-                        } else {
+                                red_add_v4(yrow + r0 + j, wslot * o[j], wslot * o[j + 1], wslot * o[j + 2], wslot * o[j + 3]);
+                        } else if (p.mode == kEpiStoreF32) {
+                            float* dst = reinterpret_cast<float*>(p.out) + prow * p.ld_out + r0;
+                            if (whole) {
 #pragma unroll
-                            for (int j = 0; j < 32; ++j)
-                                if (r0 + j < p.M) dst[j] = o[j];
-                        }
-                    } else {  // kEpiStoreAct (+ optional fp32 addend)
-                        __nv_bfloat16* dst = reinterpret_cast<__nv_bfloat16*>(p.out) + prow * p.ld_out + r0;
-                        const float* ad = p.addend ? p.addend + prow * p.ld_add + r0 : nullptr;
-                        if (whole) {
-                            if (ad) {
+                                for (int j = 0; j < 32; j += 4)
+                                    *reinterpret_cast<float4*>(dst + j) = make_float4(o[j], o[j + 1], o[j + 2], o[j + 3]);
+                            } else {
 #pragma unroll
-                                for (int j = 0; j < 32; j += 4) {
-                                    const float4 a4 = __ldcs(reinterpret_cast<const float4*>(ad + j));
-                                    o[j] += a4.x; o[j + 1] += a4.y; o[j + 2] += a4.z; o[j + 3] += a4.w;
-                                }
+                                for (int j = 0; j < 32; ++j)
+                                    if (r0 + j < p.M) dst[j] = o[j];
                             }
+                        } else {  // kEpiStoreAct (+ optional fp32 addend)
+                            __nv_bfloat16* dst = reinterpret_cast<__nv_bfloat16*>(p.out) + prow * p.ld_out + r0;
+                            const float* ad = p.addend ? p.addend + prow * p.ld_add + r0 : nullptr;
+                            if (whole) {
+                                if (ad) {
 #pragma unroll
-                            for (int w4 = 0; w4 < 4; ++w4) {
-                                uint32_t hp[4];
-#pragma unroll
-                                for (int j = 0; j < 4; ++j) {
-                                    __nv_bfloat162 v2 = __floats2bfloat162_rn(o[8 * w4 + 2 * j], o[8 * w4 + 2 * j + 1]);
-                                    hp[j] = *reinterpret_cast<uint32_t*>(&v2);
+                                    for (int j = 0; j < 32; j += 4) {
+                                        const float4 a4 = __ldcs(reinterpret_cast<const float4*>(ad + j));
+                                        o[j] += a4.x; o[j + 1] += a4.y; o[j + 2] += a4.z; o[j + 3] += a4.w;
+                                    }
                                 }
-                                reinterpret_cast<uint4*>(dst)[w4] = make_uint4(hp[0], hp[1], hp[2], hp[3]);
-                            }
-                        } else {
 #pragma unroll
-                            for (int j = 0; j < 32; ++j)
-                                if (r0 + j < p.M) dst[j] = __float2bfloat16_rn(o[j] + (ad ? ad[j] : 0.f));
+                                for (int w4 = 0; w4 < 4; ++w4) {
+                                    uint32_t hp[4];
+#pragma unroll
+                                    for (int j = 0; j < 4; ++j) {
+                                        __nv_bfloat162 v2 = __floats2bfloat162_rn(o[8 * w4 + 2 * j], o[8 * w4 + 2 * j + 1]);
+                                        hp[j] = *reinterpret_cast<uint32_t*>(&v2);
+                                    }
+                                    reinterpret_cast<uint4*>(dst)[w4] = make_uint4(hp[0], hp[1], hp[2], hp[3]);
+                                }
+                            } else {
+#pragma unroll
+                                for (int j = 0; j < 32; ++j)
+                                    if (r0 + j < p.M) dst[j] = __float2bfloat16_rn(o[j] + (ad ? ad[j] : 0.f));
+                            }
                         }
                     }
                 }
