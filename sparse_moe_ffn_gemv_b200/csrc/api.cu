@@ -72,6 +72,18 @@ bool finite_pos(float v) { return std::isfinite(v) && v > 0.f; }
 
 bool dense_q4(const moe_config* c) { return c->dense_format == MOE_DTYPE_Q4_AFFINE; }
 
+// Token rows per tensor-core tile. 128 in launches that dequantise 4-bit weights (their
+// shared memory holds the packed-weight ring as well) and in small batches (four stages of
+// weights in flight per SM, where the launch streams weights for a few tokens); 256 in bf16
+// launches of large batches, where a weight tile then serves twice the token rows (an expert
+// with 129..256 routed rows reads its weights once instead of twice). The expert launches
+// carry the routed and the shared problem, the dense launches one projection.
+int expert_bn(const moe_config* c, int64_t T) {
+    const bool q = c->weight_format == MOE_DTYPE_Q4_AFFINE || c->weight_format == MOE_DTYPE_MXFP4 || dense_q4(c);
+    return !q && T * c->top_k >= 64 * int64_t(c->num_experts) ? kTcBNWide : kTcBN;
+}
+int dense_bn(const moe_config* c, int64_t T) { return !dense_q4(c) && T >= 256 ? kTcBNWide : kTcBN; }
+
 // Weight operand(s) of a dense (one-group) tensor-core problem: bf16 [M, K], or 4-bit affine
 // words [M, K / 8] with bf16 scales / biases per dense_group_size columns (the second
 // operand w1 only in gate/up mode).
@@ -393,14 +405,15 @@ moe_status run_route(const moe_config* c, const moe_weights* w, const void* x, i
             p.K = c->hidden;
             p.m_blocks = (p.M + kTcRows - 1) / kTcRows;
             p.rows = int(T);
-            p.n_tiles = int((T + kTcBN - 1) / kTcBN);
+            p.bn = dense_bn(c, T);  // a 4-bit router never runs here
+            p.n_tiles = int((T + p.bn - 1) / p.bn);
             p.bias0 = i == 0 ? r.b0 : r.b1;
             p.out = at<float>(ws, L.logits) + (i == 0 ? 0 : c->num_experts);
             p.ld_out = L.ld_logits;
             const bool wok = i == 0 ? tc_dense_weights(c, p, &P.a0[i], nullptr, r.W0, w->router_s, w->router_z, nullptr,
                                                        nullptr, nullptr, p.M, c->hidden)
                                     : tc_weight_map(&P.a0[i], r.W1, 1, p.M, c->hidden, false);  // blend head: act dtype
-            if (!wok || !tc_token_map(P.b[i], x, T, c->hidden, kTcBN)) return MOE_ERR_CUDA;
+            if (!wok || !tc_token_map(P.b[i], x, T, c->hidden, p.bn)) return MOE_ERR_CUDA;
         }
         P.nprob = np;
         P.status = at<int>(ws, L.status);
@@ -440,7 +453,7 @@ moe_status run_permute(const moe_config* c, const int32_t* idx, int64_t T, int32
     p.n_chunks = L.n_chunks;
     p.status = at<int>(ws, L.status);
     if (tc_tiles) {
-        p.tile_bn = kTcBN;
+        p.tile_bn = expert_bn(c, T);
         p.tile_start = at<int32_t>(ws, L.tiles);
     }
     MOE_CUDA(launch_permute(p, s));
@@ -468,7 +481,8 @@ moe_status run_experts_tc(const moe_config* c, const moe_weights* w, const void*
     void* x16 = at<void>(ws, L.x16);
     const int Is = c->shared_intermediate;
     const int64_t S = T * k;
-    const int64_t n_dense = (T + kTcBN - 1) / kTcBN;
+    const int BN = expert_bn(c, T);
+    const int64_t n_dense = (T + BN - 1) / BN;
     void* uperm = at<void>(ws, L.uperm);
     // the routed token rows in sorted order (fp16 for 4-bit affine weights)
     if (rtc) MOE_CUDA(launch_gather_rows(u, K, sorted_slot, k, S, uperm, s, goff, goff + E, aff));
@@ -484,12 +498,12 @@ moe_status run_experts_tc(const moe_config* c, const moe_weights* w, const void*
             TcProblem& p = P.p[np];
             p.mode = kEpiGateUp;
             p.M = Is; p.K = H; p.m_blocks = (Is + kTcRowsGateUp - 1) / kTcRowsGateUp;
-            p.rows = int(T); p.n_tiles = int(n_dense);
+            p.rows = int(T); p.n_tiles = int(n_dense); p.bn = BN;
             p.out = hs; p.ld_out = Is;
             p.out_f16 = dq ? 1 : 0;  // fp16 hs for the fp16 shared down GEMM
             if (!tc_dense_weights(c, p, &P.a0[np], &P.a1[np], w->shared_gate_w, w->shared_gate_s, w->shared_gate_z,
                                   w->shared_up_w, w->shared_up_s, w->shared_up_z, Is, H) ||
-                !tc_token_map(P.b[np], dq ? x16 : x, T, H, kTcBN))
+                !tc_token_map(P.b[np], dq ? x16 : x, T, H, BN))
                 return MOE_ERR_CUDA;
             max_tiles += int64_t(p.m_blocks) * p.n_tiles;
             ++np;
@@ -498,7 +512,7 @@ moe_status run_experts_tc(const moe_config* c, const moe_weights* w, const void*
             TcProblem& p = P.p[np];
             p.mode = kEpiGateUp;
             p.M = I; p.K = K; p.m_blocks = (I + kTcRowsGateUp - 1) / kTcRowsGateUp;
-            p.grouped = 1; p.num_groups = E; p.offsets = goff; p.tile_start = tiles;
+            p.grouped = 1; p.num_groups = E; p.offsets = goff; p.tile_start = tiles; p.bn = BN;
             p.out = h; p.ld_out = I;
             p.interleaved = c->gate_up_interleaved;  // bf16 / f32 planes: one 4-D map
             if (c->has_expert_bias) {
@@ -542,7 +556,7 @@ moe_status run_experts_tc(const moe_config* c, const moe_weights* w, const void*
                      tc_weight_map(&P.a1[np], w->up_w, E, I, K, false);
             }
             p.out_f16 = aff ? 1 : 0;  // fp16 h for the fp16 routed down GEMM
-            if (!ok || !tc_token_map(P.b[np], uperm, S, K, kTcBN)) return MOE_ERR_CUDA;
+            if (!ok || !tc_token_map(P.b[np], uperm, S, K, BN)) return MOE_ERR_CUDA;
             max_tiles += int64_t(p.m_blocks) * max_routed_tiles(*c, T);
             ++np;
         }
@@ -561,11 +575,11 @@ moe_status run_experts_tc(const moe_config* c, const moe_weights* w, const void*
             TcProblem& p = P.p[np];
             p.mode = kEpiStoreF32;
             p.M = H; p.K = Is; p.m_blocks = (H + kTcRows - 1) / kTcRows;
-            p.rows = int(T); p.n_tiles = int(n_dense);
+            p.rows = int(T); p.n_tiles = int(n_dense); p.bn = BN;
             p.out = at<float>(ws, L.s_acc); p.ld_out = H;
             if (!tc_dense_weights(c, p, &P.a0[np], nullptr, w->shared_down_w, w->shared_down_s, w->shared_down_z,
                                   nullptr, nullptr, nullptr, H, Is) ||
-                !tc_token_map(P.b[np], hs, T, Is, kTcBN))
+                !tc_token_map(P.b[np], hs, T, Is, BN))
                 return MOE_ERR_CUDA;
             max_tiles += int64_t(p.m_blocks) * p.n_tiles;
             ++np;
@@ -574,7 +588,7 @@ moe_status run_experts_tc(const moe_config* c, const moe_weights* w, const void*
             TcProblem& p = P.p[np];
             p.mode = kEpiScatterAdd;
             p.M = K; p.K = I; p.m_blocks = (K + kTcRows - 1) / kTcRows;
-            p.grouped = 1; p.num_groups = E; p.offsets = goff; p.tile_start = tiles;
+            p.grouped = 1; p.num_groups = E; p.offsets = goff; p.tile_start = tiles; p.bn = BN;
             p.sorted_slot = sorted_slot; p.topk_w = topk_w; p.k = k;
             p.bias0 = c->has_expert_bias ? w->down_b : nullptr;
             p.out = y_acc; p.ld_out = K;
@@ -588,7 +602,7 @@ moe_status run_experts_tc(const moe_config* c, const moe_weights* w, const void*
             } else {
                 ok = tc_weight_map(&P.a0[np], w->down_w, E, K, I, false);
             }
-            if (!ok || !tc_token_map(P.b[np], h, S, I, kTcBN)) return MOE_ERR_CUDA;
+            if (!ok || !tc_token_map(P.b[np], h, S, I, BN)) return MOE_ERR_CUDA;
             max_tiles += int64_t(p.m_blocks) * max_routed_tiles(*c, T);
             ++np;
         }
@@ -721,7 +735,8 @@ moe_status run_latent_down(const moe_config* c, const moe_weights* w, const void
         TcProblem& p = P.p[0];
         p.mode = kEpiStoreAct;
         p.M = c->latent_dim; p.K = c->hidden; p.m_blocks = (p.M + kTcRows - 1) / kTcRows;
-        p.rows = int(T); p.n_tiles = int((T + kTcBN - 1) / kTcBN);
+        p.bn = dense_bn(c, T);
+        p.rows = int(T); p.n_tiles = int((T + p.bn - 1) / p.bn);
         p.out = z; p.ld_out = c->latent_dim;
         const void* xt = x;
         if (dense_q4(c)) {  // fp16 operands
@@ -730,7 +745,7 @@ moe_status run_latent_down(const moe_config* c, const moe_weights* w, const void
         }
         if (!tc_dense_weights(c, p, &P.a0[0], nullptr, w->latent_down_w, w->latent_down_s, w->latent_down_z, nullptr,
                               nullptr, nullptr, p.M, p.K) ||
-            !tc_token_map(P.b[0], xt, T, p.K, kTcBN))
+            !tc_token_map(P.b[0], xt, T, p.K, p.bn))
             return MOE_ERR_CUDA;
         P.nprob = 1;
         P.status = status;
@@ -782,7 +797,8 @@ moe_status run_output(const moe_config* c, const moe_weights* w, RoutedSum rs, c
         TcProblem& p = P.p[0];
         p.mode = kEpiStoreAct;
         p.M = c->hidden; p.K = c->latent_dim; p.m_blocks = (p.M + kTcRows - 1) / kTcRows;
-        p.rows = int(T); p.n_tiles = int((T + kTcBN - 1) / kTcBN);
+        p.bn = dense_bn(c, T);
+        p.rows = int(T); p.n_tiles = int((T + p.bn - 1) / p.bn);
         p.out = y; p.ld_out = c->hidden;
         p.addend = s_acc; p.ld_add = c->hidden;
         const void* nt = n;
@@ -792,7 +808,7 @@ moe_status run_output(const moe_config* c, const moe_weights* w, RoutedSum rs, c
         }
         if (!tc_dense_weights(c, p, &P.a0[0], nullptr, w->latent_up_w, w->latent_up_s, w->latent_up_z, nullptr,
                               nullptr, nullptr, p.M, p.K) ||
-            !tc_token_map(P.b[0], nt, T, p.K, kTcBN))
+            !tc_token_map(P.b[0], nt, T, p.K, p.bn))
             return MOE_ERR_CUDA;
         P.nprob = 1;
         P.status = at<int>(ws, L.status);
@@ -872,7 +888,7 @@ moe_status grouped_ffn_range(const moe_config* cfg, const moe_weights* w, const 
     MOE_CUDA(cudaMemsetAsync(y_acc, 0, size_t(T) * expert_in(*cfg) * sizeof(float), s));
     MOE_CUDA(launch_active_list(expert_offsets + rg.e0, rg.ne, at<int32_t>(ws, L.active), s));
     if (routed_tc(cfg, T))
-        MOE_CUDA(launch_tile_start(expert_offsets + rg.e0, rg.ne, kTcBN, at<int32_t>(ws, L.tiles), s));
+        MOE_CUDA(launch_tile_start(expert_offsets + rg.e0, rg.ne, expert_bn(cfg, T), at<int32_t>(ws, L.tiles), s));
     return run_experts(cfg, w, u, nullptr, T, expert_offsets, sorted_slot, topk_w, y_acc, true, false, ws, L, s,
                        nullptr, rg);
 }

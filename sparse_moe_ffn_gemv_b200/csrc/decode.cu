@@ -50,9 +50,16 @@ struct DecSmem {
     int doff[kDecMaxSlots + 1];  // their ranges in `sorted`
     int n_d;                     // number of distinct experts
     int flag;
+    float sstat[2 * kTT];        // softmax over all experts: each token's max and 1 / sum
     float acc_r[kDecRowsMax][kTT];  // routed sum of the block's rows
     float acc_s[kDecRowsMax][kTT];  // shared expert output of the block's rows
 };
+
+// Byte offset of the top-k keys in the dynamic shared memory: after the T staged token rows
+// (bf16) and, for 4-bit planes, their per-32 sums; 16-byte aligned.
+__host__ __device__ __forceinline__ size_t dec_keys_offset(int T, int H, bool sums) {
+    return (size_t(T) * H * 2 + (sums ? size_t(T) * (H / 32) * 4 : 0) + 15) & ~size_t(15);
+}
 
 __device__ __forceinline__ void l2_prefetch(const void* p, size_t bytes) {
     // a hint: the start is rounded up and the size down to 16 bytes, so nothing outside
@@ -78,13 +85,15 @@ __device__ __forceinline__ void copy_cg(uint4* dst, const void* src, int64_t n16
 
 // Rows per warp item. With one token the accumulators are few, so a warp keeps several rows
 // (two gate/up units, four down rows) in flight; with up to 8 tokens one unit / two rows.
+// Every phase of one format uses the same row count, so that it runs the same code.
 template <int WF, int TT> struct DecShape {
     static constexpr bool ONE = TT == 1;
-    static constexpr int RR = ONE ? 4 : 1;                          // router rows
-    static constexpr int SU = ONE ? 2 : 1;                          // shared gate/up units
+    static constexpr int ND = ONE ? 4 : 2;                          // bf16 dense rows per item
+    static constexpr int RR = ND;                                   // router / coefficient rows
+    static constexpr int SU = ND / 2;                               // shared gate/up units
+    static constexpr int SN = ND;                                   // shared down rows
     static constexpr int BU = (ONE && WF == kBF16) ? 2 : 1;         // routed gate/up units
-    static constexpr int DN = (ONE && WF == kBF16) ? 4 : 2;         // routed down rows
-    static constexpr int SN = ONE ? 4 : 2;                          // shared down rows
+    static constexpr int DN = 2 * BU;                               // routed down rows
 };
 
 // acc[r][t] = sum over the row of W_r . u_t, reduced over the warp (every lane holds it).
@@ -106,6 +115,29 @@ __device__ __forceinline__ void dot_reduce(const char* const (&rows)[NR], const 
         }
 }
 
+// One out-of-line copy of the dot product per (format, rows, tokens): every call site of
+// every phase runs the same instructions. The kernel runs each phase once per SM after an L2
+// flush could have evicted its code, so distinct instructions cost instruction-cache misses;
+// the call's argument traffic (a few words of local memory) is paid once per item.
+template <int WF, int NR, int TT>
+__device__ __noinline__ void dec_dot(const char* const* rows, const QRow* q, int K, int gs,
+                                     const __nv_bfloat16* us, const float* usum, int tt, const int* tl,
+                                     float* out) {
+    const char* r[NR];
+    QRow qq[NR];
+#pragma unroll
+    for (int j = 0; j < NR; ++j) {
+        r[j] = rows[j];
+        qq[j] = q[j];
+    }
+    float acc[NR][TT];
+    dot_reduce<WF, NR, TT>(r, qq, K, gs, us, usum, tt, acc, tl);
+#pragma unroll
+    for (int j = 0; j < NR; ++j)
+#pragma unroll
+        for (int t = 0; t < TT; ++t) out[j * TT + t] = acc[j][t];
+}
+
 template <int WF, int TT>
 __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(const DecodeArgs a) {
     using AT = __nv_bfloat16;
@@ -115,7 +147,9 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(const DecodeArgs
     __shared__ DecSmem sm;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int T = a.T, H = a.H, k = a.k, I = a.I, Is = a.Is, S = T * k, E = a.E;
-    const int gw = blockIdx.x * kDecWarps + warp, nw = gridDim.x * kDecWarps;
+    // grid-wide warp index, SM-major: item i goes to warp i / grid of SM i % grid, so that a
+    // phase with fewer items than warps, or a partial last round, is spread over every SM
+    const int gw = warp * gridDim.x + blockIdx.x, nw = gridDim.x * kDecWarps;
     const uint64_t deadline = gtimer() + kDecWaitNs;
     const int RB = (H + gridDim.x - 1) / gridDim.x;  // output rows per block
     const int r0 = min(H, int(blockIdx.x) * RB), r1 = min(H, r0 + RB), nr = r1 - r0;
@@ -135,6 +169,8 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(const DecodeArgs
     // ------------------------------------------------------------ phase A
     AT* xs = reinterpret_cast<AT*>(dsm);
     float* xsum = reinterpret_cast<float*>(xs + int64_t(T) * H);  // 4-bit affine: sums per 32
+    // selection keys of the top-k (phase B), after the staged tokens and their sums
+    uint64_t* skeys = reinterpret_cast<uint64_t*>(dsm) + dec_keys_offset(T, H, WF == kQ4 || dq) / 8;
     if (WF == kQ4 || dq) stage_tokens<kQ4>(a.x, H, 0, T, nullptr, 1, xs, xsum);
     else stage_tokens<kBF16>(a.x, H, 0, T, nullptr, 1, xs, nullptr);
     if (a.l2_prefetch && Is && threadIdx.x == 0 && nr > 0)
@@ -154,27 +190,32 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(const DecodeArgs
                     rows[j] = static_cast<const char*>(a.router_w) + int64_t(e) * dhb;
                     q[j] = dense_q(a.router_s, a.router_z, e, H);
                 }
-                float acc[RR][TT];
-                if (dq) dot_reduce<kQ4, RR, TT>(rows, q, H, dg, xs, xsum, T, acc);
-                else dot_reduce<kBF16, RR, TT>(rows, q, H, 64, xs, nullptr, T, acc);
+                float acc[RR * TT];
+                if (dq) dec_dot<kQ4, RR, TT>(rows, q, H, dg, xs, xsum, T, nullptr, acc);
+                else dec_dot<kBF16, RR, TT>(rows, q, H, 64, xs, nullptr, T, nullptr, acc);
 #pragma unroll
                 for (int j = 0; j < RR; ++j) {
                     const int e = it * RR + j;
                     const float b = a.router_b ? bf16_ld(a.router_b, min(e, E - 1)) : 0.f;
 #pragma unroll
                     for (int t = 0; t < TT; ++t)
-                        if (t < T && e < E && lane == t) a.logits[int64_t(t) * a.ld_logits + e] = acc[j][t] + b;
+                        if (t < T && e < E && lane == t) a.logits[int64_t(t) * a.ld_logits + e] = acc[j * TT + t] + b;
                 }
-            } else if (it < n_rg + n_cf) {  // one coefficient-head row (bf16)
+            } else if (it < n_rg + n_cf) {  // one coefficient-head row (bf16), in the router's item shape
                 const int c = it - n_rg;
-                const char* rows[1] = {static_cast<const char*>(a.coef_w) + int64_t(c) * H * 2};
-                const QRow q[1] = {{nullptr, nullptr, nullptr}};
-                float acc[1][TT];
-                dot_reduce<kBF16, 1, TT>(rows, q, H, 64, xs, nullptr, T, acc);
+                const char* rows[RR];
+                QRow q[RR];
+#pragma unroll
+                for (int j = 0; j < RR; ++j) {
+                    rows[j] = static_cast<const char*>(a.coef_w) + int64_t(c) * H * 2;
+                    q[j] = QRow{nullptr, nullptr, nullptr};
+                }
+                float acc[RR * TT];
+                dec_dot<kBF16, RR, TT>(rows, q, H, 64, xs, nullptr, T, nullptr, acc);
                 const float b = bf16_ld(a.coef_b, c);
 #pragma unroll
                 for (int t = 0; t < TT; ++t)
-                    if (t < T && lane == t) a.logits[int64_t(t) * a.ld_logits + E + c] = acc[0][t] + b;
+                    if (t < T && lane == t) a.logits[int64_t(t) * a.ld_logits + E + c] = acc[t] + b;
             } else {  // SU shared gate/up units
                 const int i0 = (it - n_rg - n_cf) * SU;
                 const char* rows[2 * SU];
@@ -187,16 +228,16 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(const DecodeArgs
                     q[j] = dense_q(a.sg_s, a.sg_z, i, H);
                     q[SU + j] = dense_q(a.su_s, a.su_z, i, H);
                 }
-                float acc[2 * SU][TT];
-                if (dq) dot_reduce<kQ4, 2 * SU, TT>(rows, q, H, dg, xs, xsum, T, acc);
-                else dot_reduce<kBF16, 2 * SU, TT>(rows, q, H, 64, xs, nullptr, T, acc);
+                float acc[2 * SU * TT];
+                if (dq) dec_dot<kQ4, 2 * SU, TT>(rows, q, H, dg, xs, xsum, T, nullptr, acc);
+                else dec_dot<kBF16, 2 * SU, TT>(rows, q, H, 64, xs, nullptr, T, nullptr, acc);
 #pragma unroll
                 for (int j = 0; j < SU; ++j)
 #pragma unroll
                     for (int t = 0; t < TT; ++t)
                         if (t < T && i0 + j < Is && lane == t)
                             reinterpret_cast<AT*>(a.hs)[int64_t(t) * Is + i0 + j] = __float2bfloat16_rn(
-                                act_apply(a.act, acc[j][t], acc[SU + j][t], a.limit, a.alpha));
+                                act_apply(a.act, acc[j * TT + t], acc[(SU + j) * TT + t], a.limit, a.alpha));
             }
         }
     }
@@ -204,13 +245,13 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(const DecodeArgs
 
     // ------------------------------------------------------------ phase B
     if (ok) {
-        if (warp < T) {  // top-k of token `warp`, identical in every block
+        {  // top-k of the T tokens, identical in every block
             TopkArgs ta;
             ta.logits = a.logits; ta.ld = a.ld_logits; ta.T = T; ta.E = E; ta.k = k;
             ta.scoring = a.scoring; ta.norm = a.norm; ta.has_sel = a.has_sel; ta.sel_bias = a.sel_bias;
             ta.blend = blend ? 1 : 0;
             ta.idx = sm.sidx; ta.w = sm.sw; ta.coef = sm.scoef;
-            topk_token(ta, warp);
+            topk_block(ta, skeys, sm.sstat);
         }
         __syncthreads();
         // stable counting sort of the S slots by expert (a token's k experts are distinct,
@@ -298,15 +339,15 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(const DecodeArgs
                     }
                 }
             }
-            float acc[2 * BU][TT];
-            dot_reduce<WF, 2 * BU, TT>(rows, q, H, a.group_size, xs, xsum, cnt, acc, tl);
+            float acc[2 * BU * TT];
+            dec_dot<WF, 2 * BU, TT>(rows, q, H, a.group_size, xs, xsum, cnt, tl, acc);
 #pragma unroll
             for (int j = 0; j < BU; ++j)
 #pragma unroll
                 for (int t = 0; t < TT; ++t)
                     if (t < cnt && i0 + j < I && lane == t)
                         reinterpret_cast<AT*>(a.h)[int64_t(sm.sorted[sb + t]) * I + i0 + j] = __float2bfloat16_rn(
-                            act_apply(a.act, acc[j][t] + bg[j], acc[BU + j][t] + bu[j], a.limit, a.alpha));
+                            act_apply(a.act, acc[j * TT + t] + bg[j], acc[(BU + j) * TT + t] + bu[j], a.limit, a.alpha));
         }
         ok = grid_barrier(&a.bar[1], gridDim.x, deadline, a.status, &sm.flag);
     }
@@ -371,8 +412,8 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(const DecodeArgs
                     }
                     bd[jr] = a.has_bias ? bf16_ld(a.down_b, gr) : 0.f;
                 }
-                float acc[DN][TT];
-                dot_reduce<WF, DN, TT>(rows, q, I, a.group_size, hsm, hsum, cnt, acc, tl);
+                float acc[DN * TT];
+                dec_dot<WF, DN, TT>(rows, q, I, a.group_size, hsm, hsum, cnt, tl, acc);
 #pragma unroll
                 for (int jr = 0; jr < DN; ++jr)
 #pragma unroll
@@ -380,7 +421,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(const DecodeArgs
                         const int rl = qq * DN + jr;
                         if (j < cnt && lane == 0 && rl < nr) {
                             const int slot = tl[j];
-                            atomicAdd(&sm.acc_r[rl][slot / k], sm.sw[slot] * (acc[jr][j] + bd[jr]));
+                            atomicAdd(&sm.acc_r[rl][slot / k], sm.sw[slot] * (acc[jr * TT + j] + bd[jr]));
                         }
                     }
             } else {  // SN rows of the shared expert's down projection, every token
@@ -393,15 +434,15 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(const DecodeArgs
                     rows[jr] = static_cast<const char*>(a.sd_w) + r * srb;
                     q[jr] = dense_q(a.sd_s, a.sd_z, r, Is);
                 }
-                float acc[SN][TT];
-                if (dq) dot_reduce<kQ4, SN, TT>(rows, q, Is, dg, hss, hssum, T, acc);
-                else dot_reduce<kBF16, SN, TT>(rows, q, Is, 64, hss, nullptr, T, acc);
+                float acc[SN * TT];
+                if (dq) dec_dot<kQ4, SN, TT>(rows, q, Is, dg, hss, hssum, T, nullptr, acc);
+                else dec_dot<kBF16, SN, TT>(rows, q, Is, 64, hss, nullptr, T, nullptr, acc);
 #pragma unroll
                 for (int jr = 0; jr < SN; ++jr)
 #pragma unroll
                     for (int t = 0; t < TT; ++t) {
                         const int rl = qq * SN + jr;
-                        if (t < T && lane == 0 && rl < nr) sm.acc_s[rl][t] = acc[jr][t];
+                        if (t < T && lane == 0 && rl < nr) sm.acc_s[rl][t] = acc[jr * TT + t];
                     }
             }
         }
@@ -465,7 +506,7 @@ size_t decode_smem_bytes(const DecodeArgs& a) {
     if (a.wf != kBF16 && a.wf != kQ4 && a.wf != kMX4) return 0;
     const size_t S = size_t(a.T) * a.k;
     const bool q4 = a.wf == kQ4;
-    const size_t pa = size_t(a.T) * a.H * 2 + ((q4 || a.dense_q4) ? size_t(a.T) * (a.H / 32) * 4 : 0);
+    const size_t pa = dec_keys_offset(a.T, a.H, q4 || a.dense_q4) + size_t(a.T) * a.E * 8;
     const size_t pc = S * a.I * 2 + (q4 ? S * (a.I / 32) * 4 : 0) + size_t(a.T) * a.Is * 2 +
                       (a.dense_q4 ? size_t(a.T) * (a.Is / 32) * 4 : 0);
     const size_t need = (std::max(pa, pc) + 15) & ~size_t(15);

@@ -139,7 +139,8 @@ size_t decode_smem_bytes(const DecodeArgs& a);
 cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t s);
 
 // ------------------------------------------------------------------ tensor-core GEMM
-constexpr int kTcBN = 128;       // token columns per tile
+constexpr int kTcBN = 128;       // token rows per tile (4-bit weights, small batches)
+constexpr int kTcBNWide = 256;   // token rows per tile of bf16 launches on large batches
 constexpr int kTcRowsGateUp = 128;  // intermediate units per gate/up tile (gate + up rows)
 constexpr int kTcRows = 256;        // output rows per tile of the other GEMMs
 enum { kEpiGateUp = 0, kEpiScatterAdd = 1, kEpiStoreF32 = 2, kEpiStoreAct = 3 };
@@ -149,7 +150,8 @@ struct TcProblem {
     int mode = kEpiStoreF32;
     int M = 0, K = 0, m_blocks = 0;        // m_blocks = ceil(M / rows per tile)
     int grouped = 0;                       // 1: expert groups (offsets / tile_start), 0: one dense group
-    int rows = 0, n_tiles = 0, bn = kTcBN; // dense: token rows and their tiles
+    int rows = 0, n_tiles = 0;             // dense: token rows and their tiles
+    int bn = kTcBN;                        // token rows per tile (the kernel's; checked at launch)
     int num_groups = 0;
     const int32_t* offsets = nullptr;      // [E + 1] sorted-row offsets of the groups
     const int32_t* tile_start = nullptr;   // [E + 1] prefix of token tiles per group
@@ -182,7 +184,7 @@ struct alignas(64) TcParams {
     }
     CUtensorMap a0[2];  // weights (gate / single)
     CUtensorMap a1[2];  // weights (up), gate/up mode with separate planes
-    CUtensorMap b[2][4];  // tokens, boxes of 16, 32, 64 and 128 rows (a tile loads the smallest
+    CUtensorMap b[2][5];  // tokens, boxes of 16, 32, 64, 128 and 256 rows (a tile loads the smallest
                           // box that holds its valid tokens)
     TcProblem p[2];
     int nprob = 0;
@@ -197,7 +199,7 @@ bool tc_weight_map(CUtensorMap* m, const void* w, int E, int R, int K, bool inte
 // row_step 2 views every other row of an interleaved [E, 2R, K / 8] plane from w (gate rows;
 // pass w advanced by one row for the up rows).
 bool tc_q4_weight_map(CUtensorMap* m, const void* w, int E, int R, int K, int row_step = 1);
-// Four maps m[0..3] of the token operand [rows, K] bf16, boxes of 16, 32, 64 and bn rows.
+// Five maps m[0..4] of the token operand [rows, K] bf16, boxes of 16, 32, 64, 128, 256 rows (<= bn).
 bool tc_token_map(CUtensorMap* m, const void* u, int64_t rows, int K, int bn);
 // dst[i] = fp16(src[i]) for n bf16 values (exact within fp16's range), n % 8 == 0.
 cudaError_t launch_to_f16(const void* src, int64_t n, void* dst, cudaStream_t s);

@@ -179,26 +179,35 @@ __device__ __forceinline__ TileInfo decode_tile(const TcParams& P, const GroupTa
 // [packed 0 | packed 1 | B] (TMA), then ASTAGES operand slots of [A0 | A1] (dequantised).
 template <bool GATEUP, int BN, int STAGES, bool Q4 = false>
 struct TcShape {
-    static constexpr int A_BYTES = kBM * kBK * 2;                // 16 KB
-    static constexpr int B_BYTES = BN * kBK * 2;
+    static constexpr int A_BYTES = kBM * kBK * 2;                // 16 KB: one 128-row weight tile
+    static constexpr int B_BYTES = BN * kBK * 2;                 // token tile
     static constexpr int ASTAGES = Q4 ? 2 : 0;                   // dequantised operand slots
     static constexpr int B_OFF = Q4 ? 2 * kPkBytes : 2 * A_BYTES;  // token tile within a stage
     static constexpr int STAGE_BYTES = Q4 ? 2 * kPkBytes + B_BYTES : 2 * A_BYTES + B_BYTES;
     static constexpr int ARING_OFF = STAGES * STAGE_BYTES;       // operand ring (4-bit only)
     static constexpr int RING_BYTES = STAGES * STAGE_BYTES + ASTAGES * 2 * A_BYTES;
-    // epilogue warps: 8 (two per TMEM lane quarter, one column half each), or 4 beside the
-    // dequantising warps (each taking both halves), which keeps the 4-bit block at 14 warps,
-    // at most 4 per SM sub-partition and so 128 registers per thread
+    // epilogue warps: 8, or 4 beside the dequantising warps, which keeps the 4-bit block at
+    // 14 warps, at most 4 per SM sub-partition and so 128 registers per thread
     static constexpr int EPI = Q4 ? 128 : kEpiThreads;
     static constexpr int DQ_BASE = 64 + EPI;                     // first dequantising thread
     static constexpr int THREADS = 64 + EPI + (Q4 ? kDqThreads : 0);
-    static constexpr int ACC_COLS = 2 * BN;                      // per accumulator set
-    static constexpr int TMEM_COLS = 2 * ACC_COLS;               // double-buffered
+    // TMEM: one 128 x 256 fp32 accumulator per 128 token rows of a tile; 128-row tiles keep
+    // two accumulator sets (the epilogue of one tile overlaps the next tile's main loop),
+    // 256-row tiles one set of two (512 columns either way)
+    static constexpr int MH = BN / kBM;                          // 128-row token halves per tile
+    static constexpr int NBUF = MH == 1 ? 2 : 1;                 // accumulator sets
+    static constexpr int ACC_COLS = 2 * kBM;                     // columns of one accumulator
+    static constexpr int TMEM_COLS = ACC_COLS * MH * NBUF;
     static constexpr int ROWS = GATEUP ? kBM : 2 * kBM;          // weight rows per tile
-    static constexpr int SMEM = RING_BYTES + 1024 /*align*/ + 256 /*barriers*/ + int(sizeof(GroupTables)) +
-                                8 * 128 * 4 /*epilogue bias tables*/;
-    static_assert(TMEM_COLS <= 512 && (TMEM_COLS & (TMEM_COLS - 1)) == 0, "TMEM columns");
-    static_assert(BN % 32 == 0 && BN >= 32 && BN <= 256, "BN");
+    // epilogue layout: the warps of each token half cover its 128 rows (lane quarters) and
+    // the 256 columns in NH column halves each
+    static constexpr int EPI_WARPS_PER_HALF = EPI / 32 / MH;
+    static constexpr int NH = EPI_WARPS_PER_HALF == 4 ? 2 : 1;
+    static constexpr int BIAS_BYTES = (EPI / 32) * 128 * NH * 4;
+    static constexpr int SMEM = RING_BYTES + 1024 /*align*/ + 256 /*barriers*/ + int(sizeof(GroupTables)) + BIAS_BYTES;
+    static_assert(TMEM_COLS == 512, "TMEM columns");
+    static_assert(BN == 128 || (BN == 256 && !Q4), "token tile");
+    static_assert(EPI_WARPS_PER_HALF == 4 || EPI_WARPS_PER_HALF == 8, "epilogue warps");
     static_assert(STAGE_BYTES % 1024 == 0 && B_OFF % 1024 == 0, "swizzle atoms stay 1 KB aligned");
     static_assert((2 * STAGES + 5 + 2 * ASTAGES) * 8 + 4 <= 256, "barriers fit their region");
     static_assert(SMEM <= 232448, "dynamic shared memory per block");
@@ -337,7 +346,7 @@ __global__ void __launch_bounds__(TcShape<GATEUP, BN, STAGES, Q4>::THREADS, 1)
         for (int i = 0; i < P.nprob; ++i) {
             prefetch_tmap(&P.a0[i]);
             if (GATEUP && !P.p[i].interleaved) prefetch_tmap(&P.a1[i]);
-            for (int v = 0; v < 4; ++v) prefetch_tmap(&P.b[i][v]);
+            for (int v = 0; v < 5; ++v) prefetch_tmap(&P.b[i][v]);
         }
     }
     pdl_begin();  // everything above touches no memory that earlier kernels write
@@ -373,8 +382,8 @@ __global__ void __launch_bounds__(TcShape<GATEUP, BN, STAGES, Q4>::THREADS, 1)
             const TcProblem& p = P.p[ti.prob];
             const int nk = p.K / kBK;
             const int mrow = ti.mb * S::ROWS;
-            // token rows: the smallest box (16, 32, 64, BN) that holds the valid tokens
-            const int bv = ti.nvalid <= 16 ? 0 : ti.nvalid <= 32 ? 1 : ti.nvalid <= 64 ? 2 : 3;
+            // token rows: the smallest box (16, 32, 64, 128, 256 rows) that holds the valid tokens
+            const int bv = ti.nvalid <= 16 ? 0 : ti.nvalid <= 32 ? 1 : ti.nvalid <= 64 ? 2 : ti.nvalid <= 128 ? 3 : 4;
             const uint32_t b_bytes = uint32_t(min(BN, 16 << bv)) * kBK * 2;
             for (int kb = 0; kb < nk; ++kb) {
                 int ok = 1;
@@ -429,13 +438,14 @@ __global__ void __launch_bounds__(TcShape<GATEUP, BN, STAGES, Q4>::THREADS, 1)
             for (int tile = blockIdx.x; tile < total && !timed_out; tile += gridDim.x, ++it) {
                 const TileInfo ti = decode_tile(P, gt, tile, t0);
                 const TcProblem& p = P.p[ti.prob];
-                const uint32_t ab = it & 1u, aph = (it >> 1) & 1u;
+                const uint32_t ab = it % S::NBUF, aph = (it / S::NBUF) & 1u;
                 if (!mbar_wait(&acc_empty[ab], aph ^ 1u, deadline)) {
                     timed_out = true;
                     break;
                 }
                 tc_fence_after();
-                const uint32_t d0 = tmem_base + ab * S::ACC_COLS;
+                const uint32_t d0 = tmem_base + ab * S::MH * S::ACC_COLS;
+                const int nh = S::MH == 2 && ti.nvalid > kBM ? 2 : 1;  // token halves with valid rows
                 const uint32_t idesc = (Q4 && p.q4 && !p.mx) ? idesc_h : idesc_b;
                 const int nk = p.K / kBK;
                 for (int kb = 0; kb < nk; ++kb) {
@@ -451,8 +461,12 @@ __global__ void __launch_bounds__(TcShape<GATEUP, BN, STAGES, Q4>::THREADS, 1)
                                            : su32(smem + stage * S::STAGE_BYTES);
                     const uint32_t st = su32(smem + stage * S::STAGE_BYTES + S::B_OFF);
 #pragma unroll
-                    for (int k = 0; k < kBK / 16; ++k)
-                        umma(d0, smem_desc(st + k * 32), smem_desc(sw + k * 32), idesc, (kb > 0 || k > 0) ? 1u : 0u);
+                    for (int k = 0; k < kBK / 16; ++k) {
+                        const uint32_t acc = (kb > 0 || k > 0) ? 1u : 0u;
+                        umma(d0, smem_desc(st + k * 32), smem_desc(sw + k * 32), idesc, acc);
+                        if (S::MH == 2 && nh == 2)  // token rows 128..255 (16 KB further), same weights
+                            umma(d0 + S::ACC_COLS, smem_desc(st + kBM * 128 + k * 32), smem_desc(sw + k * 32), idesc, acc);
+                    }
                     umma_commit(&empty[stage]);
                     if (++stage == STAGES) {
                         stage = 0;
@@ -538,50 +552,65 @@ __global__ void __launch_bounds__(TcShape<GATEUP, BN, STAGES, Q4>::THREADS, 1)
                 sp[ai] = static_cast<const unsigned char*>((GATEUP && a == 1) ? p.qs1 : p.qs0) + off * (p.mx ? 1 : 2);
                 zp[ai] = p.mx ? nullptr : static_cast<const unsigned char*>((GATEUP && a == 1) ? p.qz1 : p.qz0) + off * 2;
             }
-            // (scale, bias) of each tile for the first and second half of K block kb (two
-            // groups per block when group_size is 32, else the same group twice); MXFP4: one
-            // E8M0 byte per block of 32 at the same offsets, the pair carrying 2^(byte - 127) twice
-            // the K loop is instantiated per format, so that no format test sits in it
+            // (scale, bias) of each tile for the two 32-wide halves of K block kb. The raw words
+            // are loaded kPre blocks ahead into a register ring whose slots are indexed
+            // statically (the K loop is unrolled kPre times), and converted only when their
+            // block is dequantised, so that no instruction waits on a load issued since.
+            // Group 32: one 32-bit word holds the two groups of the block (scales, then
+            // biases; MXFP4: a 16-bit word of the two E8M0 bytes); larger groups: one 16-bit
+            // value serves both halves.
+            const bool two = p.group_size == 32;
             auto run = [&](auto mx_tag) {
             constexpr bool MX = decltype(mx_tag)::value;
-            auto load_sb = [&](int kb, __nv_bfloat162 (&o)[DT][2]) {
+            auto load_raw = [&](int kb, uint32_t (&rs)[DT], uint32_t (&rz)[DT]) {
+                const int g = (kb * kBK) / p.group_size;
+#pragma unroll
+                for (int ai = 0; ai < DT; ++ai) {
+                    if constexpr (MX) {
+                        rs[ai] = __ldg(reinterpret_cast<const unsigned short*>(sp[ai] + g));
+                        rz[ai] = 0;
+                    } else if (two) {
+                        rs[ai] = __ldg(reinterpret_cast<const unsigned int*>(sp[ai]) + g / 2);
+                        rz[ai] = __ldg(reinterpret_cast<const unsigned int*>(zp[ai]) + g / 2);
+                    } else {
+                        rs[ai] = __ldg(reinterpret_cast<const unsigned short*>(sp[ai]) + g);
+                        rz[ai] = __ldg(reinterpret_cast<const unsigned short*>(zp[ai]) + g);
+                    }
+                }
+            };
+            // raw words -> the pair used by the dequantisation of half h: (scale, bias) as an
+            // fp16 pair in one 32-bit register, or MXFP4's 2^(byte - 127) twice as bf16
+            auto convert = [&](const uint32_t (&rs)[DT], const uint32_t (&rz)[DT], __nv_bfloat162 (&o)[DT][2]) {
 #pragma unroll
                 for (int ai = 0; ai < DT; ++ai)
 #pragma unroll
                     for (int h = 0; h < 2; ++h) {
-                        const int g = (kb * kBK + h * 32) / p.group_size;
                         if constexpr (MX) {
-                            const uint32_t sbyte = __ldg(sp[ai] + g);
+                            const uint32_t sbyte = (rs[ai] >> (8 * h)) & 0xFFu;
                             const __nv_bfloat16 sc = __ushort_as_bfloat16(uint16_t(sbyte ? (sbyte << 7) : 0x0040u));
                             o[ai][h] = __halves2bfloat162(sc, sc);
-                        } else {  // (scale, bias) as an fp16 pair, kept in the same 32-bit register
+                        } else {
+                            const int sh = (two && h == 1) ? 16 : 0;
                             const __half2 sz = __floats2half2_rn(
-                                __bfloat162float(__ldg(reinterpret_cast<const __nv_bfloat16*>(sp[ai]) + g)),
-                                __bfloat162float(__ldg(reinterpret_cast<const __nv_bfloat16*>(zp[ai]) + g)));
+                                __bfloat162float(__ushort_as_bfloat16(uint16_t(rs[ai] >> sh))),
+                                __bfloat162float(__ushort_as_bfloat16(uint16_t(rz[ai] >> sh))));
                             o[ai][h] = *reinterpret_cast<const __nv_bfloat162*>(&sz);
                         }
                     }
             };
-            // a ring of the next kPre K blocks' pairs in registers, refilled kPre blocks ahead
-            // (the pairs come from DRAM the first time a tile row is read)
             constexpr int kPre = 8;
-            __nv_bfloat162 qr[kPre][DT][2];
+            uint32_t rs[kPre][DT], rz[kPre][DT];
 #pragma unroll
             for (int j = 0; j < kPre; ++j)
-                if (j < nk) load_sb(j, qr[j]);
-            for (int kb = 0; kb < nk; ++kb) {
+                if (j < nk) load_raw(j, rs[j], rz[j]);
+            for (int kb0 = 0; kb0 < nk && !timed_out; kb0 += kPre) {
+#pragma unroll
+            for (int j = 0; j < kPre; ++j) {
+                const int kb = kb0 + j;
+                if (kb >= nk) break;
                 __nv_bfloat162 q0[DT][2];
-#pragma unroll
-                for (int ai = 0; ai < DT; ++ai)
-#pragma unroll
-                    for (int h = 0; h < 2; ++h) q0[ai][h] = qr[0][ai][h];
-#pragma unroll
-                for (int j = 0; j + 1 < kPre; ++j)
-#pragma unroll
-                    for (int ai = 0; ai < DT; ++ai)
-#pragma unroll
-                        for (int h = 0; h < 2; ++h) qr[j][ai][h] = qr[j + 1][ai][h];
-                if (kb + kPre < nk) load_sb(kb + kPre, qr[kPre - 1]);
+                convert(rs[j], rz[j], q0);
+                if (kb + kPre < nk) load_raw(kb + kPre, rs[j], rz[j]);  // this slot's next block
                 if (!mbar_wait(&full[stage], phase, deadline) || !mbar_wait(&aempty[astage], aphase ^ 1u, deadline)) {
                     timed_out = true;
                     break;
@@ -613,6 +642,7 @@ __global__ void __launch_bounds__(TcShape<GATEUP, BN, STAGES, Q4>::THREADS, 1)
                 if (lane == 0) mbar_arrive(&dq[astage]);
                 next();
             }
+            }
             };
             if (p.mx) run(std::true_type{});
             else run(std::false_type{});
@@ -632,16 +662,17 @@ __global__ void __launch_bounds__(TcShape<GATEUP, BN, STAGES, Q4>::THREADS, 1)
         // (columns 128..255) block. Each warp stages the biases of its own columns in a
         // warp-private slice of shared memory, so that no epilogue step waits on another warp.
         const int q = warp & 3;
-        const int tok = q * 32 + lane;  // token row of the tile
         const int eid = threadIdx.x - 64;
-        constexpr int NH = S::EPI == kEpiThreads ? 1 : 2;  // column halves per warp
+        const int th = S::MH == 2 ? (eid >= 128 ? 1 : 0) : 0;  // token half of this warp
+        const int tok = th * kBM + q * 32 + lane;               // token row of the tile
+        constexpr int NH = S::NH;                               // column halves per warp
         const int h_lo = NH == 1 ? (eid >= 128 ? 1 : 0) : 0;
         float* sb = sbias + (eid >> 5) * 128 * NH;  // this warp's column biases (warp-private)
         uint32_t it = 0;
         for (int tile = blockIdx.x; tile < total; tile += gridDim.x, ++it) {
             const TileInfo ti = decode_tile(P, gt, tile, t0);
             const TcProblem& p = P.p[ti.prob];
-            const uint32_t ab = it & 1u, aph = (it >> 1) & 1u;
+            const uint32_t ab = it % S::NBUF, aph = (it / S::NBUF) & 1u;
             const bool tv = tok < ti.nvalid;
             const int64_t prow = int64_t(ti.row0) + tok;
             float wslot = 0.f;
@@ -683,7 +714,7 @@ __global__ void __launch_bounds__(TcShape<GATEUP, BN, STAGES, Q4>::THREADS, 1)
                 break;
             }
             tc_fence_after();
-            const uint32_t tb = tmem_base + (uint32_t(q * 32) << 16) + ab * S::ACC_COLS;
+            const uint32_t tb = tmem_base + (uint32_t(q * 32) << 16) + (ab * S::MH + th) * S::ACC_COLS;
             auto release = [&]() {  // the accumulator set is free for the tile after next
                 tc_fence_before();
                 __syncwarp();
@@ -878,11 +909,12 @@ bool tc_weight_map(CUtensorMap* m, const void* w, int E, int R, int K, bool inte
     return encode(m, w, 3, dims, strides, box);
 }
 
-// Token operand: [rows, K] bf16, maps m[0..3] with boxes of 16, 32, 64 and bn rows.
+// Token operand: [rows, K] bf16, maps m[0..4] with boxes of 16, 32, 64, 128 and 256 rows
+// (at most bn).
 bool tc_token_map(CUtensorMap* m, const void* u, int64_t rows, int K, int bn) {
     const cuuint64_t dims[2] = {cuuint64_t(K), cuuint64_t(rows)};
     const cuuint64_t strides[1] = {cuuint64_t(K) * 2};
-    for (int v = 0; v < 4; ++v) {
+    for (int v = 0; v < 5; ++v) {
         const cuuint32_t box[2] = {kBK, cuuint32_t(std::min(bn, 16 << v))};
         if (!encode(&m[v], u, 2, dims, strides, box)) return false;
     }
@@ -901,10 +933,20 @@ bool tc_q4_weight_map(CUtensorMap* m, const void* w, int E, int R, int K, int ro
 cudaError_t launch_tc_gemm(TcParams& P, bool gateup, int64_t max_tiles, cudaStream_t s) {
     bool q4 = false;
     for (int i = 0; i < P.nprob; ++i) q4 = q4 || P.p[i].q4;
+    // the tile lists (dense tile counts, the permutation's tile prefix) were built for one
+    // tile height, which picks the kernel: 128 rows with 4-bit weights or bf16, 256 with bf16
+    const int bn = P.p[0].bn;
+    for (int i = 0; i < P.nprob; ++i)
+        if (P.p[i].bn != bn || (q4 && bn != kTcBN) || (bn != kTcBN && bn != kTcBNWide)) return cudaErrorInvalidValue;
     if (q4) {  // six load slots (packed tiles + token tile) feed two dequantised operand slots
         if (gateup) return launch_tc_t<true, kTcBN, 6, true>(P, max_tiles, s);
         return launch_tc_t<false, kTcBN, 6, true>(P, max_tiles, s);
     }
+    if (bn == kTcBNWide) {  // 256-token tiles, three 64 KB stages
+        if (gateup) return launch_tc_t<true, kTcBNWide, 3, false>(P, max_tiles, s);
+        return launch_tc_t<false, kTcBNWide, 3, false>(P, max_tiles, s);
+    }
+    // 128-token tiles, four 48 KB stages
     if (gateup) return launch_tc_t<true, kTcBN, 4, false>(P, max_tiles, s);
     return launch_tc_t<false, kTcBN, 4, false>(P, max_tiles, s);
 }

@@ -276,6 +276,9 @@ TC_SMALL = [  # tensor-core path forced: ragged groups, partial tiles, interleav
     (ts.Q4_INTERLEAVED, 3),
     (ts.DENSE_Q4, 9),          # router, latent projections and experts on the tensor cores, 4-bit dense
     (inputs.KLEAR_Q4_DENSE, 70),
+    (ts.WIDE, 700),            # 256-token tiles: full, 129..256 and <= 128 valid rows
+    (ts.WIDE, 300),
+    (ts.LATENT_WIDE, 600),
 ]
 
 
@@ -479,7 +482,7 @@ def test_grid_barrier_wait_reports_a_timeout_and_the_next_decode_works(monkeypat
 
 
 EP_CASES = [(inputs.KLEAR_BF16, 200), (inputs.KLEAR_BF16, 5), (inputs.KLEAR_Q4, 64),
-            (inputs.CLAMPED_MXFP4_NATIVE, 40), (ts.SIG_BLEND, 9)]
+            (inputs.CLAMPED_MXFP4_NATIVE, 40), (ts.SIG_BLEND, 9), (ts.WIDE, 700)]
 
 
 @pytest.mark.parametrize("spec,T", EP_CASES, ids=[f"{s.name}-T{T}" for s, T in EP_CASES])
