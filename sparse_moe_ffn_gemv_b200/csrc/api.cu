@@ -78,11 +78,20 @@ bool dense_q4(const moe_config* c) { return c->dense_format == MOE_DTYPE_Q4_AFFI
 // launches of large batches, where a weight tile then serves twice the token rows (an expert
 // with 129..256 routed rows reads its weights once instead of twice). The expert launches
 // carry the routed and the shared problem, the dense launches one projection.
+// Wide tiles keep one accumulator set (the epilogue of a tile no longer overlaps the next
+// tile's main loop), so they pay only where most experts hold more than 128 routed rows
+// (measured: latent block at 8192 tokens, 170 rows per expert on average, expert gate/up
+// 2.97 -> 2.63 ms; Klear at 4096 tokens, 128 on average, block 0.71 -> 0.78 ms), and in dense
+// launches that still give every SM two tiles or more (a router of 384 rows at 8192 tokens has
+// 64 wide tiles: 84 -> 113 us).
 int expert_bn(const moe_config* c, int64_t T) {
     const bool q = c->weight_format == MOE_DTYPE_Q4_AFFINE || c->weight_format == MOE_DTYPE_MXFP4 || dense_q4(c);
-    return !q && T * c->top_k >= 64 * int64_t(c->num_experts) ? kTcBNWide : kTcBN;
+    return !q && T * c->top_k >= 160 * int64_t(c->num_experts) ? kTcBNWide : kTcBN;
 }
-int dense_bn(const moe_config* c, int64_t T) { return !dense_q4(c) && T >= 256 ? kTcBNWide : kTcBN; }
+int dense_bn(const moe_config* c, int64_t T, int M) {
+    const int64_t wide_tiles = int64_t((M + kTcRows - 1) / kTcRows) * ((T + kTcBNWide - 1) / kTcBNWide);
+    return !dense_q4(c) && wide_tiles >= 2 * int64_t(device_sm_count()) ? kTcBNWide : kTcBN;
+}
 
 // Weight operand(s) of a dense (one-group) tensor-core problem: bf16 [M, K], or 4-bit affine
 // words [M, K / 8] with bf16 scales / biases per dense_group_size columns (the second
@@ -405,7 +414,7 @@ moe_status run_route(const moe_config* c, const moe_weights* w, const void* x, i
             p.K = c->hidden;
             p.m_blocks = (p.M + kTcRows - 1) / kTcRows;
             p.rows = int(T);
-            p.bn = dense_bn(c, T);  // a 4-bit router never runs here
+            p.bn = dense_bn(c, T, c->num_experts);  // both problems: one tile height
             p.n_tiles = int((T + p.bn - 1) / p.bn);
             p.bias0 = i == 0 ? r.b0 : r.b1;
             p.out = at<float>(ws, L.logits) + (i == 0 ? 0 : c->num_experts);
@@ -735,7 +744,7 @@ moe_status run_latent_down(const moe_config* c, const moe_weights* w, const void
         TcProblem& p = P.p[0];
         p.mode = kEpiStoreAct;
         p.M = c->latent_dim; p.K = c->hidden; p.m_blocks = (p.M + kTcRows - 1) / kTcRows;
-        p.bn = dense_bn(c, T);
+        p.bn = dense_bn(c, T, p.M);
         p.rows = int(T); p.n_tiles = int((T + p.bn - 1) / p.bn);
         p.out = z; p.ld_out = c->latent_dim;
         const void* xt = x;
@@ -797,7 +806,7 @@ moe_status run_output(const moe_config* c, const moe_weights* w, RoutedSum rs, c
         TcProblem& p = P.p[0];
         p.mode = kEpiStoreAct;
         p.M = c->hidden; p.K = c->latent_dim; p.m_blocks = (p.M + kTcRows - 1) / kTcRows;
-        p.bn = dense_bn(c, T);
+        p.bn = dense_bn(c, T, p.M);
         p.rows = int(T); p.n_tiles = int((T + p.bn - 1) / p.bn);
         p.out = y; p.ld_out = c->hidden;
         p.addend = s_acc; p.ld_add = c->hidden;

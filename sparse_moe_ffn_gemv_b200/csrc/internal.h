@@ -139,6 +139,7 @@ size_t decode_smem_bytes(const DecodeArgs& a);
 cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t s);
 
 // ------------------------------------------------------------------ tensor-core GEMM
+int device_sm_count();          // SMs of the current device (148 if the query fails)
 constexpr int kTcBN = 128;       // token rows per tile (4-bit weights, small batches)
 constexpr int kTcBNWide = 256;   // token rows per tile of bf16 launches on large batches
 constexpr int kTcRowsGateUp = 128;  // intermediate units per gate/up tile (gate + up rows)

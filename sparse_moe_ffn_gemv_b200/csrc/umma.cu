@@ -874,11 +874,7 @@ bool encode(CUtensorMap* m, const void* base, int rank, const cuuint64_t* dims, 
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-int sm_count() {
-    int dev = 0, n = 148;
-    if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
-    return n;
-}
+int sm_count() { return device_sm_count(); }
 
 template <bool GATEUP, int BN, int STAGES, bool Q4>
 cudaError_t launch_tc_t(TcParams& P, int64_t max_tiles, cudaStream_t s) {
@@ -928,6 +924,12 @@ bool tc_q4_weight_map(CUtensorMap* m, const void* w, int E, int R, int K, int ro
     const cuuint64_t strides[2] = {cuuint64_t(K / 8) * 4 * row_step, cuuint64_t(R) * (K / 8) * 4 * row_step};
     const cuuint32_t box[3] = {8, kBM, 1};
     return encode(m, w, 3, dims, strides, box, CU_TENSOR_MAP_DATA_TYPE_UINT32, CU_TENSOR_MAP_SWIZZLE_NONE);
+}
+
+int device_sm_count() {
+    int dev = 0, n = 148;
+    if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    return n;
 }
 
 cudaError_t launch_tc_gemm(TcParams& P, bool gateup, int64_t max_tiles, cudaStream_t s) {

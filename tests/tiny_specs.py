@@ -64,15 +64,17 @@ DENSE_Q4_BLEND = Q4.replace(name="t_dense_q4_blend", config_id=112, dense_format
 
 # bf16 shapes on which a few hundred tokens give the tensor-core launches 256-token tiles with
 # ragged halves: experts holding 129..256 and more than 256 routed rows, dense tails of 188
-# rows (clamped family with biases and the blend head; latent block with the add)
+# rows (clamped family with biases and the blend head; latent block with the add, wide enough
+# that its three bf16 intermediates z, h and the normalised latent stay inside the bar: at
+# hidden 128 / latent 128 their roundings alone reach 0.022 rms)
 WIDE = MoeSpec(
     name="t_wide", config_id=113, hidden=128, num_experts=4, top_k=2, intermediate=128,
     scoring="softmax_topk", activation="swiglu_clamped", gate_up_interleaved=True,
     has_expert_bias=True, shared_mode="blend", shared_intermediate=64)
 LATENT_WIDE = MoeSpec(
-    name="t_latent_wide", config_id=114, hidden=128, num_experts=6, top_k=2, intermediate=64,
+    name="t_latent_wide", config_id=114, hidden=512, num_experts=6, top_k=2, intermediate=128,
     scoring="sigmoid", has_selection_bias=True, norm_topk_prob=True, shared_mode="add",
-    shared_intermediate=64, latent_dim=128, latent_use_norm=True)
+    shared_intermediate=128, latent_dim=256, latent_use_norm=True)
 
 ALL = [inputs.TINY_F32, SIG_BLEND, CLAMPED, Q4, LATENT, ROUTER_BIAS, SEPARATE_BIAS,
        LATENT_NONORM, MXFP4, MXFP4_NATIVE, Q4_INTERLEAVED, DENSE_Q4, DENSE_Q4_BLEND]
