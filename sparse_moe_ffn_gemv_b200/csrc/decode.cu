@@ -51,6 +51,7 @@ struct DecSmem {
     int n_d;                     // number of distinct experts
     int flag;
     float sstat[2 * kTT];        // softmax over all experts: each token's max and 1 / sum
+    float ssel[kMaxExperts];     // select-only biases, staged in phase A
     float acc_r[kDecRowsMax][kTT];  // routed sum of the block's rows
     float acc_s[kDecRowsMax][kTT];  // shared expert output of the block's rows
 };
@@ -83,21 +84,25 @@ __device__ __forceinline__ void copy_cg(uint4* dst, const void* src, int64_t n16
     for (int64_t i = threadIdx.x; i < n16; i += blockDim.x) dst[i] = __ldcg(s + i);
 }
 
-// Rows per warp item. With one token the accumulators are few, so a warp keeps several rows
-// (two gate/up units, four down rows) in flight; with up to 8 tokens one unit / two rows.
-// Every phase of one format uses the same row count, so that it runs the same code.
+// Rows per warp item and 16-byte vectors in flight per row and lane. With one token the
+// accumulators are few: phases A and B take two rows (one gate/up unit) per item with a whole
+// 2048-wide bf16 row in flight per lane pair of loads (U = 8: one round trip per item), phase
+// C four down rows. With up to 8 tokens: two rows everywhere. Every phase of one format uses
+// the same shape, so that it runs the same code.
 template <int WF, int TT> struct DecShape {
     static constexpr bool ONE = TT == 1;
-    static constexpr int ND = ONE ? 4 : 2;                          // bf16 dense rows per item
-    static constexpr int RR = ND;                                   // router / coefficient rows
-    static constexpr int SU = ND / 2;                               // shared gate/up units
-    static constexpr int SN = ND;                                   // shared down rows
-    static constexpr int BU = (ONE && WF == kBF16) ? 2 : 1;         // routed gate/up units
-    static constexpr int DN = 2 * BU;                               // routed down rows
+    static constexpr int RR = 2;                                    // router / coefficient rows
+    static constexpr int SU = 1;                                    // shared gate/up units
+    static constexpr int BU = 1;                                    // routed gate/up units
+    static constexpr int UA = ONE ? 8 : Fmt<kBF16>::U;              // bf16 rows, phases A and B
+    static constexpr int UB = (ONE && WF == kBF16) ? 8 : Fmt<WF>::U;  // routed gate/up rows
+    static constexpr int DN = (ONE && WF == kBF16) ? 4 : 2;         // routed down rows
+    static constexpr int SN = ONE ? 4 : 2;                          // shared down rows
+    static constexpr int UC = Fmt<WF>::U;                           // routed down rows, phase C
 };
 
 // acc[r][t] = sum over the row of W_r . u_t, reduced over the warp (every lane holds it).
-template <int WF, int NR, int TT>
+template <int WF, int NR, int TT, int U = Fmt<WF>::U>
 __device__ __forceinline__ void dot_reduce(const char* const (&rows)[NR], const QRow (&q)[NR], int K, int gs,
                                            const __nv_bfloat16* us, const float* usum, int tt, float (&acc)[NR][TT],
                                            const int* tl = nullptr) {
@@ -105,7 +110,7 @@ __device__ __forceinline__ void dot_reduce(const char* const (&rows)[NR], const 
     for (int r = 0; r < NR; ++r)
 #pragma unroll
         for (int t = 0; t < TT; ++t) acc[r][t] = 0.f;
-    dot_rows<WF, NR, TT>(rows, q, K, gs, us, usum, tt, acc, tl);
+    dot_rows<WF, NR, TT, U>(rows, q, K, gs, us, usum, tt, acc, tl);
 #pragma unroll
     for (int r = 0; r < NR; ++r)
 #pragma unroll
@@ -119,7 +124,7 @@ __device__ __forceinline__ void dot_reduce(const char* const (&rows)[NR], const 
 // every phase runs the same instructions. The kernel runs each phase once per SM after an L2
 // flush could have evicted its code, so distinct instructions cost instruction-cache misses;
 // the call's argument traffic (a few words of local memory) is paid once per item.
-template <int WF, int NR, int TT>
+template <int WF, int NR, int TT, int U = Fmt<WF>::U>
 __device__ __noinline__ void dec_dot(const char* const* rows, const QRow* q, int K, int gs,
                                      const __nv_bfloat16* us, const float* usum, int tt, const int* tl,
                                      float* out) {
@@ -131,7 +136,7 @@ __device__ __noinline__ void dec_dot(const char* const* rows, const QRow* q, int
         qq[j] = q[j];
     }
     float acc[NR][TT];
-    dot_reduce<WF, NR, TT>(r, qq, K, gs, us, usum, tt, acc, tl);
+    dot_reduce<WF, NR, TT, U>(r, qq, K, gs, us, usum, tt, acc, tl);
 #pragma unroll
     for (int j = 0; j < NR; ++j)
 #pragma unroll
@@ -143,6 +148,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(const DecodeArgs
     using AT = __nv_bfloat16;
     using Sh = DecShape<WF, TT>;
     constexpr int DN = Sh::DN, SN = Sh::SN, RR = Sh::RR, SU = Sh::SU, BU = Sh::BU;
+    constexpr int UA = Sh::UA, UB = Sh::UB, UC = Sh::UC;
     extern __shared__ uint4 dsm[];
     __shared__ DecSmem sm;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -171,6 +177,8 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(const DecodeArgs
     float* xsum = reinterpret_cast<float*>(xs + int64_t(T) * H);  // 4-bit affine: sums per 32
     // selection keys of the top-k (phase B), after the staged tokens and their sums
     uint64_t* skeys = reinterpret_cast<uint64_t*>(dsm) + dec_keys_offset(T, H, WF == kQ4 || dq) / 8;
+    if (a.has_sel)
+        for (int e = threadIdx.x; e < E; e += blockDim.x) sm.ssel[e] = __ldg(a.sel_bias + e);
     if (WF == kQ4 || dq) stage_tokens<kQ4>(a.x, H, 0, T, nullptr, 1, xs, xsum);
     else stage_tokens<kBF16>(a.x, H, 0, T, nullptr, 1, xs, nullptr);
     if (a.l2_prefetch && Is && threadIdx.x == 0 && nr > 0)
@@ -192,7 +200,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(const DecodeArgs
                 }
                 float acc[RR * TT];
                 if (dq) dec_dot<kQ4, RR, TT>(rows, q, H, dg, xs, xsum, T, nullptr, acc);
-                else dec_dot<kBF16, RR, TT>(rows, q, H, 64, xs, nullptr, T, nullptr, acc);
+                else dec_dot<kBF16, RR, TT, UA>(rows, q, H, 64, xs, nullptr, T, nullptr, acc);
 #pragma unroll
                 for (int j = 0; j < RR; ++j) {
                     const int e = it * RR + j;
@@ -211,7 +219,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(const DecodeArgs
                     q[j] = QRow{nullptr, nullptr, nullptr};
                 }
                 float acc[RR * TT];
-                dec_dot<kBF16, RR, TT>(rows, q, H, 64, xs, nullptr, T, nullptr, acc);
+                dec_dot<kBF16, RR, TT, UA>(rows, q, H, 64, xs, nullptr, T, nullptr, acc);
                 const float b = bf16_ld(a.coef_b, c);
 #pragma unroll
                 for (int t = 0; t < TT; ++t)
@@ -230,7 +238,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(const DecodeArgs
                 }
                 float acc[2 * SU * TT];
                 if (dq) dec_dot<kQ4, 2 * SU, TT>(rows, q, H, dg, xs, xsum, T, nullptr, acc);
-                else dec_dot<kBF16, 2 * SU, TT>(rows, q, H, 64, xs, nullptr, T, nullptr, acc);
+                else dec_dot<kBF16, 2 * SU, TT, UA>(rows, q, H, 64, xs, nullptr, T, nullptr, acc);
 #pragma unroll
                 for (int j = 0; j < SU; ++j)
 #pragma unroll
@@ -251,7 +259,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(const DecodeArgs
             ta.scoring = a.scoring; ta.norm = a.norm; ta.has_sel = a.has_sel; ta.sel_bias = a.sel_bias;
             ta.blend = blend ? 1 : 0;
             ta.idx = sm.sidx; ta.w = sm.sw; ta.coef = sm.scoef;
-            topk_block(ta, skeys, sm.sstat);
+            topk_block(ta, skeys, sm.sstat, sm.ssel, reinterpret_cast<float*>(skeys + T * E));
         }
         __syncthreads();
         // stable counting sort of the S slots by expert (a token's k experts are distinct,
@@ -340,7 +348,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(const DecodeArgs
                 }
             }
             float acc[2 * BU * TT];
-            dec_dot<WF, 2 * BU, TT>(rows, q, H, a.group_size, xs, xsum, cnt, tl, acc);
+            dec_dot<WF, 2 * BU, TT, UB>(rows, q, H, a.group_size, xs, xsum, cnt, tl, acc);
 #pragma unroll
             for (int j = 0; j < BU; ++j)
 #pragma unroll
@@ -413,7 +421,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(const DecodeArgs
                     bd[jr] = a.has_bias ? bf16_ld(a.down_b, gr) : 0.f;
                 }
                 float acc[DN * TT];
-                dec_dot<WF, DN, TT>(rows, q, I, a.group_size, hsm, hsum, cnt, tl, acc);
+                dec_dot<WF, DN, TT, UC>(rows, q, I, a.group_size, hsm, hsum, cnt, tl, acc);
 #pragma unroll
                 for (int jr = 0; jr < DN; ++jr)
 #pragma unroll
@@ -506,7 +514,7 @@ size_t decode_smem_bytes(const DecodeArgs& a) {
     if (a.wf != kBF16 && a.wf != kQ4 && a.wf != kMX4) return 0;
     const size_t S = size_t(a.T) * a.k;
     const bool q4 = a.wf == kQ4;
-    const size_t pa = dec_keys_offset(a.T, a.H, q4 || a.dense_q4) + size_t(a.T) * a.E * 8;
+    const size_t pa = dec_keys_offset(a.T, a.H, q4 || a.dense_q4) + size_t(a.T) * a.E * 12;  // keys + logits
     const size_t pc = S * a.I * 2 + (q4 ? S * (a.I / 32) * 4 : 0) + size_t(a.T) * a.Is * 2 +
                       (a.dense_q4 ? size_t(a.T) * (a.Is / 32) * 4 : 0);
     const size_t need = (std::max(pa, pc) + 15) & ~size_t(15);

@@ -37,8 +37,9 @@ struct QRow {  // 4-bit companions of one row
 };
 
 // acc[r][t] += sum_c W_r[c] * u_t[c] for NR rows and tt (<= kTT) staged tokens; u_t is row
-// t of `us` (rows of K values), or row tl[t] when a token list is given.
-template <int WF, int NR, int TT = kTT>
+// t of `us` (rows of K values), or row tl[t] when a token list is given. U: 16-byte vectors
+// per row in flight per lane.
+template <int WF, int NR, int TT = kTT, int U = Fmt<WF>::U>
 __device__ __forceinline__ void dot_rows(const char* const (&rows)[NR], const QRow (&q)[NR], int K,
                                          int group_size, const typename Fmt<WF>::AT* us,
                                          const float* xsum, int tt, float (&acc)[NR][TT],
@@ -47,17 +48,17 @@ __device__ __forceinline__ void dot_rows(const char* const (&rows)[NR], const QR
     using AT = typename F::AT;
     const int lane = threadIdx.x & 31;
     const int nvec = K / F::VE;
-    for (int base = lane; base < nvec; base += 32 * F::U) {
-        uint4 wv[NR][F::U];
+    for (int base = lane; base < nvec; base += 32 * U) {
+        uint4 wv[NR][U];
 #pragma unroll
-        for (int u = 0; u < F::U; ++u) {
+        for (int u = 0; u < U; ++u) {
             const int v = base + 32 * u;
 #pragma unroll
             for (int r = 0; r < NR; ++r)
                 wv[r][u] = v < nvec ? ld_stream16(rows[r] + int64_t(v) * 16) : make_uint4(0, 0, 0, 0);
         }
 #pragma unroll
-        for (int u = 0; u < F::U; ++u) {
+        for (int u = 0; u < U; ++u) {
             const int v = base + 32 * u;
             if (v >= nvec) break;
             const int c0 = v * F::VE;

@@ -171,8 +171,11 @@ __device__ __forceinline__ void topk_token(const TopkArgs& a, int64_t t) {
 // in shared memory (skeys: T * E words) and rolled loops: the decode kernel runs this once
 // per SM, with the instruction caches cold, so few distinct instructions matter more than
 // registers. Same keys, tie-breaking and arithmetic as topk_token (identical results).
+// ssel: the select-only biases already staged in shared memory (or null: read from global);
+// slog: T * E floats of shared memory that keep the logits for the combine weights.
 // Every thread of the block calls it; warp t < T finishes token t.
-__device__ __forceinline__ void topk_block(const TopkArgs& a, uint64_t* skeys, float* sstat) {
+__device__ __forceinline__ void topk_block(const TopkArgs& a, uint64_t* skeys, float* sstat, const float* ssel,
+                                           float* slog) {
     const int T = int(a.T), E = a.E;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     if (a.scoring == MOE_SCORING_SOFTMAX_ALL) {  // each token's max and 1 / sum, lane order as above
@@ -198,7 +201,8 @@ __device__ __forceinline__ void topk_block(const TopkArgs& a, uint64_t* skeys, f
         const int t = i / E, e = i - t * E;
         const bool sa = a.scoring == MOE_SCORING_SOFTMAX_ALL;
         const float l = __ldcg(a.logits + int64_t(t) * a.ld + e);
-        const float sb = a.has_sel ? __ldg(a.sel_bias + e) : 0.f;
+        const float sb = a.has_sel ? (ssel ? ssel[e] : __ldg(a.sel_bias + e)) : 0.f;
+        slog[i] = l;
         skeys[i] = select_key(a, l, sb, e, sa ? sstat[2 * t] : 0.f, sa ? sstat[2 * t + 1] : 1.f);
     }
     __syncthreads();
@@ -219,7 +223,7 @@ __device__ __forceinline__ void topk_block(const TopkArgs& a, uint64_t* skeys, f
         __syncwarp();
         if (lane == j) my_e = e;
     }
-    const float my_l = lane < a.k ? __ldcg(a.logits + int64_t(warp) * a.ld + my_e) : -INFINITY;
+    const float my_l = lane < a.k ? slog[warp * E + my_e] : -INFINITY;
     const bool sa = a.scoring == MOE_SCORING_SOFTMAX_ALL;
     finish_token(a, warp, my_e, my_l, sa ? sstat[2 * warp] : 0.f, sa ? sstat[2 * warp + 1] : 1.f);
 }

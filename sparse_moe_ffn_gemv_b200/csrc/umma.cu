@@ -18,16 +18,19 @@
 //               combine (down: the slot's output row times its routing weight reduced
 //               into the token's fp32 routed sum with 16-byte vector reductions), or a
 //               plain store, each thread writing contiguous 16-byte vectors
-//   warps 10..17 (4-bit weights only) dequantisation: the producer loads the packed words,
-//               these warps write w = scale * q + bias as bf16 into the swizzled operand
+//   4-bit weights: warps 2..5 epilogue (one per TMEM lane quarter, all 256 columns) and
+//   warps 6..21 dequantisation: the producer loads the packed words,
+//               these warps write w = scale * q + bias (fp16; MXFP4: bf16) into the swizzled operand
 //               layout the MMA reads (mlxcel issue #974: affine 4-bit, per-group scale
 //               and bias). With 4-bit weights the shared memory holds two rings: a deep
 //               one of small slots (the two packed tiles + the token tile of a K block)
 //               that TMA fills far ahead, and a shallow one of bf16 operand tiles that
 //               the dequantising warps fill and the MMA drains, so that load latency,
 //               dequantisation and MMA overlap instead of sharing one stage
-// TMEM holds two accumulator sets so the epilogue of one tile overlaps the main loop of
-// the next. Every mbarrier wait is bounded by %globaltimer; a wait that gives up records
+// Tiles of 128 token rows keep two accumulator sets in TMEM, so the epilogue of one tile
+// overlaps the main loop of the next; bf16 launches on large batches use tiles of 256 token
+// rows (two MMAs per K step sharing the weight tile, one accumulator set of 2 x 256 columns),
+// which read each weight tile once for up to 256 routed rows. Every mbarrier wait is bounded by %globaltimer; a wait that gives up records
 // MOE_ERR_DEVICE_TIMEOUT in the status word, drains its own outstanding copies / MMAs and
 // returns, and TMEM is always freed.
 //
@@ -51,8 +54,14 @@ namespace {
 
 constexpr int kBM = 128;          // weight rows per MMA (M)
 constexpr int kBK = 64;           // K per stage: one 128-byte swizzle atom of bf16
-constexpr int kDqThreads = 256;   // + 8 dequantising warps for 4-bit weights (4 measured 30% slower)
-constexpr int kDqTiles = 2 * kBM / kDqThreads;  // weight tiles per dequantising thread (one row each)
+// 4-bit weights: 16 dequantising warps, one thread per (weight tile, row, half of the K
+// block). With 8 warps (one whole row each) a warp took about 1100 cycles per K block, twice
+// the MMA's 512: two warps per SM sub-partition could not hide the shared-memory and fence
+// latencies of their chain.
+constexpr int kDqThreads = 512;
+constexpr int kDqParts = kDqThreads / (2 * kBM);  // parts of a K block per weight row
+constexpr int kDqWords = 8 / kDqParts;             // packed words (8 codes each) per thread
+constexpr int kDqTiles = 1;                        // weight tiles per dequantising thread
 constexpr int kEpiThreads = 256;
 constexpr int kPkBytes = kBM * kBK / 2;  // packed 4-bit weight tile: 128 rows x 32 bytes
 constexpr int kMaxGroups = 512;   // expert groups whose tile table fits in shared memory
@@ -91,28 +100,49 @@ __device__ __forceinline__ void umma_commit(uint64_t* bar) {
     asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(su32(bar))
                  : "memory");
 }
-// Issue a 32-column TMEM load without waiting; the registers are valid only after
-// tmem_ld_wait on the same array (which also keeps the compiler from using them early).
-__device__ __forceinline__ void tmem_ld_issue(uint32_t taddr, uint32_t (&r)[32]) {
-    asm volatile(
-        "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
-        "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
-        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
-          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]),
-          "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]),
-          "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]),
-          "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
-        : "r"(taddr));
+// Issue an N-column TMEM load (N = 16 or 32) without waiting; the registers are valid only
+// after tmem_ld_wait on the same array (which also keeps the compiler from using them early).
+template <int N>
+__device__ __forceinline__ void tmem_ld_issue(uint32_t taddr, uint32_t (&r)[N]) {
+    static_assert(N == 16 || N == 32, "16 or 32 columns");
+    if constexpr (N == 32) {
+        asm volatile(
+            "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+            "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+            : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+              "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]),
+              "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]),
+              "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]),
+              "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+            : "r"(taddr));
+    } else {
+        asm volatile(
+            "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+            : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+              "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]),
+              "=r"(r[15])
+            : "r"(taddr));
+    }
 }
-__device__ __forceinline__ void tmem_ld_wait(uint32_t (&r)[32]) {
-    asm volatile("tcgen05.wait::ld.sync.aligned;"
-                 : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]), "+r"(r[6]),
-                   "+r"(r[7]), "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]), "+r"(r[12]), "+r"(r[13]),
-                   "+r"(r[14]), "+r"(r[15]), "+r"(r[16]), "+r"(r[17]), "+r"(r[18]), "+r"(r[19]),
-                   "+r"(r[20]), "+r"(r[21]), "+r"(r[22]), "+r"(r[23]), "+r"(r[24]), "+r"(r[25]),
-                   "+r"(r[26]), "+r"(r[27]), "+r"(r[28]), "+r"(r[29]), "+r"(r[30]), "+r"(r[31])
-                 :
-                 : "memory");
+template <int N>
+__device__ __forceinline__ void tmem_ld_wait(uint32_t (&r)[N]) {
+    if constexpr (N == 32) {
+        asm volatile("tcgen05.wait::ld.sync.aligned;"
+                     : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]), "+r"(r[6]),
+                       "+r"(r[7]), "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]), "+r"(r[12]), "+r"(r[13]),
+                       "+r"(r[14]), "+r"(r[15]), "+r"(r[16]), "+r"(r[17]), "+r"(r[18]), "+r"(r[19]),
+                       "+r"(r[20]), "+r"(r[21]), "+r"(r[22]), "+r"(r[23]), "+r"(r[24]), "+r"(r[25]),
+                       "+r"(r[26]), "+r"(r[27]), "+r"(r[28]), "+r"(r[29]), "+r"(r[30]), "+r"(r[31])
+                     :
+                     : "memory");
+    } else {
+        asm volatile("tcgen05.wait::ld.sync.aligned;"
+                     : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]), "+r"(r[6]),
+                       "+r"(r[7]), "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]), "+r"(r[12]), "+r"(r[13]),
+                       "+r"(r[14]), "+r"(r[15])
+                     :
+                     : "memory");
+    }
 }
 
 // Where one tile lives.
@@ -490,14 +520,15 @@ __global__ void __launch_bounds__(TcShape<GATEUP, BN, STAGES, Q4>::THREADS, 1)
         }
     } else if (Q4 && int(threadIdx.x) >= S::DQ_BASE) {
         // ---------------------------------------------------------- dequantisation warps
-        // Thread d dequantises row d % 128 of kDqTiles of the two weight tiles (all 64 K
-        // elements of the block: two 16-byte loads of packed words from the load slot, eight
-        // swizzled 16-byte stores into the operand slot). Its (scale, bias) pairs are loaded
-        // eight K blocks ahead. A bf16 tile in the same launch (the shared expert) gets its
-        // operand slot filled by TMA, issued by the first dequantising thread.
+        // Thread d dequantises row d % 128 of weight tile (d / 128) % 2, part d / 256 of the
+        // K block (kDqWords packed words: one 16-byte load from the load slot, kDqWords
+        // swizzled 16-byte stores into the operand slot); a warp's threads share tile and
+        // part. Its (scale, bias) pairs are loaded eight K blocks ahead. A bf16 tile in the
+        // same launch (the shared expert) gets its operand slot filled by TMA, issued by the
+        // first dequantising thread.
         constexpr int DT = kDqTiles;
         const int d = threadIdx.x - S::DQ_BASE;
-        const int drow = d & (kBM - 1), a0 = (d / kBM) * DT;
+        const int drow = d & (kBM - 1), a0 = (d / kBM) & 1, part = d / (2 * kBM);
         const bool leader = d == 0;
         uint32_t stage = 0, phase = 0;
         uint32_t astage = 0, aphase = 0;
@@ -620,18 +651,19 @@ __global__ void __launch_bounds__(TcShape<GATEUP, BN, STAGES, Q4>::THREADS, 1)
 #pragma unroll
                 for (int ai = 0; ai < DT; ++ai) {
                     const int a = a0 + ai;
-                    const uint4* pk = reinterpret_cast<const uint4*>(lb + a * kPkBytes + drow * 32);
-                    const uint4 w0 = pk[0], w1 = pk[1];
-                    const uint32_t words[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
+                    static_assert(kDqWords == 4, "one 16-byte load of packed words per thread");
+                    const uint4 w0 = *reinterpret_cast<const uint4*>(lb + a * kPkBytes + drow * 32 + part * 16);
+                    const uint32_t words[4] = {w0.x, w0.y, w0.z, w0.w};
 #pragma unroll
-                    for (int c = 0; c < 8; ++c) {
+                    for (int j = 0; j < kDqWords; ++j) {
+                        const int c = part * kDqWords + j;  // 16-byte chunk (8 K values) of the row
                         const __nv_bfloat162 sbv = q0[ai][c >> 2];
                         uint4 v;
                         if constexpr (MX) {
-                            v = dequant8_mx(words[c], sbv);
+                            v = dequant8_mx(words[j], sbv);
                         } else {
                             const __half2 sz = *reinterpret_cast<const __half2*>(&sbv);
-                            v = dequant8_f16(words[c], __low2half2(sz), __high2half2(sz));
+                            v = dequant8_f16(words[j], __low2half2(sz), __high2half2(sz));
                         }
                         *reinterpret_cast<uint4*>(ob + a * S::A_BYTES + sw128_offset(drow, c)) = v;
                     }
@@ -663,6 +695,9 @@ __global__ void __launch_bounds__(TcShape<GATEUP, BN, STAGES, Q4>::THREADS, 1)
         // warp-private slice of shared memory, so that no epilogue step waits on another warp.
         const int q = warp & 3;
         const int eid = threadIdx.x - 64;
+        // TMEM columns per epilogue step: 16 beside the 4-bit kernel's 16 dequantising warps
+        // (704 threads leave 80 registers per thread), 32 otherwise
+        constexpr int CW = Q4 ? 16 : 32;
         const int th = S::MH == 2 ? (eid >= 128 ? 1 : 0) : 0;  // token half of this warp
         const int tok = th * kBM + q * 32 + lane;               // token row of the tile
         constexpr int NH = S::NH;                               // column halves per warp
@@ -726,23 +761,23 @@ __global__ void __launch_bounds__(TcShape<GATEUP, BN, STAGES, Q4>::THREADS, 1)
                 const bool last_half = hh == NH - 1;
                 const float* sbh = sb + hh * 128;
                 if constexpr (GATEUP) {
-                    // 32 units per chunk: gate and up of the same units -> 32 values of h (64 bytes)
+                    // CW units per chunk: gate and up of the same units -> CW values of h
                     const int u0 = ti.mb * kBM + half * 64;
 #pragma unroll 1
-                    for (int c = 0; c < 2; ++c) {
-                        uint32_t g[32], u[32];
-                        tmem_ld_issue(tb + half * 64 + 32 * c, g);
-                        tmem_ld_issue(tb + kBM + half * 64 + 32 * c, u);
+                    for (int c = 0; c < 64 / CW; ++c) {
+                        uint32_t g[CW], u[CW];
+                        tmem_ld_issue(tb + half * 64 + CW * c, g);
+                        tmem_ld_issue(tb + kBM + half * 64 + CW * c, u);
                         tmem_ld_wait(g);
                         tmem_ld_wait(u);
-                        if (c == 1 && last_half) release();
-                        const int ub = u0 + 32 * c;
+                        if (c == 64 / CW - 1 && last_half) release();
+                        const int ub = u0 + CW * c;
                         if (!tv || ub >= p.M) continue;
-                        const float* bg = sbh + 32 * c;  // gate biases of these 32 units
+                        const float* bg = sbh + CW * c;  // gate biases of these CW units
                         const float* bu = bg + 64;       // their up biases
-                        uint32_t hp[16];
+                        uint32_t hp[CW / 2];
 #pragma unroll
-                        for (int j = 0; j < 32; j += 2) {
+                        for (int j = 0; j < CW; j += 2) {
                             float gg0 = __uint_as_float(g[j]), gg1 = __uint_as_float(g[j + 1]);
                             float uu0 = __uint_as_float(u[j]), uu1 = __uint_as_float(u[j + 1]);
                             if (has_bias) {
@@ -761,47 +796,48 @@ __global__ void __launch_bounds__(TcShape<GATEUP, BN, STAGES, Q4>::THREADS, 1)
                         }
                         uint4* dst = reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(p.out) + prow * p.ld_out + ub);
 #pragma unroll
-                        for (int v = 0; v < 4; ++v) dst[v] = make_uint4(hp[4 * v], hp[4 * v + 1], hp[4 * v + 2], hp[4 * v + 3]);
+                        for (int v = 0; v < CW / 8; ++v) dst[v] = make_uint4(hp[4 * v], hp[4 * v + 1], hp[4 * v + 2], hp[4 * v + 3]);
                     }
                 } else {
-                    // 32 weight rows (output columns) per chunk; bf16 weights: the next chunk's TMEM
+                    // CW weight rows (output columns) per chunk; bf16 weights: the next chunk's TMEM
                     // load in flight while this one is stored; 4-bit weights: one at a time
                     const int rb = ti.mb * 2 * kBM + half * kBM;
                     constexpr int NB = Q4 ? 1 : 2;
-                    uint32_t v[NB][32];
+                    constexpr int NC = kBM / CW;  // chunks per half
+                    uint32_t v[NB][CW];
                     tmem_ld_issue(tb + half * kBM, v[0]);
 #pragma unroll
-                    for (int c = 0; c < 4; ++c) {
+                    for (int c = 0; c < NC; ++c) {
                         tmem_ld_wait(v[c % NB]);
-                        if (NB == 2 && c < 3) tmem_ld_issue(tb + half * kBM + 32 * (c + 1), v[(c + 1) % NB]);
-                        if (c == 3 && last_half) release();
-                        const int r0 = rb + 32 * c;
-                        float o[32];
+                        if (NB == 2 && c < NC - 1) tmem_ld_issue(tb + half * kBM + CW * (c + 1), v[(c + 1) % NB]);
+                        if (c == NC - 1 && last_half) release();
+                        const int r0 = rb + CW * c;
+                        float o[CW];
 #pragma unroll
-                        for (int j = 0; j < 32; ++j) o[j] = __uint_as_float(v[c % NB][j]);
-                        if (NB == 1 && c < 3) tmem_ld_issue(tb + half * kBM + 32 * (c + 1), v[0]);
+                        for (int j = 0; j < CW; ++j) o[j] = __uint_as_float(v[c % NB][j]);
+                        if (NB == 1 && c < NC - 1) tmem_ld_issue(tb + half * kBM + CW * (c + 1), v[0]);
                         if (!tv || r0 >= p.M) continue;
                         if (has_bias) {
 #pragma unroll
-                            for (int j = 0; j < 32; ++j) o[j] += sbh[32 * c + j];
+                            for (int j = 0; j < CW; ++j) o[j] += sbh[CW * c + j];
                         }
-                        const bool whole = r0 + 32 <= p.M;
+                        const bool whole = r0 + CW <= p.M;
                         if (p.mode == kEpiScatterAdd) {
                             // weighted combine into the token's fp32 routed sum, 16 bytes per
                             // reduction (libmir-metal execute: down weighted by routing.weights and
                             // summed per token); M is a multiple of 64 here
 #pragma unroll
-                            for (int j = 0; j < 32; j += 4)
+                            for (int j = 0; j < CW; j += 4)
                                 red_add_v4(yrow + r0 + j, wslot * o[j], wslot * o[j + 1], wslot * o[j + 2], wslot * o[j + 3]);
                         } else if (p.mode == kEpiStoreF32) {
                             float* dst = reinterpret_cast<float*>(p.out) + prow * p.ld_out + r0;
                             if (whole) {
 #pragma unroll
-                                for (int j = 0; j < 32; j += 4)
+                                for (int j = 0; j < CW; j += 4)
                                     *reinterpret_cast<float4*>(dst + j) = make_float4(o[j], o[j + 1], o[j + 2], o[j + 3]);
                             } else {
 #pragma unroll
-                                for (int j = 0; j < 32; ++j)
+                                for (int j = 0; j < CW; ++j)
                                     if (r0 + j < p.M) dst[j] = o[j];
                             }
                         } else {  // kEpiStoreAct (+ optional fp32 addend)
@@ -810,13 +846,13 @@ __global__ void __launch_bounds__(TcShape<GATEUP, BN, STAGES, Q4>::THREADS, 1)
                             if (whole) {
                                 if (ad) {
 #pragma unroll
-                                    for (int j = 0; j < 32; j += 4) {
+                                    for (int j = 0; j < CW; j += 4) {
                                         const float4 a4 = __ldcs(reinterpret_cast<const float4*>(ad + j));
                                         o[j] += a4.x; o[j + 1] += a4.y; o[j + 2] += a4.z; o[j + 3] += a4.w;
                                     }
                                 }
 #pragma unroll
-                                for (int w4 = 0; w4 < 4; ++w4) {
+                                for (int w4 = 0; w4 < CW / 8; ++w4) {
                                     uint32_t hp[4];
 #pragma unroll
                                     for (int j = 0; j < 4; ++j) {
@@ -827,7 +863,7 @@ __global__ void __launch_bounds__(TcShape<GATEUP, BN, STAGES, Q4>::THREADS, 1)
                                 }
                             } else {
 #pragma unroll
-                                for (int j = 0; j < 32; ++j)
+                                for (int j = 0; j < CW; ++j)
                                     if (r0 + j < p.M) dst[j] = __float2bfloat16_rn(o[j] + (ad ? ad[j] : 0.f));
                             }
                         }
