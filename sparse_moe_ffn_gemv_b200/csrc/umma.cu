@@ -100,6 +100,28 @@ __device__ __forceinline__ void umma_commit(uint64_t* bar) {
     asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(su32(bar))
                  : "memory");
 }
+// CTA pair: M = 256 rows (128 in each CTA's shared memory and TMEM), N = 256 (each CTA holds
+// half of the N-side operand), issued by the pair's leader.
+__host__ __device__ constexpr uint32_t idesc_bf16_pair() {
+    return (1u << 4) | (1u << 7) | (1u << 10) | (uint32_t(256 >> 3) << 17) | (uint32_t(256 >> 4) << 24);
+}
+__device__ __forceinline__ void umma_pair(uint32_t d, uint64_t a, uint64_t b, uint32_t idesc, uint32_t acc) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d),
+        "l"(a), "l"(b), "r"(idesc), "r"(acc)
+        : "memory");
+}
+// Arrive on the mbarrier at the same shared-memory offset in both CTAs of the pair once the
+// leader's MMAs issued so far have completed.
+__device__ __forceinline__ void umma_commit_pair(uint64_t* bar) {
+    asm volatile(
+        "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;" ::"r"(
+            su32(bar)),
+        "h"(uint16_t(3))
+        : "memory");
+}
 // Issue an N-column TMEM load (N = 16 or 32) without waiting; the registers are valid only
 // after tmem_ld_wait on the same array (which also keeps the compiler from using them early).
 template <int N>
@@ -207,13 +229,17 @@ __device__ __forceinline__ TileInfo decode_tile(const TcParams& P, const GroupTa
 // up rows of 128 intermediate units (gate/up), or 256 consecutive output rows (others).
 // bf16 weights: STAGES stages of [A0 | A1 | B]. 4-bit weights: STAGES load slots of
 // [packed 0 | packed 1 | B] (TMA), then ASTAGES operand slots of [A0 | A1] (dequantised).
-template <bool GATEUP, int BN, int STAGES, bool Q4 = false>
+// PAIR: a cluster of two CTAs shares each 256-token tile: CTA r holds token rows
+// 128 r .. 128 r + 127 and weight tile r (the gate or the up rows, or output rows
+// 128 r .. 128 r + 127), and the leader's M = 256, N = 256 MMAs read both CTAs' operands.
+template <bool GATEUP, int BN, int STAGES, bool Q4 = false, bool PAIR = false>
 struct TcShape {
     static constexpr int A_BYTES = kBM * kBK * 2;                // 16 KB: one 128-row weight tile
-    static constexpr int B_BYTES = BN * kBK * 2;                 // token tile
+    static constexpr int B_BYTES = (PAIR ? kBM : BN) * kBK * 2;  // this CTA's token tile
     static constexpr int ASTAGES = Q4 ? 2 : 0;                   // dequantised operand slots
-    static constexpr int B_OFF = Q4 ? 2 * kPkBytes : 2 * A_BYTES;  // token tile within a stage
-    static constexpr int STAGE_BYTES = Q4 ? 2 * kPkBytes + B_BYTES : 2 * A_BYTES + B_BYTES;
+    static constexpr int NA = PAIR ? 1 : 2;                      // weight tiles per CTA and stage
+    static constexpr int B_OFF = Q4 ? 2 * kPkBytes : NA * A_BYTES;  // token tile within a stage
+    static constexpr int STAGE_BYTES = Q4 ? 2 * kPkBytes + B_BYTES : NA * A_BYTES + B_BYTES;
     static constexpr int ARING_OFF = STAGES * STAGE_BYTES;       // operand ring (4-bit only)
     static constexpr int RING_BYTES = STAGES * STAGE_BYTES + ASTAGES * 2 * A_BYTES;
     // epilogue warps: 8, or 4 beside the dequantising warps, which keeps the 4-bit block at
@@ -224,7 +250,7 @@ struct TcShape {
     // TMEM: one 128 x 256 fp32 accumulator per 128 token rows of a tile; 128-row tiles keep
     // two accumulator sets (the epilogue of one tile overlaps the next tile's main loop),
     // 256-row tiles one set of two (512 columns either way)
-    static constexpr int MH = BN / kBM;                          // 128-row token halves per tile
+    static constexpr int MH = PAIR ? 1 : BN / kBM;               // 128-row token halves per CTA tile
     static constexpr int NBUF = MH == 1 ? 2 : 1;                 // accumulator sets
     static constexpr int ACC_COLS = 2 * kBM;                     // columns of one accumulator
     static constexpr int TMEM_COLS = ACC_COLS * MH * NBUF;
@@ -237,6 +263,7 @@ struct TcShape {
     static constexpr int SMEM = RING_BYTES + 1024 /*align*/ + 256 /*barriers*/ + int(sizeof(GroupTables)) + BIAS_BYTES;
     static_assert(TMEM_COLS == 512, "TMEM columns");
     static_assert(BN == 128 || (BN == 256 && !Q4), "token tile");
+    static_assert(!PAIR || (BN == 256 && !Q4), "CTA pairs: bf16, 256-token tiles");
     static_assert(EPI_WARPS_PER_HALF == 4 || EPI_WARPS_PER_HALF == 8, "epilogue warps");
     static_assert(STAGE_BYTES % 1024 == 0 && B_OFF % 1024 == 0, "swizzle atoms stay 1 KB aligned");
     static_assert((2 * STAGES + 5 + 2 * ASTAGES) * 8 + 4 <= 256, "barriers fit their region");
@@ -330,10 +357,21 @@ __device__ __forceinline__ void load_a_bf16(uint8_t* dst, const TcParams& P, con
     }
 }
 
-template <bool GATEUP, int BN, int STAGES, bool Q4>
-__global__ void __launch_bounds__(TcShape<GATEUP, BN, STAGES, Q4>::THREADS, 1)
+// CTA pair: this CTA's one weight tile of K block kc (rank 0: gate rows or output rows
+// [mrow, mrow + 128); rank 1: up rows or [mrow + 128, mrow + 256)), completing on the
+// leader's barrier at cluster address bar.
+template <bool GATEUP>
+__device__ __forceinline__ void load_a_pair(uint8_t* dst, const TcParams& P, const TileInfo& ti, int mrow, int kc,
+                                            uint32_t rank, uint32_t bar, uint64_t pol) {
+    if (!GATEUP) tma_3d_pair(dst, &P.a0[ti.prob], bar, kc, mrow + kBM * int(rank), ti.group, pol);
+    else if (P.p[ti.prob].interleaved) tma_4d_pair(dst, &P.a0[ti.prob], bar, kc, int(rank), mrow, ti.group, pol);
+    else tma_3d_pair(dst, rank ? &P.a1[ti.prob] : &P.a0[ti.prob], bar, kc, mrow, ti.group, pol);
+}
+
+template <bool GATEUP, int BN, int STAGES, bool Q4, bool PAIR>
+__global__ void __launch_bounds__(TcShape<GATEUP, BN, STAGES, Q4, PAIR>::THREADS, 1)
     tc_gemm_kernel(const __grid_constant__ TcParams P) {
-    using S = TcShape<GATEUP, BN, STAGES, Q4>;
+    using S = TcShape<GATEUP, BN, STAGES, Q4, PAIR>;
     constexpr int AS = S::ASTAGES > 0 ? S::ASTAGES : 1;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -349,10 +387,21 @@ __global__ void __launch_bounds__(TcShape<GATEUP, BN, STAGES, Q4>::THREADS, 1)
     float* sbias = reinterpret_cast<float*>(&gt + 1);  // epilogue: 128 column biases per warp
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    // CTA pairs: rank in the pair (0 = leader: issues the MMAs, owns the full / acc_empty
+    // barriers) and the pair's tile stride; single CTAs: rank 0, one tile per CTA
+    const uint32_t crank = PAIR ? cluster_rank() : 0u;
+    const int tile0 = PAIR ? int(blockIdx.x >> 1) : int(blockIdx.x);
+    const int tstep = PAIR ? int(gridDim.x >> 1) : int(gridDim.x);
     if (warp == 0) {
-        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(su32(tmem_slot)),
-                     "r"(uint32_t(S::TMEM_COLS)));
-        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
+        if constexpr (PAIR) {
+            asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(su32(tmem_slot)),
+                         "r"(uint32_t(S::TMEM_COLS)));
+            asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;");
+        } else {
+            asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(su32(tmem_slot)),
+                         "r"(uint32_t(S::TMEM_COLS)));
+            asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
+        }
     }
     if (warp == 1 && lane == 0) {
         for (int s = 0; s < STAGES; ++s) {
@@ -361,7 +410,7 @@ __global__ void __launch_bounds__(TcShape<GATEUP, BN, STAGES, Q4>::THREADS, 1)
         }
         for (int b = 0; b < 2; ++b) {
             mbar_init(&acc_full[b], 1);
-            mbar_init(&acc_empty[b], S::EPI / 32);  // one arrive per epilogue warp
+            mbar_init(&acc_empty[b], (PAIR ? 2 : 1) * S::EPI / 32);  // one arrive per epilogue warp (of the pair)
         }
         mbar_init(drain, 1);
         if (Q4)
@@ -389,6 +438,7 @@ __global__ void __launch_bounds__(TcShape<GATEUP, BN, STAGES, Q4>::THREADS, 1)
     }
     tc_fence_before();
     __syncthreads();
+    if constexpr (PAIR) cluster_sync();  // the peer's barriers are initialised before any remote use
     tc_fence_after();
     const uint32_t tmem_base = *tmem_slot;
 
@@ -407,14 +457,20 @@ __global__ void __launch_bounds__(TcShape<GATEUP, BN, STAGES, Q4>::THREADS, 1)
         uint32_t armed = 0;  // bit s: stage s was filled at least once
         uint32_t last_par = 0;
         const uint64_t pol_w = policy_evict_first(), pol_t = policy_evict_last();
-        for (int tile = blockIdx.x; tile < total && !timed_out; tile += gridDim.x) {
+        for (int tile = tile0; tile < total && !timed_out; tile += tstep) {
             const TileInfo ti = decode_tile(P, gt, tile, t0);
             const TcProblem& p = P.p[ti.prob];
             const int nk = p.K / kBK;
             const int mrow = ti.mb * S::ROWS;
             // token rows: the smallest box (16, 32, 64, 128, 256 rows) that holds the valid tokens
-            const int bv = ti.nvalid <= 16 ? 0 : ti.nvalid <= 32 ? 1 : ti.nvalid <= 64 ? 2 : ti.nvalid <= 128 ? 3 : 4;
+            // (CTA pairs: of this CTA's 128-row half; the leader's barrier counts both halves)
+            auto box_of = [](int nv) { return nv <= 16 ? 0 : nv <= 32 ? 1 : nv <= 64 ? 2 : nv <= 128 ? 3 : 4; };
+            auto half_nv = [&](uint32_t r) { return max(0, min(kBM, ti.nvalid - kBM * int(r))); };
+            const int bv = box_of(PAIR ? half_nv(crank) : ti.nvalid);
             const uint32_t b_bytes = uint32_t(min(BN, 16 << bv)) * kBK * 2;
+            const uint32_t pair_tx = PAIR ? 2u * S::A_BYTES + (uint32_t(16 << box_of(half_nv(0))) +
+                                                               uint32_t(16 << box_of(half_nv(1)))) * kBK * 2
+                                          : 0u;
             for (int kb = 0; kb < nk; ++kb) {
                 int ok = 1;
                 if (lane == 0) ok = mbar_wait(&empty[stage], phase ^ 1u, deadline) ? 1 : 0;
@@ -436,11 +492,18 @@ __global__ void __launch_bounds__(TcShape<GATEUP, BN, STAGES, Q4>::THREADS, 1)
                         } else {
                             mbar_expect_tx(&full[stage], b_bytes);
                         }
+                    } else if constexpr (PAIR) {
+                        // this CTA's weight tile and token half; the bytes complete on the
+                        // leader's barrier, which the leader arms with the pair's total
+                        const uint32_t fb = mapa_shared(&full[stage], 0);
+                        if (crank == 0) mbar_expect_tx(&full[stage], pair_tx);
+                        load_a_pair<GATEUP>(sb, P, ti, mrow, kc, crank, fb, pol_w);
+                        tma_2d_pair(sb + S::B_OFF, &P.b[ti.prob][bv], fb, kc, ti.row0 + kBM * int(crank), pol_t);
                     } else {
                         mbar_expect_tx(&full[stage], 2 * S::A_BYTES + b_bytes);
                         load_a_bf16<GATEUP>(sb, P, ti, mrow, kc, &full[stage], pol_w);
                     }
-                    tma_2d(sb + S::B_OFF, &P.b[ti.prob][bv], &full[stage], kc, ti.row0, pol_t);
+                    if constexpr (!PAIR) tma_2d(sb + S::B_OFF, &P.b[ti.prob][bv], &full[stage], kc, ti.row0, pol_t);
                 }
                 armed |= 1u << stage;
                 last_par = (last_par & ~(1u << stage)) | (phase << stage);
@@ -450,22 +513,23 @@ __global__ void __launch_bounds__(TcShape<GATEUP, BN, STAGES, Q4>::THREADS, 1)
                 }
             }
         }
-        // drain: every copy this warp issued has landed before the CTA can exit
+        // drain: every copy this warp issued has landed before the CTA can exit (CTA pairs:
+        // the leader's MMA has consumed it, which it does only once both halves landed)
         if (lane == 0) {
             const uint64_t dl2 = gtimer() + kWaitNs;
             for (int s = 0; s < STAGES; ++s)
-                if ((armed >> s) & 1u) mbar_wait(&full[s], (last_par >> s) & 1u, dl2);
+                if ((armed >> s) & 1u) mbar_wait(PAIR ? &empty[s] : &full[s], (last_par >> s) & 1u, dl2);
             if (timed_out) set_status(P.status, MOE_ERR_DEVICE_TIMEOUT);
         }
         __syncwarp();
     } else if (warp == 1) {
-        if (lane == 0) {
-            // ---------------------------------------------------------- MMA issuer
+        if (lane == 0 && crank == 0) {
+            // ---------------------------------------------------------- MMA issuer (pairs: the leader's)
             uint32_t stage = 0, phase = 0, it = 0;
             uint32_t astage = 0, aphase = 0;
             // M = 128 token rows, N = 256 weight rows; fp16 operands for 4-bit affine weights
             constexpr uint32_t idesc_b = idesc_bf16(2 * kBM), idesc_h = idesc_f16(2 * kBM);
-            for (int tile = blockIdx.x; tile < total && !timed_out; tile += gridDim.x, ++it) {
+            for (int tile = tile0; tile < total && !timed_out; tile += tstep, ++it) {
                 const TileInfo ti = decode_tile(P, gt, tile, t0);
                 const TcProblem& p = P.p[ti.prob];
                 const uint32_t ab = it % S::NBUF, aph = (it / S::NBUF) & 1u;
@@ -476,7 +540,7 @@ __global__ void __launch_bounds__(TcShape<GATEUP, BN, STAGES, Q4>::THREADS, 1)
                 tc_fence_after();
                 const uint32_t d0 = tmem_base + ab * S::MH * S::ACC_COLS;
                 const int nh = S::MH == 2 && ti.nvalid > kBM ? 2 : 1;  // token halves with valid rows
-                const uint32_t idesc = (Q4 && p.q4 && !p.mx) ? idesc_h : idesc_b;
+                const uint32_t idesc = PAIR ? idesc_bf16_pair() : (Q4 && p.q4 && !p.mx) ? idesc_h : idesc_b;
                 const int nk = p.K / kBK;
                 for (int kb = 0; kb < nk; ++kb) {
                     // 4-bit: the operand slot is complete once the dequantising warps have
@@ -493,11 +557,13 @@ __global__ void __launch_bounds__(TcShape<GATEUP, BN, STAGES, Q4>::THREADS, 1)
 #pragma unroll
                     for (int k = 0; k < kBK / 16; ++k) {
                         const uint32_t acc = (kb > 0 || k > 0) ? 1u : 0u;
-                        umma(d0, smem_desc(st + k * 32), smem_desc(sw + k * 32), idesc, acc);
+                        if constexpr (PAIR) umma_pair(d0, smem_desc(st + k * 32), smem_desc(sw + k * 32), idesc, acc);
+                        else umma(d0, smem_desc(st + k * 32), smem_desc(sw + k * 32), idesc, acc);
                         if (S::MH == 2 && nh == 2)  // token rows 128..255 (16 KB further), same weights
                             umma(d0 + S::ACC_COLS, smem_desc(st + kBM * 128 + k * 32), smem_desc(sw + k * 32), idesc, acc);
                     }
-                    umma_commit(&empty[stage]);
+                    if constexpr (PAIR) umma_commit_pair(&empty[stage]);  // both CTAs' slots
+                    else umma_commit(&empty[stage]);
                     if (++stage == STAGES) {
                         stage = 0;
                         phase ^= 1u;
@@ -511,10 +577,12 @@ __global__ void __launch_bounds__(TcShape<GATEUP, BN, STAGES, Q4>::THREADS, 1)
                     }
                 }
                 if (timed_out) break;
-                umma_commit(&acc_full[ab]);
+                if constexpr (PAIR) umma_commit_pair(&acc_full[ab]);  // both CTAs' epilogues
+                else umma_commit(&acc_full[ab]);
             }
             // drain: all MMAs issued by this thread have completed
-            umma_commit(drain);
+            if constexpr (PAIR) umma_commit_pair(drain);
+            else umma_commit(drain);
             mbar_wait(drain, 0, gtimer() + kWaitNs);
             if (timed_out) set_status(P.status, MOE_ERR_DEVICE_TIMEOUT);
         }
@@ -544,7 +612,7 @@ __global__ void __launch_bounds__(TcShape<GATEUP, BN, STAGES, Q4>::THREADS, 1)
                 aphase ^= 1u;
             }
         };
-        for (int tile = blockIdx.x; tile < total && !timed_out; tile += gridDim.x) {
+        for (int tile = tile0; tile < total && !timed_out; tile += tstep) {
             const TileInfo ti = decode_tile(P, gt, tile, t0);
             const TcProblem& p = P.p[ti.prob];
             const int nk = p.K / kBK;
@@ -699,12 +767,12 @@ __global__ void __launch_bounds__(TcShape<GATEUP, BN, STAGES, Q4>::THREADS, 1)
         // (704 threads leave 80 registers per thread), 32 otherwise
         constexpr int CW = Q4 ? 16 : 32;
         const int th = S::MH == 2 ? (eid >= 128 ? 1 : 0) : 0;  // token half of this warp
-        const int tok = th * kBM + q * 32 + lane;               // token row of the tile
+        const int tok = (PAIR ? int(crank) : th) * kBM + q * 32 + lane;  // token row of the tile
         constexpr int NH = S::NH;                               // column halves per warp
         const int h_lo = NH == 1 ? (eid >= 128 ? 1 : 0) : 0;
         float* sb = sbias + (eid >> 5) * 128 * NH;  // this warp's column biases (warp-private)
         uint32_t it = 0;
-        for (int tile = blockIdx.x; tile < total; tile += gridDim.x, ++it) {
+        for (int tile = tile0; tile < total; tile += tstep, ++it) {
             const TileInfo ti = decode_tile(P, gt, tile, t0);
             const TcProblem& p = P.p[ti.prob];
             const uint32_t ab = it % S::NBUF, aph = (it / S::NBUF) & 1u;
@@ -753,7 +821,10 @@ __global__ void __launch_bounds__(TcShape<GATEUP, BN, STAGES, Q4>::THREADS, 1)
             auto release = [&]() {  // the accumulator set is free for the tile after next
                 tc_fence_before();
                 __syncwarp();
-                if (lane == 0) mbar_arrive(&acc_empty[ab]);
+                if (lane == 0) {
+                    if constexpr (PAIR) mbar_arrive_cluster(mapa_shared(&acc_empty[ab], 0));  // the leader's
+                    else mbar_arrive(&acc_empty[ab]);
+                }
             };
 #pragma unroll 1
             for (int hh = 0; hh < NH; ++hh) {
@@ -874,10 +945,17 @@ __global__ void __launch_bounds__(TcShape<GATEUP, BN, STAGES, Q4>::THREADS, 1)
     }
     tc_fence_before();
     __syncthreads();
+    // CTA pairs: neither CTA leaves (nor frees its TMEM) while the other may still arrive on its
+    // barriers or the leader's MMAs may read its operands
+    if constexpr (PAIR) cluster_sync();
     if (warp == 0) {
         tc_fence_after();
-        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base),
-                     "r"(uint32_t(S::TMEM_COLS)));
+        if constexpr (PAIR)
+            asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(tmem_base),
+                         "r"(uint32_t(S::TMEM_COLS)));
+        else
+            asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base),
+                         "r"(uint32_t(S::TMEM_COLS)));
     }
 }
 
@@ -912,12 +990,37 @@ bool encode(CUtensorMap* m, const void* base, int rank, const cuuint64_t* dims, 
 
 int sm_count() { return device_sm_count(); }
 
-template <bool GATEUP, int BN, int STAGES, bool Q4>
+template <bool GATEUP, int BN, int STAGES, bool Q4, bool PAIR = false>
 cudaError_t launch_tc_t(TcParams& P, int64_t max_tiles, cudaStream_t s) {
-    using S = TcShape<GATEUP, BN, STAGES, Q4>;
-    auto kern = tc_gemm_kernel<GATEUP, BN, STAGES, Q4>;
+    using S = TcShape<GATEUP, BN, STAGES, Q4, PAIR>;
+    auto kern = tc_gemm_kernel<GATEUP, BN, STAGES, Q4, PAIR>;
     cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, S::SMEM);
     if (err != cudaSuccess) return err;
+    if constexpr (PAIR) {
+        // clusters of two CTAs; as many pairs as can be resident at once (a GPC with an odd
+        // number of free SMs holds one CTA fewer), each looping over the pair tiles
+        cudaLaunchConfig_t cfg = {};
+        cfg.blockDim = dim3(S::THREADS);
+        cfg.dynamicSmemBytes = S::SMEM;
+        cfg.stream = s;
+        cudaLaunchAttribute attr[2];
+        attr[0].id = cudaLaunchAttributeClusterDimension;
+        attr[0].val.clusterDim.x = 2;
+        attr[0].val.clusterDim.y = 1;
+        attr[0].val.clusterDim.z = 1;
+        attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[1].val.programmaticStreamSerializationAllowed = pdl_enabled() ? 1 : 0;
+        cfg.attrs = attr;
+        cfg.numAttrs = 2;
+        cfg.gridDim = dim3(2 * (sm_count() / 2));
+        int resident = 0;
+        if ((err = cudaOccupancyMaxActiveClusters(&resident, kern, &cfg)) != cudaSuccess) return err;
+        const int pairs = int(std::min<int64_t>(max_tiles, std::min(resident, sm_count() / 2)));
+        if (pairs <= 0) return resident <= 0 ? cudaErrorInvalidConfiguration : cudaSuccess;
+        cfg.gridDim = dim3(2 * pairs);
+        if ((err = cudaLaunchKernelEx(&cfg, kern, P)) != cudaSuccess) return err;
+        return cudaGetLastError();
+    }
     const int grid = int(std::min<int64_t>(max_tiles, sm_count()));
     if (grid <= 0) return cudaSuccess;
     { const cudaError_t e_ = launch_pdl(kern, dim3(grid), dim3(S::THREADS), S::SMEM, s, P); if (e_ != cudaSuccess) return e_; }
@@ -980,9 +1083,9 @@ cudaError_t launch_tc_gemm(TcParams& P, bool gateup, int64_t max_tiles, cudaStre
         if (gateup) return launch_tc_t<true, kTcBN, 6, true>(P, max_tiles, s);
         return launch_tc_t<false, kTcBN, 6, true>(P, max_tiles, s);
     }
-    if (bn == kTcBNWide) {  // 256-token tiles, three 64 KB stages
-        if (gateup) return launch_tc_t<true, kTcBNWide, 3, false>(P, max_tiles, s);
-        return launch_tc_t<false, kTcBNWide, 3, false>(P, max_tiles, s);
+    if (bn == kTcBNWide) {  // 256-token tiles on CTA pairs, six 32 KB stages per CTA
+        if (gateup) return launch_tc_t<true, kTcBNWide, 6, false, true>(P, max_tiles, s);
+        return launch_tc_t<false, kTcBNWide, 6, false, true>(P, max_tiles, s);
     }
     // 128-token tiles, four 48 KB stages
     if (gateup) return launch_tc_t<true, kTcBN, 4, false>(P, max_tiles, s);
