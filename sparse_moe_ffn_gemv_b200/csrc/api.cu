@@ -307,15 +307,16 @@ DecodeArgs decode_args(const moe_config* c, const moe_weights* w, const void* x,
 }
 
 // Chosen where it measured faster than both other engines on B200 (graph replay, L2
-// flushed): a single token, and MXFP4 weights up to 8 tokens. From two tokens on, the
-// tensor-core kernel streams bf16 and affine 4-bit weights faster (Klear 2 tokens: 98 vs
-// 82 us; 8 tokens: 186 vs 129 us).
+// flushed): a single token (Klear bf16 47 vs 62 / 72 us, clamped MXFP4 62 vs 88 / 133 us),
+// and two tokens with bf16 weights (Klear 74 vs 86 / 82 us). From there on the tensor-core
+// kernel streams the weights faster (Klear 4 tokens: 115 vs 111 us; 8 tokens: 176 vs 129 us;
+// clamped MXFP4 8 tokens: 432 vs 361 us).
 bool use_decode(const moe_config* c, int64_t T, const DecodeArgs& d) {
     if (c->latent_dim || c->act_dtype != MOE_DTYPE_BF16 || c->weight_format == MOE_DTYPE_F32) return false;
     const int o = path_override();
     if (o == kPathGemv || o == kPathTc) return false;
     if (T < 1 || T > 8 || decode_smem_bytes(d) == 0) return false;
-    return o == kPathDecode || T == 1 || c->weight_format == MOE_DTYPE_MXFP4;
+    return o == kPathDecode || T == 1 || (T == 2 && c->weight_format == MOE_DTYPE_BF16);
 }
 
 #define MOE_CHECK(expr)                          \

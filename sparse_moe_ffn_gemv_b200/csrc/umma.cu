@@ -29,8 +29,12 @@
 //               dequantisation and MMA overlap instead of sharing one stage
 // Tiles of 128 token rows keep two accumulator sets in TMEM, so the epilogue of one tile
 // overlaps the main loop of the next; bf16 launches on large batches use tiles of 256 token
-// rows (two MMAs per K step sharing the weight tile, one accumulator set of 2 x 256 columns),
-// which read each weight tile once for up to 256 routed rows. Every mbarrier wait is bounded by %globaltimer; a wait that gives up records
+// rows, which read each weight tile once for up to 256 routed rows: in grouped launches one
+// CTA per tile (two MMAs per K step sharing the weight tile, the second skipped when the tile
+// holds at most 128 rows, one accumulator set of 2 x 256 columns), in dense launches a
+// cluster of two CTAs per tile (PAIR: each CTA holds 128 token rows and one 128-row weight
+// tile, the leader issues tcgen05.mma.cta_group::2 with M = 256, N = 256 over both CTAs'
+// shared memory, two accumulator sets of 256 columns per CTA). Every mbarrier wait is bounded by %globaltimer; a wait that gives up records
 // MOE_ERR_DEVICE_TIMEOUT in the status word, drains its own outstanding copies / MMAs and
 // returns, and TMEM is always freed.
 //
@@ -1083,9 +1087,20 @@ cudaError_t launch_tc_gemm(TcParams& P, bool gateup, int64_t max_tiles, cudaStre
         if (gateup) return launch_tc_t<true, kTcBN, 6, true>(P, max_tiles, s);
         return launch_tc_t<false, kTcBN, 6, true>(P, max_tiles, s);
     }
-    if (bn == kTcBNWide) {  // 256-token tiles on CTA pairs, six 32 KB stages per CTA
-        if (gateup) return launch_tc_t<true, kTcBNWide, 6, false, true>(P, max_tiles, s);
-        return launch_tc_t<false, kTcBNWide, 6, false, true>(P, max_tiles, s);
+    if (bn == kTcBNWide) {
+        // Dense launches: CTA pairs (six 32 KB stages per CTA). A pair's M = 256 MMA computes
+        // all 256 token rows of a tile, so in grouped launches, where the last tile of most
+        // experts is partial, the one-CTA tile (which skips an empty second half) measured
+        // faster: latent block at 8192 tokens, expert gate/up 2.64 ms one CTA vs 2.78 ms
+        // pairs; with 512 routed rows per expert (every tile full) pairs win, 518 vs 570 us.
+        bool grouped = false;
+        for (int i = 0; i < P.nprob; ++i) grouped = grouped || P.p[i].grouped;
+        if (!grouped) {
+            if (gateup) return launch_tc_t<true, kTcBNWide, 6, false, true>(P, max_tiles, s);
+            return launch_tc_t<false, kTcBNWide, 6, false, true>(P, max_tiles, s);
+        }
+        if (gateup) return launch_tc_t<true, kTcBNWide, 3, false>(P, max_tiles, s);  // three 64 KB stages
+        return launch_tc_t<false, kTcBNWide, 3, false>(P, max_tiles, s);
     }
     // 128-token tiles, four 48 KB stages
     if (gateup) return launch_tc_t<true, kTcBN, 4, false>(P, max_tiles, s);
