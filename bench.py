@@ -69,7 +69,18 @@ def parse(argv=None):
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--no-e2e", action="store_true")
     p.add_argument("--no-kernel-table", action="store_true")
+    p.add_argument("--experts", type=int, default=0,
+                   help="keep only the first E routed experts of the workload (a smaller copy for ncu captures)")
     return p.parse_args(argv)
+
+
+def workload_spec(args):
+    spec = inputs.WORKLOADS[args.workload]
+    if args.experts:
+        if not spec.top_k <= args.experts <= spec.num_experts:
+            raise SystemExit("--experts must lie between top_k and the workload's expert count")
+        spec = spec.replace(num_experts=args.experts, name=f"{spec.name}_e{args.experts}")
+    return spec
 
 
 def peaks():
@@ -333,23 +344,32 @@ def label_expert_launches(table):
     return gu, dn
 
 
-def source_hash() -> str:
+# the sources a kernel is compiled from (its own file and the headers it includes)
+KERNEL_SOURCES = {
+    "tc_gemm_kernel": ("umma.cu", "ptx.cuh", "common.cuh", "internal.h"),
+    "decode_kernel": ("decode.cu", "gemv_dev.cuh", "topk_dev.cuh", "ptx.cuh", "common.cuh", "internal.h"),
+}
+
+
+def source_hash(kernel: str = "") -> str:
+    """Hash of the sources of `kernel` (its base name), or of every CUDA source."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "sparse_moe_ffn_gemv_b200", "csrc")
-    for f in sorted(os.listdir(csrc)):
+    files = KERNEL_SOURCES.get(kernel.split("<")[0], None) or sorted(os.listdir(csrc))
+    for f in files:
         h.update(open(os.path.join(csrc, f), "rb").read())
     return h.hexdigest()[:16]
 
 
 def recorded_traffic(workload: str, T: int, kernel: str):
     """DRAM bytes per launch of a kernel from a committed ncu summary, only if it was
-    taken on the current kernel sources."""
+    taken on the kernel's current sources."""
     path = os.path.join(ROOT, "profiles", "traffic.json")
     if not os.path.exists(path):
         return None
     d = json.load(open(path))
     e = d.get(f"{workload}/T{T}/{kernel}")
-    if not e or e.get("source_hash") != source_hash():
+    if not e or e.get("source_hash") != source_hash(kernel):
         return None
     return e.get("dram_bytes_per_launch")
 
@@ -412,7 +432,7 @@ def max_over_ranks(v: float, dist, device) -> float:
 def reference_arm(args, rank, world):
     if rank != 0:
         return
-    spec = inputs.WORKLOADS[args.workload]
+    spec = workload_spec(args)
     T = args.tokens
     w_cpu = inputs.make_weights(spec)
     x_cpu = inputs.make_x(spec, T)
@@ -617,7 +637,7 @@ def run(args, rank, world, local, dist):
     dev = torch.device("cuda", local)
     pk, pk_src = peaks()
     cpu_ok = rank == 0 and world == 1 and not args.no_cpu_baseline
-    spec = inputs.WORKLOADS[args.workload]
+    spec = workload_spec(args)
     T = args.tokens
     w_cpu = inputs.make_weights(spec)
     x_cpu = inputs.make_x(spec, T)

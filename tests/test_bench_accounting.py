@@ -5,6 +5,7 @@ The roofline fractions divide these counts by measured times, so a wrong count (
 """
 import os
 import sys
+import pytest
 
 sys.path.insert(0, os.path.dirname(os.path.dirname(os.path.abspath(__file__))))
 
@@ -84,3 +85,16 @@ def test_dense_bytes_count_4bit_dense_planes_at_their_width():
     q4 = lambda r, c: r * c // 2 + r * (c // g) * 4
     assert bench.dense_bytes(s) == q4(E, H) + E * 4 + 2 * H * 2 + 3 * q4(Is, H)
     assert bench.dense_bytes(s) < bench.dense_bytes(inputs.KLEAR_Q4) / 3
+
+
+def test_smaller_copy_of_a_workload_keeps_every_other_field():
+    import bench
+    a = bench.parse(["--workload", "latent_bf16", "--tokens", "8192", "--experts", "32"])
+    s = bench.workload_spec(a)
+    full = bench.inputs.WORKLOADS["latent_bf16"]
+    assert s.num_experts == 32 and s.name == "latent_bf16_e32"
+    assert (s.hidden, s.latent_dim, s.top_k, s.intermediate, s.config_id) == \
+        (full.hidden, full.latent_dim, full.top_k, full.intermediate, full.config_id)
+    assert bench.workload_spec(bench.parse(["--workload", "klear_bf16"])) is bench.inputs.WORKLOADS["klear_bf16"]
+    with pytest.raises(SystemExit):
+        bench.workload_spec(bench.parse(["--workload", "klear_bf16", "--experts", "4"]))
