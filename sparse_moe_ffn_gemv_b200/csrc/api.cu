@@ -17,7 +17,7 @@ namespace moe {
 
 int64_t max_routed_tiles(const moe_config& c, int64_t T) {
     const int64_t S = T * c.top_k;
-    return (S + kTcBN - 1) / kTcBN + std::min<int64_t>(c.num_experts, S);
+    return (S + kTcBNQ4 - 1) / kTcBNQ4 + std::min<int64_t>(c.num_experts, S);  // the smallest tile height
 }
 
 WsLayout ws_layout(const moe_config& c, int64_t T) {
@@ -72,12 +72,12 @@ bool finite_pos(float v) { return std::isfinite(v) && v > 0.f; }
 
 bool dense_q4(const moe_config* c) { return c->dense_format == MOE_DTYPE_Q4_AFFINE; }
 
-// Token rows per tensor-core tile. 128 in launches that dequantise 4-bit weights (their
-// shared memory holds the packed-weight ring as well) and in small batches (four stages of
-// weights in flight per SM, where the launch streams weights for a few tokens); 256 in bf16
-// launches of large batches, where a weight tile then serves twice the token rows (an expert
-// with 129..256 routed rows reads its weights once instead of twice). The expert launches
-// carry the routed and the shared problem, the dense launches one projection.
+// Token rows per tensor-core tile. 96 in launches with 4-bit weights (their kernel keeps the
+// dequantised operand in TMEM beside two accumulator sets of 2 x 96 columns). bf16: 128 on
+// small batches (four stages of weights in flight per SM, where the launch streams weights
+// for a few tokens); 256 on large batches, where a weight tile then serves twice the token
+// rows (an expert with 129..256 routed rows reads its weights once instead of twice). The
+// expert launches carry the routed and the shared problem, the dense launches one projection.
 // Wide tiles keep one accumulator set (the epilogue of a tile no longer overlaps the next
 // tile's main loop), so they pay only where most experts hold more than 128 routed rows
 // (measured: latent block at 8192 tokens, 170 rows per expert on average, expert gate/up
@@ -86,11 +86,13 @@ bool dense_q4(const moe_config* c) { return c->dense_format == MOE_DTYPE_Q4_AFFI
 // 64 wide tiles: 84 -> 113 us).
 int expert_bn(const moe_config* c, int64_t T) {
     const bool q = c->weight_format == MOE_DTYPE_Q4_AFFINE || c->weight_format == MOE_DTYPE_MXFP4 || dense_q4(c);
-    return !q && T * c->top_k >= 160 * int64_t(c->num_experts) ? kTcBNWide : kTcBN;
+    if (q) return kTcBNQ4;
+    return T * c->top_k >= 160 * int64_t(c->num_experts) ? kTcBNWide : kTcBN;
 }
 int dense_bn(const moe_config* c, int64_t T, int M) {
+    if (dense_q4(c)) return kTcBNQ4;
     const int64_t wide_tiles = int64_t((M + kTcRows - 1) / kTcRows) * ((T + kTcBNWide - 1) / kTcBNWide);
-    return !dense_q4(c) && wide_tiles >= 2 * int64_t(device_sm_count()) ? kTcBNWide : kTcBN;
+    return wide_tiles >= 2 * int64_t(device_sm_count()) ? kTcBNWide : kTcBN;
 }
 
 // Weight operand(s) of a dense (one-group) tensor-core problem: bf16 [M, K], or 4-bit affine
