@@ -84,13 +84,19 @@ bool dense_q4(const moe_config* c) { return c->dense_format == MOE_DTYPE_Q4_AFFI
 // 2.97 -> 2.63 ms; Klear at 4096 tokens, 128 on average, block 0.71 -> 0.78 ms), and in dense
 // launches that still give every SM two tiles or more (a router of 384 rows at 8192 tokens has
 // 64 wide tiles: 84 -> 113 us).
+// 4-bit launches: the kernel with the dequantised operand in TMEM (96-token tiles) where the
+// experts hold few routed rows each, the one with dequantised shared-memory operand slots
+// (128-token tiles) on large batches.
+int q4_bn(const moe_config* c, int64_t T) {
+    return T * c->top_k < 32 * int64_t(c->num_experts) ? kTcBNQ4 : kTcBN;
+}
 int expert_bn(const moe_config* c, int64_t T) {
     const bool q = c->weight_format == MOE_DTYPE_Q4_AFFINE || c->weight_format == MOE_DTYPE_MXFP4 || dense_q4(c);
-    if (q) return kTcBNQ4;
+    if (q) return q4_bn(c, T);
     return T * c->top_k >= 160 * int64_t(c->num_experts) ? kTcBNWide : kTcBN;
 }
 int dense_bn(const moe_config* c, int64_t T, int M) {
-    if (dense_q4(c)) return kTcBNQ4;
+    if (dense_q4(c)) return q4_bn(c, T);
     const int64_t wide_tiles = int64_t((M + kTcRows - 1) / kTcRows) * ((T + kTcBNWide - 1) / kTcBNWide);
     return wide_tiles >= 2 * int64_t(device_sm_count()) ? kTcBNWide : kTcBN;
 }

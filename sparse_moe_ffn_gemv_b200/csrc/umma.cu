@@ -979,7 +979,8 @@ __global__ void __launch_bounds__(TcShape<GATEUP, BN, STAGES, Q4, PAIR>::THREADS
 //   warps 2..5   epilogue: thread = weight row (its TMEM lane) of both tiles, one token
 //                column at a time (h of 32 consecutive units per warp and token, or the
 //                weighted down row reduced into the token's fp32 routed sum)
-//   warps 6..13  dequantisation: warp w writes TMEM lanes 32 (w % 4) .. of tile (w - 6) / 4;
+//   warps 6..21  dequantisation: warp w writes TMEM lanes 32 (w % 4) .. of tile ((w - 6) / 4) % 2,
+//                the half (w - 6) / 8 of each K block (16 columns);
 //                a bf16 problem in the same launch (the shared expert) gets its two weight
 //                tiles into a shared-memory operand slot by TMA (A from a descriptor)
 // TMEM (512 columns): two accumulator sets of 2 x kQtBN columns (the epilogue of a tile
@@ -987,7 +988,7 @@ __global__ void __launch_bounds__(TcShape<GATEUP, BN, STAGES, Q4, PAIR>::THREADS
 constexpr int kQtBN = kTcBNQ4;   // token rows per tile
 constexpr int kQtStages = 6;     // load slots
 constexpr int kQtAStages = 2;    // operand slots (TMEM for 4-bit tiles, shared memory for bf16)
-constexpr int kQtDq = 256;       // dequantising threads: one weight row of one tile each
+constexpr int kQtDq = 512;       // dequantising threads: half a K block of one weight row each
 constexpr int kQtEpi = 128;      // epilogue threads: one weight row of both tiles each
 
 struct QtShape {
@@ -1019,15 +1020,13 @@ __device__ __forceinline__ void umma_ts(uint32_t d, uint32_t a_tmem, uint64_t b,
         "r"(a_tmem), "l"(b), "r"(idesc), "r"(acc)
         : "memory");
 }
-// Store 32 consecutive 32-bit columns of this thread's TMEM lane (warp-collective).
-__device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32]) {
+// Store 16 consecutive 32-bit columns of this thread's TMEM lane (warp-collective).
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16]) {
     asm volatile(
-        "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,"
-        "%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};" ::"r"(taddr),
+        "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(
+            taddr),
         "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]),
-        "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15]), "r"(r[16]),
-        "r"(r[17]), "r"(r[18]), "r"(r[19]), "r"(r[20]), "r"(r[21]), "r"(r[22]), "r"(r[23]), "r"(r[24]),
-        "r"(r[25]), "r"(r[26]), "r"(r[27]), "r"(r[28]), "r"(r[29]), "r"(r[30]), "r"(r[31])
+        "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
         : "memory");
 }
 __device__ __forceinline__ void tmem_st_wait() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
@@ -1205,7 +1204,9 @@ __global__ void __launch_bounds__(QtShape::THREADS, 1) tc_q4t_kernel(const __gri
         }
     } else if (int(threadIdx.x) >= S::DQ_BASE) {
         // ---------------------------------------------------------- dequantisation warps
-        const int a = (warp - S::DQ_BASE / 32) / 4;  // weight tile of this warp
+        const int dw = warp - S::DQ_BASE / 32;
+        const int a = (dw / 4) & 1;                    // weight tile of this warp
+        const int part = dw / 8;                       // its half of each K block
         const int q = warp & 3;                        // its TMEM lane quarter
         const int drow = q * 32 + lane;                // its row of the tile
         const bool leader = threadIdx.x == S::DQ_BASE;
@@ -1307,18 +1308,17 @@ __global__ void __launch_bounds__(QtShape::THREADS, 1) tc_q4t_kernel(const __gri
                             break;
                         }
                         tc_fence_after();  // the slot's previous MMAs have completed
-                        const uint4* pk = reinterpret_cast<const uint4*>(smem + stage * S::STAGE_BYTES + a * kPkBytes +
-                                                                         drow * 32);
-                        const uint4 w0 = pk[0], w1 = pk[1];
-                        const uint32_t words[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
-                        uint32_t v[32];  // the row's 64 weights as 16-bit pairs, in K order
+                        const uint4 w0 = *reinterpret_cast<const uint4*>(smem + stage * S::STAGE_BYTES + a * kPkBytes +
+                                                                         drow * 32 + part * 16);
+                        const uint32_t words[4] = {w0.x, w0.y, w0.z, w0.w};
+                        uint32_t v[16];  // 32 weights of the row as 16-bit pairs, in K order
 #pragma unroll
-                        for (int c = 0; c < 8; ++c) {
+                        for (int c = 0; c < 4; ++c) {
                             uint4 o;
                             if constexpr (MX) {
-                                o = dequant8_mx(words[c], sz[c >> 2]);
+                                o = dequant8_mx(words[c], sz[part]);
                             } else {
-                                const __half2 p2 = *reinterpret_cast<const __half2*>(&sz[c >> 2]);
+                                const __half2 p2 = *reinterpret_cast<const __half2*>(&sz[part]);
                                 o = dequant8_f16(words[c], __low2half2(p2), __high2half2(p2));
                             }
                             v[4 * c] = o.x;
@@ -1326,7 +1326,7 @@ __global__ void __launch_bounds__(QtShape::THREADS, 1) tc_q4t_kernel(const __gri
                             v[4 * c + 2] = o.z;
                             v[4 * c + 3] = o.w;
                         }
-                        tmem_st32(tmem_base + (uint32_t(q * 32) << 16) + S::A_COL0 + astage * 64 + a * 32, v);
+                        tmem_st16(tmem_base + (uint32_t(q * 32) << 16) + S::A_COL0 + astage * 64 + a * 32 + part * 16, v);
                         tmem_st_wait();
                         tc_fence_before();
                         __syncwarp();
@@ -1561,11 +1561,15 @@ cudaError_t launch_tc_gemm(TcParams& P, bool gateup, int64_t max_tiles, cudaStre
     // tile height, which picks the kernel: 128 rows with 4-bit weights or bf16, 256 with bf16
     const int bn = P.p[0].bn;
     for (int i = 0; i < P.nprob; ++i)
-        if (P.p[i].bn != bn || (q4 && bn != kTcBNQ4) || (!q4 && bn != kTcBN && bn != kTcBNWide))
+        if (P.p[i].bn != bn || (q4 && bn != kTcBNQ4 && bn != kTcBN) || (!q4 && bn != kTcBN && bn != kTcBNWide))
             return cudaErrorInvalidValue;
-    if (q4) {  // dequantised operands in TMEM, 96-token tiles
+    if (q4 && bn == kTcBNQ4) {  // dequantised operands in TMEM, 96-token tiles
         if (gateup) return launch_q4t<true>(P, max_tiles, s);
         return launch_q4t<false>(P, max_tiles, s);
+    }
+    if (q4) {  // six load slots (packed tiles + token tile) feed two dequantised shared-memory operand slots
+        if (gateup) return launch_tc_t<true, kTcBN, 6, true>(P, max_tiles, s);
+        return launch_tc_t<false, kTcBN, 6, true>(P, max_tiles, s);
     }
     if (bn == kTcBNWide) {
         // Dense launches: CTA pairs (six 32 KB stages per CTA). A pair's M = 256 MMA computes
