@@ -17,7 +17,7 @@ namespace moe {
 
 int64_t max_routed_tiles(const moe_config& c, int64_t T) {
     const int64_t S = T * c.top_k;
-    return (S + kTcBNQ4 - 1) / kTcBNQ4 + std::min<int64_t>(c.num_experts, S);  // the smallest tile height
+    return (S + kTcBN - 1) / kTcBN + std::min<int64_t>(c.num_experts, S);  // the smaller tile height
 }
 
 WsLayout ws_layout(const moe_config& c, int64_t T) {
@@ -72,33 +72,25 @@ bool finite_pos(float v) { return std::isfinite(v) && v > 0.f; }
 
 bool dense_q4(const moe_config* c) { return c->dense_format == MOE_DTYPE_Q4_AFFINE; }
 
-// Token rows per tensor-core tile. 96 in launches with 4-bit weights (their kernel keeps the
-// dequantised operand in TMEM beside two accumulator sets of 2 x 96 columns). bf16: 128 on
-// small batches (four stages of weights in flight per SM, where the launch streams weights
-// for a few tokens); 256 on large batches, where a weight tile then serves twice the token
-// rows (an expert with 129..256 routed rows reads its weights once instead of twice). The
-// expert launches carry the routed and the shared problem, the dense launches one projection.
-// Wide tiles keep one accumulator set (the epilogue of a tile no longer overlaps the next
-// tile's main loop), so they pay only where most experts hold more than 128 routed rows
-// (measured: latent block at 8192 tokens, 170 rows per expert on average, expert gate/up
-// 2.97 -> 2.63 ms; Klear at 4096 tokens, 128 on average, block 0.71 -> 0.78 ms), and in dense
-// launches that still give every SM two tiles or more (a router of 384 rows at 8192 tokens has
-// 64 wide tiles: 84 -> 113 us).
-// 4-bit launches: the kernel with the dequantised operand in TMEM (96-token tiles) where the
-// experts hold few routed rows each, the one with dequantised shared-memory operand slots
-// (128-token tiles) on large batches.
-int q4_bn(const moe_config* c, int64_t T) {
-    return T * c->top_k < 32 * int64_t(c->num_experts) ? kTcBNQ4 : kTcBN;
-}
+// Token rows per tensor-core tile. 128 in launches that dequantise 4-bit weights (their
+// shared memory holds the packed-weight ring as well) and on small bf16 batches (four stages
+// of weights in flight per SM, where the launch streams weights for a few tokens); 256 on
+// large bf16 batches, where a weight tile then serves twice the token rows (an expert with
+// 129..256 routed rows reads its weights once instead of twice). The expert launches carry
+// the routed and the shared problem, the dense launches one projection. Wide tiles keep one
+// accumulator set (the epilogue of a tile no longer overlaps the next tile's main loop), so
+// they pay only where most experts hold more than 128 routed rows (measured: latent block at
+// 8192 tokens, 170 rows per expert on average, expert gate/up 2.97 -> 2.63 ms; Klear at 4096
+// tokens, 128 on average, block 0.71 -> 0.78 ms), and in dense launches that still give
+// every SM two tiles or more (a router of 384 rows at 8192 tokens has 64 wide tiles: 84 ->
+// 113 us).
 int expert_bn(const moe_config* c, int64_t T) {
     const bool q = c->weight_format == MOE_DTYPE_Q4_AFFINE || c->weight_format == MOE_DTYPE_MXFP4 || dense_q4(c);
-    if (q) return q4_bn(c, T);
-    return T * c->top_k >= 160 * int64_t(c->num_experts) ? kTcBNWide : kTcBN;
+    return !q && T * c->top_k >= 160 * int64_t(c->num_experts) ? kTcBNWide : kTcBN;
 }
 int dense_bn(const moe_config* c, int64_t T, int M) {
-    if (dense_q4(c)) return q4_bn(c, T);
     const int64_t wide_tiles = int64_t((M + kTcRows - 1) / kTcRows) * ((T + kTcBNWide - 1) / kTcBNWide);
-    return wide_tiles >= 2 * int64_t(device_sm_count()) ? kTcBNWide : kTcBN;
+    return !dense_q4(c) && wide_tiles >= 2 * int64_t(device_sm_count()) ? kTcBNWide : kTcBN;
 }
 
 // Weight operand(s) of a dense (one-group) tensor-core problem: bf16 [M, K], or 4-bit affine

@@ -140,9 +140,8 @@ cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t s);
 
 // ------------------------------------------------------------------ tensor-core GEMM
 int device_sm_count();          // SMs of the current device (148 if the query fails)
-constexpr int kTcBN = 128;       // token rows per tile of bf16 launches on small batches
+constexpr int kTcBN = 128;       // token rows per tile (4-bit weights, small batches)
 constexpr int kTcBNWide = 256;   // token rows per tile of bf16 launches on large batches
-constexpr int kTcBNQ4 = 96;      // token rows per tile of launches with 4-bit weights
 constexpr int kTcRowsGateUp = 128;  // intermediate units per gate/up tile (gate + up rows)
 constexpr int kTcRows = 256;        // output rows per tile of the other GEMMs
 enum { kEpiGateUp = 0, kEpiScatterAdd = 1, kEpiStoreF32 = 2, kEpiStoreAct = 3 };

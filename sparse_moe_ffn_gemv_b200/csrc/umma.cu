@@ -178,6 +178,7 @@ struct TileInfo {
     int mb;        // weight-row block
     int row0;      // first B row (sorted position or token) of the tile
     int nvalid;    // valid token columns
+    int ntt;       // token tiles that share this tile's weight block (of its group)
 };
 
 // Tile tables of the (at most one) grouped problem, copied to shared memory at start.
@@ -206,6 +207,7 @@ __device__ __forceinline__ TileInfo decode_tile(const TcParams& P, const GroupTa
         const int nb = local - ti.mb * p.n_tiles;
         ti.row0 = nb * p.bn;
         ti.nvalid = min(p.bn, p.rows - ti.row0);
+        ti.ntt = p.n_tiles;
         return ti;
     }
     // largest e with tile_start[e] * m_blocks <= local (that expert is non-empty)
@@ -226,6 +228,7 @@ __device__ __forceinline__ TileInfo decode_tile(const TcParams& P, const GroupTa
     const int cnt = gt.off[e + 1] - off;
     ti.row0 = off + nb * p.bn;
     ti.nvalid = min(p.bn, cnt - nb * p.bn);
+    ti.ntt = nbe;
     return ti;
 }
 
@@ -460,9 +463,10 @@ __global__ void __launch_bounds__(TcShape<GATEUP, BN, STAGES, Q4, PAIR>::THREADS
         uint32_t stage = 0, phase = 0;
         uint32_t armed = 0;  // bit s: stage s was filled at least once
         uint32_t last_par = 0;
-        const uint64_t pol_w = policy_evict_first(), pol_t = policy_evict_last();
+        const uint64_t pol_w = policy_evict_first(), pol_n = policy_evict_normal(), pol_t = policy_evict_last();
         for (int tile = tile0; tile < total && !timed_out; tile += tstep) {
             const TileInfo ti = decode_tile(P, gt, tile, t0);
+            const uint64_t pw = ti.ntt > 1 ? pol_n : pol_w;  // weights shared by several token tiles
             const TcProblem& p = P.p[ti.prob];
             const int nk = p.K / kBK;
             const int mrow = ti.mb * S::ROWS;
@@ -488,11 +492,11 @@ __global__ void __launch_bounds__(TcShape<GATEUP, BN, STAGES, Q4, PAIR>::THREADS
                     if constexpr (Q4) {
                         if (p.q4) {  // packed words of the two weight tiles (8 words per K block)
                             mbar_expect_tx(&full[stage], 2 * kPkBytes + b_bytes);
-                            tma_3d(sb, &P.a0[ti.prob], &full[stage], kb * 8, mrow, ti.group, pol_w);
+                            tma_3d(sb, &P.a0[ti.prob], &full[stage], kb * 8, mrow, ti.group, pw);
                             if (!GATEUP)
-                                tma_3d(sb + kPkBytes, &P.a0[ti.prob], &full[stage], kb * 8, mrow + kBM, ti.group, pol_w);
+                                tma_3d(sb + kPkBytes, &P.a0[ti.prob], &full[stage], kb * 8, mrow + kBM, ti.group, pw);
                             else
-                                tma_3d(sb + kPkBytes, &P.a1[ti.prob], &full[stage], kb * 8, mrow, ti.group, pol_w);
+                                tma_3d(sb + kPkBytes, &P.a1[ti.prob], &full[stage], kb * 8, mrow, ti.group, pw);
                         } else {
                             mbar_expect_tx(&full[stage], b_bytes);
                         }
@@ -501,11 +505,11 @@ __global__ void __launch_bounds__(TcShape<GATEUP, BN, STAGES, Q4, PAIR>::THREADS
                         // leader's barrier, which the leader arms with the pair's total
                         const uint32_t fb = mapa_shared(&full[stage], 0);
                         if (crank == 0) mbar_expect_tx(&full[stage], pair_tx);
-                        load_a_pair<GATEUP>(sb, P, ti, mrow, kc, crank, fb, pol_w);
+                        load_a_pair<GATEUP>(sb, P, ti, mrow, kc, crank, fb, pw);
                         tma_2d_pair(sb + S::B_OFF, &P.b[ti.prob][bv], fb, kc, ti.row0 + kBM * int(crank), pol_t);
                     } else {
                         mbar_expect_tx(&full[stage], 2 * S::A_BYTES + b_bytes);
-                        load_a_bf16<GATEUP>(sb, P, ti, mrow, kc, &full[stage], pol_w);
+                        load_a_bf16<GATEUP>(sb, P, ti, mrow, kc, &full[stage], pw);
                     }
                     if constexpr (!PAIR) tma_2d(sb + S::B_OFF, &P.b[ti.prob][bv], &full[stage], kc, ti.row0, pol_t);
                 }
@@ -605,7 +609,7 @@ __global__ void __launch_bounds__(TcShape<GATEUP, BN, STAGES, Q4, PAIR>::THREADS
         uint32_t stage = 0, phase = 0;
         uint32_t astage = 0, aphase = 0;
         uint32_t a_armed = 0, a_last = 0;  // leader: operand slots it filled by TMA
-        const uint64_t pol_w = policy_evict_first();
+        const uint64_t pol_w = policy_evict_first(), pol_n = policy_evict_normal();
         auto next = [&]() {
             if (++stage == STAGES) {
                 stage = 0;
@@ -618,6 +622,7 @@ __global__ void __launch_bounds__(TcShape<GATEUP, BN, STAGES, Q4, PAIR>::THREADS
         };
         for (int tile = tile0; tile < total && !timed_out; tile += tstep) {
             const TileInfo ti = decode_tile(P, gt, tile, t0);
+            const uint64_t pw = ti.ntt > 1 ? pol_n : pol_w;  // weights shared by several token tiles
             const TcProblem& p = P.p[ti.prob];
             const int nk = p.K / kBK;
             const int mrow = ti.mb * S::ROWS;
@@ -631,7 +636,7 @@ __global__ void __launch_bounds__(TcShape<GATEUP, BN, STAGES, Q4, PAIR>::THREADS
                     if (leader) {
                         mbar_expect_tx(&dq[astage], 2 * S::A_BYTES);  // counts as this warp's arrive
                         load_a_bf16<GATEUP>(smem + S::ARING_OFF + astage * 2 * S::A_BYTES, P, ti, mrow, kb * kBK,
-                                            &dq[astage], pol_w);
+                                            &dq[astage], pw);
                         a_armed |= 1u << astage;
                         a_last = (a_last & ~(1u << astage)) | (aphase << astage);
                     } else if (lane == 0) {
@@ -963,474 +968,6 @@ __global__ void __launch_bounds__(TcShape<GATEUP, BN, STAGES, Q4, PAIR>::THREADS
     }
 }
 
-// ------------------------------------------------------------------ 4-bit weights, operand in TMEM
-// D[256 weight rows, N tokens] = W[rows, K] . U[tokens, K]^T as two M = 128 MMAs per K step
-// (weight tile 0 and 1: the gate and the up rows of 128 intermediate units, or 256 output
-// rows) with the dequantised weights as the A operand in tensor memory
-// (tcgen05.mma ... [d], [a_tmem], b_desc) and the tile's token rows as the B operand in shared
-// memory; N = the tile's valid token rows rounded up to 16, so small tiles cost little MMA
-// work. Each dequantising thread turns one weight row's 64 codes of a K block into fp16
-// (affine: s * q + b, one rounding) or bf16 (MXFP4, exact) and stores them to its TMEM lane
-// with one tcgen05.st: no dequantised tile passes through shared memory, which carries only
-// the TMA loads (packed words and token rows) and the MMA's token reads.
-//   warp 0       TMA producer: per K block the two packed tiles + the token tile into a
-//                kQtStages-deep ring of load slots
-//   warp 1       MMA issuer (one thread)
-//   warps 2..5   epilogue: thread = weight row (its TMEM lane) of both tiles, one token
-//                column at a time (h of 32 consecutive units per warp and token, or the
-//                weighted down row reduced into the token's fp32 routed sum)
-//   warps 6..21  dequantisation: warp w writes TMEM lanes 32 (w % 4) .. of tile ((w - 6) / 4) % 2,
-//                the half (w - 6) / 8 of each K block (16 columns);
-//                a bf16 problem in the same launch (the shared expert) gets its two weight
-//                tiles into a shared-memory operand slot by TMA (A from a descriptor)
-// TMEM (512 columns): two accumulator sets of 2 x kQtBN columns (the epilogue of a tile
-// overlaps the next tile's main loop) and kQtAStages operand slots of 2 x 32 columns.
-constexpr int kQtBN = kTcBNQ4;   // token rows per tile
-constexpr int kQtStages = 6;     // load slots
-constexpr int kQtAStages = 2;    // operand slots (TMEM for 4-bit tiles, shared memory for bf16)
-constexpr int kQtDq = 512;       // dequantising threads: half a K block of one weight row each
-constexpr int kQtEpi = 128;      // epilogue threads: one weight row of both tiles each
-
-struct QtShape {
-    static constexpr int A_BYTES = kBM * kBK * 2;                 // bf16 weight tile (shared-expert path)
-    static constexpr int B_BYTES = kQtBN * kBK * 2;               // token tile
-    static constexpr int B_OFF = 2 * kPkBytes;
-    static constexpr int STAGE_BYTES = 2 * kPkBytes + B_BYTES;    // 20 KB
-    static constexpr int BSLOT_OFF = kQtStages * STAGE_BYTES;     // bf16 operand slots
-    static constexpr int RING_BYTES = BSLOT_OFF + kQtAStages * 2 * A_BYTES;
-    static constexpr int THREADS = 64 + kQtEpi + kQtDq;
-    static constexpr int DQ_BASE = 64 + kQtEpi;
-    static constexpr int ACC_COLS = 2 * kQtBN;                    // one accumulator set
-    static constexpr int A_COL0 = 2 * ACC_COLS;                   // first operand-slot column
-    static constexpr int TMEM_COLS = 512;
-    static constexpr int SMEM = RING_BYTES + 1024 /*align*/ + 256 /*barriers*/ + int(sizeof(GroupTables));
-    static_assert(A_COL0 + kQtAStages * 64 <= TMEM_COLS, "TMEM columns");
-    static_assert(STAGE_BYTES % 1024 == 0 && B_OFF % 1024 == 0 && BSLOT_OFF % 1024 == 0, "1 KB aligned slots");
-    static_assert((2 * kQtStages + 5 + 2 * kQtAStages) * 8 + 4 <= 256, "barriers fit their region");
-    static_assert(SMEM <= 232448, "dynamic shared memory per block");
-};
-
-// MMA with the A operand in tensor memory (taddr of its first column; M = 128 lanes, 16 K
-// values in 8 columns of packed 16-bit pairs per K step).
-__device__ __forceinline__ void umma_ts(uint32_t d, uint32_t a_tmem, uint64_t b, uint32_t idesc, uint32_t acc) {
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "setp.ne.b32 p, %4, 0;\n\t"
-        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d),
-        "r"(a_tmem), "l"(b), "r"(idesc), "r"(acc)
-        : "memory");
-}
-// Store 16 consecutive 32-bit columns of this thread's TMEM lane (warp-collective).
-__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16]) {
-    asm volatile(
-        "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(
-            taddr),
-        "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]),
-        "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
-        : "memory");
-}
-__device__ __forceinline__ void tmem_st_wait() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
-
-template <bool GATEUP>
-__global__ void __launch_bounds__(QtShape::THREADS, 1) tc_q4t_kernel(const __grid_constant__ TcParams P) {
-    using S = QtShape;
-    constexpr int STAGES = kQtStages, AS = kQtAStages;
-    extern __shared__ uint8_t smem_raw[];
-    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    uint64_t* full = reinterpret_cast<uint64_t*>(smem + S::RING_BYTES);
-    uint64_t* empty = full + STAGES;
-    uint64_t* acc_full = empty + STAGES;
-    uint64_t* acc_empty = acc_full + 2;
-    uint64_t* drain = acc_empty + 2;
-    uint64_t* dq = drain + 1;      // operand slot filled (dequantised into TMEM, or bf16 by TMA)
-    uint64_t* aempty = dq + AS;    // operand slot consumed by the MMA
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(aempty + AS);
-    GroupTables& gt = *reinterpret_cast<GroupTables*>(smem + S::RING_BYTES + 256);
-
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    if (warp == 0) {
-        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(su32(tmem_slot)),
-                     "r"(uint32_t(S::TMEM_COLS)));
-        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
-    }
-    if (warp == 1 && lane == 0) {
-        for (int s = 0; s < STAGES; ++s) {
-            mbar_init(&full[s], 1);
-            mbar_init(&empty[s], 1);
-        }
-        for (int b = 0; b < 2; ++b) {
-            mbar_init(&acc_full[b], 1);
-            mbar_init(&acc_empty[b], kQtEpi / 32);  // one arrive per epilogue warp
-        }
-        mbar_init(drain, 1);
-        for (int st = 0; st < AS; ++st) {
-            mbar_init(&dq[st], kQtDq / 32);  // one arrive per dequantising warp
-            mbar_init(&aempty[st], 1);       // one MMA commit
-        }
-        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-    }
-    if (warp == 2 && lane == 0) {
-        for (int i = 0; i < P.nprob; ++i) {
-            prefetch_tmap(&P.a0[i]);
-            if (GATEUP && !P.p[i].interleaved) prefetch_tmap(&P.a1[i]);
-            for (int v = 0; v < 4; ++v) prefetch_tmap(&P.b[i][v]);
-        }
-    }
-    pdl_begin();  // everything above touches no memory that earlier kernels write
-    for (int i = 0; i < P.nprob; ++i) {
-        if (!P.p[i].grouped) continue;
-        for (int e = threadIdx.x; e <= P.p[i].num_groups; e += blockDim.x) {
-            gt.ts[e] = P.p[i].tile_start[e];
-            gt.off[e] = P.p[i].offsets[e];
-        }
-    }
-    tc_fence_before();
-    __syncthreads();
-    tc_fence_after();
-    const uint32_t tmem_base = *tmem_slot;
-
-    const int t0 = problem_tiles(P.p[0], gt);
-    const int total = t0 + (P.nprob > 1 ? problem_tiles(P.p[1], gt) : 0);
-    const uint64_t deadline = gtimer() + kWaitNs;
-    bool timed_out = false;
-    constexpr int ROWS = GATEUP ? kBM : 2 * kBM;  // weight rows (units) per tile
-
-    if (warp == 0) {
-        // -------------------------------------------------------------- TMA producer
-        // 4-bit problem: the two packed tiles + the token tile per K block; bf16 problem:
-        // the token tile only (the first dequantising thread loads its weight tiles).
-        uint32_t stage = 0, phase = 0;
-        uint32_t armed = 0, last_par = 0;
-        const uint64_t pol_w = policy_evict_first(), pol_t = policy_evict_last();
-        for (int tile = blockIdx.x; tile < total && !timed_out; tile += gridDim.x) {
-            const TileInfo ti = decode_tile(P, gt, tile, t0);
-            const TcProblem& p = P.p[ti.prob];
-            const int nk = p.K / kBK;
-            const int mrow = ti.mb * ROWS;
-            // the smallest token box (16, 32, 64 or kQtBN rows) that holds the valid rows
-            const int bv = ti.nvalid <= 16 ? 0 : ti.nvalid <= 32 ? 1 : ti.nvalid <= 64 ? 2 : 3;
-            const uint32_t b_bytes = uint32_t(min(kQtBN, 16 << bv)) * kBK * 2;
-            for (int kb = 0; kb < nk; ++kb) {
-                int ok = 1;
-                if (lane == 0) ok = mbar_wait(&empty[stage], phase ^ 1u, deadline) ? 1 : 0;
-                if (!__shfl_sync(0xffffffffu, ok, 0)) {
-                    timed_out = true;
-                    break;
-                }
-                uint8_t* sb = smem + stage * S::STAGE_BYTES;
-                if (lane == 0) {
-                    if (p.q4) {  // packed words of the two weight tiles (8 words per row and K block)
-                        mbar_expect_tx(&full[stage], 2 * kPkBytes + b_bytes);
-                        tma_3d(sb, &P.a0[ti.prob], &full[stage], kb * 8, mrow, ti.group, pol_w);
-                        if (!GATEUP)
-                            tma_3d(sb + kPkBytes, &P.a0[ti.prob], &full[stage], kb * 8, mrow + kBM, ti.group, pol_w);
-                        else
-                            tma_3d(sb + kPkBytes, &P.a1[ti.prob], &full[stage], kb * 8, mrow, ti.group, pol_w);
-                    } else {
-                        mbar_expect_tx(&full[stage], b_bytes);
-                    }
-                    tma_2d(sb + S::B_OFF, &P.b[ti.prob][bv], &full[stage], kb * kBK, ti.row0, pol_t);
-                }
-                armed |= 1u << stage;
-                last_par = (last_par & ~(1u << stage)) | (phase << stage);
-                if (++stage == STAGES) {
-                    stage = 0;
-                    phase ^= 1u;
-                }
-            }
-        }
-        if (lane == 0) {  // drain: every copy this warp issued has landed
-            const uint64_t dl2 = gtimer() + kWaitNs;
-            for (int s = 0; s < STAGES; ++s)
-                if ((armed >> s) & 1u) mbar_wait(&full[s], (last_par >> s) & 1u, dl2);
-            if (timed_out) set_status(P.status, MOE_ERR_DEVICE_TIMEOUT);
-        }
-        __syncwarp();
-    } else if (warp == 1) {
-        if (lane == 0) {
-            // ---------------------------------------------------------- MMA issuer
-            uint32_t stage = 0, phase = 0, it = 0, astage = 0, aphase = 0;
-            for (int tile = blockIdx.x; tile < total && !timed_out; tile += gridDim.x, ++it) {
-                const TileInfo ti = decode_tile(P, gt, tile, t0);
-                const TcProblem& p = P.p[ti.prob];
-                const uint32_t ab = it & 1u, aph = (it >> 1) & 1u;
-                if (!mbar_wait(&acc_empty[ab], aph ^ 1u, deadline)) {
-                    timed_out = true;
-                    break;
-                }
-                tc_fence_after();
-                // N = valid token rows rounded up to 16 (the M = 128 minimum step)
-                const int n_mma = min(kQtBN, max(16, (ti.nvalid + 15) & ~15));
-                const uint32_t idesc = (p.q4 && !p.mx) ? idesc_f16(n_mma) : idesc_bf16(n_mma);
-                const uint32_t d0 = tmem_base + ab * S::ACC_COLS;
-                const int nk = p.K / kBK;
-                for (int kb = 0; kb < nk; ++kb) {
-                    // the operand slot is complete once the dequantising warps have filled it,
-                    // which they do only after the load slot (token tile) landed
-                    if (!mbar_wait(&dq[astage], aphase, deadline)) {
-                        timed_out = true;
-                        break;
-                    }
-                    tc_fence_after();
-                    const uint32_t st = su32(smem + stage * S::STAGE_BYTES + S::B_OFF);
-                    const uint32_t ta = tmem_base + S::A_COL0 + astage * 64;  // TMEM operand slot
-                    const uint32_t sw = su32(smem + S::BSLOT_OFF + astage * 2 * S::A_BYTES);
-#pragma unroll
-                    for (int a = 0; a < 2; ++a)
-#pragma unroll
-                        for (int k = 0; k < kBK / 16; ++k) {
-                            const uint32_t acc = (kb > 0 || k > 0) ? 1u : 0u;
-                            if (p.q4) umma_ts(d0 + a * kQtBN, ta + a * 32 + k * 8, smem_desc(st + k * 32), idesc, acc);
-                            else umma(d0 + a * kQtBN, smem_desc(sw + a * S::A_BYTES + k * 32), smem_desc(st + k * 32), idesc, acc);
-                        }
-                    umma_commit(&empty[stage]);
-                    umma_commit(&aempty[astage]);
-                    if (++stage == STAGES) {
-                        stage = 0;
-                        phase ^= 1u;
-                    }
-                    if (++astage == uint32_t(AS)) {
-                        astage = 0;
-                        aphase ^= 1u;
-                    }
-                }
-                if (timed_out) break;
-                umma_commit(&acc_full[ab]);
-            }
-            umma_commit(drain);  // all MMAs issued by this thread have completed
-            mbar_wait(drain, 0, gtimer() + kWaitNs);
-            if (timed_out) set_status(P.status, MOE_ERR_DEVICE_TIMEOUT);
-        }
-    } else if (int(threadIdx.x) >= S::DQ_BASE) {
-        // ---------------------------------------------------------- dequantisation warps
-        const int dw = warp - S::DQ_BASE / 32;
-        const int a = (dw / 4) & 1;                    // weight tile of this warp
-        const int part = dw / 8;                       // its half of each K block
-        const int q = warp & 3;                        // its TMEM lane quarter
-        const int drow = q * 32 + lane;                // its row of the tile
-        const bool leader = threadIdx.x == S::DQ_BASE;
-        uint32_t stage = 0, phase = 0, astage = 0, aphase = 0;
-        uint32_t a_armed = 0, a_last = 0;  // leader: operand slots it filled by TMA
-        const uint64_t pol_w = policy_evict_first();
-        auto next = [&]() {
-            if (++stage == STAGES) {
-                stage = 0;
-                phase ^= 1u;
-            }
-            if (++astage == uint32_t(AS)) {
-                astage = 0;
-                aphase ^= 1u;
-            }
-        };
-        for (int tile = blockIdx.x; tile < total && !timed_out; tile += gridDim.x) {
-            const TileInfo ti = decode_tile(P, gt, tile, t0);
-            const TcProblem& p = P.p[ti.prob];
-            const int nk = p.K / kBK;
-            const int mrow = ti.mb * ROWS;
-            if (!p.q4) {  // bf16 tile: the leader loads both weight tiles into the operand slot
-                for (int kb = 0; kb < nk; ++kb) {
-                    if (!mbar_wait(&full[stage], phase, deadline) || !mbar_wait(&aempty[astage], aphase ^ 1u, deadline)) {
-                        timed_out = true;
-                        break;
-                    }
-                    __syncwarp();
-                    if (leader) {
-                        mbar_expect_tx(&dq[astage], 2 * S::A_BYTES);  // counts as this warp's arrive
-                        load_a_bf16<GATEUP>(smem + S::BSLOT_OFF + astage * 2 * S::A_BYTES, P, ti, mrow, kb * kBK,
-                                            &dq[astage], pol_w);
-                        a_armed |= 1u << astage;
-                        a_last = (a_last & ~(1u << astage)) | (aphase << astage);
-                    } else if (lane == 0) {
-                        mbar_arrive(&dq[astage]);
-                    }
-                    next();
-                }
-                continue;
-            }
-            // this row's scale / bias companions (rows past M read row M - 1: their results
-            // are discarded); byte addresses of bf16 scales and biases, or MXFP4 scale bytes
-            const int ng = p.K / p.group_size;
-            const int r = min(mrow + (GATEUP ? 0 : a * kBM) + drow, p.M - 1);
-            const int64_t off = (int64_t(ti.group) * p.M + r) * p.qrow_step * ng;
-            const unsigned char* sp = static_cast<const unsigned char*>((GATEUP && a == 1) ? p.qs1 : p.qs0) +
-                                      off * (p.mx ? 1 : 2);
-            const unsigned char* zp =
-                p.mx ? nullptr : static_cast<const unsigned char*>((GATEUP && a == 1) ? p.qz1 : p.qz0) + off * 2;
-            const bool two = p.group_size == 32;
-            auto run = [&](auto mx_tag) {
-                constexpr bool MX = decltype(mx_tag)::value;
-                // raw scale / bias words of K block kb (group 32: both groups of the block in
-                // one word; larger groups: one value for both halves; MXFP4: two scale bytes)
-                auto load_raw = [&](int kb, uint32_t& rs, uint32_t& rz) {
-                    const int g = (kb * kBK) / p.group_size;
-                    if constexpr (MX) {
-                        rs = __ldg(reinterpret_cast<const unsigned short*>(sp + g));
-                        rz = 0;
-                    } else if (two) {
-                        rs = __ldg(reinterpret_cast<const unsigned int*>(sp) + g / 2);
-                        rz = __ldg(reinterpret_cast<const unsigned int*>(zp) + g / 2);
-                    } else {
-                        rs = __ldg(reinterpret_cast<const unsigned short*>(sp) + g);
-                        rz = __ldg(reinterpret_cast<const unsigned short*>(zp) + g);
-                    }
-                };
-                // the words of the next kPre blocks in a statically indexed register ring
-                constexpr int kPre = 2;
-                uint32_t rs[kPre], rz[kPre];
-#pragma unroll
-                for (int j = 0; j < kPre; ++j)
-                    if (j < nk) load_raw(j, rs[j], rz[j]);
-                for (int kb0 = 0; kb0 < nk && !timed_out; kb0 += kPre) {
-#pragma unroll
-                    for (int j = 0; j < kPre; ++j) {
-                        const int kb = kb0 + j;
-                        if (kb >= nk) break;
-                        __nv_bfloat162 sz[2];  // the pair of each 32-wide half of the block
-#pragma unroll
-                        for (int h = 0; h < 2; ++h) {
-                            if constexpr (MX) {
-                                const uint32_t sbyte = (rs[j] >> (8 * h)) & 0xFFu;
-                                const __nv_bfloat16 sc = __ushort_as_bfloat16(uint16_t(sbyte ? (sbyte << 7) : 0x0040u));
-                                sz[h] = __halves2bfloat162(sc, sc);
-                            } else {
-                                const int sh = (two && h == 1) ? 16 : 0;
-                                const __half2 v = __floats2half2_rn(
-                                    __bfloat162float(__ushort_as_bfloat16(uint16_t(rs[j] >> sh))),
-                                    __bfloat162float(__ushort_as_bfloat16(uint16_t(rz[j] >> sh))));
-                                sz[h] = *reinterpret_cast<const __nv_bfloat162*>(&v);
-                            }
-                        }
-                        if (kb + kPre < nk) load_raw(kb + kPre, rs[j], rz[j]);
-                        if (!mbar_wait(&full[stage], phase, deadline) ||
-                            !mbar_wait(&aempty[astage], aphase ^ 1u, deadline)) {
-                            timed_out = true;
-                            break;
-                        }
-                        tc_fence_after();  // the slot's previous MMAs have completed
-                        const uint4 w0 = *reinterpret_cast<const uint4*>(smem + stage * S::STAGE_BYTES + a * kPkBytes +
-                                                                         drow * 32 + part * 16);
-                        const uint32_t words[4] = {w0.x, w0.y, w0.z, w0.w};
-                        uint32_t v[16];  // 32 weights of the row as 16-bit pairs, in K order
-#pragma unroll
-                        for (int c = 0; c < 4; ++c) {
-                            uint4 o;
-                            if constexpr (MX) {
-                                o = dequant8_mx(words[c], sz[part]);
-                            } else {
-                                const __half2 p2 = *reinterpret_cast<const __half2*>(&sz[part]);
-                                o = dequant8_f16(words[c], __low2half2(p2), __high2half2(p2));
-                            }
-                            v[4 * c] = o.x;
-                            v[4 * c + 1] = o.y;
-                            v[4 * c + 2] = o.z;
-                            v[4 * c + 3] = o.w;
-                        }
-                        tmem_st16(tmem_base + (uint32_t(q * 32) << 16) + S::A_COL0 + astage * 64 + a * 32 + part * 16, v);
-                        tmem_st_wait();
-                        tc_fence_before();
-                        __syncwarp();
-                        if (lane == 0) mbar_arrive(&dq[astage]);
-                        next();
-                    }
-                }
-            };
-            if (p.mx) run(std::true_type{});
-            else run(std::false_type{});
-        }
-        if (leader) {  // drain: the operand loads the leader issued have landed
-            const uint64_t dl2 = gtimer() + kWaitNs;
-            for (int s = 0; s < AS; ++s)
-                if ((a_armed >> s) & 1u) mbar_wait(&dq[s], (a_last >> s) & 1u, dl2);
-        }
-        if (timed_out) set_status(P.status, MOE_ERR_DEVICE_TIMEOUT);
-    } else {
-        // -------------------------------------------------------------- epilogue (4 warps)
-        // Accumulator lane = weight row of the tile, column = token. Thread = row q * 32 + lane
-        // of both tiles: in gate/up mode the gate and the up row of one unit, else output rows
-        // r and r + 128. One token column at a time, so that a warp writes 32 consecutive
-        // units (or output rows) of one token row per store.
-        const int q = warp & 3;
-        const int rt = q * 32 + lane;
-        uint32_t it = 0;
-        for (int tile = blockIdx.x; tile < total; tile += gridDim.x, ++it) {
-            const TileInfo ti = decode_tile(P, gt, tile, t0);
-            const TcProblem& p = P.p[ti.prob];
-            const uint32_t ab = it & 1u, aph = (it >> 1) & 1u;
-            const int64_t g = ti.group;
-            const int r0 = ti.mb * ROWS + rt;               // unit (gate/up) or output row of tile 0
-            const int r1 = GATEUP ? r0 : r0 + kBM;          // its row in tile 1
-            float b0 = 0.f, b1 = 0.f;                       // biases, before the wait
-            if (p.bias0) {
-                if (GATEUP) {
-                    if (r0 < p.M) {
-                        b0 = p.bias_interleaved ? bf16_at(p.bias0, (g * p.M + r0) * 2) : bf16_at(p.bias0, g * p.M + r0);
-                        b1 = p.bias_interleaved ? bf16_at(p.bias0, (g * p.M + r0) * 2 + 1) : bf16_at(p.bias1, g * p.M + r0);
-                    }
-                } else {
-                    if (r0 < p.M) b0 = bf16_at(p.bias0, g * p.M + r0);
-                    if (r1 < p.M) b1 = bf16_at(p.bias0, g * p.M + r1);
-                }
-            }
-            if (!mbar_wait_sleep(&acc_full[ab], aph, deadline)) {
-                set_status(P.status, MOE_ERR_DEVICE_TIMEOUT);
-                break;
-            }
-            tc_fence_after();
-            const uint32_t tb = tmem_base + (uint32_t(q * 32) << 16) + ab * S::ACC_COLS;
-            const int nv = ti.nvalid;
-            for (int c0 = 0; c0 < nv; c0 += 16) {
-                uint32_t x0[16], x1[16];
-                tmem_ld_issue(tb + c0, x0);
-                tmem_ld_issue(tb + kQtBN + c0, x1);
-                tmem_ld_wait(x0);
-                tmem_ld_wait(x1);
-#pragma unroll
-                for (int j = 0; j < 16; ++j) {  // fully unrolled: the registers stay registers
-                    const int t = c0 + j;
-                    if (t >= nv) break;
-                    const int64_t prow = int64_t(ti.row0) + t;
-                    const float v0 = __uint_as_float(x0[j]) + b0, v1 = __uint_as_float(x1[j]) + b1;
-                    if constexpr (GATEUP) {
-                        if (r0 < p.M) {
-                            const float h = act_fast(P.act, v0, v1, P.limit, P.alpha);
-                            if (p.out_f16) reinterpret_cast<__half*>(p.out)[prow * p.ld_out + r0] = __float2half_rn(h);
-                            else reinterpret_cast<__nv_bfloat16*>(p.out)[prow * p.ld_out + r0] = __float2bfloat16_rn(h);
-                        }
-                    } else if (p.mode == kEpiScatterAdd) {
-                        // weighted combine into the token's fp32 routed sum (libmir-metal
-                        // execute: down weighted by routing.weights and summed per token)
-                        const int slot = p.sorted_slot[prow];
-                        const float w = p.topk_w[slot];
-                        float* yrow = reinterpret_cast<float*>(p.out) + int64_t(slot / p.k) * p.ld_out;
-                        if (r0 < p.M) atomicAdd(yrow + r0, w * v0);
-                        if (r1 < p.M) atomicAdd(yrow + r1, w * v1);
-                    } else if (p.mode == kEpiStoreF32) {
-                        float* dst = reinterpret_cast<float*>(p.out) + prow * p.ld_out;
-                        if (r0 < p.M) dst[r0] = v0;
-                        if (r1 < p.M) dst[r1] = v1;
-                    } else {  // kEpiStoreAct (+ optional fp32 addend)
-                        __nv_bfloat16* dst = reinterpret_cast<__nv_bfloat16*>(p.out) + prow * p.ld_out;
-                        const float* ad = p.addend ? p.addend + prow * p.ld_add : nullptr;
-                        if (r0 < p.M) dst[r0] = __float2bfloat16_rn(v0 + (ad ? ad[r0] : 0.f));
-                        if (r1 < p.M) dst[r1] = __float2bfloat16_rn(v1 + (ad ? ad[r1] : 0.f));
-                    }
-                }
-            }
-            tc_fence_before();  // the accumulator set is free for the tile after next
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&acc_empty[ab]);
-        }
-    }
-    tc_fence_before();
-    __syncthreads();
-    if (warp == 0) {
-        tc_fence_after();
-        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base),
-                     "r"(uint32_t(S::TMEM_COLS)));
-    }
-}
-
 // ------------------------------------------------------------------ host side
 using EncodeFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
                               const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
@@ -1499,17 +1036,6 @@ cudaError_t launch_tc_t(TcParams& P, int64_t max_tiles, cudaStream_t s) {
     return cudaGetLastError();
 }
 
-template <bool GATEUP>
-cudaError_t launch_q4t(TcParams& P, int64_t max_tiles, cudaStream_t s) {
-    auto kern = tc_q4t_kernel<GATEUP>;
-    cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, QtShape::SMEM);
-    if (err != cudaSuccess) return err;
-    const int grid = int(std::min<int64_t>(max_tiles, sm_count()));
-    if (grid <= 0) return cudaSuccess;
-    { const cudaError_t e_ = launch_pdl(kern, dim3(grid), dim3(QtShape::THREADS), QtShape::SMEM, s, P); if (e_ != cudaSuccess) return e_; }
-    return cudaGetLastError();
-}
-
 }  // namespace
 
 // Weight operand: [E, R, K] bf16 (E = 1 for a dense matrix), or the interleaved
@@ -1561,12 +1087,7 @@ cudaError_t launch_tc_gemm(TcParams& P, bool gateup, int64_t max_tiles, cudaStre
     // tile height, which picks the kernel: 128 rows with 4-bit weights or bf16, 256 with bf16
     const int bn = P.p[0].bn;
     for (int i = 0; i < P.nprob; ++i)
-        if (P.p[i].bn != bn || (q4 && bn != kTcBNQ4 && bn != kTcBN) || (!q4 && bn != kTcBN && bn != kTcBNWide))
-            return cudaErrorInvalidValue;
-    if (q4 && bn == kTcBNQ4) {  // dequantised operands in TMEM, 96-token tiles
-        if (gateup) return launch_q4t<true>(P, max_tiles, s);
-        return launch_q4t<false>(P, max_tiles, s);
-    }
+        if (P.p[i].bn != bn || (q4 && bn != kTcBN) || (bn != kTcBN && bn != kTcBNWide)) return cudaErrorInvalidValue;
     if (q4) {  // six load slots (packed tiles + token tile) feed two dequantised shared-memory operand slots
         if (gateup) return launch_tc_t<true, kTcBN, 6, true>(P, max_tiles, s);
         return launch_tc_t<false, kTcBN, 6, true>(P, max_tiles, s);
