@@ -723,6 +723,9 @@ __global__ void __launch_bounds__(TcShape<GATEUP, BN, STAGES, Q4, PAIR>::THREADS
                     timed_out = true;
                     break;
                 }
+                // this slot's last use is no longer the leader's copy (the MMA consumed it
+                // before the slot came free), so the exit drain must not wait on that phase
+                if (leader) a_armed &= ~(1u << astage);
                 const uint8_t* lb = smem + stage * S::STAGE_BYTES;
                 uint8_t* ob = smem + S::ARING_OFF + astage * 2 * S::A_BYTES;
 #pragma unroll
@@ -757,6 +760,8 @@ __global__ void __launch_bounds__(TcShape<GATEUP, BN, STAGES, Q4, PAIR>::THREADS
             else run(std::false_type{});
         }
         // drain: the operand loads the leader issued have landed before the CTA can exit
+        // (only slots whose last use was such a load: a later 4-bit use of the slot moved its
+        // barrier on, and waiting for the old parity would wait for a phase that never comes)
         if (leader) {
             const uint64_t dl2 = gtimer() + kWaitNs;
             for (int s = 0; s < S::ASTAGES; ++s)

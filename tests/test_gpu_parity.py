@@ -529,3 +529,31 @@ def test_expert_parallel_block_on_one_rank_equals_the_block():
     rms = float(ref.pow(2).mean().sqrt())
     ulp = torch.exp2(torch.floor(torch.log2(ref.abs().clamp_min(1e-30))) - 7)
     assert bool(((y.float() - ref).abs() <= 2 * 2e-2 * rms + ulp).all())
+
+
+def test_4bit_tiles_after_bf16_shared_tiles_end_without_a_stalled_drain(monkeypatch):
+    """More tensor-core tiles than SMs, so that CTAs run bf16 shared-expert tiles and then 4-bit
+    routed tiles with an odd number of K blocks (hidden 192): the dequantising warps' exit
+    drain must wait only for copies still in flight. Waiting for the parity of an operand
+    slot whose barrier later 4-bit tiles moved on gives up only at the 2 s bound (and sets no
+    status), so a forward of this size must take milliseconds. Checked against the oracle."""
+    monkeypatch.setenv("MOE_PATH", "tc")
+    spec, T = ts.Q4_ODD_K, 8192
+    wcpu, wnp = weights(spec)
+    x_cpu = inputs.make_x(spec, T)
+    blk = M.MoeBlock(spec, wcpu, max_tokens=T)
+    x = x_cpu.cuda()
+    blk.forward(x)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    y = blk.forward(x)
+    e1.record()
+    torch.cuda.synchronize()
+    assert blk.device_status() == 0
+    assert e0.elapsed_time(e1) < 200.0, f"forward took {e0.elapsed_time(e1):.1f} ms"
+    y, idx, _, _ = run_gpu(spec, wcpu, x_cpu, block=blk)
+    x_np = inputs.to_numpy_storage(x_cpu)
+    rng = np.random.default_rng(T)
+    tokens = np.unique(np.concatenate([[0], np.arange(T - 32, T), rng.choice(T, size=223, replace=False)]))
+    check_block(spec, wnp, x_np, tokens, y[tokens], idx[tokens], label=f"{spec.name} T={T}")

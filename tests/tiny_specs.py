@@ -71,6 +71,13 @@ WIDE = MoeSpec(
     name="t_wide", config_id=113, hidden=128, num_experts=4, top_k=2, intermediate=128,
     scoring="softmax_topk", activation="swiglu_clamped", gate_up_interleaved=True,
     has_expert_bias=True, shared_mode="blend", shared_intermediate=64)
+# 4-bit routed experts with a bf16 shared expert and an odd number of 64-wide K blocks
+# (hidden 192): in a batch with more tensor-core tiles than SMs a CTA runs shared-expert bf16
+# tiles and then 4-bit tiles, which move its operand-slot barriers an odd number of phases on
+Q4_ODD_K = MoeSpec(
+    name="t_q4_odd_k", config_id=115, hidden=192, num_experts=8, top_k=2, intermediate=128,
+    scoring="sigmoid", has_selection_bias=True, norm_topk_prob=True, weight_format="q4",
+    group_size=64, shared_mode="add", shared_intermediate=128)
 LATENT_WIDE = MoeSpec(
     name="t_latent_wide", config_id=114, hidden=512, num_experts=6, top_k=2, intermediate=128,
     scoring="sigmoid", has_selection_bias=True, norm_topk_prob=True, shared_mode="add",
