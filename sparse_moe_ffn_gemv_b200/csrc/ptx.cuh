@@ -90,8 +90,9 @@ __device__ bool grid_barrier(unsigned* ctr, unsigned target, uint64_t deadline, 
 
 // L2 policies: weights read by one token tile stream through once (evict first), weights
 // shared by several token tiles stay at normal priority until the other tiles, which run at
-// about the same time on other SMs, have read them; token tiles are re-read by every
-// weight-row block of their group (evict last).
+// about the same time on other SMs, have read them; the token rows of a dense problem are
+// re-read by every weight-row block of the launch (evict last); routed token rows only by
+// their expert's blocks, which run together (normal).
 __device__ __forceinline__ uint64_t policy_evict_first() {
     uint64_t p;
     asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));

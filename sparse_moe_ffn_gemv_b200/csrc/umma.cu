@@ -286,8 +286,13 @@ __device__ __forceinline__ float act_fast(int act, float g, float v, float limit
 }
 
 // Fire-and-forget add of four consecutive fp32 values in global memory (16-byte aligned).
-__device__ __forceinline__ void red_add_v4(float* p, float a, float b, float c, float d) {
-    asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(p), "f"(a), "f"(b), "f"(c), "f"(d) : "memory");
+// The routed sums are the target of every slot's reduction, spread over the whole launch:
+// they carry an L2 evict-last hint so that the streamed weights and token rows do not push
+// them out between the reductions of their token's slots.
+__device__ __forceinline__ void red_add_v4(float* p, float a, float b, float c, float d, uint64_t pol) {
+    asm volatile("red.global.add.L2::cache_hint.v4.f32 [%0], {%1, %2, %3, %4}, %5;" ::"l"(p), "f"(a), "f"(b), "f"(c),
+                 "f"(d), "l"(pol)
+                 : "memory");
 }
 
 __device__ __forceinline__ float bf16_at(const void* p, int64_t i) {
@@ -467,7 +472,10 @@ __global__ void __launch_bounds__(TcShape<GATEUP, BN, STAGES, Q4, PAIR>::THREADS
         for (int tile = tile0; tile < total && !timed_out; tile += tstep) {
             const TileInfo ti = decode_tile(P, gt, tile, t0);
             const uint64_t pw = ti.ntt > 1 ? pol_n : pol_w;  // weights shared by several token tiles
+            // token rows: a dense batch is re-read by every weight-row block (kept); routed rows
+            // are re-read only by their expert's blocks, which run at about the same time
             const TcProblem& p = P.p[ti.prob];
+            const uint64_t pt = p.grouped ? pol_n : pol_t;
             const int nk = p.K / kBK;
             const int mrow = ti.mb * S::ROWS;
             // token rows: the smallest box (16, 32, 64, 128, 256 rows) that holds the valid tokens
@@ -506,12 +514,12 @@ __global__ void __launch_bounds__(TcShape<GATEUP, BN, STAGES, Q4, PAIR>::THREADS
                         const uint32_t fb = mapa_shared(&full[stage], 0);
                         if (crank == 0) mbar_expect_tx(&full[stage], pair_tx);
                         load_a_pair<GATEUP>(sb, P, ti, mrow, kc, crank, fb, pw);
-                        tma_2d_pair(sb + S::B_OFF, &P.b[ti.prob][bv], fb, kc, ti.row0 + kBM * int(crank), pol_t);
+                        tma_2d_pair(sb + S::B_OFF, &P.b[ti.prob][bv], fb, kc, ti.row0 + kBM * int(crank), pt);
                     } else {
                         mbar_expect_tx(&full[stage], 2 * S::A_BYTES + b_bytes);
                         load_a_bf16<GATEUP>(sb, P, ti, mrow, kc, &full[stage], pw);
                     }
-                    if constexpr (!PAIR) tma_2d(sb + S::B_OFF, &P.b[ti.prob][bv], &full[stage], kc, ti.row0, pol_t);
+                    if constexpr (!PAIR) tma_2d(sb + S::B_OFF, &P.b[ti.prob][bv], &full[stage], kc, ti.row0, pt);
                 }
                 armed |= 1u << stage;
                 last_par = (last_par & ~(1u << stage)) | (phase << stage);
@@ -780,6 +788,7 @@ __global__ void __launch_bounds__(TcShape<GATEUP, BN, STAGES, Q4, PAIR>::THREADS
         // TMEM columns per epilogue step: 16 beside the 4-bit kernel's 16 dequantising warps
         // (704 threads leave 80 registers per thread), 32 otherwise
         constexpr int CW = Q4 ? 16 : 32;
+        const uint64_t pol_y = policy_evict_last();  // routed-sum reductions
         const int th = S::MH == 2 ? (eid >= 128 ? 1 : 0) : 0;  // token half of this warp
         const int tok = (PAIR ? int(crank) : th) * kBM + q * 32 + lane;  // token row of the tile
         constexpr int NH = S::NH;                               // column halves per warp
@@ -913,7 +922,8 @@ __global__ void __launch_bounds__(TcShape<GATEUP, BN, STAGES, Q4, PAIR>::THREADS
                             // summed per token); M is a multiple of 64 here
 #pragma unroll
                             for (int j = 0; j < CW; j += 4)
-                                red_add_v4(yrow + r0 + j, wslot * o[j], wslot * o[j + 1], wslot * o[j + 2], wslot * o[j + 3]);
+                                red_add_v4(yrow + r0 + j, wslot * o[j], wslot * o[j + 1], wslot * o[j + 2], wslot * o[j + 3],
+                                           pol_y);
                         } else if (p.mode == kEpiStoreF32) {
                             float* dst = reinterpret_cast<float*>(p.out) + prow * p.ld_out + r0;
                             if (whole) {
