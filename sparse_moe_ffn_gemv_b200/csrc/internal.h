@@ -153,6 +153,7 @@ struct TcProblem {
     int grouped = 0;                       // 1: expert groups (offsets / tile_start), 0: one dense group
     int rows = 0, n_tiles = 0;             // dense: token rows and their tiles
     int bn = kTcBN;                        // token rows per tile (the kernel's; checked at launch)
+    int band = 0;                          // dense: token tiles per band of the tile order (set at launch)
     int num_groups = 0;
     const int32_t* offsets = nullptr;      // [E + 1] sorted-row offsets of the groups
     const int32_t* tile_start = nullptr;   // [E + 1] prefix of token tiles per group

@@ -202,9 +202,20 @@ __device__ __forceinline__ TileInfo decode_tile(const TcParams& P, const GroupTa
     }
     const TcProblem& p = P.p[ti.prob];
     if (!p.grouped) {
+        // dense: bands of `band` token tiles, every weight-row block of a token tile in turn,
+        // so that the tiles running at the same time share a few token tiles and every weight
+        // block (each read about once per band from HBM, the rest from L2)
         ti.group = 0;
-        ti.mb = local / p.n_tiles;
-        const int nb = local - ti.mb * p.n_tiles;
+        int nb;
+        if (p.band > 0) {
+            const int bsz = p.band * p.m_blocks;
+            const int band = local / bsz, within = local - band * bsz;
+            nb = band * p.band + within / p.m_blocks;
+            ti.mb = within - (within / p.m_blocks) * p.m_blocks;
+        } else {
+            ti.mb = local / p.n_tiles;
+            nb = local - ti.mb * p.n_tiles;
+        }
         ti.row0 = nb * p.bn;
         ti.nvalid = min(p.bn, p.rows - ti.row0);
         ti.ntt = p.n_tiles;
@@ -1101,6 +1112,14 @@ cudaError_t launch_tc_gemm(TcParams& P, bool gateup, int64_t max_tiles, cudaStre
     // the tile lists (dense tile counts, the permutation's tile prefix) were built for one
     // tile height, which picks the kernel: 128 rows with 4-bit weights or bf16, 256 with bf16
     const int bn = P.p[0].bn;
+    bool grouped = false;
+    for (int i = 0; i < P.nprob; ++i) grouped = grouped || P.p[i].grouped;
+    // dense problems: as many token tiles per band as fill the resident CTAs (or pairs)
+    // together with every weight-row block
+    const int conc = (bn == kTcBNWide && !q4 && !grouped) ? sm_count() / 2 : sm_count();
+    for (int i = 0; i < P.nprob; ++i)
+        if (!P.p[i].grouped && P.p[i].m_blocks > 0)
+            P.p[i].band = std::max(1, std::min(P.p[i].n_tiles, conc / P.p[i].m_blocks));
     for (int i = 0; i < P.nprob; ++i)
         if (P.p[i].bn != bn || (q4 && bn != kTcBN) || (bn != kTcBN && bn != kTcBNWide)) return cudaErrorInvalidValue;
     if (q4) {  // six load slots (packed tiles + token tile) feed two dequantised shared-memory operand slots
@@ -1113,8 +1132,6 @@ cudaError_t launch_tc_gemm(TcParams& P, bool gateup, int64_t max_tiles, cudaStre
         // experts is partial, the one-CTA tile (which skips an empty second half) measured
         // faster: latent block at 8192 tokens, expert gate/up 2.64 ms one CTA vs 2.78 ms
         // pairs; with 512 routed rows per expert (every tile full) pairs win, 518 vs 570 us.
-        bool grouped = false;
-        for (int i = 0; i < P.nprob; ++i) grouped = grouped || P.p[i].grouped;
         if (!grouped) {
             if (gateup) return launch_tc_t<true, kTcBNWide, 6, false, true>(P, max_tiles, s);
             return launch_tc_t<false, kTcBNWide, 6, false, true>(P, max_tiles, s);
