@@ -351,13 +351,20 @@ KERNEL_SOURCES = {
 }
 
 
+def code_of(text: str) -> str:
+    """C++ source without comments and blank-line or indentation differences."""
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    text = re.sub(r"//[^\n]*", "", text)
+    return "\n".join(line.strip() for line in text.splitlines() if line.strip())
+
+
 def source_hash(kernel: str = "") -> str:
-    """Hash of the sources of `kernel` (its base name), or of every CUDA source."""
+    """Hash of the code (comments aside) of `kernel`'s sources, or of every CUDA source."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "sparse_moe_ffn_gemv_b200", "csrc")
     files = KERNEL_SOURCES.get(kernel.split("<")[0], None) or sorted(os.listdir(csrc))
     for f in files:
-        h.update(open(os.path.join(csrc, f), "rb").read())
+        h.update(code_of(open(os.path.join(csrc, f)).read()).encode())
     return h.hexdigest()[:16]
 
 

@@ -5,9 +5,11 @@
 // output rows) its N side, so that one 128 x 256 x 16 MMA per K step reads 12 KB of shared
 // memory (a 128 x 128 pair of MMAs sharing the token tile would read 16 KB for the same
 // work). Every expert group is padded only to the token tile, and each weight tile is read
-// from HBM once and shared by the token tiles of its group through L2.
+// from HBM once and shared by the token tiles of its group through L2 (those tiles run at
+// about the same time; dense problems walk their tiles in bands of token tiles so that the
+// tiles running together share token tiles and weight blocks).
 //
-// One persistent CTA per SM, warp-specialised:
+// One persistent CTA (or CTA pair) per SM (pair of SMs), warp-specialised:
 //   warp 0      TMA producer: weight tile(s) + token tile per 64-wide K block into a
 //               STAGES-deep shared-memory ring (128-byte swizzle)
 //   warp 1      MMA issuer (one thread): tcgen05.mma kind::f16, bf16 x bf16 -> fp32 in
@@ -19,10 +21,9 @@
 //               into the token's fp32 routed sum with 16-byte vector reductions), or a
 //               plain store, each thread writing contiguous 16-byte vectors
 //   4-bit weights: warps 2..5 epilogue (one per TMEM lane quarter, all 256 columns) and
-//   warps 6..21 dequantisation: the producer loads the packed words,
-//               these warps write w = scale * q + bias (fp16; MXFP4: bf16) into the swizzled operand
-//               layout the MMA reads (mlxcel issue #974: affine 4-bit, per-group scale
-//               and bias). With 4-bit weights the shared memory holds two rings: a deep
+//   warps 6..21 dequantisation: the producer loads the packed words, these warps write
+//               w = scale * q + bias (fp16; MXFP4: bf16) into the swizzled operand layout
+//               the MMA reads (mlxcel issue #974: affine 4-bit, per-group scale and bias). With 4-bit weights the shared memory holds two rings: a deep
 //               one of small slots (the two packed tiles + the token tile of a K block)
 //               that TMA fills far ahead, and a shallow one of bf16 operand tiles that
 //               the dequantising warps fill and the MMA drains, so that load latency,
@@ -34,7 +35,8 @@
 // holds at most 128 rows, one accumulator set of 2 x 256 columns), in dense launches a
 // cluster of two CTAs per tile (PAIR: each CTA holds 128 token rows and one 128-row weight
 // tile, the leader issues tcgen05.mma.cta_group::2 with M = 256, N = 256 over both CTAs'
-// shared memory, two accumulator sets of 256 columns per CTA). Every mbarrier wait is bounded by %globaltimer; a wait that gives up records
+// shared memory, two accumulator sets of 256 columns per CTA).
+// Every mbarrier wait is bounded by %globaltimer; a wait that gives up records
 // MOE_ERR_DEVICE_TIMEOUT in the status word, drains its own outstanding copies / MMAs and
 // returns, and TMEM is always freed.
 //

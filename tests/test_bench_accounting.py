@@ -98,3 +98,10 @@ def test_smaller_copy_of_a_workload_keeps_every_other_field():
     assert bench.workload_spec(bench.parse(["--workload", "klear_bf16"])) is bench.inputs.WORKLOADS["klear_bf16"]
     with pytest.raises(SystemExit):
         bench.workload_spec(bench.parse(["--workload", "klear_bf16", "--experts", "4"]))
+
+
+def test_kernel_source_hash_ignores_comments_but_not_code():
+    import bench
+    a = "int f(int x) { return x + 1; } // add one\n"
+    assert bench.code_of(a) == bench.code_of("/* doc */\nint f(int x) { return x + 1; }\n\n")
+    assert bench.code_of(a) != bench.code_of("int f(int x) { return x + 2; }\n")
