@@ -250,7 +250,11 @@ MOE_API moe_status moe_combine(const moe_config *cfg, const moe_weights *w, cons
                        const void *x, const float *coef, int64_t T, void *y,
                        void *ws, size_t ws_bytes, moe_stream_t stream);
 
-/* The whole block: y [T, H] = block(x [T, H]), act_dtype in and out. */
+/* The whole block: y [T, H] = block(x [T, H]), act_dtype in and out. The engine is chosen
+ * by the batch: one cooperative decode launch for one token (two with bf16 weights; no
+ * latent projection, bf16 activations), the CUDA-core weight-streaming kernels for few
+ * slots per expert, the tensor-core kernels from about E / 4 slots on (environment variable
+ * MOE_PATH=gemv | tc | decode forces one engine where it can run). */
 MOE_API moe_status moe_block_forward(const moe_config *cfg, const moe_weights *w, const void *x,
                              int64_t T, void *y, void *ws, size_t ws_bytes, moe_stream_t stream);
 
@@ -299,7 +303,7 @@ MOE_API moe_status moe_clear_device_status(void *ws, moe_stream_t stream);
 MOE_API moe_status moe_selftest_bounded_wait(void *ws, int64_t timeout_ns, moe_stream_t stream);
 
 /* Failure-detection self test of the grid barrier the persistent decode kernel uses
- * between its phases (moe_block_forward with up to 8 tokens): one block arrives at a
+ * between its phases (moe_block_forward on a decode-sized batch): one block arrives at a
  * barrier that needs two arrivals and polls it with the same %globaltimer deadline
  * (timeout_ns, 0 < timeout_ns <= 1e9); when it gives up it records
  * MOE_ERR_DEVICE_TIMEOUT in the status word of `ws` and returns, and the counter is put
