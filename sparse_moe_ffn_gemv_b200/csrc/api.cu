@@ -298,11 +298,6 @@ DecodeArgs decode_args(const moe_config* c, const moe_weights* w, const void* x,
     d.hs = static_cast<char*>(ws) + L.hs;
     d.status = reinterpret_cast<int*>(static_cast<char*>(ws) + L.status);
     d.bar = reinterpret_cast<unsigned*>(static_cast<char*>(ws) + L.status + kDecodeBarOffset);
-    // the down rows of the activated experts are prefetched into L2 only where they fit
-    // comfortably beside the gate/up stream
-    const int64_t drow = c->weight_format == MOE_DTYPE_BF16 ? int64_t(c->intermediate) * 2 : c->intermediate / 2;
-    const int64_t most = std::min<int64_t>(c->num_experts, T * c->top_k);
-    d.l2_prefetch = most * c->hidden * drow + int64_t(c->hidden) * c->shared_intermediate * 2 <= (int64_t(40) << 20);
     return d;
 }
 

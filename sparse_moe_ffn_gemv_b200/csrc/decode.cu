@@ -17,8 +17,8 @@
 //      and for the shared expert, and writes y = y_r | y_r + s | c0 y_r + c1 s for its
 //      rows (libmir-metal execute: down weighted by routing.weights and summed; ferrox
 //      KimiExpertWeights::forward: down(act(gate, up))).
-// While phase B streams the gate/up rows, each block asks L2 to prefetch its phase-C down
-// rows when they fit in L2, so phase C reads them from L2.
+// (An L2 prefetch of each block's phase-C down rows issued at the start of phase B
+// measured slower: Klear, one token, 47.1 vs 45.1 us without it.)
 // Every grid-barrier wait is bounded by %globaltimer: a wait that gives up records
 // MOE_ERR_DEVICE_TIMEOUT in the status word, and the block skips the remaining phases.
 // The last block to finish resets the barrier counters, so the next launch starts from 0.
@@ -60,18 +60,6 @@ struct DecSmem {
 // (bf16) and, for 4-bit planes, their per-32 sums; 16-byte aligned.
 __host__ __device__ __forceinline__ size_t dec_keys_offset(int T, int H, bool sums) {
     return (size_t(T) * H * 2 + (sums ? size_t(T) * (H / 32) * 4 : 0) + 15) & ~size_t(15);
-}
-
-__device__ __forceinline__ void l2_prefetch(const void* p, size_t bytes) {
-    // a hint: the start is rounded up and the size down to 16 bytes, so nothing outside
-    // [p, p + bytes) is named
-    uintptr_t a = (reinterpret_cast<uintptr_t>(p) + 15) & ~uintptr_t(15);
-    const uintptr_t end = (reinterpret_cast<uintptr_t>(p) + bytes) & ~uintptr_t(15);
-    while (a < end) {
-        const uint32_t n = uint32_t(end - a < (uintptr_t(1) << 20) ? end - a : (uintptr_t(1) << 20));
-        asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(a), "r"(n) : "memory");
-        a += n;
-    }
 }
 
 __device__ __forceinline__ float bf16_ld(const void* p, int64_t i) {
@@ -181,8 +169,6 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(const DecodeArgs
         for (int e = threadIdx.x; e < E; e += blockDim.x) sm.ssel[e] = __ldg(a.sel_bias + e);
     if (WF == kQ4 || dq) stage_tokens<kQ4>(a.x, H, 0, T, nullptr, 1, xs, xsum);
     else stage_tokens<kBF16>(a.x, H, 0, T, nullptr, 1, xs, nullptr);
-    if (a.l2_prefetch && Is && threadIdx.x == 0 && nr > 0)
-        l2_prefetch(static_cast<const char*>(a.sd_w) + int64_t(r0) * srb, size_t(nr) * srb);
     __syncthreads();
     {
         const int n_rg = (E + RR - 1) / RR;           // router row groups
@@ -289,11 +275,6 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(const DecodeArgs
             sm.n_d = n_d;
         }
         __syncthreads();
-        // this block's phase-C down rows of every distinct expert, into L2
-        if (a.l2_prefetch && nr > 0)
-            for (int d = threadIdx.x; d < n_d; d += blockDim.x)
-                l2_prefetch(static_cast<const char*>(a.down_w) + (int64_t(sm.dexp[d]) * H + r0) * drb,
-                            size_t(nr) * drb);
         // routed gate/up: BU units (gate + up rows) of one distinct expert per warp item
         const int ub = (I + BU - 1) / BU;
         const int64_t rbh = row_bytes<WF>(H);

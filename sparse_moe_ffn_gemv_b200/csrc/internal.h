@@ -132,7 +132,6 @@ struct DecodeArgs {
     void* hs = nullptr;                           // workspace: bf16 [T, Is]
     unsigned* bar = nullptr;                      // workspace: three zeroed counters
     int* status = nullptr;
-    int l2_prefetch = 0;                          // prefetch each block's down rows into L2
 };
 // Dynamic shared memory the decode kernel needs for a config and T (0 if it cannot run it).
 size_t decode_smem_bytes(const DecodeArgs& a);
